@@ -1,0 +1,499 @@
+"""Benchmark of the Nectar hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload qwen3_1p7b]
+
+One step = the whole hot path over one decode batch of the workload:
+(i) exact cached-token attention (alpha, A) over the document (Eq. (3.1))
+and the Nectar decode -- (ii) the score / target MLPs (Eq. (3.6)) fused with
+(iii) the merge with exact causal local attention (Eqs. (3.4)-(3.5)).  The
+metric is query vectors (layer x query head x token) per second through the
+step; the dominant kernel is (i), which is HBM-bound, so its roofline is
+reported as achieved / measured HBM bandwidth.
+
+Multi-GPU: one process per GPU under torchrun; every rank runs an
+independent replica (the path has no exchange step), value = all ranks'
+queries / max-over-ranks time, scaling "weak".
+
+--impl reference times the CPU oracle (oracle/, plain C in fp64) on the
+box's host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from nectar_inputs import PRESETS, make_workload  # noqa: E402
+
+METRIC = "Nectar decode queries/s & exact (α,A) HBM GB/s at 1 B200; % of roofline"
+UNIT = "queries/s"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# distributed helpers (also exercised by the gloo tests)
+# ---------------------------------------------------------------------------
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max over ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(value: float, device=None) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate(units_per_rank: float, max_ms: float, steps: int) -> float:
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    total_units = reduce_sum(units_per_rank * steps)
+    return total_units / (max_ms / 1e3)
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        try:
+            rows = [ln.split(",") for ln in open(self.path).read().strip().splitlines() if ln.strip()]
+        except Exception:
+            rows = []
+        sm = []
+        mx = None
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+                for nm, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(nm)
+            except Exception:
+                pass
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# workload bookkeeping
+# ---------------------------------------------------------------------------
+def describe(wl):
+    H = sorted(set(wl.widths)) if wl.widths else []
+    return (f"{wl.name}: L={wl.L} Hkv={wl.Hkv} G={wl.G} d={wl.d} n={wl.n} B={wl.B} T={wl.T} "
+            f"nq={wl.nq} H={H[0] if len(H) == 1 else H} depth={wl.depth}")
+
+
+def queries_per_step(wl) -> int:
+    return wl.L * wl.Hkv * wl.G * wl.nq
+
+
+def attn_bytes(wl) -> int:
+    """Algorithmic bytes of (i): K and V once per (l, h), Q in, alpha and A out."""
+    heads, rows = wl.heads, wl.rows
+    return heads * (4 * wl.n * wl.d + rows * 2 * wl.d + rows * 4 * (wl.d + 1))
+
+
+def decode_bytes(wl, weight_bytes: int) -> int:
+    """Algorithmic bytes of the fused decode: module weights, the visible local
+    K/V of every sequence, Q in, out."""
+    vis = (wl.local_len.long().clamp(max=wl.T)).sum().item()
+    return weight_bytes + wl.heads * vis * 4 * wl.d + wl.heads * wl.rows * (2 + 4) * wl.d
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import long_context_attention_split_b200 as nx
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    hbm_peak, tc_peak, peak_kind = load_peaks()
+
+    wl = make_workload(args.workload, seed=args.seed + rank, device=dev)
+    mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G, device=dev)
+    Q = wl.Q
+    alpha = torch.empty(Q.shape[:4], dtype=torch.float32, device=dev)
+    A = torch.empty(Q.shape, dtype=torch.float32, device=dev)
+    out = torch.empty(Q.shape, dtype=torch.float32, device=dev)
+    wsb = nx.cache_attn_workspace_size(wl.L, wl.Hkv, wl.G, wl.n, wl.nq)
+    work = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    local_args = (wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len)
+    n_split = math.ceil(wl.rows / 8)       # CUDA-core split launches per (i) call
+    launches_per_step = n_split + 1 + 1    # split kernel(s) + combine + fused decode
+
+    ev_a0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_a1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_d1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    def step(i=None):
+        if i is not None:
+            ev_a0[i].record(stream)
+        nx.cache_attn_lse(wl.K, wl.V, Q, alpha=alpha, A=A, workspace=work, stream=stream)
+        if i is not None:
+            ev_a1[i].record(stream)
+        nx.decode(mods, Q, *local_args, out=out, stream=stream)
+        if i is not None:
+            ev_d1[i].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    flags = nx.device_error_flags(clear=True)
+
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+    total_ms = t0.elapsed_time(t1)
+    max_ms = reduce_max(total_ms, dev)
+    attn_ms = [ev_a0[i].elapsed_time(ev_a1[i]) for i in range(args.steps)]
+    dec_ms = [ev_a1[i].elapsed_time(ev_d1[i]) for i in range(args.steps)]
+    attn_avg = sum(attn_ms) / len(attn_ms)
+    dec_avg = sum(dec_ms) / len(dec_ms)
+    flags |= nx.device_error_flags(clear=True)
+
+    qps = queries_per_step(wl)
+    value = aggregate(qps, max_ms, args.steps)
+    ab = attn_bytes(wl)
+    achieved = ab / (attn_avg / 1e3) / 1e9
+    db = decode_bytes(wl, mods.bytes)
+
+    # ---- end to end through the public API with host buffers ----
+    pin = lambda t: t.cpu().pin_memory()
+    hQ, hseq, hpos, hlen = pin(Q), pin(wl.q_seq), pin(wl.q_pos), pin(wl.local_len)
+    h_alpha = torch.empty(alpha.shape, dtype=torch.float32).pin_memory()
+    h_A = torch.empty(A.shape, dtype=torch.float32).pin_memory()
+    h_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    dQ = torch.empty_like(Q)
+    dseq, dpos, dlen = torch.empty_like(wl.q_seq), torch.empty_like(wl.q_pos), torch.empty_like(wl.local_len)
+    h2d = sum(t.numel() * t.element_size() for t in (hQ, hseq, hpos, hlen))
+    d2h = sum(t.numel() * t.element_size() for t in (h_alpha, h_A, h_out))
+
+    def e2e_step():
+        dQ.copy_(hQ, non_blocking=True)
+        dseq.copy_(hseq, non_blocking=True)
+        dpos.copy_(hpos, non_blocking=True)
+        dlen.copy_(hlen, non_blocking=True)
+        nx.cache_attn_lse(wl.K, wl.V, dQ, alpha=alpha, A=A, workspace=work, stream=stream)
+        nx.decode(mods, dQ, dseq, dpos, wl.Kloc, wl.Vloc, dlen, out=out, stream=stream)
+        h_alpha.copy_(alpha, non_blocking=True)
+        h_A.copy_(A, non_blocking=True)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_max = reduce_max(e0.elapsed_time(e1), dev)
+    e2e_value = aggregate(qps, e2e_max, args.steps)
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, mods_host=None, budget_s=args.cpu_budget)
+
+    if rank == 0:
+        traffic = traffic_from_profile(args.workload)
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": UNIT,
+            "n_gpus": ws,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": max_ms / args.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {
+                "workload": describe(wl),
+                "global_batch": wl.B * ws,
+                "seq_len": wl.n,
+                "parallelism": f"replicas{ws}",
+                "queries_per_step_per_gpu": qps,
+                "l2": "inputs larger than L2 (document K/V 3.76 GB streamed every step)",
+            },
+            "parts": {
+                "exact_attn_ms": attn_avg,
+                "exact_attn_GBps": achieved,
+                "decode_ms": dec_avg,
+                "decode_queries_per_s": qps / (dec_avg / 1e3),
+                "decode_alg_bytes": db,
+                "decode_GBps": db / (dec_avg / 1e3) / 1e9,
+                "decode_frac_of_hbm": db / (dec_avg / 1e3) / 1e9 / hbm_peak,
+            },
+            "roofline": {
+                "kernel": "cache_attn_split+combine (exact alpha, A)",
+                "bound": "hbm",
+                "achieved": achieved,
+                "peak": hbm_peak,
+                "peak_kind": peak_kind,
+                "unit": "GB/s",
+                "frac": achieved / hbm_peak,
+                "alg_bytes_per_launch": ab,
+                "traffic": traffic,
+            },
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+            "device_error_flags": flags,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def traffic_from_profile(workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary (profiles/), or None."""
+    path = os.path.join(ROOT, "profiles", f"cache_attn_split_{workload}.json")
+    try:
+        with open(path) as f:
+            return json.load(f).get("dram_bytes_per_launch")
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline
+# ---------------------------------------------------------------------------
+def _oracle_sample(wl, layers):
+    """One pass of the whole path on the oracle for the given layers
+    (all their KV heads).  Returns query vectors processed."""
+    import numpy as np
+    import oracle
+    H = len(layers) * wl.Hkv
+    K = wl.K[layers].reshape(H, wl.n, wl.d)
+    V = wl.V[layers].reshape(H, wl.n, wl.d)
+    Q = wl.Q[layers].reshape(H, wl.rows, wl.d)
+    alpha, A = oracle.cache_attn(K, V, Q, wl.scale)
+    sel = [(l, h) for l in layers for h in range(wl.Hkv)]
+    a, At = oracle.module_forward(wl, sel)
+    a = np.stack([a[k] for k in sel])
+    At = np.stack([At[k] for k in sel])
+    oracle.merge_local(a, At, Q, wl.q_seq, wl.q_pos, wl.Kloc[layers].reshape(H, wl.B, wl.T, wl.d),
+                       wl.Vloc[layers].reshape(H, wl.B, wl.T, wl.d), wl.local_len, wl.scale)
+    return H * wl.rows
+
+
+def cpu_baseline(wl, mods_host=None, budget_s=20.0, layers_per_sample=1):
+    import oracle
+    oracle.build()
+    cores = oracle.num_threads()
+    # host copies of what one sample touches
+    layers = list(range(min(layers_per_sample, wl.L)))
+    host = _host_view(wl, layers)
+    t0 = time.perf_counter()
+    done = 0
+    samples = 0
+    while True:
+        done += _oracle_sample(host, list(range(len(layers))))
+        samples += 1
+        if time.perf_counter() - t0 > budget_s * 0.5 or samples >= 4:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{samples} pass(es) of the whole path over layer(s) {layers} "
+                      f"({len(layers) * wl.Hkv} of {wl.heads} KV heads, all their query rows), "
+                      f"{dt:.1f} s on {cores} threads; queries/s = query vectors done / time"}
+
+
+class _HostWL:
+    pass
+
+
+def _host_view(wl, layers):
+    """CPU copy of the workload restricted to `layers` (renumbered 0..)."""
+    h = _HostWL()
+    for k in ("name", "Hkv", "G", "d", "n", "nq", "B", "T", "scale", "depth"):
+        setattr(h, k, getattr(wl, k))
+    h.L = len(layers)
+    h.rows = wl.rows
+    h.heads = h.L * wl.Hkv
+    idx = torch.tensor(layers)
+    h.K = wl.K[idx.to(wl.K.device)].cpu()
+    h.V = wl.V[idx.to(wl.V.device)].cpu()
+    h.Q = wl.Q[idx.to(wl.Q.device)].cpu()
+    h.Kloc = wl.Kloc[idx.to(wl.Kloc.device)].cpu()
+    h.Vloc = wl.Vloc[idx.to(wl.Vloc.device)].cpu()
+    h.q_seq, h.q_pos, h.local_len = wl.q_seq.cpu(), wl.q_pos.cpu(), wl.local_len.cpu()
+    h.widths = [wl.widths[l] for l in layers]
+    h.modules = []
+    for l in layers:
+        layer = {}
+        for net, p in wl.modules[l].items():
+            layer[net] = {k: ([x.cpu() if x is not None else None for x in v] if isinstance(v, list)
+                              else (v.cpu() if torch.is_tensor(v) else v)) for k, v in p.items()}
+        h.modules.append(layer)
+    return h
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    wl = make_workload(args.workload, seed=args.seed, device="cpu") if args.workload == "toy" else None
+    if wl is None:
+        # the oracle's sample needs one layer of the workload on the host
+        wl = make_workload(args.workload, seed=args.seed, device="cpu", L=1)
+    host = _host_view(wl, [0])
+    cores = oracle.num_threads()
+    for _ in range(max(args.warmup, 0)):
+        pass   # the oracle has no warm-up state; a warm-up pass would only repeat the work
+    t0 = time.perf_counter()
+    done = 0
+    for _ in range(args.steps):
+        done += _oracle_sample(host, [0])
+    dt = time.perf_counter() - t0
+    value = done / dt
+    full = PRESETS[args.workload]
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": describe(make_workload(args.workload, seed=args.seed, device="meta"))
+                   if False else f"{args.workload}: L={full['L']} Hkv={full['Hkv']} G={full['G']} n={full['n']}",
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step = the whole path on layer 0 ({wl.Hkv} KV heads, all query rows) "
+                                   f"of {args.workload}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qwen3_1p7b", choices=sorted(PRESETS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,213 @@
+/*
+ * nectar.h -- C ABI of libnectar.so, the B200 (sm_100a) hot path of Nectar.
+ *
+ * Method: "Nectar: Neural Estimation of Cached-Token Attention via
+ * Regression" (Monteiro, Klein, Ablin, Cuturi; arXiv 2605.09778).  For a
+ * fixed document cache K, V (RoPE already applied) of one (layer, KV-head),
+ * a query q has the document log-normalizer alpha(q) and the
+ * document-normalised readout A(q) of Eq. (3.1).  A trained pair of small
+ * networks (score a_theta, target A_theta; Eq. (3.6)) replaces them at
+ * inference, and the document then acts as ONE virtual logit a_theta with
+ * value A_theta, softmaxed jointly with the exact causal local tokens
+ * (Eqs. (3.4)-(3.5)).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - d (head dimension) must be 128; any other value returns
+ *    NECTAR_ERR_UNSUPPORTED.
+ *  - GQA: query head h' = h*G + g belongs to KV head h and uses its cache and
+ *    its module pair (§2.1).  All query tensors are laid out
+ *    [L][Hkv][G][nq][d] (bf16), so the G*nq query vectors ("rows") of one
+ *    (l, h) are contiguous; row r = g*nq + i is token i of query head g.
+ *  - Per-query outputs (alpha, a: fp32 [L][Hkv][G][nq]; A, A_theta, out:
+ *    fp32 [L][Hkv][G][nq][d]) follow the same row order.  Outputs are fp32
+ *    because the paper stores its regression targets in float32 (App. A).
+ *  - Pointers marked DEVICE are device memory owned by the caller; HOST
+ *    pointers are read during the call only.  Device pointers must be
+ *    16-byte aligned and the tensors contiguous.  The library never
+ *    allocates, frees or synchronises in these calls: all work is enqueued on
+ *    `stream` and the outputs are valid once the stream reaches that point.
+ *  - Every call validates its arguments on the host first and returns a
+ *    status.  On any error nothing is enqueued.  nectar_last_error() then
+ *    gives a one-line reason (thread-local).
+ *  - Values that the host cannot see (device arrays q_seq, q_pos,
+ *    local_len) are checked in the kernels: an out-of-range q_seq entry is
+ *    treated as a sequence with no local tokens, a local_len above T_max is
+ *    clamped to T_max, and both raise a bit readable with
+ *    nectar_device_error_flags().
+ *  - `scale` multiplies q.k; pass 1/sqrt(d) for Eq. (3.1)'s scores.
+ */
+#ifndef NECTAR_H_
+#define NECTAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NECTAR_API __attribute__((visibility("default")))
+#else
+#define NECTAR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t nectar_bf16;            /* raw bfloat16 bit pattern */
+typedef struct CUstream_st *nectar_stream_t;   /* same type as cudaStream_t */
+
+typedef enum {
+  NECTAR_OK = 0,
+  NECTAR_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size */
+  NECTAR_ERR_UNSUPPORTED = 2,   /* d != 128, width or depth out of range */
+  NECTAR_ERR_WORKSPACE = 3,     /* workspace missing or too small */
+  NECTAR_ERR_CUDA = 4           /* a CUDA call failed (see nectar_last_error) */
+} nectar_status;
+
+/* Model shape: L layers, Hkv KV heads, G query heads per KV head, head dim d. */
+typedef struct {
+  int32_t L, Hkv, G, d;
+} nectar_dims;
+
+#define NECTAR_MAX_DEPTH 4
+#define NECTAR_MAX_LAYERS 256
+#define NECTAR_MAX_WIDTH 1024
+
+/* ------------------------------------------------------------------------
+ * (i) Exact cached-token attention, Eq. (3.1), §2.1:
+ *   s_j = scale * q . k_j,   alpha(q) = log sum_j e^{s_j},
+ *   A(q) = sum_j e^{s_j} v_j / sum_j e^{s_j},
+ * for every query row of every (l, h) over that head's n document tokens.
+ * The sum is split over n and the parts are joined by their log-sum-exp
+ * (the grouping of the softmax sum that Eq. (3.4) rests on), so the result
+ * does not depend on how the cache is split.
+ *
+ *   K, V   DEVICE bf16 [L][Hkv][n][d]       document cache
+ *   Q      DEVICE bf16 [L][Hkv][G][nq][d]
+ *   alpha  DEVICE fp32 [L][Hkv][G][nq]      (-inf when n == 0)
+ *   A      DEVICE fp32 [L][Hkv][G][nq][d]   (0 when n == 0)
+ *   workspace  DEVICE scratch of at least
+ *              nectar_cache_attn_workspace_size(dims, n, nq) bytes (may be
+ *              NULL when that size is 0).  Its contents on entry do not
+ *              matter; two calls that overlap on the GPU must not share one.
+ * n >= 0, nq >= 0 (nq == 0: nothing to do).  Returns NECTAR_ERR_WORKSPACE
+ * when the workspace is too small.
+ * ------------------------------------------------------------------------ */
+NECTAR_API size_t nectar_cache_attn_workspace_size(nectar_dims dims, int64_t n, int64_t nq);
+
+NECTAR_API nectar_status nectar_cache_attn_lse(nectar_dims dims, const nectar_bf16 *K,
+                                    const nectar_bf16 *V, int64_t n,
+                                    const nectar_bf16 *Q, int64_t nq, float scale,
+                                    float *alpha, float *A, void *workspace,
+                                    size_t workspace_bytes, nectar_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Module set: one score net a_theta: R^d -> R and one target net
+ * A_theta: R^d -> R^d per (l, h), shared by the G query heads of that KV
+ * head (§2.1), each an MLP with input re-injection, Eq. (3.6), §2.4:
+ *   h_0 = SiLU(U_0 q + b_0),  h_k = SiLU(V_k q + U_k h_{k-1} + b_k),
+ *   k = 1..depth-1, followed by a linear readout y = W_out h_{depth-1} + c
+ *   (dout = 1 for the score net, d for the target net).
+ * Width H_l may differ between layers (App. C.1); both nets of a layer use
+ * it.  Weights and biases are bf16.
+ *
+ * The device copy is one packed blob built by nectar_module_pack.  Its
+ * layout is private to the library (tiled for TMA); size it with
+ * nectar_module_packed_elems.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int32_t depth;          /* hidden layers per net, 1..NECTAR_MAX_DEPTH */
+  const int32_t *width;   /* HOST [L]: H_l, a multiple of 16 in [16, 1024] */
+  const nectar_bf16 *weights;   /* DEVICE packed blob */
+  int64_t weights_elems;  /* bf16 elements in the blob */
+} nectar_module_set;
+
+/* Plain row-major HOST tensors of one net for all Hkv heads of a layer. */
+typedef struct {
+  const nectar_bf16 *U[NECTAR_MAX_DEPTH]; /* k=0: [Hkv][H][d]; k>=1: [Hkv][H][H] */
+  const nectar_bf16 *V[NECTAR_MAX_DEPTH]; /* k>=1: [Hkv][H][d] (V[0] unused) */
+  const nectar_bf16 *b[NECTAR_MAX_DEPTH]; /* [Hkv][H] */
+  const nectar_bf16 *Wout;                /* [Hkv][dout][H] */
+  const nectar_bf16 *c;                   /* [Hkv][dout] */
+} nectar_net_host;
+
+/* Elements of the packed blob for these widths (0 on invalid arguments). */
+NECTAR_API int64_t nectar_module_packed_elems(nectar_dims dims, int32_t depth, const int32_t *width);
+
+/* Pack HOST tensors into a HOST blob of `blob_elems` elements.
+ * nets: HOST [L][2] -- nets[2*l + 0] the score net, nets[2*l + 1] the target
+ * net of layer l.  Padding in the blob is written as zeros. */
+NECTAR_API nectar_status nectar_module_pack(nectar_dims dims, int32_t depth, const int32_t *width,
+                                 const nectar_net_host *nets, nectar_bf16 *blob,
+                                 int64_t blob_elems);
+
+/* ------------------------------------------------------------------------
+ * (ii) Module forward, Eq. (3.6): for every query row of every (l, h),
+ *   a[row]       = a_theta(q)     DEVICE fp32 [L][Hkv][G][nq]
+ *   A_theta[row] = A_theta(q)     DEVICE fp32 [L][Hkv][G][nq][d]
+ * Runs on the tensor cores (tcgen05, bf16 operands, fp32 accumulation);
+ * hidden activations are rounded to bf16 between layers.
+ * ------------------------------------------------------------------------ */
+NECTAR_API nectar_status nectar_module_forward(nectar_dims dims, const nectar_module_set *mods,
+                                    const nectar_bf16 *Q, int64_t nq, float *a,
+                                    float *A_theta, nectar_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * (iii) Merge with exact causal local attention, Eqs. (3.4)-(3.5), §2.2:
+ *   out = (e^{a} A_doc + sum_{i vis} e^{s_i} v_i) / (e^{a} + sum_{i vis} e^{s_i}),
+ *   s_i = scale * q . k_i over the visible local tokens of the row's token.
+ * With (a, A_doc) = the exact (alpha, A) of nectar_cache_attn_lse this is
+ * full attention over document + local tokens (Eq. (3.4) is an identity);
+ * with (a_theta, A_theta) it is the Nectar output (Eq. (3.5)).
+ *
+ *   a       DEVICE fp32 [L][Hkv][G][nq]
+ *   A_doc   DEVICE fp32 [L][Hkv][G][nq][d]
+ *   Q       DEVICE bf16 [L][Hkv][G][nq][d]
+ *   q_seq   DEVICE int32 [nq]   sequence of token i, in [0, B)
+ *   q_pos   DEVICE int32 [nq]   local position t of token i
+ *   Kloc, Vloc  DEVICE bf16 [L][Hkv][B][T_max][d]   local cache per sequence
+ *   local_len   DEVICE int32 [B]   valid local tokens of each sequence
+ *   out     DEVICE fp32 [L][Hkv][G][nq][d]
+ * Visible set of token i (reading of §2.2, Eq. (3.4) indexes i <= t):
+ *   { j : j <= q_pos[i] and j < local_len[q_seq[i]] }  -- the token itself
+ * included.  An empty visible set gives out = A_doc.
+ * ------------------------------------------------------------------------ */
+NECTAR_API nectar_status nectar_merge_local(nectar_dims dims, const float *a, const float *A_doc,
+                                 const nectar_bf16 *Q, int64_t nq, const int32_t *q_seq,
+                                 const int32_t *q_pos, const nectar_bf16 *Kloc,
+                                 const nectar_bf16 *Vloc, int32_t B, int32_t T_max,
+                                 const int32_t *local_len, float scale, float *out,
+                                 nectar_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Fused Nectar decode: (ii) and (iii) in one launch -- the module forward of
+ * every row followed by the merge of its (a_theta, A_theta) with its exact
+ * causal local attention.  Arguments as in nectar_module_forward and
+ * nectar_merge_local; out DEVICE fp32 [L][Hkv][G][nq][d].  Equal (up to
+ * rounding order) to nectar_module_forward followed by nectar_merge_local.
+ * ------------------------------------------------------------------------ */
+NECTAR_API nectar_status nectar_decode(nectar_dims dims, const nectar_module_set *mods,
+                            const nectar_bf16 *Q, int64_t nq, const int32_t *q_seq,
+                            const int32_t *q_pos, const nectar_bf16 *Kloc,
+                            const nectar_bf16 *Vloc, int32_t B, int32_t T_max,
+                            const int32_t *local_len, float scale, float *out,
+                            nectar_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Diagnostics
+ * ------------------------------------------------------------------------ */
+NECTAR_API const char *nectar_status_string(nectar_status s);
+/* One-line reason for the last non-OK status returned on this thread. */
+NECTAR_API const char *nectar_last_error(void);
+/* Reads (and, if `clear` is non-zero, resets) the device error word of the
+ * current device: bit 0 = a bounded wait gave up, bit 1 = a q_seq entry out
+ * of range, bit 2 = a local_len entry out of range.  SYNCHRONISES the
+ * device; meant for tests and debugging, not for the hot path. */
+NECTAR_API nectar_status nectar_device_error_flags(int32_t *flags, int32_t clear);
+/* Library version, "major.minor.patch". */
+NECTAR_API const char *nectar_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NECTAR_H_ */

@@ -1,0 +1,296 @@
+"""Nectar hot path on B200: Python binding of libnectar.so.
+
+Argument marshalling only -- every step of the path runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the stream.  The entry
+points mirror include/nectar.h:
+
+    cache_attn_lse   (i)   exact alpha(q), A(q) of Eq. (3.1) over the document
+    module_forward   (ii)  score / target MLPs a_theta, A_theta of Eq. (3.6)
+    merge_local      (iii) merge with exact causal local attention, Eqs. (3.4)-(3.5)
+    decode           (ii)+(iii) in one launch
+
+"Nectar: Neural Estimation of Cached-Token Attention via Regression"
+(Monteiro, Klein, Ablin, Cuturi).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnectar.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "nectar.h")
+
+NECTAR_MAX_DEPTH = 4
+STATUS = {0: "NECTAR_OK", 1: "NECTAR_ERR_INVALID_ARG", 2: "NECTAR_ERR_UNSUPPORTED",
+          3: "NECTAR_ERR_WORKSPACE", 4: "NECTAR_ERR_CUDA"}
+
+
+class NectarError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("L", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("G", ctypes.c_int32), ("d", ctypes.c_int32)]
+
+
+class _ModuleSetC(ctypes.Structure):
+    _fields_ = [("depth", ctypes.c_int32), ("width", ctypes.POINTER(ctypes.c_int32)),
+                ("weights", ctypes.c_void_p), ("weights_elems", ctypes.c_int64)]
+
+
+class _NetHostC(ctypes.Structure):
+    _fields_ = [("U", ctypes.c_void_p * NECTAR_MAX_DEPTH), ("V", ctypes.c_void_p * NECTAR_MAX_DEPTH),
+                ("b", ctypes.c_void_p * NECTAR_MAX_DEPTH), ("Wout", ctypes.c_void_p), ("c", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libnectar.so (built in-tree by build.py).  Raises if it is missing:
+    there is no fallback path."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m long_context_attention_split_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I64, I32, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
+    S = ctypes.c_int
+    L.nectar_cache_attn_workspace_size.argtypes = [Dims, I64, I64]
+    L.nectar_cache_attn_workspace_size.restype = ctypes.c_size_t
+    L.nectar_cache_attn_lse.argtypes = [Dims, P, P, I64, P, I64, F, P, P, P, ctypes.c_size_t, P]
+    L.nectar_cache_attn_lse.restype = S
+    L.nectar_module_packed_elems.argtypes = [Dims, I32, P]
+    L.nectar_module_packed_elems.restype = I64
+    L.nectar_module_pack.argtypes = [Dims, I32, P, P, P, I64]
+    L.nectar_module_pack.restype = S
+    L.nectar_module_forward.argtypes = [Dims, ctypes.POINTER(_ModuleSetC), P, I64, P, P, P]
+    L.nectar_module_forward.restype = S
+    L.nectar_merge_local.argtypes = [Dims, P, P, P, I64, P, P, P, P, I32, I32, P, F, P, P]
+    L.nectar_merge_local.restype = S
+    L.nectar_decode.argtypes = [Dims, ctypes.POINTER(_ModuleSetC), P, I64, P, P, P, P, I32, I32, P, F, P, P]
+    L.nectar_decode.restype = S
+    L.nectar_status_string.argtypes = [S]
+    L.nectar_status_string.restype = ctypes.c_char_p
+    L.nectar_last_error.restype = ctypes.c_char_p
+    L.nectar_device_error_flags.argtypes = [ctypes.POINTER(ctypes.c_int32), I32]
+    L.nectar_device_error_flags.restype = S
+    L.nectar_version.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def header_functions() -> List[str]:
+    """Names of the functions declared in include/nectar.h."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nectar_[a-z0-9_]+)\s*\(", text)))
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise NectarError(status, f"{what}: {lib().nectar_last_error().decode()}")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, device=True) -> None:
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def dims_of(Q: torch.Tensor) -> Tuple[Dims, int]:
+    """Q: [L][Hkv][G][nq][d] -> (dims, nq)."""
+    if Q.dim() != 5:
+        raise ValueError("Q must be [L, Hkv, G, nq, d]")
+    L_, Hkv, G, nq, d = Q.shape
+    return Dims(L_, Hkv, G, d), nq
+
+
+def version() -> str:
+    return lib().nectar_version().decode()
+
+
+# ---------------------------------------------------------------------------
+# (i) exact cached-token attention
+# ---------------------------------------------------------------------------
+def cache_attn_workspace_size(L: int, Hkv: int, G: int, n: int, nq: int, d: int = 128) -> int:
+    return int(lib().nectar_cache_attn_workspace_size(Dims(L, Hkv, G, d), n, nq))
+
+
+def cache_attn_lse(K, V, Q, scale: Optional[float] = None, alpha=None, A=None, workspace=None, stream=None):
+    """alpha [L,Hkv,G,nq] fp32 and A [L,Hkv,G,nq,d] fp32 of Eq. (3.1).
+
+    K, V: bf16 [L, Hkv, n, d]; Q: bf16 [L, Hkv, G, nq, d] (CUDA)."""
+    dims, nq = dims_of(Q)
+    n = K.shape[2]
+    for t, nm in ((K, "K"), (V, "V"), (Q, "Q")):
+        _need(t, nm, torch.bfloat16)
+    if scale is None:
+        scale = 1.0 / math.sqrt(dims.d)
+    if alpha is None:
+        alpha = torch.empty(Q.shape[:4], dtype=torch.float32, device=Q.device)
+    if A is None:
+        A = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    ws_bytes = cache_attn_workspace_size(dims.L, dims.Hkv, dims.G, n, nq, dims.d)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    st = lib().nectar_cache_attn_lse(dims, _ptr(K), _ptr(V), n, _ptr(Q), nq, float(scale), _ptr(alpha), _ptr(A),
+                                     _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                     _stream(stream))
+    _check(st, "nectar_cache_attn_lse")
+    return alpha, A
+
+
+# ---------------------------------------------------------------------------
+# module set
+# ---------------------------------------------------------------------------
+class ModuleSet:
+    """A packed module set on the device (nectar_module_set)."""
+
+    def __init__(self, blob: torch.Tensor, widths: Sequence[int], depth: int, L: int, Hkv: int):
+        self.blob = blob
+        self.widths = [int(w) for w in widths]
+        self.depth = int(depth)
+        self.L, self.Hkv = L, Hkv
+        self._w = (ctypes.c_int32 * len(self.widths))(*self.widths)
+        self._c = _ModuleSetC(self.depth, ctypes.cast(self._w, ctypes.POINTER(ctypes.c_int32)),
+                              blob.data_ptr(), blob.numel())
+
+    def c(self):
+        return ctypes.byref(self._c)
+
+    @property
+    def bytes(self) -> int:
+        return self.blob.numel() * 2
+
+
+def packed_elems(L: int, Hkv: int, G: int, widths: Sequence[int], depth: int, d: int = 128) -> int:
+    w = (ctypes.c_int32 * L)(*widths)
+    return int(lib().nectar_module_packed_elems(Dims(L, Hkv, G, d), depth, w))
+
+
+def pack_modules(modules, widths: Sequence[int], depth: int, Hkv: int, G: int, d: int = 128,
+                 device="cuda") -> ModuleSet:
+    """Pack per-layer nets (dicts with U, V, b, Wout, c as bf16 tensors with a
+    leading Hkv axis) with nectar_module_pack and copy the blob to `device`."""
+    L_ = len(modules)
+    total = packed_elems(L_, Hkv, G, widths, depth, d)
+    if total <= 0:
+        raise NectarError(1, lib().nectar_last_error().decode())
+    blob = torch.zeros(total, dtype=torch.bfloat16)
+    keep = []
+    nets = (_NetHostC * (2 * L_))()
+    for l, layer in enumerate(modules):
+        for j, name in enumerate(("score", "target")):
+            net = layer[name]
+            nh = nets[2 * l + j]
+            for k in range(depth):
+                u = net["U"][k].detach().cpu().contiguous()
+                b = net["b"][k].detach().cpu().contiguous()
+                keep += [u, b]
+                nh.U[k] = u.data_ptr()
+                nh.b[k] = b.data_ptr()
+                if k > 0:
+                    v = net["V"][k].detach().cpu().contiguous()
+                    keep.append(v)
+                    nh.V[k] = v.data_ptr()
+            wo = net["Wout"].detach().cpu().contiguous()
+            cc = net["c"].detach().cpu().contiguous()
+            keep += [wo, cc]
+            nh.Wout, nh.c = wo.data_ptr(), cc.data_ptr()
+    w = (ctypes.c_int32 * L_)(*widths)
+    st = lib().nectar_module_pack(Dims(L_, Hkv, G, d), depth, w, nets, blob.data_ptr(), total)
+    _check(st, "nectar_module_pack")
+    dev_blob = blob.to(device) if device is not None else blob
+    return ModuleSet(dev_blob, widths, depth, L_, Hkv)
+
+
+# ---------------------------------------------------------------------------
+# (ii) module forward, (iii) merge, fused decode
+# ---------------------------------------------------------------------------
+def module_forward(mods: ModuleSet, Q, a=None, A_theta=None, stream=None):
+    """(a [L,Hkv,G,nq], A_theta [L,Hkv,G,nq,d]) fp32 for every query row."""
+    dims, nq = dims_of(Q)
+    _need(Q, "Q", torch.bfloat16)
+    if a is None:
+        a = torch.empty(Q.shape[:4], dtype=torch.float32, device=Q.device)
+    if A_theta is None:
+        A_theta = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    st = lib().nectar_module_forward(dims, mods.c(), _ptr(Q), nq, _ptr(a), _ptr(A_theta), _stream(stream))
+    _check(st, "nectar_module_forward")
+    return a, A_theta
+
+
+def _local_args(q_seq, q_pos, Kloc, Vloc, local_len):
+    for t, nm in ((q_seq, "q_seq"), (q_pos, "q_pos"), (local_len, "local_len")):
+        _need(t, nm, torch.int32)
+    for t, nm in ((Kloc, "Kloc"), (Vloc, "Vloc")):
+        _need(t, nm, torch.bfloat16)
+    B, T = Kloc.shape[2], Kloc.shape[3]
+    return B, T
+
+
+def merge_local(a, A_doc, Q, q_seq, q_pos, Kloc, Vloc, local_len, scale: Optional[float] = None, out=None,
+                stream=None):
+    """out [L,Hkv,G,nq,d] fp32: Eqs. (3.4)-(3.5) merge of (a, A_doc) with the
+    exact causal attention over Kloc, Vloc [L,Hkv,B,T,d]."""
+    dims, nq = dims_of(Q)
+    _need(Q, "Q", torch.bfloat16)
+    _need(a, "a", torch.float32)
+    _need(A_doc, "A_doc", torch.float32)
+    B, T = _local_args(q_seq, q_pos, Kloc, Vloc, local_len)
+    if scale is None:
+        scale = 1.0 / math.sqrt(dims.d)
+    if out is None:
+        out = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    st = lib().nectar_merge_local(dims, _ptr(a), _ptr(A_doc), _ptr(Q), nq, _ptr(q_seq), _ptr(q_pos), _ptr(Kloc),
+                                  _ptr(Vloc), B, T, _ptr(local_len), float(scale), _ptr(out), _stream(stream))
+    _check(st, "nectar_merge_local")
+    return out
+
+
+def decode(mods: ModuleSet, Q, q_seq, q_pos, Kloc, Vloc, local_len, scale: Optional[float] = None, out=None,
+           stream=None):
+    """Fused module forward + merge: out [L,Hkv,G,nq,d] fp32."""
+    dims, nq = dims_of(Q)
+    _need(Q, "Q", torch.bfloat16)
+    B, T = _local_args(q_seq, q_pos, Kloc, Vloc, local_len)
+    if scale is None:
+        scale = 1.0 / math.sqrt(dims.d)
+    if out is None:
+        out = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    st = lib().nectar_decode(dims, mods.c(), _ptr(Q), nq, _ptr(q_seq), _ptr(q_pos), _ptr(Kloc), _ptr(Vloc), B, T,
+                             _ptr(local_len), float(scale), _ptr(out), _stream(stream))
+    _check(st, "nectar_decode")
+    return out
+
+
+def device_error_flags(clear: bool = True) -> int:
+    """Device error word (bit 0 wait timeout, 1 bad q_seq, 2 bad local_len).
+    Synchronises the device."""
+    v = ctypes.c_int32(0)
+    _check(lib().nectar_device_error_flags(ctypes.byref(v), 1 if clear else 0), "nectar_device_error_flags")
+    return int(v.value)

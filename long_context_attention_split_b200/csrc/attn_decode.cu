@@ -1,0 +1,280 @@
+// (i) Exact cached-token attention, decode regime (few query rows per KV
+// head): Eq. (3.1) of "Nectar: Neural Estimation of Cached-Token Attention
+// via Regression" (§2.1), split over n and joined by log-sum-exp.
+//
+// Schedule.  The document of every (l, h) is cut into 64-key tiles and all
+// heads' tiles are laid end to end (head-major).  CTA c of C takes the
+// contiguous range [c*T/C, (c+1)*T/C) of that list, so every CTA streams the
+// same number of bytes whatever n and the head count are; a CTA whose range
+// crosses a head boundary emits one partial (m, l, acc) per head it touched.
+// The combine kernel then joins, for each head, the partials of the CTAs
+// that covered it -- a separate launch, so no CTA ever waits on another.
+//
+// Data movement.  One producer warp streams K and V tiles (16 KB each, whole
+// contiguous rows) into a 3-stage ring with TMA bulk copies (evict-first L2
+// policy: the document is read once); 8 consumer warps score and accumulate
+// on the CUDA cores (see common.cuh).
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nectar {
+
+constexpr int kDecTile = 64;
+constexpr int kDecWarps = 8;
+constexpr int kDecStages = 3;
+constexpr int kDecThreads = (kDecWarps + 1) * 32;
+
+__host__ __device__ __forceinline__ int first_cta_of_tile(int64_t t, int64_t total, int C) {
+  return static_cast<int>(((t + 1) * static_cast<int64_t>(C) - 1) / total);
+}
+
+template <int R>
+__host__ __device__ constexpr size_t dec_smem_bytes() {
+  return size_t(2) * kDecStages * kDecTile * kRowBytes      // K, V ring
+         + size_t(kDecWarps) * R * (kD + 2) * sizeof(float)  // cross-warp reduction
+         + 2 * kDecStages * sizeof(uint64_t);                // full / empty barriers
+}
+
+template <int R, int LPK>
+__global__ void __launch_bounds__(kDecThreads)
+cache_attn_split_kernel(const DecParams p) {
+  using St = RowState<R, LPK>;
+  constexpr int NG = St::NG;
+  constexpr int KPW = kDecTile / kDecWarps;  // keys per warp per tile
+  constexpr int KPG = KPW / NG;              // keys per group per tile
+  static_assert(KPG >= 1, "tile too small");
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + kDecStages * kDecTile * kRowBytes;
+  float* sRed = reinterpret_cast<float*>(smem + 2 * kDecStages * kDecTile * kRowBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sRed + kDecWarps * R * (kD + 2));
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kDecStages);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x;
+  const int64_t t0 = static_cast<int64_t>(c) * p.total / p.C;
+  const int64_t t1 = static_cast<int64_t>(c + 1) * p.total / p.C;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, kDecWarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kDecWarps) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      int64_t i = 0;
+      for (int64_t tt = t0; tt < t1; ++tt, ++i) {
+        const int s = static_cast<int>(i % kDecStages);
+        if (i >= kDecStages && !mbar_wait(empty0 + 8 * s, static_cast<uint32_t>(((i / kDecStages) - 1) & 1), p.err))
+          break;
+        const int64_t hd = tt / p.tph;
+        const int64_t j0 = (tt - hd * p.tph) * kDecTile;
+        const int64_t cnt = (p.n - j0 < kDecTile) ? (p.n - j0) : kDecTile;
+        const uint32_t bytes = static_cast<uint32_t>(cnt) * kRowBytes;
+        const size_t off = (static_cast<size_t>(hd) * p.n + j0) * kD;
+        mbar_arrive_expect_tx(full0 + 8 * s, 2 * bytes);
+        bulk_g2s(smem_u32(sK + s * kDecTile * kRowBytes), p.K + off, bytes, full0 + 8 * s, pol);
+        bulk_g2s(smem_u32(sV + s * kDecTile * kRowBytes), p.V + off, bytes, full0 + 8 * s, pol);
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int g = lane / LPK, t = lane % LPK;
+  St st;
+  int64_t cur = -1;
+  bool ok = true;
+
+  auto finalize = [&](int64_t hd) {
+    st.merge_groups();
+    if (g == 0) {
+      float* dst = sRed + (warp * R) * (kD + 2);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+#pragma unroll
+        for (int ci = 0; ci < St::CPL; ++ci)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dst[r * (kD + 2) + St::dim_of(t, ci, e)] = st.acc[r][ci * 8 + e];
+        if (t == 0) {
+          dst[r * (kD + 2) + kD] = st.m[r];
+          dst[r * (kD + 2) + kD + 1] = st.l[r];
+        }
+      }
+    }
+    named_bar_sync(1, kDecWarps * 32);
+    const int slot = c - first_cta_of_tile(hd * p.tph, p.total, p.C);
+    for (int it = threadIdx.x; it < R * kD; it += kDecWarps * 32) {
+      const int r = it / kD, dim = it % kD;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sRed[(w * R + r) * (kD + 2) + kD]);
+      float ls = 0.f, as = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) {
+        const float* src = sRed + (w * R + r) * (kD + 2);
+        const float wgt = exp2_shift(src[kD], M);
+        ls = fmaf(src[kD + 1], wgt, ls);
+        as = fmaf(src[dim], wgt, as);
+      }
+      const int64_t prow = (hd * p.S_max + slot) * p.rows_total + p.row0 + r;
+      p.ws_acc[prow * kD + dim] = as;
+      if (dim == 0) {
+        p.ws_ml[prow * 2] = M;
+        p.ws_ml[prow * 2 + 1] = ls;
+      }
+    }
+    named_bar_sync(1, kDecWarps * 32);
+  };
+
+  int64_t i = 0;
+  for (int64_t tt = t0; tt < t1; ++tt, ++i) {
+    const int64_t hd = tt / p.tph;
+    if (hd != cur) {
+      if (cur >= 0) finalize(cur);
+      cur = hd;
+      st.reset();
+      st.load_q(p.Q + (hd * p.rows_total + p.row0) * kD, kD, R, t, p.qmul);
+    }
+    const int s = static_cast<int>(i % kDecStages);
+    if (ok) ok = mbar_wait(full0 + 8 * s, static_cast<uint32_t>((i / kDecStages) & 1), p.err);
+    if (ok) {
+      const int64_t j0 = (tt - hd * p.tph) * kDecTile;
+      const int cnt = static_cast<int>((p.n - j0 < kDecTile) ? (p.n - j0) : kDecTile);
+      const uint8_t* kt = sK + s * kDecTile * kRowBytes;
+      const uint8_t* vt = sV + s * kDecTile * kRowBytes;
+      const uint8_t* kr[KPG];
+      const uint8_t* vr[KPG];
+      bool valid[KPG];
+#pragma unroll
+      for (int k = 0; k < KPG; ++k) {
+        const int key = warp * KPW + k * NG + g;
+        valid[k] = key < cnt;
+        kr[k] = kt + key * kRowBytes;
+        vr[k] = vt + key * kRowBytes;
+      }
+      st.template step<KPG>(kr, vr, valid, t, SmemLoader{});
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * s);
+  }
+  if (cur >= 0) finalize(cur);
+}
+
+// One warp per (head, row): join the partials of every CTA that covered the
+// head.  alpha = ln2 * (M + log2 sum_s l_s 2^{m_s - M}), A = sum_s acc_s
+// 2^{m_s - M} / sum_s l_s 2^{m_s - M}.
+__global__ void cache_attn_combine_kernel(const DecParams p, float* __restrict__ alpha,
+                                          float* __restrict__ A) {
+  const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= static_cast<int64_t>(p.heads) * p.rows_total) return;
+  const int64_t hd = gw / p.rows_total, r = gw % p.rows_total;
+  float4* out = reinterpret_cast<float4*>(A + gw * kD) + lane;
+  if (p.tph == 0) {
+    if (lane == 0) alpha[gw] = -INFINITY;
+    *out = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
+  const int f = first_cta_of_tile(hd * p.tph, p.total, p.C);
+  const int la = first_cta_of_tile(hd * p.tph + p.tph - 1, p.total, p.C);
+  float M = -INFINITY;
+  for (int s = 0; s <= la - f; ++s) M = fmaxf(M, p.ws_ml[((hd * p.S_max + s) * p.rows_total + r) * 2]);
+  float ls = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s <= la - f; ++s) {
+    const int64_t prow = (hd * p.S_max + s) * p.rows_total + r;
+    const float w = exp2_shift(p.ws_ml[prow * 2], M);
+    ls = fmaf(p.ws_ml[prow * 2 + 1], w, ls);
+    const float4 a4 = reinterpret_cast<const float4*>(p.ws_acc + prow * kD)[lane];
+    acc.x = fmaf(a4.x, w, acc.x);
+    acc.y = fmaf(a4.y, w, acc.y);
+    acc.z = fmaf(a4.z, w, acc.z);
+    acc.w = fmaf(a4.w, w, acc.w);
+  }
+  const float inv = 1.0f / ls;
+  *out = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (lane == 0) alpha[gw] = (M + log2f(ls)) * kLn2;
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+template <int R, int LPK>
+static cudaError_t launch_split(const DecParams& p, cudaStream_t stream) {
+  const size_t smem = dec_smem_bytes<R>();
+  cudaError_t e = cudaFuncSetAttribute(cache_attn_split_kernel<R, LPK>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  cache_attn_split_kernel<R, LPK><<<p.C, kDecThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+int dec_max_rows() { return 8; }
+
+size_t dec_smem_for_rows(int R) {
+  switch (R) {
+    case 1: return dec_smem_bytes<1>();
+    case 2: return dec_smem_bytes<2>();
+    case 3: return dec_smem_bytes<3>();
+    case 4: return dec_smem_bytes<4>();
+    case 5: return dec_smem_bytes<5>();
+    case 6: return dec_smem_bytes<6>();
+    case 7: return dec_smem_bytes<7>();
+    default: return dec_smem_bytes<8>();
+  }
+}
+
+// Plan: tiles per head, total tiles, CTA count and partial slots per head.
+DecPlan plan_decode(int heads, int64_t n, int num_sms, int ctas_per_sm) {
+  DecPlan pl{};
+  pl.tph = (n + kDecTile - 1) / kDecTile;
+  pl.total = static_cast<int64_t>(heads) * pl.tph;
+  int64_t C = static_cast<int64_t>(num_sms) * ctas_per_sm;
+  if (C > pl.total) C = pl.total;
+  if (C < 1) C = 1;
+  pl.C = static_cast<int>(C);
+  pl.S_max = 0;
+  if (pl.total > 0) {
+    for (int64_t hd = 0; hd < heads; ++hd) {
+      const int f = first_cta_of_tile(hd * pl.tph, pl.total, pl.C);
+      const int la = first_cta_of_tile(hd * pl.tph + pl.tph - 1, pl.total, pl.C);
+      if (la - f + 1 > pl.S_max) pl.S_max = la - f + 1;
+    }
+  }
+  return pl;
+}
+
+cudaError_t launch_cache_attn_split(const DecParams& p, int R, cudaStream_t stream) {
+  switch (R) {
+    case 1: return launch_split<1, 8>(p, stream);
+    case 2: return launch_split<2, 8>(p, stream);
+    case 3: return launch_split<3, 8>(p, stream);
+    case 4: return launch_split<4, 8>(p, stream);
+    case 5: return launch_split<5, 16>(p, stream);
+    case 6: return launch_split<6, 16>(p, stream);
+    case 7: return launch_split<7, 16>(p, stream);
+    case 8: return launch_split<8, 16>(p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_cache_attn_combine(const DecParams& p, float* alpha, float* A, cudaStream_t stream) {
+  const int64_t warps = static_cast<int64_t>(p.heads) * p.rows_total;
+  if (warps == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (warps * 32 + threads - 1) / threads;
+  cache_attn_combine_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(p, alpha, A);
+  return cudaGetLastError();
+}
+
+}  // namespace nectar

@@ -1,0 +1,219 @@
+// Shared pieces of the CUDA-core attention path.
+//
+// A group of LPK lanes owns one key at a time: lane t of the group holds the
+// 16-byte chunks t, t+LPK, ... of the key's 256-byte row (d = 128 bf16), so
+// one group reads a row with conflict-free 16-byte accesses and the lane keeps
+// DPL = 128 / LPK dimensions of every query row in registers.  A warp runs
+// NG = 32 / LPK key slots side by side.  Scores are reduced across the LPK
+// lanes with xor shuffles, so every lane of a group ends with the full score.
+//
+// Scores are kept in log2 units (q is pre-multiplied by scale * log2 e), so
+// exp becomes exp2.  The running maximum is only moved when a block maximum
+// exceeds it by more than kRescaleSlack (2^8): until then the weights
+// 2^{s - m} stay below 256, and the final normalisation divides numerator
+// and denominator by the same 2^m, so the result is the same quantity.
+#pragma once
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+
+namespace nectar {
+
+constexpr int kD = 128;                 // head dimension (the only one supported)
+constexpr int kRowBytes = kD * 2;       // one bf16 key / value row
+constexpr float kRescaleSlack = 8.0f;   // log2 units
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ float neg_inf() { return -INFINITY; }
+
+// exp2(x - m) for a finite or -inf x, 0 for x == -inf (also when m == -inf).
+__device__ __forceinline__ float exp2_shift(float x, float m) {
+  return (x == -INFINITY) ? 0.0f : ex2(x - m);
+}
+
+// Load 8 bf16 (one 16-byte chunk) as floats.
+__device__ __forceinline__ void unpack8(const uint4 w, float* f) {
+  f[0] = bf16lo(w.x); f[1] = bf16hi(w.x);
+  f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
+  f[4] = bf16lo(w.z); f[5] = bf16hi(w.z);
+  f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
+}
+
+struct SmemLoader {
+  __device__ __forceinline__ uint4 operator()(const uint8_t* p) const {
+    return *reinterpret_cast<const uint4*>(p);
+  }
+};
+struct GlobalLoader {
+  __device__ __forceinline__ uint4 operator()(const uint8_t* p) const { return ld_nc_v4(p); }
+};
+
+// Online-softmax state of R query rows held by one lane.
+template <int R, int LPK>
+struct RowState {
+  static constexpr int NG = 32 / LPK;     // key slots per warp
+  static constexpr int DPL = kD / LPK;    // dims per lane
+  static constexpr int CPL = DPL / 8;     // 16-byte chunks per lane
+
+  float q[R][DPL];
+  float m[R], l[R];
+  float acc[R][DPL];
+
+  // dimension index of acc[.][ci*8 + e] for lane-in-group t
+  __device__ __forceinline__ static int dim_of(int t, int ci, int e) { return 8 * (t + LPK * ci) + e; }
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      m[r] = -INFINITY;
+      l[r] = 0.f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[r][e] = 0.f;
+    }
+  }
+
+  // rows: pointer to row 0 of R consecutive bf16 query rows (d = 128 each),
+  // row_stride in elements.  qmul = scale * log2 e.  Rows >= nrows read 0.
+  __device__ __forceinline__ void load_q(const __nv_bfloat16* rows, int64_t row_stride, int nrows,
+                                         int t, float qmul) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+#pragma unroll
+      for (int ci = 0; ci < CPL; ++ci) {
+        float f[8];
+        if (r < nrows) {
+          const uint8_t* p = reinterpret_cast<const uint8_t*>(rows + r * row_stride) + 16 * (t + LPK * ci);
+          unpack8(ld_nc_v4(p), f);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) q[r][ci * 8 + e] = f[e] * qmul;
+      }
+    }
+  }
+
+  // Process KPG keys of this group.  krow[k] / vrow[k] point at the 256-byte
+  // rows; invalid keys are skipped (their rows are never read).
+  template <int KPG, class Loader>
+  __device__ __forceinline__ void step(const uint8_t* const* krow, const uint8_t* const* vrow,
+                                       const bool* valid, int t, const Loader& ld) {
+    float sc[KPG][R];
+    uint4 kw[KPG][CPL];
+#pragma unroll
+    for (int k = 0; k < KPG; ++k)
+#pragma unroll
+      for (int ci = 0; ci < CPL; ++ci)
+        kw[k][ci] = valid[k] ? ld(krow[k] + 16 * (t + LPK * ci)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int k = 0; k < KPG; ++k) {
+      float part[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) part[r] = 0.f;
+#pragma unroll
+      for (int ci = 0; ci < CPL; ++ci) {
+        float kf[8];
+        unpack8(kw[k][ci], kf);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) part[r] = fmaf(q[r][ci * 8 + e], kf[e], part[r]);
+      }
+#pragma unroll
+      for (int off = LPK / 2; off >= 1; off >>= 1)
+#pragma unroll
+        for (int r = 0; r < R; ++r) part[r] += __shfl_xor_sync(0xffffffffu, part[r], off);
+#pragma unroll
+      for (int r = 0; r < R; ++r) sc[k][r] = valid[k] ? part[r] : -INFINITY;
+    }
+    // block maximum, lazy rescale
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float bm = sc[0][r];
+#pragma unroll
+      for (int k = 1; k < KPG; ++k) bm = fmaxf(bm, sc[k][r]);
+      if (bm > m[r] + kRescaleSlack) {
+        const float corr = exp2_shift(m[r], bm);
+        l[r] *= corr;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[r][e] *= corr;
+        m[r] = bm;
+      }
+    }
+    float pw[KPG][R];
+#pragma unroll
+    for (int k = 0; k < KPG; ++k)
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        pw[k][r] = exp2_shift(sc[k][r], m[r]);
+        l[r] += pw[k][r];
+      }
+    uint4 vw[KPG][CPL];
+#pragma unroll
+    for (int k = 0; k < KPG; ++k)
+#pragma unroll
+      for (int ci = 0; ci < CPL; ++ci)
+        vw[k][ci] = valid[k] ? ld(vrow[k] + 16 * (t + LPK * ci)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int k = 0; k < KPG; ++k)
+#pragma unroll
+      for (int ci = 0; ci < CPL; ++ci) {
+        float vf[8];
+        unpack8(vw[k][ci], vf);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[r][ci * 8 + e] = fmaf(pw[k][r], vf[e], acc[r][ci * 8 + e]);
+      }
+  }
+
+  // Join the NG groups of the warp (xor over lane bits >= LPK); afterwards
+  // every group holds the warp's combined state.
+  __device__ __forceinline__ void merge_groups() {
+#pragma unroll
+    for (int off = LPK; off < 32; off <<= 1) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m[r], off);
+        const float lo = __shfl_xor_sync(0xffffffffu, l[r], off);
+        const float M = fmaxf(m[r], mo);
+        const float wa = exp2_shift(m[r], M), wb = exp2_shift(mo, M);
+        l[r] = l[r] * wa + lo * wb;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) {
+          const float ao = __shfl_xor_sync(0xffffffffu, acc[r][e], off);
+          acc[r][e] = acc[r][e] * wa + ao * wb;
+        }
+        m[r] = M;
+      }
+    }
+  }
+};
+
+// Visible local tokens of a query token; flags bad metadata (reading of
+// §2.2: token i sees local j <= q_pos[i], j < local_len[q_seq[i]]).
+__device__ __forceinline__ int visible_local(const int32_t* q_seq, const int32_t* q_pos,
+                                             const int32_t* local_len, int64_t i, int B, int T,
+                                             int* seq_out, int* err) {
+  const int b = q_seq[i];
+  *seq_out = b;
+  if (b < 0 || b >= B) {
+    record_error(err, DEVERR_BAD_SEQ);
+    return 0;
+  }
+  int len = local_len[b];
+  if (len < 0 || len > T) {
+    record_error(err, DEVERR_BAD_LEN);
+    len = len < 0 ? 0 : T;
+  }
+  int nv = q_pos[i] + 1;
+  if (nv > len) nv = len;
+  if (nv < 0) nv = 0;
+  return nv;
+}
+
+}  // namespace nectar

@@ -1,0 +1,92 @@
+// Internal launch interface between the C ABI (nectar_api.cu) and the
+// kernels.  Not part of the public header.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nectar {
+
+// ----- (i) split-n decode attention (CUDA cores) + LSE combine -------------
+struct DecParams {
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  const __nv_bfloat16* Q;
+  int64_t n;
+  int heads;
+  int64_t rows_total;   // query rows per head (G * nq)
+  int row0;             // first row handled by this launch
+  int64_t tph;          // 64-key tiles per head
+  int64_t total;        // heads * tph
+  int C;                // CTAs of the split launch
+  int S_max;            // partial slots per head
+  float qmul;           // scale * log2(e)
+  float* ws_ml;         // [heads][S_max][rows_total][2]  (m in log2 units, l)
+  float* ws_acc;        // [heads][S_max][rows_total][128]
+  int* err;             // device error word
+};
+
+struct DecPlan {
+  int64_t tph, total;
+  int C, S_max;
+};
+
+DecPlan plan_decode(int heads, int64_t n, int num_sms, int ctas_per_sm);
+int dec_max_rows();
+size_t dec_smem_for_rows(int R);
+cudaError_t launch_cache_attn_split(const DecParams& p, int R, cudaStream_t stream);
+cudaError_t launch_cache_attn_combine(const DecParams& p, float* alpha, float* A, cudaStream_t stream);
+
+// ----- (iii) merge with exact causal local attention -----------------------
+struct MergeParams {
+  const float* a;
+  const float* A_doc;
+  const __nv_bfloat16* Q;
+  const int32_t* q_seq;
+  const int32_t* q_pos;
+  const __nv_bfloat16* Kloc;
+  const __nv_bfloat16* Vloc;
+  const int32_t* local_len;
+  float* out;
+  int heads, G;
+  int64_t nq;
+  int B, T;
+  float qmul;           // scale * log2(e)
+  int* err;             // device error word
+};
+cudaError_t launch_merge_local(const MergeParams& p, cudaStream_t stream);
+
+// ----- (ii) module forward and the fused decode (tcgen05) ------------------
+constexpr int kModMaxLayers = 256;
+struct ModParams {
+  int Hkv, G, depth;
+  int64_t nq;
+  int N, TPC, nblk, Hmax, tmem_cols;
+  const __nv_bfloat16* blob;
+  const __nv_bfloat16* Q;
+  float* a_out;         // module forward outputs
+  float* A_out;
+  // fused decode
+  const int32_t* q_seq;
+  const int32_t* q_pos;
+  const __nv_bfloat16* Kloc;
+  const __nv_bfloat16* Vloc;
+  const int32_t* local_len;
+  int B, T;
+  float qmul;
+  float* out;
+  int* err;
+  int32_t width[kModMaxLayers];
+  int64_t layer_base[kModMaxLayers];   // blob element offset of layer l
+  uint8_t order[kModMaxLayers];        // layers by decreasing width
+};
+struct ModShape {
+  int TPC, N, nblk, tmem_cols;
+  size_t smem;
+};
+ModShape mod_shape(int G, int64_t nq, int Hmax, bool fuse);
+cudaError_t launch_module(const CUtensorMap& tw, const CUtensorMap& tq, const ModParams& p, int units, size_t smem,
+                          bool fuse, cudaStream_t stream);
+
+}  // namespace nectar

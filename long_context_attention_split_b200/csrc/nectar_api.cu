@@ -1,0 +1,504 @@
+// C ABI of libnectar.so: argument validation, work planning and dispatch.
+// Every entry point validates on the host and enqueues nothing on error.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
+#include "../../include/nectar.h"
+#include "common.cuh"
+#include "kernels.h"
+#include "module_layout.h"
+
+namespace nectar {
+// The device error word (see nectar_device_error_flags).  Kernels get its
+// address through their parameters.
+__device__ int g_error_word = 0;
+}
+
+using namespace nectar;
+
+namespace {
+
+thread_local char t_last_error[512] = "";
+
+nectar_status fail(nectar_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof t_last_error, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+nectar_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(NECTAR_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+nectar_status check_dims(const nectar_dims& d) {
+  if (d.L < 1 || d.Hkv < 1 || d.G < 1) return fail(NECTAR_ERR_INVALID_ARG, "dims: L, Hkv, G must be >= 1");
+  if (d.d != kD) return fail(NECTAR_ERR_UNSUPPORTED, "dims: d = %d, only d = 128 is supported", d.d);
+  if (static_cast<int64_t>(d.L) * d.Hkv > (1 << 20)) return fail(NECTAR_ERR_INVALID_ARG, "dims: too many heads");
+  return NECTAR_OK;
+}
+
+nectar_status check_ptr(const void* p, const char* name) {
+  if (p == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(NECTAR_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return NECTAR_OK;
+}
+
+#define NECTAR_TRY(expr)              \
+  do {                                \
+    nectar_status _s = (expr);        \
+    if (_s != NECTAR_OK) return _s;   \
+  } while (0)
+
+struct DeviceInfo {
+  int sms = 0;
+  int* err = nullptr;   // device address of g_error_word on this device
+};
+
+DeviceInfo device_info() {
+  static std::mutex mu;
+  static std::vector<DeviceInfo> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DeviceInfo{};
+  std::lock_guard<std::mutex> lk(mu);
+  if (static_cast<int>(cache.size()) <= dev) cache.resize(dev + 1);
+  if (cache[dev].sms == 0) {
+    int sms = 0;
+    void* err = nullptr;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaGetSymbolAddress(&err, nectar::g_error_word) != cudaSuccess)
+      return DeviceInfo{};
+    cache[dev].err = static_cast<int*>(err);
+    cache[dev].sms = sms;
+  }
+  return cache[dev];
+}
+
+// CTAs of the split kernel resident per SM (shared memory bound).
+int dec_ctas_per_sm(int R) {
+  const size_t per = dec_smem_for_rows(R) + 1024;
+  int c = static_cast<int>((228 * 1024) / per);
+  return c < 1 ? 1 : (c > 2 ? 2 : c);
+}
+
+// Row blocks handled by one launch of the CUDA-core split kernel.
+int dec_row_block(int64_t rows) { return rows < dec_max_rows() ? static_cast<int>(rows) : dec_max_rows(); }
+
+DecPlan cache_attn_plan(const nectar_dims& d, int64_t n, int64_t nq, int sms) {
+  const int64_t rows = static_cast<int64_t>(d.G) * nq;
+  const int R = dec_row_block(rows);
+  return plan_decode(d.L * d.Hkv, n, sms, dec_ctas_per_sm(R < 1 ? 1 : R));
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// link-time dependency on libcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims / strides innermost first,
+// strides in bytes for dims 1..rank-1.
+nectar_status make_tmap(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                        const cuuint64_t* strides, const cuuint32_t* box, const char* what) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return fail(NECTAR_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NECTAR_ERR_CUDA, "tensor map for %s: CUresult %d", what, static_cast<int>(r));
+  return NECTAR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nectar_version(void) { return "0.1.0"; }
+
+const char* nectar_status_string(nectar_status s) {
+  switch (s) {
+    case NECTAR_OK: return "ok";
+    case NECTAR_ERR_INVALID_ARG: return "invalid argument";
+    case NECTAR_ERR_UNSUPPORTED: return "unsupported";
+    case NECTAR_ERR_WORKSPACE: return "workspace too small";
+    case NECTAR_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* nectar_last_error(void) { return t_last_error; }
+
+nectar_status nectar_device_error_flags(int32_t* flags, int32_t clear) {
+  if (flags == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "flags is NULL");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "nectar_device_error_flags");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, nectar::g_error_word, sizeof v);
+  if (e != cudaSuccess) return cuda_fail(e, "nectar_device_error_flags");
+  *flags = v;
+  if (clear) {
+    const int z = 0;
+    e = cudaMemcpyToSymbol(nectar::g_error_word, &z, sizeof z);
+    if (e != cudaSuccess) return cuda_fail(e, "nectar_device_error_flags");
+  }
+  return NECTAR_OK;
+}
+
+// ---------------------------------------------------------------------------
+// (i) exact cached-token attention
+// ---------------------------------------------------------------------------
+size_t nectar_cache_attn_workspace_size(nectar_dims dims, int64_t n, int64_t nq) {
+  if (check_dims(dims) != NECTAR_OK || n < 0 || nq < 0) return 0;
+  const int64_t rows = static_cast<int64_t>(dims.G) * nq;
+  if (rows == 0 || n == 0) return 0;
+  const DeviceInfo di = device_info();
+  if (di.sms == 0) return 0;
+  const DecPlan pl = cache_attn_plan(dims, n, nq, di.sms);
+  const int64_t prow = static_cast<int64_t>(dims.L) * dims.Hkv * pl.S_max * rows;
+  return static_cast<size_t>(prow) * (kD + 2) * sizeof(float) + 256;
+}
+
+nectar_status nectar_cache_attn_lse(nectar_dims dims, const nectar_bf16* K, const nectar_bf16* V,
+                                    int64_t n, const nectar_bf16* Q, int64_t nq, float scale,
+                                    float* alpha, float* A, void* workspace, size_t workspace_bytes,
+                                    nectar_stream_t stream) {
+  NECTAR_TRY(check_dims(dims));
+  if (n < 0 || nq < 0) return fail(NECTAR_ERR_INVALID_ARG, "n and nq must be >= 0");
+  if (!(scale == scale)) return fail(NECTAR_ERR_INVALID_ARG, "scale is NaN");
+  if (nq == 0) return NECTAR_OK;
+  const int heads = dims.L * dims.Hkv;
+  const int64_t rows = static_cast<int64_t>(dims.G) * nq;
+  if (rows > (int64_t(1) << 30)) return fail(NECTAR_ERR_INVALID_ARG, "too many query rows");
+  NECTAR_TRY(check_ptr(Q, "Q"));
+  if (alpha == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "alpha is NULL");
+  NECTAR_TRY(check_ptr(A, "A"));
+  if (n > 0) {
+    NECTAR_TRY(check_ptr(K, "K"));
+    NECTAR_TRY(check_ptr(V, "V"));
+  }
+  const DeviceInfo di = device_info();
+  if (di.sms == 0) return fail(NECTAR_ERR_CUDA, "no CUDA device");
+
+  DecParams p{};
+  p.K = reinterpret_cast<const __nv_bfloat16*>(K);
+  p.V = reinterpret_cast<const __nv_bfloat16*>(V);
+  p.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  p.n = n;
+  p.heads = heads;
+  p.rows_total = rows;
+  p.qmul = scale * kLog2e;
+  p.err = di.err;
+  const DecPlan pl = cache_attn_plan(dims, n, nq, di.sms);
+  p.tph = pl.tph;
+  p.total = pl.total;
+  p.C = pl.C;
+  p.S_max = pl.S_max;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (n == 0) {
+    cudaError_t e = launch_cache_attn_combine(p, alpha, A, st);
+    return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "cache_attn (n = 0)");
+  }
+  const size_t need = nectar_cache_attn_workspace_size(dims, n, nq);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(NECTAR_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
+  if (!aligned16(workspace)) return fail(NECTAR_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+  const int64_t prow = static_cast<int64_t>(heads) * pl.S_max * rows;
+  p.ws_acc = reinterpret_cast<float*>(workspace);
+  p.ws_ml = p.ws_acc + prow * kD;
+
+  const int RB = dec_row_block(rows);
+  for (int64_t r0 = 0; r0 < rows; r0 += RB) {
+    p.row0 = static_cast<int>(r0);
+    const int R = static_cast<int>((rows - r0) < RB ? (rows - r0) : RB);
+    cudaError_t e = launch_cache_attn_split(p, R, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cache_attn split kernel");
+  }
+  cudaError_t e = launch_cache_attn_combine(p, alpha, A, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cache_attn combine kernel");
+  return NECTAR_OK;
+}
+
+// ---------------------------------------------------------------------------
+// (iii) merge with local attention
+// ---------------------------------------------------------------------------
+static nectar_status check_local(const int32_t* q_seq, const int32_t* q_pos, const nectar_bf16* Kloc,
+                                 const nectar_bf16* Vloc, int32_t B, int32_t T_max,
+                                 const int32_t* local_len) {
+  if (B < 0 || T_max < 0) return fail(NECTAR_ERR_INVALID_ARG, "B and T_max must be >= 0");
+  if (q_seq == nullptr || q_pos == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "q_seq / q_pos is NULL");
+  if (B > 0) {
+    if (local_len == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "local_len is NULL");
+    if (T_max > 0) {
+      NECTAR_TRY(check_ptr(Kloc, "Kloc"));
+      NECTAR_TRY(check_ptr(Vloc, "Vloc"));
+    }
+  }
+  return NECTAR_OK;
+}
+
+nectar_status nectar_merge_local(nectar_dims dims, const float* a, const float* A_doc, const nectar_bf16* Q,
+                                 int64_t nq, const int32_t* q_seq, const int32_t* q_pos,
+                                 const nectar_bf16* Kloc, const nectar_bf16* Vloc, int32_t B, int32_t T_max,
+                                 const int32_t* local_len, float scale, float* out, nectar_stream_t stream) {
+  NECTAR_TRY(check_dims(dims));
+  if (nq < 0) return fail(NECTAR_ERR_INVALID_ARG, "nq must be >= 0");
+  if (nq == 0) return NECTAR_OK;
+  if (!(scale == scale)) return fail(NECTAR_ERR_INVALID_ARG, "scale is NaN");
+  if (a == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "a is NULL");
+  NECTAR_TRY(check_ptr(A_doc, "A_doc"));
+  NECTAR_TRY(check_ptr(Q, "Q"));
+  NECTAR_TRY(check_ptr(out, "out"));
+  NECTAR_TRY(check_local(q_seq, q_pos, Kloc, Vloc, B, T_max, local_len));
+  if (static_cast<int64_t>(dims.L) * dims.Hkv * nq * ((dims.G + 7) / 8) > 0x7fffffffLL)
+    return fail(NECTAR_ERR_INVALID_ARG, "too many (head, token) units");
+  MergeParams p{};
+  p.a = a;
+  p.A_doc = A_doc;
+  p.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  p.q_seq = q_seq;
+  p.q_pos = q_pos;
+  p.Kloc = reinterpret_cast<const __nv_bfloat16*>(Kloc);
+  p.Vloc = reinterpret_cast<const __nv_bfloat16*>(Vloc);
+  p.local_len = local_len;
+  p.out = out;
+  p.heads = dims.L * dims.Hkv;
+  p.G = dims.G;
+  p.nq = nq;
+  p.B = B;
+  p.T = T_max;
+  p.qmul = scale * kLog2e;
+  const DeviceInfo di = device_info();
+  if (di.sms == 0) return fail(NECTAR_ERR_CUDA, "no CUDA device");
+  p.err = di.err;
+  cudaError_t e = launch_merge_local(p, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "merge_local kernel");
+}
+
+// ---------------------------------------------------------------------------
+// module packing (host only)
+// ---------------------------------------------------------------------------
+static nectar_status check_modules_shape(const nectar_dims& dims, int32_t depth, const int32_t* width) {
+  NECTAR_TRY(check_dims(dims));
+  if (depth < 1 || depth > NECTAR_MAX_DEPTH)
+    return fail(NECTAR_ERR_UNSUPPORTED, "depth %d outside [1, %d]", depth, NECTAR_MAX_DEPTH);
+  if (width == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "width is NULL");
+  if (dims.L > NECTAR_MAX_LAYERS) return fail(NECTAR_ERR_UNSUPPORTED, "L = %d > %d", dims.L, NECTAR_MAX_LAYERS);
+  for (int l = 0; l < dims.L; ++l) {
+    const int H = width[l];
+    if (H < 16 || H > NECTAR_MAX_WIDTH || H % 16 != 0)
+      return fail(NECTAR_ERR_UNSUPPORTED, "width[%d] = %d: need a multiple of 16 in [16, %d]", l, H,
+                  NECTAR_MAX_WIDTH);
+  }
+  return NECTAR_OK;
+}
+
+int64_t nectar_module_packed_elems(nectar_dims dims, int32_t depth, const int32_t* width) {
+  if (check_modules_shape(dims, depth, width) != NECTAR_OK) return 0;
+  int64_t tot = 0;
+  for (int l = 0; l < dims.L; ++l) tot += static_cast<int64_t>(dims.Hkv) * layout::head_elems(width[l], depth);
+  return tot;
+}
+
+nectar_status nectar_module_pack(nectar_dims dims, int32_t depth, const int32_t* width,
+                                 const nectar_net_host* nets, nectar_bf16* blob, int64_t blob_elems) {
+  NECTAR_TRY(check_modules_shape(dims, depth, width));
+  if (nets == nullptr || blob == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "nets / blob is NULL");
+  const int64_t need = nectar_module_packed_elems(dims, depth, width);
+  if (blob_elems < need) return fail(NECTAR_ERR_INVALID_ARG, "blob has %lld elements, %lld needed",
+                                     (long long)blob_elems, (long long)need);
+  for (int l = 0; l < dims.L; ++l)
+    for (int net = 0; net < 2; ++net) {
+      const nectar_net_host& nh = nets[2 * l + net];
+      for (int k = 0; k < depth; ++k) {
+        if (nh.U[k] == nullptr || nh.b[k] == nullptr || (k > 0 && nh.V[k] == nullptr))
+          return fail(NECTAR_ERR_INVALID_ARG, "layer %d net %d: missing U/V/b[%d]", l, net, k);
+      }
+      if (nh.Wout == nullptr || nh.c == nullptr)
+        return fail(NECTAR_ERR_INVALID_ARG, "layer %d net %d: missing Wout / c", l, net);
+    }
+  memset(blob, 0, sizeof(nectar_bf16) * need);
+  int64_t base = 0;
+  for (int l = 0; l < dims.L; ++l) {
+    const int H = width[l];
+    const int64_t per_head = layout::head_elems(H, depth);
+    for (int h = 0; h < dims.Hkv; ++h) {
+      for (int net = 0; net < 2; ++net) {
+        const nectar_net_host& nh = nets[2 * l + net];
+        const int dout = net == 0 ? 1 : kD;
+        const int64_t nb = base + h * per_head + (net ? layout::net_elems(H, depth, 1) : 0);
+        for (int k = 0; k < depth; ++k) {
+          const int Kk = layout::hidden_k(H, k);
+          // logical W_k[i][c]: c < d from V_k (k>=1) or U_0 (k=0); c >= d from U_k
+          nectar_bf16* W = blob + nb + layout::hidden_w_off(H, depth, k);
+          for (int i = 0; i < H; ++i)
+            for (int c = 0; c < Kk; ++c) {
+              nectar_bf16 v;
+              if (k == 0) v = nh.U[0][(static_cast<int64_t>(h) * H + i) * kD + c];
+              else if (c < kD) v = nh.V[k][(static_cast<int64_t>(h) * H + i) * kD + c];
+              else v = nh.U[k][(static_cast<int64_t>(h) * H + i) * H + (c - kD)];
+              W[layout::chunked_index(H, c, i)] = v;
+            }
+          nectar_bf16* bb = blob + nb + layout::hidden_b_off(H, depth, k);
+          for (int i = 0; i < H; ++i) bb[i] = nh.b[k][static_cast<int64_t>(h) * H + i];
+        }
+        nectar_bf16* Wo = blob + nb + layout::out_w_off(H, depth);
+        if (dout == 1) {
+          for (int i = 0; i < H; ++i) Wo[i] = nh.Wout[static_cast<int64_t>(h) * H + i];
+        } else {
+          for (int o = 0; o < dout; ++o)
+            for (int c = 0; c < H; ++c)
+              Wo[layout::chunked_index(kD, c, o)] = nh.Wout[(static_cast<int64_t>(h) * dout + o) * H + c];
+        }
+        nectar_bf16* cb = blob + nb + layout::out_b_off(H, depth, dout);
+        for (int o = 0; o < dout; ++o) cb[o] = nh.c[static_cast<int64_t>(h) * dout + o];
+      }
+    }
+    base += static_cast<int64_t>(dims.Hkv) * per_head;
+  }
+  return NECTAR_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// (ii) module forward and the fused decode
+// ---------------------------------------------------------------------------
+namespace {
+
+nectar_status prepare_modules(const nectar_dims& dims, const nectar_module_set* mods, const nectar_bf16* Q,
+                              int64_t nq, bool fuse, ModParams* p, CUtensorMap* tw, CUtensorMap* tq,
+                              ModShape* sh) {
+  if (mods == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "mods is NULL");
+  NECTAR_TRY(check_modules_shape(dims, mods->depth, mods->width));
+  if (dims.G > 64) return fail(NECTAR_ERR_UNSUPPORTED, "G = %d > 64", dims.G);
+  NECTAR_TRY(check_ptr(mods->weights, "mods->weights"));
+  const int64_t need = nectar_module_packed_elems(dims, mods->depth, mods->width);
+  if (mods->weights_elems < need)
+    return fail(NECTAR_ERR_INVALID_ARG, "weights_elems = %lld, the widths need %lld", (long long)mods->weights_elems,
+                (long long)need);
+  NECTAR_TRY(check_ptr(Q, "Q"));
+  if (nq > 0x7fffffffLL) return fail(NECTAR_ERR_INVALID_ARG, "nq too large");
+  const DeviceInfo di = device_info();
+  if (di.sms == 0) return fail(NECTAR_ERR_CUDA, "no CUDA device");
+  memset(p, 0, sizeof(*p));
+  p->Hkv = dims.Hkv;
+  p->G = dims.G;
+  p->depth = mods->depth;
+  p->nq = nq;
+  p->blob = reinterpret_cast<const __nv_bfloat16*>(mods->weights);
+  p->Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  p->err = di.err;
+  int Hmax = 0;
+  int64_t base = 0;
+  for (int l = 0; l < dims.L; ++l) {
+    p->width[l] = mods->width[l];
+    p->layer_base[l] = base;
+    base += static_cast<int64_t>(dims.Hkv) * layout::head_elems(mods->width[l], mods->depth);
+    if (mods->width[l] > Hmax) Hmax = mods->width[l];
+  }
+  // widest layers first: their CTAs run longest
+  std::vector<int> ord(dims.L);
+  for (int l = 0; l < dims.L; ++l) ord[l] = l;
+  std::stable_sort(ord.begin(), ord.end(), [&](int a, int b) { return mods->width[a] > mods->width[b]; });
+  for (int l = 0; l < dims.L; ++l) p->order[l] = static_cast<uint8_t>(ord[l]);
+  p->Hmax = Hmax;
+  *sh = mod_shape(dims.G, nq, Hmax, fuse);
+  if (sh->smem > 227 * 1024) return fail(NECTAR_ERR_UNSUPPORTED, "width %d needs too much shared memory", Hmax);
+  p->N = sh->N;
+  p->TPC = sh->TPC;
+  p->nblk = sh->nblk;
+  p->tmem_cols = sh->tmem_cols;
+  // weights: the blob viewed as [rows][64]; box = 64 columns x 128 rows
+  {
+    const cuuint64_t dimsw[2] = {64, static_cast<cuuint64_t>(mods->weights_elems / 64)};
+    const cuuint64_t strw[1] = {128};
+    const cuuint32_t boxw[2] = {64, 128};
+    NECTAR_TRY(make_tmap(tw, mods->weights, 2, dimsw, strw, boxw, "module weights"));
+  }
+  // queries: [heads][G][nq][128]; box = 64 columns x TPC tokens x G heads x 1
+  {
+    const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
+    const cuuint64_t dimsq[4] = {128, static_cast<cuuint64_t>(nq), static_cast<cuuint64_t>(dims.G),
+                                 static_cast<cuuint64_t>(heads)};
+    const cuuint64_t strq[3] = {256, static_cast<cuuint64_t>(nq) * 256, static_cast<cuuint64_t>(nq) * 256 * dims.G};
+    const cuuint32_t boxq[4] = {64, static_cast<cuuint32_t>(sh->TPC), static_cast<cuuint32_t>(dims.G), 1};
+    NECTAR_TRY(make_tmap(tq, Q, 4, dimsq, strq, boxq, "queries"));
+  }
+  return NECTAR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nectar_status nectar_module_forward(nectar_dims dims, const nectar_module_set* mods, const nectar_bf16* Q, int64_t nq,
+                                    float* a, float* A_theta, nectar_stream_t stream) {
+  NECTAR_TRY(check_dims(dims));
+  if (nq < 0) return fail(NECTAR_ERR_INVALID_ARG, "nq must be >= 0");
+  if (nq == 0) return NECTAR_OK;
+  if (a == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "a is NULL");
+  NECTAR_TRY(check_ptr(A_theta, "A_theta"));
+  ModParams p;
+  CUtensorMap tw, tq;
+  ModShape sh;
+  NECTAR_TRY(prepare_modules(dims, mods, Q, nq, false, &p, &tw, &tq, &sh));
+  p.a_out = a;
+  p.A_out = A_theta;
+  const int units = dims.L * dims.Hkv * sh.nblk;
+  cudaError_t e = launch_module(tw, tq, p, units, sh.smem, false, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "module kernel");
+}
+
+nectar_status nectar_decode(nectar_dims dims, const nectar_module_set* mods, const nectar_bf16* Q, int64_t nq,
+                            const int32_t* q_seq, const int32_t* q_pos, const nectar_bf16* Kloc,
+                            const nectar_bf16* Vloc, int32_t B, int32_t T_max, const int32_t* local_len,
+                            float scale, float* out, nectar_stream_t stream) {
+  NECTAR_TRY(check_dims(dims));
+  if (nq < 0) return fail(NECTAR_ERR_INVALID_ARG, "nq must be >= 0");
+  if (nq == 0) return NECTAR_OK;
+  if (!(scale == scale)) return fail(NECTAR_ERR_INVALID_ARG, "scale is NaN");
+  NECTAR_TRY(check_ptr(out, "out"));
+  NECTAR_TRY(check_local(q_seq, q_pos, Kloc, Vloc, B, T_max, local_len));
+  ModParams p;
+  CUtensorMap tw, tq;
+  ModShape sh;
+  NECTAR_TRY(prepare_modules(dims, mods, Q, nq, true, &p, &tw, &tq, &sh));
+  p.q_seq = q_seq;
+  p.q_pos = q_pos;
+  p.Kloc = reinterpret_cast<const __nv_bfloat16*>(Kloc);
+  p.Vloc = reinterpret_cast<const __nv_bfloat16*>(Vloc);
+  p.local_len = local_len;
+  p.B = B;
+  p.T = T_max;
+  p.qmul = scale * kLog2e;
+  p.out = out;
+  const int units = dims.L * dims.Hkv * sh.nblk;
+  cudaError_t e = launch_module(tw, tq, p, units, sh.smem, true, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "decode kernel");
+}
+
+}  // extern "C"

@@ -1,0 +1,120 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+that include/nectar.h declares, validates arguments on the host, and packs
+module weights in the documented layout."""
+import ctypes
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import long_context_attention_split_b200 as nx
+from nectar_inputs import make_modules
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from long_context_attention_split_b200 import build
+    build.build()
+
+
+def test_exports_every_header_function():
+    names = nx.header_functions()
+    assert len(names) >= 10
+    lib = ctypes.CDLL(nx.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    for n in ["nectar_cache_attn_lse", "nectar_module_forward", "nectar_merge_local", "nectar_decode"]:
+        assert n in names
+
+
+def test_status_strings_and_version():
+    L = nx.lib()
+    for s in range(5):
+        assert L.nectar_status_string(s)
+    assert nx.version().count(".") == 2
+
+
+def test_host_validation_without_device():
+    L = nx.lib()
+    bad_d = nx.Dims(1, 1, 1, 64)
+    st = L.nectar_cache_attn_lse(bad_d, None, None, 10, None, 1, 1.0, None, None, None, 0, None)
+    assert st == 2 and b"d = 64" in L.nectar_last_error()
+    st = L.nectar_cache_attn_lse(nx.Dims(0, 1, 1, 128), None, None, 10, None, 1, 1.0, None, None, None, 0, None)
+    assert st == 1
+    st = L.nectar_cache_attn_lse(nx.Dims(1, 1, 1, 128), None, None, -1, None, 1, 1.0, None, None, None, 0, None)
+    assert st == 1
+    # nq == 0 is a no-op even with no buffers
+    assert L.nectar_cache_attn_lse(nx.Dims(1, 1, 1, 128), None, None, 5, None, 0, 1.0, None, None, None, 0, None) == 0
+    assert L.nectar_cache_attn_workspace_size(bad_d, 10, 1) == 0
+    st = L.nectar_merge_local(nx.Dims(1, 1, 1, 128), None, None, None, 1, None, None, None, None, 1, 1, None, 1.0,
+                              None, None)
+    assert st == 1
+    w = (ctypes.c_int32 * 2)(64, 40)      # 40 is not a multiple of 16
+    assert L.nectar_module_packed_elems(nx.Dims(2, 1, 1, 128), 2, w) == 0
+    w = (ctypes.c_int32 * 1)(2048)        # too wide
+    assert L.nectar_module_packed_elems(nx.Dims(1, 1, 1, 128), 2, w) == 0
+    w = (ctypes.c_int32 * 1)(64)
+    assert L.nectar_module_packed_elems(nx.Dims(1, 1, 1, 128), 0, w) == 0
+
+
+# -- independent reader of the packed layout (as documented in module_layout.h) --
+def r64(x):
+    return (x + 63) // 64 * 64
+
+
+def kch(K):
+    return (K + 63) // 64
+
+
+def read_chunked(blob, off, rows, K):
+    """K-chunked [ceil(K/64)][rows][64] -> dense [rows][K]."""
+    n = kch(K) * rows * 64
+    a = blob[off:off + n].reshape(kch(K), rows, 64)
+    return np.concatenate(list(a), axis=1)[:, :K], off + n
+
+
+def read_net(blob, off, H, depth, dout, d=128):
+    out = {"W": [], "b": []}
+    for k in range(depth):
+        Kk = d if k == 0 else d + H
+        W, off = read_chunked(blob, off, H, Kk)
+        out["W"].append(W)
+        out["b"].append(blob[off:off + H]); off += r64(H)
+    if dout == 1:
+        out["Wout"] = blob[off:off + H][None]; off += r64(H)
+        out["c"] = blob[off:off + 1]; off += 64
+    else:
+        W, off = read_chunked(blob, off, d, H)
+        out["Wout"] = W
+        out["c"] = blob[off:off + d]; off += d
+    return out, off
+
+
+@pytest.mark.parametrize("widths,depth,hkv", [([64, 32], 2, 2), ([48], 3, 1), ([16, 208], 1, 3)])
+def test_pack_layout(widths, depth, hkv):
+    mods = make_modules(len(widths), hkv, widths, 128, seed=3, device="cpu", depth=depth)
+    ms = nx.pack_modules(mods, widths, depth, hkv, G=2, device=None)
+    blob = ms.blob.float().numpy()
+    assert ms.blob.numel() == nx.packed_elems(len(widths), hkv, 2, widths, depth)
+    off = 0
+    for l, H in enumerate(widths):
+        for h in range(hkv):
+            for name, dout in (("score", 1), ("target", 128)):
+                net = mods[l][name]
+                got, off = read_net(blob, off, H, depth, dout)
+                for k in range(depth):
+                    if k == 0:
+                        ref = net["U"][0][h].float().numpy()
+                    else:
+                        ref = np.concatenate([net["V"][k][h].float().numpy(), net["U"][k][h].float().numpy()], 1)
+                    np.testing.assert_array_equal(got["W"][k], ref)
+                    np.testing.assert_array_equal(got["b"][k], net["b"][k][h].float().numpy())
+                np.testing.assert_array_equal(got["Wout"], net["Wout"][h].float().numpy())
+                np.testing.assert_array_equal(got["c"], net["c"][h].float().numpy())
+    assert off == blob.size
+    # padding (K columns beyond d + H inside the last chunk) is zero
+    H = widths[0]
+    if depth >= 2 and (128 + H) % 64:
+        W1, _ = read_chunked(blob, r64(0) + kch(128) * H * 64 + r64(H), H, r64(128 + H))
+        assert np.all(W1[:, 128 + H:] == 0)
