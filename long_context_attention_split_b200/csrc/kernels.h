@@ -38,6 +38,32 @@ size_t dec_smem_for_rows(int R);
 cudaError_t launch_cache_attn_split(const DecParams& p, int R, cudaStream_t stream);
 cudaError_t launch_cache_attn_combine(const DecParams& p, float* alpha, float* A, cudaStream_t stream);
 
+// ----- (i) tensor-core path for many query rows per head -------------------
+struct TcParams {
+  int64_t n;
+  int heads;
+  int64_t rows_total;
+  int qtiles;           // 128-row query tiles per head
+  int64_t tph;          // 128-key tiles per head
+  int64_t total;        // heads * qtiles * tph
+  int C, S_max;
+  float qmul;           // scale * log2(e)
+  float* alpha;
+  float* A;
+  float* ws_ml;         // [C][S_max][128][2]
+  float* ws_acc;        // [C][S_max][128][128]
+  int* err;
+};
+struct TcPlan {
+  int qtiles;
+  int64_t tph, total;
+  int C, S_max;
+  size_t ws_bytes, smem;
+};
+TcPlan plan_tc(int heads, int64_t n, int64_t rows, int num_sms);
+cudaError_t launch_cache_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                 const TcParams& p, cudaStream_t stream);
+
 // ----- (iii) merge with exact causal local attention -----------------------
 struct MergeParams {
   const float* a;

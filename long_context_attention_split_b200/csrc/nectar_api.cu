@@ -177,6 +177,10 @@ size_t nectar_cache_attn_workspace_size(nectar_dims dims, int64_t n, int64_t nq)
   if (rows == 0 || n == 0) return 0;
   const DeviceInfo di = device_info();
   if (di.sms == 0) return 0;
+  if (rows > dec_max_rows()) {
+    const TcPlan tp = plan_tc(dims.L * dims.Hkv, n, rows, di.sms);
+    return tp.ws_bytes + 256;
+  }
   const DecPlan pl = cache_attn_plan(dims, n, nq, di.sms);
   const int64_t prow = static_cast<int64_t>(dims.L) * dims.Hkv * pl.S_max * rows;
   return static_cast<size_t>(prow) * (kD + 2) * sizeof(float) + 256;
@@ -226,6 +230,36 @@ nectar_status nectar_cache_attn_lse(nectar_dims dims, const nectar_bf16* K, cons
   if (workspace == nullptr || workspace_bytes < need)
     return fail(NECTAR_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
   if (!aligned16(workspace)) return fail(NECTAR_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+  if (rows > dec_max_rows()) {
+    // many query rows per head: tcgen05 flash-style kernel
+    const TcPlan tp = plan_tc(heads, n, rows, di.sms);
+    TcParams tpar{};
+    tpar.n = n;
+    tpar.heads = heads;
+    tpar.rows_total = rows;
+    tpar.qtiles = tp.qtiles;
+    tpar.tph = tp.tph;
+    tpar.total = tp.total;
+    tpar.C = tp.C;
+    tpar.S_max = tp.S_max;
+    tpar.qmul = scale * kLog2e;
+    tpar.alpha = alpha;
+    tpar.A = A;
+    tpar.ws_acc = reinterpret_cast<float*>(workspace);
+    tpar.ws_ml = tpar.ws_acc + static_cast<int64_t>(tp.C) * tp.S_max * 128 * kD;
+    tpar.err = di.err;
+    CUtensorMap tq, tk, tv;
+    const cuuint64_t dq[3] = {128, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(heads)};
+    const cuuint64_t sq[2] = {256, static_cast<cuuint64_t>(rows) * 256};
+    const cuuint64_t dk[3] = {128, static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(heads)};
+    const cuuint64_t sk[2] = {256, static_cast<cuuint64_t>(n) * 256};
+    const cuuint32_t box[3] = {64, 128, 1};
+    NECTAR_TRY(make_tmap(&tq, Q, 3, dq, sq, box, "Q"));
+    NECTAR_TRY(make_tmap(&tk, K, 3, dk, sk, box, "K"));
+    NECTAR_TRY(make_tmap(&tv, V, 3, dk, sk, box, "V"));
+    cudaError_t e = launch_cache_attn_tc(tq, tk, tv, tpar, st);
+    return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "cache_attn tensor-core kernel");
+  }
   const int64_t prow = static_cast<int64_t>(heads) * pl.S_max * rows;
   p.ws_acc = reinterpret_cast<float*>(workspace);
   p.ws_ml = p.ws_acc + prow * kD;

@@ -63,7 +63,14 @@ def run_cache_attn(L, Hkv, G, n, nq, seed=0, key_scale=None):
     (1, 2, 7, 333, 1),        # R = 7 (16-lane groups)
     (2, 1, 8, 64, 1),         # R = 8, exactly one tile
     (1, 1, 3, 1, 1),          # n = 1
-    (3, 2, 2, 5000, 3),       # 6 rows -> blocks of 8, several heads per CTA range
+    (3, 2, 2, 5000, 3),       # 6 rows, several heads per CTA range
+    # tensor-core path (more than 8 query rows per KV head)
+    (1, 1, 3, 777, 3),        # 9 rows: one partial 128-row tile, ragged keys
+    (1, 2, 2, 1000, 65),      # 130 rows: two row tiles, the second with 2 rows
+    (4, 8, 4, 1000, 4),       # 16 rows, 32 heads: units cut between CTAs
+    (1, 2, 8, 128, 128),      # 1024 rows, n = one key tile: units whole in a CTA
+    (1, 1, 4, 100, 32),       # n < one key tile
+    (2, 2, 4, 8192, 128),     # 512 rows x 64 key tiles
 ])
 def test_cache_attn_parity(L, Hkv, G, n, nq):
     wl, ag, Ag, ao, Ao = run_cache_attn(L, Hkv, G, n, nq, seed=n + G)
@@ -105,6 +112,40 @@ def test_cache_attn_workspace_errors():
     with pytest.raises(nx.NectarError) as e:
         nx.cache_attn_lse(cuda(wl.K), cuda(wl.V), cuda(wl.Q), workspace=small)
     assert e.value.status == 3
+
+
+def test_cache_attn_tc_heavy_hitters_config3_shape():
+    """Regression-target shape (4096 query rows per head) on a reduced cache:
+    heavy-hitter keys with a +6 logit, tensor-core path."""
+    wl = make_workload("qwen3_4b_targets", L=1, Hkv=2, n=4096, nq=1024, seed=11)
+    alpha, A = nx.cache_attn_lse(cuda(wl.K), cuda(wl.V), cuda(wl.Q))
+    torch.cuda.synchronize()
+    sel = torch.arange(0, wl.rows, 37)      # sampled rows, recomputed by the oracle
+    for h in range(2):
+        ao, Ao = oracle.cache_attn(wl.K[0, h][None], wl.V[0, h][None], wl.Q[0, h].reshape(1, -1, 128)[:, sel],
+                                   wl.scale)
+        check_attn(alpha[0, h].reshape(1, -1)[:, sel].cpu().numpy(),
+                   A[0, h].reshape(1, -1, 128)[:, sel].cpu().numpy(), ao, Ao, wl.V.float().abs().max().item())
+
+
+def test_cache_attn_tc_running_max_moves():
+    """A key deep in the cache that scores far above everything before it, for
+    half of the query rows only: the running maximum moves by more than 2^8
+    inside a unit for some rows of a warp and not for others."""
+    g = torch.Generator().manual_seed(21)
+    L, Hkv, G, nq, n = 2, 2, 4, 64, 3000
+    K = torch.randn(L, Hkv, n, 128, generator=g)
+    V = torch.randn(L, Hkv, n, 128, generator=g).to(torch.bfloat16)
+    Q = torch.randn(L, Hkv, G, nq, 128, generator=g)
+    u = torch.nn.functional.normalize(torch.randn(128, generator=g), dim=0)
+    Q[..., ::2, :] += 3.0 * u           # every other token of every query head
+    K[:, :, 2345] = 40.0 * u            # scores ~ +10 (natural log units) for those rows
+    K, Q = K.to(torch.bfloat16), Q.to(torch.bfloat16)
+    alpha, A = nx.cache_attn_lse(cuda(K), cuda(V), cuda(Q))
+    torch.cuda.synchronize()
+    ao, Ao = oracle.cache_attn(K, V, Q.reshape(L, Hkv, G * nq, 128), 1 / math.sqrt(128))
+    check_attn(alpha.cpu().numpy().reshape(ao.shape), A.cpu().numpy().reshape(Ao.shape), ao, Ao,
+               V.float().abs().max().item(), "rescale")
 
 
 def test_cache_attn_full_size_sampled():
