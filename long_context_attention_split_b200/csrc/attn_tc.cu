@@ -9,7 +9,9 @@
 // per SM) takes the contiguous range [c*T/C, (c+1)*T/C): a unit wholly
 // inside one range is finished by that CTA (alpha, A written directly); a
 // unit cut by range boundaries leaves one (m, l, acc) partial per piece, and
-// the combine kernel joins them by log-sum-exp (a separate launch).
+// the combine kernel joins them by log-sum-exp (a separate launch).  A CTA
+// can cut at most two units (the first and the last of its range), so the
+// partials take two slots per CTA whatever the shape.
 //
 // Per tile, tcgen05 (kind::f16, cta_group::1, fp32 accumulation in TMEM):
 //   S = Q K^T   M = 128 rows, N = 128 keys, K = d    (A, B K-major, SW128)
@@ -237,7 +239,8 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         dst = p.A + (hd * p.rows_total + r) * kD;
         inv = 1.0f / l;
       } else {
-        const int64_t prow = (static_cast<int64_t>(f) * p.S_max + (c - f)) * kTcRows + row;
+        const int slot = (u == t0 / p.tph) ? 0 : 1;    // first or last unit of this CTA's range
+        const int64_t prow = (static_cast<int64_t>(c) * 2 + slot) * kTcRows + row;
         dst = p.ws_acc + prow * kD;
         if (r < p.rows_total) {
           p.ws_ml[prow * 2] = m;
@@ -362,13 +365,17 @@ __global__ void cache_attn_tc_combine_kernel(const TcParams p) {
   const int f = tc_first_cta(u * p.tph, p.total, p.C);
   const int la = tc_first_cta(u * p.tph + p.tph - 1, p.total, p.C);
   if (f == la) return;
+  // the piece of CTA cc sits in slot 0 if u is the first unit of cc's range
+  auto prow_of = [&](int cc) {
+    const int64_t first_unit = (static_cast<int64_t>(cc) * p.total / p.C) / p.tph;
+    return (static_cast<int64_t>(cc) * 2 + (u == first_unit ? 0 : 1)) * kTcRows + rr;
+  };
   float M = -INFINITY;
-  for (int s = 0; s <= la - f; ++s)
-    M = fmaxf(M, p.ws_ml[((static_cast<int64_t>(f) * p.S_max + s) * kTcRows + rr) * 2]);
+  for (int cc = f; cc <= la; ++cc) M = fmaxf(M, p.ws_ml[prow_of(cc) * 2]);
   float ls = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s <= la - f; ++s) {
-    const int64_t prow = (static_cast<int64_t>(f) * p.S_max + s) * kTcRows + rr;
+  for (int cc = f; cc <= la; ++cc) {
+    const int64_t prow = prow_of(cc);
     const float w = exp2_shift(p.ws_ml[prow * 2], M);
     ls = fmaf(p.ws_ml[prow * 2 + 1], w, ls);
     const float4 a4 = reinterpret_cast<const float4*>(p.ws_acc + prow * kD)[lane];
@@ -395,15 +402,8 @@ TcPlan plan_tc(int heads, int64_t n, int64_t rows, int num_sms) {
   if (C > pl.total) C = pl.total;
   if (C < 1) C = 1;
   pl.C = static_cast<int>(C);
-  pl.S_max = 1;
-  if (pl.total > 0) {
-    for (int64_t u = 0; u < units; ++u) {
-      const int f = tc_first_cta(u * pl.tph, pl.total, pl.C);
-      const int la = tc_first_cta(u * pl.tph + pl.tph - 1, pl.total, pl.C);
-      if (la - f + 1 > pl.S_max) pl.S_max = la - f + 1;
-    }
-  }
-  pl.ws_bytes = static_cast<size_t>(pl.C) * pl.S_max * kTcRows * (kD + 2) * sizeof(float);
+  pl.S_max = 2;    // partial slots per CTA
+  pl.ws_bytes = static_cast<size_t>(pl.C) * 2 * kTcRows * (kD + 2) * sizeof(float);
   pl.smem = TcSmem::total + 1024;
   return pl;
 }

@@ -46,12 +46,12 @@ struct TcParams {
   int qtiles;           // 128-row query tiles per head
   int64_t tph;          // 128-key tiles per head
   int64_t total;        // heads * qtiles * tph
-  int C, S_max;
+  int C, S_max;         // S_max = 2 partial slots per CTA
   float qmul;           // scale * log2(e)
   float* alpha;
   float* A;
-  float* ws_ml;         // [C][S_max][128][2]
-  float* ws_acc;        // [C][S_max][128][128]
+  float* ws_ml;         // [C][2][128][2]
+  float* ws_acc;        // [C][2][128][128]
   int* err;
 };
 struct TcPlan {
