@@ -1,0 +1,54 @@
+"""bench.py's multi-rank bookkeeping on CPU with gloo, world size 2: the
+step time is the max over ranks and the throughput counts every rank's
+units over that time."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    import bench
+    assert bench.dist_env() == (world, rank, rank)
+    ms = [10.0, 25.0][rank]                     # rank 1 is the slow one
+    mx = bench.reduce_max(ms)
+    value = bench.aggregate(448, mx, steps=20)  # 448 query vectors per rank-step
+    bench.barrier()
+    out[rank] = (mx, value)
+    dist.destroy_process_group()
+
+
+def test_bench_aggregation_gloo_two_ranks():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    for r in range(2):
+        mx, value = out[r]
+        assert mx == 25.0
+        assert value == pytest.approx(2 * 448 * 20 / 0.025)
+
+
+def test_bench_single_process_identity():
+    import bench
+    assert bench.reduce_max(3.5) == 3.5
+    assert bench.aggregate(448, 10.0, steps=10) == pytest.approx(448 * 10 / 0.010)
