@@ -102,6 +102,39 @@ NECTAR_API nectar_status nectar_cache_attn_lse(nectar_dims dims, const nectar_bf
                                     size_t workspace_bytes, nectar_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * nectar_cache_attn_lse_static -- the same computation as
+ * nectar_cache_attn_lse (same validation, kernels and outputs) with no
+ * workspace argument and no allocation anywhere.  The paper has no
+ * counterpart: this is an interface for callers that cannot create device
+ * buffers -- code inside a host application or serving runtime whose memory
+ * manager owns the whole device pool, plugin interfaces that receive only
+ * input and output pointers, and latency-bound decode loops where cudaMalloc
+ * (which may synchronise the device) is not acceptable.
+ *
+ * Scratch comes from a fixed area that is part of the library's device
+ * image: NECTAR_STATIC_SCRATCH_BYTES on every GPU that loads the library,
+ * held until the process exits.  A call whose scratch need
+ * (nectar_cache_attn_workspace_size) exceeds it returns
+ * NECTAR_ERR_WORKSPACE with the two sizes in nectar_last_error().
+ *  - The first call on a device looks up the area's device address (with
+ *    that device current) and remembers it; make that first call before
+ *    any stream capture.
+ *  - All calls on a device share the one area, and it keeps whatever the
+ *    last call left there.  Nothing in it has to start at zero (every value
+ *    read is first written by the same call), but two calls that overlap on
+ *    the GPU -- on different streams, or on one stream from different host
+ *    threads without ordering -- race on it.
+ * Arguments and outputs as for nectar_cache_attn_lse.
+ * ------------------------------------------------------------------------ */
+#define NECTAR_STATIC_SCRATCH_BYTES (32u << 20)
+
+NECTAR_API nectar_status nectar_cache_attn_lse_static(nectar_dims dims, const nectar_bf16 *K,
+                                                      const nectar_bf16 *V, int64_t n,
+                                                      const nectar_bf16 *Q, int64_t nq, float scale,
+                                                      float *alpha, float *A,
+                                                      nectar_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Module set: one score net a_theta: R^d -> R and one target net
  * A_theta: R^d -> R^d per (l, h), shared by the G query heads of that KV
  * head (§2.1), each an MLP with input re-injection, Eq. (3.6), §2.4:

@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
     L.nectar_cache_attn_workspace_size.restype = ctypes.c_size_t
     L.nectar_cache_attn_lse.argtypes = [Dims, P, P, I64, P, I64, F, P, P, P, ctypes.c_size_t, P]
     L.nectar_cache_attn_lse.restype = S
+    L.nectar_cache_attn_lse_static.argtypes = [Dims, P, P, I64, P, I64, F, P, P, P]
+    L.nectar_cache_attn_lse_static.restype = S
     L.nectar_module_packed_elems.argtypes = [Dims, I32, P]
     L.nectar_module_packed_elems.restype = I64
     L.nectar_module_pack.argtypes = [Dims, I32, P, P, P, I64]
@@ -162,6 +164,28 @@ def cache_attn_lse(K, V, Q, scale: Optional[float] = None, alpha=None, A=None, w
                                      _stream(stream))
     _check(st, "nectar_cache_attn_lse")
     return alpha, A
+
+
+def cache_attn_lse_static(K, V, Q, scale: Optional[float] = None, alpha=None, A=None, stream=None):
+    """As cache_attn_lse, through nectar_cache_attn_lse_static: no workspace is
+    passed or allocated; the library's fixed device scratch area is used."""
+    dims, nq = dims_of(Q)
+    n = K.shape[2]
+    for t, nm in ((K, "K"), (V, "V"), (Q, "Q")):
+        _need(t, nm, torch.bfloat16)
+    if scale is None:
+        scale = 1.0 / math.sqrt(dims.d)
+    if alpha is None:
+        alpha = torch.empty(Q.shape[:4], dtype=torch.float32, device=Q.device)
+    if A is None:
+        A = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    st = lib().nectar_cache_attn_lse_static(dims, _ptr(K), _ptr(V), n, _ptr(Q), nq, float(scale), _ptr(alpha),
+                                            _ptr(A), _stream(stream))
+    _check(st, "nectar_cache_attn_lse_static")
+    return alpha, A
+
+
+STATIC_SCRATCH_BYTES = 32 << 20
 
 
 # ---------------------------------------------------------------------------

@@ -8,6 +8,9 @@
 
 namespace nectar {
 
+// Sets the thread's nectar_last_error() text (defined with the C ABI).
+void set_last_error(const char* msg);
+
 // ----- (i) split-n decode attention (CUDA cores) + LSE combine -------------
 struct DecParams {
   const __nv_bfloat16* K;

@@ -24,8 +24,12 @@ __device__ int g_error_word = 0;
 using namespace nectar;
 
 namespace {
-
 thread_local char t_last_error[512] = "";
+}
+
+void nectar::set_last_error(const char* msg) { snprintf(t_last_error, sizeof t_last_error, "%s", msg); }
+
+namespace {
 
 nectar_status fail(nectar_status s, const char* fmt, ...) {
   va_list ap;
