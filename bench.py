@@ -40,6 +40,14 @@ METRIC = "Nectar decode queries/s & exact (α,A) HBM GB/s at 1 B200; % of roofli
 UNIT = "queries/s"
 
 
+def load_sustained(default):
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"])
+    except Exception:
+        return default
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -171,6 +179,19 @@ def attn_bytes(wl) -> int:
     return heads * (4 * wl.n * wl.d + rows * 2 * wl.d + rows * 4 * (wl.d + 1))
 
 
+def attn_flops(wl) -> int:
+    """FLOPs of (i): q.k and p.v, 2 d each, for every (key, row) of every head."""
+    return wl.heads * wl.rows * wl.n * 4 * wl.d
+
+
+def decode_flops(wl) -> int:
+    """FLOPs of the fused decode: 2 per module weight per row, plus local q.k
+    and p.v over the visible tokens."""
+    params = sum(wl.Hkv * (2 * H * H + 645 * H + 129) if wl.depth == 2 else 0 for H in wl.widths)
+    vis = (torch.minimum(wl.q_pos.long().cpu() + 1, wl.local_len.long().cpu()[wl.q_seq.long().cpu()])).clamp(min=0)
+    return 2 * params * wl.G * wl.nq + wl.heads * wl.G * int(vis.sum()) * 4 * wl.d
+
+
 def decode_bytes(wl, weight_bytes: int) -> int:
     """Algorithmic bytes of the fused decode: module weights, the visible local
     K/V of every sequence, Q in, out."""
@@ -192,10 +213,12 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     hbm_peak, tc_peak, peak_kind = load_peaks()
+    tc_peak_sust = load_sustained(tc_peak)
 
-    over = {"L": args.layers} if args.layers else {}
+    over = workload_overrides(args)
     wl = make_workload(args.workload, seed=args.seed + rank, device=dev, **over)
-    mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G, device=dev)
+    has_decode = wl.modules is not None and wl.Kloc is not None
+    mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G, device=dev) if has_decode else None
     Q = wl.Q
     alpha = torch.empty(Q.shape[:4], dtype=torch.float32, device=dev)
     A = torch.empty(Q.shape, dtype=torch.float32, device=dev)
@@ -203,9 +226,8 @@ def run_ours(args):
     wsb = nx.cache_attn_workspace_size(wl.L, wl.Hkv, wl.G, wl.n, wl.nq)
     work = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    local_args = (wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len)
-    n_split = math.ceil(wl.rows / 8)       # CUDA-core split launches per (i) call
-    launches_per_step = n_split + 1 + 1    # split kernel(s) + combine + fused decode
+    local_args = (wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len) if has_decode else None
+    launches_per_step = 2 + (1 if has_decode else 0)   # (i) main kernel + combine, fused decode
 
     ev_a0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ev_a1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -217,7 +239,8 @@ def run_ours(args):
         nx.cache_attn_lse(wl.K, wl.V, Q, alpha=alpha, A=A, workspace=work, stream=stream)
         if i is not None:
             ev_a1[i].record(stream)
-        nx.decode(mods, Q, *local_args, out=out, stream=stream)
+        if has_decode:
+            nx.decode(mods, Q, *local_args, out=out, stream=stream)
         if i is not None:
             ev_d1[i].record(stream)
 
@@ -248,30 +271,42 @@ def run_ours(args):
     qps = queries_per_step(wl)
     value = aggregate(qps, max_ms, args.steps)
     ab = attn_bytes(wl)
-    achieved = ab / (attn_avg / 1e3) / 1e9
-    db = decode_bytes(wl, mods.bytes)
+    af = attn_flops(wl)
+    db = decode_bytes(wl, mods.bytes) if has_decode else 0
+    # dominant kernel: exact attention; HBM-bound below the ridge point
+    # (query rows per KV head = FLOP per byte of K/V), tensor-bound above
+    tensor_bound = wl.rows > tc_peak * 1e12 / (hbm_peak * 1e9)
+    long_step = attn_avg > 10.0
+    tc_use = tc_peak_sust if long_step else tc_peak
+    if tensor_bound:
+        achieved = af / (attn_avg / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_use,
+                "peak_kind": f"{peak_kind} bf16 {'sustained' if long_step else 'burst'}",
+                "unit": "TFLOP/s", "frac": achieved / tc_use, "alg_flops_per_launch": af,
+                "alg_bytes_per_launch": ab, "hbm_GBps": ab / (attn_avg / 1e3) / 1e9}
+    else:
+        achieved = ab / (attn_avg / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "peak_kind": f"{peak_kind} copy",
+                "unit": "GB/s", "frac": achieved / hbm_peak, "alg_bytes_per_launch": ab}
 
     # ---- end to end through the public API with host buffers ----
     pin = lambda t: t.cpu().pin_memory()
-    hQ, hseq, hpos, hlen = pin(Q), pin(wl.q_seq), pin(wl.q_pos), pin(wl.local_len)
-    h_alpha = torch.empty(alpha.shape, dtype=torch.float32).pin_memory()
-    h_A = torch.empty(A.shape, dtype=torch.float32).pin_memory()
-    h_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-    dQ = torch.empty_like(Q)
-    dseq, dpos, dlen = torch.empty_like(wl.q_seq), torch.empty_like(wl.q_pos), torch.empty_like(wl.local_len)
-    h2d = sum(t.numel() * t.element_size() for t in (hQ, hseq, hpos, hlen))
-    d2h = sum(t.numel() * t.element_size() for t in (h_alpha, h_A, h_out))
+    meta = (wl.q_seq, wl.q_pos, wl.local_len) if has_decode else ()
+    h_in = [pin(Q)] + [pin(t) for t in meta]
+    d_in = [torch.empty_like(Q)] + [torch.empty_like(t) for t in meta]
+    d_out = [alpha, A] + ([out] if has_decode else [])
+    h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in d_out]
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
 
     def e2e_step():
-        dQ.copy_(hQ, non_blocking=True)
-        dseq.copy_(hseq, non_blocking=True)
-        dpos.copy_(hpos, non_blocking=True)
-        dlen.copy_(hlen, non_blocking=True)
-        nx.cache_attn_lse(wl.K, wl.V, dQ, alpha=alpha, A=A, workspace=work, stream=stream)
-        nx.decode(mods, dQ, dseq, dpos, wl.Kloc, wl.Vloc, dlen, out=out, stream=stream)
-        h_alpha.copy_(alpha, non_blocking=True)
-        h_A.copy_(A, non_blocking=True)
-        h_out.copy_(out, non_blocking=True)
+        for d, h in zip(d_in, h_in):
+            d.copy_(h, non_blocking=True)
+        nx.cache_attn_lse(wl.K, wl.V, d_in[0], alpha=alpha, A=A, workspace=work, stream=stream)
+        if has_decode:
+            nx.decode(mods, d_in[0], d_in[1], d_in[2], wl.Kloc, wl.Vloc, d_in[3], out=out, stream=stream)
+        for h, d in zip(h_out, d_out):
+            h.copy_(d, non_blocking=True)
 
     e2e_value = None
     if not args.no_e2e:
@@ -291,7 +326,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, mods_host=None, budget_s=args.cpu_budget)
+        cpu = cpu_baseline(wl, budget_s=args.cpu_budget)
 
     if rank == 0:
         traffic = traffic_from_profile(args.workload)
@@ -316,26 +351,9 @@ def run_ours(args):
                 "queries_per_step_per_gpu": qps,
                 "l2": "inputs larger than L2 (document K/V 3.76 GB streamed every step)",
             },
-            "parts": {
-                "exact_attn_ms": attn_avg,
-                "exact_attn_GBps": achieved,
-                "decode_ms": dec_avg,
-                "decode_queries_per_s": qps / (dec_avg / 1e3),
-                "decode_alg_bytes": db,
-                "decode_GBps": db / (dec_avg / 1e3) / 1e9,
-                "decode_frac_of_hbm": db / (dec_avg / 1e3) / 1e9 / hbm_peak,
-            },
-            "roofline": {
-                "kernel": "cache_attn_split+combine (exact alpha, A)",
-                "bound": "hbm",
-                "achieved": achieved,
-                "peak": hbm_peak,
-                "peak_kind": peak_kind,
-                "unit": "GB/s",
-                "frac": achieved / hbm_peak,
-                "alg_bytes_per_launch": ab,
-                "traffic": traffic,
-            },
+            "parts": parts(wl, attn_avg, dec_avg, ab, db, qps, hbm_peak, tc_peak, has_decode),
+            "roofline": dict(kernel=("cache_attn_tc+combine" if wl.rows > 8 else "cache_attn_split+combine")
+                             + " (exact alpha, A)", traffic=traffic, **roof),
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
@@ -346,6 +364,42 @@ def run_ours(args):
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def parts(wl, attn_ms, dec_ms, ab, db, qps, hbm_peak, tc_peak, has_decode):
+    out = {"exact_attn_ms": attn_ms, "exact_attn_GBps": ab / (attn_ms / 1e3) / 1e9,
+           "exact_attn_TFLOPs": attn_flops(wl) / (attn_ms / 1e3) / 1e12,
+           "exact_attn_queries_per_s": qps / (attn_ms / 1e3)}
+    if has_decode:
+        wbytes = db - wl.heads * (wl.local_len.long().clamp(max=wl.T)).sum().item() * 4 * wl.d \
+            - wl.heads * wl.rows * 6 * wl.d
+        dflops = decode_flops(wl)
+        t = dec_ms / 1e3
+        out.update({
+            "decode_ms": dec_ms,
+            "decode_queries_per_s": qps / t,
+            "decode_alg_bytes": db,
+            "decode_GBps": db / t / 1e9,
+            "decode_flops": dflops,
+            # full form: weights + local K/V bytes at HBM vs FLOPs at the tensor peak
+            "decode_roofline_us_full": max(db / (hbm_peak * 1e9), dflops / (tc_peak * 1e12)) * 1e6,
+            # weights-or-FLOPs form (module weights only)
+            "decode_roofline_us_weights": max(wbytes / (hbm_peak * 1e9), dflops / (tc_peak * 1e12)) * 1e6,
+        })
+        out["decode_frac_full"] = out["decode_roofline_us_full"] / (dec_ms * 1e3)
+        out["decode_frac_weights_form"] = out["decode_roofline_us_weights"] / (dec_ms * 1e3)
+    return out
+
+
+def workload_overrides(args) -> dict:
+    over = {}
+    if args.layers:
+        over["L"] = args.layers
+    if args.batch:
+        over["B"] = args.batch
+    if args.rho:
+        over["rho"] = args.rho
+    return over
 
 
 def traffic_from_profile(workload: str):
@@ -363,8 +417,9 @@ def traffic_from_profile(workload: str):
 # CPU oracle baseline
 # ---------------------------------------------------------------------------
 def _oracle_sample(wl, layers):
-    """One pass of the whole path on the oracle for the given layers
-    (all their KV heads).  Returns query vectors processed."""
+    """One pass of the whole path on the oracle for the given layers (all
+    their KV heads, the tokens kept in the host view).  Returns query
+    vectors processed."""
     import numpy as np
     import oracle
     H = len(layers) * wl.Hkv
@@ -372,6 +427,8 @@ def _oracle_sample(wl, layers):
     V = wl.V[layers].reshape(H, wl.n, wl.d)
     Q = wl.Q[layers].reshape(H, wl.rows, wl.d)
     alpha, A = oracle.cache_attn(K, V, Q, wl.scale)
+    if wl.modules is None:
+        return H * wl.rows
     sel = [(l, h) for l in layers for h in range(wl.Hkv)]
     a, At = oracle.module_forward(wl, sel)
     a = np.stack([a[k] for k in sel])
@@ -381,13 +438,14 @@ def _oracle_sample(wl, layers):
     return H * wl.rows
 
 
-def cpu_baseline(wl, mods_host=None, budget_s=20.0, layers_per_sample=1):
+def cpu_baseline(wl, budget_s=12.0, layers_per_sample=1):
     import oracle
     oracle.build()
     cores = oracle.num_threads()
-    # host copies of what one sample touches
+    # host copies of what one sample touches: layer 0, and at most enough
+    # tokens that one pass stays around a second
     layers = list(range(min(layers_per_sample, wl.L)))
-    host = _host_view(wl, layers)
+    host = _host_view(wl, layers, token_cap=_token_cap(wl))
     t0 = time.perf_counter()
     done = 0
     samples = 0
@@ -399,29 +457,42 @@ def cpu_baseline(wl, mods_host=None, budget_s=20.0, layers_per_sample=1):
     dt = time.perf_counter() - t0
     return {"value": done / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{samples} pass(es) of the whole path over layer(s) {layers} "
-                      f"({len(layers) * wl.Hkv} of {wl.heads} KV heads, all their query rows), "
-                      f"{dt:.1f} s on {cores} threads; queries/s = query vectors done / time"}
+                      f"({len(layers) * wl.Hkv} of {wl.heads} KV heads, {host.nq} of {wl.nq} tokens x {wl.G} "
+                      f"query heads), {dt:.1f} s on {cores} threads; queries/s = query vectors done / time"}
+
+
+def _token_cap(wl) -> int:
+    """Tokens per sample so that the exact part of one pass is ~1e9 MACs."""
+    per_token = wl.Hkv * wl.G * wl.n * wl.d * 3
+    return max(1, min(wl.nq, int(1e9 // max(per_token, 1))))
 
 
 class _HostWL:
     pass
 
 
-def _host_view(wl, layers):
-    """CPU copy of the workload restricted to `layers` (renumbered 0..)."""
+def _host_view(wl, layers, token_cap=None):
+    """CPU copy of the workload restricted to `layers` (renumbered 0..) and
+    to the first `token_cap` query tokens."""
     h = _HostWL()
-    for k in ("name", "Hkv", "G", "d", "n", "nq", "B", "T", "scale", "depth"):
+    for k in ("name", "Hkv", "G", "d", "n", "B", "T", "scale", "depth"):
         setattr(h, k, getattr(wl, k))
+    nq = wl.nq if token_cap is None else min(token_cap, wl.nq)
+    h.nq = nq
     h.L = len(layers)
-    h.rows = wl.rows
+    h.rows = wl.G * nq
     h.heads = h.L * wl.Hkv
     idx = torch.tensor(layers)
     h.K = wl.K[idx.to(wl.K.device)].cpu()
     h.V = wl.V[idx.to(wl.V.device)].cpu()
-    h.Q = wl.Q[idx.to(wl.Q.device)].cpu()
+    h.Q = wl.Q[idx.to(wl.Q.device)][:, :, :, :nq].contiguous().cpu()
+    h.modules = None
+    h.widths = None
+    if wl.Kloc is None or wl.modules is None:
+        return h
     h.Kloc = wl.Kloc[idx.to(wl.Kloc.device)].cpu()
     h.Vloc = wl.Vloc[idx.to(wl.Vloc.device)].cpu()
-    h.q_seq, h.q_pos, h.local_len = wl.q_seq.cpu(), wl.q_pos.cpu(), wl.local_len.cpu()
+    h.q_seq, h.q_pos, h.local_len = wl.q_seq[:nq].cpu(), wl.q_pos[:nq].cpu(), wl.local_len.cpu()
     h.widths = [wl.widths[l] for l in layers]
     h.modules = []
     for l in layers:
@@ -442,11 +513,10 @@ def run_reference(args):
         return
     import oracle
     oracle.build()
-    over = {"L": 1}
-    if args.layers:
-        over = {"L": 1}
+    over = workload_overrides(args)
+    over["L"] = 1
     wl = make_workload(args.workload, seed=args.seed, device="cpu", **over)
-    host = _host_view(wl, [0])
+    host = _host_view(wl, [0], token_cap=_token_cap(wl))
     cores = oracle.num_threads()
     t0 = time.perf_counter()
     done = 0
@@ -455,8 +525,8 @@ def run_reference(args):
     dt = time.perf_counter() - t0
     value = done / dt
     full = PRESETS[args.workload]
-    sample = (f"each step = the whole path (exact attention, both MLPs, merge) over layer 0 of {full['L']} "
-              f"({wl.Hkv} KV heads x {wl.rows} query rows) of {args.workload}")
+    sample = (f"each step = the whole path over layer 0 of {full['L']} ({wl.Hkv} KV heads, {host.nq} of {wl.nq} "
+              f"tokens x {wl.G} query heads) of {args.workload}")
     line = {
         "impl": "reference",
         "metric": METRIC,
@@ -495,6 +565,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="decode batch B (llama8b_sweep: 1, 16, 256)")
+    ap.add_argument("--rho", type=float, default=0.0, help="module capacity (llama8b_sweep: 0.01, 0.05, 0.10)")
     ap.add_argument("--layers", type=int, default=0,
                     help="run only the first LAYERS layers (small cases for profiling; not a bench line)")
     args = ap.parse_args()

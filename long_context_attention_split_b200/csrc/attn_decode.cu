@@ -37,8 +37,9 @@ __host__ __device__ constexpr size_t dec_smem_bytes() {
          + 2 * kDecStages * sizeof(uint64_t);                // full / empty barriers
 }
 
+// Two CTAs per SM for up to 2 rows (register cap 113), one otherwise.
 template <int R, int LPK>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecThreads, (R <= 2 ? 2 : 1))
 cache_attn_split_kernel(const DecParams p) {
   using St = RowState<R, LPK>;
   constexpr int NG = St::NG;
@@ -220,6 +221,33 @@ static cudaError_t launch_split(const DecParams& p, cudaStream_t stream) {
 }
 
 int dec_max_rows() { return 8; }
+
+// Resident CTAs per SM of the split kernel for R rows (occupancy calculator).
+template <int R, int LPK>
+static int occ_t() {
+  const size_t smem = dec_smem_bytes<R>();
+  if (cudaFuncSetAttribute(cache_attn_split_kernel<R, LPK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, cache_attn_split_kernel<R, LPK>, kDecThreads, smem) !=
+      cudaSuccess)
+    return 1;
+  return n < 1 ? 1 : n;
+}
+
+int dec_ctas_per_sm(int R) {
+  switch (R) {
+    case 1: return occ_t<1, 8>();
+    case 2: return occ_t<2, 8>();
+    case 3: return occ_t<3, 8>();
+    case 4: return occ_t<4, 8>();
+    case 5: return occ_t<5, 16>();
+    case 6: return occ_t<6, 16>();
+    case 7: return occ_t<7, 16>();
+    default: return occ_t<8, 16>();
+  }
+}
 
 size_t dec_smem_for_rows(int R) {
   switch (R) {

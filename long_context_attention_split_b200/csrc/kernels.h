@@ -37,6 +37,7 @@ struct DecPlan {
 
 DecPlan plan_decode(int heads, int64_t n, int num_sms, int ctas_per_sm);
 int dec_max_rows();
+int dec_ctas_per_sm(int R);
 size_t dec_smem_for_rows(int R);
 cudaError_t launch_cache_attn_split(const DecParams& p, int R, cudaStream_t stream);
 cudaError_t launch_cache_attn_combine(const DecParams& p, float* alpha, float* A, cudaStream_t stream);
@@ -91,7 +92,7 @@ constexpr int kModMaxLayers = 256;
 struct ModParams {
   int Hkv, G, depth;
   int64_t nq;
-  int N, TPC, nblk, Hmax, tmem_cols;
+  int N, TPC, nblk, Hmax, tmem_cols, stages, cps;
   const __nv_bfloat16* blob;
   const __nv_bfloat16* Q;
   float* a_out;         // module forward outputs
@@ -111,11 +112,11 @@ struct ModParams {
   uint8_t order[kModMaxLayers];        // layers by decreasing width
 };
 struct ModShape {
-  int TPC, N, nblk, tmem_cols;
+  int TPC, N, nblk, tmem_cols, stages, cps;
   size_t smem;
 };
 ModShape mod_shape(int G, int64_t nq, int Hmax, bool fuse);
-cudaError_t launch_module(const CUtensorMap& tw, const CUtensorMap& tq, const ModParams& p, int units, size_t smem,
-                          bool fuse, cudaStream_t stream);
+cudaError_t launch_module(const CUtensorMap& tq, const ModParams& p, int units, size_t smem, bool fuse,
+                          cudaStream_t stream);
 
 }  // namespace nectar

@@ -5,120 +5,89 @@
 // keys; with the exact (alpha, A) this is full attention (Eq. (3.4) is an
 // identity), with (a_theta, A_theta) it is the Nectar output (Eq. (3.5)).
 //
-// One CTA (4 warps) per (KV head, query token, block of <= 8 query heads):
-// the G query heads of a token share the token's local K/V and its causal
-// mask, so the local rows are read once for all of them, straight from
-// global memory with 16-byte non-coherent loads.
+// One CTA per (KV head, query token): the G query heads of the token share
+// its local rows and causal mask, so the rows are streamed once (blocks of
+// up to 8 heads are jobs of the same CTA) through a 4-stage shared-memory
+// ring filled by TMA bulk copies (local_attn.cuh).
 #include <cuda_runtime.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "local_attn.cuh"
 
 namespace nectar {
 
-constexpr int kMergeWarps = 4;
+constexpr int kMergeCW = 4;                       // consumer warps
+constexpr int kMergeThreads = (kMergeCW + 1) * 32;  // + 1 producer warp
+constexpr int kMergeStages = 4;
 
-template <int R, int LPK>
-__global__ void __launch_bounds__(kMergeWarps * 32)
-merge_local_kernel(const MergeParams p) {
-  using St = RowState<R, LPK>;
-  constexpr int NG = St::NG;
-  constexpr int KPG = 2;
-  constexpr int kStride = kMergeWarps * NG;   // key slots per CTA step
-
-  __shared__ float sRed[kMergeWarps][R][kD + 2];
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane / LPK, t = lane % LPK;
-  // unit = (head, token, g-block)
-  const int64_t unit = blockIdx.x;
-  const int gblocks = (p.G + R - 1) / R;
-  const int64_t hd = unit / (p.nq * gblocks);
-  const int64_t rem = unit % (p.nq * gblocks);
-  const int64_t i = rem / gblocks;
-  const int g0 = static_cast<int>(rem % gblocks) * R;
-  const int nrows = (p.G - g0 < R) ? (p.G - g0) : R;
-  const int64_t rows = static_cast<int64_t>(p.G) * p.nq;
-
-  int b;
-  const int nv = visible_local(p.q_seq, p.q_pos, p.local_len, i, p.B, p.T, &b, p.err);
-
-  St st;
-  st.reset();
-  // query rows g0..g0+nrows-1 of token i: row (g0+gg)*nq + i, stride nq rows
-  st.load_q(p.Q + (hd * rows + static_cast<int64_t>(g0) * p.nq + i) * kD, p.nq * kD, nrows, t, p.qmul);
-
-  if (nv > 0) {
-    const uint8_t* kbase = reinterpret_cast<const uint8_t*>(p.Kloc + ((hd * p.B + b) * p.T) * kD);
-    const uint8_t* vbase = reinterpret_cast<const uint8_t*>(p.Vloc + ((hd * p.B + b) * p.T) * kD);
-    for (int j0 = 0; j0 < nv; j0 += kStride * KPG) {
-      const uint8_t* kr[KPG];
-      const uint8_t* vr[KPG];
-      bool valid[KPG];
-#pragma unroll
-      for (int k = 0; k < KPG; ++k) {
-        const int j = j0 + k * kStride + warp * NG + g;
-        valid[k] = j < nv;
-        kr[k] = kbase + static_cast<int64_t>(j) * kRowBytes;
-        vr[k] = vbase + static_cast<int64_t>(j) * kRowBytes;
-      }
-      st.template step<KPG>(kr, vr, valid, t, GlobalLoader{});
-    }
-  }
-  st.merge_groups();
-  if (g == 0) {
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-#pragma unroll
-      for (int ci = 0; ci < St::CPL; ++ci)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sRed[warp][r][St::dim_of(t, ci, e)] = st.acc[r][ci * 8 + e];
-      if (t == 0) {
-        sRed[warp][r][kD] = st.m[r];
-        sRed[warp][r][kD + 1] = st.l[r];
-      }
-    }
-  }
-  __syncthreads();
-  for (int it = threadIdx.x; it < nrows * kD; it += kMergeWarps * 32) {
-    const int r = it / kD, dim = it % kD;
-    const int64_t row = hd * rows + static_cast<int64_t>(g0 + r) * p.nq + i;
-    const float ad = p.a[row] * kLog2e;       // document logit in log2 units
-    float M = ad;
-#pragma unroll
-    for (int w = 0; w < kMergeWarps; ++w) M = fmaxf(M, sRed[w][r][kD]);
-    const float wd = exp2_shift(ad, M);
-    float den = wd;
-    float num = wd * p.A_doc[row * kD + dim];
-#pragma unroll
-    for (int w = 0; w < kMergeWarps; ++w) {
-      const float wl = exp2_shift(sRed[w][r][kD], M);
-      den = fmaf(sRed[w][r][kD + 1], wl, den);
-      num = fmaf(sRed[w][r][dim], wl, num);
-    }
-    p.out[row * kD + dim] = num / den;
-  }
+template <int RG>
+__host__ __device__ constexpr size_t merge_smem_bytes() {
+  return size_t(kMergeStages) * kLocStageBytes + size_t(kMergeCW) * RG * (kD + 2) * sizeof(float) +
+         2 * kMergeStages * sizeof(uint64_t);
 }
 
-template <int R, int LPK>
+template <int RG>
+__global__ void __launch_bounds__(kMergeThreads)
+merge_local_kernel(const MergeParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* ring = smem;
+  float* scratch = reinterpret_cast<float*>(smem + kMergeStages * kLocStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(scratch + kMergeCW * RG * (kD + 2));
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kMergeStages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t hd = blockIdx.x / p.nq;
+  const int64_t i = blockIdx.x % p.nq;
+  const int64_t rows = static_cast<int64_t>(p.G) * p.nq;
+  const LocalJobs J{p.q_seq, p.q_pos, p.local_len, p.Kloc, p.Vloc, p.B, p.T, p.G, p.err};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kMergeStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, kMergeCW);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (warp == kMergeCW) {
+    if (lane == 0) local_produce<RG>(J, hd, i, 1, smem_u32(ring), kMergeStages, full0, empty0);
+    return;
+  }
+  const __nv_bfloat16* q0 = p.Q + (hd * rows + i) * kD;   // row (g = 0, token i)
+  local_consume<RG, kMergeCW>(
+      J, hd, i, 1, q0, p.nq * kD, p.qmul, ring, kMergeStages, full0, empty0, scratch, 1, warp, lane,
+      [&](int /*t*/, int g, int dim, float M, float ls, float as) {
+        // document term as one more logit a with value A_doc, Eqs. (3.4)-(3.5)
+        const int64_t row = hd * rows + static_cast<int64_t>(g) * p.nq + i;
+        const float ad = p.a[row] * kLog2e;
+        const float Mx = fmaxf(ad, M);
+        const float wd = exp2_shift(ad, Mx), wl = exp2_shift(M, Mx);
+        p.out[row * kD + dim] = (wd * p.A_doc[row * kD + dim] + wl * as) / (wd + wl * ls);
+      });
+}
+
+template <int RG>
 static cudaError_t launch_merge_t(const MergeParams& p, cudaStream_t stream) {
-  const int gblocks = (p.G + R - 1) / R;
-  const int64_t units = static_cast<int64_t>(p.heads) * p.nq * gblocks;
+  const int64_t units = static_cast<int64_t>(p.heads) * p.nq;
   if (units == 0) return cudaSuccess;
-  merge_local_kernel<R, LPK><<<static_cast<unsigned>(units), kMergeWarps * 32, 0, stream>>>(p);
+  const size_t smem = merge_smem_bytes<RG>();
+  cudaError_t e = cudaFuncSetAttribute(merge_local_kernel<RG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  merge_local_kernel<RG><<<static_cast<unsigned>(units), kMergeThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_merge_local(const MergeParams& p, cudaStream_t stream) {
   switch (p.G < 8 ? p.G : 8) {
-    case 1: return launch_merge_t<1, 8>(p, stream);
-    case 2: return launch_merge_t<2, 8>(p, stream);
-    case 3: return launch_merge_t<3, 8>(p, stream);
-    case 4: return launch_merge_t<4, 8>(p, stream);
-    case 5: return launch_merge_t<5, 16>(p, stream);
-    case 6: return launch_merge_t<6, 16>(p, stream);
-    case 7: return launch_merge_t<7, 16>(p, stream);
-    default: return launch_merge_t<8, 16>(p, stream);
+    case 1: return launch_merge_t<1>(p, stream);
+    case 2: return launch_merge_t<2>(p, stream);
+    case 3: return launch_merge_t<3>(p, stream);
+    case 4: return launch_merge_t<4>(p, stream);
+    case 5: return launch_merge_t<5>(p, stream);
+    case 6: return launch_merge_t<6>(p, stream);
+    case 7: return launch_merge_t<7>(p, stream);
+    default: return launch_merge_t<8>(p, stream);
   }
 }
 

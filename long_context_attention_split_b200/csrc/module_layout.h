@@ -6,15 +6,21 @@
 //   layer_base(l) + h * head_elems(H_l) + net * net_elems(H_l, depth, 1).
 // Inside a net (every piece a multiple of 64 elements = 128 bytes):
 //   for k = 0..depth-1:
-//     W_k  K-chunked [ceil(K_k/64)][H][64], K_k = d (k = 0) or d + H (k >= 1),
+//     W_k  tiled [ceil(H/128)][ceil(K_k/64)][tr][64], K_k = d (k = 0) or d + H,
 //          row i = hidden unit, column c = input feature: c < d multiplies q
 //          (U_0 for k = 0, V_k for k >= 1), c >= d multiplies h_{k-1} (U_k);
 //     b_k  [round64(H)]
 //   score:  w [round64(H)], c [64]            (readout W_out row, bias)
-//   target: W_out K-chunked [ceil(H/64)][d][64], c [d]
-// K-chunked means each 64-wide column block of the matrix is stored as
-// rows x 128 bytes, so a TMA box of (64 columns x 128 rows) over the blob
-// viewed as [rows][64] lands as one K-major tile.  Padding columns are 0.
+//   target: W_out tiled [1][ceil(H/64)][d][64], c [d]
+// Tiled means: the rows are cut into tiles of 128 (the last one holding
+// tr = rows - 128 * m rows), and each row tile stores its 64-column chunks
+// one after another, tr rows x 128 bytes each.  Inside every row the eight
+// 16-byte pieces sit in the order of the 128-byte swizzle (piece j of row i
+// at slot j ^ (i % 8)).  Any run of consecutive chunks of one row tile is
+// then a single contiguous block, and its bulk copy to a 1024-byte aligned
+// shared-memory address yields, chunk after chunk, exactly the K-major,
+// 128-byte-swizzled operand tiles the tensor cores read.  Padding columns
+// are 0.
 #pragma once
 #include <stdint.h>
 
@@ -33,9 +39,17 @@ NECTAR_HD int round64(int x) { return (x + 63) & ~63; }
 NECTAR_HD int kchunks(int K) { return (K + 63) / 64; }
 NECTAR_HD int hidden_k(int H, int k) { return k == 0 ? kDm : kDm + H; }
 NECTAR_HD int64_t chunked_elems(int rows, int K) { return static_cast<int64_t>(kchunks(K)) * rows * 64; }
-// element (row i, column c) of a K-chunked matrix with `rows` rows
-NECTAR_HD int64_t chunked_index(int rows, int c, int i) {
-  return (static_cast<int64_t>(c / 64) * rows + i) * 64 + (c % 64);
+// rows of row tile m of a matrix with `rows` rows
+NECTAR_HD int tile_rows(int rows, int m) { return (rows - 128 * m < 128) ? (rows - 128 * m) : 128; }
+// element offset of chunk c of row tile m (matrix with `rows` rows, K columns)
+NECTAR_HD int64_t tile_chunk_off(int rows, int K, int m, int c) {
+  return (static_cast<int64_t>(m) * kchunks(K) * 128 + static_cast<int64_t>(c) * tile_rows(rows, m)) * 64;
+}
+// element (row i, column c) of a tiled, swizzled matrix with `rows` rows and K columns
+NECTAR_HD int64_t chunked_index(int rows, int K, int c, int i) {
+  const int m = i >> 7, r = i & 127;
+  return tile_chunk_off(rows, K, m, c / 64) + static_cast<int64_t>(r) * 64 + ((((c % 64) >> 3) ^ (r & 7)) << 3) +
+         (c & 7);
 }
 NECTAR_HD int64_t hidden_w_off(int H, int depth, int k) {
   (void)depth;

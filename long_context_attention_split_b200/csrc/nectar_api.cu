@@ -88,13 +88,6 @@ DeviceInfo device_info() {
   return cache[dev];
 }
 
-// CTAs of the split kernel resident per SM (shared memory bound).
-int dec_ctas_per_sm(int R) {
-  const size_t per = dec_smem_for_rows(R) + 1024;
-  int c = static_cast<int>((228 * 1024) / per);
-  return c < 1 ? 1 : (c > 2 ? 2 : c);
-}
-
 // Row blocks handled by one launch of the CUDA-core split kernel.
 int dec_row_block(int64_t rows) { return rows < dec_max_rows() ? static_cast<int>(rows) : dec_max_rows(); }
 
@@ -398,7 +391,7 @@ nectar_status nectar_module_pack(nectar_dims dims, int32_t depth, const int32_t*
               if (k == 0) v = nh.U[0][(static_cast<int64_t>(h) * H + i) * kD + c];
               else if (c < kD) v = nh.V[k][(static_cast<int64_t>(h) * H + i) * kD + c];
               else v = nh.U[k][(static_cast<int64_t>(h) * H + i) * H + (c - kD)];
-              W[layout::chunked_index(H, c, i)] = v;
+              W[layout::chunked_index(H, Kk, c, i)] = v;
             }
           nectar_bf16* bb = blob + nb + layout::hidden_b_off(H, depth, k);
           for (int i = 0; i < H; ++i) bb[i] = nh.b[k][static_cast<int64_t>(h) * H + i];
@@ -409,7 +402,7 @@ nectar_status nectar_module_pack(nectar_dims dims, int32_t depth, const int32_t*
         } else {
           for (int o = 0; o < dout; ++o)
             for (int c = 0; c < H; ++c)
-              Wo[layout::chunked_index(kD, c, o)] = nh.Wout[(static_cast<int64_t>(h) * dout + o) * H + c];
+              Wo[layout::chunked_index(kD, H, c, o)] = nh.Wout[(static_cast<int64_t>(h) * dout + o) * H + c];
         }
         nectar_bf16* cb = blob + nb + layout::out_b_off(H, depth, dout);
         for (int o = 0; o < dout; ++o) cb[o] = nh.c[static_cast<int64_t>(h) * dout + o];
@@ -428,8 +421,7 @@ nectar_status nectar_module_pack(nectar_dims dims, int32_t depth, const int32_t*
 namespace {
 
 nectar_status prepare_modules(const nectar_dims& dims, const nectar_module_set* mods, const nectar_bf16* Q,
-                              int64_t nq, bool fuse, ModParams* p, CUtensorMap* tw, CUtensorMap* tq,
-                              ModShape* sh) {
+                              int64_t nq, bool fuse, ModParams* p, CUtensorMap* tq, ModShape* sh) {
   if (mods == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "mods is NULL");
   NECTAR_TRY(check_modules_shape(dims, mods->depth, mods->width));
   if (dims.G > 64) return fail(NECTAR_ERR_UNSUPPORTED, "G = %d > 64", dims.G);
@@ -470,13 +462,8 @@ nectar_status prepare_modules(const nectar_dims& dims, const nectar_module_set* 
   p->TPC = sh->TPC;
   p->nblk = sh->nblk;
   p->tmem_cols = sh->tmem_cols;
-  // weights: the blob viewed as [rows][64]; box = 64 columns x 128 rows
-  {
-    const cuuint64_t dimsw[2] = {64, static_cast<cuuint64_t>(mods->weights_elems / 64)};
-    const cuuint64_t strw[1] = {128};
-    const cuuint32_t boxw[2] = {64, 128};
-    NECTAR_TRY(make_tmap(tw, mods->weights, 2, dimsw, strw, boxw, "module weights"));
-  }
+  p->stages = sh->stages;
+  p->cps = sh->cps;
   // queries: [heads][G][nq][128]; box = 64 columns x TPC tokens x G heads x 1
   {
     const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
@@ -501,13 +488,13 @@ nectar_status nectar_module_forward(nectar_dims dims, const nectar_module_set* m
   if (a == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "a is NULL");
   NECTAR_TRY(check_ptr(A_theta, "A_theta"));
   ModParams p;
-  CUtensorMap tw, tq;
+  CUtensorMap tq;
   ModShape sh;
-  NECTAR_TRY(prepare_modules(dims, mods, Q, nq, false, &p, &tw, &tq, &sh));
+  NECTAR_TRY(prepare_modules(dims, mods, Q, nq, false, &p, &tq, &sh));
   p.a_out = a;
   p.A_out = A_theta;
   const int units = dims.L * dims.Hkv * sh.nblk;
-  cudaError_t e = launch_module(tw, tq, p, units, sh.smem, false, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_module(tq, p, units, sh.smem, false, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "module kernel");
 }
 
@@ -522,9 +509,9 @@ nectar_status nectar_decode(nectar_dims dims, const nectar_module_set* mods, con
   NECTAR_TRY(check_ptr(out, "out"));
   NECTAR_TRY(check_local(q_seq, q_pos, Kloc, Vloc, B, T_max, local_len));
   ModParams p;
-  CUtensorMap tw, tq;
+  CUtensorMap tq;
   ModShape sh;
-  NECTAR_TRY(prepare_modules(dims, mods, Q, nq, true, &p, &tw, &tq, &sh));
+  NECTAR_TRY(prepare_modules(dims, mods, Q, nq, true, &p, &tq, &sh));
   p.q_seq = q_seq;
   p.q_pos = q_pos;
   p.Kloc = reinterpret_cast<const __nv_bfloat16*>(Kloc);
@@ -535,7 +522,7 @@ nectar_status nectar_decode(nectar_dims dims, const nectar_module_set* mods, con
   p.qmul = scale * kLog2e;
   p.out = out;
   const int units = dims.L * dims.Hkv * sh.nblk;
-  cudaError_t e = launch_module(tw, tq, p, units, sh.smem, true, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_module(tq, p, units, sh.smem, true, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "decode kernel");
 }
 

@@ -68,10 +68,19 @@ def kch(K):
 
 
 def read_chunked(blob, off, rows, K):
-    """K-chunked [ceil(K/64)][rows][64] -> dense [rows][K]."""
-    n = kch(K) * rows * 64
-    a = blob[off:off + n].reshape(kch(K), rows, 64)
-    return np.concatenate(list(a), axis=1)[:, :K], off + n
+    """Tiled [ceil(rows/128)][ceil(K/64)][tile rows][64], the 16-byte pieces of
+    row i stored in 128-byte-swizzle order (piece j at slot j ^ (i % 8))
+    -> dense [rows][K]."""
+    out = []
+    for m in range((rows + 127) // 128):
+        tr = min(128, rows - 128 * m)
+        n = kch(K) * tr * 64
+        a = blob[off:off + n].reshape(kch(K), tr, 8, 8)
+        slot = np.arange(8)[None, :] ^ (np.arange(tr)[:, None] % 8)      # [row][piece] -> stored slot
+        a = np.take_along_axis(a, np.broadcast_to(slot[None, :, :, None], a.shape), axis=2)
+        out.append(np.concatenate(list(a.reshape(kch(K), tr, 64)), axis=1)[:, :K])
+        off += n
+    return np.concatenate(out, axis=0), off
 
 
 def read_net(blob, off, H, depth, dout, d=128):
@@ -91,7 +100,7 @@ def read_net(blob, off, H, depth, dout, d=128):
     return out, off
 
 
-@pytest.mark.parametrize("widths,depth,hkv", [([64, 32], 2, 2), ([48], 3, 1), ([16, 208], 1, 3)])
+@pytest.mark.parametrize("widths,depth,hkv", [([64, 32], 2, 2), ([48], 3, 1), ([16, 208], 1, 3), ([272], 2, 1)])
 def test_pack_layout(widths, depth, hkv):
     mods = make_modules(len(widths), hkv, widths, 128, seed=3, device="cpu", depth=depth)
     ms = nx.pack_modules(mods, widths, depth, hkv, G=2, device=None)

@@ -1,0 +1,111 @@
+"""Parity at the full sizes of the workloads, in the launch configuration
+bench.py times: every (l, h) runs on the GPU, and sampled heads and tokens
+are recomputed by the oracle one by one."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import long_context_attention_split_b200 as nx
+import oracle
+from nectar_inputs import make_workload
+
+pytestmark = pytest.mark.gpu
+
+ALPHA_TOL = 1e-3
+ATT_TOL = 2e-3
+MLP_TOL = 1e-2
+
+
+def sample_heads(wl, k, seed):
+    rng = np.random.default_rng(seed)
+    hs = {(0, 0), (wl.L - 1, wl.Hkv - 1)}
+    while len(hs) < k:
+        hs.add((int(rng.integers(wl.L)), int(rng.integers(wl.Hkv))))
+    return sorted(hs)
+
+
+def check_exact(wl, alpha, A, heads, tokens):
+    """(alpha, A) of the rows of `tokens` (all G query heads) against the oracle."""
+    for (l, h) in heads:
+        X = wl.Q[l, h][:, tokens].reshape(1, -1, 128).cpu()
+        ao, Ao = oracle.cache_attn(wl.K[l, h][None].cpu(), wl.V[l, h][None].cpu(), X, wl.scale)
+        ag = alpha[l, h][:, tokens].reshape(1, -1).cpu().numpy()
+        Ag = A[l, h][:, tokens].reshape(1, -1, 128).cpu().numpy()
+        vmax = wl.V[l, h].float().abs().max().item()
+        assert np.abs(ag - ao).max() <= ALPHA_TOL, ((l, h), np.abs(ag - ao).max())
+        assert np.abs(Ag - Ao).max() <= ATT_TOL * vmax, ((l, h), np.abs(Ag - Ao).max())
+
+
+def check_decode(wl, out, heads, tokens):
+    """Fused decode output of the rows of `tokens` against the oracle's
+    module forward + merge for those rows."""
+    tok = torch.as_tensor(tokens)
+    for (l, h) in heads:
+        H = wl.widths[l]
+        X = wl.Q[l, h][:, tok].reshape(1, -1, 128).cpu()
+        a = oracle.mlp(oracle.flatten_net(wl.modules[l]["score"], [h]), X, wl.depth, H, 1)[..., 0]
+        At = oracle.mlp(oracle.flatten_net(wl.modules[l]["target"], [h]), X, wl.depth, H, 128)
+        ref = oracle.merge_local(a, At, X, wl.q_seq[tok].cpu(), wl.q_pos[tok].cpu(),
+                                 wl.Kloc[l, h][None].cpu(), wl.Vloc[l, h][None].cpu(), wl.local_len.cpu(), wl.scale)
+        got = out[l, h][:, tok].reshape(1, -1, 128).cpu().numpy()
+        vmax = max(wl.Vloc[l, h].float().abs().max().item(), np.abs(At).max())
+        bound = MLP_TOL * np.abs(a).max() * (np.abs(At).max() + np.abs(ref).max()) + MLP_TOL * np.abs(At).max() \
+            + ATT_TOL * vmax
+        err = np.abs(got - ref).max()
+        assert err <= bound, ((l, h), err, bound)
+
+
+def test_qwen3_4b_targets_full():
+    """36 x 8 heads, n = 61440 with heavy hitters, 4096 query rows per head."""
+    wl = make_workload("qwen3_4b_targets", device="cuda")
+    alpha, A = nx.cache_attn_lse(wl.K, wl.V, wl.Q)
+    torch.cuda.synchronize()
+    assert nx.device_error_flags() == 0
+    check_exact(wl, alpha, A, sample_heads(wl, 3, 1), [0, 511, 1023])
+    del wl, alpha, A
+    torch.cuda.empty_cache()
+
+
+def test_qwen25_7b_decode_full():
+    """28 x 4 heads, G = 7, n = 131072, 64 sequences x 256 local tokens, H = 768."""
+    wl = make_workload("qwen25_7b_decode", device="cuda")
+    mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G, device="cuda")
+    alpha, A = nx.cache_attn_lse(wl.K, wl.V, wl.Q)
+    out = nx.decode(mods, wl.Q, wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len)
+    full = nx.merge_local(alpha, A, wl.Q, wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len)
+    torch.cuda.synchronize()
+    assert nx.device_error_flags() == 0
+    heads = sample_heads(wl, 3, 2)
+    check_exact(wl, alpha, A, heads, [0, 37, 63])
+    check_decode(wl, out, heads, [0, 37, 63])
+    # Eq. (3.4): merging the exact (alpha, A) is full attention over document + local
+    (l, h) = heads[0]
+    tok = torch.tensor([5])
+    ref = oracle.full_attention(wl.K[l, h][None].cpu(), wl.V[l, h][None].cpu(),
+                                wl.Q[l, h][:, tok].reshape(1, -1, 128).cpu(), wl.q_seq[tok].cpu(),
+                                wl.q_pos[tok].cpu(), wl.Kloc[l, h][None].cpu(), wl.Vloc[l, h][None].cpu(),
+                                wl.local_len.cpu(), wl.scale)
+    got = full[l, h][:, tok].reshape(1, -1, 128).cpu().numpy()
+    vmax = max(wl.V[l, h].float().abs().max().item(), wl.Vloc[l, h].float().abs().max().item())
+    assert np.abs(got - ref).max() <= ATT_TOL * vmax
+    del wl, mods, alpha, A, out, full
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("B,rho", [(1, 0.10), (16, 0.10), (256, 0.10), (16, 0.01), (16, 0.05)])
+def test_llama8b_sweep_full(B, rho):
+    """32 x 8 heads, G = 4, n = 65536, 128 local tokens, non-uniform widths."""
+    wl = make_workload("llama8b_sweep", device="cuda", B=B, rho=rho)
+    mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G, device="cuda")
+    alpha, A = nx.cache_attn_lse(wl.K, wl.V, wl.Q)
+    out = nx.decode(mods, wl.Q, wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len)
+    torch.cuda.synchronize()
+    assert nx.device_error_flags() == 0
+    heads = sample_heads(wl, 3, B)
+    tokens = sorted({0, B // 2, B - 1})
+    check_exact(wl, alpha, A, heads, tokens)
+    check_decode(wl, out, heads, tokens)
+    del wl, mods, alpha, A, out
+    torch.cuda.empty_cache()
