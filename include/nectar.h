@@ -126,7 +126,7 @@ NECTAR_API nectar_status nectar_cache_attn_lse(nectar_dims dims, const nectar_bf
  *    threads without ordering -- race on it.
  * Arguments and outputs as for nectar_cache_attn_lse.
  * ------------------------------------------------------------------------ */
-#define NECTAR_STATIC_SCRATCH_BYTES (32u << 20)
+#define NECTAR_STATIC_SCRATCH_BYTES (48u << 20)
 
 NECTAR_API nectar_status nectar_cache_attn_lse_static(nectar_dims dims, const nectar_bf16 *K,
                                                       const nectar_bf16 *V, int64_t n,

@@ -185,7 +185,7 @@ def cache_attn_lse_static(K, V, Q, scale: Optional[float] = None, alpha=None, A=
     return alpha, A
 
 
-STATIC_SCRATCH_BYTES = 32 << 20
+STATIC_SCRATCH_BYTES = 48 << 20
 
 
 # ---------------------------------------------------------------------------

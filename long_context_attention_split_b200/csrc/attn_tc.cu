@@ -1,31 +1,34 @@
 // (i) Exact cached-token attention with many query rows per KV head, on the
 // tensor cores: Eq. (3.1) of "Nectar: Neural Estimation of Cached-Token
-// Attention via Regression" (§2.1) for regression-target generation and
-// large decode batches, where the query rows of one (l, h) reuse each
-// K / V tile enough times that the contraction, not HBM, bounds the time.
+// Attention via Regression" (§2.1), for regression-target generation and
+// large decode batches, where the query rows of one (l, h) reuse each K / V
+// tile often enough that the contraction, not HBM, bounds the time.
 //
-// Work: a unit is (KV head, tile of 128 query rows); its n keys are cut into
-// 128-key tiles and all units' tiles are laid end to end.  CTA c of C (one
-// per SM) takes the contiguous range [c*T/C, (c+1)*T/C): a unit wholly
-// inside one range is finished by that CTA (alpha, A written directly); a
-// unit cut by range boundaries leaves one (m, l, acc) partial per piece, and
-// the combine kernel joins them by log-sum-exp (a separate launch).  A CTA
-// can cut at most two units (the first and the last of its range), so the
-// partials take two slots per CTA whatever the shape.
+// Work unit: (KV head, pair of 128-row query tiles); the pair shares every
+// K / V tile, so each byte of K and V brought on chip serves 256 query rows.
+// Keys come in tiles of 64.  Units are dealt to the CTAs (one per SM) round
+// by round, so the CTAs that work on the query tiles of one head at the same
+// time walk its K / V in step and the repeats hit L2; the last one or two
+// rounds are cut into equal ranges of key tiles (stream-K) so that every CTA
+// ends together.  A unit wholly inside one CTA is finished there (alpha, A
+// written directly); a unit cut between CTAs leaves one (m, l, acc) partial
+// per piece -- at most two per CTA -- joined by log-sum-exp in a second
+// launch, so no CTA ever waits on another.
 //
-// Per tile, tcgen05 (kind::f16, cta_group::1, fp32 accumulation in TMEM):
-//   S = Q K^T   M = 128 rows, N = 128 keys, K = d    (A, B K-major, SW128)
-//   O += P V    M = 128 rows, N = d, K = 128 keys    (P K-major from smem,
-//                                                     V MN-major, SW128)
-// S is double-buffered in TMEM so S_{j+1} runs while the softmax warps turn
-// S_j into P_j.  Softmax keeps a per-row running maximum m and moves it only
-// when a tile's maximum exceeds it by more than 2^8; O is then rescaled in
-// TMEM (rare), and the final normalisation by the same 2^m makes the result
-// the exact quantity.  The row sum l adds the bf16-rounded weights that the
-// P V product uses, so A stays a convex combination of the v_j.
+// Per key tile and query tile t (tcgen05 kind::f16, cta_group::1, fp32 in
+// TMEM):
+//   S_t = Q_t K^T    M = 128, N = 64 keys, K = d     A, B K-major SW128
+//   O_t += P_t V     M = 128, N = d, K = 64 keys     P K-major, V MN-major
+// S_t is double-buffered in TMEM (S_t of the next tile runs while softmax
+// warpgroup t turns this one into bf16 P_t in shared memory, also double-
+// buffered).  The running row maximum moves only when a tile's maximum
+// exceeds it by more than 2^8; O_t is then rescaled in TMEM (warp-uniform
+// decision, as TMEM access is warp-collective), and the final division by
+// the same 2^m makes the result exact.  The row sum adds the bf16-rounded
+// weights that the P V product uses, so A stays a convex combination.
 //
-// Warps: 0..3 softmax / epilogue (thread = query row = TMEM lane),
-//        4 TMA producer, 5 MMA issuer and TMEM owner.
+// Warps: 0..3 softmax / epilogue of query tile 0, 4..7 of tile 1 (thread =
+// row = TMEM lane), 8 Q and K producer, 9 V producer, 10 MMA issuer.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -34,18 +37,22 @@
 
 namespace nectar {
 
-constexpr int kTcRows = 128;     // query rows per unit
-constexpr int kTcKeys = 128;     // keys per tile
-constexpr int kTcThreads = 192;
-constexpr uint32_t kTcTileBytes = 128 * 128 * 2;   // 32 KB: 128 x 128 bf16
+constexpr int kTcRows = 128;                       // query rows per tile
+constexpr int kTcUnitRows = 2 * kTcRows;           // two tiles per unit
+constexpr int kTcKeys = 64;                        // keys per tile
+constexpr int kTcStages = 3;                       // K and V ring depth
+constexpr int kTcThreads = 11 * 32;
+constexpr uint32_t kQBytes = kTcRows * kD * 2;     // 32 KB
+constexpr uint32_t kKVBytes = kTcKeys * kD * 2;    // 16 KB
+constexpr uint32_t kPBytes = kTcRows * kTcKeys * 2;   // 16 KB
 
 struct TcSmem {
-  static constexpr uint32_t q = 0;                           // 32 KB
-  static constexpr uint32_t k = q + kTcTileBytes;            // 2 x 32 KB
-  static constexpr uint32_t v = k + 2 * kTcTileBytes;        // 2 x 32 KB
-  static constexpr uint32_t p = v + 2 * kTcTileBytes;        // 2 x 32 KB
-  static constexpr uint32_t bars = p + 2 * kTcTileBytes;     // 20 barriers
-  static constexpr uint32_t tslot = bars + 20 * 8;
+  static constexpr uint32_t q = 0;                                  // 2 x 32 KB
+  static constexpr uint32_t k = q + 2 * kQBytes;                    // 3 x 16 KB
+  static constexpr uint32_t v = k + kTcStages * kKVBytes;           // 3 x 16 KB
+  static constexpr uint32_t p = v + kTcStages * kKVBytes;           // [tile][buf] 4 x 16 KB
+  static constexpr uint32_t bars = p + 4 * kPBytes;                 // 40 barriers
+  static constexpr uint32_t tslot = bars + 40 * 8;
   static constexpr uint32_t total = tslot + 16;
 };
 
@@ -53,11 +60,47 @@ __host__ __device__ __forceinline__ int tc_first_cta(int64_t t, int64_t total, i
   return static_cast<int>(((t + 1) * static_cast<int64_t>(C) - 1) / total);
 }
 
-// element (row, key) of a K-major SW128 128 x 128 bf16 tile stored as two
-// 64-column halves of 128 rows x 128 bytes
-__device__ __forceinline__ uint32_t tile_off(int row, int col) {
-  return static_cast<uint32_t>((col >> 6) * (128 * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) +
-                               ((col & 7) << 1));
+// One contiguous piece of a unit's key tiles handled by a CTA.
+struct TcSeg {
+  int64_t unit;     // global unit index
+  int64_t k0, k1;   // key tiles [k0, k1)
+  bool whole;       // the CTA does every key tile of the unit
+  int slot;         // partial slot when not whole (0: first unit of the CTA's range, 1: last)
+};
+
+// CTA c's segments: R data-parallel units c + r*C, then its stream-K range.
+__device__ __forceinline__ int tc_num_segs(const TcParams& p, int c) {
+  const int64_t Tsk = p.sk_units * p.tph;
+  if (Tsk == 0) return p.dp_rounds;
+  const int64_t s0 = static_cast<int64_t>(c) * Tsk / p.C, s1 = static_cast<int64_t>(c + 1) * Tsk / p.C;
+  if (s1 <= s0) return p.dp_rounds;
+  return p.dp_rounds + static_cast<int>((s1 - 1) / p.tph - s0 / p.tph + 1);
+}
+__device__ __forceinline__ TcSeg tc_seg(const TcParams& p, int c, int i) {
+  TcSeg sg;
+  if (i < p.dp_rounds) {
+    sg.unit = c + static_cast<int64_t>(i) * p.C;
+    sg.k0 = 0;
+    sg.k1 = p.tph;
+    sg.whole = true;
+    sg.slot = 0;
+    return sg;
+  }
+  const int64_t Tsk = p.sk_units * p.tph;
+  const int64_t s0 = static_cast<int64_t>(c) * Tsk / p.C, s1 = static_cast<int64_t>(c + 1) * Tsk / p.C;
+  const int64_t ul = s0 / p.tph + (i - p.dp_rounds);
+  const int64_t b = ul * p.tph;
+  sg.unit = static_cast<int64_t>(p.dp_rounds) * p.C + ul;
+  sg.k0 = (s0 > b ? s0 : b) - b;
+  sg.k1 = (s1 < b + p.tph ? s1 : b + p.tph) - b;
+  sg.whole = (sg.k0 == 0 && sg.k1 == p.tph);
+  sg.slot = (ul == s0 / p.tph) ? 0 : 1;
+  return sg;
+}
+
+// element (row, key) of a K-major SW128 tile of 128 rows x 64 keys
+__device__ __forceinline__ uint32_t p_off(int row, int col) {
+  return static_cast<uint32_t>(row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + ((col & 7) << 1));
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -67,35 +110,38 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TcSmem::bars);
   const uint32_t b_qfull = smem_u32(bars + 0), b_qempty = smem_u32(bars + 1);
-  const uint32_t b_kfull = smem_u32(bars + 2), b_kempty = smem_u32(bars + 4);     // [2] each
-  const uint32_t b_vfull = smem_u32(bars + 6), b_vempty = smem_u32(bars + 8);
-  const uint32_t b_sfull = smem_u32(bars + 10), b_sfree = smem_u32(bars + 12);
-  const uint32_t b_pfull = smem_u32(bars + 14), b_pvdone = smem_u32(bars + 16);
-  const uint32_t b_ofree = smem_u32(bars + 18);
+  const uint32_t b_kfull = smem_u32(bars + 2), b_kempty = smem_u32(bars + 5);     // [3]
+  const uint32_t b_vfull = smem_u32(bars + 8), b_vempty = smem_u32(bars + 11);    // [3]
+  // [tile t][buf b] at + 8 * (2 t + b)
+  const uint32_t b_sfull = smem_u32(bars + 14), b_sfree = smem_u32(bars + 18);
+  const uint32_t b_pfull = smem_u32(bars + 22), b_pvdone = smem_u32(bars + 26);
+  const uint32_t b_ofree = smem_u32(bars + 30);                                   // [tile]
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + TcSmem::tslot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x;
-  const int64_t t0 = static_cast<int64_t>(c) * p.total / p.C;
-  const int64_t t1 = static_cast<int64_t>(c + 1) * p.total / p.C;
+  const int nseg = tc_num_segs(p, c);
 
   if (threadIdx.x == 0) {
     mbar_init(b_qfull, 1);
     mbar_init(b_qempty, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kTcStages; ++s) {
       mbar_init(b_kfull + 8 * s, 1);
       mbar_init(b_kempty + 8 * s, 1);
       mbar_init(b_vfull + 8 * s, 1);
       mbar_init(b_vempty + 8 * s, 1);
-      mbar_init(b_sfull + 8 * s, 1);
-      mbar_init(b_sfree + 8 * s, 128);
-      mbar_init(b_pfull + 8 * s, 128);
-      mbar_init(b_pvdone + 8 * s, 1);
     }
-    mbar_init(b_ofree, 128);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(b_sfull + 8 * i, 1);
+      mbar_init(b_sfree + 8 * i, 128);
+      mbar_init(b_pfull + 8 * i, 128);
+      mbar_init(b_pvdone + 8 * i, 1);
+    }
+    mbar_init(b_ofree + 0, 128);
+    mbar_init(b_ofree + 8, 128);
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 10) {
     tmem_alloc(smem_u32(tslot), 512);
     tmem_relinquish();
   }
@@ -103,144 +149,223 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const uint32_t tmem_o = tmem + 256;
+  // TMEM columns: S[t][b] at 128 t + 64 b, O[t] at 256 + 128 t
 
-  if (warp == 4) {
-    // --------------------------- TMA producer ---------------------------
+  auto two_tiles = [&](int64_t unit) {
+    const int64_t qp = unit % p.qpairs;
+    return qp * kTcUnitRows + kTcRows < p.rows_total;
+  };
+
+  if (warp == 8) {
+    // ----------------------- Q and K producer -----------------------
     if (lane == 0) {
       prefetch_tmap(&tmap_q);
       prefetch_tmap(&tmap_k);
-      prefetch_tmap(&tmap_v);
-      const uint64_t pol_kv = policy_evict_first();
-      const uint64_t pol_q = policy_evict_last();
-      int64_t cur = -1;
-      uint32_t qn = 0;
+      const uint64_t pol_kv = policy_evict_normal();
+      const uint64_t pol_q = policy_evict_first();
       bool ok = true;
-      int64_t jj = 0;
-      for (int64_t t = t0; t < t1 && ok; ++t, ++jj) {
-        const int64_t u = t / p.tph;
-        if (u != cur) {
-          if (cur >= 0) ok = mbar_wait(b_qempty, (qn - 1) & 1, p.err);
-          if (!ok) break;
-          const int64_t hd = u / p.qtiles;
-          const int qt = static_cast<int>(u % p.qtiles);
-          mbar_arrive_expect_tx(b_qfull, kTcTileBytes);
-          tma_load_3d(smem_u32(smem + TcSmem::q), &tmap_q, 0, qt * kTcRows, static_cast<int>(hd), b_qfull, pol_q);
-          tma_load_3d(smem_u32(smem + TcSmem::q + kTcTileBytes / 2), &tmap_q, 64, qt * kTcRows, static_cast<int>(hd),
-                      b_qfull, pol_q);
-          ++qn;
-          cur = u;
+      uint32_t qn = 0, it = 0;
+      for (int si = 0; si < nseg && ok; ++si) {
+        const TcSeg sg = tc_seg(p, c, si);
+        const int64_t hd = sg.unit / p.qpairs;
+        const int qp = static_cast<int>(sg.unit % p.qpairs);
+        if (qn > 0 && !(ok = mbar_wait(b_qempty, (qn - 1) & 1, p.err))) break;
+        const bool two = two_tiles(sg.unit);
+        mbar_arrive_expect_tx(b_qfull, (two ? 2 : 1) * kQBytes);
+        tma_load_4d(smem_u32(smem + TcSmem::q), &tmap_q, 0, qp * kTcUnitRows, 0, static_cast<int>(hd), b_qfull, pol_q);
+        if (two)
+          tma_load_4d(smem_u32(smem + TcSmem::q + kQBytes), &tmap_q, 0, qp * kTcUnitRows + kTcRows, 0,
+                      static_cast<int>(hd), b_qfull, pol_q);
+        ++qn;
+        for (int64_t kt = sg.k0; kt < sg.k1; ++kt, ++it) {
+          const uint32_t s = it % kTcStages;
+          if (it >= kTcStages && !(ok = mbar_wait(b_kempty + 8 * s, ((it / kTcStages) - 1) & 1, p.err))) break;
+          mbar_arrive_expect_tx(b_kfull + 8 * s, kKVBytes);
+          tma_load_4d(smem_u32(smem + TcSmem::k + s * kKVBytes), &tmap_k, 0, static_cast<int>(kt * kTcKeys), 0,
+                      static_cast<int>(hd), b_kfull + 8 * s, pol_kv);
         }
-        const int64_t hd = u / p.qtiles;
-        const int key0 = static_cast<int>((t - u * p.tph) * kTcKeys);
-        const int s = static_cast<int>(jj & 1);
-        const uint32_t ph = static_cast<uint32_t>(((jj >> 1) - 1) & 1);
-        if (jj >= 2 && !(ok = mbar_wait(b_kempty + 8 * s, ph, p.err))) break;
-        mbar_arrive_expect_tx(b_kfull + 8 * s, kTcTileBytes);
-        tma_load_3d(smem_u32(smem + TcSmem::k + s * kTcTileBytes), &tmap_k, 0, key0, static_cast<int>(hd),
-                    b_kfull + 8 * s, pol_kv);
-        tma_load_3d(smem_u32(smem + TcSmem::k + s * kTcTileBytes + kTcTileBytes / 2), &tmap_k, 64, key0,
-                    static_cast<int>(hd), b_kfull + 8 * s, pol_kv);
-        if (jj >= 2 && !(ok = mbar_wait(b_vempty + 8 * s, ph, p.err))) break;
-        mbar_arrive_expect_tx(b_vfull + 8 * s, kTcTileBytes);
-        tma_load_3d(smem_u32(smem + TcSmem::v + s * kTcTileBytes), &tmap_v, 0, key0, static_cast<int>(hd),
-                    b_vfull + 8 * s, pol_kv);
-        tma_load_3d(smem_u32(smem + TcSmem::v + s * kTcTileBytes + kTcTileBytes / 2), &tmap_v, 64, key0,
-                    static_cast<int>(hd), b_vfull + 8 * s, pol_kv);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
+    // --------------------------- V producer ---------------------------
+    if (lane == 0) {
+      prefetch_tmap(&tmap_v);
+      const uint64_t pol_kv = policy_evict_normal();
+      bool ok = true;
+      uint32_t it = 0;
+      for (int si = 0; si < nseg && ok; ++si) {
+        const TcSeg sg = tc_seg(p, c, si);
+        const int64_t hd = sg.unit / p.qpairs;
+        for (int64_t kt = sg.k0; kt < sg.k1; ++kt, ++it) {
+          const uint32_t s = it % kTcStages;
+          if (it >= kTcStages && !(ok = mbar_wait(b_vempty + 8 * s, ((it / kTcStages) - 1) & 1, p.err))) break;
+          mbar_arrive_expect_tx(b_vfull + 8 * s, kKVBytes);
+          tma_load_4d(smem_u32(smem + TcSmem::v + s * kKVBytes), &tmap_v, 0, static_cast<int>(kt * kTcKeys), 0,
+                      static_cast<int>(hd), b_vfull + 8 * s, pol_kv);
+        }
+      }
+    }
+  } else if (warp == 10) {
     // ---------------------------- MMA issuer ----------------------------
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
-      const uint32_t idesc_o = idesc_bf16_f32(128, 128, 0, 1);
-      const uint32_t sq = smem_u32(smem + TcSmem::q);
+      const uint32_t idesc_s = idesc_bf16_f32(128, kTcKeys, 0, 0);
+      const uint32_t idesc_o = idesc_bf16_f32(128, kD, 0, 1);
       bool ok = true;
-      uint32_t qn = 0;      // units whose Q has been consumed
-      uint32_t un = 0;      // units whose first P V has been issued
-      // O += P_x V_x for local tile x; the first P V of a unit starts O
-      // from zero, after the epilogue has read the previous unit's O.
-      auto issue_pv = [&](int64_t x) {
-        const int s = static_cast<int>(x & 1);
-        const int64_t tx = t0 + x;
-        const bool first = (x == 0) || (tx / p.tph != (tx - 1) / p.tph);
-        if (ok) ok = mbar_wait(b_pfull + 8 * s, static_cast<uint32_t>((x >> 1) & 1), p.err);
-        if (ok) ok = mbar_wait(b_vfull + 8 * s, static_cast<uint32_t>((x >> 1) & 1), p.err);
-        if (ok && first && un > 0) ok = mbar_wait(b_ofree, (un - 1) & 1, p.err);
-        if (first) ++un;
-        if (!ok) return;
-        tc_fence_after();
-        const uint32_t pa = smem_u32(smem + TcSmem::p + s * kTcTileBytes);
-        const uint32_t vb = smem_u32(smem + TcSmem::v + s * kTcTileBytes);
+      uint32_t qn = 0, it = 0;
+      uint32_t cs[2] = {0, 0};   // S tiles issued per query tile
+      uint32_t cp[2] = {0, 0};   // P V products issued per query tile
+      uint32_t un[2] = {0, 0};   // units whose O was started, per query tile
+      // O_t += P_t V for key tile `vit` (the ring index of its V)
+      auto issue_pv = [&](uint32_t vit, bool two, bool first) {
+        const uint32_t vs = vit % kTcStages;
+        if (ok) ok = mbar_wait(b_vfull + 8 * vs, (vit / kTcStages) & 1, p.err);
+        for (int t = 0; t < (two ? 2 : 1); ++t) {
+          const uint32_t b = cp[t] & 1;
+          if (ok) ok = mbar_wait(b_pfull + 8 * (2 * t + b), (cp[t] >> 1) & 1, p.err);
+          if (ok && first && un[t] > 0) ok = mbar_wait(b_ofree + 8 * t, (un[t] - 1) & 1, p.err);
+          if (first) ++un[t];
+          ++cp[t];
+          if (!ok) continue;
+          tc_fence_after();
+          const uint32_t pa = smem_u32(smem + TcSmem::p + (2 * t + b) * kPBytes);
+          const uint32_t vb = smem_u32(smem + TcSmem::v + vs * kKVBytes);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          // A = P, K-major: keys 16kk.. sit in half kk/4 at byte (kk%4)*32
-          const uint64_t ad = sdesc_sw128(pa + (kk >> 2) * (kTcTileBytes / 2) + (kk & 3) * 32, 16, 1024);
-          // B = V, MN-major: 16 keys = two 8-row groups of 128 B; the two
-          // 64-wide d halves are kTcTileBytes / 2 apart
-          const uint64_t bd = sdesc_sw128(vb + kk * 2048, kTcTileBytes / 2, 1024);
-          mma_bf16_ss(tmem_o, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
+          for (int kk = 0; kk < kTcKeys / 16; ++kk) {
+            // A = P (K-major, one 64-key chunk): keys 16 kk.. at byte 32 kk.
+            // B = V (MN-major): 16 keys = two 8-row groups of 128 B; the two
+            // 64-wide d halves are kKVBytes / 2 apart
+            mma_bf16_ss(tmem + 256 + 128 * t, sdesc_sw128(pa + kk * 32, 16, 1024),
+                        sdesc_sw128(vb + kk * 2048, kKVBytes / 2, 1024), idesc_o, (first && kk == 0) ? 0u : 1u);
+          }
+          mma_commit(b_pvdone + 8 * (2 * t + b));
         }
-        mma_commit(b_vempty + 8 * s);
-        mma_commit(b_pvdone + 8 * s);
+        mma_commit(b_vempty + 8 * vs);
       };
-      int64_t jj = 0;
-      for (int64_t t = t0; t < t1 && ok; ++t, ++jj) {
-        const int64_t u = t / p.tph;
-        const bool unit_first = (t == t0) || (t % p.tph == 0);
-        const bool unit_last = (t + 1 == t1) || ((t + 1) % p.tph == 0);
-        if (unit_first) {
-          ok = mbar_wait(b_qfull, qn & 1, p.err);
-          ++qn;
-          if (!ok) break;
-        }
-        (void)u;
-        const int s = static_cast<int>(jj & 1);
-        if (!(ok = mbar_wait(b_kfull + 8 * s, static_cast<uint32_t>((jj >> 1) & 1), p.err))) break;
-        if (jj >= 2 && !(ok = mbar_wait(b_sfree + 8 * s, static_cast<uint32_t>(((jj >> 1) - 1) & 1), p.err))) break;
-        tc_fence_after();
-        const uint32_t kb = smem_u32(smem + TcSmem::k + s * kTcTileBytes);
+      bool prev_two = false, prev_first = false, have_prev = false;
+      for (int si = 0; si < nseg && ok; ++si) {
+        const TcSeg sg = tc_seg(p, c, si);
+        const bool two = two_tiles(sg.unit);
+        ok = mbar_wait(b_qfull, qn & 1, p.err);
+        ++qn;
+        for (int64_t kt = sg.k0; kt < sg.k1 && ok; ++kt, ++it) {
+          const uint32_t ks = it % kTcStages;
+          if (!(ok = mbar_wait(b_kfull + 8 * ks, (it / kTcStages) & 1, p.err))) break;
+          for (int t = 0; t < (two ? 2 : 1) && ok; ++t) {
+            const uint32_t b = cs[t] & 1;
+            if (cs[t] >= 2 && !(ok = mbar_wait(b_sfree + 8 * (2 * t + b), ((cs[t] >> 1) - 1) & 1, p.err))) break;
+            tc_fence_after();
+            const uint32_t qa = smem_u32(smem + TcSmem::q + t * kQBytes);
+            const uint32_t kb = smem_u32(smem + TcSmem::k + ks * kKVBytes);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * (kTcTileBytes / 2) + (kk & 3) * 32;
-          mma_bf16_ss(tmem + s * 128, sdesc_sw128(sq + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_s,
-                      kk != 0);
+            for (int kk = 0; kk < 8; ++kk) {
+              // d 16 kk..: half kk / 4, byte (kk % 4) * 32 inside the 128-B rows
+              mma_bf16_ss(tmem + 128 * t + 64 * b,
+                          sdesc_sw128(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024),
+                          sdesc_sw128(kb + (kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32, 16, 1024), idesc_s, kk != 0);
+            }
+            mma_commit(b_sfull + 8 * (2 * t + b));
+            ++cs[t];
+          }
+          mma_commit(b_kempty + 8 * ks);
+          if (kt + 1 == sg.k1) mma_commit(b_qempty);
+          if (have_prev) issue_pv(it - 1, prev_two, prev_first);
+          prev_two = two;
+          prev_first = (kt == sg.k0);
+          have_prev = true;
         }
-        mma_commit(b_kempty + 8 * s);
-        mma_commit(b_sfull + 8 * s);
-        if (unit_last) mma_commit(b_qempty);
-        if (jj >= 1) issue_pv(jj - 1);
       }
-      if (ok && jj >= 1) issue_pv(jj - 1);
+      if (ok && have_prev) issue_pv(it - 1, prev_two, prev_first);
     }
   } else {
-    // ------------------------ softmax + epilogue ------------------------
-    const int row = (warp & 3) * 32 + lane;              // TMEM lane = query row in the tile
+    // --------------------- softmax + epilogue (tile t) ---------------------
+    const int t = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;               // TMEM lane = row of the tile
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    float m = -INFINITY, l = 0.f;
-    int64_t cur = -1;
+    const uint32_t tS = tmem + 128 * t, tO = tmem + 256 + 128 * t;
     bool ok = true;
-    uint32_t on = 0;
-    int64_t jj = 0;
-    auto finalize = [&](int64_t u, int64_t jlast) {
-      // wait for the unit's last P V, then write alpha, A (or a partial)
-      const int s = static_cast<int>(jlast & 1);
-      if (ok) ok = mbar_wait(b_pvdone + 8 * s, static_cast<uint32_t>((jlast >> 1) & 1), p.err);
+    uint32_t cnt = 0;   // S tiles consumed by this tile
+    for (int si = 0; si < nseg; ++si) {
+      const TcSeg sg = tc_seg(p, c, si);
+      if (t == 1 && !two_tiles(sg.unit)) continue;
+      float m = -INFINITY, l = 0.f;
+      for (int64_t kt = sg.k0; kt < sg.k1; ++kt, ++cnt) {
+        const uint32_t b = cnt & 1;
+        const int64_t nvalid = p.n - kt * kTcKeys;
+        if (ok) ok = mbar_wait(b_sfull + 8 * (2 * t + b), (cnt >> 1) & 1, p.err);
+        tc_fence_after();
+        float sc[kTcKeys];
+#pragma unroll
+        for (int cb = 0; cb < kTcKeys; cb += 32) {
+          uint32_t v[32];
+          NECTAR_TMEM_LD32(tS + 64 * b + lane_base + cb, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sc[cb + e] = __uint_as_float(v[e]) * p.qmul;
+        }
+        tc_fence_before();
+        mbar_arrive(b_sfree + 8 * (2 * t + b));
+        float bm = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < kTcKeys; ++e) {
+          if (e >= nvalid) sc[e] = -INFINITY;
+          bm = fmaxf(bm, sc[e]);
+        }
+        const bool need = bm > m + kRescaleSlack;
+        const float corr = need ? exp2_shift(m, bm) : 1.0f;
+        if (need) {
+          l *= corr;
+          m = bm;
+        }
+        if (__any_sync(0xffffffffu, need) && kt != sg.k0) {
+          // O_t holds the earlier key tiles of this unit: wait for their
+          // last P V, then rescale it in TMEM (warp-collective)
+          const uint32_t pc = cnt - 1;
+          if (ok) ok = mbar_wait(b_pvdone + 8 * (2 * t + (pc & 1)), (pc >> 1) & 1, p.err);
+          tc_fence_after();
+#pragma unroll
+          for (int cb = 0; cb < kD; cb += 32) {
+            uint32_t v[32];
+            NECTAR_TMEM_LD32(tO + lane_base + cb, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * corr);
+            NECTAR_TMEM_ST32(tO + lane_base + cb, v);
+          }
+          tmem_st_wait();
+        }
+        // P buffer b was last read by the P V of this tile's S count cnt - 2
+        if (cnt >= 2 && ok) ok = mbar_wait(b_pvdone + 8 * (2 * t + b), ((cnt >> 1) - 1) & 1, p.err);
+        uint8_t* pt = smem + TcSmem::p + (2 * t + b) * kPBytes;
+        float rs = 0.f;
+#pragma unroll
+        for (int c8 = 0; c8 < kTcKeys / 8; ++c8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            w[e] = pack_bf16x2(exp2_shift(sc[c8 * 8 + 2 * e], m), exp2_shift(sc[c8 * 8 + 2 * e + 1], m));
+            rs += bf16lo(w[e]) + bf16hi(w[e]);
+          }
+          *reinterpret_cast<uint4*>(pt + p_off(row, c8 * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        l += rs;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(b_pfull + 8 * (2 * t + b));
+      }
+      // ------------- epilogue of this unit for tile t -------------
+      const uint32_t pc = cnt - 1;
+      if (ok) ok = mbar_wait(b_pvdone + 8 * (2 * t + (pc & 1)), (pc >> 1) & 1, p.err);
       tc_fence_after();
-      const int64_t hd = u / p.qtiles;
-      const int qt = static_cast<int>(u % p.qtiles);
-      const int64_t r = static_cast<int64_t>(qt) * kTcRows + row;
-      const int f = tc_first_cta(u * p.tph, p.total, p.C);
-      const int la = tc_first_cta(u * p.tph + p.tph - 1, p.total, p.C);
-      const bool whole = (f == la);
+      const int64_t hd = sg.unit / p.qpairs;
+      const int64_t qp = sg.unit % p.qpairs;
+      const int64_t r = qp * kTcUnitRows + t * kTcRows + row;
       float* dst;
       float inv = 1.f;
-      if (whole) {
+      if (sg.whole) {
         dst = p.A + (hd * p.rows_total + r) * kD;
         inv = 1.0f / l;
       } else {
-        const int slot = (u == t0 / p.tph) ? 0 : 1;    // first or last unit of this CTA's range
-        const int64_t prow = (static_cast<int64_t>(c) * 2 + slot) * kTcRows + row;
+        const int64_t prow = (static_cast<int64_t>(c) * 2 + sg.slot) * kTcUnitRows + t * kTcRows + row;
         dst = p.ws_acc + prow * kD;
         if (r < p.rows_total) {
           p.ws_ml[prow * 2] = m;
@@ -248,9 +373,9 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         }
       }
 #pragma unroll
-      for (int cb = 0; cb < 128; cb += 32) {
+      for (int cb = 0; cb < kD; cb += 32) {
         uint32_t v[32];
-        NECTAR_TMEM_LD32(tmem_o + lane_base + cb, v);
+        NECTAR_TMEM_LD32(tO + lane_base + cb, v);
         tmem_ld_wait();
         if (ok && r < p.rows_total) {
 #pragma unroll
@@ -260,115 +385,39 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
                             __uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv);
         }
       }
-      if (whole && ok && r < p.rows_total) p.alpha[hd * p.rows_total + r] = (m + log2f(l)) * kLn2;
+      if (sg.whole && ok && r < p.rows_total) p.alpha[hd * p.rows_total + r] = (m + log2f(l)) * kLn2;
       tc_fence_before();
-      mbar_arrive(b_ofree);
-      ++on;
-    };
-    for (int64_t t = t0; t < t1; ++t, ++jj) {
-      const int64_t u = t / p.tph;
-      if (u != cur) {
-        if (cur >= 0) finalize(cur, jj - 1);
-        cur = u;
-        m = -INFINITY;
-        l = 0.f;
-      }
-      const bool unit_first = (t == t0) || (t % p.tph == 0);
-      const int s = static_cast<int>(jj & 1);
-      const int nvalid = static_cast<int>(p.n - (t - u * p.tph) * kTcKeys);   // keys of this tile < n
-      if (ok) ok = mbar_wait(b_sfull + 8 * s, static_cast<uint32_t>((jj >> 1) & 1), p.err);
-      tc_fence_after();
-      float sc[128];
-#pragma unroll
-      for (int cb = 0; cb < 128; cb += 32) {
-        uint32_t v[32];
-        NECTAR_TMEM_LD32(tmem + s * 128 + lane_base + cb, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) sc[cb + e] = __uint_as_float(v[e]) * p.qmul;
-      }
-      tc_fence_before();
-      mbar_arrive(b_sfree + 8 * s);
-      float bm = -INFINITY;
-#pragma unroll
-      for (int e = 0; e < 128; ++e) {
-        if (e >= nvalid) sc[e] = -INFINITY;
-        bm = fmaxf(bm, sc[e]);
-      }
-      // Moving the maximum is decided per row, but the TMEM load / store of O
-      // is warp-collective (.sync.aligned), so the whole warp takes that path
-      // and rows that keep their maximum scale by 1.
-      const bool need = bm > m + kRescaleSlack;
-      const float corr = need ? exp2_shift(m, bm) : 1.0f;
-      if (need) {
-        l *= corr;
-        m = bm;
-      }
-      if (__any_sync(0xffffffffu, need) && !unit_first) {
-        // O holds the previous tiles of this unit: wait for their last P V,
-        // then rescale O in TMEM
-        const int64_t jp = jj - 1;
-        if (ok) ok = mbar_wait(b_pvdone + 8 * (jp & 1), static_cast<uint32_t>((jp >> 1) & 1), p.err);
-        tc_fence_after();
-#pragma unroll
-        for (int cb = 0; cb < 128; cb += 32) {
-          uint32_t v[32];
-          NECTAR_TMEM_LD32(tmem_o + lane_base + cb, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * corr);
-          NECTAR_TMEM_ST32(tmem_o + lane_base + cb, v);
-        }
-        tmem_st_wait();
-      }
-      // P buffer s was last read by the P V of tile jj - 2
-      if (jj >= 2 && ok) ok = mbar_wait(b_pvdone + 8 * s, static_cast<uint32_t>(((jj >> 1) - 1) & 1), p.err);
-      uint8_t* pt = smem + TcSmem::p + s * kTcTileBytes;
-      float rs = 0.f;
-#pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = exp2_shift(sc[c8 * 8 + 2 * e], m);
-          const float p1 = exp2_shift(sc[c8 * 8 + 2 * e + 1], m);
-          w[e] = pack_bf16x2(p0, p1);
-          rs += bf16lo(w[e]) + bf16hi(w[e]);
-        }
-        *reinterpret_cast<uint4*>(pt + tile_off(row, c8 * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      l += rs;
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(b_pfull + 8 * s);
+      mbar_arrive(b_ofree + 8 * t);
     }
-    if (cur >= 0) finalize(cur, jj - 1);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 10) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
-// One warp per (head, row) of a unit that was cut between CTAs: join its
-// partials (units inside one CTA were written by the main kernel).
+// One warp per (head, row) of a stream-K unit that was cut between CTAs:
+// join its partials (every other unit was written by the main kernel).
 __global__ void cache_attn_tc_combine_kernel(const TcParams p) {
   const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= static_cast<int64_t>(p.heads) * p.rows_total) return;
   const int64_t hd = gw / p.rows_total, r = gw % p.rows_total;
-  const int64_t u = hd * p.qtiles + r / kTcRows;
-  const int rr = static_cast<int>(r % kTcRows);
-  const int f = tc_first_cta(u * p.tph, p.total, p.C);
-  const int la = tc_first_cta(u * p.tph + p.tph - 1, p.total, p.C);
+  const int64_t unit = hd * p.qpairs + r / kTcUnitRows;
+  const int rr = static_cast<int>(r % kTcUnitRows);
+  const int64_t ul = unit - static_cast<int64_t>(p.dp_rounds) * p.C;   // stream-K local unit
+  if (ul < 0) return;
+  const int64_t Tsk = p.sk_units * p.tph;
+  const int f = tc_first_cta(ul * p.tph, Tsk, p.C);
+  const int la = tc_first_cta(ul * p.tph + p.tph - 1, Tsk, p.C);
   if (f == la) return;
-  // the piece of CTA cc sits in slot 0 if u is the first unit of cc's range
+  // the piece of CTA cc sits in slot 0 if ul is the first unit of cc's range
   auto prow_of = [&](int cc) {
-    const int64_t first_unit = (static_cast<int64_t>(cc) * p.total / p.C) / p.tph;
-    return (static_cast<int64_t>(cc) * 2 + (u == first_unit ? 0 : 1)) * kTcRows + rr;
+    const int64_t first = (static_cast<int64_t>(cc) * Tsk / p.C) / p.tph;
+    return (static_cast<int64_t>(cc) * 2 + (ul == first ? 0 : 1)) * kTcUnitRows + rr;
   };
   float M = -INFINITY;
   for (int cc = f; cc <= la; ++cc) M = fmaxf(M, p.ws_ml[prow_of(cc) * 2]);
@@ -394,16 +443,20 @@ __global__ void cache_attn_tc_combine_kernel(const TcParams p) {
 // ---------------------------------------------------------------------------
 TcPlan plan_tc(int heads, int64_t n, int64_t rows, int num_sms) {
   TcPlan pl{};
-  pl.qtiles = static_cast<int>((rows + kTcRows - 1) / kTcRows);
+  pl.qpairs = static_cast<int>((rows + kTcUnitRows - 1) / kTcUnitRows);
   pl.tph = (n + kTcKeys - 1) / kTcKeys;
-  const int64_t units = static_cast<int64_t>(heads) * pl.qtiles;
-  pl.total = units * pl.tph;
+  const int64_t units = static_cast<int64_t>(heads) * pl.qpairs;
   int64_t C = num_sms;
-  if (C > pl.total) C = pl.total;
+  if (C > units * pl.tph) C = units * pl.tph;
   if (C < 1) C = 1;
   pl.C = static_cast<int>(C);
-  pl.S_max = 2;    // partial slots per CTA
-  pl.ws_bytes = static_cast<size_t>(pl.C) * 2 * kTcRows * (kD + 2) * sizeof(float);
+  // whole rounds of units first (the CTAs of one head then read its K / V
+  // in step), the rest cut evenly by key tiles
+  int64_t R = units / C;
+  if (units % C != 0 && R > 0) R -= 1;
+  pl.dp_rounds = static_cast<int>(R);
+  pl.sk_units = units - R * C;
+  pl.ws_bytes = static_cast<size_t>(pl.C) * 2 * kTcUnitRows * (kD + 2) * sizeof(float);
   pl.smem = TcSmem::total + 1024;
   return pl;
 }
@@ -417,6 +470,7 @@ cudaError_t launch_cache_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk, c
   cache_attn_tc_kernel<<<p.C, kTcThreads, smem, stream>>>(tq, tk, tv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (p.sk_units == 0) return cudaSuccess;
   const int64_t warps = static_cast<int64_t>(p.heads) * p.rows_total;
   const int64_t blocks = (warps * 32 + 255) / 256;
   cache_attn_tc_combine_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);

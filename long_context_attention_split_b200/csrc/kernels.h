@@ -47,21 +47,23 @@ struct TcParams {
   int64_t n;
   int heads;
   int64_t rows_total;
-  int qtiles;           // 128-row query tiles per head
-  int64_t tph;          // 128-key tiles per head
-  int64_t total;        // heads * qtiles * tph
-  int C, S_max;         // S_max = 2 partial slots per CTA
+  int qpairs;           // units (pairs of 128-row query tiles) per head
+  int64_t tph;          // 64-key tiles per head
+  int C;                // CTAs (one per SM)
+  int dp_rounds;        // whole-unit rounds before the stream-K part
+  int64_t sk_units;     // units cut by key tiles across the CTAs
   float qmul;           // scale * log2(e)
   float* alpha;
   float* A;
-  float* ws_ml;         // [C][2][128][2]
-  float* ws_acc;        // [C][2][128][128]
+  float* ws_ml;         // [C][2][256][2]
+  float* ws_acc;        // [C][2][256][128]
   int* err;
 };
 struct TcPlan {
-  int qtiles;
-  int64_t tph, total;
-  int C, S_max;
+  int qpairs;
+  int64_t tph;
+  int C, dp_rounds;
+  int64_t sk_units;
   size_t ws_bytes, smem;
 };
 TcPlan plan_tc(int heads, int64_t n, int64_t rows, int num_sms);

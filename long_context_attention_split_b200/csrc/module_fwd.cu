@@ -38,11 +38,11 @@ namespace nectar {
 constexpr int kModMaxStages = 12;             // weight stages (upper bound)
 constexpr int kWTileBytes = 128 * 128;        // one chunk: 128 rows x 64 bf16
 constexpr int kModEpiWarps = 4;
-// local-attention warps of the fused decode: 8 light ones for up to 4 query
-// heads per token, 4 with room for 8 heads' registers otherwise
-__host__ __device__ constexpr int loc_warps(int RG) { return RG <= 4 ? 8 : 4; }
+// local-attention warps of the fused decode (the local keys are a small part
+// of its bytes; the rest of the SM's registers go to the epilogue)
+__host__ __device__ constexpr int loc_warps(int RG) { return (void)RG, 4; }
 __host__ __device__ constexpr int mod_threads(bool fuse, int RG) { return (6 + (fuse ? 1 + loc_warps(RG) : 0)) * 32; }
-constexpr int kModLocStages = 4;              // local K/V ring of the fused decode
+constexpr int kModLocStages = 2;              // local K/V ring of the fused decode
 
 struct ModSmem {
   // offsets in bytes from the 1024-aligned dynamic smem base
@@ -261,12 +261,21 @@ module_kernel(const __grid_constant__ CUtensorMap tmap_q, const ModParams p) {
     for (int net = 0; net < 2; ++net) {
     const int64_t nb = head_base + (net ? layout::net_elems(H, depth, 1) : 0);
     for (int k = 0; k < depth; ++k) {
-      if (ok) ok = mbar_wait(b_acc, accp & 1, p.err);
-      ++accp;
-      tc_fence_after();
       const __nv_bfloat16* bias = blob + nb + layout::hidden_b_off(H, depth, k);
       const bool readout = (net == 0 && k == depth - 1);   // score net: reduce w . h here
       const __nv_bfloat16* wsc = blob + nb + layout::out_w_off(H, depth);
+      // this thread's biases (and readout weights) do not depend on the
+      // accumulators: fetch them while the layer's MMAs run
+      float bvs[8], wvs[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int i = m * 128 + u;
+        bvs[m] = (m < mt && i < H) ? __bfloat162float(bias[i]) : 0.f;
+        wvs[m] = (readout && m < mt && i < H) ? __bfloat162float(wsc[i]) : 0.f;
+      }
+      if (ok) ok = mbar_wait(b_acc, accp & 1, p.err);
+      ++accp;
+      tc_fence_after();
       for (int n0 = 0; n0 < N; n0 += 16) {
         float part[16];
 #pragma unroll
@@ -282,8 +291,13 @@ module_kernel(const __grid_constant__ CUtensorMap tmap_q, const ModParams p) {
           for (int mm = 0; mm < 4; ++mm) {
             const int i = (m0 + mm) * 128 + u;
             if (mm < mc && ok && i < H) {
-              const float bv = __bfloat162float(bias[i]);
-              const float wv = readout ? __bfloat162float(wsc[i]) : 0.f;
+              float bv = 0.f, wv = 0.f;
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                if (q == m0 + mm) {
+                  bv = bvs[q];
+                  wv = wvs[q];
+                }
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
                 const __nv_bfloat16 hb = __float2bfloat16_rn(silu(__uint_as_float(v[mm][j]) + bv));
@@ -318,12 +332,11 @@ module_kernel(const __grid_constant__ CUtensorMap tmap_q, const ModParams p) {
     }
     }
     // target readout A_theta[row][u] = acc[u][row] + c[u], then (fused) the merge
+    const float cb = __bfloat162float(blob[head_base + layout::net_elems(H, depth, 1) + layout::out_b_off(H, depth, kD) + u]);
     if (ok) ok = mbar_wait(b_acc, accp & 1, p.err);
     if (kFuse && ok) ok = mbar_wait(b_loc, 0, p.err);
     named_bar_sync(2, kModEpiWarps * 32);     // sa complete
     tc_fence_after();
-    const int64_t nbt = head_base + layout::net_elems(H, depth, 1);
-    const float cb = __bfloat162float(blob[nbt + layout::out_b_off(H, depth, kD) + u]);
     for (int n0 = 0; n0 < N; n0 += 16) {
       uint32_t v[16];
       NECTAR_TMEM_LD16(trow + n0, v);
@@ -403,10 +416,10 @@ ModShape mod_shape(int G, int64_t nq, int Hmax, bool fuse) {
     if (sh.smem <= kBudget || tpc == 1) break;
     tpc = (tpc + 1) / 2;
   }
-  // weight stages: prefer big copies (up to 4 chunks = 64 KB each) with at
-  // least 3 stages in flight, then as many stages as shared memory takes
-  int cps = 4;
-  while (cps > 1 && mod_smem_layout(Hmax, sh.N, fuse, RG, 3, cps).total + 1024 > kBudget) cps >>= 1;
+  // weight stages: copies of 2 chunks (32 KB) with at least 5 in flight if
+  // they fit, else smaller; then as many stages as shared memory takes
+  int cps = 2;
+  if (mod_smem_layout(Hmax, sh.N, fuse, RG, 4, 2).total + 1024 > kBudget) cps = 1;
   int stages = 3;
   while (stages < kModMaxStages && mod_smem_layout(Hmax, sh.N, fuse, RG, stages + 1, cps).total + 1024 <= kBudget)
     ++stages;

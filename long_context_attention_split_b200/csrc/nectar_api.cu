@@ -234,26 +234,30 @@ nectar_status nectar_cache_attn_lse(nectar_dims dims, const nectar_bf16* K, cons
     tpar.n = n;
     tpar.heads = heads;
     tpar.rows_total = rows;
-    tpar.qtiles = tp.qtiles;
+    tpar.qpairs = tp.qpairs;
     tpar.tph = tp.tph;
-    tpar.total = tp.total;
     tpar.C = tp.C;
-    tpar.S_max = tp.S_max;
+    tpar.dp_rounds = tp.dp_rounds;
+    tpar.sk_units = tp.sk_units;
     tpar.qmul = scale * kLog2e;
     tpar.alpha = alpha;
     tpar.A = A;
     tpar.ws_acc = reinterpret_cast<float*>(workspace);
-    tpar.ws_ml = tpar.ws_acc + static_cast<int64_t>(tp.C) * tp.S_max * 128 * kD;
+    tpar.ws_ml = tpar.ws_acc + static_cast<int64_t>(tp.C) * 2 * 256 * kD;
     tpar.err = di.err;
+    // 4-D views [heads][2 halves of d][rows][64] so that one box brings both
+    // 64-column halves of a tile (each then a K-major, 128-byte-swizzled
+    // operand of 128-byte rows)
     CUtensorMap tq, tk, tv;
-    const cuuint64_t dq[3] = {128, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(heads)};
-    const cuuint64_t sq[2] = {256, static_cast<cuuint64_t>(rows) * 256};
-    const cuuint64_t dk[3] = {128, static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(heads)};
-    const cuuint64_t sk[2] = {256, static_cast<cuuint64_t>(n) * 256};
-    const cuuint32_t box[3] = {64, 128, 1};
-    NECTAR_TRY(make_tmap(&tq, Q, 3, dq, sq, box, "Q"));
-    NECTAR_TRY(make_tmap(&tk, K, 3, dk, sk, box, "K"));
-    NECTAR_TRY(make_tmap(&tv, V, 3, dk, sk, box, "V"));
+    const cuuint64_t dq[4] = {64, static_cast<cuuint64_t>(rows), 2, static_cast<cuuint64_t>(heads)};
+    const cuuint64_t sq[3] = {256, 128, static_cast<cuuint64_t>(rows) * 256};
+    const cuuint64_t dk[4] = {64, static_cast<cuuint64_t>(n), 2, static_cast<cuuint64_t>(heads)};
+    const cuuint64_t sk[3] = {256, 128, static_cast<cuuint64_t>(n) * 256};
+    const cuuint32_t boxq[4] = {64, 128, 2, 1};
+    const cuuint32_t boxk[4] = {64, 64, 2, 1};
+    NECTAR_TRY(make_tmap(&tq, Q, 4, dq, sq, boxq, "Q"));
+    NECTAR_TRY(make_tmap(&tk, K, 4, dk, sk, boxk, "K"));
+    NECTAR_TRY(make_tmap(&tv, V, 4, dk, sk, boxk, "V"));
     cudaError_t e = launch_cache_attn_tc(tq, tk, tv, tpar, st);
     return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "cache_attn tensor-core kernel");
   }

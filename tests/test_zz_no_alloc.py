@@ -68,9 +68,9 @@ def test_static_matches_workspace_entry_point(case):
 
 
 def test_static_rejects_oversize():
-    # 8192 (layer, KV head) pairs with 8 query rows each leave one partial per
-    # head in the decode-regime kernel: 8192 * 8 * 520 B > the static area
-    L, Hkv, G, n = 64, 128, 8, 64
+    # 16384 (layer, KV head) pairs with 8 query rows each leave one partial per
+    # head in the decode-regime kernel: 16384 * 8 * 520 B > the static area
+    L, Hkv, G, n = 128, 128, 8, 64
     assert nx.cache_attn_workspace_size(L, Hkv, G, n, 1) > nx.STATIC_SCRATCH_BYTES
     g = torch.Generator(device="cuda").manual_seed(7)
     K = torch.randn(L, Hkv, n, 128, generator=g, device="cuda").to(torch.bfloat16)
