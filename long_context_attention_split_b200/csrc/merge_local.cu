@@ -19,17 +19,21 @@ namespace nectar {
 
 constexpr int kMergeCW = 4;                       // consumer warps
 constexpr int kMergeThreads = (kMergeCW + 1) * 32;  // + 1 producer warp
-constexpr int kMergeStages = 4;
+// ring depth: 4 stages for up to 4 query heads (several CTAs share an SM),
+// 8 when the heads' registers leave one CTA per SM
+template <int RG>
+__host__ __device__ constexpr int merge_stages() { return RG <= 4 ? 4 : 8; }
 
 template <int RG>
 __host__ __device__ constexpr size_t merge_smem_bytes() {
-  return size_t(kMergeStages) * kLocStageBytes + size_t(kMergeCW) * RG * (kD + 2) * sizeof(float) +
-         2 * kMergeStages * sizeof(uint64_t);
+  return size_t(merge_stages<RG>()) * kLocStageBytes + size_t(kMergeCW) * RG * (kD + 2) * sizeof(float) +
+         2 * merge_stages<RG>() * sizeof(uint64_t);
 }
 
 template <int RG>
 __global__ void __launch_bounds__(kMergeThreads)
 merge_local_kernel(const MergeParams p) {
+  constexpr int kMergeStages = merge_stages<RG>();
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* ring = smem;
   float* scratch = reinterpret_cast<float*>(smem + kMergeStages * kLocStageBytes);
