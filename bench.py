@@ -227,7 +227,10 @@ def run_ours(args):
     work = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     local_args = (wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len) if has_decode else None
-    launches_per_step = 2 + (1 if has_decode else 0)   # (i) main kernel + combine, fused decode
+    dwork = None
+    if has_decode:
+        dwork = torch.empty(nx.decode_workspace_size(wl.L, wl.Hkv, wl.G, wl.nq), dtype=torch.uint8, device=dev)
+    launches_per_step = 2 + (2 if has_decode else 0)   # (i) main kernel + combine; decode + its merge
 
     ev_a0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ev_a1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -240,7 +243,7 @@ def run_ours(args):
         if i is not None:
             ev_a1[i].record(stream)
         if has_decode:
-            nx.decode(mods, Q, *local_args, out=out, stream=stream)
+            nx.decode(mods, Q, *local_args, out=out, workspace=dwork, stream=stream)
         if i is not None:
             ev_d1[i].record(stream)
 
@@ -304,7 +307,8 @@ def run_ours(args):
             d.copy_(h, non_blocking=True)
         nx.cache_attn_lse(wl.K, wl.V, d_in[0], alpha=alpha, A=A, workspace=work, stream=stream)
         if has_decode:
-            nx.decode(mods, d_in[0], d_in[1], d_in[2], wl.Kloc, wl.Vloc, d_in[3], out=out, stream=stream)
+            nx.decode(mods, d_in[0], d_in[1], d_in[2], wl.Kloc, wl.Vloc, d_in[3], out=out, workspace=dwork,
+                      stream=stream)
         for h, d in zip(h_out, d_out):
             h.copy_(d, non_blocking=True)
 
@@ -402,15 +406,36 @@ def workload_overrides(args) -> dict:
     return over
 
 
+# sources of the exact-attention kernels whose DRAM counters profiles/ records
+_SPLIT_SOURCES = ("attn_decode.cu", "common.cuh", "ptx.cuh")
+
+
+def split_sources_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in _SPLIT_SOURCES:
+        with open(os.path.join(ROOT, "long_context_attention_split_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def traffic_from_profile(workload: str):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary (profiles/), or None."""
-    path = os.path.join(ROOT, "profiles", f"cache_attn_split_{workload}.json")
+    """DRAM bytes per full launch of the dominant kernel, read from the ncu
+    summary in profiles/ (lines `dram_bytes_per_launch: B` and
+    `sources_digest: X`); None when absent or when the kernel sources have
+    changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", f"cache_attn_split_{workload}.md")
     try:
         with open(path) as f:
-            return json.load(f).get("dram_bytes_per_launch")
-    except Exception:
+            text = f.read()
+    except OSError:
         return None
+    import re
+    mb = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    md = re.search(r"sources_digest:\s*([0-9a-f]+)", text)
+    if not mb or not md or md.group(1) != split_sources_digest():
+        return None
+    return int(mb.group(1))
 
 
 # ---------------------------------------------------------------------------

@@ -213,17 +213,30 @@ NECTAR_API nectar_status nectar_merge_local(nectar_dims dims, const float *a, co
                                  nectar_stream_t stream);
 
 /* ------------------------------------------------------------------------
- * Fused Nectar decode: (ii) and (iii) in one launch -- the module forward of
- * every row followed by the merge of its (a_theta, A_theta) with its exact
- * causal local attention.  Arguments as in nectar_module_forward and
- * nectar_merge_local; out DEVICE fp32 [L][Hkv][G][nq][d].  Equal (up to
+ * Nectar decode: (ii) and (iii) together -- the module forward of every row
+ * and the merge of its (a_theta, A_theta) with its exact causal local
+ * attention, Eq. (3.5) (§2.2, §2.4).  Arguments as in nectar_module_forward
+ * and nectar_merge_local; out DEVICE fp32 [L][Hkv][G][nq][d].  Equal (up to
  * rounding order) to nectar_module_forward followed by nectar_merge_local.
+ *
+ * Two launches on `stream`: one whose CTAs run the module forward (writing
+ * A_theta into out) side by side with CTAs that compute each row's local
+ * attention state, then a small merge that rewrites out in place.
+ *
+ *   workspace  DEVICE scratch, 256-byte aligned, of at least
+ *              nectar_decode_workspace_size(dims, nq) bytes
+ *              (= rows * 4, rounded up to 256, + rows * (d + 2) * 4 with
+ *              rows = L * Hkv * G * nq); owned by the caller, overwritten,
+ *              must not be used by another call in flight.
+ * Returns NECTAR_ERR_WORKSPACE when it is missing or too small.
  * ------------------------------------------------------------------------ */
+NECTAR_API size_t nectar_decode_workspace_size(nectar_dims dims, int64_t nq);
 NECTAR_API nectar_status nectar_decode(nectar_dims dims, const nectar_module_set *mods,
                             const nectar_bf16 *Q, int64_t nq, const int32_t *q_seq,
                             const int32_t *q_pos, const nectar_bf16 *Kloc,
                             const nectar_bf16 *Vloc, int32_t B, int32_t T_max,
                             const int32_t *local_len, float scale, float *out,
+                            void *workspace, size_t workspace_bytes,
                             nectar_stream_t stream);
 
 /* ------------------------------------------------------------------------

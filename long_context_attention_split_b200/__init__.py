@@ -79,7 +79,10 @@ def lib() -> ctypes.CDLL:
     L.nectar_module_forward.restype = S
     L.nectar_merge_local.argtypes = [Dims, P, P, P, I64, P, P, P, P, I32, I32, P, F, P, P]
     L.nectar_merge_local.restype = S
-    L.nectar_decode.argtypes = [Dims, ctypes.POINTER(_ModuleSetC), P, I64, P, P, P, P, I32, I32, P, F, P, P]
+    L.nectar_decode_workspace_size.argtypes = [Dims, I64]
+    L.nectar_decode_workspace_size.restype = ctypes.c_size_t
+    L.nectar_decode.argtypes = [Dims, ctypes.POINTER(_ModuleSetC), P, I64, P, P, P, P, I32, I32, P, F, P, P,
+                                ctypes.c_size_t, P]
     L.nectar_decode.restype = S
     L.nectar_status_string.argtypes = [S]
     L.nectar_status_string.restype = ctypes.c_char_p
@@ -296,9 +299,15 @@ def merge_local(a, A_doc, Q, q_seq, q_pos, Kloc, Vloc, local_len, scale: Optiona
     return out
 
 
+def decode_workspace_size(L: int, Hkv: int, G: int, nq: int, d: int = 128) -> int:
+    return int(lib().nectar_decode_workspace_size(Dims(L, Hkv, G, d), nq))
+
+
 def decode(mods: ModuleSet, Q, q_seq, q_pos, Kloc, Vloc, local_len, scale: Optional[float] = None, out=None,
-           stream=None):
-    """Fused module forward + merge: out [L,Hkv,G,nq,d] fp32."""
+           workspace=None, stream=None):
+    """Module forward + merge with local attention: out [L,Hkv,G,nq,d] fp32.
+    workspace: uint8 CUDA tensor of decode_workspace_size(...) bytes, made
+    here when None."""
     dims, nq = dims_of(Q)
     _need(Q, "Q", torch.bfloat16)
     B, T = _local_args(q_seq, q_pos, Kloc, Vloc, local_len)
@@ -306,8 +315,12 @@ def decode(mods: ModuleSet, Q, q_seq, q_pos, Kloc, Vloc, local_len, scale: Optio
         scale = 1.0 / math.sqrt(dims.d)
     if out is None:
         out = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    ws_bytes = decode_workspace_size(dims.L, dims.Hkv, dims.G, nq, dims.d)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
     st = lib().nectar_decode(dims, mods.c(), _ptr(Q), nq, _ptr(q_seq), _ptr(q_pos), _ptr(Kloc), _ptr(Vloc), B, T,
-                             _ptr(local_len), float(scale), _ptr(out), _stream(stream))
+                             _ptr(local_len), float(scale), _ptr(out), _ptr(workspace),
+                             0 if workspace is None else workspace.numel(), _stream(stream))
     _check(st, "nectar_decode")
     return out
 

@@ -108,6 +108,8 @@ struct ModParams {
   int B, T;
   float qmul;
   float* out;
+  float* ws_loc;        // decode: local state per row [(hd * rows + row)][d + 2]
+  int64_t n_local;      // decode: local CTAs (heads * nq) ahead of the module CTAs
   int* err;
   int32_t width[kModMaxLayers];
   int64_t layer_base[kModMaxLayers];   // blob element offset of layer l
@@ -120,5 +122,6 @@ struct ModShape {
 ModShape mod_shape(int G, int64_t nq, int Hmax, bool fuse);
 cudaError_t launch_module(const CUtensorMap& tq, const ModParams& p, int units, size_t smem, bool fuse,
                           cudaStream_t stream);
+cudaError_t launch_decode(const CUtensorMap& tq, const ModParams& p, int units, size_t smem, cudaStream_t stream);
 
 }  // namespace nectar

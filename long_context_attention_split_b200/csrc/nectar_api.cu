@@ -424,6 +424,10 @@ nectar_status nectar_module_pack(nectar_dims dims, int32_t depth, const int32_t*
 // ---------------------------------------------------------------------------
 namespace {
 
+// bytes of the decode workspace's a_theta part (rounded so the local states
+// that follow start 256-byte aligned)
+size_t decode_ws_a_bytes(int64_t rows) { return (static_cast<size_t>(rows) * sizeof(float) + 255) & ~size_t(255); }
+
 nectar_status prepare_modules(const nectar_dims& dims, const nectar_module_set* mods, const nectar_bf16* Q,
                               int64_t nq, bool fuse, ModParams* p, CUtensorMap* tq, ModShape* sh) {
   if (mods == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "mods is NULL");
@@ -502,20 +506,37 @@ nectar_status nectar_module_forward(nectar_dims dims, const nectar_module_set* m
   return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "module kernel");
 }
 
+size_t nectar_decode_workspace_size(nectar_dims dims, int64_t nq) {
+  if (check_dims(dims) != NECTAR_OK || nq <= 0) return 0;
+  const int64_t rows = static_cast<int64_t>(dims.L) * dims.Hkv * dims.G * nq;
+  return decode_ws_a_bytes(rows) + static_cast<size_t>(rows) * (kD + 2) * sizeof(float);
+}
+
 nectar_status nectar_decode(nectar_dims dims, const nectar_module_set* mods, const nectar_bf16* Q, int64_t nq,
                             const int32_t* q_seq, const int32_t* q_pos, const nectar_bf16* Kloc,
                             const nectar_bf16* Vloc, int32_t B, int32_t T_max, const int32_t* local_len,
-                            float scale, float* out, nectar_stream_t stream) {
+                            float scale, float* out, void* workspace, size_t workspace_bytes,
+                            nectar_stream_t stream) {
   NECTAR_TRY(check_dims(dims));
   if (nq < 0) return fail(NECTAR_ERR_INVALID_ARG, "nq must be >= 0");
   if (nq == 0) return NECTAR_OK;
   if (!(scale == scale)) return fail(NECTAR_ERR_INVALID_ARG, "scale is NaN");
   NECTAR_TRY(check_ptr(out, "out"));
   NECTAR_TRY(check_local(q_seq, q_pos, Kloc, Vloc, B, T_max, local_len));
+  const size_t need = nectar_decode_workspace_size(dims, nq);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(NECTAR_ERR_WORKSPACE, "decode workspace of %zu bytes given, %zu needed",
+                workspace == nullptr ? size_t(0) : workspace_bytes, need);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0)
+    return fail(NECTAR_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   ModParams p;
   CUtensorMap tq;
   ModShape sh;
   NECTAR_TRY(prepare_modules(dims, mods, Q, nq, true, &p, &tq, &sh));
+  const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
+  const int64_t rows = heads * dims.G * nq;
+  if (heads * nq + static_cast<int64_t>(dims.L) * dims.Hkv * sh.nblk > 0x7fffffffLL)
+    return fail(NECTAR_ERR_UNSUPPORTED, "too many CTAs for one launch");
   p.q_seq = q_seq;
   p.q_pos = q_pos;
   p.Kloc = reinterpret_cast<const __nv_bfloat16*>(Kloc);
@@ -525,9 +546,13 @@ nectar_status nectar_decode(nectar_dims dims, const nectar_module_set* mods, con
   p.T = T_max;
   p.qmul = scale * kLog2e;
   p.out = out;
+  p.a_out = static_cast<float*>(workspace);
+  p.A_out = out;                    // A_theta lands in out, merged in place
+  p.ws_loc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + decode_ws_a_bytes(rows));
+  p.n_local = heads * nq;
   const int units = dims.L * dims.Hkv * sh.nblk;
-  cudaError_t e = launch_module(tq, p, units, sh.smem, true, reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "decode kernel");
+  cudaError_t e = launch_decode(tq, p, units, sh.smem, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "decode kernels");
 }
 
 }  // extern "C"

@@ -317,9 +317,30 @@ def test_decode_toy_prefill():
     dict(L=2, Hkv=2, G=2, n=16, B=3, T=40, widths=[512, 512]),
     dict(L=1, Hkv=2, G=7, n=16, B=10, T=33, widths=[208]),
     dict(L=2, Hkv=1, G=4, n=16, B=20, T=17, widths=[1024, 64]),
+    dict(L=1, Hkv=2, G=8, n=16, B=5, T=70, widths=[256]),      # 8 heads per local job
+    dict(L=1, Hkv=1, G=12, n=16, B=4, T=45, widths=[128]),     # two local jobs per token (8 + 4 heads)
 ])
 def test_decode_shapes(kw):
     wl = make_workload("qwen3_1p7b", seed=2, key_scale=None, **kw)
     wl.local_len = torch.randint(0, wl.T + 1, (wl.B,), generator=torch.Generator().manual_seed(3)).to(torch.int32)
     wl.q_pos = (wl.local_len[wl.q_seq.long()] - 1).clamp(min=0).to(torch.int32)
     decode_case(wl)
+
+
+def test_decode_workspace_checked():
+    wl = make_workload("toy", seed=4)
+    mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G)
+    args = (cuda(wl.Q), cuda(wl.q_seq), cuda(wl.q_pos), cuda(wl.Kloc), cuda(wl.Vloc), cuda(wl.local_len))
+    need = nx.decode_workspace_size(wl.L, wl.Hkv, wl.G, wl.nq)
+    assert need == (wl.heads * wl.rows * 4 + 255) // 256 * 256 + wl.heads * wl.rows * 130 * 4
+    out = torch.full(wl.Q.shape, float("nan"), device="cuda")
+    small = torch.empty(need - 4, dtype=torch.uint8, device="cuda")
+    with pytest.raises(RuntimeError, match="workspace"):
+        nx.decode(mods, *args, out=out, workspace=small)
+    torch.cuda.synchronize()
+    assert torch.isnan(out).all()       # nothing was enqueued
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    nx.decode(mods, *args, out=out, workspace=ws)
+    ref = nx.decode(mods, *args)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
