@@ -179,11 +179,24 @@ NECTAR_API nectar_status nectar_module_pack(nectar_dims dims, int32_t depth, con
  *   a[row]       = a_theta(q)     DEVICE fp32 [L][Hkv][G][nq]
  *   A_theta[row] = A_theta(q)     DEVICE fp32 [L][Hkv][G][nq][d]
  * Runs on the tensor cores (tcgen05, bf16 operands, fp32 accumulation);
- * hidden activations are rounded to bf16 between layers.
+ * hidden activations are rounded to bf16 between layers.  Fewer than 128
+ * query rows per KV head: one launch, each CTA carrying <= 64 rows through
+ * all layers in shared memory (workspace unused, may be NULL).  More rows:
+ * one grouped-GEMM launch per hidden layer plus one for the readouts, the
+ * hidden activations kept in `workspace` (DEVICE, 256-byte aligned, owned
+ * by the caller, overwritten; NECTAR_ERR_WORKSPACE when missing or small).
  * ------------------------------------------------------------------------ */
+/* Workspace of nectar_module_forward, in bytes: 0 when the KV heads have
+ * fewer than 128 query rows (G * nq), else the hidden activations of the
+ * layer-by-layer path, (depth >= 2 ? 2 : 1) * align256(2 * rows * Hp * 2)
+ * + align256(rows * ceil(Hmax / 128) * 4), with rows = L * Hkv * G * nq,
+ * Hmax the widest layer and Hp = Hmax rounded up to 64. */
+NECTAR_API size_t nectar_module_workspace_size(nectar_dims dims, const nectar_module_set *mods,
+                                               int64_t nq);
 NECTAR_API nectar_status nectar_module_forward(nectar_dims dims, const nectar_module_set *mods,
                                     const nectar_bf16 *Q, int64_t nq, float *a,
-                                    float *A_theta, nectar_stream_t stream);
+                                    float *A_theta, void *workspace, size_t workspace_bytes,
+                                    nectar_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * (iii) Merge with exact causal local attention, Eqs. (3.4)-(3.5), §2.2:
@@ -219,18 +232,23 @@ NECTAR_API nectar_status nectar_merge_local(nectar_dims dims, const float *a, co
  * and nectar_merge_local; out DEVICE fp32 [L][Hkv][G][nq][d].  Equal (up to
  * rounding order) to nectar_module_forward followed by nectar_merge_local.
  *
- * Two launches on `stream`: one whose CTAs run the module forward (writing
- * A_theta into out) side by side with CTAs that compute each row's local
- * attention state, then a small merge that rewrites out in place.
+ * Fewer than 128 query rows per KV head: one launch whose CTAs run the
+ * module forward (writing A_theta into out) side by side with CTAs that
+ * compute each row's local attention state, then a small merge that
+ * rewrites out in place.  More rows: the local states first, then the
+ * layer-by-layer module, whose last launch merges and writes out.
  *
  *   workspace  DEVICE scratch, 256-byte aligned, of at least
- *              nectar_decode_workspace_size(dims, nq) bytes
- *              (= rows * 4, rounded up to 256, + rows * (d + 2) * 4 with
- *              rows = L * Hkv * G * nq); owned by the caller, overwritten,
- *              must not be used by another call in flight.
+ *              nectar_decode_workspace_size(dims, mods, nq) bytes: the
+ *              local state of every row, rows * (d + 2) * 4 with
+ *              rows = L * Hkv * G * nq, plus rows * 4 (fewer than 128 query
+ *              rows per KV head) or nectar_module_workspace_size (else);
+ *              owned by the caller, overwritten, must not be used by
+ *              another call in flight.
  * Returns NECTAR_ERR_WORKSPACE when it is missing or too small.
  * ------------------------------------------------------------------------ */
-NECTAR_API size_t nectar_decode_workspace_size(nectar_dims dims, int64_t nq);
+NECTAR_API size_t nectar_decode_workspace_size(nectar_dims dims, const nectar_module_set *mods,
+                                               int64_t nq);
 NECTAR_API nectar_status nectar_decode(nectar_dims dims, const nectar_module_set *mods,
                             const nectar_bf16 *Q, int64_t nq, const int32_t *q_seq,
                             const int32_t *q_pos, const nectar_bf16 *Kloc,

@@ -75,11 +75,13 @@ def lib() -> ctypes.CDLL:
     L.nectar_module_packed_elems.restype = I64
     L.nectar_module_pack.argtypes = [Dims, I32, P, P, P, I64]
     L.nectar_module_pack.restype = S
-    L.nectar_module_forward.argtypes = [Dims, ctypes.POINTER(_ModuleSetC), P, I64, P, P, P]
+    L.nectar_module_workspace_size.argtypes = [Dims, ctypes.POINTER(_ModuleSetC), I64]
+    L.nectar_module_workspace_size.restype = ctypes.c_size_t
+    L.nectar_module_forward.argtypes = [Dims, ctypes.POINTER(_ModuleSetC), P, I64, P, P, P, ctypes.c_size_t, P]
     L.nectar_module_forward.restype = S
     L.nectar_merge_local.argtypes = [Dims, P, P, P, I64, P, P, P, P, I32, I32, P, F, P, P]
     L.nectar_merge_local.restype = S
-    L.nectar_decode_workspace_size.argtypes = [Dims, I64]
+    L.nectar_decode_workspace_size.argtypes = [Dims, ctypes.POINTER(_ModuleSetC), I64]
     L.nectar_decode_workspace_size.restype = ctypes.c_size_t
     L.nectar_decode.argtypes = [Dims, ctypes.POINTER(_ModuleSetC), P, I64, P, P, P, P, I32, I32, P, F, P, P,
                                 ctypes.c_size_t, P]
@@ -213,6 +215,13 @@ class ModuleSet:
     def bytes(self) -> int:
         return self.blob.numel() * 2
 
+    def layer(self, l: int) -> "ModuleSet":
+        """The modules of layer l alone, as a one-layer set viewing the same
+        blob (blocks are stored layer after layer)."""
+        off = packed_elems(l, self.Hkv, 1, self.widths[:l], self.depth) if l > 0 else 0
+        n = packed_elems(1, self.Hkv, 1, self.widths[l:l + 1], self.depth)
+        return ModuleSet(self.blob[off:off + n], self.widths[l:l + 1], self.depth, 1, self.Hkv)
+
 
 def packed_elems(L: int, Hkv: int, G: int, widths: Sequence[int], depth: int, d: int = 128) -> int:
     w = (ctypes.c_int32 * L)(*widths)
@@ -258,15 +267,25 @@ def pack_modules(modules, widths: Sequence[int], depth: int, Hkv: int, G: int, d
 # ---------------------------------------------------------------------------
 # (ii) module forward, (iii) merge, fused decode
 # ---------------------------------------------------------------------------
-def module_forward(mods: ModuleSet, Q, a=None, A_theta=None, stream=None):
-    """(a [L,Hkv,G,nq], A_theta [L,Hkv,G,nq,d]) fp32 for every query row."""
+def module_workspace_size(mods: ModuleSet, G: int, nq: int, d: int = 128) -> int:
+    return int(lib().nectar_module_workspace_size(Dims(mods.L, mods.Hkv, G, d), mods.c(), nq))
+
+
+def module_forward(mods: ModuleSet, Q, a=None, A_theta=None, workspace=None, stream=None):
+    """(a [L,Hkv,G,nq], A_theta [L,Hkv,G,nq,d]) fp32 for every query row.
+    workspace: uint8 CUDA tensor of module_workspace_size(...) bytes (made
+    here when None and needed)."""
     dims, nq = dims_of(Q)
     _need(Q, "Q", torch.bfloat16)
     if a is None:
         a = torch.empty(Q.shape[:4], dtype=torch.float32, device=Q.device)
     if A_theta is None:
         A_theta = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
-    st = lib().nectar_module_forward(dims, mods.c(), _ptr(Q), nq, _ptr(a), _ptr(A_theta), _stream(stream))
+    ws_bytes = module_workspace_size(mods, dims.G, nq, dims.d)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    st = lib().nectar_module_forward(dims, mods.c(), _ptr(Q), nq, _ptr(a), _ptr(A_theta), _ptr(workspace),
+                                     0 if workspace is None else workspace.numel(), _stream(stream))
     _check(st, "nectar_module_forward")
     return a, A_theta
 
@@ -299,8 +318,8 @@ def merge_local(a, A_doc, Q, q_seq, q_pos, Kloc, Vloc, local_len, scale: Optiona
     return out
 
 
-def decode_workspace_size(L: int, Hkv: int, G: int, nq: int, d: int = 128) -> int:
-    return int(lib().nectar_decode_workspace_size(Dims(L, Hkv, G, d), nq))
+def decode_workspace_size(mods: ModuleSet, G: int, nq: int, d: int = 128) -> int:
+    return int(lib().nectar_decode_workspace_size(Dims(mods.L, mods.Hkv, G, d), mods.c(), nq))
 
 
 def decode(mods: ModuleSet, Q, q_seq, q_pos, Kloc, Vloc, local_len, scale: Optional[float] = None, out=None,
@@ -315,7 +334,7 @@ def decode(mods: ModuleSet, Q, q_seq, q_pos, Kloc, Vloc, local_len, scale: Optio
         scale = 1.0 / math.sqrt(dims.d)
     if out is None:
         out = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
-    ws_bytes = decode_workspace_size(dims.L, dims.Hkv, dims.G, nq, dims.d)
+    ws_bytes = decode_workspace_size(mods, dims.G, nq, dims.d)
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
     st = lib().nectar_decode(dims, mods.c(), _ptr(Q), nq, _ptr(q_seq), _ptr(q_pos), _ptr(Kloc), _ptr(Vloc), B, T,

@@ -40,6 +40,11 @@ namespace nectar {
 constexpr int kTcRows = 128;                       // query rows per tile
 constexpr int kTcUnitRows = 2 * kTcRows;           // two tiles per unit
 constexpr int kTcKeys = 64;                        // keys per tile
+#ifndef NECTAR_TC_POLY_PAIRS
+#define NECTAR_TC_POLY_PAIRS 1
+#endif
+// of every 4 pairs of softmax weights, how many use exp2_poly (0..4)
+constexpr int kTcPolyPairs = NECTAR_TC_POLY_PAIRS;
 constexpr int kTcStages = 3;                       // K and V ring depth
 constexpr int kTcThreads = 11 * 32;
 constexpr uint32_t kQBytes = kTcRows * kD * 2;     // 32 KB
@@ -293,6 +298,10 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         const int64_t nvalid = p.n - kt * kTcKeys;
         if (ok) ok = mbar_wait(b_sfull + 8 * (2 * t + b), (cnt >> 1) & 1, p.err);
         tc_fence_after();
+        // a whole tile of valid keys (every tile but a head's last): keep
+        // the raw scores, take the max on them and fold the scale into the
+        // exponent's FMA; the last tile scales and masks element by element
+        const bool full = nvalid >= kTcKeys;
         float sc[kTcKeys];
 #pragma unroll
         for (int cb = 0; cb < kTcKeys; cb += 32) {
@@ -300,15 +309,27 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
           NECTAR_TMEM_LD32(tS + 64 * b + lane_base + cb, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) sc[cb + e] = __uint_as_float(v[e]) * p.qmul;
+          for (int e = 0; e < 32; ++e) sc[cb + e] = __uint_as_float(v[e]);
         }
         tc_fence_before();
         mbar_arrive(b_sfree + 8 * (2 * t + b));
         float bm = -INFINITY;
+        if (full) {
+          float x = sc[0];
+          if (p.qmul >= 0.f) {
 #pragma unroll
-        for (int e = 0; e < kTcKeys; ++e) {
-          if (e >= nvalid) sc[e] = -INFINITY;
-          bm = fmaxf(bm, sc[e]);
+            for (int e = 1; e < kTcKeys; ++e) x = fmaxf(x, sc[e]);
+          } else {
+#pragma unroll
+            for (int e = 1; e < kTcKeys; ++e) x = fminf(x, sc[e]);
+          }
+          bm = x * p.qmul;
+        } else {
+#pragma unroll
+          for (int e = 0; e < kTcKeys; ++e) {
+            sc[e] = (e < nvalid) ? sc[e] * p.qmul : -INFINITY;
+            bm = fmaxf(bm, sc[e]);
+          }
         }
         const bool need = bm > m + kRescaleSlack;
         const float corr = need ? exp2_shift(m, bm) : 1.0f;
@@ -336,18 +357,30 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         // P buffer b was last read by the P V of this tile's S count cnt - 2
         if (cnt >= 2 && ok) ok = mbar_wait(b_pvdone + 8 * (2 * t + b), ((cnt >> 1) - 1) & 1, p.err);
         uint8_t* pt = smem + TcSmem::p + (2 * t + b) * kPBytes;
-        float rs = 0.f;
+        float2 rs2 = make_float2(0.f, 0.f);
+        const float2 q2 = make_float2(p.qmul, p.qmul), nm2 = make_float2(-m, -m);
 #pragma unroll
         for (int c8 = 0; c8 < kTcKeys / 8; ++c8) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            w[e] = pack_bf16x2(exp2_shift(sc[c8 * 8 + 2 * e], m), exp2_shift(sc[c8 * 8 + 2 * e + 1], m));
-            rs += bf16lo(w[e]) + bf16hi(w[e]);
+            const float s0 = sc[c8 * 8 + 2 * e], s1 = sc[c8 * 8 + 2 * e + 1];
+            if (full) {
+              // 2^(s * scale * log2 e - m) for two keys: one paired FMA; the
+              // last kTcPolyPairs of every 4 pairs take the polynomial exp2 so
+              // the special-function unit is not the limit
+              const float2 x = ffma2(make_float2(s0, s1), q2, nm2);
+              if (e >= 4 - kTcPolyPairs) w[e] = pack_bf16x2(exp2_poly(x.x), exp2_poly(x.y));
+              else w[e] = pack_bf16x2(ex2(x.x), ex2(x.y));
+            } else {
+              w[e] = pack_bf16x2(exp2_shift(s0, m), exp2_shift(s1, m));
+            }
+            // the row sum adds the rounded weights that P V uses
+            rs2 = fadd2(rs2, make_float2(bf16lo(w[e]), bf16hi(w[e])));
           }
           *reinterpret_cast<uint4*>(pt + p_off(row, c8 * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        l += rs;
+        l += rs2.x + rs2.y;
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(b_pfull + 8 * (2 * t + b));

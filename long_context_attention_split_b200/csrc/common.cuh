@@ -34,6 +34,27 @@ __device__ __forceinline__ float exp2_shift(float x, float m) {
   return (x == -INFINITY) ? 0.0f : ex2(x - m);
 }
 
+// 2^x on the FMA and integer pipes instead of the special-function unit,
+// for arguments x <= 127 (softmax exponents, <= the lazy-rescale slack).
+// Cody-Waite argument reduction x = n + f with n = round(x), done by adding
+// and subtracting 1.5 * 2^23 (n lands in the low mantissa bits of j),
+// f in [-0.5, 0.5]; 2^f by a degree-3 polynomial fitted by the Remez
+// exchange to minimise the relative error on that interval (coefficients
+// from fit_exp2_poly.py; max relative error 7.5e-5, far below the 2^-9 of
+// the bf16 rounding the softmax weights get next); 2^n is added to the
+// exponent field.  Arguments below -126 give ~2^-126 instead of 0.
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float j = x + 12582912.0f;             // 1.5 * 2^23
+  const float f = x - (j - 12582912.0f);
+  const float pf = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  return __int_as_float(__float_as_int(pf) + (__float_as_int(j) << 23));
+}
+
 // Load 8 bf16 (one 16-byte chunk) as floats.
 __device__ __forceinline__ void unpack8(const uint4 w, float* f) {
   f[0] = bf16lo(w.x); f[1] = bf16hi(w.x);

@@ -115,6 +115,54 @@ struct ModParams {
   int64_t layer_base[kModMaxLayers];   // blob element offset of layer l
   uint8_t order[kModMaxLayers];        // layers by decreasing width
 };
+// Layer-by-layer grouped GEMM path of the module forward (module_gemm.cu),
+// used when a KV head has at least kGemmMinRows query rows.
+constexpr int kGemmMaxStages = 8;
+constexpr int kGemmMinRows = 128;
+struct GemmParams {
+  int L, Hkv, depth, stage, readout, nlayers;
+  int R, NR, rtiles, Hp, MT, stages, tmem_cols;
+  int64_t ntiles;
+  const __nv_bfloat16* blob;
+  __nv_bfloat16* h_out;     // [2 nets][heads * R][Hp] bf16 (hidden stages)
+  float* part;              // score partials [heads * R][MT]
+  float* a_out;             // readout: [heads * R]
+  float* A_out;             // readout: [heads * R][d] (A_theta, or the merged output)
+  const float* ws_loc;      // decode: local state per row [(heads * R)][d + 2], else null
+  int* err;
+  int32_t width[kModMaxLayers];
+  int64_t layer_base[kModMaxLayers];
+  int64_t tile_start[kModMaxLayers + 1];
+  uint8_t order[kModMaxLayers];
+};
+struct GemmShape {
+  int NR, rtiles, stages, tmem_cols;
+  size_t smem;
+};
+GemmShape gemm_shape(int64_t R);
+cudaError_t launch_module_gemm(const CUtensorMap& tq, const CUtensorMap& th, const GemmParams& p, int grid,
+                               size_t smem, cudaStream_t stream);
+cudaError_t launch_local_state(const ModParams& p, cudaStream_t stream);
+
+// Tensor-core local attention (local_tc.cu).
+struct LocTcParams {
+  int64_t njobs;            // heads * nq
+  int64_t nq;
+  int G, B, T, kbox;        // kbox = keys per TMA box, min(128, T)
+  const int32_t* q_seq;
+  const int32_t* q_pos;
+  const int32_t* local_len;
+  float qmul;               // scale * log2 e
+  float* ws_loc;            // state per row [(hd * rows + row)][d + 2] (when out is null)
+  const float* a;           // merge: document logit per row
+  const float* A_doc;       // merge: document term per row [.][d]
+  float* out;               // merge output, or null
+  int* err;
+};
+size_t local_tc_smem();
+cudaError_t launch_local_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const LocTcParams& p, int grid, cudaStream_t stream);
+
 struct ModShape {
   int TPC, N, nblk, tmem_cols, stages, cps;
   size_t smem;

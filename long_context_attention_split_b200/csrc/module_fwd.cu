@@ -493,6 +493,31 @@ static cudaError_t launch_decode_t(const CUtensorMap& tq, const ModParams& p, in
   return cudaGetLastError();
 }
 
+template <int RG>
+static cudaError_t launch_local_t(const ModParams& p, cudaStream_t stream) {
+  const size_t smem = dec_local_smem(RG) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<RG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  CUtensorMap unused{};                      // local CTAs read no tensor map
+  decode_kernel<RG><<<static_cast<unsigned>(p.n_local), kModThreads, smem, stream>>>(unused, p);
+  return cudaGetLastError();
+}
+
+// Local attention states only (every CTA a local CTA), into p.ws_loc.
+cudaError_t launch_local_state(const ModParams& p, cudaStream_t stream) {
+  switch (p.G < 8 ? p.G : 8) {
+    case 1: return launch_local_t<1>(p, stream);
+    case 2: return launch_local_t<2>(p, stream);
+    case 3: return launch_local_t<3>(p, stream);
+    case 4: return launch_local_t<4>(p, stream);
+    case 5: return launch_local_t<5>(p, stream);
+    case 6: return launch_local_t<6>(p, stream);
+    case 7: return launch_local_t<7>(p, stream);
+    default: return launch_local_t<8>(p, stream);
+  }
+}
+
 cudaError_t launch_decode(const CUtensorMap& tq, const ModParams& p, int units, size_t smem, cudaStream_t stream) {
   switch (p.G < 8 ? p.G : 8) {
     case 1: return launch_decode_t<1>(tq, p, units, smem, stream);

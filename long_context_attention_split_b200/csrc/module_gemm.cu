@@ -1,0 +1,354 @@
+// (ii) Nectar module forward for many query rows per KV head, layer by
+// layer: Eq. (3.6) of "Nectar: Neural Estimation of Cached-Token Attention
+// via Regression" (§2.4), with the Eq. (3.5) merge folded into the last
+// layer when it serves the decode (§2.2).
+//
+// When a KV head has many query rows (a decode batch, a prompt), one CTA per
+// block of 64 rows holding all hidden activations in shared memory would
+// stream the head's weights once per block.  Here each hidden layer of both
+// nets is instead one grouped GEMM over all (layer, KV head) pairs:
+//   D[hidden unit, row] = W_k[hidden unit, :] . X[row, :],
+//   X = q (k = 0) or [q | h_{k-1}] (k >= 1),
+// on tcgen05 (kind::f16, cta_group::1): M = 128 hidden units (A = one row
+// tile of the packed, pre-swizzled weights, fetched by bulk copies), N = up
+// to 256 rows (B = rows of Q and of the previous layer's activations, by 2-D
+// TMA boxes with the 128-byte swizzle), fp32 accumulators in TMEM.  The
+// epilogue adds the bias, applies SiLU and stores h_k (bf16, row-major
+// [rows][Hp]) for the next launch; the score net's last hidden layer is not
+// stored but reduced at once against the readout row w (one fp32 partial per
+// 128 hidden units and row).  A last launch runs the target readout GEMM
+// (M = d), adds the score partials and the biases, and either writes
+// (a_theta, A_theta) or merges them with each row's exact local attention
+// state (decode).
+//
+// Persistent CTAs (one per SM) walk a static list of tiles, widest layers
+// first.  Warp roles: 0 TMA producer, 1 MMA issuer (+ TMEM owner), 2..5
+// epilogue.  Two TMEM accumulators let the epilogue of one tile run under
+// the MMAs of the next.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "module_layout.h"
+
+namespace nectar {
+
+constexpr int kGemmThreads = 6 * 32;
+constexpr int kGemmWBytes = 128 * 128;        // one weight chunk: 128 rows x 64 bf16
+
+__host__ __device__ inline uint32_t gemm_stage_bytes(int NR) {
+  return (static_cast<uint32_t>(kGemmWBytes + NR * 128) + 1023u) & ~1023u;
+}
+
+struct GemmSmem {
+  uint32_t ring, red, bars, tslot, total;
+};
+
+__host__ __device__ inline GemmSmem gemm_smem_layout(int NR, int stages) {
+  GemmSmem s{};
+  uint32_t off = 0;
+  s.ring = off;
+  off += static_cast<uint32_t>(stages) * gemm_stage_bytes(NR);
+  s.red = off;                                    // score partials [4 warps][NR]
+  off += 4u * NR * 4;
+  off = (off + 15) & ~15u;
+  s.bars = off;
+  off += 2 * kGemmMaxStages * 8 + 4 * 8;
+  s.tslot = off;
+  off += 16;
+  s.total = off;
+  return s;
+}
+
+struct GemmTile {
+  int l, H, net, m, rt;
+  int64_t hd;
+};
+
+__device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int64_t t) {
+  int li = 0;
+  while (li + 1 < p.nlayers && t >= p.tile_start[li + 1]) ++li;
+  GemmTile g;
+  g.l = p.order[li];
+  g.H = p.width[g.l];
+  const int mt = p.readout ? 1 : (g.H + 127) / 128;
+  const int nets = p.readout ? 1 : 2;
+  int64_t rem = t - p.tile_start[li];
+  g.rt = static_cast<int>(rem % p.rtiles);
+  rem /= p.rtiles;
+  g.m = static_cast<int>(rem % mt);
+  rem /= mt;
+  g.net = p.readout ? 1 : static_cast<int>(rem % nets);
+  const int h = static_cast<int>(rem / nets);
+  g.hd = static_cast<int64_t>(g.l) * p.Hkv + h;
+  return g;
+}
+
+__device__ __forceinline__ float gemm_silu(float v) { return __fdividef(v, 1.0f + ex2(-v * kLog2e)); }
+
+// Sum over the 32 lanes of v[j] for j = 0..31; lane j returns the total of
+// row j (halving exchange: 31 shuffles instead of 160).
+__device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int k = 0; k < off; ++k) {
+      const float send = upper ? v[k] : v[k + off];
+      const float keep = upper ? v[k + off] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0];
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_h,
+                   const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int NR = p.NR;
+  const GemmSmem L = gemm_smem_layout(NR, p.stages);
+  const uint32_t S = static_cast<uint32_t>(p.stages);
+  const uint32_t SB = gemm_stage_bytes(NR);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  const uint32_t b_full = smem_u32(bars);
+  const uint32_t b_empty = smem_u32(bars + kGemmMaxStages);
+  const uint32_t b_accf = smem_u32(bars + 2 * kGemmMaxStages);       // [2]
+  const uint32_t b_acce = smem_u32(bars + 2 * kGemmMaxStages + 2);   // [2]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L.tslot);
+  float* red = reinterpret_cast<float*>(smem + L.red);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t heads = static_cast<int64_t>(p.L) * p.Hkv;
+  const int R = p.R;
+
+  if (threadIdx.x == 0) {
+    for (uint32_t s = 0; s < S; ++s) {
+      mbar_init(b_full + 8 * s, 1);
+      mbar_init(b_empty + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(b_accf + 8 * b, 1);
+      mbar_init(b_acce + 8 * b, 4);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tslot), static_cast<uint32_t>(p.tmem_cols));
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      prefetch_tmap(&tmap_q);
+      prefetch_tmap(&tmap_h);
+      const uint64_t pol_w = policy_evict_last();     // weight tiles are re-read by the row tiles
+      const uint64_t pol_x = policy_evict_normal();
+      uint32_t it = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x) {
+        const GemmTile g = gemm_tile(p, t);
+        const int64_t nb = p.layer_base[g.l] + (g.hd - static_cast<int64_t>(g.l) * p.Hkv) * layout::head_elems(g.H, p.depth) +
+                           (g.net ? layout::net_elems(g.H, p.depth, 1) : 0);
+        const int rows = p.readout ? kD : g.H;
+        const int K = p.readout ? g.H : layout::hidden_k(g.H, p.stage);
+        const int kc = layout::kchunks(K);
+        const __nv_bfloat16* wbase =
+            p.blob + nb + (p.readout ? layout::out_w_off(g.H, p.depth) : layout::hidden_w_off(g.H, p.depth, p.stage));
+        const uint32_t wbytes = static_cast<uint32_t>(layout::tile_rows(rows, g.m)) * 128;
+        const int qrow = static_cast<int>(g.hd * R + static_cast<int64_t>(g.rt) * NR);
+        const int hrow = static_cast<int>((g.net * heads + g.hd) * R + static_cast<int64_t>(g.rt) * NR);
+        const int qch = p.readout ? 0 : 2;             // leading chunks taken from q
+        for (int c = 0; c < kc; ++c, ++it) {
+          const uint32_t s = it % S;
+          if (it >= S && !mbar_wait(b_empty + 8 * s, ((it / S) - 1) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = smem_u32(smem + L.ring + s * SB);
+          mbar_arrive_expect_tx(b_full + 8 * s, wbytes + static_cast<uint32_t>(NR) * 128);
+          bulk_g2s(dst, wbase + layout::tile_chunk_off(rows, K, g.m, c), wbytes, b_full + 8 * s, pol_w);
+          if (c < qch) tma_load_2d(dst + kGemmWBytes, &tmap_q, c * 64, qrow, b_full + 8 * s, pol_x);
+          else tma_load_2d(dst + kGemmWBytes, &tmap_h, (c - qch) * 64, hrow, b_full + 8 * s, pol_x);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, NR, 0, 0);
+      uint32_t it = 0, tc = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x, ++tc) {
+        const GemmTile g = gemm_tile(p, t);
+        const int K = p.readout ? g.H : layout::hidden_k(g.H, p.stage);
+        const int kc = layout::kchunks(K);
+        const uint32_t b = tc & 1;
+        if (tc >= 2 && !mbar_wait(b_acce + 8 * b, ((tc >> 1) - 1) & 1, p.err)) break;
+        tc_fence_after();
+        const uint32_t dacc = tmem + b * static_cast<uint32_t>(NR);
+        for (int c = 0; c < kc; ++c, ++it) {
+          const uint32_t s = it % S;
+          if (!mbar_wait(b_full + 8 * s, (it / S) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t wa = smem_u32(smem + L.ring + s * SB);
+          const uint32_t xb = wa + kGemmWBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(dacc, sdesc_sw128(wa + kk * 32, 16, 1024), sdesc_sw128(xb + kk * 32, 16, 1024), idesc,
+                        (c | kk) != 0);
+          mma_commit(b_empty + 8 * s);
+        }
+        if (ok) mma_commit(b_accf + 8 * b);
+      }
+    }
+  } else {
+    // ------------------------------ epilogue ------------------------------
+    const int q4 = warp & 3;                  // TMEM lane quarter of this warp
+    const int u = q4 * 32 + lane;             // accumulator lane: hidden unit or output dim
+    const uint32_t tlane = static_cast<uint32_t>(q4 * 32) << 16;
+    uint32_t tc = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++tc) {
+      const GemmTile g = gemm_tile(p, t);
+      const int64_t hb = p.layer_base[g.l] + (g.hd - static_cast<int64_t>(g.l) * p.Hkv) * layout::head_elems(g.H, p.depth);
+      const int64_t nb = hb + (g.net ? layout::net_elems(g.H, p.depth, 1) : 0);
+      const uint32_t b = tc & 1;
+      const int r0 = g.rt * NR;
+      // rows of this tile; a 32-column batch may run 16 columns past NR
+      const int rend = (R < r0 + NR) ? R : r0 + NR;
+      // per-thread constants, fetched before the accumulator is ready
+      const int i = g.m * 128 + u;
+      float bias = 0.f, wsc = 0.f;
+      const bool score_last = !p.readout && g.net == 0 && p.stage == p.depth - 1;
+      if (p.readout) {
+        bias = __bfloat162float(p.blob[nb + layout::out_b_off(g.H, p.depth, kD) + u]);
+      } else if (i < g.H) {
+        bias = __bfloat162float(p.blob[nb + layout::hidden_b_off(g.H, p.depth, p.stage) + i]);
+        if (score_last) wsc = __bfloat162float(p.blob[nb + layout::out_w_off(g.H, p.depth) + i]);
+      }
+      if (ok) ok = mbar_wait(b_accf + 8 * b, (tc >> 1) & 1, p.err);
+      ok = __all_sync(0xffffffffu, ok);         // keeps the shuffles below warp-uniform
+      tc_fence_after();
+      const uint32_t dacc = tmem + tlane + b * static_cast<uint32_t>(NR);
+      for (int n0 = 0; n0 < NR; n0 += 32) {
+        uint32_t v[32];
+        NECTAR_TMEM_LD32(dacc + n0, v);
+        tmem_ld_wait();
+        if (!ok) continue;
+        if (!p.readout) {
+          if (score_last) {
+            float part[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float hv = __bfloat162float(__float2bfloat16_rn(gemm_silu(__uint_as_float(v[j]) + bias)));
+              part[j] = (i < g.H) ? wsc * hv : 0.f;
+            }
+            const float tot = warp_transpose_sum32(part, lane);
+            if (n0 + lane < NR) red[q4 * NR + n0 + lane] = tot;
+          } else {
+            const int Hp = p.Hp;
+            const int64_t hrow0 = (g.net * heads + g.hd) * R;
+            if (i < layout::round64(g.H)) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int r = r0 + n0 + j;
+                const float hv = (i < g.H) ? gemm_silu(__uint_as_float(v[j]) + bias) : 0.f;
+                if (r < rend) p.h_out[(hrow0 + r) * Hp + i] = __float2bfloat16_rn(hv);
+              }
+            }
+          }
+        } else {
+          // readout: u = output dim; a per row from the score partials
+          float a_l = 0.f;
+          {
+            const int r = r0 + n0 + lane;
+            if (r < rend) {
+              const float* pr = p.part + (g.hd * R + r) * p.MT;
+              const int mts = (g.H + 127) / 128;
+              for (int m = 0; m < mts; ++m) a_l += pr[m];
+              a_l += __bfloat162float(p.blob[hb + layout::out_b_off(g.H, p.depth, 1)]);
+              if (q4 == 0 && p.a_out != nullptr) p.a_out[g.hd * R + r] = a_l;
+            }
+          }
+#pragma unroll 4
+          for (int j = 0; j < 32; ++j) {
+            const int r = r0 + n0 + j;
+            const float aj = __shfl_sync(0xffffffffu, a_l, j);
+            if (r >= rend) continue;
+            const int64_t row = g.hd * R + r;
+            const float At = __uint_as_float(v[j]) + bias;
+            if (p.ws_loc == nullptr) {
+              p.A_out[row * kD + u] = At;
+            } else {
+              const float* st = p.ws_loc + row * (kD + 2);
+              const float ad = aj * kLog2e;
+              const float M = fmaxf(ad, st[kD]);
+              const float wd = exp2_shift(ad, M), wl = exp2_shift(st[kD], M);
+              p.A_out[row * kD + u] = (wd * At + wl * st[u]) / (wd + wl * st[kD + 1]);
+            }
+          }
+        }
+      }
+      // this tile's accumulator may be overwritten now
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_acce + 8 * b);
+      if (score_last) {
+        named_bar_sync(2, 4 * 32);
+        for (int n = u; n < NR; n += 128) {
+          const int r = r0 + n;
+          if (ok && r < rend)
+            p.part[(g.hd * R + r) * p.MT + g.m] = (red[n] + red[NR + n]) + (red[2 * NR + n] + red[3 * NR + n]);
+        }
+        named_bar_sync(2, 4 * 32);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, static_cast<uint32_t>(p.tmem_cols));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+GemmShape gemm_shape(int64_t R) {
+  GemmShape sh{};
+  sh.rtiles = static_cast<int>((R + 255) / 256);
+  const int64_t per = (R + sh.rtiles - 1) / sh.rtiles;
+  sh.NR = static_cast<int>((per + 15) / 16 * 16);
+  constexpr size_t kBudget = 227 * 1024;
+  int stages = 2;
+  while (stages < kGemmMaxStages && gemm_smem_layout(sh.NR, stages + 1).total + 1024 <= kBudget) ++stages;
+  sh.stages = stages;
+  sh.smem = gemm_smem_layout(sh.NR, stages).total + 1024;
+  int c = 32;
+  while (c < 2 * sh.NR) c <<= 1;
+  sh.tmem_cols = c;
+  return sh;
+}
+
+cudaError_t launch_module_gemm(const CUtensorMap& tq, const CUtensorMap& th, const GemmParams& p, int grid,
+                               size_t smem, cudaStream_t stream) {
+  cudaError_t e =
+      cudaFuncSetAttribute(module_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  module_gemm_kernel<<<grid, kGemmThreads, smem, stream>>>(tq, th, p);
+  return cudaGetLastError();
+}
+
+}  // namespace nectar

@@ -295,6 +295,58 @@ static nectar_status check_local(const int32_t* q_seq, const int32_t* q_pos, con
   return NECTAR_OK;
 }
 
+// Many query tokens: the local attention runs on the tensor cores
+// (local_tc.cu), one job per (KV head, token).
+static bool use_local_tc(const nectar_dims& dims, int64_t nq, int32_t B, int32_t T_max) {
+  return static_cast<int64_t>(dims.G) * nq >= kGemmMinRows && dims.G <= 64 && B > 0 && T_max > 0;
+}
+
+// Either leaves each row's local state in ws_loc (out == nullptr) or merges
+// it with (a, A_doc) into out.
+static nectar_status run_local_tc(const nectar_dims& dims, const nectar_bf16* Q, int64_t nq, const int32_t* q_seq,
+                                  const int32_t* q_pos, const nectar_bf16* Kloc, const nectar_bf16* Vloc, int32_t B,
+                                  int32_t T_max, const int32_t* local_len, float scale, float* ws_loc,
+                                  const float* a, const float* A_doc, float* out, cudaStream_t st) {
+  const DeviceInfo di = device_info();
+  if (di.sms == 0) return fail(NECTAR_ERR_CUDA, "no CUDA device");
+  const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
+  if (heads * B > 0x7fffffffLL || heads > 0x7fffffffLL || nq > 0x7fffffffLL)
+    return fail(NECTAR_ERR_UNSUPPORTED, "local cache too large for one call");
+  LocTcParams p{};
+  p.njobs = heads * nq;
+  p.nq = nq;
+  p.G = dims.G;
+  p.B = B;
+  p.T = T_max;
+  p.kbox = T_max < 128 ? T_max : 128;
+  p.q_seq = q_seq;
+  p.q_pos = q_pos;
+  p.local_len = local_len;
+  p.qmul = scale * kLog2e;
+  p.ws_loc = ws_loc;
+  p.a = a;
+  p.A_doc = A_doc;
+  p.out = out;
+  p.err = di.err;
+  CUtensorMap tq, tk, tv;
+  {
+    const cuuint64_t dq[4] = {128, static_cast<cuuint64_t>(nq), static_cast<cuuint64_t>(dims.G),
+                              static_cast<cuuint64_t>(heads)};
+    const cuuint64_t sq[3] = {256, static_cast<cuuint64_t>(nq) * 256, static_cast<cuuint64_t>(nq) * 256 * dims.G};
+    const cuuint32_t bq[4] = {64, 1, static_cast<cuuint32_t>(dims.G), 1};
+    NECTAR_TRY(make_tmap(&tq, Q, 4, dq, sq, bq, "queries (per token)"));
+    // local caches as [heads * B][2 halves][T][64]: one box = kbox keys of one half
+    const cuuint64_t dk[4] = {64, static_cast<cuuint64_t>(T_max), 2, static_cast<cuuint64_t>(heads * B)};
+    const cuuint64_t sk[3] = {256, 128, static_cast<cuuint64_t>(T_max) * 256};
+    const cuuint32_t bk[4] = {64, static_cast<cuuint32_t>(p.kbox), 1, 1};
+    NECTAR_TRY(make_tmap(&tk, Kloc, 4, dk, sk, bk, "local keys"));
+    NECTAR_TRY(make_tmap(&tv, Vloc, 4, dk, sk, bk, "local values"));
+  }
+  const int grid = static_cast<int>(p.njobs < di.sms ? p.njobs : di.sms);
+  cudaError_t e = launch_local_tc(tq, tk, tv, p, grid, st);
+  return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "local attention kernel");
+}
+
 nectar_status nectar_merge_local(nectar_dims dims, const float* a, const float* A_doc, const nectar_bf16* Q,
                                  int64_t nq, const int32_t* q_seq, const int32_t* q_pos,
                                  const nectar_bf16* Kloc, const nectar_bf16* Vloc, int32_t B, int32_t T_max,
@@ -308,6 +360,9 @@ nectar_status nectar_merge_local(nectar_dims dims, const float* a, const float* 
   NECTAR_TRY(check_ptr(Q, "Q"));
   NECTAR_TRY(check_ptr(out, "out"));
   NECTAR_TRY(check_local(q_seq, q_pos, Kloc, Vloc, B, T_max, local_len));
+  if (use_local_tc(dims, nq, B, T_max))
+    return run_local_tc(dims, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, nullptr, a, A_doc, out,
+                        reinterpret_cast<cudaStream_t>(stream));
   if (static_cast<int64_t>(dims.L) * dims.Hkv * nq * ((dims.G + 7) / 8) > 0x7fffffffLL)
     return fail(NECTAR_ERR_INVALID_ARG, "too many (head, token) units");
   MergeParams p{};
@@ -424,9 +479,107 @@ nectar_status nectar_module_pack(nectar_dims dims, int32_t depth, const int32_t*
 // ---------------------------------------------------------------------------
 namespace {
 
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
 // bytes of the decode workspace's a_theta part (rounded so the local states
 // that follow start 256-byte aligned)
-size_t decode_ws_a_bytes(int64_t rows) { return (static_cast<size_t>(rows) * sizeof(float) + 255) & ~size_t(255); }
+size_t decode_ws_a_bytes(int64_t rows) { return align256(static_cast<size_t>(rows) * sizeof(float)); }
+
+// Many query rows per KV head: the module runs layer by layer as grouped
+// GEMMs (module_gemm.cu) instead of one CTA per block of <= 64 rows.
+bool use_gemm_path(const nectar_dims& dims, int64_t nq) {
+  return static_cast<int64_t>(dims.G) * nq >= kGemmMinRows;
+}
+
+int mods_hmax(const nectar_dims& dims, const int32_t* width) {
+  int Hmax = 0;
+  for (int l = 0; l < dims.L; ++l) Hmax = width[l] > Hmax ? width[l] : Hmax;
+  return Hmax;
+}
+
+// Workspace of the layer-by-layer path: hidden activations (two buffers
+// when depth >= 2, each [2 nets][rows][Hp] bf16), then the score partials
+// [rows][MT] fp32.
+size_t gemm_h_bytes(const nectar_dims& dims, int Hmax, int64_t nq) {
+  const int64_t rows = static_cast<int64_t>(dims.L) * dims.Hkv * dims.G * nq;
+  return align256(static_cast<size_t>(2 * rows) * layout::round64(Hmax) * 2);
+}
+size_t gemm_ws_bytes(const nectar_dims& dims, int Hmax, int depth, int64_t nq) {
+  const int64_t rows = static_cast<int64_t>(dims.L) * dims.Hkv * dims.G * nq;
+  const int MT = (Hmax + 127) / 128;
+  return (depth >= 2 ? 2 : 1) * gemm_h_bytes(dims, Hmax, nq) + align256(static_cast<size_t>(rows) * MT * 4);
+}
+
+// The layer-by-layer module forward: depth hidden-layer launches and one
+// readout launch.  With ws_loc the readout merges with the local states
+// (decode) and writes the output into A_out.
+nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, const nectar_bf16* Q, int64_t nq,
+                              float* a, float* A_out, const float* ws_loc, void* ws, cudaStream_t st) {
+  const DeviceInfo di = device_info();
+  const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
+  const int64_t R = static_cast<int64_t>(dims.G) * nq;
+  if (heads * R * 2 > 0x7fffffffLL) return fail(NECTAR_ERR_UNSUPPORTED, "too many query rows for one call");
+  const GemmShape sh = gemm_shape(R);
+  GemmParams g;
+  memset(&g, 0, sizeof(g));
+  g.L = dims.L;
+  g.Hkv = dims.Hkv;
+  g.depth = mp.depth;
+  g.nlayers = dims.L;
+  g.R = static_cast<int>(R);
+  g.NR = sh.NR;
+  g.rtiles = sh.rtiles;
+  g.Hp = layout::round64(mp.Hmax);
+  g.MT = (mp.Hmax + 127) / 128;
+  g.stages = sh.stages;
+  g.tmem_cols = sh.tmem_cols;
+  g.blob = mp.blob;
+  g.err = mp.err;
+  for (int l = 0; l < dims.L; ++l) {
+    g.width[l] = mp.width[l];
+    g.layer_base[l] = mp.layer_base[l];
+    g.order[l] = mp.order[l];
+  }
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const size_t hb = gemm_h_bytes(dims, mp.Hmax, nq);
+  __nv_bfloat16* hbuf[2] = {reinterpret_cast<__nv_bfloat16*>(base),
+                            reinterpret_cast<__nv_bfloat16*>(base + (mp.depth >= 2 ? hb : 0))};
+  g.part = reinterpret_cast<float*>(base + (mp.depth >= 2 ? 2 : 1) * hb);
+  CUtensorMap tq, th[2];
+  {
+    const cuuint64_t dq[2] = {128, static_cast<cuuint64_t>(heads * R)};
+    const cuuint64_t sq[1] = {256};
+    const cuuint32_t bq[2] = {64, static_cast<cuuint32_t>(sh.NR)};
+    NECTAR_TRY(make_tmap(&tq, Q, 2, dq, sq, bq, "queries (rows)"));
+    for (int b = 0; b < 2; ++b) {
+      const cuuint64_t dh[2] = {static_cast<cuuint64_t>(g.Hp), static_cast<cuuint64_t>(2 * heads * R)};
+      const cuuint64_t shs[1] = {static_cast<cuuint64_t>(g.Hp) * 2};
+      NECTAR_TRY(make_tmap(&th[b], hbuf[b], 2, dh, shs, bq, "hidden activations"));
+    }
+  }
+  for (int stage = 0; stage <= mp.depth; ++stage) {
+    g.stage = stage;
+    g.readout = stage == mp.depth;
+    g.h_out = g.readout ? nullptr : hbuf[stage & 1];
+    g.a_out = g.readout ? a : nullptr;
+    g.A_out = g.readout ? A_out : nullptr;
+    g.ws_loc = g.readout ? ws_loc : nullptr;
+    int64_t acc = 0;
+    for (int li = 0; li < dims.L; ++li) {
+      g.tile_start[li] = acc;
+      const int H = mp.width[mp.order[li]];
+      const int mt = g.readout ? 1 : (H + 127) / 128;
+      acc += static_cast<int64_t>(dims.Hkv) * (g.readout ? 1 : 2) * mt * sh.rtiles;
+    }
+    g.tile_start[dims.L] = acc;
+    g.ntiles = acc;
+    const int grid = static_cast<int>(acc < di.sms ? acc : di.sms);
+    const CUtensorMap& tin = stage == 0 ? tq : th[(stage - 1) & 1];
+    cudaError_t e = launch_module_gemm(tq, tin, g, grid, sh.smem, st);
+    if (e != cudaSuccess) return cuda_fail(e, "module GEMM kernel");
+  }
+  return NECTAR_OK;
+}
 
 nectar_status prepare_modules(const nectar_dims& dims, const nectar_module_set* mods, const nectar_bf16* Q,
                               int64_t nq, bool fuse, ModParams* p, CUtensorMap* tq, ModShape* sh) {
@@ -464,6 +617,7 @@ nectar_status prepare_modules(const nectar_dims& dims, const nectar_module_set* 
   std::stable_sort(ord.begin(), ord.end(), [&](int a, int b) { return mods->width[a] > mods->width[b]; });
   for (int l = 0; l < dims.L; ++l) p->order[l] = static_cast<uint8_t>(ord[l]);
   p->Hmax = Hmax;
+  if (use_gemm_path(dims, nq)) return NECTAR_OK;      // the layer-by-layer path needs no fused shape
   *sh = mod_shape(dims.G, nq, Hmax, fuse);
   if (sh->smem > 227 * 1024) return fail(NECTAR_ERR_UNSUPPORTED, "width %d needs too much shared memory", Hmax);
   p->N = sh->N;
@@ -488,8 +642,16 @@ nectar_status prepare_modules(const nectar_dims& dims, const nectar_module_set* 
 
 extern "C" {
 
+size_t nectar_module_workspace_size(nectar_dims dims, const nectar_module_set* mods, int64_t nq) {
+  if (check_dims(dims) != NECTAR_OK || nq <= 0 || mods == nullptr) return 0;
+  if (check_modules_shape(dims, mods->depth, mods->width) != NECTAR_OK) return 0;
+  if (!use_gemm_path(dims, nq)) return 0;
+  return gemm_ws_bytes(dims, mods_hmax(dims, mods->width), mods->depth, nq);
+}
+
 nectar_status nectar_module_forward(nectar_dims dims, const nectar_module_set* mods, const nectar_bf16* Q, int64_t nq,
-                                    float* a, float* A_theta, nectar_stream_t stream) {
+                                    float* a, float* A_theta, void* workspace, size_t workspace_bytes,
+                                    nectar_stream_t stream) {
   NECTAR_TRY(check_dims(dims));
   if (nq < 0) return fail(NECTAR_ERR_INVALID_ARG, "nq must be >= 0");
   if (nq == 0) return NECTAR_OK;
@@ -499,17 +661,30 @@ nectar_status nectar_module_forward(nectar_dims dims, const nectar_module_set* m
   CUtensorMap tq;
   ModShape sh;
   NECTAR_TRY(prepare_modules(dims, mods, Q, nq, false, &p, &tq, &sh));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (use_gemm_path(dims, nq)) {
+    const size_t need = gemm_ws_bytes(dims, p.Hmax, p.depth, nq);
+    if (workspace == nullptr || workspace_bytes < need)
+      return fail(NECTAR_ERR_WORKSPACE, "module workspace of %zu bytes given, %zu needed",
+                  workspace == nullptr ? size_t(0) : workspace_bytes, need);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0)
+      return fail(NECTAR_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    return run_module_gemm(dims, p, Q, nq, a, A_theta, nullptr, workspace, st);
+  }
   p.a_out = a;
   p.A_out = A_theta;
   const int units = dims.L * dims.Hkv * sh.nblk;
-  cudaError_t e = launch_module(tq, p, units, sh.smem, false, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_module(tq, p, units, sh.smem, false, st);
   return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "module kernel");
 }
 
-size_t nectar_decode_workspace_size(nectar_dims dims, int64_t nq) {
-  if (check_dims(dims) != NECTAR_OK || nq <= 0) return 0;
+size_t nectar_decode_workspace_size(nectar_dims dims, const nectar_module_set* mods, int64_t nq) {
+  if (check_dims(dims) != NECTAR_OK || nq <= 0 || mods == nullptr) return 0;
+  if (check_modules_shape(dims, mods->depth, mods->width) != NECTAR_OK) return 0;
   const int64_t rows = static_cast<int64_t>(dims.L) * dims.Hkv * dims.G * nq;
-  return decode_ws_a_bytes(rows) + static_cast<size_t>(rows) * (kD + 2) * sizeof(float);
+  const size_t loc = align256(static_cast<size_t>(rows) * (kD + 2) * sizeof(float));
+  if (use_gemm_path(dims, nq)) return loc + gemm_ws_bytes(dims, mods_hmax(dims, mods->width), mods->depth, nq);
+  return decode_ws_a_bytes(rows) + loc;
 }
 
 nectar_status nectar_decode(nectar_dims dims, const nectar_module_set* mods, const nectar_bf16* Q, int64_t nq,
@@ -523,7 +698,9 @@ nectar_status nectar_decode(nectar_dims dims, const nectar_module_set* mods, con
   if (!(scale == scale)) return fail(NECTAR_ERR_INVALID_ARG, "scale is NaN");
   NECTAR_TRY(check_ptr(out, "out"));
   NECTAR_TRY(check_local(q_seq, q_pos, Kloc, Vloc, B, T_max, local_len));
-  const size_t need = nectar_decode_workspace_size(dims, nq);
+  if (mods == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "mods is NULL");
+  NECTAR_TRY(check_modules_shape(dims, mods->depth, mods->width));
+  const size_t need = nectar_decode_workspace_size(dims, mods, nq);
   if (workspace == nullptr || workspace_bytes < need)
     return fail(NECTAR_ERR_WORKSPACE, "decode workspace of %zu bytes given, %zu needed",
                 workspace == nullptr ? size_t(0) : workspace_bytes, need);
@@ -535,7 +712,8 @@ nectar_status nectar_decode(nectar_dims dims, const nectar_module_set* mods, con
   NECTAR_TRY(prepare_modules(dims, mods, Q, nq, true, &p, &tq, &sh));
   const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
   const int64_t rows = heads * dims.G * nq;
-  if (heads * nq + static_cast<int64_t>(dims.L) * dims.Hkv * sh.nblk > 0x7fffffffLL)
+  const bool gemm = use_gemm_path(dims, nq);
+  if (heads * nq + (gemm ? 0 : static_cast<int64_t>(dims.L) * dims.Hkv * sh.nblk) > 0x7fffffffLL)
     return fail(NECTAR_ERR_UNSUPPORTED, "too many CTAs for one launch");
   p.q_seq = q_seq;
   p.q_pos = q_pos;
@@ -546,12 +724,27 @@ nectar_status nectar_decode(nectar_dims dims, const nectar_module_set* mods, con
   p.T = T_max;
   p.qmul = scale * kLog2e;
   p.out = out;
+  p.n_local = heads * nq;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (gemm) {
+    // local states first, then the layer-by-layer module whose readout merges
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    p.ws_loc = reinterpret_cast<float*>(base);
+    if (use_local_tc(dims, nq, B, T_max)) {
+      NECTAR_TRY(run_local_tc(dims, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, p.ws_loc, nullptr,
+                              nullptr, nullptr, st));
+    } else {
+      cudaError_t e = launch_local_state(p, st);
+      if (e != cudaSuccess) return cuda_fail(e, "local attention kernel");
+    }
+    return run_module_gemm(dims, p, Q, nq, nullptr, out, p.ws_loc,
+                           base + align256(static_cast<size_t>(rows) * (kD + 2) * sizeof(float)), st);
+  }
   p.a_out = static_cast<float*>(workspace);
   p.A_out = out;                    // A_theta lands in out, merged in place
   p.ws_loc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + decode_ws_a_bytes(rows));
-  p.n_local = heads * nq;
   const int units = dims.L * dims.Hkv * sh.nblk;
-  cudaError_t e = launch_decode(tq, p, units, sh.smem, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_decode(tq, p, units, sh.smem, st);
   return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "decode kernels");
 }
 

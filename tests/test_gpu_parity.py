@@ -226,6 +226,72 @@ def test_merge_bad_metadata_flags():
     assert torch.equal(out[..., 1, :], Ad[..., 1, :])
 
 
+# many query rows per KV head: the tensor-core local kernel (one job per
+# (KV head, token), 128-key tiles)
+@pytest.mark.parametrize("G,T", [(1, 300), (4, 33), (7, 256), (33, 130)])
+def test_merge_many_tokens(G, T):
+    nq = max(128 // G + 1, 8)
+    B = 5
+    g = torch.Generator().manual_seed(G * 1000 + T)
+    q_seq = torch.randint(0, B, (nq,), generator=g).tolist()
+    local_len = [T, 0, 1, T // 2 + 3, T - 1]
+    q_pos = torch.randint(0, T, (nq,), generator=g).tolist()
+    q_pos[0] = 0
+    out, Ad = merge_case(G, nq, B, T, q_seq, q_pos, local_len, seed=G + T)
+    # tokens of the sequence with no local tokens keep the document term
+    o = out.cpu().reshape(2, G, nq, 128)
+    A = Ad.reshape(2, G, nq, 128)
+    for i, b in enumerate(q_seq):
+        if b == 1:
+            assert torch.equal(o[:, :, i], A[:, :, i])
+
+
+def test_merge_prefill_causal_many_tiles():
+    T = 300
+    merge_case(4, T, 1, T, [0] * T, list(range(T)), [T], L=1, Hkv=1, seed=13)
+
+
+def test_merge_tc_running_max_moves():
+    # keys of the second 128-key tile score far above the first: the running
+    # maximum jumps by more than the lazy-rescale slack inside one job
+    G, nq, B, T = 4, 40, 2, 256
+    g = torch.Generator().manual_seed(21)
+    rows = G * nq
+    Q = torch.randn(1, 2, G, nq, 128, generator=g).to(torch.bfloat16)
+    Kl = torch.randn(1, 2, B, T, 128, generator=g)
+    Kl[:, :, :, 128:] *= 8.0
+    Kl = Kl.to(torch.bfloat16)
+    Vl = torch.randn(1, 2, B, T, 128, generator=g).to(torch.bfloat16)
+    a = torch.randn(1, 2, G, nq, generator=g).float()
+    Ad = torch.randn(1, 2, G, nq, 128, generator=g).float()
+    qs = torch.tensor([i % B for i in range(nq)], dtype=torch.int32)
+    qp = torch.full((nq,), T - 1, dtype=torch.int32)
+    ll = torch.tensor([T, T], dtype=torch.int32)
+    out = nx.merge_local(cuda(a), cuda(Ad), cuda(Q), cuda(qs), cuda(qp), cuda(Kl), cuda(Vl), cuda(ll))
+    torch.cuda.synchronize()
+    ref = oracle.merge_local(a.reshape(2, rows), Ad.reshape(2, rows, 128), Q.reshape(2, rows, 128), qs, qp,
+                             Kl.reshape(2, B, T, 128), Vl.reshape(2, B, T, 128), ll, 1 / math.sqrt(128))
+    vmax = max(Vl.float().abs().max().item(), Ad.abs().max().item())
+    assert np.abs(out.cpu().numpy().reshape(2, rows, 128) - ref).max() <= ATT_TOL * vmax
+
+
+def test_merge_tc_bad_metadata_flags():
+    nx.device_error_flags(clear=True)
+    G, nq, B, T = 4, 64, 2, 16
+    g = torch.Generator().manual_seed(2)
+    Q = torch.randn(1, 1, G, nq, 128, generator=g).to(torch.bfloat16).cuda()
+    Kl = torch.randn(1, 1, B, T, 128, generator=g).to(torch.bfloat16).cuda()
+    a = torch.zeros(1, 1, G, nq).cuda()
+    Ad = torch.randn(1, 1, G, nq, 128).cuda()
+    qs = torch.zeros(nq, dtype=torch.int32)
+    qs[5] = 7                                                  # not a sequence
+    qp = torch.full((nq,), T - 1, dtype=torch.int32)
+    ll = torch.tensor([T, T], dtype=torch.int32)
+    out = nx.merge_local(a, Ad, Q, qs.cuda(), qp.cuda(), Kl, Kl, ll.cuda())
+    assert nx.device_error_flags(clear=True) & 2
+    assert torch.equal(out[..., 5, :], Ad[..., 5, :])
+
+
 def test_split_identity_on_gpu():
     """merge(exact alpha, A) == full attention over document + local (Eq. (3.4))."""
     wl = make_workload("toy", L=1, Hkv=2, G=2, n=1500, nq=6, B=2, T=20, mode="decode", with_modules=False, seed=8)
@@ -272,6 +338,11 @@ def test_module_forward_toy():
     dict(L=3, Hkv=1, G=4, nq=20, widths=[16, 1024, 144], depth=2),
     dict(L=1, Hkv=2, G=1, nq=33, widths=[64], depth=1),
     dict(L=1, Hkv=1, G=3, nq=7, widths=[128], depth=3),
+    # >= 128 rows per KV head: the layer-by-layer grouped-GEMM path
+    dict(L=2, Hkv=2, G=7, nq=40, widths=[208, 96], depth=2),    # 280 rows: two ragged row tiles
+    dict(L=3, Hkv=1, G=4, nq=300, widths=[16, 1024, 144], depth=3),   # 1200 rows, 5 row tiles
+    dict(L=1, Hkv=2, G=1, nq=130, widths=[64], depth=1),        # depth 1: readout straight from h_0
+    dict(L=1, Hkv=1, G=2, nq=64, widths=[512], depth=2),        # exactly 128 rows
 ])
 def test_module_forward_shapes(kw):
     kw = dict(kw)
@@ -319,6 +390,8 @@ def test_decode_toy_prefill():
     dict(L=2, Hkv=1, G=4, n=16, B=20, T=17, widths=[1024, 64]),
     dict(L=1, Hkv=2, G=8, n=16, B=5, T=70, widths=[256]),      # 8 heads per local job
     dict(L=1, Hkv=1, G=12, n=16, B=4, T=45, widths=[128]),     # two local jobs per token (8 + 4 heads)
+    dict(L=2, Hkv=2, G=4, n=16, B=40, T=50, widths=[256, 512]),   # 160 rows per KV head: GEMM path
+    dict(L=1, Hkv=2, G=7, n=16, B=64, T=33, widths=[768]),     # 448 rows: two row tiles of 224
 ])
 def test_decode_shapes(kw):
     wl = make_workload("qwen3_1p7b", seed=2, key_scale=None, **kw)
@@ -331,8 +404,12 @@ def test_decode_workspace_checked():
     wl = make_workload("toy", seed=4)
     mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G)
     args = (cuda(wl.Q), cuda(wl.q_seq), cuda(wl.q_pos), cuda(wl.Kloc), cuda(wl.Vloc), cuda(wl.local_len))
-    need = nx.decode_workspace_size(wl.L, wl.Hkv, wl.G, wl.nq)
-    assert need == (wl.heads * wl.rows * 4 + 255) // 256 * 256 + wl.heads * wl.rows * 130 * 4
+    need = nx.decode_workspace_size(mods, wl.G, wl.nq)
+    loc = (wl.heads * wl.rows * 130 * 4 + 255) // 256 * 256
+    if wl.rows < 128:
+        assert need == (wl.heads * wl.rows * 4 + 255) // 256 * 256 + loc
+    else:
+        assert need == loc + nx.module_workspace_size(mods, wl.G, wl.nq) > loc
     out = torch.full(wl.Q.shape, float("nan"), device="cuda")
     small = torch.empty(need - 4, dtype=torch.uint8, device="cuda")
     with pytest.raises(RuntimeError, match="workspace"):
