@@ -41,9 +41,11 @@ constexpr int kTcRows = 128;                       // query rows per tile
 constexpr int kTcUnitRows = 2 * kTcRows;           // two tiles per unit
 constexpr int kTcKeys = 64;                        // keys per tile
 #ifndef NECTAR_TC_POLY_PAIRS
-#define NECTAR_TC_POLY_PAIRS 1
+#define NECTAR_TC_POLY_PAIRS 0
 #endif
-// of every 4 pairs of softmax weights, how many use exp2_poly (0..4)
+// of every 4 pairs of softmax weights, how many use exp2_poly (0..4); 0:
+// measured on B200, moving exponentials to the FMA pipe made the softmax
+// slower (the special-function unit is not its limit)
 constexpr int kTcPolyPairs = NECTAR_TC_POLY_PAIRS;
 constexpr int kTcStages = 3;                       // K and V ring depth
 constexpr int kTcThreads = 11 * 32;
@@ -315,15 +317,28 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         mbar_arrive(b_sfree + 8 * (2 * t + b));
         float bm = -INFINITY;
         if (full) {
-          float x = sc[0];
+          // four independent chains (a 64-deep dependent chain would
+          // expose its latency on every tile)
+          float x0 = sc[0], x1 = sc[1], x2 = sc[2], x3 = sc[3];
           if (p.qmul >= 0.f) {
 #pragma unroll
-            for (int e = 1; e < kTcKeys; ++e) x = fmaxf(x, sc[e]);
+            for (int e = 4; e < kTcKeys; e += 4) {
+              x0 = fmaxf(x0, sc[e]);
+              x1 = fmaxf(x1, sc[e + 1]);
+              x2 = fmaxf(x2, sc[e + 2]);
+              x3 = fmaxf(x3, sc[e + 3]);
+            }
+            bm = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)) * p.qmul;
           } else {
 #pragma unroll
-            for (int e = 1; e < kTcKeys; ++e) x = fminf(x, sc[e]);
+            for (int e = 4; e < kTcKeys; e += 4) {
+              x0 = fminf(x0, sc[e]);
+              x1 = fminf(x1, sc[e + 1]);
+              x2 = fminf(x2, sc[e + 2]);
+              x3 = fminf(x3, sc[e + 3]);
+            }
+            bm = fminf(fminf(x0, x1), fminf(x2, x3)) * p.qmul;
           }
-          bm = x * p.qmul;
         } else {
 #pragma unroll
           for (int e = 0; e < kTcKeys; ++e) {
@@ -357,7 +372,7 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         // P buffer b was last read by the P V of this tile's S count cnt - 2
         if (cnt >= 2 && ok) ok = mbar_wait(b_pvdone + 8 * (2 * t + b), ((cnt >> 1) - 1) & 1, p.err);
         uint8_t* pt = smem + TcSmem::p + (2 * t + b) * kPBytes;
-        float2 rs2 = make_float2(0.f, 0.f);
+        float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const float2 q2 = make_float2(p.qmul, p.qmul), nm2 = make_float2(-m, -m);
 #pragma unroll
         for (int c8 = 0; c8 < kTcKeys / 8; ++c8) {
@@ -376,11 +391,11 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
               w[e] = pack_bf16x2(exp2_shift(s0, m), exp2_shift(s1, m));
             }
             // the row sum adds the rounded weights that P V uses
-            rs2 = fadd2(rs2, make_float2(bf16lo(w[e]), bf16hi(w[e])));
+            rs2[e & 1] = fadd2(rs2[e & 1], make_float2(bf16lo(w[e]), bf16hi(w[e])));
           }
           *reinterpret_cast<uint4*>(pt + p_off(row, c8 * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        l += rs2.x + rs2.y;
+        l += (rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y);
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(b_pfull + 8 * (2 * t + b));

@@ -118,18 +118,23 @@ struct RowState {
     }
   }
 
-  // Process KPG keys of this group.  krow[k] / vrow[k] point at the 256-byte
-  // rows; invalid keys are skipped (their rows are never read).
+  // Load this lane's 16-byte pieces of KPG key (or value) rows; invalid
+  // keys read nothing and give zeros.
   template <int KPG, class Loader>
-  __device__ __forceinline__ void step(const uint8_t* const* krow, const uint8_t* const* vrow,
-                                       const bool* valid, int t, const Loader& ld) {
-    float sc[KPG][R];
-    uint4 kw[KPG][CPL];
+  __device__ __forceinline__ static void load_rows(const uint8_t* const* row, const bool* valid, int t,
+                                                   const Loader& ld, uint4 (&w)[KPG][CPL]) {
 #pragma unroll
     for (int k = 0; k < KPG; ++k)
 #pragma unroll
       for (int ci = 0; ci < CPL; ++ci)
-        kw[k][ci] = valid[k] ? ld(krow[k] + 16 * (t + LPK * ci)) : make_uint4(0, 0, 0, 0);
+        w[k][ci] = valid[k] ? ld(row[k] + 16 * (t + LPK * ci)) : make_uint4(0, 0, 0, 0);
+  }
+
+  // Scores of KPG keys (log2 units, -inf for invalid keys), the lazy
+  // rescale of the running state, and the keys' weights pw.
+  template <int KPG>
+  __device__ __forceinline__ void weigh(const uint4 (&kw)[KPG][CPL], const bool* valid, float (&pw)[KPG][R]) {
+    float sc[KPG][R];
 #pragma unroll
     for (int k = 0; k < KPG; ++k) {
       float part[R];
@@ -165,7 +170,6 @@ struct RowState {
         m[r] = bm;
       }
     }
-    float pw[KPG][R];
 #pragma unroll
     for (int k = 0; k < KPG; ++k)
 #pragma unroll
@@ -173,12 +177,12 @@ struct RowState {
         pw[k][r] = exp2_shift(sc[k][r], m[r]);
         l[r] += pw[k][r];
       }
-    uint4 vw[KPG][CPL];
-#pragma unroll
-    for (int k = 0; k < KPG; ++k)
-#pragma unroll
-      for (int ci = 0; ci < CPL; ++ci)
-        vw[k][ci] = valid[k] ? ld(vrow[k] + 16 * (t + LPK * ci)) : make_uint4(0, 0, 0, 0);
+  }
+
+  // acc += pw * v over KPG value rows.  (Paired f32x2 FMAs here measured
+  // slower in the decode kernel: the accumulators are separate registers.)
+  template <int KPG>
+  __device__ __forceinline__ void accumulate(const uint4 (&vw)[KPG][CPL], const float (&pw)[KPG][R]) {
 #pragma unroll
     for (int k = 0; k < KPG; ++k)
 #pragma unroll
@@ -190,6 +194,23 @@ struct RowState {
 #pragma unroll
           for (int e = 0; e < 8; ++e) acc[r][ci * 8 + e] = fmaf(pw[k][r], vf[e], acc[r][ci * 8 + e]);
       }
+  }
+
+  // Process KPG keys of this group.  krow[k] / vrow[k] point at the 256-byte
+  // rows; invalid keys are skipped (their rows are never read).  kEarlyV
+  // issues the V loads together with the K loads (more bytes in flight when
+  // the rows come straight from global memory).
+  template <int KPG, class Loader, bool kEarlyV = false>
+  __device__ __forceinline__ void step(const uint8_t* const* krow, const uint8_t* const* vrow,
+                                       const bool* valid, int t, const Loader& ld) {
+    uint4 kw[KPG][CPL];
+    uint4 vw[KPG][CPL];
+    float pw[KPG][R];
+    load_rows<KPG>(krow, valid, t, ld, kw);
+    if (kEarlyV) load_rows<KPG>(vrow, valid, t, ld, vw);
+    weigh<KPG>(kw, valid, pw);
+    if (!kEarlyV) load_rows<KPG>(vrow, valid, t, ld, vw);
+    accumulate<KPG>(vw, pw);
   }
 
   // Join the NG groups of the warp (xor over lane bits >= LPK); afterwards

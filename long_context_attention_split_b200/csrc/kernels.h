@@ -144,11 +144,16 @@ cudaError_t launch_module_gemm(const CUtensorMap& tq, const CUtensorMap& th, con
                                size_t smem, cudaStream_t stream);
 cudaError_t launch_local_state(const ModParams& p, cudaStream_t stream);
 
-// Tensor-core local attention (local_tc.cu).
-struct LocTcParams {
+// Local attention for many query tokens: one job per (KV head, token) on the
+// tensor cores (local_tc.cu) or per (KV head, token, block of <= 4 heads)
+// on one warp (local_warp.cu).
+struct LocalParams {
   int64_t njobs;            // heads * nq
   int64_t nq;
   int G, B, T, kbox;        // kbox = keys per TMA box, min(128, T)
+  const __nv_bfloat16* Q;   // [heads][G][nq][d]
+  const __nv_bfloat16* Kloc;  // [heads][B][T][d]
+  const __nv_bfloat16* Vloc;
   const int32_t* q_seq;
   const int32_t* q_pos;
   const int32_t* local_len;
@@ -161,7 +166,8 @@ struct LocTcParams {
 };
 size_t local_tc_smem();
 cudaError_t launch_local_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const LocTcParams& p, int grid, cudaStream_t stream);
+                            const LocalParams& p, int grid, cudaStream_t stream);
+cudaError_t launch_local_warp(const LocalParams& p, int sms, cudaStream_t stream);
 
 struct ModShape {
   int TPC, N, nblk, tmem_cols, stages, cps;

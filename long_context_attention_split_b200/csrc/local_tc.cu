@@ -62,7 +62,7 @@ struct LJob {
   int b, nv, ntiles;
 };
 
-__device__ __forceinline__ LJob local_job(const LocTcParams& p, int64_t j) {
+__device__ __forceinline__ LJob local_job(const LocalParams& p, int64_t j) {
   LJob J;
   J.hd = j / p.nq;
   J.i = j % p.nq;
@@ -75,7 +75,7 @@ __device__ __forceinline__ LJob local_job(const LocTcParams& p, int64_t j) {
 
 __global__ void __launch_bounds__(kLThreads, 1)
 local_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-                const __grid_constant__ CUtensorMap tmap_v, const LocTcParams p) {
+                const __grid_constant__ CUtensorMap tmap_v, const LocalParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LSmem::bars);
@@ -385,7 +385,7 @@ local_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
 size_t local_tc_smem() { return LSmem::total + 1024; }
 
 cudaError_t launch_local_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const LocTcParams& p, int grid, cudaStream_t stream) {
+                            const LocalParams& p, int grid, cudaStream_t stream) {
   const size_t smem = local_tc_smem();
   cudaError_t e =
       cudaFuncSetAttribute(local_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

@@ -80,13 +80,13 @@ __host__ __device__ inline size_t dec_local_smem(int RG) {
   return size_t(kDecLocStages) * kLocStageBytes + size_t(kDecLocCW) * RG * (kD + 2) * 4 + 2 * kDecLocStages * 8;
 }
 
+__device__ __forceinline__ float mod_silu(float v) { return __fdividef(v, 1.0f + ex2(-v * kLog2e)); }
+
 // element (row n, column c) of the swizzled K-major activation matrix X
 __device__ __forceinline__ uint32_t x_offset(int N, int n, int c) {
   return static_cast<uint32_t>((c >> 6) * (N * 128) + n * 128 + ((((c & 63) >> 3) ^ (n & 7)) << 4) +
                                ((c & 7) << 1));
 }
-
-__device__ __forceinline__ float silu(float v) { return __fdividef(v, 1.0f + ex2(-v * kLog2e)); }
 
 // One module CTA: (a_theta, A_theta) of the rows of `unit`.  smem is the
 // 1024-aligned dynamic shared memory.  a goes to p.a_out[hd * rows + row],
@@ -289,10 +289,19 @@ __device__ __forceinline__ void module_cta(const CUtensorMap* tmap_q, const ModP
                     wv = wvs[q];
                   }
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                  const __nv_bfloat16 hb = __float2bfloat16_rn(silu(__uint_as_float(v[mm][j]) + bv));
-                  if (readout) part[j] = fmaf(wv, __bfloat162float(hb), part[j]);
-                  else *reinterpret_cast<__nv_bfloat16*>(smem + L.x + x_offset(N, n0 + j, kD + i)) = hb;
+                for (int j = 0; j < 16; j += 2) {
+                  // two rows rounded to bf16 by one packed conversion
+                  const uint32_t w = pack_bf16x2(mod_silu(__uint_as_float(v[mm][j]) + bv),
+                                                 mod_silu(__uint_as_float(v[mm][j + 1]) + bv));
+                  if (readout) {
+                    part[j] = fmaf(wv, bf16lo(w), part[j]);
+                    part[j + 1] = fmaf(wv, bf16hi(w), part[j + 1]);
+                  } else {
+                    *reinterpret_cast<uint16_t*>(smem + L.x + x_offset(N, n0 + j, kD + i)) =
+                        static_cast<uint16_t>(w & 0xFFFFu);
+                    *reinterpret_cast<uint16_t*>(smem + L.x + x_offset(N, n0 + j + 1, kD + i)) =
+                        static_cast<uint16_t>(w >> 16);
+                  }
                 }
               }
             }

@@ -34,7 +34,8 @@
 
 namespace nectar {
 
-constexpr int kGemmThreads = 6 * 32;
+constexpr int kGemmEpiWarps = 8;             // two per TMEM lane quarter
+constexpr int kGemmThreads = (2 + kGemmEpiWarps) * 32;
 constexpr int kGemmWBytes = 128 * 128;        // one weight chunk: 128 rows x 64 bf16
 
 __host__ __device__ inline uint32_t gemm_stage_bytes(int NR) {
@@ -61,6 +62,8 @@ __host__ __device__ inline GemmSmem gemm_smem_layout(int NR, int stages) {
   return s;
 }
 
+__device__ __forceinline__ float gemm_silu(float v) { return __fdividef(v, 1.0f + ex2(-v * kLog2e)); }
+
 struct GemmTile {
   int l, H, net, m, rt;
   int64_t hd;
@@ -84,8 +87,6 @@ __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int64_t t) {
   g.hd = static_cast<int64_t>(g.l) * p.Hkv + h;
   return g;
 }
-
-__device__ __forceinline__ float gemm_silu(float v) { return __fdividef(v, 1.0f + ex2(-v * kLog2e)); }
 
 // Sum over the 32 lanes of v[j] for j = 0..31; lane j returns the total of
 // row j (halving exchange: 31 shuffles instead of 160).
@@ -130,7 +131,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(b_accf + 8 * b, 1);
-      mbar_init(b_acce + 8 * b, 4);
+      mbar_init(b_acce + 8 * b, kGemmEpiWarps);
     }
     fence_barrier_init();
   }
@@ -214,6 +215,8 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   } else {
     // ------------------------------ epilogue ------------------------------
     const int q4 = warp & 3;                  // TMEM lane quarter of this warp
+    const int eh = (warp - 2) >> 2;           // which of the quarter's two warps
+    const int et = threadIdx.x - 64;          // 0 .. 32 * kGemmEpiWarps - 1
     const int u = q4 * 32 + lane;             // accumulator lane: hidden unit or output dim
     const uint32_t tlane = static_cast<uint32_t>(q4 * 32) << 16;
     uint32_t tc = 0;
@@ -240,7 +243,8 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       ok = __all_sync(0xffffffffu, ok);         // keeps the shuffles below warp-uniform
       tc_fence_after();
       const uint32_t dacc = tmem + tlane + b * static_cast<uint32_t>(NR);
-      for (int n0 = 0; n0 < NR; n0 += 32) {
+      // the two warps of a lane quarter take alternate 32-column batches
+      for (int n0 = 32 * eh; n0 < NR; n0 += 64) {
         uint32_t v[32];
         NECTAR_TMEM_LD32(dacc + n0, v);
         tmem_ld_wait();
@@ -249,9 +253,12 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
           if (score_last) {
             float part[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float hv = __bfloat162float(__float2bfloat16_rn(gemm_silu(__uint_as_float(v[j]) + bias)));
-              part[j] = (i < g.H) ? wsc * hv : 0.f;
+            for (int j = 0; j < 32; j += 2) {
+              // bf16 rounding of two rows at once (one packed conversion)
+              const uint32_t w = pack_bf16x2(gemm_silu(__uint_as_float(v[j]) + bias),
+                                             gemm_silu(__uint_as_float(v[j + 1]) + bias));
+              part[j] = (i < g.H) ? wsc * bf16lo(w) : 0.f;
+              part[j + 1] = (i < g.H) ? wsc * bf16hi(w) : 0.f;
             }
             const float tot = warp_transpose_sum32(part, lane);
             if (n0 + lane < NR) red[q4 * NR + n0 + lane] = tot;
@@ -259,11 +266,15 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
             const int Hp = p.Hp;
             const int64_t hrow0 = (g.net * heads + g.hd) * R;
             if (i < layout::round64(g.H)) {
+              uint16_t* hcol = reinterpret_cast<uint16_t*>(p.h_out) + hrow0 * Hp + i;
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
+              for (int j = 0; j < 32; j += 2) {
                 const int r = r0 + n0 + j;
-                const float hv = (i < g.H) ? gemm_silu(__uint_as_float(v[j]) + bias) : 0.f;
-                if (r < rend) p.h_out[(hrow0 + r) * Hp + i] = __float2bfloat16_rn(hv);
+                const uint32_t w = (i < g.H) ? pack_bf16x2(gemm_silu(__uint_as_float(v[j]) + bias),
+                                                           gemm_silu(__uint_as_float(v[j + 1]) + bias))
+                                             : 0u;
+                if (r < rend) hcol[static_cast<int64_t>(r) * Hp] = static_cast<uint16_t>(w & 0xFFFFu);
+                if (r + 1 < rend) hcol[static_cast<int64_t>(r + 1) * Hp] = static_cast<uint16_t>(w >> 16);
               }
             }
           }
@@ -280,7 +291,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
               if (q4 == 0 && p.a_out != nullptr) p.a_out[g.hd * R + r] = a_l;
             }
           }
-#pragma unroll 4
+#pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int r = r0 + n0 + j;
             const float aj = __shfl_sync(0xffffffffu, a_l, j);
@@ -304,13 +315,13 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       __syncwarp();
       if (lane == 0) mbar_arrive(b_acce + 8 * b);
       if (score_last) {
-        named_bar_sync(2, 4 * 32);
-        for (int n = u; n < NR; n += 128) {
+        named_bar_sync(2, kGemmEpiWarps * 32);
+        for (int n = et; n < NR; n += kGemmEpiWarps * 32) {
           const int r = r0 + n;
           if (ok && r < rend)
             p.part[(g.hd * R + r) * p.MT + g.m] = (red[n] + red[NR + n]) + (red[2 * NR + n] + red[3 * NR + n]);
         }
-        named_bar_sync(2, 4 * 32);
+        named_bar_sync(2, kGemmEpiWarps * 32);
       }
     }
   }

@@ -89,6 +89,16 @@ DeviceInfo device_info() {
 }
 
 // Row blocks handled by one launch of the CUDA-core split kernel.
+#ifndef NECTAR_TC_ROUTE_ROWS
+#define NECTAR_TC_ROUTE_ROWS 8
+#endif
+// More query rows per KV head than this: the tensor-core kernel; else the
+// split kernel on the CUDA cores (at most dec_max_rows() rows).
+bool use_tc_attn(int64_t rows) {
+  const int64_t lim = NECTAR_TC_ROUTE_ROWS < dec_max_rows() ? NECTAR_TC_ROUTE_ROWS : dec_max_rows();
+  return rows > lim;
+}
+
 int dec_row_block(int64_t rows) { return rows < dec_max_rows() ? static_cast<int>(rows) : dec_max_rows(); }
 
 DecPlan cache_attn_plan(const nectar_dims& d, int64_t n, int64_t nq, int sms) {
@@ -174,7 +184,7 @@ size_t nectar_cache_attn_workspace_size(nectar_dims dims, int64_t n, int64_t nq)
   if (rows == 0 || n == 0) return 0;
   const DeviceInfo di = device_info();
   if (di.sms == 0) return 0;
-  if (rows > dec_max_rows()) {
+  if (use_tc_attn(rows)) {
     const TcPlan tp = plan_tc(dims.L * dims.Hkv, n, rows, di.sms);
     return tp.ws_bytes + 256;
   }
@@ -227,7 +237,7 @@ nectar_status nectar_cache_attn_lse(nectar_dims dims, const nectar_bf16* K, cons
   if (workspace == nullptr || workspace_bytes < need)
     return fail(NECTAR_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
   if (!aligned16(workspace)) return fail(NECTAR_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
-  if (rows > dec_max_rows()) {
+  if (use_tc_attn(rows)) {
     // many query rows per head: tcgen05 flash-style kernel
     const TcPlan tp = plan_tc(heads, n, rows, di.sms);
     TcParams tpar{};
@@ -312,13 +322,16 @@ static nectar_status run_local_tc(const nectar_dims& dims, const nectar_bf16* Q,
   const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
   if (heads * B > 0x7fffffffLL || heads > 0x7fffffffLL || nq > 0x7fffffffLL)
     return fail(NECTAR_ERR_UNSUPPORTED, "local cache too large for one call");
-  LocTcParams p{};
+  LocalParams p{};
   p.njobs = heads * nq;
   p.nq = nq;
   p.G = dims.G;
   p.B = B;
   p.T = T_max;
   p.kbox = T_max < 128 ? T_max : 128;
+  p.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  p.Kloc = reinterpret_cast<const __nv_bfloat16*>(Kloc);
+  p.Vloc = reinterpret_cast<const __nv_bfloat16*>(Vloc);
   p.q_seq = q_seq;
   p.q_pos = q_pos;
   p.local_len = local_len;
@@ -347,6 +360,49 @@ static nectar_status run_local_tc(const nectar_dims& dims, const nectar_bf16* Q,
   return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "local attention kernel");
 }
 
+// The same result from the warp-per-job CUDA-core kernel (local_warp.cu).
+static nectar_status run_local_warp(const nectar_dims& dims, const nectar_bf16* Q, int64_t nq,
+                                    const int32_t* q_seq, const int32_t* q_pos, const nectar_bf16* Kloc,
+                                    const nectar_bf16* Vloc, int32_t B, int32_t T_max, const int32_t* local_len,
+                                    float scale, float* ws_loc, const float* a, const float* A_doc, float* out,
+                                    cudaStream_t st) {
+  const DeviceInfo di = device_info();
+  if (di.sms == 0) return fail(NECTAR_ERR_CUDA, "no CUDA device");
+  LocalParams p{};
+  p.njobs = static_cast<int64_t>(dims.L) * dims.Hkv * nq;
+  p.nq = nq;
+  p.G = dims.G;
+  p.B = B;
+  p.T = T_max;
+  p.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  p.Kloc = reinterpret_cast<const __nv_bfloat16*>(Kloc);
+  p.Vloc = reinterpret_cast<const __nv_bfloat16*>(Vloc);
+  p.q_seq = q_seq;
+  p.q_pos = q_pos;
+  p.local_len = local_len;
+  p.qmul = scale * kLog2e;
+  p.ws_loc = ws_loc;
+  p.a = a;
+  p.A_doc = A_doc;
+  p.out = out;
+  p.err = di.err;
+  cudaError_t e = launch_local_warp(p, di.sms, st);
+  return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "local attention kernel");
+}
+
+// Many query tokens: up to 8 query heads per KV head on warps, more on the
+// tensor cores.
+static nectar_status run_local_many(const nectar_dims& dims, const nectar_bf16* Q, int64_t nq,
+                                    const int32_t* q_seq, const int32_t* q_pos, const nectar_bf16* Kloc,
+                                    const nectar_bf16* Vloc, int32_t B, int32_t T_max, const int32_t* local_len,
+                                    float scale, float* ws_loc, const float* a, const float* A_doc, float* out,
+                                    cudaStream_t st) {
+  if (dims.G <= 8)
+    return run_local_warp(dims, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, ws_loc, a, A_doc, out,
+                          st);
+  return run_local_tc(dims, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, ws_loc, a, A_doc, out, st);
+}
+
 nectar_status nectar_merge_local(nectar_dims dims, const float* a, const float* A_doc, const nectar_bf16* Q,
                                  int64_t nq, const int32_t* q_seq, const int32_t* q_pos,
                                  const nectar_bf16* Kloc, const nectar_bf16* Vloc, int32_t B, int32_t T_max,
@@ -361,8 +417,8 @@ nectar_status nectar_merge_local(nectar_dims dims, const float* a, const float* 
   NECTAR_TRY(check_ptr(out, "out"));
   NECTAR_TRY(check_local(q_seq, q_pos, Kloc, Vloc, B, T_max, local_len));
   if (use_local_tc(dims, nq, B, T_max))
-    return run_local_tc(dims, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, nullptr, a, A_doc, out,
-                        reinterpret_cast<cudaStream_t>(stream));
+    return run_local_many(dims, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, nullptr, a, A_doc, out,
+                          reinterpret_cast<cudaStream_t>(stream));
   if (static_cast<int64_t>(dims.L) * dims.Hkv * nq * ((dims.G + 7) / 8) > 0x7fffffffLL)
     return fail(NECTAR_ERR_INVALID_ARG, "too many (head, token) units");
   MergeParams p{};
@@ -731,8 +787,8 @@ nectar_status nectar_decode(nectar_dims dims, const nectar_module_set* mods, con
     uint8_t* base = static_cast<uint8_t*>(workspace);
     p.ws_loc = reinterpret_cast<float*>(base);
     if (use_local_tc(dims, nq, B, T_max)) {
-      NECTAR_TRY(run_local_tc(dims, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, p.ws_loc, nullptr,
-                              nullptr, nullptr, st));
+      NECTAR_TRY(run_local_many(dims, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, p.ws_loc,
+                                nullptr, nullptr, nullptr, st));
     } else {
       cudaError_t e = launch_local_state(p, st);
       if (e != cudaSuccess) return cuda_fail(e, "local attention kernel");
