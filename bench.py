@@ -422,6 +422,7 @@ def per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args):
     replayed; None when the workload has one layer."""
     if wl.L < 2:
         return None
+    import long_context_attention_split_b200 as nx
     try:
         s = torch.cuda.Stream(dev)
         ws = torch.empty(max(nx.cache_attn_workspace_size(1, wl.Hkv, wl.G, wl.n, wl.nq), 16), dtype=torch.uint8,

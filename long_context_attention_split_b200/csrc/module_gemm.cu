@@ -239,7 +239,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         bias = __bfloat162float(p.blob[nb + layout::hidden_b_off(g.H, p.depth, p.stage) + i]);
         if (score_last) wsc = __bfloat162float(p.blob[nb + layout::out_w_off(g.H, p.depth) + i]);
       }
-      if (ok) ok = mbar_wait(b_accf + 8 * b, (tc >> 1) & 1, p.err);
+      if (ok) ok = mbar_wait_sleep(b_accf + 8 * b, (tc >> 1) & 1, p.err);   // waits out a main loop
       ok = __all_sync(0xffffffffu, ok);         // keeps the shuffles below warp-uniform
       tc_fence_after();
       const uint32_t dacc = tmem + tlane + b * static_cast<uint32_t>(NR);
@@ -266,15 +266,28 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
             const int Hp = p.Hp;
             const int64_t hrow0 = (g.net * heads + g.hd) * R;
             if (i < layout::round64(g.H)) {
-              uint16_t* hcol = reinterpret_cast<uint16_t*>(p.h_out) + hrow0 * Hp + i;
+              // column i of rows r0 + n0 .. ; 32-bit offsets from one base
+              uint16_t* hb = reinterpret_cast<uint16_t*>(p.h_out) + (hrow0 + r0 + n0) * Hp + i;
+              const int nrow = rend - (r0 + n0);       // rows of this batch inside the tile
+              const bool live = i < g.H;
+              if (nrow >= 32) {
 #pragma unroll
-              for (int j = 0; j < 32; j += 2) {
-                const int r = r0 + n0 + j;
-                const uint32_t w = (i < g.H) ? pack_bf16x2(gemm_silu(__uint_as_float(v[j]) + bias),
-                                                           gemm_silu(__uint_as_float(v[j + 1]) + bias))
-                                             : 0u;
-                if (r < rend) hcol[static_cast<int64_t>(r) * Hp] = static_cast<uint16_t>(w & 0xFFFFu);
-                if (r + 1 < rend) hcol[static_cast<int64_t>(r + 1) * Hp] = static_cast<uint16_t>(w >> 16);
+                for (int j = 0; j < 32; j += 2) {
+                  const uint32_t w = live ? pack_bf16x2(gemm_silu(__uint_as_float(v[j]) + bias),
+                                                        gemm_silu(__uint_as_float(v[j + 1]) + bias))
+                                          : 0u;
+                  hb[j * Hp] = static_cast<uint16_t>(w & 0xFFFFu);
+                  hb[(j + 1) * Hp] = static_cast<uint16_t>(w >> 16);
+                }
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                  const uint32_t w = live ? pack_bf16x2(gemm_silu(__uint_as_float(v[j]) + bias),
+                                                        gemm_silu(__uint_as_float(v[j + 1]) + bias))
+                                          : 0u;
+                  if (j < nrow) hb[j * Hp] = static_cast<uint16_t>(w & 0xFFFFu);
+                  if (j + 1 < nrow) hb[(j + 1) * Hp] = static_cast<uint16_t>(w >> 16);
+                }
               }
             }
           }

@@ -60,6 +60,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait with a suspend-time hint: a thread whose phase is not complete is
+// parked by the hardware (it issues nothing) until the phase completes or
+// the hint expires.  For long waits of whole warpgroups (an epilogue waiting
+// out a tile's main loop), where spinning lanes would take issue slots from
+// the warps doing the work; on short, latency-critical waits the wake-up
+// costs more than the spinning (measured on B200).
+constexpr uint32_t kSuspendHintNs = 500000;    // 0.5 ms per try
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
 // Wait for the phase with the given parity to complete.  Returns false (and
 // records DEVERR_WAIT_TIMEOUT) if it has not completed within kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
@@ -67,6 +85,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* er
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      record_error(err, DEVERR_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+}
+// As mbar_wait, parking the thread between tries (mbar_try_wait_sleep).
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
     if (globaltimer() - t0 > kWaitLimitNs) {
       record_error(err, DEVERR_WAIT_TIMEOUT);
       return false;
