@@ -27,6 +27,12 @@
 // the same 2^m makes the result exact.  The row sum adds the bf16-rounded
 // weights that the P V product uses, so A stays a convex combination.
 //
+// A unit with one query tile (at most 128 rows left for it) would leave the
+// second softmax warpgroup idle; its key range is then split between the
+// two warpgroups (interleaved in the K / V ring, both reading query tile
+// 0), and warpgroup 1 hands its (m, l, O) to warpgroup 0 through shared
+// memory at the end of the unit.
+//
 // Warps: 0..3 softmax / epilogue of query tile 0, 4..7 of tile 1 (thread =
 // row = TMEM lane), 8 Q and K producer, 9 V producer, 10 MMA issuer.
 #include <cuda.h>
@@ -58,7 +64,8 @@ struct TcSmem {
   static constexpr uint32_t k = q + 2 * kQBytes;                    // 3 x 16 KB
   static constexpr uint32_t v = k + kTcStages * kKVBytes;           // 3 x 16 KB
   static constexpr uint32_t p = v + kTcStages * kKVBytes;           // [tile][buf] 4 x 16 KB
-  static constexpr uint32_t bars = p + 4 * kPBytes;                 // 40 barriers
+  static constexpr uint32_t xml = p + 4 * kPBytes;                  // split units: (m, l) of warpgroup 1
+  static constexpr uint32_t bars = xml + 2 * kTcRows * 4;           // 40 barriers
   static constexpr uint32_t tslot = bars + 40 * 8;
   static constexpr uint32_t total = tslot + 16;
 };
@@ -105,11 +112,142 @@ __device__ __forceinline__ TcSeg tc_seg(const TcParams& p, int c, int i) {
   return sg;
 }
 
+// The key tiles of a segment in ring order.  With two query tiles every
+// key tile serves both softmax warpgroups; with one, warpgroup 0 alone --
+// unless the segment has two or more key tiles: then the warpgroups take
+// the two halves of its range (split), interleaved in the ring, and merge
+// their partial states at the end.  All roles walk the same sequence.
+struct TcItem {
+  int64_t kt;        // key tile
+  uint32_t mask;     // bit t: consumed by softmax warpgroup t
+  bool first;        // first key tile of this segment for the warpgroup(s)
+};
+template <bool kSplit>
+__device__ __forceinline__ bool tc_split(const TcSeg& sg, bool two) { return kSplit && !two && sg.k1 - sg.k0 >= 2; }
+template <bool kSplit>
+__device__ __forceinline__ TcItem tc_item(const TcSeg& sg, bool two, int64_t i) {
+  TcItem it;
+  if (!tc_split<kSplit>(sg, two)) {
+    it.kt = sg.k0 + i;
+    it.mask = two ? 3u : 1u;
+    it.first = i == 0;
+    return it;
+  }
+  const int64_t n0 = (sg.k1 - sg.k0 + 1) / 2;     // warpgroup 0: [k0, k0 + n0), 1: the rest
+  const int64_t pair = i >> 1;
+  if (i & 1) {
+    it.kt = sg.k0 + n0 + pair;
+    it.mask = 2u;
+  } else {
+    it.kt = sg.k0 + pair;
+    it.mask = 1u;
+  }
+  it.first = pair == 0;
+  return it;
+}
+
 // element (row, key) of a K-major SW128 tile of 128 rows x 64 keys
 __device__ __forceinline__ uint32_t p_off(int row, int col) {
   return static_cast<uint32_t>(row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + ((col & 7) << 1));
 }
 
+// End of a unit for softmax warpgroup t, once its last P V is complete:
+// the split hand-off (split units) and the output -- alpha and A, or the
+// partial (m, l, acc) of a unit cut between CTAs.  tO: this thread's TMEM
+// lane of O_t.
+template <bool kSplit>
+__device__ __forceinline__ void tc_unit_epilogue(const TcParams& p, uint8_t* smem, uint32_t tO, uint32_t b_ofree_t,
+                                              const TcSeg& sg, bool split_, int t, int row, float m, float l, bool ok,
+                                              int c) {
+  const bool split = kSplit && split_;
+  // split unit: warpgroup 1 parks its O rows in the P buffers (free once
+  // both warpgroups' last P V is done; 16-byte chunks swizzled by row)
+  // and its (m, l); warpgroup 0 joins the two states by log-sum-exp
+  float4* xo = reinterpret_cast<float4*>(smem + TcSmem::p) + row * (kD / 4);
+  float* xml = reinterpret_cast<float*>(smem + TcSmem::xml);
+  float w0 = 1.f, w1 = 0.f;
+  if (split) {
+    named_bar_sync(1, 2 * kTcRows);
+    if (t == 1) {
+#pragma unroll
+      for (int cb = 0; cb < kD; cb += 16) {
+        uint32_t v[16];
+        NECTAR_TMEM_LD16(tO + cb, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          xo[((cb >> 2) + q4) ^ (row & 31)] =
+              make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                          __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
+      }
+      xml[row] = m;
+      xml[kTcRows + row] = l;
+      tc_fence_before();
+      mbar_arrive(b_ofree_t);
+      named_bar_sync(1, 2 * kTcRows);   // parked
+      named_bar_sync(1, 2 * kTcRows);   // read by warpgroup 0: the P buffers are free again
+      return;
+    }
+    named_bar_sync(1, 2 * kTcRows);     // warpgroup 1's state is parked
+    const float m1 = xml[row], l1 = xml[kTcRows + row];
+    const float M = fmaxf(m, m1);
+    w0 = exp2_shift(m, M);
+    w1 = exp2_shift(m1, M);
+    l = w0 * l + w1 * l1;
+    m = M;
+  }
+  const int64_t hd = sg.unit / p.qpairs;
+  const int64_t qp = sg.unit % p.qpairs;
+  const int64_t r = qp * kTcUnitRows + t * kTcRows + row;
+  float* dst;
+  float inv = 1.f;
+  if (sg.whole) {
+    dst = p.A + (hd * p.rows_total + r) * kD;
+    inv = 1.0f / l;
+  } else {
+    const int64_t prow = (static_cast<int64_t>(c) * 2 + sg.slot) * kTcUnitRows + t * kTcRows + row;
+    dst = p.ws_acc + prow * kD;
+    if (r < p.rows_total) {
+      p.ws_ml[prow * 2] = m;
+      p.ws_ml[prow * 2 + 1] = l;
+    }
+  }
+#pragma unroll
+  for (int cb = 0; cb < kD; cb += 16) {
+    uint32_t v[16];
+    NECTAR_TMEM_LD16(tO + cb, v);
+    tmem_ld_wait();
+    if (ok && r < p.rows_total) {
+#pragma unroll
+      for (int e = 0; e < 16; e += 4) {
+        float4 o = make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
+                               __uint_as_float(v[e + 3]));
+        if (split) {
+          const float4 o1 = xo[((cb + e) >> 2) ^ (row & 31)];
+          o = make_float4(w0 * o.x + w1 * o1.x, w0 * o.y + w1 * o1.y, w0 * o.z + w1 * o1.z, w0 * o.w + w1 * o1.w);
+        }
+        *reinterpret_cast<float4*>(dst + cb + e) = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+      }
+    }
+  }
+  if (sg.whole && ok && r < p.rows_total) p.alpha[hd * p.rows_total + r] = (m + log2f(l)) * kLn2;
+  tc_fence_before();
+  mbar_arrive(b_ofree_t);
+  if (split) named_bar_sync(1, 2 * kTcRows);   // done with the parked state
+}
+
+// The split instance out of line: inlined, its hand-off makes the softmax
+// loop spill; the other instance inlines it with no spill.
+__device__ __noinline__ void tc_unit_epilogue_split(const TcParams& p, uint8_t* smem, uint32_t tO, uint32_t b_ofree_t,
+                                                    const TcSeg& sg, bool split, int t, int row, float m, float l,
+                                                    bool ok, int c) {
+  tc_unit_epilogue<true>(p, smem, tO, b_ofree_t, sg, split, t, row, m, l, ok, c);
+}
+
+// kSplit: units with one query tile split their keys between the two
+// softmax warpgroups (compiled only into the instance used when every unit
+// has one query tile: the hand-off costs registers)
+template <bool kSplit>
 __global__ void __launch_bounds__(kTcThreads, 1)
 cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const TcParams p) {
@@ -184,7 +322,8 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
           tma_load_4d(smem_u32(smem + TcSmem::q + kQBytes), &tmap_q, 0, qp * kTcUnitRows + kTcRows, 0,
                       static_cast<int>(hd), b_qfull, pol_q);
         ++qn;
-        for (int64_t kt = sg.k0; kt < sg.k1; ++kt, ++it) {
+        for (int64_t i = 0; i < sg.k1 - sg.k0; ++i, ++it) {
+          const int64_t kt = tc_item<kSplit>(sg, two, i).kt;
           const uint32_t s = it % kTcStages;
           if (it >= kTcStages && !(ok = mbar_wait(b_kempty + 8 * s, ((it / kTcStages) - 1) & 1, p.err))) break;
           mbar_arrive_expect_tx(b_kfull + 8 * s, kKVBytes);
@@ -203,7 +342,9 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
       for (int si = 0; si < nseg && ok; ++si) {
         const TcSeg sg = tc_seg(p, c, si);
         const int64_t hd = sg.unit / p.qpairs;
-        for (int64_t kt = sg.k0; kt < sg.k1; ++kt, ++it) {
+        const bool two = two_tiles(sg.unit);
+        for (int64_t i = 0; i < sg.k1 - sg.k0; ++i, ++it) {
+          const int64_t kt = tc_item<kSplit>(sg, two, i).kt;
           const uint32_t s = it % kTcStages;
           if (it >= kTcStages && !(ok = mbar_wait(b_vempty + 8 * s, ((it / kTcStages) - 1) & 1, p.err))) break;
           mbar_arrive_expect_tx(b_vfull + 8 * s, kKVBytes);
@@ -222,11 +363,12 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
       uint32_t cs[2] = {0, 0};   // S tiles issued per query tile
       uint32_t cp[2] = {0, 0};   // P V products issued per query tile
       uint32_t un[2] = {0, 0};   // units whose O was started, per query tile
-      // O_t += P_t V for key tile `vit` (the ring index of its V)
-      auto issue_pv = [&](uint32_t vit, bool two, bool first) {
+      // O_t += P_t V for the ring entry `vit`, for every warpgroup t in mask
+      auto issue_pv = [&](uint32_t vit, uint32_t mask, bool first) {
         const uint32_t vs = vit % kTcStages;
         if (ok) ok = mbar_wait(b_vfull + 8 * vs, (vit / kTcStages) & 1, p.err);
-        for (int t = 0; t < (two ? 2 : 1); ++t) {
+        for (int t = 0; t < 2; ++t) {
+          if (!(mask >> t & 1u)) continue;
           const uint32_t b = cp[t] & 1;
           if (ok) ok = mbar_wait(b_pfull + 8 * (2 * t + b), (cp[t] >> 1) & 1, p.err);
           if (ok && first && un[t] > 0) ok = mbar_wait(b_ofree + 8 * t, (un[t] - 1) & 1, p.err);
@@ -248,20 +390,25 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         }
         mma_commit(b_vempty + 8 * vs);
       };
-      bool prev_two = false, prev_first = false, have_prev = false;
+      uint32_t prev_mask = 0;
+      bool prev_first = false, have_prev = false;
       for (int si = 0; si < nseg && ok; ++si) {
         const TcSeg sg = tc_seg(p, c, si);
         const bool two = two_tiles(sg.unit);
         ok = mbar_wait(b_qfull, qn & 1, p.err);
         ++qn;
-        for (int64_t kt = sg.k0; kt < sg.k1 && ok; ++kt, ++it) {
+        const int64_t nit = sg.k1 - sg.k0;
+        for (int64_t i = 0; i < nit && ok; ++i, ++it) {
+          const TcItem itm = tc_item<kSplit>(sg, two, i);
           const uint32_t ks = it % kTcStages;
           if (!(ok = mbar_wait(b_kfull + 8 * ks, (it / kTcStages) & 1, p.err))) break;
-          for (int t = 0; t < (two ? 2 : 1) && ok; ++t) {
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (!(itm.mask >> t & 1u)) continue;
             const uint32_t b = cs[t] & 1;
             if (cs[t] >= 2 && !(ok = mbar_wait(b_sfree + 8 * (2 * t + b), ((cs[t] >> 1) - 1) & 1, p.err))) break;
             tc_fence_after();
-            const uint32_t qa = smem_u32(smem + TcSmem::q + t * kQBytes);
+            // one query tile (split or not): both warpgroups read tile 0
+            const uint32_t qa = smem_u32(smem + TcSmem::q + (two ? t : 0) * kQBytes);
             const uint32_t kb = smem_u32(smem + TcSmem::k + ks * kKVBytes);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
@@ -274,14 +421,14 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
             ++cs[t];
           }
           mma_commit(b_kempty + 8 * ks);
-          if (kt + 1 == sg.k1) mma_commit(b_qempty);
-          if (have_prev) issue_pv(it - 1, prev_two, prev_first);
-          prev_two = two;
-          prev_first = (kt == sg.k0);
+          if (i + 1 == nit) mma_commit(b_qempty);
+          if (have_prev) issue_pv(it - 1, prev_mask, prev_first);
+          prev_mask = itm.mask;
+          prev_first = itm.first;
           have_prev = true;
         }
       }
-      if (ok && have_prev) issue_pv(it - 1, prev_two, prev_first);
+      if (ok && have_prev) issue_pv(it - 1, prev_mask, prev_first);
     }
   } else {
     // --------------------- softmax + epilogue (tile t) ---------------------
@@ -293,12 +440,18 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
     uint32_t cnt = 0;   // S tiles consumed by this tile
     for (int si = 0; si < nseg; ++si) {
       const TcSeg sg = tc_seg(p, c, si);
-      if (t == 1 && !two_tiles(sg.unit)) continue;
+      const bool two = two_tiles(sg.unit);
+      const bool split = tc_split<kSplit>(sg, two);
+      if (t == 1 && !two && !split) continue;
       float m = -INFINITY, l = 0.f;
-      for (int64_t kt = sg.k0; kt < sg.k1; ++kt, ++cnt) {
-        const uint32_t b = cnt & 1;
+      for (int64_t i = 0; i < sg.k1 - sg.k0; ++i) {
+        const TcItem itm = tc_item<kSplit>(sg, two, i);
+        if (!(itm.mask >> t & 1u)) continue;
+        const int64_t kt = itm.kt;
+        const uint32_t ci = cnt++;               // this warpgroup's S tiles so far
+        const uint32_t b = ci & 1;
         const int64_t nvalid = p.n - kt * kTcKeys;
-        if (ok) ok = mbar_wait(b_sfull + 8 * (2 * t + b), (cnt >> 1) & 1, p.err);
+        if (ok) ok = mbar_wait(b_sfull + 8 * (2 * t + b), (ci >> 1) & 1, p.err);
         tc_fence_after();
         // a whole tile of valid keys (every tile but a head's last): keep
         // the raw scores, take the max on them and fold the scale into the
@@ -317,27 +470,23 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         mbar_arrive(b_sfree + 8 * (2 * t + b));
         float bm = -INFINITY;
         if (full) {
-          // four independent chains (a 64-deep dependent chain would
-          // expose its latency on every tile)
-          float x0 = sc[0], x1 = sc[1], x2 = sc[2], x3 = sc[3];
+          // two independent chains (a 64-deep dependent chain would expose
+          // its latency on every tile)
+          float x0 = sc[0], x1 = sc[1];
           if (p.qmul >= 0.f) {
 #pragma unroll
-            for (int e = 4; e < kTcKeys; e += 4) {
+            for (int e = 2; e < kTcKeys; e += 2) {
               x0 = fmaxf(x0, sc[e]);
               x1 = fmaxf(x1, sc[e + 1]);
-              x2 = fmaxf(x2, sc[e + 2]);
-              x3 = fmaxf(x3, sc[e + 3]);
             }
-            bm = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)) * p.qmul;
+            bm = fmaxf(x0, x1) * p.qmul;
           } else {
 #pragma unroll
-            for (int e = 4; e < kTcKeys; e += 4) {
+            for (int e = 2; e < kTcKeys; e += 2) {
               x0 = fminf(x0, sc[e]);
               x1 = fminf(x1, sc[e + 1]);
-              x2 = fminf(x2, sc[e + 2]);
-              x3 = fminf(x3, sc[e + 3]);
             }
-            bm = fminf(fminf(x0, x1), fminf(x2, x3)) * p.qmul;
+            bm = fminf(x0, x1) * p.qmul;
           }
         } else {
 #pragma unroll
@@ -352,10 +501,10 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
           l *= corr;
           m = bm;
         }
-        if (__any_sync(0xffffffffu, need) && kt != sg.k0) {
+        if (__any_sync(0xffffffffu, need) && !itm.first) {
           // O_t holds the earlier key tiles of this unit: wait for their
           // last P V, then rescale it in TMEM (warp-collective)
-          const uint32_t pc = cnt - 1;
+          const uint32_t pc = ci - 1;
           if (ok) ok = mbar_wait(b_pvdone + 8 * (2 * t + (pc & 1)), (pc >> 1) & 1, p.err);
           tc_fence_after();
 #pragma unroll
@@ -369,8 +518,8 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
           }
           tmem_st_wait();
         }
-        // P buffer b was last read by the P V of this tile's S count cnt - 2
-        if (cnt >= 2 && ok) ok = mbar_wait(b_pvdone + 8 * (2 * t + b), ((cnt >> 1) - 1) & 1, p.err);
+        // P buffer b was last read by the P V of this warpgroup's S tile ci - 2
+        if (ci >= 2 && ok) ok = mbar_wait(b_pvdone + 8 * (2 * t + b), ((ci >> 1) - 1) & 1, p.err);
         uint8_t* pt = smem + TcSmem::p + (2 * t + b) * kPBytes;
         float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const float2 q2 = make_float2(p.qmul, p.qmul), nm2 = make_float2(-m, -m);
@@ -404,38 +553,13 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
       const uint32_t pc = cnt - 1;
       if (ok) ok = mbar_wait(b_pvdone + 8 * (2 * t + (pc & 1)), (pc >> 1) & 1, p.err);
       tc_fence_after();
-      const int64_t hd = sg.unit / p.qpairs;
-      const int64_t qp = sg.unit % p.qpairs;
-      const int64_t r = qp * kTcUnitRows + t * kTcRows + row;
-      float* dst;
-      float inv = 1.f;
-      if (sg.whole) {
-        dst = p.A + (hd * p.rows_total + r) * kD;
-        inv = 1.0f / l;
+      if constexpr (kSplit) {
+        tc_unit_epilogue_split(p, smem, tmem + 256 + 128 * t + lane_base, b_ofree + 8 * t, sg, split, t, row, m, l,
+                               ok, c);
       } else {
-        const int64_t prow = (static_cast<int64_t>(c) * 2 + sg.slot) * kTcUnitRows + t * kTcRows + row;
-        dst = p.ws_acc + prow * kD;
-        if (r < p.rows_total) {
-          p.ws_ml[prow * 2] = m;
-          p.ws_ml[prow * 2 + 1] = l;
-        }
+        tc_unit_epilogue<false>(p, smem, tmem + 256 + 128 * t + lane_base, b_ofree + 8 * t, sg, split, t, row, m, l,
+                                ok, c);
       }
-#pragma unroll
-      for (int cb = 0; cb < kD; cb += 32) {
-        uint32_t v[32];
-        NECTAR_TMEM_LD32(tO + lane_base + cb, v);
-        tmem_ld_wait();
-        if (ok && r < p.rows_total) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + cb + e) =
-                make_float4(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv,
-                            __uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv);
-        }
-      }
-      if (sg.whole && ok && r < p.rows_total) p.alpha[hd * p.rows_total + r] = (m + log2f(l)) * kLn2;
-      tc_fence_before();
-      mbar_arrive(b_ofree + 8 * t);
     }
   }
 
@@ -512,10 +636,15 @@ TcPlan plan_tc(int heads, int64_t n, int64_t rows, int num_sms) {
 cudaError_t launch_cache_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                  const TcParams& p, cudaStream_t stream) {
   const size_t smem = TcSmem::total + 1024;
-  cudaError_t e = cudaFuncSetAttribute(cache_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  // every unit has one query tile when a head has at most 128 rows
+  const bool split = p.rows_total <= kTcRows;
+  cudaError_t e = split ? cudaFuncSetAttribute(cache_attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem))
+                        : cudaFuncSetAttribute(cache_attn_tc_kernel<false>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  cache_attn_tc_kernel<<<p.C, kTcThreads, smem, stream>>>(tq, tk, tv, p);
+  if (split) cache_attn_tc_kernel<true><<<p.C, kTcThreads, smem, stream>>>(tq, tk, tv, p);
+  else cache_attn_tc_kernel<false><<<p.C, kTcThreads, smem, stream>>>(tq, tk, tv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (p.sk_units == 0) return cudaSuccess;

@@ -132,7 +132,9 @@ struct RowState {
 
   // Scores of KPG keys (log2 units, -inf for invalid keys), the lazy
   // rescale of the running state, and the keys' weights pw.
-  template <int KPG>
+  // kPaired: the dot products as paired f32x2 FMAs (even and odd dims in
+  // two accumulators) -- fewer instructions, two more registers per row.
+  template <int KPG, bool kPaired = false>
   __device__ __forceinline__ void weigh(const uint4 (&kw)[KPG][CPL], const bool* valid, float (&pw)[KPG][R]) {
     float sc[KPG][R];
 #pragma unroll
@@ -140,14 +142,33 @@ struct RowState {
       float part[R];
 #pragma unroll
       for (int r = 0; r < R; ++r) part[r] = 0.f;
+      if (kPaired) {
+        float2 part2[R];
 #pragma unroll
-      for (int ci = 0; ci < CPL; ++ci) {
-        float kf[8];
-        unpack8(kw[k][ci], kf);
+        for (int r = 0; r < R; ++r) part2[r] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int r = 0; r < R; ++r)
+        for (int ci = 0; ci < CPL; ++ci) {
+          float kf[8];
+          unpack8(kw[k][ci], kf);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) part[r] = fmaf(q[r][ci * 8 + e], kf[e], part[r]);
+          for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int e = 0; e < 8; e += 2)
+              part2[r] = ffma2(make_float2(q[r][ci * 8 + e], q[r][ci * 8 + e + 1]), make_float2(kf[e], kf[e + 1]),
+                               part2[r]);
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) part[r] = part2[r].x + part2[r].y;
+      } else {
+#pragma unroll
+        for (int ci = 0; ci < CPL; ++ci) {
+          float kf[8];
+          unpack8(kw[k][ci], kf);
+#pragma unroll
+          for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) part[r] = fmaf(q[r][ci * 8 + e], kf[e], part[r]);
+        }
       }
 #pragma unroll
       for (int off = LPK / 2; off >= 1; off >>= 1)
@@ -179,9 +200,9 @@ struct RowState {
       }
   }
 
-  // acc += pw * v over KPG value rows.  (Paired f32x2 FMAs here measured
-  // slower in the decode kernel: the accumulators are separate registers.)
-  template <int KPG>
+  // acc += pw * v over KPG value rows; kPaired as in weigh (it measured
+  // slower in the split decode kernel, whose 96-register cap then spills).
+  template <int KPG, bool kPaired = false>
   __device__ __forceinline__ void accumulate(const uint4 (&vw)[KPG][CPL], const float (&pw)[KPG][R]) {
 #pragma unroll
     for (int k = 0; k < KPG; ++k)
@@ -190,9 +211,21 @@ struct RowState {
         float vf[8];
         unpack8(vw[k][ci], vf);
 #pragma unroll
-        for (int r = 0; r < R; ++r)
+        for (int r = 0; r < R; ++r) {
+          if (kPaired) {
+            const float2 w2 = make_float2(pw[k][r], pw[k][r]);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[r][ci * 8 + e] = fmaf(pw[k][r], vf[e], acc[r][ci * 8 + e]);
+            for (int e = 0; e < 8; e += 2) {
+              const float2 a2 = ffma2(w2, make_float2(vf[e], vf[e + 1]),
+                                      make_float2(acc[r][ci * 8 + e], acc[r][ci * 8 + e + 1]));
+              acc[r][ci * 8 + e] = a2.x;
+              acc[r][ci * 8 + e + 1] = a2.y;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[r][ci * 8 + e] = fmaf(pw[k][r], vf[e], acc[r][ci * 8 + e]);
+          }
+        }
       }
   }
 

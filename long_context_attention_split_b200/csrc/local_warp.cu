@@ -24,6 +24,10 @@ namespace nectar {
 namespace {
 
 constexpr int kLWWarps = 4;
+#ifndef NECTAR_LW_PAIRED
+#define NECTAR_LW_PAIRED 1
+#endif
+constexpr bool kLWPaired = NECTAR_LW_PAIRED != 0;   // paired f32x2 FMAs (RowState)
 constexpr int kLWThreads = kLWWarps * 32;
 
 template <int RG>
@@ -83,12 +87,12 @@ __global__ void __launch_bounds__(kLWThreads, lw_min_blocks<RG>()) local_warp_ke
       for (int j0 = 0; j0 < nv; j0 += 2 * kStep) {
         if (j0 + kStep < nv) issue(1, j0 + kStep);
         float pw[KPG][RG];
-        st.template weigh<KPG>(kw[0], valid[0], pw);
-        st.template accumulate<KPG>(vw[0], pw);
+        st.template weigh<KPG, kLWPaired>(kw[0], valid[0], pw);
+        st.template accumulate<KPG, kLWPaired>(vw[0], pw);
         if (j0 + kStep >= nv) break;
         if (j0 + 2 * kStep < nv) issue(0, j0 + 2 * kStep);
-        st.template weigh<KPG>(kw[1], valid[1], pw);
-        st.template accumulate<KPG>(vw[1], pw);
+        st.template weigh<KPG, kLWPaired>(kw[1], valid[1], pw);
+        st.template accumulate<KPG, kLWPaired>(vw[1], pw);
       }
     }
     st.merge_groups();

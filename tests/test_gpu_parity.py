@@ -71,6 +71,10 @@ def run_cache_attn(L, Hkv, G, n, nq, seed=0, key_scale=None):
     (1, 2, 8, 128, 128),      # 1024 rows, n = one key tile: units whole in a CTA
     (1, 1, 4, 100, 32),       # n < one key tile
     (2, 2, 4, 8192, 128),     # 512 rows x 64 key tiles
+    # one query tile per unit: the key range split between the warpgroups
+    (1, 2, 4, 266, 16),       # 64 rows, 5 key tiles: halves of 3 and 2, ragged last tile
+    (2, 8, 4, 3000, 16),      # 64 rows, 16 heads: units cut into short segments between CTAs
+    (1, 1, 2, 64 * 2, 40),    # 80 rows, exactly two key tiles: one each
 ])
 def test_cache_attn_parity(L, Hkv, G, n, nq):
     wl, ag, Ag, ao, Ao = run_cache_attn(L, Hkv, G, n, nq, seed=n + G)
@@ -128,12 +132,15 @@ def test_cache_attn_tc_heavy_hitters_config3_shape():
                    A[0, h].reshape(1, -1, 128)[:, sel].cpu().numpy(), ao, Ao, wl.V.float().abs().max().item())
 
 
-def test_cache_attn_tc_running_max_moves():
+@pytest.mark.parametrize("nq", [64, 16])
+def test_cache_attn_tc_running_max_moves(nq):
     """A key deep in the cache that scores far above everything before it, for
     half of the query rows only: the running maximum moves by more than 2^8
-    inside a unit for some rows of a warp and not for others."""
+    inside a unit for some rows of a warp and not for others.  nq = 16 gives
+    64 rows per KV head, one query tile: the two softmax warpgroups take the
+    two halves of the keys, and the spike falls inside the second half."""
     g = torch.Generator().manual_seed(21)
-    L, Hkv, G, nq, n = 2, 2, 4, 64, 3000
+    L, Hkv, G, n = 2, 2, 4, 3000
     K = torch.randn(L, Hkv, n, 128, generator=g)
     V = torch.randn(L, Hkv, n, 128, generator=g).to(torch.bfloat16)
     Q = torch.randn(L, Hkv, G, nq, 128, generator=g)
