@@ -30,20 +30,29 @@ __host__ __device__ __forceinline__ int first_cta_of_tile(int64_t t, int64_t tot
   return static_cast<int>(((t + 1) * static_cast<int64_t>(C) - 1) / total);
 }
 
-template <int R>
+// RW: query rows held by one warp (R rows in NRG groups of RW).
+template <int RW>
 __host__ __device__ constexpr size_t dec_smem_bytes() {
-  return size_t(2) * kDecStages * kDecTile * kRowBytes      // K, V ring
-         + size_t(kDecWarps) * R * (kD + 2) * sizeof(float)  // cross-warp reduction
-         + 2 * kDecStages * sizeof(uint64_t);                // full / empty barriers
+  return size_t(2) * kDecStages * kDecTile * kRowBytes       // K, V ring
+         + size_t(kDecWarps) * RW * (kD + 2) * sizeof(float)  // cross-warp reduction
+         + 2 * kDecStages * sizeof(uint64_t);                 // full / empty barriers
 }
 
-// Two CTAs per SM for up to 2 rows (register cap 113), one otherwise.
-template <int R, int LPK>
-__global__ void __launch_bounds__(kDecThreads, (R <= 2 ? 2 : 1))
+// R query rows per CTA pass, in NRG row groups: the consumer warps form NRG
+// groups of kDecWarps / NRG, each group scores its RW = R / NRG rows against
+// every key of a tile (the group's warps split the keys).  A warp's registers
+// grow with RW, so 4 rows as 2 groups of 2 keep the 2-row register budget
+// and two CTAs per SM, at the cost of reading each tile from shared memory
+// twice.  Two CTAs per SM for up to 2 rows per warp (register cap 113).
+template <int R, int LPK, int NRG>
+__global__ void __launch_bounds__(kDecThreads, (R / NRG <= 2 ? 2 : 1))
 cache_attn_split_kernel(const DecParams p) {
-  using St = RowState<R, LPK>;
+  constexpr int RW = R / NRG;
+  constexpr int WPG = kDecWarps / NRG;       // warps per row group
+  static_assert(RW * NRG == R && WPG * NRG == kDecWarps, "row groups");
+  using St = RowState<RW, LPK>;
   constexpr int NG = St::NG;
-  constexpr int KPW = kDecTile / kDecWarps;  // keys per warp per tile
+  constexpr int KPW = kDecTile / WPG;        // keys per warp per tile
   constexpr int KPG = KPW / NG;              // keys per group per tile
   static_assert(KPG >= 1, "tile too small");
 
@@ -51,7 +60,7 @@ cache_attn_split_kernel(const DecParams p) {
   uint8_t* sK = smem;
   uint8_t* sV = smem + kDecStages * kDecTile * kRowBytes;
   float* sRed = reinterpret_cast<float*>(smem + 2 * kDecStages * kDecTile * kRowBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sRed + kDecWarps * R * (kD + 2));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sRed + kDecWarps * RW * (kD + 2));
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kDecStages);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -92,6 +101,10 @@ cache_attn_split_kernel(const DecParams p) {
 
   // ---------------- consumers ----------------
   const int g = lane / LPK, t = lane % LPK;
+  const int rg = warp / WPG, wk = warp % WPG;   // row group, warp within it
+  // rows of this pass (the last pass of a head may have fewer than R)
+  const int rows_here = static_cast<int>((p.rows_total - p.row0 < R) ? (p.rows_total - p.row0) : R);
+  const int nr_w = (rows_here - rg * RW < RW) ? (rows_here - rg * RW) : RW;   // may be <= 0
   St st;
   int64_t cur = -1;
   bool ok = true;
@@ -99,9 +112,9 @@ cache_attn_split_kernel(const DecParams p) {
   auto finalize = [&](int64_t hd) {
     st.merge_groups();
     if (g == 0) {
-      float* dst = sRed + (warp * R) * (kD + 2);
+      float* dst = sRed + (warp * RW) * (kD + 2);
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
+      for (int r = 0; r < RW; ++r) {
 #pragma unroll
         for (int ci = 0; ci < St::CPL; ++ci)
 #pragma unroll
@@ -114,15 +127,16 @@ cache_attn_split_kernel(const DecParams p) {
     }
     named_bar_sync(1, kDecWarps * 32);
     const int slot = c - first_cta_of_tile(hd * p.tph, p.total, p.C);
-    for (int it = threadIdx.x; it < R * kD; it += kDecWarps * 32) {
+    for (int it = threadIdx.x; it < (NRG == 1 ? R : rows_here) * kD; it += kDecWarps * 32) {
       const int r = it / kD, dim = it % kD;
+      const int wg0 = (r / RW) * WPG, rr = r % RW;   // the row's group: warps wg0 .. wg0 + WPG - 1
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sRed[(w * R + r) * (kD + 2) + kD]);
+      for (int w = 0; w < WPG; ++w) M = fmaxf(M, sRed[((wg0 + w) * RW + rr) * (kD + 2) + kD]);
       float ls = 0.f, as = 0.f;
 #pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) {
-        const float* src = sRed + (w * R + r) * (kD + 2);
+      for (int w = 0; w < WPG; ++w) {
+        const float* src = sRed + ((wg0 + w) * RW + rr) * (kD + 2);
         const float wgt = exp2_shift(src[kD], M);
         ls = fmaf(src[kD + 1], wgt, ls);
         as = fmaf(src[dim], wgt, as);
@@ -144,7 +158,8 @@ cache_attn_split_kernel(const DecParams p) {
       if (cur >= 0) finalize(cur);
       cur = hd;
       st.reset();
-      st.load_q(p.Q + (hd * p.rows_total + p.row0) * kD, kD, R, t, p.qmul);
+      if constexpr (NRG == 1) st.load_q(p.Q + (hd * p.rows_total + p.row0) * kD, kD, R, t, p.qmul);
+      else st.load_q(p.Q + (hd * p.rows_total + p.row0 + rg * RW) * kD, kD, nr_w, t, p.qmul);
     }
     const int s = static_cast<int>(i % kDecStages);
     if (ok) ok = mbar_wait(full0 + 8 * s, static_cast<uint32_t>((i / kDecStages) & 1), p.err);
@@ -153,17 +168,36 @@ cache_attn_split_kernel(const DecParams p) {
       const int cnt = static_cast<int>((p.n - j0 < kDecTile) ? (p.n - j0) : kDecTile);
       const uint8_t* kt = sK + s * kDecTile * kRowBytes;
       const uint8_t* vt = sV + s * kDecTile * kRowBytes;
-      const uint8_t* kr[KPG];
-      const uint8_t* vr[KPG];
-      bool valid[KPG];
+      if constexpr (NRG == 1) {
+        const uint8_t* kr[KPG];
+        const uint8_t* vr[KPG];
+        bool valid[KPG];
 #pragma unroll
-      for (int k = 0; k < KPG; ++k) {
-        const int key = warp * KPW + k * NG + g;
-        valid[k] = key < cnt;
-        kr[k] = kt + key * kRowBytes;
-        vr[k] = vt + key * kRowBytes;
+        for (int k = 0; k < KPG; ++k) {
+          const int key = warp * KPW + k * NG + g;
+          valid[k] = key < cnt;
+          kr[k] = kt + key * kRowBytes;
+          vr[k] = vt + key * kRowBytes;
+        }
+        st.template step<KPG>(kr, vr, valid, t, SmemLoader{});
+      } else {
+        // the warp's KPG keys per lane group, at most 2 per step (registers)
+        constexpr int KS = KPG > 2 ? 2 : KPG;
+#pragma unroll
+        for (int k0 = 0; k0 < KPG; k0 += KS) {
+          const uint8_t* kr[KS];
+          const uint8_t* vr[KS];
+          bool valid[KS];
+#pragma unroll
+          for (int k = 0; k < KS; ++k) {
+            const int key = wk * KPW + (k0 + k) * NG + g;
+            valid[k] = key < cnt;
+            kr[k] = kt + key * kRowBytes;
+            vr[k] = vt + key * kRowBytes;
+          }
+          st.template step<KS>(kr, vr, valid, t, SmemLoader{});
+        }
       }
-      st.template step<KPG>(kr, vr, valid, t, SmemLoader{});
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * s);
@@ -210,27 +244,27 @@ __global__ void cache_attn_combine_kernel(const DecParams p, float* __restrict__
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-template <int R, int LPK>
+template <int R, int LPK, int NRG>
 static cudaError_t launch_split(const DecParams& p, cudaStream_t stream) {
-  const size_t smem = dec_smem_bytes<R>();
-  cudaError_t e = cudaFuncSetAttribute(cache_attn_split_kernel<R, LPK>,
+  const size_t smem = dec_smem_bytes<R / NRG>();
+  cudaError_t e = cudaFuncSetAttribute(cache_attn_split_kernel<R, LPK, NRG>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  cache_attn_split_kernel<R, LPK><<<p.C, kDecThreads, smem, stream>>>(p);
+  cache_attn_split_kernel<R, LPK, NRG><<<p.C, kDecThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
 int dec_max_rows() { return 8; }
 
 // Resident CTAs per SM of the split kernel for R rows (occupancy calculator).
-template <int R, int LPK>
+template <int R, int LPK, int NRG>
 static int occ_t() {
-  const size_t smem = dec_smem_bytes<R>();
-  if (cudaFuncSetAttribute(cache_attn_split_kernel<R, LPK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const size_t smem = dec_smem_bytes<R / NRG>();
+  if (cudaFuncSetAttribute(cache_attn_split_kernel<R, LPK, NRG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, cache_attn_split_kernel<R, LPK>, kDecThreads, smem) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, cache_attn_split_kernel<R, LPK, NRG>, kDecThreads, smem) !=
       cudaSuccess)
     return 1;
   return n < 1 ? 1 : n;
@@ -238,14 +272,14 @@ static int occ_t() {
 
 int dec_ctas_per_sm(int R) {
   switch (R) {
-    case 1: return occ_t<1, 8>();
-    case 2: return occ_t<2, 8>();
-    case 3: return occ_t<3, 8>();
-    case 4: return occ_t<4, 8>();
-    case 5: return occ_t<5, 16>();
-    case 6: return occ_t<6, 16>();
-    case 7: return occ_t<7, 16>();
-    default: return occ_t<8, 16>();
+    case 1: return occ_t<1, 8, 1>();
+    case 2: return occ_t<2, 8, 1>();
+    case 3:
+    case 4: return occ_t<4, 8, 2>();
+    case 5: return occ_t<5, 16, 1>();
+    case 6: return occ_t<6, 16, 1>();
+    case 7: return occ_t<7, 16, 1>();
+    default: return occ_t<8, 16, 1>();
   }
 }
 
@@ -253,8 +287,8 @@ size_t dec_smem_for_rows(int R) {
   switch (R) {
     case 1: return dec_smem_bytes<1>();
     case 2: return dec_smem_bytes<2>();
-    case 3: return dec_smem_bytes<3>();
-    case 4: return dec_smem_bytes<4>();
+    case 3:
+    case 4: return dec_smem_bytes<2>();
     case 5: return dec_smem_bytes<5>();
     case 6: return dec_smem_bytes<6>();
     case 7: return dec_smem_bytes<7>();
@@ -284,14 +318,14 @@ DecPlan plan_decode(int heads, int64_t n, int num_sms, int ctas_per_sm) {
 
 cudaError_t launch_cache_attn_split(const DecParams& p, int R, cudaStream_t stream) {
   switch (R) {
-    case 1: return launch_split<1, 8>(p, stream);
-    case 2: return launch_split<2, 8>(p, stream);
-    case 3: return launch_split<3, 8>(p, stream);
-    case 4: return launch_split<4, 8>(p, stream);
-    case 5: return launch_split<5, 16>(p, stream);
-    case 6: return launch_split<6, 16>(p, stream);
-    case 7: return launch_split<7, 16>(p, stream);
-    case 8: return launch_split<8, 16>(p, stream);
+    case 1: return launch_split<1, 8, 1>(p, stream);
+    case 2: return launch_split<2, 8, 1>(p, stream);
+    case 3:   // 3 rows run as 4, the last one empty
+    case 4: return launch_split<4, 8, 2>(p, stream);
+    case 5: return launch_split<5, 16, 1>(p, stream);
+    case 6: return launch_split<6, 16, 1>(p, stream);
+    case 7: return launch_split<7, 16, 1>(p, stream);
+    case 8: return launch_split<8, 16, 1>(p, stream);
     default: return cudaErrorInvalidValue;
   }
 }

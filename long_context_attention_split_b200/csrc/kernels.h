@@ -118,7 +118,10 @@ struct ModParams {
 // Layer-by-layer grouped GEMM path of the module forward (module_gemm.cu),
 // used when a KV head has at least kGemmMinRows query rows.
 constexpr int kGemmMaxStages = 8;
-constexpr int kGemmMinRows = 128;
+#ifndef NECTAR_GEMM_MIN_ROWS
+#define NECTAR_GEMM_MIN_ROWS 128
+#endif
+constexpr int kGemmMinRows = NECTAR_GEMM_MIN_ROWS;
 struct GemmParams {
   int L, Hkv, depth, stage, readout, nlayers;
   int R, NR, rtiles, Hp, MT, stages, tmem_cols;
