@@ -187,7 +187,7 @@ NECTAR_API nectar_status nectar_module_pack(nectar_dims dims, int32_t depth, con
  * by the caller, overwritten; NECTAR_ERR_WORKSPACE when missing or small).
  * ------------------------------------------------------------------------ */
 /* Workspace of nectar_module_forward, in bytes: 0 when the KV heads have
- * fewer than 128 query rows (G * nq), else the hidden activations of the
+ * fewer than 64 query rows (G * nq), else the hidden activations of the
  * layer-by-layer path, (depth >= 2 ? 2 : 1) * align256(2 * rows * Hp * 2)
  * + align256(rows * ceil(Hmax / 128) * 4), with rows = L * Hkv * G * nq,
  * Hmax the widest layer and Hp = Hmax rounded up to 64. */
@@ -232,7 +232,7 @@ NECTAR_API nectar_status nectar_merge_local(nectar_dims dims, const float *a, co
  * and nectar_merge_local; out DEVICE fp32 [L][Hkv][G][nq][d].  Equal (up to
  * rounding order) to nectar_module_forward followed by nectar_merge_local.
  *
- * Fewer than 128 query rows per KV head: one launch whose CTAs run the
+ * Fewer than 64 query rows per KV head: one launch whose CTAs run the
  * module forward (writing A_theta into out) side by side with CTAs that
  * compute each row's local attention state, then a small merge that
  * rewrites out in place.  More rows: the local states first, then the
@@ -241,7 +241,7 @@ NECTAR_API nectar_status nectar_merge_local(nectar_dims dims, const float *a, co
  *   workspace  DEVICE scratch, 256-byte aligned, of at least
  *              nectar_decode_workspace_size(dims, mods, nq) bytes: the
  *              local state of every row, rows * (d + 2) * 4 with
- *              rows = L * Hkv * G * nq, plus rows * 4 (fewer than 128 query
+ *              rows = L * Hkv * G * nq, plus rows * 4 (fewer than 64 query
  *              rows per KV head) or nectar_module_workspace_size (else);
  *              owned by the caller, overwritten, must not be used by
  *              another call in flight.

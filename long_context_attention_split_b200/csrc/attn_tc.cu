@@ -522,27 +522,36 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         if (ci >= 2 && ok) ok = mbar_wait(b_pvdone + 8 * (2 * t + b), ((ci >> 1) - 1) & 1, p.err);
         uint8_t* pt = smem + TcSmem::p + (2 * t + b) * kPBytes;
         float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        const float2 q2 = make_float2(p.qmul, p.qmul), nm2 = make_float2(-m, -m);
+        // the row sum adds the rounded weights that P V uses; full tiles and
+        // the last (masked) tile in separate loops, so that the unrolled
+        // loop body carries no per-pair branch
+        if (full) {
+          const float2 q2 = make_float2(p.qmul, p.qmul), nm2 = make_float2(-m, -m);
 #pragma unroll
-        for (int c8 = 0; c8 < kTcKeys / 8; ++c8) {
-          uint32_t w[4];
+          for (int c8 = 0; c8 < kTcKeys / 8; ++c8) {
+            uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float s0 = sc[c8 * 8 + 2 * e], s1 = sc[c8 * 8 + 2 * e + 1];
-            if (full) {
+            for (int e = 0; e < 4; ++e) {
               // 2^(s * scale * log2 e - m) for two keys: one paired FMA; the
-              // last kTcPolyPairs of every 4 pairs take the polynomial exp2 so
-              // the special-function unit is not the limit
-              const float2 x = ffma2(make_float2(s0, s1), q2, nm2);
+              // last kTcPolyPairs of every 4 pairs take the polynomial exp2
+              const float2 x = ffma2(make_float2(sc[c8 * 8 + 2 * e], sc[c8 * 8 + 2 * e + 1]), q2, nm2);
               if (e >= 4 - kTcPolyPairs) w[e] = pack_bf16x2(exp2_poly(x.x), exp2_poly(x.y));
               else w[e] = pack_bf16x2(ex2(x.x), ex2(x.y));
-            } else {
-              w[e] = pack_bf16x2(exp2_shift(s0, m), exp2_shift(s1, m));
+              rs2[e & 1] = fadd2(rs2[e & 1], make_float2(bf16lo(w[e]), bf16hi(w[e])));
             }
-            // the row sum adds the rounded weights that P V uses
-            rs2[e & 1] = fadd2(rs2[e & 1], make_float2(bf16lo(w[e]), bf16hi(w[e])));
+            *reinterpret_cast<uint4*>(pt + p_off(row, c8 * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
-          *reinterpret_cast<uint4*>(pt + p_off(row, c8 * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+#pragma unroll
+          for (int c8 = 0; c8 < kTcKeys / 8; ++c8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              w[e] = pack_bf16x2(exp2_shift(sc[c8 * 8 + 2 * e], m), exp2_shift(sc[c8 * 8 + 2 * e + 1], m));
+              rs2[e & 1] = fadd2(rs2[e & 1], make_float2(bf16lo(w[e]), bf16hi(w[e])));
+            }
+            *reinterpret_cast<uint4*>(pt + p_off(row, c8 * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
         l += (rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y);
         fence_proxy_async_smem();

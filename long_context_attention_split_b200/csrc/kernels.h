@@ -119,7 +119,7 @@ struct ModParams {
 // used when a KV head has at least kGemmMinRows query rows.
 constexpr int kGemmMaxStages = 8;
 #ifndef NECTAR_GEMM_MIN_ROWS
-#define NECTAR_GEMM_MIN_ROWS 128
+#define NECTAR_GEMM_MIN_ROWS 64
 #endif
 constexpr int kGemmMinRows = NECTAR_GEMM_MIN_ROWS;
 struct GemmParams {
@@ -142,7 +142,7 @@ struct GemmShape {
   int NR, rtiles, stages, tmem_cols;
   size_t smem;
 };
-GemmShape gemm_shape(int64_t R);
+GemmShape gemm_shape(int64_t R, int max_rows);
 cudaError_t launch_module_gemm(const CUtensorMap& tq, const CUtensorMap& th, const GemmParams& p, int grid,
                                size_t smem, cudaStream_t stream);
 cudaError_t launch_local_state(const ModParams& p, cudaStream_t stream);

@@ -350,9 +350,12 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-GemmShape gemm_shape(int64_t R) {
+// max_rows: rows per tile at most (256 for the hidden layers; the readout
+// uses smaller tiles -- it has one M tile per head, and its merge epilogue
+// per row is long -- so that all SMs get work)
+GemmShape gemm_shape(int64_t R, int max_rows) {
   GemmShape sh{};
-  sh.rtiles = static_cast<int>((R + 255) / 256);
+  sh.rtiles = static_cast<int>((R + max_rows - 1) / max_rows);
   const int64_t per = (R + sh.rtiles - 1) / sh.rtiles;
   sh.NR = static_cast<int>((per + 15) / 16 * 16);
   constexpr size_t kBudget = 227 * 1024;

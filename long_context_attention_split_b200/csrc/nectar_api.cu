@@ -575,7 +575,8 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
   const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
   const int64_t R = static_cast<int64_t>(dims.G) * nq;
   if (heads * R * 2 > 0x7fffffffLL) return fail(NECTAR_ERR_UNSUPPORTED, "too many query rows for one call");
-  const GemmShape sh = gemm_shape(R);
+  const GemmShape sh = gemm_shape(R, 256);
+  const GemmShape shr = gemm_shape(R, 64);     // readout tiles
   GemmParams g;
   memset(&g, 0, sizeof(g));
   g.L = dims.L;
@@ -601,7 +602,7 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
   __nv_bfloat16* hbuf[2] = {reinterpret_cast<__nv_bfloat16*>(base),
                             reinterpret_cast<__nv_bfloat16*>(base + (mp.depth >= 2 ? hb : 0))};
   g.part = reinterpret_cast<float*>(base + (mp.depth >= 2 ? 2 : 1) * hb);
-  CUtensorMap tq, th[2];
+  CUtensorMap tq, th[2], thr;
   {
     const cuuint64_t dq[2] = {128, static_cast<cuuint64_t>(heads * R)};
     const cuuint64_t sq[1] = {256};
@@ -612,6 +613,11 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
       const cuuint64_t shs[1] = {static_cast<cuuint64_t>(g.Hp) * 2};
       NECTAR_TRY(make_tmap(&th[b], hbuf[b], 2, dh, shs, bq, "hidden activations"));
     }
+    // the readout reads the last hidden layer in its own, smaller row tiles
+    const cuuint64_t dh[2] = {static_cast<cuuint64_t>(g.Hp), static_cast<cuuint64_t>(2 * heads * R)};
+    const cuuint64_t shs[1] = {static_cast<cuuint64_t>(g.Hp) * 2};
+    const cuuint32_t br[2] = {64, static_cast<cuuint32_t>(shr.NR)};
+    NECTAR_TRY(make_tmap(&thr, hbuf[(mp.depth - 1) & 1], 2, dh, shs, br, "hidden activations (readout)"));
   }
   for (int stage = 0; stage <= mp.depth; ++stage) {
     g.stage = stage;
@@ -620,18 +626,23 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
     g.a_out = g.readout ? a : nullptr;
     g.A_out = g.readout ? A_out : nullptr;
     g.ws_loc = g.readout ? ws_loc : nullptr;
+    const GemmShape& ss = g.readout ? shr : sh;
+    g.NR = ss.NR;
+    g.rtiles = ss.rtiles;
+    g.stages = ss.stages;
+    g.tmem_cols = ss.tmem_cols;
     int64_t acc = 0;
     for (int li = 0; li < dims.L; ++li) {
       g.tile_start[li] = acc;
       const int H = mp.width[mp.order[li]];
       const int mt = g.readout ? 1 : (H + 127) / 128;
-      acc += static_cast<int64_t>(dims.Hkv) * (g.readout ? 1 : 2) * mt * sh.rtiles;
+      acc += static_cast<int64_t>(dims.Hkv) * (g.readout ? 1 : 2) * mt * ss.rtiles;
     }
     g.tile_start[dims.L] = acc;
     g.ntiles = acc;
     const int grid = static_cast<int>(acc < di.sms ? acc : di.sms);
-    const CUtensorMap& tin = stage == 0 ? tq : th[(stage - 1) & 1];
-    cudaError_t e = launch_module_gemm(tq, tin, g, grid, sh.smem, st);
+    const CUtensorMap& tin = g.readout ? thr : (stage == 0 ? tq : th[(stage - 1) & 1]);
+    cudaError_t e = launch_module_gemm(tq, tin, g, grid, ss.smem, st);
     if (e != cudaSuccess) return cuda_fail(e, "module GEMM kernel");
   }
   return NECTAR_OK;

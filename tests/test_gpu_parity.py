@@ -345,11 +345,13 @@ def test_module_forward_toy():
     dict(L=3, Hkv=1, G=4, nq=20, widths=[16, 1024, 144], depth=2),
     dict(L=1, Hkv=2, G=1, nq=33, widths=[64], depth=1),
     dict(L=1, Hkv=1, G=3, nq=7, widths=[128], depth=3),
-    # >= 128 rows per KV head: the layer-by-layer grouped-GEMM path
+    # >= 64 rows per KV head: the layer-by-layer grouped-GEMM path
     dict(L=2, Hkv=2, G=7, nq=40, widths=[208, 96], depth=2),    # 280 rows: two ragged row tiles
     dict(L=3, Hkv=1, G=4, nq=300, widths=[16, 1024, 144], depth=3),   # 1200 rows, 5 row tiles
     dict(L=1, Hkv=2, G=1, nq=130, widths=[64], depth=1),        # depth 1: readout straight from h_0
-    dict(L=1, Hkv=1, G=2, nq=64, widths=[512], depth=2),        # exactly 128 rows
+    dict(L=1, Hkv=1, G=2, nq=64, widths=[512], depth=2),        # 128 rows
+    dict(L=1, Hkv=2, G=4, nq=16, widths=[256], depth=2),        # exactly 64 rows: the first grouped-GEMM size
+    dict(L=1, Hkv=1, G=7, nq=9, widths=[144], depth=2),         # 63 rows: still one CTA per block of tokens
 ])
 def test_module_forward_shapes(kw):
     kw = dict(kw)
@@ -399,6 +401,7 @@ def test_decode_toy_prefill():
     dict(L=1, Hkv=1, G=12, n=16, B=4, T=45, widths=[128]),     # two local jobs per token (8 + 4 heads)
     dict(L=2, Hkv=2, G=4, n=16, B=40, T=50, widths=[256, 512]),   # 160 rows per KV head: GEMM path
     dict(L=1, Hkv=2, G=7, n=16, B=64, T=33, widths=[768]),     # 448 rows: two row tiles of 224
+    dict(L=2, Hkv=2, G=4, n=16, B=16, T=40, widths=[256, 128]),   # exactly 64 rows: grouped-GEMM decode
 ])
 def test_decode_shapes(kw):
     wl = make_workload("qwen3_1p7b", seed=2, key_scale=None, **kw)
@@ -413,7 +416,7 @@ def test_decode_workspace_checked():
     args = (cuda(wl.Q), cuda(wl.q_seq), cuda(wl.q_pos), cuda(wl.Kloc), cuda(wl.Vloc), cuda(wl.local_len))
     need = nx.decode_workspace_size(mods, wl.G, wl.nq)
     loc = (wl.heads * wl.rows * 130 * 4 + 255) // 256 * 256
-    if wl.rows < 128:
+    if wl.rows < 64:
         assert need == (wl.heads * wl.rows * 4 + 255) // 256 * 256 + loc
     else:
         assert need == loc + nx.module_workspace_size(mods, wl.G, wl.nq) > loc
