@@ -288,19 +288,24 @@ __device__ __forceinline__ void module_cta(const CUtensorMap* tmap_q, const ModP
                     bv = bvs[q];
                     wv = wvs[q];
                   }
+                uint32_t ws[8];
 #pragma unroll
                 for (int j = 0; j < 16; j += 2) {
                   // two rows rounded to bf16 by one packed conversion
                   const uint32_t w = pack_bf16x2(mod_silu(__uint_as_float(v[mm][j]) + bv),
                                                  mod_silu(__uint_as_float(v[mm][j + 1]) + bv));
-                  if (readout) {
-                    part[j] = fmaf(wv, bf16lo(w), part[j]);
-                    part[j + 1] = fmaf(wv, bf16hi(w), part[j + 1]);
-                  } else {
+                  part[j] = fmaf(wv, bf16lo(w), part[j]);          // wv = 0 outside the readout layer
+                  part[j + 1] = fmaf(wv, bf16hi(w), part[j + 1]);
+                  ws[j >> 1] = w;
+                }
+                if (!readout) {
+                  // h back into X (the readout layer's h is reduced, not stored)
+#pragma unroll
+                  for (int j = 0; j < 16; j += 2) {
                     *reinterpret_cast<uint16_t*>(smem + L.x + x_offset(N, n0 + j, kD + i)) =
-                        static_cast<uint16_t>(w & 0xFFFFu);
+                        static_cast<uint16_t>(ws[j >> 1] & 0xFFFFu);
                     *reinterpret_cast<uint16_t*>(smem + L.x + x_offset(N, n0 + j + 1, kD + i)) =
-                        static_cast<uint16_t>(w >> 16);
+                        static_cast<uint16_t>(ws[j >> 1] >> 16);
                   }
                 }
               }

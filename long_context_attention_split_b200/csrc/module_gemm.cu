@@ -304,21 +304,25 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
               if (q4 == 0 && p.a_out != nullptr) p.a_out[g.hd * R + r] = a_l;
             }
           }
+          const int nrow = rend - (r0 + n0);          // rows of this batch inside the tile
+          float* arow = p.A_out + (g.hd * R + r0 + n0) * kD + u;
+          if (p.ws_loc == nullptr) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int r = r0 + n0 + j;
-            const float aj = __shfl_sync(0xffffffffu, a_l, j);
-            if (r >= rend) continue;
-            const int64_t row = g.hd * R + r;
-            const float At = __uint_as_float(v[j]) + bias;
-            if (p.ws_loc == nullptr) {
-              p.A_out[row * kD + u] = At;
-            } else {
-              const float* st = p.ws_loc + row * (kD + 2);
-              const float ad = aj * kLog2e;
-              const float M = fmaxf(ad, st[kD]);
-              const float wd = exp2_shift(ad, M), wl = exp2_shift(st[kD], M);
-              p.A_out[row * kD + u] = (wd * At + wl * st[u]) / (wd + wl * st[kD + 1]);
+            for (int j = 0; j < 32; ++j)
+              if (j < nrow) arow[j * kD] = __uint_as_float(v[j]) + bias;
+          } else {
+            // merge with the row's local state (decode)
+            const float* st0 = p.ws_loc + (g.hd * R + r0 + n0) * (kD + 2);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float aj = __shfl_sync(0xffffffffu, a_l, j);
+              if (j < nrow) {
+                const float* st = st0 + j * (kD + 2);
+                const float ad = aj * kLog2e;
+                const float M = fmaxf(ad, st[kD]);
+                const float wd = exp2_shift(ad, M), wl = exp2_shift(st[kD], M);
+                arow[j * kD] = (wd * (__uint_as_float(v[j]) + bias) + wl * st[u]) / (wd + wl * st[kD + 1]);
+              }
             }
           }
         }
