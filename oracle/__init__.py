@@ -54,6 +54,7 @@ def _load():
                                               ctypes.c_double, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_fit_metrics.argtypes = [I, I, ctypes.c_int, P, P, P, P, P, P]
         _lib = lib
     return _lib
 
@@ -203,3 +204,26 @@ def full_attention(K, V, Q, q_seq, q_pos, Kloc, Vloc, local_len, scale: float):
     _load().oracle_full_attention(heads, n, rows, nq, d, _p(Kb), _p(Vb), _p(Qb), _p(qs), _p(qp),
                                   _p(Klb), _p(Vlb), B, T, _p(ll), float(scale), _p(out))
     return out
+
+
+def quadrature_forward(W, Z, Q, scale: float):
+    """Quadrature module of §2.4: a_theta(q) = log sum_j exp((W q)_j / sqrt d),
+    A_theta(q) = softmax(W q / sqrt d)^T Z, with W, Z [..., p, d] the learned
+    rows (initialised to the first p rows of K and V).  By its definition this
+    is the exact attention of Eq. (3.1) over (W, Z), computed as such."""
+    return cache_attn(W, Z, Q, scale)
+
+
+def fit_metrics(alpha, A, a, At, Q):
+    """Per (l, h) score MSE, target MSE (per element) and mean log error ratio
+    of Eq. (C.1) (App. C.4); returns [heads, 3] float64 and the RTE (the sum
+    of the last column).  alpha, a: [..., rows]; A, At: [..., rows, d];
+    Q: bf16 [..., rows, d]."""
+    al, aa = _f64(alpha), _f64(a)
+    Ad, At_ = _f64(A), _f64(At)
+    Qb = _bf16_bits(Q)
+    rows, d = Ad.shape[-2], Ad.shape[-1]
+    heads = int(np.prod(Ad.shape[:-2])) if Ad.ndim > 2 else 1
+    out = np.zeros((heads, 3), np.float64)
+    _load().oracle_fit_metrics(heads, rows, d, _p(al), _p(Ad), _p(aa), _p(At_), _p(Qb), _p(out))
+    return out, float(out[:, 2].sum())

@@ -247,6 +247,43 @@ void oracle_full_attention(int64_t heads, int64_t n, int64_t rows, int64_t nq, i
 }
 
 /* Threads OpenMP will use (for reporting the CPU baseline's core count). */
+/*
+ * Fitting metrics of a module against the exact targets, per (l, h)
+ * (notes §4 "score / target MSE"; App. C.4, Eq. (C.1)):
+ *   score_mse  = mean_q (a(q) - alpha(q))^2
+ *   target_mse = mean_q (1/d) sum_c (A_theta(q)_c - A(q)_c)^2
+ *   rte        = mean_q log( ||A_theta(q) - A(q)||^2 / ||q - A(q)||^2 )
+ * (the RTE of Eq. (C.1) is the sum of rte over (l, h)).  q is the bf16 query
+ * row as stored; the others are double.
+ *
+ * alpha, a: [heads][rows]   A, At: [heads][rows][d]   Q: [heads][rows][d] bf16
+ * out: [heads][3] = {score_mse, target_mse, rte}
+ */
+void oracle_fit_metrics(int64_t heads, int64_t rows, int d, const double *alpha, const double *A,
+                        const double *a, const double *At, const uint16_t *Q, double *out) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t hd = 0; hd < heads; ++hd) {
+        double s_sum = 0.0, t_sum = 0.0, r_sum = 0.0;
+        for (int64_t r = 0; r < rows; ++r) {
+            const int64_t it = hd * rows + r;
+            const double ds = a[it] - alpha[it];
+            s_sum += ds * ds;
+            double num = 0.0, den = 0.0;
+            for (int c = 0; c < d; ++c) {
+                const double e = At[it * d + c] - A[it * d + c];
+                const double b = bf16_to_double(Q[it * d + c]) - A[it * d + c];
+                num += e * e;
+                den += b * b;
+            }
+            t_sum += num / d;
+            r_sum += log(num / den);
+        }
+        out[hd * 3 + 0] = rows > 0 ? s_sum / rows : 0.0;
+        out[hd * 3 + 1] = rows > 0 ? t_sum / rows : 0.0;
+        out[hd * 3 + 2] = rows > 0 ? r_sum / rows : 0.0;
+    }
+}
+
 #ifdef _OPENMP
 #include <omp.h>
 int oracle_num_threads(void) { return omp_get_max_threads(); }

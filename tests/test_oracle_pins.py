@@ -393,3 +393,63 @@ def test_capacity_and_widths():
         total = sum(module_params_per_head(x) for x in w)
         assert abs(total / (rho * 2 * 65536 * 128 * 32) - 1) < 0.04
         assert w[0] > w[10] and w[0] == w[31] and w[4] == w[27]
+
+
+# ---------------------------------------------------------------------------
+# next rows: the Quadrature module (§2.4) and the fitting metrics (App. C.4)
+# ---------------------------------------------------------------------------
+def test_quadrature_is_attention_over_the_first_p_rows():
+    """§2.4: a_theta = log sum_j exp((W q)_j / sqrt d), A_theta = softmax(.)^T Z,
+    W, Z initialised to the first p rows of K, V -- brute force with fsum."""
+    g = torch.Generator().manual_seed(77)
+    n, p, d, rows = 12, 5, 6, 3
+    K, V, Q = rand_bf16(g, 2, n, d), rand_bf16(g, 2, n, d), rand_bf16(g, 2, rows, d)
+    W, Z = K[:, :p].contiguous(), V[:, :p].contiguous()
+    a, At = oracle.quadrature_forward(W, Z, Q, 1 / math.sqrt(d))
+    for h in range(2):
+        for r in range(rows):
+            ba, bA = brute_alpha_A(f64(Q[h, r]), f64(K[h, :p]), f64(V[h, :p]), 1 / math.sqrt(d))
+            assert abs(a[h, r] - ba) < 1e-12
+            assert np.abs(At[h, r] - bA).max() < 1e-12
+    # p = 1: the softmax has one term, A_theta = z_1, a_theta = w_1 . q / sqrt d
+    a1, At1 = oracle.quadrature_forward(K[:, :1].contiguous(), V[:, :1].contiguous(), Q, 1 / math.sqrt(d))
+    assert np.abs(At1 - f64(V[:, :1]).numpy()).max() == 0.0
+    s = (f64(Q) @ f64(K[:, :1]).transpose(1, 2)).squeeze(-1) / math.sqrt(d)
+    assert np.abs(a1 - s.numpy()).max() < 1e-12
+
+
+def test_fit_metrics_worked_example():
+    """d = 2, one row: A = (0, 0), A_theta = (3, 4), q = (1, 0), alpha = 1,
+    a = 3: score MSE 4, target MSE (9 + 16) / 2, RTE term log(25 / 1)."""
+    A = np.zeros((1, 1, 2))
+    At = np.array([[[3.0, 4.0]]])
+    Q = bf16([[[1.0, 0.0]]])
+    out, rte = oracle.fit_metrics(np.array([[1.0]]), A, np.array([[3.0]]), At, Q)
+    assert out[0, 0] == 4.0 and out[0, 1] == 12.5
+    assert abs(out[0, 2] - math.log(25.0)) < 1e-15 and abs(rte - math.log(25.0)) < 1e-15
+
+
+def test_fit_metrics_special_cases_and_scaling():
+    g = torch.Generator().manual_seed(5)
+    heads, rows, d = 3, 7, 8
+    alpha = torch.randn(heads, rows, generator=g, dtype=torch.float64)
+    A = torch.randn(heads, rows, d, generator=g, dtype=torch.float64)
+    Q = rand_bf16(g, heads, rows, d)
+    E = torch.randn(heads, rows, d, generator=g, dtype=torch.float64)
+    # a perfect module: both MSEs 0, every log ratio -inf
+    out, _ = oracle.fit_metrics(alpha, A, alpha, A, Q)
+    assert np.all(out[:, :2] == 0.0) and np.all(np.isneginf(out[:, 2]))
+    # A_theta = q (the baseline of Eq. (C.1)): every log ratio is exactly 0
+    out, rte = oracle.fit_metrics(alpha, A, alpha, f64(Q), Q)
+    assert np.all(out[:, 2] == 0.0) and rte == 0.0
+    # scaling the error by c scales the target MSE by c^2 and shifts each
+    # log ratio by log c^2; the score MSE of a + c is c^2
+    out1, rte1 = oracle.fit_metrics(alpha, A, alpha + 0.5, A + E, Q)
+    out3, rte3 = oracle.fit_metrics(alpha, A, alpha + 1.5, A + 3.0 * E, Q)
+    assert np.allclose(out1[:, 0], 0.25, rtol=0, atol=1e-15) and np.allclose(out3[:, 0], 2.25, rtol=0, atol=1e-15)
+    assert np.allclose(out3[:, 1], 9.0 * out1[:, 1], rtol=1e-12)
+    assert np.allclose(out3[:, 2], out1[:, 2] + math.log(9.0), rtol=0, atol=1e-12)
+    assert abs(rte3 - (rte1 + heads * math.log(9.0))) < 1e-10
+    # heads are independent: the metrics of a head do not see the others
+    out_h, _ = oracle.fit_metrics(alpha[1:2], A[1:2], alpha[1:2] + 0.5, A[1:2] + E[1:2], Q[1:2])
+    assert np.array_equal(out_h[0], out1[1])
