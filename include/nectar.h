@@ -258,6 +258,70 @@ NECTAR_API nectar_status nectar_decode(nectar_dims dims, const nectar_module_set
                             nectar_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * The decode as a base-model attention layer ("Nectar layer"): the same
+ * computation as nectar_decode, written in bf16 straight into the layer
+ * layout of the base model's attention output,
+ *   out   DEVICE bf16 [L][nq][Hkv * G][d], query head h * G + g
+ * (token-major; one [nq][Hkv * G][d] block per layer), rounded to nearest
+ * even from the fp32 value nectar_decode would write.  Works for decode
+ * (one token per sequence) and for prompts (several tokens of a sequence,
+ * q_pos giving each its causal prefix).
+ *   workspace  as nectar_decode, of nectar_decode_layer_out_workspace_size
+ *              bytes (below 64 query rows per KV head it adds rows * d * 4
+ *              bytes, rounded up to 256, for A_theta in fp32).
+ * ------------------------------------------------------------------------ */
+NECTAR_API size_t nectar_decode_layer_out_workspace_size(nectar_dims dims,
+                                                         const nectar_module_set *mods, int64_t nq);
+NECTAR_API nectar_status nectar_decode_layer_out(nectar_dims dims, const nectar_module_set *mods,
+                                                 const nectar_bf16 *Q, int64_t nq,
+                                                 const int32_t *q_seq, const int32_t *q_pos,
+                                                 const nectar_bf16 *Kloc, const nectar_bf16 *Vloc,
+                                                 int32_t B, int32_t T_max, const int32_t *local_len,
+                                                 float scale, nectar_bf16 *out, void *workspace,
+                                                 size_t workspace_bytes, nectar_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Quadrature module (§2.4): per (l, h), p learned key / value rows W, Z
+ * (DEVICE bf16 [L][Hkv][p][d]), initialised to the first p rows of the cache;
+ *   a_theta(q) = log sum_j exp((W q)_j * scale),
+ *   A_theta(q) = softmax(W q * scale)^T Z,
+ * i.e. the exact attention of Eq. (3.1) over (W, Z) -- computed by the same
+ * kernels as nectar_cache_attn_lse, with the same arguments, outputs,
+ * workspace rules and errors (n replaced by p).
+ * nectar_quadrature_init copies W[l][h] = K[l][h][0:p], Z[l][h] = V[l][h][0:p]
+ * (K, V: DEVICE bf16 [L][Hkv][n][d]; 1 <= p <= n; W, Z must not overlap K, V).
+ * ------------------------------------------------------------------------ */
+NECTAR_API nectar_status nectar_quadrature_init(nectar_dims dims, const nectar_bf16 *K,
+                                                const nectar_bf16 *V, int64_t n, int64_t p,
+                                                nectar_bf16 *W, nectar_bf16 *Z,
+                                                nectar_stream_t stream);
+NECTAR_API size_t nectar_quadrature_workspace_size(nectar_dims dims, int64_t p, int64_t nq);
+NECTAR_API nectar_status nectar_quadrature_forward(nectar_dims dims, const nectar_bf16 *W,
+                                                   const nectar_bf16 *Z, int64_t p,
+                                                   const nectar_bf16 *Q, int64_t nq, float scale,
+                                                   float *a, float *A_theta, void *workspace,
+                                                   size_t workspace_bytes, nectar_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Fitting metrics of a module against the exact targets (notes §4 and
+ * App. C.4, Eq. (C.1)), per (l, h):
+ *   metrics[l][h][0] = mean_q (a - alpha)^2                         score MSE
+ *   metrics[l][h][1] = mean_q (1/d) ||A_theta - A||^2               target MSE
+ *   metrics[l][h][2] = mean_q log(||A_theta - A||^2 / ||q - A||^2)  RTE term
+ * The RTE of Eq. (C.1) is the sum of the third column over (l, h).
+ *   alpha, a      DEVICE fp32 [L][Hkv][G][nq]
+ *   A, A_theta    DEVICE fp32 [L][Hkv][G][nq][d]
+ *   Q             DEVICE bf16 [L][Hkv][G][nq][d]
+ *   metrics       DEVICE double [L][Hkv][3], overwritten
+ * A row whose ||A_theta - A|| is 0 adds -inf to its RTE term (log 0), one
+ * whose q equals A adds +inf or NaN: the definition, unguarded.
+ * ------------------------------------------------------------------------ */
+NECTAR_API nectar_status nectar_fit_metrics(nectar_dims dims, int64_t nq, const float *alpha,
+                                            const float *A, const float *a, const float *A_theta,
+                                            const nectar_bf16 *Q, double *metrics,
+                                            nectar_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Diagnostics
  * ------------------------------------------------------------------------ */
 NECTAR_API const char *nectar_status_string(nectar_status s);

@@ -86,6 +86,19 @@ def lib() -> ctypes.CDLL:
     L.nectar_decode.argtypes = [Dims, ctypes.POINTER(_ModuleSetC), P, I64, P, P, P, P, I32, I32, P, F, P, P,
                                 ctypes.c_size_t, P]
     L.nectar_decode.restype = S
+    L.nectar_decode_layer_out_workspace_size.argtypes = [Dims, ctypes.POINTER(_ModuleSetC), I64]
+    L.nectar_decode_layer_out_workspace_size.restype = ctypes.c_size_t
+    L.nectar_decode_layer_out.argtypes = [Dims, ctypes.POINTER(_ModuleSetC), P, I64, P, P, P, P, I32, I32, P, F, P,
+                                          P, ctypes.c_size_t, P]
+    L.nectar_decode_layer_out.restype = S
+    L.nectar_quadrature_init.argtypes = [Dims, P, P, I64, I64, P, P, P]
+    L.nectar_quadrature_init.restype = S
+    L.nectar_quadrature_workspace_size.argtypes = [Dims, I64, I64]
+    L.nectar_quadrature_workspace_size.restype = ctypes.c_size_t
+    L.nectar_quadrature_forward.argtypes = [Dims, P, P, I64, P, I64, F, P, P, P, ctypes.c_size_t, P]
+    L.nectar_quadrature_forward.restype = S
+    L.nectar_fit_metrics.argtypes = [Dims, I64, P, P, P, P, P, P, P]
+    L.nectar_fit_metrics.restype = S
     L.nectar_status_string.argtypes = [S]
     L.nectar_status_string.restype = ctypes.c_char_p
     L.nectar_last_error.restype = ctypes.c_char_p
@@ -342,6 +355,82 @@ def decode(mods: ModuleSet, Q, q_seq, q_pos, Kloc, Vloc, local_len, scale: Optio
                              0 if workspace is None else workspace.numel(), _stream(stream))
     _check(st, "nectar_decode")
     return out
+
+
+def decode_layer_out(mods: ModuleSet, Q, q_seq, q_pos, Kloc, Vloc, local_len, scale: Optional[float] = None,
+                     out=None, workspace=None, stream=None):
+    """The decode as a base-model attention layer: bf16 out [L, nq, Hkv*G, d]
+    (query head h*G + g), the fp32 result of decode() rounded to nearest."""
+    dims, nq = dims_of(Q)
+    _need(Q, "Q", torch.bfloat16)
+    B, T = _local_args(q_seq, q_pos, Kloc, Vloc, local_len)
+    if scale is None:
+        scale = 1.0 / math.sqrt(dims.d)
+    if out is None:
+        out = torch.empty((dims.L, nq, dims.Hkv * dims.G, dims.d), dtype=torch.bfloat16, device=Q.device)
+    ws_bytes = int(lib().nectar_decode_layer_out_workspace_size(dims, mods.c(), nq))
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    st = lib().nectar_decode_layer_out(dims, mods.c(), _ptr(Q), nq, _ptr(q_seq), _ptr(q_pos), _ptr(Kloc),
+                                       _ptr(Vloc), B, T, _ptr(local_len), float(scale), _ptr(out), _ptr(workspace),
+                                       0 if workspace is None else workspace.numel(), _stream(stream))
+    _check(st, "nectar_decode_layer_out")
+    return out
+
+
+def quadrature_init(K, V, p: int, W=None, Z=None, stream=None):
+    """Quadrature module rows (section 2.4) initialised to the first p rows of
+    the cache: W, Z bf16 [L, Hkv, p, d] (made here when None)."""
+    for t, nm in ((K, "K"), (V, "V")):
+        _need(t, nm, torch.bfloat16)
+    L_, Hkv, n, d = K.shape
+    if W is None:
+        W = torch.empty((L_, Hkv, p, d), dtype=torch.bfloat16, device=K.device)
+    if Z is None:
+        Z = torch.empty((L_, Hkv, p, d), dtype=torch.bfloat16, device=K.device)
+    st = lib().nectar_quadrature_init(Dims(L_, Hkv, 1, d), _ptr(K), _ptr(V), n, p, _ptr(W), _ptr(Z),
+                                      _stream(stream))
+    _check(st, "nectar_quadrature_init")
+    return W, Z
+
+
+def quadrature_forward(W, Z, Q, scale: Optional[float] = None, a=None, A_theta=None, workspace=None, stream=None):
+    """(a_theta [L,Hkv,G,nq], A_theta [L,Hkv,G,nq,d]) fp32 of the Quadrature
+    module with rows W, Z bf16 [L, Hkv, p, d]."""
+    dims, nq = dims_of(Q)
+    p = W.shape[2]
+    for t, nm in ((W, "W"), (Z, "Z"), (Q, "Q")):
+        _need(t, nm, torch.bfloat16)
+    if scale is None:
+        scale = 1.0 / math.sqrt(dims.d)
+    if a is None:
+        a = torch.empty(Q.shape[:4], dtype=torch.float32, device=Q.device)
+    if A_theta is None:
+        A_theta = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    ws_bytes = int(lib().nectar_quadrature_workspace_size(dims, p, nq))
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    st = lib().nectar_quadrature_forward(dims, _ptr(W), _ptr(Z), p, _ptr(Q), nq, float(scale), _ptr(a),
+                                         _ptr(A_theta), _ptr(workspace),
+                                         0 if workspace is None else workspace.numel(), _stream(stream))
+    _check(st, "nectar_quadrature_forward")
+    return a, A_theta
+
+
+def fit_metrics(alpha, A, a, A_theta, Q, metrics=None, stream=None):
+    """Per (l, h) [score MSE, target MSE, RTE term] (float64 [L, Hkv, 3]) of a
+    module's (a, A_theta) against the exact (alpha, A); the RTE of Eq. (C.1)
+    is metrics[..., 2].sum()."""
+    dims, nq = dims_of(Q)
+    _need(Q, "Q", torch.bfloat16)
+    for t, nm in ((alpha, "alpha"), (A, "A"), (a, "a"), (A_theta, "A_theta")):
+        _need(t, nm, torch.float32)
+    if metrics is None:
+        metrics = torch.empty((dims.L, dims.Hkv, 3), dtype=torch.float64, device=Q.device)
+    st = lib().nectar_fit_metrics(dims, nq, _ptr(alpha), _ptr(A), _ptr(a), _ptr(A_theta), _ptr(Q), _ptr(metrics),
+                                  _stream(stream))
+    _check(st, "nectar_fit_metrics")
+    return metrics
 
 
 def device_error_flags(clear: bool = True) -> int:

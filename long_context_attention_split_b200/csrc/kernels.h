@@ -110,6 +110,7 @@ struct ModParams {
   float* out;
   float* ws_loc;        // decode: local state per row [(hd * rows + row)][d + 2]
   int64_t n_local;      // decode: local CTAs (heads * nq) ahead of the module CTAs
+  __nv_bfloat16* out_bf16;   // decode: if set, the output goes here, bf16 [L][nq][Hkv][G][d]
   int* err;
   int32_t width[kModMaxLayers];
   int64_t layer_base[kModMaxLayers];   // blob element offset of layer l
@@ -132,6 +133,9 @@ struct GemmParams {
   float* a_out;             // readout: [heads * R]
   float* A_out;             // readout: [heads * R][d] (A_theta, or the merged output)
   const float* ws_loc;      // decode: local state per row [(heads * R)][d + 2], else null
+  __nv_bfloat16* out_bf16;  // decode: if set, the merged output goes here, bf16 [L][nq][Hkv][G][d]
+  int G;
+  int64_t nq;
   int* err;
   int32_t width[kModMaxLayers];
   int64_t layer_base[kModMaxLayers];
@@ -171,6 +175,14 @@ size_t local_tc_smem();
 cudaError_t launch_local_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const LocalParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_local_warp(const LocalParams& p, int sms, cudaStream_t stream);
+
+// metrics.cu
+cudaError_t launch_fit_metrics(const float* alpha, const float* A, const float* a, const float* At,
+                               const __nv_bfloat16* Q, int64_t heads, int64_t rows, double* out,
+                               cudaStream_t stream);
+cudaError_t launch_quadrature_init(const __nv_bfloat16* K, const __nv_bfloat16* V, __nv_bfloat16* W,
+                                   __nv_bfloat16* Z, int64_t heads, int64_t n, int64_t p, int sms,
+                                   cudaStream_t stream);
 
 struct ModShape {
   int TPC, N, nblk, tmem_cols, stages, cps;

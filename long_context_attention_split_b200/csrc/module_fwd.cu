@@ -35,6 +35,7 @@
 #include "kernels.h"
 #include "local_attn.cuh"
 #include "module_layout.h"
+#include "out_layout.cuh"
 
 namespace nectar {
 
@@ -430,7 +431,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_q, const ModParams p) {
 }
 
 // Merge of every row's document term (a_theta from the workspace, A_theta
-// already in out) with its local state, Eqs. (3.4)-(3.5); in place in out.
+// in A_out) with its local state, Eqs. (3.4)-(3.5), into out (in place when
+// A_out is out) or, bf16, into out_bf16 in the layer layout.
 __global__ void decode_merge_kernel(const ModParams p, int64_t nrows) {
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= nrows * kD) return;
@@ -440,7 +442,9 @@ __global__ void decode_merge_kernel(const ModParams p, int64_t nrows) {
   const float ad = p.a_out[row] * kLog2e;       // document logit in log2 units
   const float M = fmaxf(ad, st[kD]);
   const float wd = exp2_shift(ad, M), wl = exp2_shift(st[kD], M);
-  p.out[idx] = (wd * p.out[idx] + wl * st[dim]) / (wd + wl * st[kD + 1]);
+  const float v = (wd * p.A_out[idx] + wl * st[dim]) / (wd + wl * st[kD + 1]);
+  if (p.out_bf16 != nullptr) p.out_bf16[layer_layout_index(row, dim, p.Hkv, p.G, p.nq)] = __float2bfloat16_rn(v);
+  else p.out[idx] = v;
 }
 
 // ---------------------------------------------------------------------------

@@ -31,6 +31,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "module_layout.h"
+#include "out_layout.cuh"
 
 namespace nectar {
 
@@ -313,16 +314,29 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
           } else {
             // merge with the row's local state (decode)
             const float* st0 = p.ws_loc + (g.hd * R + r0 + n0) * (kD + 2);
+            float mv[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const float aj = __shfl_sync(0xffffffffu, a_l, j);
+              mv[j] = 0.f;
               if (j < nrow) {
                 const float* st = st0 + j * (kD + 2);
                 const float ad = aj * kLog2e;
                 const float M = fmaxf(ad, st[kD]);
                 const float wd = exp2_shift(ad, M), wl = exp2_shift(st[kD], M);
-                arow[j * kD] = (wd * (__uint_as_float(v[j]) + bias) + wl * st[u]) / (wd + wl * st[kD + 1]);
+                mv[j] = (wd * (__uint_as_float(v[j]) + bias) + wl * st[u]) / (wd + wl * st[kD + 1]);
               }
+            }
+            if (p.out_bf16 == nullptr) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < nrow) arow[j * kD] = mv[j];
+            } else {
+              const int64_t row0 = g.hd * R + r0 + n0;
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < nrow)
+                  p.out_bf16[layer_layout_index(row0 + j, u, p.Hkv, p.G, p.nq)] = __float2bfloat16_rn(mv[j]);
             }
           }
         }

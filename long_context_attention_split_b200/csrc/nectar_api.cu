@@ -570,7 +570,8 @@ size_t gemm_ws_bytes(const nectar_dims& dims, int Hmax, int depth, int64_t nq) {
 // readout launch.  With ws_loc the readout merges with the local states
 // (decode) and writes the output into A_out.
 nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, const nectar_bf16* Q, int64_t nq,
-                              float* a, float* A_out, const float* ws_loc, void* ws, cudaStream_t st) {
+                              float* a, float* A_out, const float* ws_loc, void* ws, cudaStream_t st,
+                              __nv_bfloat16* out_bf16 = nullptr) {
   const DeviceInfo di = device_info();
   const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
   const int64_t R = static_cast<int64_t>(dims.G) * nq;
@@ -592,6 +593,8 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
   g.tmem_cols = sh.tmem_cols;
   g.blob = mp.blob;
   g.err = mp.err;
+  g.G = dims.G;
+  g.nq = nq;
   for (int l = 0; l < dims.L; ++l) {
     g.width[l] = mp.width[l];
     g.layer_base[l] = mp.layer_base[l];
@@ -626,6 +629,7 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
     g.a_out = g.readout ? a : nullptr;
     g.A_out = g.readout ? A_out : nullptr;
     g.ws_loc = g.readout ? ws_loc : nullptr;
+    g.out_bf16 = g.readout ? out_bf16 : nullptr;
     const GemmShape& ss = g.readout ? shr : sh;
     g.NR = ss.NR;
     g.rtiles = ss.rtiles;
@@ -754,20 +758,34 @@ size_t nectar_decode_workspace_size(nectar_dims dims, const nectar_module_set* m
   return decode_ws_a_bytes(rows) + loc;
 }
 
-nectar_status nectar_decode(nectar_dims dims, const nectar_module_set* mods, const nectar_bf16* Q, int64_t nq,
-                            const int32_t* q_seq, const int32_t* q_pos, const nectar_bf16* Kloc,
-                            const nectar_bf16* Vloc, int32_t B, int32_t T_max, const int32_t* local_len,
-                            float scale, float* out, void* workspace, size_t workspace_bytes,
-                            nectar_stream_t stream) {
+size_t nectar_decode_layer_out_workspace_size(nectar_dims dims, const nectar_module_set* mods, int64_t nq) {
+  const size_t base = nectar_decode_workspace_size(dims, mods, nq);
+  if (base == 0 || use_gemm_path(dims, nq)) return base;
+  // the one-launch path keeps A_theta in fp32 until the merge
+  const int64_t rows = static_cast<int64_t>(dims.L) * dims.Hkv * dims.G * nq;
+  return base + align256(static_cast<size_t>(rows) * kD * sizeof(float));
+}
+
+}  // extern "C"
+
+namespace {
+
+// The decode, into out (fp32, per KV head) or out_bf16 (bf16, layer layout).
+nectar_status decode_impl(nectar_dims dims, const nectar_module_set* mods, const nectar_bf16* Q, int64_t nq,
+                          const int32_t* q_seq, const int32_t* q_pos, const nectar_bf16* Kloc,
+                          const nectar_bf16* Vloc, int32_t B, int32_t T_max, const int32_t* local_len, float scale,
+                          float* out, __nv_bfloat16* out_bf16, void* workspace, size_t workspace_bytes,
+                          nectar_stream_t stream) {
   NECTAR_TRY(check_dims(dims));
   if (nq < 0) return fail(NECTAR_ERR_INVALID_ARG, "nq must be >= 0");
   if (nq == 0) return NECTAR_OK;
   if (!(scale == scale)) return fail(NECTAR_ERR_INVALID_ARG, "scale is NaN");
-  NECTAR_TRY(check_ptr(out, "out"));
+  NECTAR_TRY(check_ptr(out != nullptr ? static_cast<const void*>(out) : static_cast<const void*>(out_bf16), "out"));
   NECTAR_TRY(check_local(q_seq, q_pos, Kloc, Vloc, B, T_max, local_len));
   if (mods == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "mods is NULL");
   NECTAR_TRY(check_modules_shape(dims, mods->depth, mods->width));
-  const size_t need = nectar_decode_workspace_size(dims, mods, nq);
+  const size_t need = out != nullptr ? nectar_decode_workspace_size(dims, mods, nq)
+                                     : nectar_decode_layer_out_workspace_size(dims, mods, nq);
   if (workspace == nullptr || workspace_bytes < need)
     return fail(NECTAR_ERR_WORKSPACE, "decode workspace of %zu bytes given, %zu needed",
                 workspace == nullptr ? size_t(0) : workspace_bytes, need);
@@ -791,11 +809,12 @@ nectar_status nectar_decode(nectar_dims dims, const nectar_module_set* mods, con
   p.T = T_max;
   p.qmul = scale * kLog2e;
   p.out = out;
+  p.out_bf16 = out_bf16;
   p.n_local = heads * nq;
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
   if (gemm) {
     // local states first, then the layer-by-layer module whose readout merges
-    uint8_t* base = static_cast<uint8_t*>(workspace);
     p.ws_loc = reinterpret_cast<float*>(base);
     if (use_local_tc(dims, nq, B, T_max)) {
       NECTAR_TRY(run_local_many(dims, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, p.ws_loc,
@@ -805,14 +824,93 @@ nectar_status nectar_decode(nectar_dims dims, const nectar_module_set* mods, con
       if (e != cudaSuccess) return cuda_fail(e, "local attention kernel");
     }
     return run_module_gemm(dims, p, Q, nq, nullptr, out, p.ws_loc,
-                           base + align256(static_cast<size_t>(rows) * (kD + 2) * sizeof(float)), st);
+                           base + align256(static_cast<size_t>(rows) * (kD + 2) * sizeof(float)), st, out_bf16);
   }
-  p.a_out = static_cast<float*>(workspace);
-  p.A_out = out;                    // A_theta lands in out, merged in place
-  p.ws_loc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + decode_ws_a_bytes(rows));
+  p.a_out = reinterpret_cast<float*>(base);
+  p.ws_loc = reinterpret_cast<float*>(base + decode_ws_a_bytes(rows));
+  // A_theta lands in out and is merged in place; for the bf16 layer output it
+  // is kept in fp32 after the local states
+  p.A_out = out != nullptr ? out
+                           : reinterpret_cast<float*>(base + decode_ws_a_bytes(rows) +
+                                                      align256(static_cast<size_t>(rows) * (kD + 2) * sizeof(float)));
   const int units = dims.L * dims.Hkv * sh.nblk;
   cudaError_t e = launch_decode(tq, p, units, sh.smem, st);
   return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "decode kernels");
+}
+
+}  // namespace
+
+extern "C" {
+
+nectar_status nectar_decode(nectar_dims dims, const nectar_module_set* mods, const nectar_bf16* Q, int64_t nq,
+                            const int32_t* q_seq, const int32_t* q_pos, const nectar_bf16* Kloc,
+                            const nectar_bf16* Vloc, int32_t B, int32_t T_max, const int32_t* local_len,
+                            float scale, float* out, void* workspace, size_t workspace_bytes,
+                            nectar_stream_t stream) {
+  if (out == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "out is NULL");
+  return decode_impl(dims, mods, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, out, nullptr,
+                     workspace, workspace_bytes, stream);
+}
+
+nectar_status nectar_decode_layer_out(nectar_dims dims, const nectar_module_set* mods, const nectar_bf16* Q,
+                                      int64_t nq, const int32_t* q_seq, const int32_t* q_pos,
+                                      const nectar_bf16* Kloc, const nectar_bf16* Vloc, int32_t B, int32_t T_max,
+                                      const int32_t* local_len, float scale, nectar_bf16* out, void* workspace,
+                                      size_t workspace_bytes, nectar_stream_t stream) {
+  if (out == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "out is NULL");
+  return decode_impl(dims, mods, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, nullptr,
+                     reinterpret_cast<__nv_bfloat16*>(out), workspace, workspace_bytes, stream);
+}
+
+// ---------------------------------------------------------------------------
+// next rows: Quadrature module, fitting metrics
+// ---------------------------------------------------------------------------
+nectar_status nectar_quadrature_init(nectar_dims dims, const nectar_bf16* K, const nectar_bf16* V, int64_t n,
+                                     int64_t p, nectar_bf16* W, nectar_bf16* Z, nectar_stream_t stream) {
+  NECTAR_TRY(check_dims(dims));
+  if (p < 1 || p > n) return fail(NECTAR_ERR_INVALID_ARG, "p = %lld must be in [1, n = %lld]", (long long)p,
+                                  (long long)n);
+  NECTAR_TRY(check_ptr(K, "K"));
+  NECTAR_TRY(check_ptr(V, "V"));
+  NECTAR_TRY(check_ptr(W, "W"));
+  NECTAR_TRY(check_ptr(Z, "Z"));
+  const DeviceInfo di = device_info();
+  if (di.sms == 0) return fail(NECTAR_ERR_CUDA, "no CUDA device");
+  const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
+  cudaError_t e = launch_quadrature_init(reinterpret_cast<const __nv_bfloat16*>(K),
+                                         reinterpret_cast<const __nv_bfloat16*>(V),
+                                         reinterpret_cast<__nv_bfloat16*>(W), reinterpret_cast<__nv_bfloat16*>(Z),
+                                         heads, n, p, di.sms, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "quadrature init kernel");
+}
+
+size_t nectar_quadrature_workspace_size(nectar_dims dims, int64_t p, int64_t nq) {
+  return nectar_cache_attn_workspace_size(dims, p, nq);
+}
+
+nectar_status nectar_quadrature_forward(nectar_dims dims, const nectar_bf16* W, const nectar_bf16* Z, int64_t p,
+                                        const nectar_bf16* Q, int64_t nq, float scale, float* a, float* A_theta,
+                                        void* workspace, size_t workspace_bytes, nectar_stream_t stream) {
+  // the exact attention of Eq. (3.1) over the p learned rows
+  return nectar_cache_attn_lse(dims, W, Z, p, Q, nq, scale, a, A_theta, workspace, workspace_bytes, stream);
+}
+
+nectar_status nectar_fit_metrics(nectar_dims dims, int64_t nq, const float* alpha, const float* A, const float* a,
+                                 const float* A_theta, const nectar_bf16* Q, double* metrics,
+                                 nectar_stream_t stream) {
+  NECTAR_TRY(check_dims(dims));
+  if (nq < 0) return fail(NECTAR_ERR_INVALID_ARG, "nq must be >= 0");
+  if (alpha == nullptr || a == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "alpha / a is NULL");
+  NECTAR_TRY(check_ptr(A, "A"));
+  NECTAR_TRY(check_ptr(A_theta, "A_theta"));
+  NECTAR_TRY(check_ptr(Q, "Q"));
+  if (metrics == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "metrics is NULL");
+  const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
+  if (heads > 0x7fffffffLL) return fail(NECTAR_ERR_UNSUPPORTED, "too many heads");
+  cudaError_t e = launch_fit_metrics(alpha, A, a, A_theta, reinterpret_cast<const __nv_bfloat16*>(Q), heads,
+                                     static_cast<int64_t>(dims.G) * nq, metrics,
+                                     reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "fit metrics kernel");
 }
 
 }  // extern "C"
