@@ -175,6 +175,9 @@ size_t local_tc_smem();
 cudaError_t launch_local_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const LocalParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_local_warp(const LocalParams& p, int sms, cudaStream_t stream);
+size_t local_tct_smem();
+cudaError_t launch_local_tct(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const LocalParams& p, int sms, cudaStream_t stream);
 
 // metrics.cu
 cudaError_t launch_fit_metrics(const float* alpha, const float* A, const float* a, const float* At,

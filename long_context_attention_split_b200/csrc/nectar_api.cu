@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -312,11 +313,14 @@ static bool use_local_tc(const nectar_dims& dims, int64_t nq, int32_t B, int32_t
 }
 
 // Either leaves each row's local state in ws_loc (out == nullptr) or merges
-// it with (a, A_doc) into out.
-static nectar_status run_local_tc(const nectar_dims& dims, const nectar_bf16* Q, int64_t nq, const int32_t* q_seq,
-                                  const int32_t* q_pos, const nectar_bf16* Kloc, const nectar_bf16* Vloc, int32_t B,
-                                  int32_t T_max, const int32_t* local_len, float scale, float* ws_loc,
-                                  const float* a, const float* A_doc, float* out, cudaStream_t st) {
+// it with (a, A_doc) into out.  `transposed` picks local_tct_kernel (keys on
+// the TMEM lanes; G <= 16, T_max <= 512) over local_tc_kernel (query heads
+// on the TMEM lanes); both take the same parameters and tensor maps.
+static nectar_status run_local_tc(bool transposed, const nectar_dims& dims, const nectar_bf16* Q, int64_t nq,
+                                  const int32_t* q_seq, const int32_t* q_pos, const nectar_bf16* Kloc,
+                                  const nectar_bf16* Vloc, int32_t B, int32_t T_max, const int32_t* local_len,
+                                  float scale, float* ws_loc, const float* a, const float* A_doc, float* out,
+                                  cudaStream_t st) {
   const DeviceInfo di = device_info();
   if (di.sms == 0) return fail(NECTAR_ERR_CUDA, "no CUDA device");
   const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
@@ -355,8 +359,13 @@ static nectar_status run_local_tc(const nectar_dims& dims, const nectar_bf16* Q,
     NECTAR_TRY(make_tmap(&tk, Kloc, 4, dk, sk, bk, "local keys"));
     NECTAR_TRY(make_tmap(&tv, Vloc, 4, dk, sk, bk, "local values"));
   }
-  const int grid = static_cast<int>(p.njobs < di.sms ? p.njobs : di.sms);
-  cudaError_t e = launch_local_tc(tq, tk, tv, p, grid, st);
+  cudaError_t e;
+  if (transposed) {
+    e = launch_local_tct(tq, tk, tv, p, di.sms, st);
+  } else {
+    const int grid = static_cast<int>(p.njobs < di.sms ? p.njobs : di.sms);
+    e = launch_local_tc(tq, tk, tv, p, grid, st);
+  }
   return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "local attention kernel");
 }
 
@@ -390,17 +399,29 @@ static nectar_status run_local_warp(const nectar_dims& dims, const nectar_bf16* 
   return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "local attention kernel");
 }
 
-// Many query tokens: up to 8 query heads per KV head on warps, more on the
-// tensor cores.
+// Which kernel runs the local attention of many query tokens.  Default: the
+// transposed tensor-core kernel where it applies (G <= 16, at most 512 local
+// tokens), else warps for G <= 8 and the row-per-head tensor-core kernel
+// above.  NECTAR_LOCAL_TCT=0 turns the transposed kernel off.
+static bool use_local_tct(const nectar_dims& dims, int32_t T_max) {
+  if (dims.G > 16 || T_max > 512) return false;
+  const char* env = getenv("NECTAR_LOCAL_TCT");
+  return env == nullptr || atoi(env) != 0;
+}
+
 static nectar_status run_local_many(const nectar_dims& dims, const nectar_bf16* Q, int64_t nq,
                                     const int32_t* q_seq, const int32_t* q_pos, const nectar_bf16* Kloc,
                                     const nectar_bf16* Vloc, int32_t B, int32_t T_max, const int32_t* local_len,
                                     float scale, float* ws_loc, const float* a, const float* A_doc, float* out,
                                     cudaStream_t st) {
+  if (use_local_tct(dims, T_max))
+    return run_local_tc(true, dims, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, ws_loc, a, A_doc,
+                        out, st);
   if (dims.G <= 8)
     return run_local_warp(dims, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, ws_loc, a, A_doc, out,
                           st);
-  return run_local_tc(dims, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, ws_loc, a, A_doc, out, st);
+  return run_local_tc(false, dims, Q, nq, q_seq, q_pos, Kloc, Vloc, B, T_max, local_len, scale, ws_loc, a, A_doc,
+                      out, st);
 }
 
 nectar_status nectar_merge_local(nectar_dims dims, const float* a, const float* A_doc, const nectar_bf16* Q,

@@ -233,9 +233,11 @@ def test_merge_bad_metadata_flags():
     assert torch.equal(out[..., 1, :], Ad[..., 1, :])
 
 
-# many query rows per KV head: the tensor-core local kernel (one job per
-# (KV head, token), 128-key tiles)
-@pytest.mark.parametrize("G,T", [(1, 300), (4, 33), (7, 256), (33, 130)])
+# many query rows per KV head: the tensor-core local kernels (one job per
+# (KV head, token), 128-key tiles).  G <= 16 with at most 512 local tokens
+# runs the transposed kernel (keys on the TMEM lanes), G = 33 the kernel with
+# the query heads on the lanes, T = 600 the warp kernel.
+@pytest.mark.parametrize("G,T", [(1, 300), (4, 33), (7, 256), (9, 200), (16, 512), (33, 130), (4, 600)])
 def test_merge_many_tokens(G, T):
     nq = max(128 // G + 1, 8)
     B = 5
@@ -251,6 +253,13 @@ def test_merge_many_tokens(G, T):
     for i, b in enumerate(q_seq):
         if b == 1:
             assert torch.equal(o[:, :, i], A[:, :, i])
+
+
+@pytest.mark.parametrize("G,T", [(4, 33), (7, 256), (16, 130)])
+def test_merge_many_tokens_without_transposed_kernel(G, T, monkeypatch):
+    # the warp kernel (G <= 8) and the row-per-head tensor-core kernel (G > 8)
+    monkeypatch.setenv("NECTAR_LOCAL_TCT", "0")
+    test_merge_many_tokens(G, T)
 
 
 def test_merge_prefill_causal_many_tiles():
@@ -402,6 +411,7 @@ def test_decode_toy_prefill():
     dict(L=2, Hkv=2, G=4, n=16, B=40, T=50, widths=[256, 512]),   # 160 rows per KV head: GEMM path
     dict(L=1, Hkv=2, G=7, n=16, B=64, T=33, widths=[768]),     # 448 rows: two row tiles of 224
     dict(L=2, Hkv=2, G=4, n=16, B=16, T=40, widths=[256, 128]),   # exactly 64 rows: grouped-GEMM decode
+    dict(L=1, Hkv=2, G=16, n=16, B=8, T=300, widths=[256]),    # 128 rows, 16 heads per local job, 3 tiles
 ])
 def test_decode_shapes(kw):
     wl = make_workload("qwen3_1p7b", seed=2, key_scale=None, **kw)
