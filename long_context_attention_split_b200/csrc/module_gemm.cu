@@ -63,7 +63,23 @@ __host__ __device__ inline GemmSmem gemm_smem_layout(int NR, int stages) {
   return s;
 }
 
-__device__ __forceinline__ float gemm_silu(float v) { return __fdividef(v, 1.0f + ex2(-v * kLog2e)); }
+// SiLU of two pre-activations x = acc + b, packed to bf16x2.  With h = x / 2,
+// SiLU(x) = x sigmoid(x) = h (1 + tanh h) = h + h tanh h: one tanh.approx
+// (the hardware approximation, relative error ~2^-11) per value instead of
+// an exp2 and a reciprocal, and the bias folded into the first (paired)
+// FMA as b / 2.  The absolute error, |x| 2^-12 at most, stays below the
+// bf16 rounding of the stored activation for |x| < 8.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t gemm_silu2(uint32_t acc0, uint32_t acc1, float half_bias) {
+  const float2 h = ffma2(make_float2(__uint_as_float(acc0), __uint_as_float(acc1)), make_float2(0.5f, 0.5f),
+                         make_float2(half_bias, half_bias));
+  const float2 y = ffma2(h, make_float2(tanh_approx(h.x), tanh_approx(h.y)), h);
+  return pack_bf16x2(y.x, y.y);
+}
 
 struct GemmTile {
   int l, H, net, m, rt;
@@ -240,6 +256,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         bias = __bfloat162float(p.blob[nb + layout::hidden_b_off(g.H, p.depth, p.stage) + i]);
         if (score_last) wsc = __bfloat162float(p.blob[nb + layout::out_w_off(g.H, p.depth) + i]);
       }
+      const float hbias = 0.5f * bias;
       if (ok) ok = mbar_wait_sleep(b_accf + 8 * b, (tc >> 1) & 1, p.err);   // waits out a main loop
       ok = __all_sync(0xffffffffu, ok);         // keeps the shuffles below warp-uniform
       tc_fence_after();
@@ -256,8 +273,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
               // bf16 rounding of two rows at once (one packed conversion)
-              const uint32_t w = pack_bf16x2(gemm_silu(__uint_as_float(v[j]) + bias),
-                                             gemm_silu(__uint_as_float(v[j + 1]) + bias));
+              const uint32_t w = gemm_silu2(v[j], v[j + 1], hbias);
               part[j] = (i < g.H) ? wsc * bf16lo(w) : 0.f;
               part[j + 1] = (i < g.H) ? wsc * bf16hi(w) : 0.f;
             }
@@ -274,18 +290,14 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
               if (nrow >= 32) {
 #pragma unroll
                 for (int j = 0; j < 32; j += 2) {
-                  const uint32_t w = live ? pack_bf16x2(gemm_silu(__uint_as_float(v[j]) + bias),
-                                                        gemm_silu(__uint_as_float(v[j + 1]) + bias))
-                                          : 0u;
+                  const uint32_t w = live ? gemm_silu2(v[j], v[j + 1], hbias) : 0u;
                   hb[j * Hp] = static_cast<uint16_t>(w & 0xFFFFu);
                   hb[(j + 1) * Hp] = static_cast<uint16_t>(w >> 16);
                 }
               } else {
 #pragma unroll
                 for (int j = 0; j < 32; j += 2) {
-                  const uint32_t w = live ? pack_bf16x2(gemm_silu(__uint_as_float(v[j]) + bias),
-                                                        gemm_silu(__uint_as_float(v[j + 1]) + bias))
-                                          : 0u;
+                  const uint32_t w = live ? gemm_silu2(v[j], v[j + 1], hbias) : 0u;
                   if (j < nrow) hb[j * Hp] = static_cast<uint16_t>(w & 0xFFFFu);
                   if (j + 1 < nrow) hb[(j + 1) * Hp] = static_cast<uint16_t>(w >> 16);
                 }
@@ -311,22 +323,28 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
 #pragma unroll
             for (int j = 0; j < 32; ++j)
               if (j < nrow) arow[j * kD] = __uint_as_float(v[j]) + bias;
-          } else {
-            // merge with the row's local state (decode)
+          } else if (nrow > 0) {
+            // merge with the row's local state (decode).  Lane j forms the two
+            // weights of row j once (an exp2 pair and a division per row, not
+            // per element); then every lane loads its dim of all the batch's
+            // local sums at once (row index clamped into the tile), so the 32
+            // loads are in flight together, and combines.
             const float* st0 = p.ws_loc + (g.hd * R + r0 + n0) * (kD + 2);
+            const float* stl = st0 + (lane < nrow ? lane : 0) * (kD + 2);
+            const float ml = stl[kD], ll = stl[kD + 1];
+            const float ad = a_l * kLog2e;                  // document logit, log2 units
+            const float M = fmaxf(ad, ml);
+            const float wd = exp2_shift(ad, M), wl = exp2_shift(ml, M);
+            const float inv = 1.0f / (wd + wl * ll);
+            const float cd = wd * inv, cl = wl * inv;
+            float xs[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) xs[j] = st0[(j < nrow ? j : 0) * (kD + 2) + u];
             float mv[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float aj = __shfl_sync(0xffffffffu, a_l, j);
-              mv[j] = 0.f;
-              if (j < nrow) {
-                const float* st = st0 + j * (kD + 2);
-                const float ad = aj * kLog2e;
-                const float M = fmaxf(ad, st[kD]);
-                const float wd = exp2_shift(ad, M), wl = exp2_shift(st[kD], M);
-                mv[j] = (wd * (__uint_as_float(v[j]) + bias) + wl * st[u]) / (wd + wl * st[kD + 1]);
-              }
-            }
+            for (int j = 0; j < 32; ++j)
+              mv[j] = __shfl_sync(0xffffffffu, cd, j) * (__uint_as_float(v[j]) + bias) +
+                      __shfl_sync(0xffffffffu, cl, j) * xs[j];
             if (p.out_bf16 == nullptr) {
 #pragma unroll
               for (int j = 0; j < 32; ++j)
@@ -369,8 +387,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
 // host side
 // ---------------------------------------------------------------------------
 // max_rows: rows per tile at most (256 for the hidden layers; the readout
-// uses smaller tiles -- it has one M tile per head, and its merge epilogue
-// per row is long -- so that all SMs get work)
+// picks its own, see readout_rows)
 GemmShape gemm_shape(int64_t R, int max_rows) {
   GemmShape sh{};
   sh.rtiles = static_cast<int>((R + max_rows - 1) / max_rows);

@@ -587,6 +587,17 @@ size_t gemm_ws_bytes(const nectar_dims& dims, int Hmax, int depth, int64_t nq) {
   return (depth >= 2 ? 2 : 1) * gemm_h_bytes(dims, Hmax, nq) + align256(static_cast<size_t>(rows) * MT * 4);
 }
 
+// Rows per readout tile.  The readout has a single 128-dim M tile per head,
+// and every row tile streams the head's whole W_out again, so tiles are as
+// tall as possible (up to 256 rows) while there are still at least four
+// tiles per SM; with fewer rows per head they shrink (down to 64) so that
+// all SMs get work.
+int readout_rows(int64_t heads, int64_t R, int sms) {
+  for (int mr = 256; mr > 64; mr /= 2)
+    if (heads * ((R + mr - 1) / mr) >= 4 * static_cast<int64_t>(sms)) return mr;
+  return 64;
+}
+
 // The layer-by-layer module forward: depth hidden-layer launches and one
 // readout launch.  With ws_loc the readout merges with the local states
 // (decode) and writes the output into A_out.
@@ -598,7 +609,7 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
   const int64_t R = static_cast<int64_t>(dims.G) * nq;
   if (heads * R * 2 > 0x7fffffffLL) return fail(NECTAR_ERR_UNSUPPORTED, "too many query rows for one call");
   const GemmShape sh = gemm_shape(R, 256);
-  const GemmShape shr = gemm_shape(R, 64);     // readout tiles
+  const GemmShape shr = gemm_shape(R, readout_rows(heads, R, di.sms));
   GemmParams g;
   memset(&g, 0, sizeof(g));
   g.L = dims.L;
