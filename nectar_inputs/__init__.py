@@ -213,6 +213,48 @@ def make_modules(L: int, Hkv: int, widths: Sequence[int], d: int, seed: int,
     return mods
 
 
+def make_modules_general(L: int, Hkv: int, d: int, seed: int, device, depths: Sequence[int],
+                         width_b: Sequence[int], width_s: Sequence[int],
+                         width_t: Sequence[int]) -> List[Dict[str, dict]]:
+    """Random-init module sets with a shared backbone: depths (D_b, D_s, D_t)
+    of the backbone, score and target branches, per-layer widths of each.
+    The backbone is D_b layers of the Eq. (3.6) recursion; each branch
+    continues it from the backbone's last hidden state (its first layer sees
+    q and that state), then its linear readout.  A layer that starts a chain
+    (D_b = 0) sees only q: U [H][d], V None.  Weights N(0, 1/fan_in), biases
+    N(0, BIAS_STD^2), bf16.  With D_b = 0 and equal widths the draws are
+    those of make_modules."""
+    Db, Ds, Dt = depths
+    mods = []
+    for l in range(L):
+        layer = {}
+        Hb = width_b[l] if Db > 0 else 0
+        g = _gen(device, seed, "module", l, "backbone")
+        U, Vs, b = [], [], []
+        for k in range(Db):
+            prev = 0 if k == 0 else Hb
+            std = 1.0 / math.sqrt(d + prev)
+            U.append((_randn((Hkv, Hb, prev if prev else d), g, device) * std).to(torch.bfloat16))
+            Vs.append(None if prev == 0 else (_randn((Hkv, Hb, d), g, device) * std).to(torch.bfloat16))
+            b.append((_randn((Hkv, Hb), g, device) * BIAS_STD).to(torch.bfloat16))
+        layer["backbone"] = dict(U=U, V=Vs, b=b, H=Hb)
+        for net, dout, D, Ws in (("score", 1, Ds, width_s), ("target", d, Dt, width_t)):
+            H = Ws[l]
+            g = _gen(device, seed, "module", l, net)
+            U, Vs, b = [], [], []
+            for k in range(D):
+                prev = Hb if k == 0 else H
+                std = 1.0 / math.sqrt(d + prev)
+                U.append((_randn((Hkv, H, prev if prev else d), g, device) * std).to(torch.bfloat16))
+                Vs.append(None if prev == 0 else (_randn((Hkv, H, d), g, device) * std).to(torch.bfloat16))
+                b.append((_randn((Hkv, H), g, device) * BIAS_STD).to(torch.bfloat16))
+            Wout = (_randn((Hkv, dout, H), g, device) / math.sqrt(H)).to(torch.bfloat16)
+            c = (_randn((Hkv, dout), g, device) * BIAS_STD).to(torch.bfloat16)
+            layer[net] = dict(U=U, V=Vs, b=b, Wout=Wout, c=c, H=H, dout=dout)
+        mods.append(layer)
+    return mods
+
+
 def make_workload(name: str, *, seed: int = 0, device="cpu", **overrides) -> Workload:
     """Build a preset workload (optionally with overridden sizes).
 

@@ -48,6 +48,9 @@ def _load():
         lib.oracle_mlp_param_count.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
         lib.oracle_mlp_param_count.restype = I
         lib.oracle_mlp.argtypes = [I, I, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P]
+        lib.oracle_chain_param_count.argtypes = [ctypes.c_int, ctypes.c_int, P, ctypes.c_int]
+        lib.oracle_chain_param_count.restype = I
+        lib.oracle_chain.argtypes = [I, I, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, P, P]
         lib.oracle_merge_local.argtypes = [I, I, I, ctypes.c_int, P, P, P, P, P, P, P, I, I, P,
                                            ctypes.c_double, P]
         lib.oracle_full_attention.argtypes = [I, I, I, I, ctypes.c_int, P, P, P, P, P, P, P, I, I, P,
@@ -166,6 +169,72 @@ def module_forward(wl, heads=None):
         X = wl.Q[l, hs].reshape(len(hs), wl.rows, wl.d)
         for net, dout in (("score", 1), ("target", wl.d)):
             Y = mlp(flatten_net(wl.modules[l][net], hs), X, wl.depth, H, dout)
+            for j, h in enumerate(hs):
+                if net == "score":
+                    out_a[(l, h)] = Y[j, :, 0]
+                else:
+                    out_A[(l, h)] = Y[j]
+    return out_a, out_A
+
+
+def flatten_chain(backbone: Optional[dict], net: dict, heads: Optional[List[int]] = None):
+    """The parameters of one net with a shared backbone in front (dicts from
+    nectar_inputs.make_modules_general), as the chain the oracle runs: the
+    backbone's layers, then the branch's, then the readout.  Returns
+    (params [Hkv][P] float64, per-layer widths)."""
+    layers = []
+    if backbone is not None:
+        layers += [(backbone["U"][k], backbone["V"][k], backbone["b"][k]) for k in range(len(backbone["U"]))]
+    layers += [(net["U"][k], net["V"][k], net["b"][k]) for k in range(len(net["U"]))]
+    widths = [int(U.shape[1]) for (U, _, _) in layers]
+    hs = range(net["Wout"].shape[0]) if heads is None else heads
+    rows = []
+    for h in hs:
+        parts = []
+        for k, (U, V, b) in enumerate(layers):
+            # the chain's first layer sees only q (through U); later ones see
+            # q through V and the previous layer through U
+            assert (V is None) == (k == 0)
+            parts += ([U[h], b[h]] if k == 0 else [V[h], U[h], b[h]])
+        parts += [net["Wout"][h], net["c"][h]]
+        rows.append(np.concatenate([p.detach().cpu().double().numpy().ravel() for p in parts]))
+    return np.ascontiguousarray(np.stack(rows)), widths
+
+
+def chain(params: np.ndarray, X, widths: List[int], dout: int):
+    """A chain of Eq. (3.6) layers with per-layer widths, then the linear
+    readout.  params [units][P] (flatten_chain order); X bf16 [units, rows, d].
+    Returns Y [units, rows, dout] float64."""
+    Xb = _bf16_bits(X)
+    units, rows, d = Xb.shape
+    W = np.ascontiguousarray(np.asarray(widths, dtype=np.int32))
+    P = int(_load().oracle_chain_param_count(d, len(widths), _p(W), dout))
+    params = _f64(params)
+    assert params.shape == (units, P), (params.shape, units, P)
+    Y = np.zeros((units, rows, dout), np.float64)
+    _load().oracle_chain(units, rows, d, len(widths), _p(W), dout, _p(params), _p(Xb), _p(Y))
+    return Y
+
+
+def module_forward_general(mods, Q, heads=None):
+    """(a, A_theta) of module sets with a shared backbone (depths
+    (D_b, D_s, D_t), App. A.3; mods from nectar_inputs.make_modules_general):
+    the score output is the chain backbone -> score branch -> readout, the
+    target output the chain backbone -> target branch -> readout.
+    Q bf16 [L][Hkv][G][nq][d].  Returns dicts keyed by (l, h): a [rows],
+    A_theta [rows, d]."""
+    L, Hkv, G, nq, d = Q.shape
+    sel = heads if heads is not None else [(l, h) for l in range(L) for h in range(Hkv)]
+    by_layer: Dict[int, List[int]] = {}
+    for (l, h) in sel:
+        by_layer.setdefault(l, []).append(h)
+    out_a, out_A = {}, {}
+    for l, hs in by_layer.items():
+        X = Q[l, hs].reshape(len(hs), G * nq, d)
+        bb = mods[l]["backbone"] if mods[l]["backbone"]["U"] else None
+        for net, dout in (("score", 1), ("target", d)):
+            params, widths = flatten_chain(bb, mods[l][net], hs)
+            Y = chain(params, X, widths, dout)
             for j, h in enumerate(hs):
                 if net == "score":
                     out_a[(l, h)] = Y[j, :, 0]

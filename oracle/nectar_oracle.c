@@ -146,6 +146,74 @@ void oracle_mlp(int64_t units, int64_t rows, int d, int depth, int H, int dout,
 }
 
 /*
+ * A chain of `nl` hidden layers of the Eq. (3.6) recursion with its own
+ * width per layer, then the linear readout -- the shape of a score or a
+ * target net when a backbone is shared (§2.4, App. A.3: depths
+ * (D_b, D_s, D_t)).  Layer 0 sees only q, layer k >= 1 sees q and layer
+ * k - 1 (width W[k-1]):
+ *   h_0 = SiLU(U_0 q + b_0),  h_k = SiLU(V_k q + U_k h_{k-1} + b_k).
+ * params per unit, in order:
+ *   U_0 [W0][d], b_0 [W0],
+ *   for k = 1..nl-1:  V_k [Wk][d], U_k [Wk][W(k-1)], b_k [Wk],
+ *   W_out [dout][W(nl-1)], c [dout]
+ */
+int64_t oracle_chain_param_count(int d, int nl, const int *W, int dout) {
+    int64_t P = (int64_t)W[0] * d + W[0];
+    for (int k = 1; k < nl; ++k) P += (int64_t)W[k] * d + (int64_t)W[k] * W[k - 1] + W[k];
+    return P + (int64_t)dout * W[nl - 1] + dout;
+}
+
+void oracle_chain(int64_t units, int64_t rows, int d, int nl, const int *W, int dout,
+                  const double *params, const uint16_t *X, double *Y) {
+    int64_t P = oracle_chain_param_count(d, nl, W, dout);
+    int Wmax = 0;
+    for (int k = 0; k < nl; ++k) Wmax = W[k] > Wmax ? W[k] : Wmax;
+    int64_t items = units * rows;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t it = 0; it < items; ++it) {
+        int64_t u = it / rows;
+        const double *p = params + u * P;
+        const uint16_t *xq = X + it * d;
+        double *q = (double *)malloc(sizeof(double) * d);
+        double *h = (double *)malloc(sizeof(double) * Wmax);
+        double *hn = (double *)malloc(sizeof(double) * Wmax);
+        for (int c = 0; c < d; ++c) q[c] = bf16_to_double(xq[c]);
+        const double *U0 = p;
+        const double *b0 = U0 + (int64_t)W[0] * d;
+        for (int i = 0; i < W[0]; ++i) {
+            double z = b0[i];
+            for (int c = 0; c < d; ++c) z += U0[(int64_t)i * d + c] * q[c];
+            h[i] = silu(z);
+        }
+        p = b0 + W[0];
+        for (int k = 1; k < nl; ++k) {
+            const int Hk = W[k], Hp = W[k - 1];
+            const double *Vk = p;
+            const double *Uk = Vk + (int64_t)Hk * d;
+            const double *bk = Uk + (int64_t)Hk * Hp;
+            for (int i = 0; i < Hk; ++i) {
+                double z = bk[i];
+                for (int c = 0; c < d; ++c) z += Vk[(int64_t)i * d + c] * q[c];
+                for (int j = 0; j < Hp; ++j) z += Uk[(int64_t)i * Hp + j] * h[j];
+                hn[i] = silu(z);
+            }
+            memcpy(h, hn, sizeof(double) * Hk);
+            p = bk + Hk;
+        }
+        const int Hl = W[nl - 1];
+        const double *Wo = p;
+        const double *cb = Wo + (int64_t)dout * Hl;
+        double *y = Y + it * dout;
+        for (int o = 0; o < dout; ++o) {
+            double z = cb[o];
+            for (int j = 0; j < Hl; ++j) z += Wo[(int64_t)o * Hl + j] * h[j];
+            y[o] = z;
+        }
+        free(q); free(h); free(hn);
+    }
+}
+
+/*
  * Visible local set of a query token (§2.2): local tokens i of its sequence
  * with i <= t (t = its local position, the token itself included) and
  * i < local_len.  Returns the count of visible tokens.

@@ -453,3 +453,142 @@ def test_fit_metrics_special_cases_and_scaling():
     # heads are independent: the metrics of a head do not see the others
     out_h, _ = oracle.fit_metrics(alpha[1:2], A[1:2], alpha[1:2] + 0.5, A[1:2] + E[1:2], Q[1:2])
     assert np.array_equal(out_h[0], out1[1])
+
+
+# ---------------------------------------------------------------------------
+# (ii) with a shared backbone: depths (D_b, D_s, D_t) and per-net widths
+# (App. A.3, Eq. (3.6)).  The oracle runs each net as one chain (backbone
+# layers, then the branch, then the readout).
+# ---------------------------------------------------------------------------
+def _general(L, Hkv, d, depths, wb, ws, wt, seed):
+    from nectar_inputs import make_modules_general
+    return make_modules_general(L, Hkv, d, seed, "cpu", depths, wb, ws, wt)
+
+
+def _torch_general_forward(mods, Q):
+    """The backbone run once with torch fp64 linear + silu, its last state
+    handed to both branches (an independent implementation)."""
+    L, Hkv, G, nq, d = Q.shape
+    a, A = {}, {}
+    for l in range(L):
+        for h in range(Hkv):
+            q = Q[l, h].reshape(G * nq, d).double()
+            bb = mods[l]["backbone"]
+            x = None
+            for k in range(len(bb["U"])):
+                z = F.linear(q, bb["U"][k][h].double(), bb["b"][k][h].double()) if k == 0 else \
+                    F.linear(q, bb["V"][k][h].double()) + F.linear(x, bb["U"][k][h].double(), bb["b"][k][h].double())
+                x = F.silu(z)
+            outs = []
+            for net in ("score", "target"):
+                nt = mods[l][net]
+                y = x
+                for k in range(len(nt["U"])):
+                    if nt["V"][k] is None:
+                        z = F.linear(q, nt["U"][k][h].double(), nt["b"][k][h].double())
+                    else:
+                        z = F.linear(q, nt["V"][k][h].double()) + F.linear(y, nt["U"][k][h].double(),
+                                                                          nt["b"][k][h].double())
+                    y = F.silu(z)
+                outs.append(F.linear(y, nt["Wout"][h].double(), nt["c"][h].double()).numpy())
+            a[(l, h)] = outs[0][:, 0]
+            A[(l, h)] = outs[1]
+    return a, A
+
+
+def test_general_module_without_backbone_is_the_separate_nets():
+    # D_b = 0, equal widths: the chain oracle gives the (pinned) per-net MLP
+    wl = make_workload("toy", L=2, Hkv=2, G=2, n=16, nq=3, with_local=False, with_modules=True,
+                       widths=[32, 48], seed=5)
+    mods = _general(2, 2, 128, (0, 2, 2), [0, 0], [32, 48], [32, 48], seed=5)
+    a, A = oracle.module_forward_general(mods, wl.Q)
+    a0, A0 = oracle.module_forward(wl)
+    for key in a0:
+        np.testing.assert_array_equal(a[key], a0[key])
+        np.testing.assert_array_equal(A[key], A0[key])
+
+
+@pytest.mark.parametrize("depths,wb,ws,wt", [((2, 1, 2), [48, 32], [32, 16], [16, 64]),
+                                            ((0, 2, 3), [0, 0], [16, 48], [64, 32]),
+                                            ((1, 1, 1), [64, 16], [32, 32], [48, 16])])
+def test_general_module_against_torch(depths, wb, ws, wt):
+    g = torch.Generator().manual_seed(7)
+    Q = torch.randn(2, 2, 2, 3, 128, generator=g).to(torch.bfloat16)
+    mods = _general(2, 2, 128, depths, wb, ws, wt, seed=11)
+    a, A = oracle.module_forward_general(mods, Q)
+    ta, tA = _torch_general_forward(mods, Q)
+    for key in a:
+        np.testing.assert_allclose(a[key], ta[key], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(A[key], tA[key], rtol=1e-12, atol=1e-12)
+
+
+def test_general_module_brute_force_tiny():
+    # d = 4, widths 3 / 2 / 5, depths (2, 1, 2): plain Python with math.fsum
+    d = 4
+    g = torch.Generator().manual_seed(3)
+    Q = torch.randn(1, 1, 1, 2, d, generator=g).to(torch.bfloat16)
+    mods = _general(1, 1, d, (2, 1, 2), [3], [2], [5], seed=13)
+    a, A = oracle.module_forward_general(mods, Q)
+
+    def silu(z):
+        return z / (1.0 + math.exp(-z))
+
+    def lin(W, x, b=None):
+        W = W.double().tolist()
+        out = [math.fsum(W[i][j] * x[j] for j in range(len(x))) for i in range(len(W))]
+        if b is not None:
+            out = [o + float(bb) for o, bb in zip(out, b.double().tolist())]
+        return out
+
+    for t in range(2):
+        q = Q[0, 0, 0, t].double().tolist()
+        bb = mods[0]["backbone"]
+        x = [silu(z) for z in lin(bb["U"][0][0], q, bb["b"][0][0])]
+        x = [silu(u + v) for u, v in zip(lin(bb["V"][1][0], q), lin(bb["U"][1][0], x, bb["b"][1][0]))]
+        res = []
+        for net in ("score", "target"):
+            nt = mods[0][net]
+            y = x
+            for k in range(len(nt["U"])):
+                y = [silu(u + v) for u, v in zip(lin(nt["V"][k][0], q), lin(nt["U"][k][0], y, nt["b"][k][0]))]
+            res.append(lin(nt["Wout"][0], y, nt["c"][0]))
+        assert abs(a[(0, 0)][t] - res[0][0]) <= 1e-12
+        np.testing.assert_allclose(A[(0, 0)][t], res[1], rtol=0, atol=1e-12)
+
+
+def test_general_module_zero_weights_closed_form():
+    # U = V = 0: every layer is SiLU of its bias; the readout is W_out SiLU(b_last) + c
+    mods = _general(1, 2, 128, (2, 1, 2), [32], [16], [48], seed=17)
+    for part in ("backbone", "score", "target"):
+        for k in range(len(mods[0][part]["U"])):
+            mods[0][part]["U"][k] = torch.zeros_like(mods[0][part]["U"][k])
+            if mods[0][part]["V"][k] is not None:
+                mods[0][part]["V"][k] = torch.zeros_like(mods[0][part]["V"][k])
+    Q = torch.randn(1, 2, 1, 4, 128, generator=torch.Generator().manual_seed(2)).to(torch.bfloat16)
+    a, A = oracle.module_forward_general(mods, Q)
+    for h in range(2):
+        for net, out in (("score", a), ("target", A)):
+            nt = mods[0][net]
+            s = F.silu(nt["b"][-1][h].double())
+            want = (nt["Wout"][h].double() @ s + nt["c"][h].double()).numpy()
+            got = out[(0, h)]
+            if net == "score":
+                np.testing.assert_allclose(got, np.full(4, want[0]), rtol=1e-14, atol=1e-14)
+            else:
+                np.testing.assert_allclose(got, np.tile(want, (4, 1)), rtol=1e-14, atol=1e-14)
+
+
+def test_general_module_routes_backbone_to_both_branches():
+    # changing a branch moves only its own output; changing the backbone moves both
+    Q = torch.randn(1, 1, 2, 3, 128, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
+    mods = _general(1, 1, 128, (2, 1, 2), [32], [16], [32], seed=19)
+    a0, A0 = oracle.module_forward_general(mods, Q)
+    mods[0]["score"]["b"][0] = mods[0]["score"]["b"][0] + 0.5
+    a1, A1 = oracle.module_forward_general(mods, Q)
+    assert not np.allclose(a1[(0, 0)], a0[(0, 0)]) and np.array_equal(A1[(0, 0)], A0[(0, 0)])
+    mods[0]["target"]["b"][1] = mods[0]["target"]["b"][1] + 0.5
+    a2, A2 = oracle.module_forward_general(mods, Q)
+    assert np.array_equal(a2[(0, 0)], a1[(0, 0)]) and not np.allclose(A2[(0, 0)], A1[(0, 0)])
+    mods[0]["backbone"]["b"][1] = mods[0]["backbone"]["b"][1] + 0.5
+    a3, A3 = oracle.module_forward_general(mods, Q)
+    assert not np.allclose(a3[(0, 0)], a2[(0, 0)]) and not np.allclose(A3[(0, 0)], A2[(0, 0)])
