@@ -148,11 +148,32 @@ NECTAR_API nectar_status nectar_cache_attn_lse_static(nectar_dims dims, const ne
  * layout is private to the library (tiled for TMA); size it with
  * nectar_module_packed_elems.
  * ------------------------------------------------------------------------ */
+/* Module sets with a shared backbone and nets of their own depth and
+ * width ("Nectar", §2.4 and App. A.3: depths (D_b, D_s, D_t)).  The
+ * backbone is D_b layers of the recursion above (width width_b[l]); the
+ * score branch continues it from the backbone's last hidden state with
+ * depth_s layers of width width_s[l] (its first layer sees q and that
+ * state: g_0 = SiLU(V_0 q + U_0 h_{D_b - 1} + b_0)), then the score
+ * readout; the target branch likewise (depth_t, width_t[l]).  With
+ * depth_b = 0 each branch starts from q alone, so depth_b = 0 with equal
+ * branches is the classic set above. */
 typedef struct {
-  int32_t depth;          /* hidden layers per net, 1..NECTAR_MAX_DEPTH */
-  const int32_t *width;   /* HOST [L]: H_l, a multiple of 16 in [16, 1024] */
+  int32_t depth_b;          /* backbone layers, 0..NECTAR_MAX_DEPTH - 1 */
+  int32_t depth_s, depth_t; /* branch layers, >= 1; depth_b + max(depth_s, depth_t) <= NECTAR_MAX_DEPTH */
+  const int32_t *width_b;   /* HOST [L], multiples of 16 in [16, 1024]; may be NULL when depth_b = 0 */
+  const int32_t *width_s;   /* HOST [L] */
+  const int32_t *width_t;   /* HOST [L] */
+} nectar_module_arch;
+
+typedef struct {
+  int32_t depth;          /* hidden layers per net, 1..NECTAR_MAX_DEPTH (classic sets) */
+  const int32_t *width;   /* HOST [L]: H_l, a multiple of 16 in [16, 1024] (classic sets) */
   const nectar_bf16 *weights;   /* DEVICE packed blob */
   int64_t weights_elems;  /* bf16 elements in the blob */
+  const nectar_module_arch *arch;   /* HOST; NULL: the classic set (depth, width); else the
+                                       architecture, and depth / width are not read.  Sets
+                                       with a backbone or unequal branches run layer by layer
+                                       (grouped GEMMs) whatever the number of query rows. */
 } nectar_module_set;
 
 /* Plain row-major HOST tensors of one net for all Hkv heads of a layer. */
@@ -163,6 +184,21 @@ typedef struct {
   const nectar_bf16 *Wout;                /* [Hkv][dout][H] */
   const nectar_bf16 *c;                   /* [Hkv][dout] */
 } nectar_net_host;
+
+/* Elements of the packed blob of an architecture (0 on invalid arguments). */
+NECTAR_API int64_t nectar_module_packed_elems_arch(nectar_dims dims, const nectar_module_arch *arch);
+
+/* Pack HOST tensors of an architecture into a HOST blob.  nets: HOST
+ * [L][3] -- nets[3*l + 0] the backbone (U, V, b of its depth_b layers;
+ * Wout, c unused), nets[3*l + 1] the score branch, nets[3*l + 2] the target
+ * branch.  Branch layer j: U[j] [Hkv][H][P] with P the width of the layer
+ * before it (the backbone's for j = 0) and V[j] [Hkv][H][d] -- except for a
+ * layer that starts a chain (the backbone's layer 0, or a branch's layer 0
+ * when depth_b = 0), whose U is [Hkv][H][d] (it multiplies q) and whose V
+ * is unused.  Padding in the blob is written as zeros. */
+NECTAR_API nectar_status nectar_module_pack_arch(nectar_dims dims, const nectar_module_arch *arch,
+                                      const nectar_net_host *nets, nectar_bf16 *blob,
+                                      int64_t blob_elems);
 
 /* Elements of the packed blob for these widths (0 on invalid arguments). */
 NECTAR_API int64_t nectar_module_packed_elems(nectar_dims dims, int32_t depth, const int32_t *width);
@@ -179,18 +215,21 @@ NECTAR_API nectar_status nectar_module_pack(nectar_dims dims, int32_t depth, con
  *   a[row]       = a_theta(q)     DEVICE fp32 [L][Hkv][G][nq]
  *   A_theta[row] = A_theta(q)     DEVICE fp32 [L][Hkv][G][nq][d]
  * Runs on the tensor cores (tcgen05, bf16 operands, fp32 accumulation);
- * hidden activations are rounded to bf16 between layers.  Fewer than 128
- * query rows per KV head: one launch, each CTA carrying <= 64 rows through
- * all layers in shared memory (workspace unused, may be NULL).  More rows:
+ * hidden activations are rounded to bf16 between layers.  Fewer than 64
+ * query rows per KV head (classic sets): one launch, each CTA carrying
+ * <= 64 rows through all layers in shared memory (workspace unused, may be
+ * NULL).  More rows, or a set with a backbone or unequal branches:
  * one grouped-GEMM launch per hidden layer plus one for the readouts, the
  * hidden activations kept in `workspace` (DEVICE, 256-byte aligned, owned
  * by the caller, overwritten; NECTAR_ERR_WORKSPACE when missing or small).
  * ------------------------------------------------------------------------ */
-/* Workspace of nectar_module_forward, in bytes: 0 when the KV heads have
- * fewer than 64 query rows (G * nq), else the hidden activations of the
- * layer-by-layer path, (depth >= 2 ? 2 : 1) * align256(2 * rows * Hp * 2)
- * + align256(rows * ceil(Hmax / 128) * 4), with rows = L * Hkv * G * nq,
- * Hmax the widest layer and Hp = Hmax rounded up to 64. */
+/* Workspace of nectar_module_forward, in bytes: 0 when the one-launch path
+ * runs (classic sets, fewer than 64 query rows G * nq per KV head), else
+ * the hidden activations of the layer-by-layer path,
+ * (S >= 2 ? 2 : 1) * align256(2 * rows * Hp * 2) + align256(rows * ceil(Hsmax / 128) * 4),
+ * with rows = L * Hkv * G * nq, S the hidden layers of the longest chain
+ * (depth, or depth_b + max(depth_s, depth_t)), Hp the widest layer of any
+ * part rounded up to 64 and Hsmax the widest score net. */
 NECTAR_API size_t nectar_module_workspace_size(nectar_dims dims, const nectar_module_set *mods,
                                                int64_t nq);
 NECTAR_API nectar_status nectar_module_forward(nectar_dims dims, const nectar_module_set *mods,

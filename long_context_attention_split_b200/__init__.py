@@ -41,9 +41,16 @@ class Dims(ctypes.Structure):
     _fields_ = [("L", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("G", ctypes.c_int32), ("d", ctypes.c_int32)]
 
 
+class _ArchC(ctypes.Structure):
+    _fields_ = [("depth_b", ctypes.c_int32), ("depth_s", ctypes.c_int32), ("depth_t", ctypes.c_int32),
+                ("width_b", ctypes.POINTER(ctypes.c_int32)), ("width_s", ctypes.POINTER(ctypes.c_int32)),
+                ("width_t", ctypes.POINTER(ctypes.c_int32))]
+
+
 class _ModuleSetC(ctypes.Structure):
     _fields_ = [("depth", ctypes.c_int32), ("width", ctypes.POINTER(ctypes.c_int32)),
-                ("weights", ctypes.c_void_p), ("weights_elems", ctypes.c_int64)]
+                ("weights", ctypes.c_void_p), ("weights_elems", ctypes.c_int64),
+                ("arch", ctypes.POINTER(_ArchC))]
 
 
 class _NetHostC(ctypes.Structure):
@@ -75,6 +82,10 @@ def lib() -> ctypes.CDLL:
     L.nectar_module_packed_elems.restype = I64
     L.nectar_module_pack.argtypes = [Dims, I32, P, P, P, I64]
     L.nectar_module_pack.restype = S
+    L.nectar_module_packed_elems_arch.argtypes = [Dims, ctypes.POINTER(_ArchC)]
+    L.nectar_module_packed_elems_arch.restype = I64
+    L.nectar_module_pack_arch.argtypes = [Dims, ctypes.POINTER(_ArchC), P, P, I64]
+    L.nectar_module_pack_arch.restype = S
     L.nectar_module_workspace_size.argtypes = [Dims, ctypes.POINTER(_ModuleSetC), I64]
     L.nectar_module_workspace_size.restype = ctypes.c_size_t
     L.nectar_module_forward.argtypes = [Dims, ctypes.POINTER(_ModuleSetC), P, I64, P, P, P, ctypes.c_size_t, P]
@@ -209,17 +220,47 @@ STATIC_SCRATCH_BYTES = 48 << 20
 # ---------------------------------------------------------------------------
 # module set
 # ---------------------------------------------------------------------------
-class ModuleSet:
-    """A packed module set on the device (nectar_module_set)."""
+class Arch:
+    """Depths (D_b, D_s, D_t) and per-layer widths of a module set with a
+    shared backbone (nectar_module_arch)."""
 
-    def __init__(self, blob: torch.Tensor, widths: Sequence[int], depth: int, L: int, Hkv: int):
+    def __init__(self, depths: Sequence[int], width_b: Sequence[int], width_s: Sequence[int],
+                 width_t: Sequence[int]):
+        self.depths = tuple(int(x) for x in depths)
+        self.width_b = [int(w) for w in width_b]
+        self.width_s = [int(w) for w in width_s]
+        self.width_t = [int(w) for w in width_t]
+        i32 = ctypes.POINTER(ctypes.c_int32)
+        self._wb = (ctypes.c_int32 * max(len(self.width_b), 1))(*self.width_b)
+        self._ws = (ctypes.c_int32 * len(self.width_s))(*self.width_s)
+        self._wt = (ctypes.c_int32 * len(self.width_t))(*self.width_t)
+        self._c = _ArchC(self.depths[0], self.depths[1], self.depths[2], ctypes.cast(self._wb, i32),
+                         ctypes.cast(self._ws, i32), ctypes.cast(self._wt, i32))
+
+    def layers(self, lo: int, hi: int) -> "Arch":
+        return Arch(self.depths, self.width_b[lo:hi] if self.depths[0] else [], self.width_s[lo:hi],
+                    self.width_t[lo:hi])
+
+    def packed_elems(self, Hkv: int, d: int = 128) -> int:
+        return int(lib().nectar_module_packed_elems_arch(Dims(len(self.width_s), Hkv, 1, d), ctypes.byref(self._c)))
+
+
+class ModuleSet:
+    """A packed module set on the device (nectar_module_set): the classic
+    one (both nets `depth` layers of `widths`) or, with `arch`, one with a
+    shared backbone and nets of their own depths and widths."""
+
+    def __init__(self, blob: torch.Tensor, widths: Sequence[int], depth: int, L: int, Hkv: int,
+                 arch: Optional[Arch] = None):
         self.blob = blob
         self.widths = [int(w) for w in widths]
         self.depth = int(depth)
         self.L, self.Hkv = L, Hkv
-        self._w = (ctypes.c_int32 * len(self.widths))(*self.widths)
+        self.arch = arch
+        self._w = (ctypes.c_int32 * max(len(self.widths), 1))(*self.widths)
         self._c = _ModuleSetC(self.depth, ctypes.cast(self._w, ctypes.POINTER(ctypes.c_int32)),
-                              blob.data_ptr(), blob.numel())
+                              blob.data_ptr(), blob.numel(),
+                              ctypes.pointer(arch._c) if arch is not None else None)
 
     def c(self):
         return ctypes.byref(self._c)
@@ -231,6 +272,11 @@ class ModuleSet:
     def layer(self, l: int) -> "ModuleSet":
         """The modules of layer l alone, as a one-layer set viewing the same
         blob (blocks are stored layer after layer)."""
+        if self.arch is not None:
+            off = self.arch.layers(0, l).packed_elems(self.Hkv) if l > 0 else 0
+            one = self.arch.layers(l, l + 1)
+            n = one.packed_elems(self.Hkv)
+            return ModuleSet(self.blob[off:off + n], self.widths[l:l + 1], self.depth, 1, self.Hkv, arch=one)
         off = packed_elems(l, self.Hkv, 1, self.widths[:l], self.depth) if l > 0 else 0
         n = packed_elems(1, self.Hkv, 1, self.widths[l:l + 1], self.depth)
         return ModuleSet(self.blob[off:off + n], self.widths[l:l + 1], self.depth, 1, self.Hkv)
@@ -275,6 +321,42 @@ def pack_modules(modules, widths: Sequence[int], depth: int, Hkv: int, G: int, d
     _check(st, "nectar_module_pack")
     dev_blob = blob.to(device) if device is not None else blob
     return ModuleSet(dev_blob, widths, depth, L_, Hkv)
+
+
+def pack_modules_arch(modules, arch: Arch, Hkv: int, G: int, d: int = 128, device="cuda") -> ModuleSet:
+    """Pack per-layer module sets with a shared backbone (dicts "backbone",
+    "score", "target" with U, V, b lists, and Wout, c for the branches; V[k]
+    None for a layer that starts a chain) with nectar_module_pack_arch and
+    copy the blob to `device`."""
+    L_ = len(modules)
+    dims = Dims(L_, Hkv, G, d)
+    total = int(lib().nectar_module_packed_elems_arch(dims, ctypes.byref(arch._c)))
+    if total <= 0:
+        raise NectarError(1, lib().nectar_last_error().decode())
+    blob = torch.zeros(total, dtype=torch.bfloat16)
+    keep = []
+    nets = (_NetHostC * (3 * L_))()
+
+    def ptr(t):
+        t = t.detach().cpu().contiguous()
+        keep.append(t)
+        return t.data_ptr()
+
+    for l, layer in enumerate(modules):
+        for j, name in enumerate(("backbone", "score", "target")):
+            part = layer[name]
+            nh = nets[3 * l + j]
+            for k in range(len(part["U"])):
+                nh.U[k] = ptr(part["U"][k])
+                nh.b[k] = ptr(part["b"][k])
+                if part["V"][k] is not None:
+                    nh.V[k] = ptr(part["V"][k])
+            if name != "backbone":
+                nh.Wout, nh.c = ptr(part["Wout"]), ptr(part["c"])
+    st = lib().nectar_module_pack_arch(dims, ctypes.byref(arch._c), nets, blob.data_ptr(), total)
+    _check(st, "nectar_module_pack_arch")
+    dev_blob = blob.to(device) if device is not None else blob
+    return ModuleSet(dev_blob, arch.width_s, arch.depths[1], L_, Hkv, arch=arch)
 
 
 # ---------------------------------------------------------------------------

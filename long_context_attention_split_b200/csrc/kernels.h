@@ -92,7 +92,9 @@ cudaError_t launch_merge_local(const MergeParams& p, cudaStream_t stream);
 // ----- (ii) module forward and the fused decode (tcgen05) ------------------
 constexpr int kModMaxLayers = 256;
 struct ModParams {
-  int Hkv, G, depth;
+  int Hkv, G, depth;            // depth: of both nets when the set has no backbone and equal nets
+  int depth_b, depth_s, depth_t;
+  bool general;                 // a backbone, or unequal nets: layer-by-layer path only
   int64_t nq;
   int N, TPC, nblk, Hmax, tmem_cols, stages, cps;
   const __nv_bfloat16* blob;
@@ -112,7 +114,9 @@ struct ModParams {
   int64_t n_local;      // decode: local CTAs (heads * nq) ahead of the module CTAs
   __nv_bfloat16* out_bf16;   // decode: if set, the output goes here, bf16 [L][nq][Hkv][G][d]
   int* err;
-  int32_t width[kModMaxLayers];
+  int32_t width[kModMaxLayers];        // score width (= target width unless general)
+  int32_t width_b[kModMaxLayers];
+  int32_t width_t[kModMaxLayers];
   int64_t layer_base[kModMaxLayers];   // blob element offset of layer l
   uint8_t order[kModMaxLayers];        // layers by decreasing width
 };
@@ -124,11 +128,12 @@ constexpr int kGemmMaxStages = 8;
 #endif
 constexpr int kGemmMinRows = NECTAR_GEMM_MIN_ROWS;
 struct GemmParams {
-  int L, Hkv, depth, stage, readout, nlayers;
+  int L, Hkv, stage, readout, nlayers;
+  int depth_b, depth_s, depth_t;   // backbone, score and target depths (depth_b = 0: separate nets)
   int R, NR, rtiles, Hp, MT, stages, tmem_cols;
   int64_t ntiles;
   const __nv_bfloat16* blob;
-  __nv_bfloat16* h_out;     // [2 nets][heads * R][Hp] bf16 (hidden stages)
+  __nv_bfloat16* h_out;     // [2 slots][heads * R][Hp] bf16 (hidden stages; the backbone uses slot 0)
   float* part;              // score partials [heads * R][MT]
   float* a_out;             // readout: [heads * R]
   float* A_out;             // readout: [heads * R][d] (A_theta, or the merged output)
@@ -137,7 +142,9 @@ struct GemmParams {
   int G;
   int64_t nq;
   int* err;
-  int32_t width[kModMaxLayers];
+  int32_t width_b[kModMaxLayers];   // backbone width of layer l (unused when depth_b = 0)
+  int32_t width_s[kModMaxLayers];   // score branch width
+  int32_t width_t[kModMaxLayers];   // target branch width
   int64_t layer_base[kModMaxLayers];
   int64_t tile_start[kModMaxLayers + 1];
   uint8_t order[kModMaxLayers];

@@ -81,9 +81,21 @@ __device__ __forceinline__ uint32_t gemm_silu2(uint32_t acc0, uint32_t acc1, flo
   return pack_bf16x2(y.x, y.y);
 }
 
+// One tile of the current launch: layer l, KV head hd, output part (0: the
+// backbone or the score branch, 1: the target branch; the readout is part
+// 1), 128-unit tile m, row tile rt -- and what the part's layer reads and
+// where its weights are.
 struct GemmTile {
-  int l, H, net, m, rt;
+  int l, net, m, rt;
   int64_t hd;
+  int H;            // output units of this layer (d for the readout)
+  int K;            // reduction length: d + the width of the h it reads (readout: the target width)
+  int in_slot;      // h slot read for the columns past d
+  int64_t w_off;    // blob offset of the layer's tiled weights
+  int64_t b_off;    // blob offset of its bias
+  bool score_last;  // the score branch's last layer: its readout is fused
+  int64_t score_base;   // blob offset of the score branch
+  int Hs;           // score width (readout: the number of partials per row)
 };
 
 __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int64_t t) {
@@ -91,17 +103,56 @@ __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int64_t t) {
   while (li + 1 < p.nlayers && t >= p.tile_start[li + 1]) ++li;
   GemmTile g;
   g.l = p.order[li];
-  g.H = p.width[g.l];
-  const int mt = p.readout ? 1 : (g.H + 127) / 128;
-  const int nets = p.readout ? 1 : 2;
+  const int Db = p.depth_b, Ds = p.depth_s, Dt = p.depth_t;
+  const int Hb = p.width_b[g.l], Hs = p.width_s[g.l], Ht = p.width_t[g.l];
+  const int s = p.stage;
+  const int j = s - Db;                                   // branch layer (s >= Db)
+  int mt0, mt1;
+  if (p.readout) {
+    mt0 = 0;
+    mt1 = 1;
+  } else if (s < Db) {
+    mt0 = (Hb + 127) / 128;
+    mt1 = 0;
+  } else {
+    mt0 = j < Ds ? (Hs + 127) / 128 : 0;
+    mt1 = j < Dt ? (Ht + 127) / 128 : 0;
+  }
   int64_t rem = t - p.tile_start[li];
   g.rt = static_cast<int>(rem % p.rtiles);
   rem /= p.rtiles;
-  g.m = static_cast<int>(rem % mt);
-  rem /= mt;
-  g.net = p.readout ? 1 : static_cast<int>(rem % nets);
-  const int h = static_cast<int>(rem / nets);
+  const int mm = static_cast<int>(rem % (mt0 + mt1));
+  const int h = static_cast<int>(rem / (mt0 + mt1));
+  g.net = mm < mt0 ? 0 : 1;
+  g.m = g.net ? mm - mt0 : mm;
   g.hd = static_cast<int64_t>(g.l) * p.Hkv + h;
+  const int64_t hb = p.layer_base[g.l] + static_cast<int64_t>(h) * layout::head_elems_arch(Db, Hb, Ds, Hs, Dt, Ht);
+  g.score_base = hb + layout::branch_base(Db, Hb, Ds, Hs, 0);
+  g.Hs = Hs;
+  g.score_last = false;
+  if (p.readout) {
+    const int64_t tb = hb + layout::branch_base(Db, Hb, Ds, Hs, 1);
+    g.H = kD;
+    g.K = Ht;
+    g.in_slot = 1;
+    g.w_off = tb + layout::branch_out_w_off(Db, Hb, Ht, Dt);
+    g.b_off = tb + layout::branch_out_b_off(Db, Hb, Ht, Dt, kD);
+  } else if (s < Db) {
+    g.H = Hb;
+    g.K = kD + (s > 0 ? Hb : 0);
+    g.in_slot = 0;
+    g.w_off = hb + layout::backbone_w_off(Hb, s);
+    g.b_off = g.w_off + layout::chunked_elems(Hb, g.K);
+  } else {
+    const int Hn = g.net ? Ht : Hs;
+    const int64_t nb = hb + layout::branch_base(Db, Hb, Ds, Hs, g.net);
+    g.H = Hn;
+    g.K = kD + layout::branch_prev(Db, Hb, Hn, j);
+    g.in_slot = j == 0 ? 0 : g.net;                         // a branch's first layer reads the backbone
+    g.w_off = nb + layout::branch_w_off(Db, Hb, Hn, j);
+    g.b_off = nb + layout::branch_b_off(Db, Hb, Hn, j);
+    g.score_last = g.net == 0 && j == Ds - 1;
+  }
   return g;
 }
 
@@ -172,16 +223,13 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       bool ok = true;
       for (int64_t t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x) {
         const GemmTile g = gemm_tile(p, t);
-        const int64_t nb = p.layer_base[g.l] + (g.hd - static_cast<int64_t>(g.l) * p.Hkv) * layout::head_elems(g.H, p.depth) +
-                           (g.net ? layout::net_elems(g.H, p.depth, 1) : 0);
-        const int rows = p.readout ? kD : g.H;
-        const int K = p.readout ? g.H : layout::hidden_k(g.H, p.stage);
+        const int rows = g.H;
+        const int K = g.K;
         const int kc = layout::kchunks(K);
-        const __nv_bfloat16* wbase =
-            p.blob + nb + (p.readout ? layout::out_w_off(g.H, p.depth) : layout::hidden_w_off(g.H, p.depth, p.stage));
+        const __nv_bfloat16* wbase = p.blob + g.w_off;
         const uint32_t wbytes = static_cast<uint32_t>(layout::tile_rows(rows, g.m)) * 128;
         const int qrow = static_cast<int>(g.hd * R + static_cast<int64_t>(g.rt) * NR);
-        const int hrow = static_cast<int>((g.net * heads + g.hd) * R + static_cast<int64_t>(g.rt) * NR);
+        const int hrow = static_cast<int>((g.in_slot * heads + g.hd) * R + static_cast<int64_t>(g.rt) * NR);
         const int qch = p.readout ? 0 : 2;             // leading chunks taken from q
         for (int c = 0; c < kc; ++c, ++it) {
           const uint32_t s = it % S;
@@ -205,8 +253,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       bool ok = true;
       for (int64_t t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x, ++tc) {
         const GemmTile g = gemm_tile(p, t);
-        const int K = p.readout ? g.H : layout::hidden_k(g.H, p.stage);
-        const int kc = layout::kchunks(K);
+        const int kc = layout::kchunks(g.K);
         const uint32_t b = tc & 1;
         if (tc >= 2 && !mbar_wait(b_acce + 8 * b, ((tc >> 1) - 1) & 1, p.err)) break;
         tc_fence_after();
@@ -240,8 +287,6 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     bool ok = true;
     for (int64_t t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++tc) {
       const GemmTile g = gemm_tile(p, t);
-      const int64_t hb = p.layer_base[g.l] + (g.hd - static_cast<int64_t>(g.l) * p.Hkv) * layout::head_elems(g.H, p.depth);
-      const int64_t nb = hb + (g.net ? layout::net_elems(g.H, p.depth, 1) : 0);
       const uint32_t b = tc & 1;
       const int r0 = g.rt * NR;
       // rows of this tile; a 32-column batch may run 16 columns past NR
@@ -249,12 +294,14 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       // per-thread constants, fetched before the accumulator is ready
       const int i = g.m * 128 + u;
       float bias = 0.f, wsc = 0.f;
-      const bool score_last = !p.readout && g.net == 0 && p.stage == p.depth - 1;
+      const bool score_last = g.score_last;
       if (p.readout) {
-        bias = __bfloat162float(p.blob[nb + layout::out_b_off(g.H, p.depth, kD) + u]);
+        bias = __bfloat162float(p.blob[g.b_off + u]);
       } else if (i < g.H) {
-        bias = __bfloat162float(p.blob[nb + layout::hidden_b_off(g.H, p.depth, p.stage) + i]);
-        if (score_last) wsc = __bfloat162float(p.blob[nb + layout::out_w_off(g.H, p.depth) + i]);
+        bias = __bfloat162float(p.blob[g.b_off + i]);
+        if (score_last)
+          wsc = __bfloat162float(
+              p.blob[g.score_base + layout::branch_out_w_off(p.depth_b, p.width_b[g.l], g.Hs, p.depth_s) + i]);
       }
       const float hbias = 0.5f * bias;
       if (ok) ok = mbar_wait_sleep(b_accf + 8 * b, (tc >> 1) & 1, p.err);   // waits out a main loop
@@ -311,9 +358,10 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
             const int r = r0 + n0 + lane;
             if (r < rend) {
               const float* pr = p.part + (g.hd * R + r) * p.MT;
-              const int mts = (g.H + 127) / 128;
+              const int mts = (g.Hs + 127) / 128;
               for (int m = 0; m < mts; ++m) a_l += pr[m];
-              a_l += __bfloat162float(p.blob[hb + layout::out_b_off(g.H, p.depth, 1)]);
+              a_l += __bfloat162float(
+                  p.blob[g.score_base + layout::branch_out_b_off(p.depth_b, p.width_b[g.l], g.Hs, p.depth_s, 1)]);
               if (q4 == 0 && p.a_out != nullptr) p.a_out[g.hd * R + r] = a_l;
             }
           }
@@ -398,8 +446,11 @@ GemmShape gemm_shape(int64_t R, int max_rows) {
   while (stages < kGemmMaxStages && gemm_smem_layout(sh.NR, stages + 1).total + 1024 <= kBudget) ++stages;
   sh.stages = stages;
   sh.smem = gemm_smem_layout(sh.NR, stages).total + 1024;
+  // two accumulators of NR columns; the epilogue reads in 32-column batches,
+  // so the second one's last batch may reach NR % 32 columns past 2 NR
+  const int need = 2 * sh.NR + (sh.NR % 32 ? 32 - sh.NR % 32 : 0);
   int c = 32;
-  while (c < 2 * sh.NR) c <<= 1;
+  while (c < need) c <<= 1;
   sh.tmem_cols = c;
   return sh;
 }

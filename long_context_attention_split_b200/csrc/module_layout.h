@@ -69,6 +69,51 @@ NECTAR_HD int64_t net_elems(int H, int depth, int dout) {
 }
 NECTAR_HD int64_t head_elems(int H, int depth) { return net_elems(H, depth, 1) + net_elems(H, depth, kDm); }
 
+// ---------------------------------------------------------------------------
+// Module sets with a shared backbone (depths Db, Ds, Dt; widths Hb, Hs, Ht
+// of one layer l).  Block of one (l, h):
+//   backbone: for k = 0..Db-1: W_k tiled [Hb][K], K = d (k = 0) or d + Hb; b_k
+//   score:    for j = 0..Ds-1: W_j tiled [Hs][d + P_j]; b_j; then w, c
+//   target:   for j = 0..Dt-1: W_j tiled [Ht][d + P_j]; b_j; then W_out, c
+// with P_0 = Hb (0 when Db = 0: the first layer then sees only q) and
+// P_j = the branch width for j >= 1.  With Db = 0 and equal branches this is
+// exactly the block above (head_elems), so either layout reads the other.
+// ---------------------------------------------------------------------------
+// input width (besides q) of layer j of a branch of width Hn
+NECTAR_HD int branch_prev(int Db, int Hb, int Hn, int j) { return j == 0 ? (Db > 0 ? Hb : 0) : Hn; }
+NECTAR_HD int64_t layer_elems(int H, int K) { return chunked_elems(H, K) + round64(H); }
+NECTAR_HD int64_t backbone_elems(int Db, int Hb) {
+  int64_t off = 0;
+  for (int k = 0; k < Db; ++k) off += layer_elems(Hb, k == 0 ? kDm : kDm + Hb);
+  return off;
+}
+// offset, inside the backbone, of the weights of layer k
+NECTAR_HD int64_t backbone_w_off(int Hb, int k) { return backbone_elems(k, Hb); }
+// offset, inside its branch, of the weights of layer j
+NECTAR_HD int64_t branch_w_off(int Db, int Hb, int Hn, int j) {
+  int64_t off = 0;
+  for (int jj = 0; jj < j; ++jj) off += layer_elems(Hn, kDm + branch_prev(Db, Hb, Hn, jj));
+  return off;
+}
+NECTAR_HD int64_t branch_b_off(int Db, int Hb, int Hn, int j) {
+  return branch_w_off(Db, Hb, Hn, j) + chunked_elems(Hn, kDm + branch_prev(Db, Hb, Hn, j));
+}
+// readout weights / bias of a branch with Dn layers (dout 1: score, d: target)
+NECTAR_HD int64_t branch_out_w_off(int Db, int Hb, int Hn, int Dn) { return branch_w_off(Db, Hb, Hn, Dn); }
+NECTAR_HD int64_t branch_out_b_off(int Db, int Hb, int Hn, int Dn, int dout) {
+  return branch_out_w_off(Db, Hb, Hn, Dn) + (dout == 1 ? round64(Hn) : chunked_elems(kDm, Hn));
+}
+NECTAR_HD int64_t branch_elems(int Db, int Hb, int Hn, int Dn, int dout) {
+  return branch_out_b_off(Db, Hb, Hn, Dn, dout) + (dout == 1 ? 64 : kDm);
+}
+// start of the score (net 0) or target (net 1) branch inside the block
+NECTAR_HD int64_t branch_base(int Db, int Hb, int Ds, int Hs, int net) {
+  return backbone_elems(Db, Hb) + (net ? branch_elems(Db, Hb, Hs, Ds, 1) : 0);
+}
+NECTAR_HD int64_t head_elems_arch(int Db, int Hb, int Ds, int Hs, int Dt, int Ht) {
+  return branch_base(Db, Hb, Ds, Hs, 1) + branch_elems(Db, Hb, Ht, Dt, kDm);
+}
+
 #undef NECTAR_HD
 }  // namespace layout
 }  // namespace nectar

@@ -483,6 +483,151 @@ static nectar_status check_modules_shape(const nectar_dims& dims, int32_t depth,
   return NECTAR_OK;
 }
 
+// The architecture of a module set: the classic one (both nets `depth`
+// layers of width[l], no backbone) or the one mods->arch gives.
+struct Arch {
+  int Db, Ds, Dt;
+  const int32_t* wb;   // null when Db = 0
+  const int32_t* ws;
+  const int32_t* wt;
+  bool general;        // a backbone or unequal nets: layer-by-layer path only
+};
+
+static nectar_status check_widths(const nectar_dims& dims, const int32_t* w, const char* what) {
+  if (w == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "%s is NULL", what);
+  for (int l = 0; l < dims.L; ++l)
+    if (w[l] < 16 || w[l] > NECTAR_MAX_WIDTH || w[l] % 16 != 0)
+      return fail(NECTAR_ERR_UNSUPPORTED, "%s[%d] = %d: need a multiple of 16 in [16, %d]", what, l, w[l],
+                  NECTAR_MAX_WIDTH);
+  return NECTAR_OK;
+}
+
+static nectar_status arch_check(const nectar_dims& dims, const nectar_module_arch* a, Arch* out) {
+  NECTAR_TRY(check_dims(dims));
+  if (a == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "arch is NULL");
+  if (dims.L > NECTAR_MAX_LAYERS) return fail(NECTAR_ERR_UNSUPPORTED, "L = %d > %d", dims.L, NECTAR_MAX_LAYERS);
+  if (a->depth_b < 0 || a->depth_s < 1 || a->depth_t < 1 ||
+      a->depth_b + (a->depth_s > a->depth_t ? a->depth_s : a->depth_t) > NECTAR_MAX_DEPTH)
+    return fail(NECTAR_ERR_UNSUPPORTED, "depths (%d, %d, %d): need depth_b >= 0, branches >= 1 and chains <= %d",
+                a->depth_b, a->depth_s, a->depth_t, NECTAR_MAX_DEPTH);
+  if (a->depth_b > 0) NECTAR_TRY(check_widths(dims, a->width_b, "width_b"));
+  NECTAR_TRY(check_widths(dims, a->width_s, "width_s"));
+  NECTAR_TRY(check_widths(dims, a->width_t, "width_t"));
+  out->Db = a->depth_b;
+  out->Ds = a->depth_s;
+  out->Dt = a->depth_t;
+  out->wb = a->depth_b > 0 ? a->width_b : nullptr;
+  out->ws = a->width_s;
+  out->wt = a->width_t;
+  bool eq = a->depth_b == 0 && a->depth_s == a->depth_t;
+  for (int l = 0; eq && l < dims.L; ++l) eq = a->width_s[l] == a->width_t[l];
+  out->general = !eq;
+  return NECTAR_OK;
+}
+
+static nectar_status arch_of(const nectar_dims& dims, const nectar_module_set* mods, Arch* out) {
+  if (mods == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "mods is NULL");
+  if (mods->arch != nullptr) return arch_check(dims, mods->arch, out);
+  NECTAR_TRY(check_modules_shape(dims, mods->depth, mods->width));
+  *out = Arch{0, mods->depth, mods->depth, nullptr, mods->width, mods->width, false};
+  return NECTAR_OK;
+}
+
+static int arch_hb(const Arch& a, int l) { return a.Db > 0 ? a.wb[l] : 0; }
+
+static int64_t arch_head_elems(const Arch& a, int l) {
+  return layout::head_elems_arch(a.Db, arch_hb(a, l), a.Ds, a.ws[l], a.Dt, a.wt[l]);
+}
+
+static int64_t arch_packed_elems(const nectar_dims& dims, const Arch& a) {
+  int64_t tot = 0;
+  for (int l = 0; l < dims.L; ++l) tot += static_cast<int64_t>(dims.Hkv) * arch_head_elems(a, l);
+  return tot;
+}
+
+// Writes one hidden layer of Hkv heads' weights into the tiled layout: the
+// logical matrix [H][d + P] takes its first d columns from Vq (or, for a
+// layer that starts a chain, P = 0, from U) and the rest from U [H][P].
+static void pack_hidden(nectar_bf16* W, nectar_bf16* bias, int h, int H, int P, const nectar_bf16* U,
+                        const nectar_bf16* Vq, const nectar_bf16* b) {
+  const int K = kD + P;
+  for (int i = 0; i < H; ++i)
+    for (int c = 0; c < K; ++c) {
+      nectar_bf16 v;
+      if (P == 0) v = U[(static_cast<int64_t>(h) * H + i) * kD + c];
+      else if (c < kD) v = Vq[(static_cast<int64_t>(h) * H + i) * kD + c];
+      else v = U[(static_cast<int64_t>(h) * H + i) * P + (c - kD)];
+      W[layout::chunked_index(H, K, c, i)] = v;
+    }
+  for (int i = 0; i < H; ++i) bias[i] = b[static_cast<int64_t>(h) * H + i];
+}
+
+int64_t nectar_module_packed_elems_arch(nectar_dims dims, const nectar_module_arch* arch) {
+  Arch a;
+  if (arch_check(dims, arch, &a) != NECTAR_OK) return 0;
+  return arch_packed_elems(dims, a);
+}
+
+nectar_status nectar_module_pack_arch(nectar_dims dims, const nectar_module_arch* arch, const nectar_net_host* nets,
+                                      nectar_bf16* blob, int64_t blob_elems) {
+  Arch a;
+  NECTAR_TRY(arch_check(dims, arch, &a));
+  if (nets == nullptr || blob == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "nets / blob is NULL");
+  const int64_t need = arch_packed_elems(dims, a);
+  if (blob_elems < need) return fail(NECTAR_ERR_INVALID_ARG, "blob has %lld elements, %lld needed",
+                                     (long long)blob_elems, (long long)need);
+  for (int l = 0; l < dims.L; ++l) {
+    const int depths[3] = {a.Db, a.Ds, a.Dt};
+    for (int part = 0; part < 3; ++part) {
+      const nectar_net_host& nh = nets[3 * l + part];
+      for (int k = 0; k < depths[part]; ++k) {
+        const bool starts = (part == 0 && k == 0) || (part > 0 && k == 0 && a.Db == 0);
+        if (nh.U[k] == nullptr || nh.b[k] == nullptr || (!starts && nh.V[k] == nullptr))
+          return fail(NECTAR_ERR_INVALID_ARG, "layer %d part %d: missing U/V/b[%d]", l, part, k);
+      }
+      if (part > 0 && (nh.Wout == nullptr || nh.c == nullptr))
+        return fail(NECTAR_ERR_INVALID_ARG, "layer %d part %d: missing Wout / c", l, part);
+    }
+  }
+  memset(blob, 0, sizeof(nectar_bf16) * need);
+  int64_t base = 0;
+  for (int l = 0; l < dims.L; ++l) {
+    const int Hb = arch_hb(a, l), Hs = a.ws[l], Ht = a.wt[l];
+    const int64_t per_head = arch_head_elems(a, l);
+    for (int h = 0; h < dims.Hkv; ++h) {
+      const int64_t hb = base + h * per_head;
+      const nectar_net_host& bb = nets[3 * l];
+      for (int k = 0; k < a.Db; ++k) {
+        nectar_bf16* W = blob + hb + layout::backbone_w_off(Hb, k);
+        const int P = k == 0 ? 0 : Hb;
+        pack_hidden(W, W + layout::chunked_elems(Hb, kD + P), h, Hb, P, bb.U[k], bb.V[k], bb.b[k]);
+      }
+      for (int net = 0; net < 2; ++net) {
+        const nectar_net_host& nh = nets[3 * l + 1 + net];
+        const int Hn = net ? Ht : Hs, Dn = net ? a.Dt : a.Ds, dout = net ? kD : 1;
+        const int64_t nb = hb + layout::branch_base(a.Db, Hb, a.Ds, Hs, net);
+        for (int j = 0; j < Dn; ++j) {
+          const int P = layout::branch_prev(a.Db, Hb, Hn, j);
+          pack_hidden(blob + nb + layout::branch_w_off(a.Db, Hb, Hn, j), blob + nb + layout::branch_b_off(a.Db, Hb, Hn, j),
+                      h, Hn, P, nh.U[j], nh.V[j], nh.b[j]);
+        }
+        nectar_bf16* Wo = blob + nb + layout::branch_out_w_off(a.Db, Hb, Hn, Dn);
+        if (dout == 1) {
+          for (int i = 0; i < Hn; ++i) Wo[i] = nh.Wout[static_cast<int64_t>(h) * Hn + i];
+        } else {
+          for (int o = 0; o < dout; ++o)
+            for (int c = 0; c < Hn; ++c)
+              Wo[layout::chunked_index(kD, Hn, c, o)] = nh.Wout[(static_cast<int64_t>(h) * dout + o) * Hn + c];
+        }
+        nectar_bf16* cb = blob + nb + layout::branch_out_b_off(a.Db, Hb, Hn, Dn, dout);
+        for (int o = 0; o < dout; ++o) cb[o] = nh.c[static_cast<int64_t>(h) * dout + o];
+      }
+    }
+    base += static_cast<int64_t>(dims.Hkv) * per_head;
+  }
+  return NECTAR_OK;
+}
+
 int64_t nectar_module_packed_elems(nectar_dims dims, int32_t depth, const int32_t* width) {
   if (check_modules_shape(dims, depth, width) != NECTAR_OK) return 0;
   int64_t tot = 0;
@@ -562,29 +707,41 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // that follow start 256-byte aligned)
 size_t decode_ws_a_bytes(int64_t rows) { return align256(static_cast<size_t>(rows) * sizeof(float)); }
 
-// Many query rows per KV head: the module runs layer by layer as grouped
-// GEMMs (module_gemm.cu) instead of one CTA per block of <= 64 rows.
-bool use_gemm_path(const nectar_dims& dims, int64_t nq) {
-  return static_cast<int64_t>(dims.G) * nq >= kGemmMinRows;
+// Many query rows per KV head, or a set with a backbone or unequal nets:
+// the module runs layer by layer as grouped GEMMs (module_gemm.cu) instead
+// of one CTA per block of <= 64 rows.
+bool use_gemm_path(const nectar_dims& dims, int64_t nq, bool general) {
+  return general || static_cast<int64_t>(dims.G) * nq >= kGemmMinRows;
 }
 
-int mods_hmax(const nectar_dims& dims, const int32_t* width) {
-  int Hmax = 0;
-  for (int l = 0; l < dims.L; ++l) Hmax = width[l] > Hmax ? width[l] : Hmax;
-  return Hmax;
+// widest layer of any part, widest score net, hidden layers of the longest chain
+int arch_hmax(const nectar_dims& dims, const Arch& a) {
+  int H = 0;
+  for (int l = 0; l < dims.L; ++l) {
+    H = std::max(H, std::max(a.ws[l], a.wt[l]));
+    if (a.Db > 0) H = std::max(H, a.wb[l]);
+  }
+  return H;
 }
+int arch_hsmax(const nectar_dims& dims, const Arch& a) {
+  int H = 0;
+  for (int l = 0; l < dims.L; ++l) H = std::max(H, a.ws[l]);
+  return H;
+}
+int arch_stages(const Arch& a) { return a.Db + std::max(a.Ds, a.Dt); }
 
 // Workspace of the layer-by-layer path: hidden activations (two buffers
-// when depth >= 2, each [2 nets][rows][Hp] bf16), then the score partials
-// [rows][MT] fp32.
+// when the longest chain has >= 2 layers, each [2 slots][rows][Hp] bf16),
+// then the score partials [rows][MT] fp32.
 size_t gemm_h_bytes(const nectar_dims& dims, int Hmax, int64_t nq) {
   const int64_t rows = static_cast<int64_t>(dims.L) * dims.Hkv * dims.G * nq;
   return align256(static_cast<size_t>(2 * rows) * layout::round64(Hmax) * 2);
 }
-size_t gemm_ws_bytes(const nectar_dims& dims, int Hmax, int depth, int64_t nq) {
+size_t gemm_ws_bytes(const nectar_dims& dims, const Arch& a, int64_t nq) {
   const int64_t rows = static_cast<int64_t>(dims.L) * dims.Hkv * dims.G * nq;
-  const int MT = (Hmax + 127) / 128;
-  return (depth >= 2 ? 2 : 1) * gemm_h_bytes(dims, Hmax, nq) + align256(static_cast<size_t>(rows) * MT * 4);
+  const int MT = (arch_hsmax(dims, a) + 127) / 128;
+  return (arch_stages(a) >= 2 ? 2 : 1) * gemm_h_bytes(dims, arch_hmax(dims, a), nq) +
+         align256(static_cast<size_t>(rows) * MT * 4);
 }
 
 // Rows per readout tile.  The readout has a single 128-dim M tile per head,
@@ -614,13 +771,17 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
   memset(&g, 0, sizeof(g));
   g.L = dims.L;
   g.Hkv = dims.Hkv;
-  g.depth = mp.depth;
+  g.depth_b = mp.depth_b;
+  g.depth_s = mp.depth_s;
+  g.depth_t = mp.depth_t;
   g.nlayers = dims.L;
   g.R = static_cast<int>(R);
   g.NR = sh.NR;
   g.rtiles = sh.rtiles;
   g.Hp = layout::round64(mp.Hmax);
-  g.MT = (mp.Hmax + 127) / 128;
+  int Hsmax = 0;
+  for (int l = 0; l < dims.L; ++l) Hsmax = std::max(Hsmax, mp.width[l]);
+  g.MT = (Hsmax + 127) / 128;
   g.stages = sh.stages;
   g.tmem_cols = sh.tmem_cols;
   g.blob = mp.blob;
@@ -628,15 +789,21 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
   g.G = dims.G;
   g.nq = nq;
   for (int l = 0; l < dims.L; ++l) {
-    g.width[l] = mp.width[l];
+    g.width_b[l] = mp.width_b[l];
+    g.width_s[l] = mp.width[l];
+    g.width_t[l] = mp.width_t[l];
     g.layer_base[l] = mp.layer_base[l];
     g.order[l] = mp.order[l];
   }
+  // hidden layers of the longest chain; the launches are stages 0..nst-1
+  // (stage s < depth_b: the backbone, else branch layer s - depth_b of the
+  // branches that have it), then the readout
+  const int nst = mp.depth_b + std::max(mp.depth_s, mp.depth_t);
   uint8_t* base = static_cast<uint8_t*>(ws);
   const size_t hb = gemm_h_bytes(dims, mp.Hmax, nq);
   __nv_bfloat16* hbuf[2] = {reinterpret_cast<__nv_bfloat16*>(base),
-                            reinterpret_cast<__nv_bfloat16*>(base + (mp.depth >= 2 ? hb : 0))};
-  g.part = reinterpret_cast<float*>(base + (mp.depth >= 2 ? 2 : 1) * hb);
+                            reinterpret_cast<__nv_bfloat16*>(base + (nst >= 2 ? hb : 0))};
+  g.part = reinterpret_cast<float*>(base + (nst >= 2 ? 2 : 1) * hb);
   CUtensorMap tq, th[2], thr;
   {
     const cuuint64_t dq[2] = {128, static_cast<cuuint64_t>(heads * R)};
@@ -652,11 +819,13 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
     const cuuint64_t dh[2] = {static_cast<cuuint64_t>(g.Hp), static_cast<cuuint64_t>(2 * heads * R)};
     const cuuint64_t shs[1] = {static_cast<cuuint64_t>(g.Hp) * 2};
     const cuuint32_t br[2] = {64, static_cast<cuuint32_t>(shr.NR)};
-    NECTAR_TRY(make_tmap(&thr, hbuf[(mp.depth - 1) & 1], 2, dh, shs, br, "hidden activations (readout)"));
+    // the target branch's last layer (stage depth_b + depth_t - 1) wrote its buffer
+    NECTAR_TRY(make_tmap(&thr, hbuf[(mp.depth_b + mp.depth_t - 1) & 1], 2, dh, shs, br,
+                         "hidden activations (readout)"));
   }
-  for (int stage = 0; stage <= mp.depth; ++stage) {
+  for (int stage = 0; stage <= nst; ++stage) {
     g.stage = stage;
-    g.readout = stage == mp.depth;
+    g.readout = stage == nst;
     g.h_out = g.readout ? nullptr : hbuf[stage & 1];
     g.a_out = g.readout ? a : nullptr;
     g.A_out = g.readout ? A_out : nullptr;
@@ -670,9 +839,13 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
     int64_t acc = 0;
     for (int li = 0; li < dims.L; ++li) {
       g.tile_start[li] = acc;
-      const int H = mp.width[mp.order[li]];
-      const int mt = g.readout ? 1 : (H + 127) / 128;
-      acc += static_cast<int64_t>(dims.Hkv) * (g.readout ? 1 : 2) * mt * ss.rtiles;
+      const int l = mp.order[li];
+      const int j = stage - mp.depth_b;
+      int mt;                                   // 128-unit tiles per head, as gemm_tile counts them
+      if (g.readout) mt = 1;
+      else if (j < 0) mt = (mp.width_b[l] + 127) / 128;
+      else mt = (j < mp.depth_s ? (mp.width[l] + 127) / 128 : 0) + (j < mp.depth_t ? (mp.width_t[l] + 127) / 128 : 0);
+      acc += static_cast<int64_t>(dims.Hkv) * mt * ss.rtiles;
     }
     g.tile_start[dims.L] = acc;
     g.ntiles = acc;
@@ -686,11 +859,11 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
 
 nectar_status prepare_modules(const nectar_dims& dims, const nectar_module_set* mods, const nectar_bf16* Q,
                               int64_t nq, bool fuse, ModParams* p, CUtensorMap* tq, ModShape* sh) {
-  if (mods == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "mods is NULL");
-  NECTAR_TRY(check_modules_shape(dims, mods->depth, mods->width));
+  Arch ar;
+  NECTAR_TRY(arch_of(dims, mods, &ar));
   if (dims.G > 64) return fail(NECTAR_ERR_UNSUPPORTED, "G = %d > 64", dims.G);
   NECTAR_TRY(check_ptr(mods->weights, "mods->weights"));
-  const int64_t need = nectar_module_packed_elems(dims, mods->depth, mods->width);
+  const int64_t need = arch_packed_elems(dims, ar);
   if (mods->weights_elems < need)
     return fail(NECTAR_ERR_INVALID_ARG, "weights_elems = %lld, the widths need %lld", (long long)mods->weights_elems,
                 (long long)need);
@@ -701,26 +874,33 @@ nectar_status prepare_modules(const nectar_dims& dims, const nectar_module_set* 
   memset(p, 0, sizeof(*p));
   p->Hkv = dims.Hkv;
   p->G = dims.G;
-  p->depth = mods->depth;
+  p->depth = ar.Ds;
+  p->depth_b = ar.Db;
+  p->depth_s = ar.Ds;
+  p->depth_t = ar.Dt;
+  p->general = ar.general;
   p->nq = nq;
   p->blob = reinterpret_cast<const __nv_bfloat16*>(mods->weights);
   p->Q = reinterpret_cast<const __nv_bfloat16*>(Q);
   p->err = di.err;
-  int Hmax = 0;
   int64_t base = 0;
+  std::vector<int> cost(dims.L);
   for (int l = 0; l < dims.L; ++l) {
-    p->width[l] = mods->width[l];
+    p->width[l] = ar.ws[l];
+    p->width_b[l] = arch_hb(ar, l);
+    p->width_t[l] = ar.wt[l];
     p->layer_base[l] = base;
-    base += static_cast<int64_t>(dims.Hkv) * layout::head_elems(mods->width[l], mods->depth);
-    if (mods->width[l] > Hmax) Hmax = mods->width[l];
+    base += static_cast<int64_t>(dims.Hkv) * arch_head_elems(ar, l);
+    cost[l] = std::max(std::max(ar.ws[l], ar.wt[l]), arch_hb(ar, l));
   }
   // widest layers first: their CTAs run longest
   std::vector<int> ord(dims.L);
   for (int l = 0; l < dims.L; ++l) ord[l] = l;
-  std::stable_sort(ord.begin(), ord.end(), [&](int a, int b) { return mods->width[a] > mods->width[b]; });
+  std::stable_sort(ord.begin(), ord.end(), [&](int a, int b) { return cost[a] > cost[b]; });
   for (int l = 0; l < dims.L; ++l) p->order[l] = static_cast<uint8_t>(ord[l]);
+  const int Hmax = arch_hmax(dims, ar);
   p->Hmax = Hmax;
-  if (use_gemm_path(dims, nq)) return NECTAR_OK;      // the layer-by-layer path needs no fused shape
+  if (use_gemm_path(dims, nq, ar.general)) return NECTAR_OK;   // the layer-by-layer path needs no fused shape
   *sh = mod_shape(dims.G, nq, Hmax, fuse);
   if (sh->smem > 227 * 1024) return fail(NECTAR_ERR_UNSUPPORTED, "width %d needs too much shared memory", Hmax);
   p->N = sh->N;
@@ -747,9 +927,10 @@ extern "C" {
 
 size_t nectar_module_workspace_size(nectar_dims dims, const nectar_module_set* mods, int64_t nq) {
   if (check_dims(dims) != NECTAR_OK || nq <= 0 || mods == nullptr) return 0;
-  if (check_modules_shape(dims, mods->depth, mods->width) != NECTAR_OK) return 0;
-  if (!use_gemm_path(dims, nq)) return 0;
-  return gemm_ws_bytes(dims, mods_hmax(dims, mods->width), mods->depth, nq);
+  Arch ar;
+  if (arch_of(dims, mods, &ar) != NECTAR_OK) return 0;
+  if (!use_gemm_path(dims, nq, ar.general)) return 0;
+  return gemm_ws_bytes(dims, ar, nq);
 }
 
 nectar_status nectar_module_forward(nectar_dims dims, const nectar_module_set* mods, const nectar_bf16* Q, int64_t nq,
@@ -765,8 +946,8 @@ nectar_status nectar_module_forward(nectar_dims dims, const nectar_module_set* m
   ModShape sh;
   NECTAR_TRY(prepare_modules(dims, mods, Q, nq, false, &p, &tq, &sh));
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (use_gemm_path(dims, nq)) {
-    const size_t need = gemm_ws_bytes(dims, p.Hmax, p.depth, nq);
+  if (use_gemm_path(dims, nq, p.general)) {
+    const size_t need = nectar_module_workspace_size(dims, mods, nq);
     if (workspace == nullptr || workspace_bytes < need)
       return fail(NECTAR_ERR_WORKSPACE, "module workspace of %zu bytes given, %zu needed",
                   workspace == nullptr ? size_t(0) : workspace_bytes, need);
@@ -783,16 +964,18 @@ nectar_status nectar_module_forward(nectar_dims dims, const nectar_module_set* m
 
 size_t nectar_decode_workspace_size(nectar_dims dims, const nectar_module_set* mods, int64_t nq) {
   if (check_dims(dims) != NECTAR_OK || nq <= 0 || mods == nullptr) return 0;
-  if (check_modules_shape(dims, mods->depth, mods->width) != NECTAR_OK) return 0;
+  Arch ar;
+  if (arch_of(dims, mods, &ar) != NECTAR_OK) return 0;
   const int64_t rows = static_cast<int64_t>(dims.L) * dims.Hkv * dims.G * nq;
   const size_t loc = align256(static_cast<size_t>(rows) * (kD + 2) * sizeof(float));
-  if (use_gemm_path(dims, nq)) return loc + gemm_ws_bytes(dims, mods_hmax(dims, mods->width), mods->depth, nq);
+  if (use_gemm_path(dims, nq, ar.general)) return loc + gemm_ws_bytes(dims, ar, nq);
   return decode_ws_a_bytes(rows) + loc;
 }
 
 size_t nectar_decode_layer_out_workspace_size(nectar_dims dims, const nectar_module_set* mods, int64_t nq) {
   const size_t base = nectar_decode_workspace_size(dims, mods, nq);
-  if (base == 0 || use_gemm_path(dims, nq)) return base;
+  Arch ar;
+  if (base == 0 || arch_of(dims, mods, &ar) != NECTAR_OK || use_gemm_path(dims, nq, ar.general)) return base;
   // the one-launch path keeps A_theta in fp32 until the merge
   const int64_t rows = static_cast<int64_t>(dims.L) * dims.Hkv * dims.G * nq;
   return base + align256(static_cast<size_t>(rows) * kD * sizeof(float));
@@ -814,8 +997,8 @@ nectar_status decode_impl(nectar_dims dims, const nectar_module_set* mods, const
   if (!(scale == scale)) return fail(NECTAR_ERR_INVALID_ARG, "scale is NaN");
   NECTAR_TRY(check_ptr(out != nullptr ? static_cast<const void*>(out) : static_cast<const void*>(out_bf16), "out"));
   NECTAR_TRY(check_local(q_seq, q_pos, Kloc, Vloc, B, T_max, local_len));
-  if (mods == nullptr) return fail(NECTAR_ERR_INVALID_ARG, "mods is NULL");
-  NECTAR_TRY(check_modules_shape(dims, mods->depth, mods->width));
+  Arch ar;
+  NECTAR_TRY(arch_of(dims, mods, &ar));
   const size_t need = out != nullptr ? nectar_decode_workspace_size(dims, mods, nq)
                                      : nectar_decode_layer_out_workspace_size(dims, mods, nq);
   if (workspace == nullptr || workspace_bytes < need)
@@ -829,7 +1012,7 @@ nectar_status decode_impl(nectar_dims dims, const nectar_module_set* mods, const
   NECTAR_TRY(prepare_modules(dims, mods, Q, nq, true, &p, &tq, &sh));
   const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
   const int64_t rows = heads * dims.G * nq;
-  const bool gemm = use_gemm_path(dims, nq);
+  const bool gemm = use_gemm_path(dims, nq, ar.general);
   if (heads * nq + (gemm ? 0 : static_cast<int64_t>(dims.L) * dims.Hkv * sh.nblk) > 0x7fffffffLL)
     return fail(NECTAR_ERR_UNSUPPORTED, "too many CTAs for one launch");
   p.q_seq = q_seq;

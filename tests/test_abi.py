@@ -127,3 +127,19 @@ def test_pack_layout(widths, depth, hkv):
     if depth >= 2 and (128 + H) % 64:
         W1, _ = read_chunked(blob, r64(0) + kch(128) * H * 64 + r64(H), H, r64(128 + H))
         assert np.all(W1[:, 128 + H:] == 0)
+
+
+def test_arch_packing_without_backbone_is_the_classic_blob():
+    # host-only: nectar_module_pack_arch with D_b = 0 and equal nets writes the
+    # classic nectar_module_pack blob, element for element
+    from nectar_inputs import make_modules, make_modules_general
+    import long_context_attention_split_b200 as nx
+    widths = [48, 32, 1024]
+    classic = nx.pack_modules(make_modules(3, 2, widths, 128, 5, "cpu", depth=3), widths, 3, 2, 2, device=None)
+    mods = make_modules_general(3, 2, 128, 5, "cpu", (0, 3, 3), [], widths, widths)
+    arch = nx.pack_modules_arch(mods, nx.Arch((0, 3, 3), [], widths, widths), 2, 2, device=None)
+    assert torch.equal(classic.blob, arch.blob)
+    # a backbone makes the blob bigger by exactly its layers
+    wb = [64, 16, 32]
+    with_bb = nx.Arch((1, 3, 3), wb, widths, widths)
+    assert with_bb.packed_elems(2) > nx.Arch((0, 3, 3), [], widths, widths).packed_elems(2)
