@@ -230,7 +230,15 @@ def run_ours(args):
     dwork = None
     if has_decode:
         dwork = torch.empty(nx.decode_workspace_size(mods, wl.G, wl.nq), dtype=torch.uint8, device=dev)
-    launches_per_step = 2 + (2 if has_decode else 0)   # (i) main kernel + combine; decode + its merge
+    # (i): main kernel + combine; decode: one launch + its merge, or with
+    # >= 64 rows per KV head the local kernel, one GEMM per hidden layer and the readout
+    if not has_decode:
+        dec_launches = 0
+    elif wl.rows >= 64:
+        dec_launches = 1 + wl.depth + 1
+    else:
+        dec_launches = 2
+    launches_per_step = 2 + dec_launches
 
     ev_a0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ev_a1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -294,6 +302,7 @@ def run_ours(args):
 
     # ---- the same step as L per-layer calls captured in one CUDA graph ----
     per_layer = per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args)
+    nextr = next_rows(wl, mods, alpha, A, has_decode, dev, hbm_peak, tc_peak) if args.next_rows else None
 
     # ---- end to end through the public API with host buffers ----
     pin = lambda t: t.cpu().pin_memory()
@@ -359,7 +368,7 @@ def run_ours(args):
                 "l2": l2_note(ab),
             },
             "parts": dict(parts(wl, attn_avg, dec_avg, ab, db, qps, hbm_peak, tc_peak, has_decode),
-                          per_layer_graph=per_layer),
+                          per_layer_graph=per_layer, **({"next_rows": nextr} if nextr else {})),
             "roofline": dict(kernel=("cache_attn_tc+combine" if wl.rows > 8 else "cache_attn_split+combine")
                              + " (exact alpha, A)", traffic=traffic, **roof),
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -397,6 +406,86 @@ def parts(wl, attn_ms, dec_ms, ab, db, qps, hbm_peak, tc_peak, has_decode):
         out["decode_frac_full"] = out["decode_roofline_us_full"] / (dec_ms * 1e3)
         out["decode_frac_weights_form"] = out["decode_roofline_us_weights"] / (dec_ms * 1e3)
     return out
+
+
+def _timed(fn, iters=10, warm=3):
+    """Median device time (ms) of fn() on the current stream, CUDA events."""
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(iters):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ts.sort()
+    return ts[len(ts) // 2]
+
+
+def next_rows(wl, mods, alpha, A, has_decode, dev, hbm_peak, tc_peak) -> dict:
+    """The rows after the hot path, each on this workload's shapes, timed
+    alone (inputs larger than L2 unless noted):
+      quadrature: the Quadrature module forward at p = 10% of n;
+      fit_metrics: score / target MSE and RTE over this step's targets;
+      backbone_decode: the decode with a (2, 1, 2) module set (backbone,
+        score, target depths) of this workload's widths."""
+    import long_context_attention_split_b200 as nx
+    from nectar_inputs import make_modules_general
+    res = {}
+    p = max(1, int(round(0.10 * wl.n)))
+    W, Z = nx.quadrature_init(wl.K, wl.V, p)
+    qa = torch.empty(wl.Q.shape[:4], dtype=torch.float32, device=dev)
+    qA = torch.empty(wl.Q.shape, dtype=torch.float32, device=dev)
+    qws = torch.empty(max(int(nx.lib().nectar_quadrature_workspace_size(nx.Dims(wl.L, wl.Hkv, wl.G, 128), p, wl.nq)),
+                          16), dtype=torch.uint8, device=dev)
+    t = _timed(lambda: nx.quadrature_forward(W, Z, wl.Q, a=qa, A_theta=qA, workspace=qws))
+    # exact attention over p keys: bytes as (i) with n = p, FLOPs 4 p d per query row
+    qbytes = 4 * p * 128 * wl.heads + wl.heads * wl.rows * (256 + 4 * 129)
+    qflops = 4 * p * 128 * wl.heads * wl.rows
+    q_roof_us = max(qbytes / (hbm_peak * 1e9), qflops / (tc_peak * 1e12)) * 1e6
+    res["quadrature"] = {"p": p, "ms": t, "GBps": qbytes / (t / 1e3) / 1e9, "TFLOPs": qflops / (t / 1e3) / 1e12,
+                         "bound": "hbm" if qbytes / (hbm_peak * 1e9) >= qflops / (tc_peak * 1e12) else "tensor",
+                         "roofline_us": q_roof_us, "frac": q_roof_us / (t * 1e3), "alg_bytes": qbytes}
+    del W, Z, qa, qA, qws
+    # fit metrics: against the module's outputs, or -- for a workload without
+    # modules (regression targets) -- against the targets shifted by 0.1 as
+    # stand-in module outputs (the kernel reads the same bytes either way)
+    if has_decode:
+        mws = torch.empty(max(nx.module_workspace_size(mods, wl.G, wl.nq), 16), dtype=torch.uint8, device=dev)
+        a, At = nx.module_forward(mods, wl.Q, workspace=mws)
+    else:
+        mws = None
+        a, At = alpha + 0.1, A + 0.1
+    met = torch.empty(wl.L, wl.Hkv, 3, dtype=torch.float64, device=dev)
+    t = _timed(lambda: nx.fit_metrics(alpha, A, a, At, wl.Q, metrics=met))
+    fbytes = wl.heads * wl.rows * (4 + 512 + 4 + 512 + 256)
+    res["fit_metrics"] = {"ms": t, "GBps": fbytes / (t / 1e3) / 1e9,
+                          "frac_hbm": fbytes / (t / 1e3) / 1e9 / hbm_peak, "alg_bytes": fbytes,
+                          "l2": "inputs smaller than L2" if fbytes < 126e6 else "inputs larger than L2"}
+    del a, At, mws
+    if has_decode:
+        widths = list(wl.widths)
+        gm = make_modules_general(wl.L, wl.Hkv, 128, 1, dev, (2, 1, 2), widths, widths, widths)
+        arch = nx.Arch((2, 1, 2), widths, widths, widths)
+        ms = nx.pack_modules_arch(gm, arch, wl.Hkv, wl.G, device=dev)
+        params = sum(t.numel() for layer in gm for part in layer.values()
+                     for key in ("U", "V", "b") for t in part[key] if t is not None) + \
+            sum(layer[n][k].numel() for layer in gm for n in ("score", "target") for k in ("Wout", "c"))
+        out = torch.empty(wl.Q.shape, dtype=torch.float32, device=dev)
+        dws = torch.empty(nx.decode_workspace_size(ms, wl.G, wl.nq), dtype=torch.uint8, device=dev)
+        args = (wl.Q, wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len)
+        t = _timed(lambda: nx.decode(ms, *args, out=out, workspace=dws))
+        dbytes = decode_bytes(wl, 2 * params)           # bf16 weights + visible local K/V + Q + out
+        classic = sum(wl.Hkv * (2 * H * H + 645 * H + 129) for H in wl.widths) if wl.depth == 2 else 0
+        dflops = decode_flops(wl) - 2 * classic * wl.G * wl.nq + 2 * params * wl.G * wl.nq
+        roof_us = max(dbytes / (hbm_peak * 1e9), dflops / (tc_peak * 1e12)) * 1e6
+        res["backbone_decode"] = {"depths": [2, 1, 2], "ms": t, "params": params, "alg_bytes": dbytes,
+                                  "roofline_us": roof_us, "frac": roof_us / (t * 1e3)}
+    return res
 
 
 def workload_overrides(args) -> dict:
@@ -648,6 +737,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--next-rows", action="store_true",
+                    help="also time the Quadrature module, the fit metrics and a decode with a shared backbone")
     ap.add_argument("--batch", type=int, default=0, help="decode batch B (llama8b_sweep: 1, 16, 256)")
     ap.add_argument("--rho", type=float, default=0.0, help="module capacity (llama8b_sweep: 0.01, 0.05, 0.10)")
     ap.add_argument("--layers", type=int, default=0,
