@@ -113,7 +113,8 @@ __device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uin
 }
 
 // ---------------------------------------------------------------------------
-// bulk copies (TMA engine).  No .multicast::cluster form is used anywhere.
+// bulk copies (TMA engine).  Every copy lands in the issuing CTA's own
+// shared memory: none is shared across a cluster.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;

@@ -1,7 +1,8 @@
 """GPU parity: every entry point of libnectar.so against the CPU oracle on the
 same seeded inputs.
 
-Tolerances (stated by the method's acceptance bar and derived in the design doc):
+Tolerances (the method's acceptance bar; the fused-decode bound is derived
+from the MLP and attention tolerances below):
   alpha            |gpu - oracle| <= 1e-3 absolute
   A, merged out    max|gpu - oracle| <= 2e-3 * ||v||_inf  (v: the values involved)
   MLP outputs      max|gpu - oracle| / max|oracle| <= 1e-2 per (l, h) and tensor
