@@ -146,6 +146,14 @@ struct GemmParams {
   int32_t width_s[kModMaxLayers];   // score branch width
   int32_t width_t[kModMaxLayers];   // target branch width
   int64_t layer_base[kModMaxLayers];
+  // per layer l, filled by the host for the current launch: the element
+  // stride between the blocks of its KV heads, the offset inside a head's
+  // block of the weights each part reads (part 0: the backbone or the score
+  // branch, part 1: the target branch; the readout: W_out as part 1), and
+  // aux: the score readout's w (the score's last layer) or c (the readout)
+  int64_t hstride[kModMaxLayers];
+  int64_t woff[kModMaxLayers][2];
+  int64_t aux[kModMaxLayers];
   int64_t tile_start[kModMaxLayers + 1];
   uint8_t order[kModMaxLayers];
 };

@@ -84,7 +84,7 @@ __device__ __forceinline__ uint32_t gemm_silu2(uint32_t acc0, uint32_t acc1, flo
 // One tile of the current launch: layer l, KV head hd, output part (0: the
 // backbone or the score branch, 1: the target branch; the readout is part
 // 1), 128-unit tile m, row tile rt -- and what the part's layer reads and
-// where its weights are.
+// where its weights are (offsets from the host's per-layer tables).
 struct GemmTile {
   int l, net, m, rt;
   int64_t hd;
@@ -93,14 +93,20 @@ struct GemmTile {
   int in_slot;      // h slot read for the columns past d
   int64_t w_off;    // blob offset of the layer's tiled weights
   int64_t b_off;    // blob offset of its bias
+  int64_t aux_off;  // blob offset of the score readout's w (score_last) or c (readout)
   bool score_last;  // the score branch's last layer: its readout is fused
-  int64_t score_base;   // blob offset of the score branch
   int Hs;           // score width (readout: the number of partials per row)
 };
 
 __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int64_t t) {
-  int li = 0;
-  while (li + 1 < p.nlayers && t >= p.tile_start[li + 1]) ++li;
+  // the layer slot holding tile t: the last li with tile_start[li] <= t
+  int lo = 0, hi = p.nlayers - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.tile_start[mid] <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  const int li = lo;
   GemmTile g;
   g.l = p.order[li];
   const int Db = p.depth_b, Ds = p.depth_s, Dt = p.depth_t;
@@ -126,33 +132,26 @@ __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int64_t t) {
   g.net = mm < mt0 ? 0 : 1;
   g.m = g.net ? mm - mt0 : mm;
   g.hd = static_cast<int64_t>(g.l) * p.Hkv + h;
-  const int64_t hb = p.layer_base[g.l] + static_cast<int64_t>(h) * layout::head_elems_arch(Db, Hb, Ds, Hs, Dt, Ht);
-  g.score_base = hb + layout::branch_base(Db, Hb, Ds, Hs, 0);
+  const int64_t hb = p.layer_base[g.l] + static_cast<int64_t>(h) * p.hstride[g.l];
   g.Hs = Hs;
   g.score_last = false;
+  g.w_off = hb + p.woff[g.l][g.net];
+  g.aux_off = hb + p.aux[g.l];
   if (p.readout) {
-    const int64_t tb = hb + layout::branch_base(Db, Hb, Ds, Hs, 1);
     g.H = kD;
     g.K = Ht;
     g.in_slot = 1;
-    g.w_off = tb + layout::branch_out_w_off(Db, Hb, Ht, Dt);
-    g.b_off = tb + layout::branch_out_b_off(Db, Hb, Ht, Dt, kD);
   } else if (s < Db) {
     g.H = Hb;
     g.K = kD + (s > 0 ? Hb : 0);
     g.in_slot = 0;
-    g.w_off = hb + layout::backbone_w_off(Hb, s);
-    g.b_off = g.w_off + layout::chunked_elems(Hb, g.K);
   } else {
-    const int Hn = g.net ? Ht : Hs;
-    const int64_t nb = hb + layout::branch_base(Db, Hb, Ds, Hs, g.net);
-    g.H = Hn;
-    g.K = kD + layout::branch_prev(Db, Hb, Hn, j);
+    g.H = g.net ? Ht : Hs;
+    g.K = kD + layout::branch_prev(Db, Hb, g.H, j);
     g.in_slot = j == 0 ? 0 : g.net;                         // a branch's first layer reads the backbone
-    g.w_off = nb + layout::branch_w_off(Db, Hb, Hn, j);
-    g.b_off = nb + layout::branch_b_off(Db, Hb, Hn, j);
     g.score_last = g.net == 0 && j == Ds - 1;
   }
+  g.b_off = g.w_off + layout::chunked_elems(g.H, g.K);     // the bias follows the tiled weights
   return g;
 }
 
@@ -299,9 +298,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         bias = __bfloat162float(p.blob[g.b_off + u]);
       } else if (i < g.H) {
         bias = __bfloat162float(p.blob[g.b_off + i]);
-        if (score_last)
-          wsc = __bfloat162float(
-              p.blob[g.score_base + layout::branch_out_w_off(p.depth_b, p.width_b[g.l], g.Hs, p.depth_s) + i]);
+        if (score_last) wsc = __bfloat162float(p.blob[g.aux_off + i]);
       }
       const float hbias = 0.5f * bias;
       if (ok) ok = mbar_wait_sleep(b_accf + 8 * b, (tc >> 1) & 1, p.err);   // waits out a main loop
@@ -360,8 +357,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
               const float* pr = p.part + (g.hd * R + r) * p.MT;
               const int mts = (g.Hs + 127) / 128;
               for (int m = 0; m < mts; ++m) a_l += pr[m];
-              a_l += __bfloat162float(
-                  p.blob[g.score_base + layout::branch_out_b_off(p.depth_b, p.width_b[g.l], g.Hs, p.depth_s, 1)]);
+              a_l += __bfloat162float(p.blob[g.aux_off]);
               if (q4 == 0 && p.a_out != nullptr) p.a_out[g.hd * R + r] = a_l;
             }
           }

@@ -788,12 +788,14 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
   g.err = mp.err;
   g.G = dims.G;
   g.nq = nq;
+  const int Db = mp.depth_b, Ds = mp.depth_s, Dt = mp.depth_t;
   for (int l = 0; l < dims.L; ++l) {
     g.width_b[l] = mp.width_b[l];
     g.width_s[l] = mp.width[l];
     g.width_t[l] = mp.width_t[l];
     g.layer_base[l] = mp.layer_base[l];
     g.order[l] = mp.order[l];
+    g.hstride[l] = layout::head_elems_arch(Db, mp.width_b[l], Ds, mp.width[l], Dt, mp.width_t[l]);
   }
   // hidden layers of the longest chain; the launches are stages 0..nst-1
   // (stage s < depth_b: the backbone, else branch layer s - depth_b of the
@@ -836,6 +838,23 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
     g.rtiles = ss.rtiles;
     g.stages = ss.stages;
     g.tmem_cols = ss.tmem_cols;
+    // per-layer weight offsets inside a head's block for this launch
+    for (int l = 0; l < dims.L; ++l) {
+      const int Hb = mp.width_b[l], Hs = mp.width[l], Ht = mp.width_t[l];
+      const int64_t sb = layout::branch_base(Db, Hb, Ds, Hs, 0), tb = layout::branch_base(Db, Hb, Ds, Hs, 1);
+      const int j = stage - Db;
+      g.woff[l][0] = g.woff[l][1] = g.aux[l] = 0;
+      if (g.readout) {
+        g.woff[l][1] = tb + layout::branch_out_w_off(Db, Hb, Ht, Dt);
+        g.aux[l] = sb + layout::branch_out_b_off(Db, Hb, Hs, Ds, 1);            // score c
+      } else if (j < 0) {
+        g.woff[l][0] = layout::backbone_w_off(Hb, stage);
+      } else {
+        if (j < Ds) g.woff[l][0] = sb + layout::branch_w_off(Db, Hb, Hs, j);
+        if (j < Dt) g.woff[l][1] = tb + layout::branch_w_off(Db, Hb, Ht, j);
+        if (j == Ds - 1) g.aux[l] = sb + layout::branch_out_w_off(Db, Hb, Hs, Ds);   // score w
+      }
+    }
     int64_t acc = 0;
     for (int li = 0; li < dims.L; ++li) {
       g.tile_start[li] = acc;
