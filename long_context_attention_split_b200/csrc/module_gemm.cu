@@ -98,6 +98,7 @@ struct GemmTile {
   int Hs;           // score width (readout: the number of partials per row)
 };
 
+template <bool kReadout>
 __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int64_t t) {
   // the layer slot holding tile t: the last li with tile_start[li] <= t
   int lo = 0, hi = p.nlayers - 1;
@@ -114,7 +115,7 @@ __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int64_t t) {
   const int s = p.stage;
   const int j = s - Db;                                   // branch layer (s >= Db)
   int mt0, mt1;
-  if (p.readout) {
+  if (kReadout) {
     mt0 = 0;
     mt1 = 1;
   } else if (s < Db) {
@@ -137,7 +138,7 @@ __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int64_t t) {
   g.score_last = false;
   g.w_off = hb + p.woff[g.l][g.net];
   g.aux_off = hb + p.aux[g.l];
-  if (p.readout) {
+  if (kReadout) {
     g.H = kD;
     g.K = Ht;
     g.in_slot = 1;
@@ -171,6 +172,9 @@ __device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) 
   return v[0];
 }
 
+// kReadout: the readout launch (target GEMM, merge epilogue) or a hidden
+// layer; separate instances keep each launch's code to its own epilogue.
+template <bool kReadout>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_h,
                    const GemmParams p) {
@@ -221,7 +225,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       uint32_t it = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x) {
-        const GemmTile g = gemm_tile(p, t);
+        const GemmTile g = gemm_tile<kReadout>(p, t);
         const int rows = g.H;
         const int K = g.K;
         const int kc = layout::kchunks(K);
@@ -229,7 +233,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         const uint32_t wbytes = static_cast<uint32_t>(layout::tile_rows(rows, g.m)) * 128;
         const int qrow = static_cast<int>(g.hd * R + static_cast<int64_t>(g.rt) * NR);
         const int hrow = static_cast<int>((g.in_slot * heads + g.hd) * R + static_cast<int64_t>(g.rt) * NR);
-        const int qch = p.readout ? 0 : 2;             // leading chunks taken from q
+        const int qch = kReadout ? 0 : 2;             // leading chunks taken from q
         for (int c = 0; c < kc; ++c, ++it) {
           const uint32_t s = it % S;
           if (it >= S && !mbar_wait(b_empty + 8 * s, ((it / S) - 1) & 1, p.err)) {
@@ -251,7 +255,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       uint32_t it = 0, tc = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x, ++tc) {
-        const GemmTile g = gemm_tile(p, t);
+        const GemmTile g = gemm_tile<kReadout>(p, t);
         const int kc = layout::kchunks(g.K);
         const uint32_t b = tc & 1;
         if (tc >= 2 && !mbar_wait(b_acce + 8 * b, ((tc >> 1) - 1) & 1, p.err)) break;
@@ -285,7 +289,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     uint32_t tc = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++tc) {
-      const GemmTile g = gemm_tile(p, t);
+      const GemmTile g = gemm_tile<kReadout>(p, t);
       const uint32_t b = tc & 1;
       const int r0 = g.rt * NR;
       // rows of this tile; a 32-column batch may run 16 columns past NR
@@ -294,7 +298,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       const int i = g.m * 128 + u;
       float bias = 0.f, wsc = 0.f;
       const bool score_last = g.score_last;
-      if (p.readout) {
+      if (kReadout) {
         bias = __bfloat162float(p.blob[g.b_off + u]);
       } else if (i < g.H) {
         bias = __bfloat162float(p.blob[g.b_off + i]);
@@ -311,7 +315,7 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         NECTAR_TMEM_LD32(dacc + n0, v);
         tmem_ld_wait();
         if (!ok) continue;
-        if (!p.readout) {
+        if constexpr (!kReadout) {
           if (score_last) {
             float part[32];
 #pragma unroll
@@ -453,10 +457,17 @@ GemmShape gemm_shape(int64_t R, int max_rows) {
 
 cudaError_t launch_module_gemm(const CUtensorMap& tq, const CUtensorMap& th, const GemmParams& p, int grid,
                                size_t smem, cudaStream_t stream) {
-  cudaError_t e =
-      cudaFuncSetAttribute(module_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  module_gemm_kernel<<<grid, kGemmThreads, smem, stream>>>(tq, th, p);
+  if (p.readout) {
+    cudaError_t e = cudaFuncSetAttribute(module_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    module_gemm_kernel<true><<<grid, kGemmThreads, smem, stream>>>(tq, th, p);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(module_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    module_gemm_kernel<false><<<grid, kGemmThreads, smem, stream>>>(tq, th, p);
+  }
   return cudaGetLastError();
 }
 
