@@ -95,6 +95,7 @@ struct ModParams {
   int Hkv, G, depth;            // depth: of both nets when the set has no backbone and equal nets
   int depth_b, depth_s, depth_t;
   bool general;                 // a backbone, or unequal nets: layer-by-layer path only
+  int net_split;                // one-launch path: one CTA per net (else one per head, both nets)
   int64_t nq;
   int N, TPC, nblk, Hmax, tmem_cols, stages, cps;
   const __nv_bfloat16* blob;

@@ -2,7 +2,10 @@
 // adds (iii): Eq. (3.6) and Eqs. (3.4)-(3.5) of "Nectar: Neural Estimation
 // of Cached-Token Attention via Regression" (§2.2, §2.4).
 //
-// Module CTA: one per (layer l, KV head h, block of TPC query tokens).  Its N
+// Module CTA: one per (layer l, KV head h, block of TPC query tokens), doing
+// the score net and then the target net -- or, when every net streams at
+// least 1 MB of weights (p.net_split), one per (l, h, block, net), so that
+// the two nets' weight streams run side by side on different SMs.  Its N
 // activation rows are the G query heads of those tokens (row g*TPC + t),
 // fetched by one 4-D TMA box.
 //
@@ -108,11 +111,14 @@ __device__ __forceinline__ void module_cta(const CUtensorMap* tmap_q, const ModP
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = p.N, TPC = p.TPC;
 
-  // unit -> (layer, head, token block); layers visited widest first
+  // unit -> (layer, head, token block[, net]); layers visited widest first
+  const int nlo = p.net_split ? (unit & 1) : 0;                // nets [nlo, nhi]: 0 score, 1 target
+  const int nhi = p.net_split ? (unit & 1) : 1;
+  const int hunit = p.net_split ? (unit >> 1) : unit;
   const int nblk = p.nblk;
-  const int li = unit / (p.Hkv * nblk);
-  const int h = (unit / nblk) % p.Hkv;
-  const int blk = unit % nblk;
+  const int li = hunit / (p.Hkv * nblk);
+  const int h = (hunit / nblk) % p.Hkv;
+  const int blk = hunit % nblk;
   const int l = p.order[li];
   const int H = p.width[l];
   const int mt = (H + 127) / 128;
@@ -164,7 +170,7 @@ __device__ __forceinline__ void module_cta(const CUtensorMap* tmap_q, const ModP
       tma_load_4d(smem_u32(smem + L.x + N * 128), tmap_q, 64, t0, 0, static_cast<int>(hd), b_qfull, pol_w);
       uint32_t it = 0;
       bool ok = true;
-      for (int net = 0; net < 2 && ok; ++net) {
+      for (int net = nlo; net <= nhi && ok; ++net) {
         const int64_t nb = head_base + (net ? layout::net_elems(H, depth, 1) : 0);
         const int nlayers = depth + net;                           // the target net adds its output GEMM
         for (int k = 0; k < nlayers && ok; ++k) {
@@ -201,11 +207,14 @@ __device__ __forceinline__ void module_cta(const CUtensorMap* tmap_q, const ModP
       uint32_t it = 0, xr = 0;
       const uint32_t idesc = idesc_bf16_f32(128, N, 0, 0);
       const uint32_t xbase = smem_u32(smem + L.x);
-      for (int net = 0; net < 2 && ok; ++net) {
+      for (int net = nlo; net <= nhi && ok; ++net) {
         const int nlayers = depth + net;
         for (int k = 0; k < nlayers && ok; ++k) {
           const bool out = (k == depth);
-          if (net > 0 || k > 0) {
+          // the accumulators and X are free once the previous layer's
+          // epilogue is done (in a CTA with both nets, also at the target's
+          // first layer)
+          if (net > nlo || k > 0) {
             ok = mbar_wait(b_xready, xr & 1, p.err);
             ++xr;
             if (!ok) break;
@@ -249,7 +258,7 @@ __device__ __forceinline__ void module_cta(const CUtensorMap* tmap_q, const ModP
     const __nv_bfloat16* blob = p.blob;
     bool ok = true;
     uint32_t accp = 0;
-    for (int net = 0; net < 2; ++net) {
+    for (int net = nlo; net <= nhi; ++net) {
       const int64_t nb = head_base + (net ? layout::net_elems(H, depth, 1) : 0);
       for (int k = 0; k < depth; ++k) {
         const __nv_bfloat16* bias = blob + nb + layout::hidden_b_off(H, depth, k);
@@ -338,24 +347,34 @@ __device__ __forceinline__ void module_cta(const CUtensorMap* tmap_q, const ModP
         mbar_arrive(b_xready);
       }
     }
-    // target readout A_theta[row][u] = acc[u][row] + c[u]
-    const float cb =
-        __bfloat162float(blob[head_base + layout::net_elems(H, depth, 1) + layout::out_b_off(H, depth, kD) + u]);
-    if (ok) ok = mbar_wait(b_acc, accp & 1, p.err);
-    named_bar_sync(2, kModEpiWarps * 32);     // sa complete
-    tc_fence_after();
-    for (int n0 = 0; n0 < N; n0 += 16) {
-      uint32_t v[16];
-      NECTAR_TMEM_LD16(trow + n0, v);
-      tmem_ld_wait();
+    if (nlo == 0) {
+      // score net: a[row] = its reduced readout (sa complete once every
+      // epilogue thread has passed the readout layer)
+      named_bar_sync(2, kModEpiWarps * 32);
+      if (et < N && ok) {
+        const int g = et / TPC, t = et % TPC;
+        if (g < p.G && t0 + t < p.nq)
+          p.a_out[hd * rows_per_head + static_cast<int64_t>(g) * p.nq + t0 + t] = sa[4 * N + et];
+      }
+    }
+    if (nhi == 1) {
+      // target net: A_theta[row][u] = acc[u][row] + c[u]
+      const float cb =
+          __bfloat162float(blob[head_base + layout::net_elems(H, depth, 1) + layout::out_b_off(H, depth, kD) + u]);
+      if (ok) ok = mbar_wait(b_acc, accp & 1, p.err);
+      tc_fence_after();
+      for (int n0 = 0; n0 < N; n0 += 16) {
+        uint32_t v[16];
+        NECTAR_TMEM_LD16(trow + n0, v);
+        tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int n = n0 + j;
-        const int g = n / TPC, t = n % TPC;
-        if (!ok || g >= p.G || t0 + t >= p.nq) continue;
-        const int64_t row = hd * rows_per_head + static_cast<int64_t>(g) * p.nq + t0 + t;
-        p.A_out[row * kD + u] = __uint_as_float(v[j]) + cb;
-        if (u == 0) p.a_out[row] = sa[4 * N + n];
+        for (int j = 0; j < 16; ++j) {
+          const int n = n0 + j;
+          const int g = n / TPC, t = n % TPC;
+          if (!ok || g >= p.G || t0 + t >= p.nq) continue;
+          const int64_t row = hd * rows_per_head + static_cast<int64_t>(g) * p.nq + t0 + t;
+          p.A_out[row * kD + u] = __uint_as_float(v[j]) + cb;
+        }
       }
     }
     tc_fence_before();

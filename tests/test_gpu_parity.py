@@ -362,6 +362,8 @@ def test_module_forward_toy():
     dict(L=1, Hkv=1, G=2, nq=64, widths=[512], depth=2),        # 128 rows
     dict(L=1, Hkv=2, G=4, nq=16, widths=[256], depth=2),        # exactly 64 rows: the first grouped-GEMM size
     dict(L=1, Hkv=1, G=7, nq=9, widths=[144], depth=2),         # 63 rows: still one CTA per block of tokens
+    dict(L=2, Hkv=2, G=2, nq=5, widths=[768, 1024], depth=2),   # >= 1 MB per net: one CTA per net
+    dict(L=1, Hkv=1, G=3, nq=4, widths=[1024], depth=3),
 ])
 def test_module_forward_shapes(kw):
     kw = dict(kw)
@@ -413,6 +415,7 @@ def test_decode_toy_prefill():
     dict(L=1, Hkv=2, G=7, n=16, B=64, T=33, widths=[768]),     # 448 rows: two row tiles of 224
     dict(L=2, Hkv=2, G=4, n=16, B=16, T=40, widths=[256, 128]),   # exactly 64 rows: grouped-GEMM decode
     dict(L=1, Hkv=2, G=16, n=16, B=8, T=300, widths=[256]),    # 128 rows, 16 heads per local job, 3 tiles
+    dict(L=2, Hkv=2, G=2, n=16, B=3, T=40, widths=[768, 896]),   # one CTA per net in the one-launch decode
 ])
 def test_decode_shapes(kw):
     wl = make_workload("qwen3_1p7b", seed=2, key_scale=None, **kw)
