@@ -112,7 +112,9 @@ struct ModParams {
   float qmul;
   float* out;
   float* ws_loc;        // decode: local state per row [(hd * rows + row)][d + 2]
-  int64_t n_local;      // decode: local CTAs (heads * nq) ahead of the module CTAs
+  int64_t n_local;      // decode: local CTAs (heads * nq), after the module CTAs
+  int64_t n_module;     // decode: module CTAs (set at launch)
+  int module_first;     // decode: module CTAs ahead of the local CTAs in the grid
   __nv_bfloat16* out_bf16;   // decode: if set, the output goes here, bf16 [L][nq][Hkv][G][d]
   int* err;
   int32_t width[kModMaxLayers];        // score width (= target width unless general)

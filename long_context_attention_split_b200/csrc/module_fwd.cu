@@ -436,16 +436,24 @@ __device__ __forceinline__ void local_state_cta(const ModParams& p, int64_t luni
   }
 }
 
-// Decode launch: CTAs [0, n_local) are local CTAs, the rest module CTAs.
+// Decode launch: n_module module CTAs and n_local local CTAs.  When the
+// local CTAs are short next to the module CTAs (p.module_first), the module
+// CTAs come first in the grid, two per SM where there are enough, and the
+// local CTAs fill the slots left, which keeps the bytes each SM streams
+// closer to even; when they are long, they come first, so that they do not
+// end the launch as a tail.
 template <int RG>
 __global__ void __launch_bounds__(kModThreads, 2)
 decode_kernel(const __grid_constant__ CUtensorMap tmap_q, const ModParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw);
-  if (static_cast<int64_t>(blockIdx.x) < p.n_local) {
-    local_state_cta<RG>(p, blockIdx.x, smem);
+  const int64_t b = blockIdx.x;
+  if (p.module_first) {
+    if (b < p.n_module) module_cta(&tmap_q, p, static_cast<int>(b), smem);
+    else local_state_cta<RG>(p, b - p.n_module, smem);
   } else {
-    module_cta(&tmap_q, p, static_cast<int>(blockIdx.x - p.n_local), smem);
+    if (b < p.n_local) local_state_cta<RG>(p, b, smem);
+    else module_cta(&tmap_q, p, static_cast<int>(b - p.n_local), smem);
   }
 }
 
@@ -521,7 +529,9 @@ static cudaError_t launch_decode_t(const CUtensorMap& tq, const ModParams& p, in
   cudaError_t e = cudaFuncSetAttribute(decode_kernel<RG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  decode_kernel<RG><<<static_cast<unsigned>(p.n_local + units), kModThreads, smem, stream>>>(tq, p);
+  ModParams q = p;
+  q.n_module = units;
+  decode_kernel<RG><<<static_cast<unsigned>(p.n_local + units), kModThreads, smem, stream>>>(tq, q);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t nrows = static_cast<int64_t>(p.n_local / p.nq) * p.G * p.nq;
@@ -537,7 +547,10 @@ static cudaError_t launch_local_t(const ModParams& p, cudaStream_t stream) {
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   CUtensorMap unused{};                      // local CTAs read no tensor map
-  decode_kernel<RG><<<static_cast<unsigned>(p.n_local), kModThreads, smem, stream>>>(unused, p);
+  ModParams q = p;
+  q.n_module = 0;                            // every CTA a local CTA
+  q.module_first = 0;
+  decode_kernel<RG><<<static_cast<unsigned>(p.n_local), kModThreads, smem, stream>>>(unused, q);
   return cudaGetLastError();
 }
 
