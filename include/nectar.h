@@ -271,17 +271,19 @@ NECTAR_API nectar_status nectar_merge_local(nectar_dims dims, const float *a, co
  * and nectar_merge_local; out DEVICE fp32 [L][Hkv][G][nq][d].  Equal (up to
  * rounding order) to nectar_module_forward followed by nectar_merge_local.
  *
- * Fewer than 64 query rows per KV head: one launch whose CTAs run the
- * module forward (writing A_theta into out) side by side with CTAs that
- * compute each row's local attention state, then a small merge that
- * rewrites out in place.  More rows: the local states first, then the
- * layer-by-layer module, whose last launch merges and writes out.
+ * Fewer than 64 query rows per KV head (classic module sets): one launch
+ * whose CTAs run the module forward (writing A_theta into out) side by side
+ * with CTAs that compute each row's local attention state, then a small
+ * merge that rewrites out in place.  More rows, or a set with a backbone or
+ * unequal nets: the local states first, then the layer-by-layer module,
+ * whose last launch merges and writes out.
  *
  *   workspace  DEVICE scratch, 256-byte aligned, of at least
  *              nectar_decode_workspace_size(dims, mods, nq) bytes: the
  *              local state of every row, rows * (d + 2) * 4 with
- *              rows = L * Hkv * G * nq, plus rows * 4 (fewer than 64 query
- *              rows per KV head) or nectar_module_workspace_size (else);
+ *              rows = L * Hkv * G * nq, plus rows * 4 (the one-launch
+ *              path) or nectar_module_workspace_size (the layer-by-layer
+ *              path);
  *              owned by the caller, overwritten, must not be used by
  *              another call in flight.
  * Returns NECTAR_ERR_WORKSPACE when it is missing or too small.
