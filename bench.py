@@ -412,21 +412,20 @@ def parts(wl, attn_ms, dec_ms, ab, db, qps, hbm_peak, tc_peak, has_decode):
 
 
 def _timed(fn, iters=10, warm=3):
-    """Median device time (ms) of fn() on the current stream, CUDA events."""
+    """Device time (ms) per call of fn() on the current stream: `iters` calls
+    back to back between two CUDA events, so that the host's launch work
+    overlaps the device's instead of sitting inside the timed region."""
     for _ in range(warm):
         fn()
     torch.cuda.synchronize()
-    ts = []
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
     for _ in range(iters):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
         fn()
-        e1.record()
-        torch.cuda.synchronize()
-        ts.append(e0.elapsed_time(e1))
-    ts.sort()
-    return ts[len(ts) // 2]
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
 
 
 def next_rows(wl, mods, alpha, A, has_decode, dev, hbm_peak, tc_peak) -> dict:
