@@ -143,3 +143,17 @@ def test_arch_packing_without_backbone_is_the_classic_blob():
     wb = [64, 16, 32]
     with_bb = nx.Arch((1, 3, 3), wb, widths, widths)
     assert with_bb.packed_elems(2) > nx.Arch((0, 3, 3), [], widths, widths).packed_elems(2)
+
+
+def test_arch_validation_on_the_host():
+    # depths and widths outside the supported set are refused (0 elements)
+    import long_context_attention_split_b200 as nx
+    ok = nx.Arch((2, 1, 2), [64, 32], [32, 16], [48, 96])
+    assert ok.packed_elems(2) > 0
+    for depths, wb, ws, wt in [((2, 0, 2), [64, 32], [32, 16], [48, 96]),     # a branch without layers
+                               ((0, 1, 0), [], [32, 16], [48, 96]),
+                               ((3, 1, 2), [64, 32], [32, 16], [48, 96]),     # chain of 5 > NECTAR_MAX_DEPTH
+                               ((1, 1, 1), [64, 40], [32, 16], [48, 96]),     # width not a multiple of 16
+                               ((0, 2, 2), [], [32, 2048], [48, 96]),         # width above the maximum
+                               ((-1, 1, 1), [], [32, 16], [48, 96])]:
+        assert nx.Arch(depths, wb, ws, wt).packed_elems(2) == 0, depths
