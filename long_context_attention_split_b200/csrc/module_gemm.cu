@@ -21,10 +21,19 @@
 // (a_theta, A_theta) or merges them with each row's exact local attention
 // state (decode).
 //
+// Module sets with a shared backbone (§2.4, App. A.3: depths D_b, D_s, D_t)
+// take one launch per chain layer: launch s < D_b runs the backbone (its h
+// in activation slot 0), later launches run layer s - D_b of each branch
+// that has one (a branch's first layer reads slot 0, the others their own
+// slot); the classic pair of nets is the case D_b = 0.
+//
 // Persistent CTAs (one per SM) walk a static list of tiles, widest layers
-// first.  Warp roles: 0 TMA producer, 1 MMA issuer (+ TMEM owner), 2..5
-// epilogue.  Two TMEM accumulators let the epilogue of one tile run under
-// the MMAs of the next.
+// first; the host gives each launch per-layer tables (head stride, weight
+// offsets) so that decoding a tile costs a binary search and a few adds.
+// Warp roles: 0 TMA producer, 1 MMA issuer (+ TMEM owner), 2..9 epilogue
+// (two per TMEM lane quarter, alternating 32-column batches).  Two TMEM
+// accumulators let the epilogue of one tile run under the MMAs of the next.
+// Hidden-layer and readout launches are separate instances of the kernel.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
