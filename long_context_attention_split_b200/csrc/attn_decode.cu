@@ -2,7 +2,9 @@
 // head): Eq. (3.1) of "Nectar: Neural Estimation of Cached-Token Attention
 // via Regression" (§2.1), split over n and joined by log-sum-exp.
 //
-// Schedule.  The document of every (l, h) is cut into 64-key tiles and all
+// Schedule.  The document of every (l, h) is cut into tiles of 128 keys (up
+// to 2 query rows per pass) or 64 (more rows: their register state needs
+// the room), and all
 // heads' tiles are laid end to end (head-major).  CTA c of C takes the
 // contiguous range [c*T/C, (c+1)*T/C) of that list, so every CTA streams the
 // same number of bytes whatever n and the head count are; a CTA whose range
@@ -10,7 +12,7 @@
 // The combine kernel then joins, for each head, the partials of the CTAs
 // that covered it -- a separate launch, so no CTA ever waits on another.
 //
-// Data movement.  One producer warp streams K and V tiles (16 KB each, whole
+// Data movement.  One producer warp streams K and V tiles (32 or 16 KB each, whole
 // contiguous rows) into a 3-stage ring with TMA bulk copies (evict-first L2
 // policy: the document is read once); 8 consumer warps score and accumulate
 // on the CUDA cores (see common.cuh).
@@ -21,7 +23,6 @@
 
 namespace nectar {
 
-constexpr int kDecTile = 64;
 constexpr int kDecWarps = 8;
 constexpr int kDecStages = 3;
 constexpr int kDecThreads = (kDecWarps + 1) * 32;
@@ -30,10 +31,10 @@ __host__ __device__ __forceinline__ int first_cta_of_tile(int64_t t, int64_t tot
   return static_cast<int>(((t + 1) * static_cast<int64_t>(C) - 1) / total);
 }
 
-// RW: query rows held by one warp (R rows in NRG groups of RW).
-template <int RW>
+// RW: query rows held by one warp (R rows in NRG groups of RW); TILE keys per tile.
+template <int RW, int TILE>
 __host__ __device__ constexpr size_t dec_smem_bytes() {
-  return size_t(2) * kDecStages * kDecTile * kRowBytes       // K, V ring
+  return size_t(2) * kDecStages * TILE * kRowBytes            // K, V ring
          + size_t(kDecWarps) * RW * (kD + 2) * sizeof(float)  // cross-warp reduction
          + 2 * kDecStages * sizeof(uint64_t);                 // full / empty barriers
 }
@@ -43,23 +44,26 @@ __host__ __device__ constexpr size_t dec_smem_bytes() {
 // every key of a tile (the group's warps split the keys).  A warp's registers
 // grow with RW, so 4 rows as 2 groups of 2 keep the 2-row register budget
 // and two CTAs per SM, at the cost of reading each tile from shared memory
-// twice.  Two CTAs per SM for up to 2 rows per warp (register cap 113).
+// twice.  With 64-key tiles, two CTAs per SM for up to 2 rows per warp
+// (register cap 113); 128-key tiles fill most of an SM's shared memory with
+// one CTA's ring, which then has the register file to itself.
 template <int R, int LPK, int NRG>
-__global__ void __launch_bounds__(kDecThreads, (R / NRG <= 2 ? 2 : 1))
+__global__ void __launch_bounds__(kDecThreads, (dec_tile(R) == 64 && R / NRG <= 2 ? 2 : 1))
 cache_attn_split_kernel(const DecParams p) {
+  constexpr int TILE = dec_tile(R);
   constexpr int RW = R / NRG;
   constexpr int WPG = kDecWarps / NRG;       // warps per row group
   static_assert(RW * NRG == R && WPG * NRG == kDecWarps, "row groups");
   using St = RowState<RW, LPK>;
   constexpr int NG = St::NG;
-  constexpr int KPW = kDecTile / WPG;        // keys per warp per tile
+  constexpr int KPW = TILE / WPG;            // keys per warp per tile
   constexpr int KPG = KPW / NG;              // keys per group per tile
   static_assert(KPG >= 1, "tile too small");
 
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* sK = smem;
-  uint8_t* sV = smem + kDecStages * kDecTile * kRowBytes;
-  float* sRed = reinterpret_cast<float*>(smem + 2 * kDecStages * kDecTile * kRowBytes);
+  uint8_t* sV = smem + kDecStages * TILE * kRowBytes;
+  float* sRed = reinterpret_cast<float*>(smem + 2 * kDecStages * TILE * kRowBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sRed + kDecWarps * RW * (kD + 2));
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kDecStages);
 
@@ -87,13 +91,13 @@ cache_attn_split_kernel(const DecParams p) {
         if (i >= kDecStages && !mbar_wait(empty0 + 8 * s, static_cast<uint32_t>(((i / kDecStages) - 1) & 1), p.err))
           break;
         const int64_t hd = tt / p.tph;
-        const int64_t j0 = (tt - hd * p.tph) * kDecTile;
-        const int64_t cnt = (p.n - j0 < kDecTile) ? (p.n - j0) : kDecTile;
+        const int64_t j0 = (tt - hd * p.tph) * TILE;
+        const int64_t cnt = (p.n - j0 < TILE) ? (p.n - j0) : TILE;
         const uint32_t bytes = static_cast<uint32_t>(cnt) * kRowBytes;
         const size_t off = (static_cast<size_t>(hd) * p.n + j0) * kD;
         mbar_arrive_expect_tx(full0 + 8 * s, 2 * bytes);
-        bulk_g2s(smem_u32(sK + s * kDecTile * kRowBytes), p.K + off, bytes, full0 + 8 * s, pol);
-        bulk_g2s(smem_u32(sV + s * kDecTile * kRowBytes), p.V + off, bytes, full0 + 8 * s, pol);
+        bulk_g2s(smem_u32(sK + s * TILE * kRowBytes), p.K + off, bytes, full0 + 8 * s, pol);
+        bulk_g2s(smem_u32(sV + s * TILE * kRowBytes), p.V + off, bytes, full0 + 8 * s, pol);
       }
     }
     return;
@@ -164,10 +168,10 @@ cache_attn_split_kernel(const DecParams p) {
     const int s = static_cast<int>(i % kDecStages);
     if (ok) ok = mbar_wait(full0 + 8 * s, static_cast<uint32_t>((i / kDecStages) & 1), p.err);
     if (ok) {
-      const int64_t j0 = (tt - hd * p.tph) * kDecTile;
-      const int cnt = static_cast<int>((p.n - j0 < kDecTile) ? (p.n - j0) : kDecTile);
-      const uint8_t* kt = sK + s * kDecTile * kRowBytes;
-      const uint8_t* vt = sV + s * kDecTile * kRowBytes;
+      const int64_t j0 = (tt - hd * p.tph) * TILE;
+      const int cnt = static_cast<int>((p.n - j0 < TILE) ? (p.n - j0) : TILE);
+      const uint8_t* kt = sK + s * TILE * kRowBytes;
+      const uint8_t* vt = sV + s * TILE * kRowBytes;
       if constexpr (NRG == 1) {
         const uint8_t* kr[KPG];
         const uint8_t* vr[KPG];
@@ -246,7 +250,8 @@ __global__ void cache_attn_combine_kernel(const DecParams p, float* __restrict__
 // ---------------------------------------------------------------------------
 template <int R, int LPK, int NRG>
 static cudaError_t launch_split(const DecParams& p, cudaStream_t stream) {
-  const size_t smem = dec_smem_bytes<R / NRG>();
+  if (p.tile != dec_tile(R)) return cudaErrorInvalidValue;   // planned for another tile size
+  const size_t smem = dec_smem_bytes<R / NRG, dec_tile(R)>();
   cudaError_t e = cudaFuncSetAttribute(cache_attn_split_kernel<R, LPK, NRG>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -259,7 +264,7 @@ int dec_max_rows() { return 8; }
 // Resident CTAs per SM of the split kernel for R rows (occupancy calculator).
 template <int R, int LPK, int NRG>
 static int occ_t() {
-  const size_t smem = dec_smem_bytes<R / NRG>();
+  const size_t smem = dec_smem_bytes<R / NRG, dec_tile(R)>();
   if (cudaFuncSetAttribute(cache_attn_split_kernel<R, LPK, NRG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return 1;
@@ -285,21 +290,22 @@ int dec_ctas_per_sm(int R) {
 
 size_t dec_smem_for_rows(int R) {
   switch (R) {
-    case 1: return dec_smem_bytes<1>();
-    case 2: return dec_smem_bytes<2>();
+    case 1: return dec_smem_bytes<1, dec_tile(1)>();
+    case 2: return dec_smem_bytes<2, dec_tile(2)>();
     case 3:
-    case 4: return dec_smem_bytes<2>();
-    case 5: return dec_smem_bytes<5>();
-    case 6: return dec_smem_bytes<6>();
-    case 7: return dec_smem_bytes<7>();
-    default: return dec_smem_bytes<8>();
+    case 4: return dec_smem_bytes<2, dec_tile(4)>();
+    case 5: return dec_smem_bytes<5, dec_tile(5)>();
+    case 6: return dec_smem_bytes<6, dec_tile(6)>();
+    case 7: return dec_smem_bytes<7, dec_tile(7)>();
+    default: return dec_smem_bytes<8, dec_tile(8)>();
   }
 }
 
 // Plan: tiles per head, total tiles, CTA count and partial slots per head.
-DecPlan plan_decode(int heads, int64_t n, int num_sms, int ctas_per_sm) {
+DecPlan plan_decode(int heads, int64_t n, int num_sms, int ctas_per_sm, int tile) {
   DecPlan pl{};
-  pl.tph = (n + kDecTile - 1) / kDecTile;
+  pl.tile = tile;
+  pl.tph = (n + tile - 1) / tile;
   pl.total = static_cast<int64_t>(heads) * pl.tph;
   int64_t C = static_cast<int64_t>(num_sms) * ctas_per_sm;
   if (C > pl.total) C = pl.total;

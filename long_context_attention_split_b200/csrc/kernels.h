@@ -20,7 +20,8 @@ struct DecParams {
   int heads;
   int64_t rows_total;   // query rows per head (G * nq)
   int row0;             // first row handled by this launch
-  int64_t tph;          // 64-key tiles per head
+  int tile;             // keys per tile: dec_tile(rows of a pass)
+  int64_t tph;          // tiles per head
   int64_t total;        // heads * tph
   int C;                // CTAs of the split launch
   int S_max;            // partial slots per head
@@ -32,10 +33,16 @@ struct DecParams {
 
 struct DecPlan {
   int64_t tph, total;
-  int C, S_max;
+  int C, S_max, tile;
 };
 
-DecPlan plan_decode(int heads, int64_t n, int num_sms, int ctas_per_sm);
+// Keys per tile of the split kernel for R query rows per pass: 128 up to 2
+// rows (one CTA per SM streaming 32 KB bulk copies: measured 0.549 against
+// 0.683 ms on a 28 x 8-head, 32768-key, 2-row document), 64 above (at 4
+// rows the 64-key tiles with two CTAs per SM measured 1 % faster; from 5
+// rows the row state needs the registers of a smaller tile).
+__host__ __device__ constexpr int dec_tile(int R) { return R <= 2 ? 128 : 64; }
+DecPlan plan_decode(int heads, int64_t n, int num_sms, int ctas_per_sm, int tile);
 int dec_max_rows();
 int dec_ctas_per_sm(int R);
 size_t dec_smem_for_rows(int R);
@@ -48,7 +55,8 @@ struct TcParams {
   int heads;
   int64_t rows_total;
   int qpairs;           // units (pairs of 128-row query tiles) per head
-  int64_t tph;          // 64-key tiles per head
+  int tile;             // keys per tile: dec_tile(rows of a pass)
+  int64_t tph;          // tiles per head
   int C;                // CTAs (one per SM)
   int dp_rounds;        // whole-unit rounds before the stream-K part
   int64_t sk_units;     // units cut by key tiles across the CTAs

@@ -95,6 +95,9 @@ __device__ __forceinline__ uint32_t x_offset(int N, int n, int c) {
 // One module CTA: (a_theta, A_theta) of the rows of `unit`.  smem is the
 // 1024-aligned dynamic shared memory.  a goes to p.a_out[hd * rows + row],
 // A_theta to p.A_out[(hd * rows + row) * d].
+// kNetSplit: one net per CTA (p.net_split); a compile-time choice, so that
+// the usual two-net CTA keeps constant loop bounds over the nets.
+template <bool kNetSplit>
 __device__ __forceinline__ void module_cta(const CUtensorMap* tmap_q, const ModParams& p, int unit, uint8_t* smem) {
   const ModSmem L = mod_smem_layout(p.Hmax, p.N, p.stages, p.cps);
   const uint32_t S = static_cast<uint32_t>(p.stages);
@@ -112,9 +115,9 @@ __device__ __forceinline__ void module_cta(const CUtensorMap* tmap_q, const ModP
   const int N = p.N, TPC = p.TPC;
 
   // unit -> (layer, head, token block[, net]); layers visited widest first
-  const int nlo = p.net_split ? (unit & 1) : 0;                // nets [nlo, nhi]: 0 score, 1 target
-  const int nhi = p.net_split ? (unit & 1) : 1;
-  const int hunit = p.net_split ? (unit >> 1) : unit;
+  const int nlo = kNetSplit ? (unit & 1) : 0;                  // nets [nlo, nhi]: 0 score, 1 target
+  const int nhi = kNetSplit ? (unit & 1) : 1;
+  const int hunit = kNetSplit ? (unit >> 1) : unit;
   const int nblk = p.nblk;
   const int li = hunit / (p.Hkv * nblk);
   const int h = (hunit / nblk) % p.Hkv;
@@ -393,10 +396,11 @@ __device__ __forceinline__ uint8_t* aligned_smem(uint8_t* raw) {
 }
 
 // Standalone module forward.  Two CTAs per SM where the plan fits half an SM.
+template <bool kNetSplit>
 __global__ void __launch_bounds__(kModThreads, 2)
 module_kernel(const __grid_constant__ CUtensorMap tmap_q, const ModParams p) {
   extern __shared__ uint8_t smem_raw[];
-  module_cta(&tmap_q, p, blockIdx.x, aligned_smem(smem_raw));
+  module_cta<kNetSplit>(&tmap_q, p, blockIdx.x, aligned_smem(smem_raw));
 }
 
 // One local CTA of the decode: the exact causal attention state of every
@@ -442,18 +446,18 @@ __device__ __forceinline__ void local_state_cta(const ModParams& p, int64_t luni
 // local CTAs fill the slots left, which keeps the bytes each SM streams
 // closer to even; when they are long, they come first, so that they do not
 // end the launch as a tail.
-template <int RG>
+template <int RG, bool kNetSplit>
 __global__ void __launch_bounds__(kModThreads, 2)
 decode_kernel(const __grid_constant__ CUtensorMap tmap_q, const ModParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw);
   const int64_t b = blockIdx.x;
   if (p.module_first) {
-    if (b < p.n_module) module_cta(&tmap_q, p, static_cast<int>(b), smem);
+    if (b < p.n_module) module_cta<kNetSplit>(&tmap_q, p, static_cast<int>(b), smem);
     else local_state_cta<RG>(p, b - p.n_module, smem);
   } else {
     if (b < p.n_local) local_state_cta<RG>(p, b, smem);
-    else module_cta(&tmap_q, p, static_cast<int>(b - p.n_local), smem);
+    else module_cta<kNetSplit>(&tmap_q, p, static_cast<int>(b - p.n_local), smem);
   }
 }
 
@@ -516,23 +520,36 @@ ModShape mod_shape(int G, int64_t nq, int Hmax, bool fuse) {
 cudaError_t launch_module(const CUtensorMap& tq, const ModParams& p, int units, size_t smem, bool fuse,
                           cudaStream_t stream) {
   (void)fuse;
-  cudaError_t e = cudaFuncSetAttribute(module_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (p.net_split) {
+    cudaError_t e = cudaFuncSetAttribute(module_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    module_kernel<true><<<units, kModThreads, smem, stream>>>(tq, p);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(module_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    module_kernel<false><<<units, kModThreads, smem, stream>>>(tq, p);
+  }
+  return cudaGetLastError();
+}
+
+template <int RG, bool kNetSplit>
+static cudaError_t launch_decode_s(const CUtensorMap& tq, const ModParams& q, size_t smem, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<RG, kNetSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  module_kernel<<<units, kModThreads, smem, stream>>>(tq, p);
+  decode_kernel<RG, kNetSplit><<<static_cast<unsigned>(q.n_local + q.n_module), kModThreads, smem, stream>>>(tq, q);
   return cudaGetLastError();
 }
 
 template <int RG>
 static cudaError_t launch_decode_t(const CUtensorMap& tq, const ModParams& p, int units, size_t smem,
                                    cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<RG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
   ModParams q = p;
   q.n_module = units;
-  decode_kernel<RG><<<static_cast<unsigned>(p.n_local + units), kModThreads, smem, stream>>>(tq, q);
-  e = cudaGetLastError();
+  cudaError_t e = p.net_split ? launch_decode_s<RG, true>(tq, q, smem, stream)
+                              : launch_decode_s<RG, false>(tq, q, smem, stream);
   if (e != cudaSuccess) return e;
   const int64_t nrows = static_cast<int64_t>(p.n_local / p.nq) * p.G * p.nq;
   const int64_t threads = nrows * kD;
@@ -543,14 +560,14 @@ static cudaError_t launch_decode_t(const CUtensorMap& tq, const ModParams& p, in
 template <int RG>
 static cudaError_t launch_local_t(const ModParams& p, cudaStream_t stream) {
   const size_t smem = dec_local_smem(RG) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<RG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<RG, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   CUtensorMap unused{};                      // local CTAs read no tensor map
   ModParams q = p;
   q.n_module = 0;                            // every CTA a local CTA
   q.module_first = 0;
-  decode_kernel<RG><<<static_cast<unsigned>(p.n_local), kModThreads, smem, stream>>>(unused, q);
+  decode_kernel<RG, false><<<static_cast<unsigned>(p.n_local), kModThreads, smem, stream>>>(unused, q);
   return cudaGetLastError();
 }
 

@@ -105,7 +105,7 @@ int dec_row_block(int64_t rows) { return rows < dec_max_rows() ? static_cast<int
 DecPlan cache_attn_plan(const nectar_dims& d, int64_t n, int64_t nq, int sms) {
   const int64_t rows = static_cast<int64_t>(d.G) * nq;
   const int R = dec_row_block(rows);
-  return plan_decode(d.L * d.Hkv, n, sms, dec_ctas_per_sm(R < 1 ? 1 : R));
+  return plan_decode(d.L * d.Hkv, n, sms, dec_ctas_per_sm(R < 1 ? 1 : R), dec_tile(R < 1 ? 1 : R));
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no
@@ -225,6 +225,7 @@ nectar_status nectar_cache_attn_lse(nectar_dims dims, const nectar_bf16* K, cons
   p.qmul = scale * kLog2e;
   p.err = di.err;
   const DecPlan pl = cache_attn_plan(dims, n, nq, di.sms);
+  p.tile = pl.tile;
   p.tph = pl.tph;
   p.total = pl.total;
   p.C = pl.C;
