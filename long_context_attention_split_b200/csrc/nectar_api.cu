@@ -89,12 +89,12 @@ DeviceInfo device_info() {
   return cache[dev];
 }
 
-// Row blocks handled by one launch of the CUDA-core split kernel.
+// Query rows per KV head up to which exact attention stays on the CUDA-core
+// split kernel (capped at dec_max_rows()).
 #ifndef NECTAR_TC_ROUTE_ROWS
 #define NECTAR_TC_ROUTE_ROWS 8
 #endif
-// More query rows per KV head than this: the tensor-core kernel; else the
-// split kernel on the CUDA cores (at most dec_max_rows() rows).
+// More query rows per KV head than that: the tensor-core kernel.
 bool use_tc_attn(int64_t rows) {
   const int64_t lim = NECTAR_TC_ROUTE_ROWS < dec_max_rows() ? NECTAR_TC_ROUTE_ROWS : dec_max_rows();
   return rows > lim;
