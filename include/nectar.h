@@ -90,6 +90,10 @@ typedef struct {
  *              nectar_cache_attn_workspace_size(dims, n, nq) bytes (may be
  *              NULL when that size is 0).  Its contents on entry do not
  *              matter; two calls that overlap on the GPU must not share one.
+ *              The size depends on the current device's SM count; it is 0
+ *              when n == 0 or nq == 0 (no scratch needed), and also for
+ *              invalid dims or when no CUDA device is current, cases in
+ *              which nectar_cache_attn_lse itself returns an error.
  * n >= 0, nq >= 0 (nq == 0: nothing to do).  Returns NECTAR_ERR_WORKSPACE
  * when the workspace is too small.
  * ------------------------------------------------------------------------ */
@@ -280,10 +284,11 @@ NECTAR_API nectar_status nectar_merge_local(nectar_dims dims, const float *a, co
  *
  *   workspace  DEVICE scratch, 256-byte aligned, of at least
  *              nectar_decode_workspace_size(dims, mods, nq) bytes: the
- *              local state of every row, rows * (d + 2) * 4 with
- *              rows = L * Hkv * G * nq, plus rows * 4 (the one-launch
- *              path) or nectar_module_workspace_size (the layer-by-layer
- *              path);
+ *              local state of every row, align256(rows * (d + 2) * 4) with
+ *              rows = L * Hkv * G * nq, plus align256(rows * 4) (the
+ *              one-launch path) or nectar_module_workspace_size (the
+ *              layer-by-layer path), align256(x) rounding x up to a
+ *              multiple of 256;
  *              owned by the caller, overwritten, must not be used by
  *              another call in flight.
  * Returns NECTAR_ERR_WORKSPACE when it is missing or too small.

@@ -157,3 +157,65 @@ def test_arch_validation_on_the_host():
                                ((0, 2, 2), [], [32, 2048], [48, 96]),         # width above the maximum
                                ((-1, 1, 1), [], [32, 16], [48, 96])]:
         assert nx.Arch(depths, wb, ws, wt).packed_elems(2) == 0, depths
+
+
+def a256(x):
+    return (x + 255) // 256 * 256
+
+
+def _host_set(L, Hkv, widths, depth, arch=None):
+    # the size functions read only the shapes: a host blob of the packed size will do
+    if arch is not None:
+        n = arch.packed_elems(Hkv)
+        return nx.ModuleSet(torch.zeros(n, dtype=torch.bfloat16), arch.width_s, arch.depths[1], L, Hkv, arch=arch)
+    n = nx.packed_elems(L, Hkv, 1, widths, depth)
+    return nx.ModuleSet(torch.zeros(n, dtype=torch.bfloat16), widths, depth, L, Hkv)
+
+
+@pytest.mark.parametrize("widths,depth", [([256, 512, 384], 2), ([208, 144, 80], 1), ([128, 128, 1024], 3)])
+@pytest.mark.parametrize("G,nq", [(2, 1), (4, 8), (2, 32), (8, 40)])
+def test_workspace_sizes_follow_the_header(widths, depth, G, nq):
+    """nectar_module_workspace_size, nectar_decode_workspace_size and
+    nectar_decode_layer_out_workspace_size equal the formulas include/nectar.h
+    states for them (classic sets; 64 query rows per KV head or more take the
+    layer-by-layer path)."""
+    L, Hkv, d = len(widths), 2, 128
+    mods = _host_set(L, Hkv, widths, depth)
+    rows = L * Hkv * G * nq
+    gemm = G * nq >= 64
+    Hp = r64(max(widths))
+    mod_ws = ((2 if depth >= 2 else 1) * a256(2 * rows * Hp * 2) + a256(rows * math.ceil(max(widths) / 128) * 4)
+              if gemm else 0)
+    assert nx.module_workspace_size(mods, G, nq) == mod_ws
+    loc = a256(rows * (d + 2) * 4)
+    dec_ws = loc + (mod_ws if gemm else a256(rows * 4))
+    assert nx.decode_workspace_size(mods, G, nq) == dec_ws
+    lo = int(nx.lib().nectar_decode_layer_out_workspace_size(nx.Dims(L, Hkv, G, d), mods.c(), nq))
+    assert lo == dec_ws + (0 if gemm else a256(rows * d * 4))
+
+
+@pytest.mark.parametrize("depths", [(2, 1, 2), (0, 2, 3), (1, 1, 1)])
+def test_workspace_sizes_of_backbone_sets(depths):
+    """A set with a backbone or unequal nets takes the layer-by-layer path at
+    any row count; its chain has D_b + max(D_s, D_t) hidden layers and Hp is
+    the widest layer of any part."""
+    L, Hkv, G, nq, d = 2, 2, 2, 1, 128
+    wb = [640, 256] if depths[0] else []
+    arch = nx.Arch(depths, wb, [384, 192], [512, 1008])
+    mods = _host_set(L, Hkv, None, None, arch)
+    rows = L * Hkv * G * nq
+    S = depths[0] + max(depths[1], depths[2])
+    Hp = r64(max([384, 192, 512, 1008] + wb))
+    mod_ws = (2 if S >= 2 else 1) * a256(2 * rows * Hp * 2) + a256(rows * math.ceil(384 / 128) * 4)
+    assert nx.module_workspace_size(mods, G, nq) == mod_ws
+    assert nx.decode_workspace_size(mods, G, nq) == a256(rows * (d + 2) * 4) + mod_ws
+
+
+def test_cache_attn_workspace_needs_a_device():
+    """The exact-attention scratch is planned for the current device's SM
+    count: with no device the size is 0 (and the compute call fails)."""
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    assert nx.cache_attn_workspace_size(2, 2, 2, 4096, 1) == 0
+    dims = nx.Dims(2, 2, 2, 128)
+    assert nx.lib().nectar_quadrature_workspace_size(dims, 512, 1) == 0
