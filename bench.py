@@ -519,7 +519,7 @@ def per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args):
         ws = torch.empty(max(nx.cache_attn_workspace_size(1, wl.Hkv, wl.G, wl.n, wl.nq), 16), dtype=torch.uint8,
                          device=dev)
         lmods = [mods.layer(l) for l in range(wl.L)] if has_decode else None
-        dws = torch.empty(max(nx.decode_workspace_size(lmods[0], wl.G, wl.nq) if has_decode else 16, 16),
+        dws = torch.empty(max(max(nx.decode_workspace_size(m, wl.G, wl.nq) for m in lmods) if has_decode else 16, 16),
                           dtype=torch.uint8, device=dev)
 
         def issue():

@@ -143,19 +143,54 @@ def _stream(stream) -> int:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def _need(t: torch.Tensor, name: str, dtype, device=True) -> None:
+def _need(t: torch.Tensor, name: str, dtype, shape=None, device=None) -> None:
+    """Checks that the library can take `t` as a pointer to `shape` elements
+    of `dtype` in CUDA memory: the C ABI sees only the pointer, so a host
+    tensor or a short buffer must be refused here."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
-    if device and not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
+    if shape is not None and tuple(t.shape) != tuple(int(x) for x in shape):
+        raise ValueError(f"{name} must have shape {tuple(int(x) for x in shape)}, got {tuple(t.shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the call runs on {device}")
+
+
+def _out(t: Optional[torch.Tensor], name: str, dtype, shape, device) -> torch.Tensor:
+    """A caller's output tensor, checked, or a new one."""
+    if t is None:
+        return torch.empty(tuple(shape), dtype=dtype, device=device)
+    _need(t, name, dtype, shape, device)
+    return t
+
+
+def _workspace(t: Optional[torch.Tensor], nbytes: int, device) -> Optional[torch.Tensor]:
+    """A caller's workspace (uint8, its size is checked by the library), or a
+    new one of `nbytes` when needed."""
+    if t is None:
+        return torch.empty(nbytes, dtype=torch.uint8, device=device) if nbytes > 0 else None
+    _need(t, "workspace", torch.uint8, device=device)
+    return t
+
+
+def _need_mods(mods: "ModuleSet", dims: Dims) -> None:
+    if not isinstance(mods, ModuleSet):
+        raise TypeError(f"mods must be a ModuleSet, got {type(mods).__name__}")
+    if (mods.L, mods.Hkv) != (dims.L, dims.Hkv):
+        raise ValueError(f"module set is for L={mods.L}, Hkv={mods.Hkv}; Q has L={dims.L}, Hkv={dims.Hkv}")
+    if mods.blob.device.type != "cuda":
+        raise ValueError("module weights must be on a CUDA device")
 
 
 def dims_of(Q: torch.Tensor) -> Tuple[Dims, int]:
     """Q: [L][Hkv][G][nq][d] -> (dims, nq)."""
-    if Q.dim() != 5:
-        raise ValueError("Q must be [L, Hkv, G, nq, d]")
+    if not isinstance(Q, torch.Tensor) or Q.dim() != 5:
+        raise ValueError("Q must be a tensor [L, Hkv, G, nq, d]")
     L_, Hkv, G, nq, d = Q.shape
     return Dims(L_, Hkv, G, d), nq
 
@@ -171,23 +206,28 @@ def cache_attn_workspace_size(L: int, Hkv: int, G: int, n: int, nq: int, d: int 
     return int(lib().nectar_cache_attn_workspace_size(Dims(L, Hkv, G, d), n, nq))
 
 
+def _cache_args(K, V, Q, dims: Dims) -> int:
+    """Checks K, V [L, Hkv, n, d] against Q [L, Hkv, G, nq, d]; returns n."""
+    _need(Q, "Q", torch.bfloat16)
+    if not isinstance(K, torch.Tensor) or K.dim() != 4:
+        raise ValueError("K must be a tensor [L, Hkv, n, d]")
+    n = K.shape[2]
+    for t, nm in ((K, "K"), (V, "V")):
+        _need(t, nm, torch.bfloat16, (dims.L, dims.Hkv, n, dims.d), Q.device)
+    return n
+
+
 def cache_attn_lse(K, V, Q, scale: Optional[float] = None, alpha=None, A=None, workspace=None, stream=None):
     """alpha [L,Hkv,G,nq] fp32 and A [L,Hkv,G,nq,d] fp32 of Eq. (3.1).
 
     K, V: bf16 [L, Hkv, n, d]; Q: bf16 [L, Hkv, G, nq, d] (CUDA)."""
     dims, nq = dims_of(Q)
-    n = K.shape[2]
-    for t, nm in ((K, "K"), (V, "V"), (Q, "Q")):
-        _need(t, nm, torch.bfloat16)
+    n = _cache_args(K, V, Q, dims)
     if scale is None:
         scale = 1.0 / math.sqrt(dims.d)
-    if alpha is None:
-        alpha = torch.empty(Q.shape[:4], dtype=torch.float32, device=Q.device)
-    if A is None:
-        A = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
-    ws_bytes = cache_attn_workspace_size(dims.L, dims.Hkv, dims.G, n, nq, dims.d)
-    if workspace is None and ws_bytes > 0:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    alpha = _out(alpha, "alpha", torch.float32, Q.shape[:4], Q.device)
+    A = _out(A, "A", torch.float32, Q.shape, Q.device)
+    workspace = _workspace(workspace, cache_attn_workspace_size(dims.L, dims.Hkv, dims.G, n, nq, dims.d), Q.device)
     st = lib().nectar_cache_attn_lse(dims, _ptr(K), _ptr(V), n, _ptr(Q), nq, float(scale), _ptr(alpha), _ptr(A),
                                      _ptr(workspace), 0 if workspace is None else workspace.numel(),
                                      _stream(stream))
@@ -199,15 +239,11 @@ def cache_attn_lse_static(K, V, Q, scale: Optional[float] = None, alpha=None, A=
     """As cache_attn_lse, through nectar_cache_attn_lse_static: no workspace is
     passed or allocated; the library's fixed device scratch area is used."""
     dims, nq = dims_of(Q)
-    n = K.shape[2]
-    for t, nm in ((K, "K"), (V, "V"), (Q, "Q")):
-        _need(t, nm, torch.bfloat16)
+    n = _cache_args(K, V, Q, dims)
     if scale is None:
         scale = 1.0 / math.sqrt(dims.d)
-    if alpha is None:
-        alpha = torch.empty(Q.shape[:4], dtype=torch.float32, device=Q.device)
-    if A is None:
-        A = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    alpha = _out(alpha, "alpha", torch.float32, Q.shape[:4], Q.device)
+    A = _out(A, "A", torch.float32, Q.shape, Q.device)
     st = lib().nectar_cache_attn_lse_static(dims, _ptr(K), _ptr(V), n, _ptr(Q), nq, float(scale), _ptr(alpha),
                                             _ptr(A), _stream(stream))
     _check(st, "nectar_cache_attn_lse_static")
@@ -372,25 +408,27 @@ def module_forward(mods: ModuleSet, Q, a=None, A_theta=None, workspace=None, str
     here when None and needed)."""
     dims, nq = dims_of(Q)
     _need(Q, "Q", torch.bfloat16)
-    if a is None:
-        a = torch.empty(Q.shape[:4], dtype=torch.float32, device=Q.device)
-    if A_theta is None:
-        A_theta = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
-    ws_bytes = module_workspace_size(mods, dims.G, nq, dims.d)
-    if workspace is None and ws_bytes > 0:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    _need_mods(mods, dims)
+    a = _out(a, "a", torch.float32, Q.shape[:4], Q.device)
+    A_theta = _out(A_theta, "A_theta", torch.float32, Q.shape, Q.device)
+    workspace = _workspace(workspace, module_workspace_size(mods, dims.G, nq, dims.d), Q.device)
     st = lib().nectar_module_forward(dims, mods.c(), _ptr(Q), nq, _ptr(a), _ptr(A_theta), _ptr(workspace),
                                      0 if workspace is None else workspace.numel(), _stream(stream))
     _check(st, "nectar_module_forward")
     return a, A_theta
 
 
-def _local_args(q_seq, q_pos, Kloc, Vloc, local_len):
-    for t, nm in ((q_seq, "q_seq"), (q_pos, "q_pos"), (local_len, "local_len")):
-        _need(t, nm, torch.int32)
-    for t, nm in ((Kloc, "Kloc"), (Vloc, "Vloc")):
-        _need(t, nm, torch.bfloat16)
+def _local_args(q_seq, q_pos, Kloc, Vloc, local_len, Q):
+    """Checks the local caches Kloc, Vloc [L, Hkv, B, T, d], q_seq, q_pos [nq]
+    and local_len [B] against Q [L, Hkv, G, nq, d]; returns (B, T)."""
+    L_, Hkv, _, nq, d = Q.shape
+    if not isinstance(Kloc, torch.Tensor) or Kloc.dim() != 5:
+        raise ValueError("Kloc must be a tensor [L, Hkv, B, T, d]")
     B, T = Kloc.shape[2], Kloc.shape[3]
+    for t, nm in ((Kloc, "Kloc"), (Vloc, "Vloc")):
+        _need(t, nm, torch.bfloat16, (L_, Hkv, B, T, d), Q.device)
+    for t, nm, n in ((q_seq, "q_seq", nq), (q_pos, "q_pos", nq), (local_len, "local_len", B)):
+        _need(t, nm, torch.int32, (n,), Q.device)
     return B, T
 
 
@@ -400,13 +438,12 @@ def merge_local(a, A_doc, Q, q_seq, q_pos, Kloc, Vloc, local_len, scale: Optiona
     exact causal attention over Kloc, Vloc [L,Hkv,B,T,d]."""
     dims, nq = dims_of(Q)
     _need(Q, "Q", torch.bfloat16)
-    _need(a, "a", torch.float32)
-    _need(A_doc, "A_doc", torch.float32)
-    B, T = _local_args(q_seq, q_pos, Kloc, Vloc, local_len)
+    _need(a, "a", torch.float32, Q.shape[:4], Q.device)
+    _need(A_doc, "A_doc", torch.float32, Q.shape, Q.device)
+    B, T = _local_args(q_seq, q_pos, Kloc, Vloc, local_len, Q)
     if scale is None:
         scale = 1.0 / math.sqrt(dims.d)
-    if out is None:
-        out = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    out = _out(out, "out", torch.float32, Q.shape, Q.device)
     st = lib().nectar_merge_local(dims, _ptr(a), _ptr(A_doc), _ptr(Q), nq, _ptr(q_seq), _ptr(q_pos), _ptr(Kloc),
                                   _ptr(Vloc), B, T, _ptr(local_len), float(scale), _ptr(out), _stream(stream))
     _check(st, "nectar_merge_local")
@@ -424,14 +461,12 @@ def decode(mods: ModuleSet, Q, q_seq, q_pos, Kloc, Vloc, local_len, scale: Optio
     here when None."""
     dims, nq = dims_of(Q)
     _need(Q, "Q", torch.bfloat16)
-    B, T = _local_args(q_seq, q_pos, Kloc, Vloc, local_len)
+    _need_mods(mods, dims)
+    B, T = _local_args(q_seq, q_pos, Kloc, Vloc, local_len, Q)
     if scale is None:
         scale = 1.0 / math.sqrt(dims.d)
-    if out is None:
-        out = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
-    ws_bytes = decode_workspace_size(mods, dims.G, nq, dims.d)
-    if workspace is None and ws_bytes > 0:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    out = _out(out, "out", torch.float32, Q.shape, Q.device)
+    workspace = _workspace(workspace, decode_workspace_size(mods, dims.G, nq, dims.d), Q.device)
     st = lib().nectar_decode(dims, mods.c(), _ptr(Q), nq, _ptr(q_seq), _ptr(q_pos), _ptr(Kloc), _ptr(Vloc), B, T,
                              _ptr(local_len), float(scale), _ptr(out), _ptr(workspace),
                              0 if workspace is None else workspace.numel(), _stream(stream))
@@ -445,14 +480,13 @@ def decode_layer_out(mods: ModuleSet, Q, q_seq, q_pos, Kloc, Vloc, local_len, sc
     (query head h*G + g), the fp32 result of decode() rounded to nearest."""
     dims, nq = dims_of(Q)
     _need(Q, "Q", torch.bfloat16)
-    B, T = _local_args(q_seq, q_pos, Kloc, Vloc, local_len)
+    _need_mods(mods, dims)
+    B, T = _local_args(q_seq, q_pos, Kloc, Vloc, local_len, Q)
     if scale is None:
         scale = 1.0 / math.sqrt(dims.d)
-    if out is None:
-        out = torch.empty((dims.L, nq, dims.Hkv * dims.G, dims.d), dtype=torch.bfloat16, device=Q.device)
-    ws_bytes = int(lib().nectar_decode_layer_out_workspace_size(dims, mods.c(), nq))
-    if workspace is None and ws_bytes > 0:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    out = _out(out, "out", torch.bfloat16, (dims.L, nq, dims.Hkv * dims.G, dims.d), Q.device)
+    workspace = _workspace(workspace, int(lib().nectar_decode_layer_out_workspace_size(dims, mods.c(), nq)),
+                           Q.device)
     st = lib().nectar_decode_layer_out(dims, mods.c(), _ptr(Q), nq, _ptr(q_seq), _ptr(q_pos), _ptr(Kloc),
                                        _ptr(Vloc), B, T, _ptr(local_len), float(scale), _ptr(out), _ptr(workspace),
                                        0 if workspace is None else workspace.numel(), _stream(stream))
@@ -463,13 +497,15 @@ def decode_layer_out(mods: ModuleSet, Q, q_seq, q_pos, Kloc, Vloc, local_len, sc
 def quadrature_init(K, V, p: int, W=None, Z=None, stream=None):
     """Quadrature module rows (section 2.4) initialised to the first p rows of
     the cache: W, Z bf16 [L, Hkv, p, d] (made here when None)."""
-    for t, nm in ((K, "K"), (V, "V")):
-        _need(t, nm, torch.bfloat16)
+    if not isinstance(K, torch.Tensor) or K.dim() != 4:
+        raise ValueError("K must be a tensor [L, Hkv, n, d]")
     L_, Hkv, n, d = K.shape
-    if W is None:
-        W = torch.empty((L_, Hkv, p, d), dtype=torch.bfloat16, device=K.device)
-    if Z is None:
-        Z = torch.empty((L_, Hkv, p, d), dtype=torch.bfloat16, device=K.device)
+    for t, nm in ((K, "K"), (V, "V")):
+        _need(t, nm, torch.bfloat16, K.shape, K.device)
+    if p < 0:
+        raise ValueError(f"p = {p}: need 1 <= p <= n")
+    W = _out(W, "W", torch.bfloat16, (L_, Hkv, p, d), K.device)
+    Z = _out(Z, "Z", torch.bfloat16, (L_, Hkv, p, d), K.device)
     st = lib().nectar_quadrature_init(Dims(L_, Hkv, 1, d), _ptr(K), _ptr(V), n, p, _ptr(W), _ptr(Z),
                                       _stream(stream))
     _check(st, "nectar_quadrature_init")
@@ -480,18 +516,12 @@ def quadrature_forward(W, Z, Q, scale: Optional[float] = None, a=None, A_theta=N
     """(a_theta [L,Hkv,G,nq], A_theta [L,Hkv,G,nq,d]) fp32 of the Quadrature
     module with rows W, Z bf16 [L, Hkv, p, d]."""
     dims, nq = dims_of(Q)
-    p = W.shape[2]
-    for t, nm in ((W, "W"), (Z, "Z"), (Q, "Q")):
-        _need(t, nm, torch.bfloat16)
+    p = _cache_args(W, Z, Q, dims)
     if scale is None:
         scale = 1.0 / math.sqrt(dims.d)
-    if a is None:
-        a = torch.empty(Q.shape[:4], dtype=torch.float32, device=Q.device)
-    if A_theta is None:
-        A_theta = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
-    ws_bytes = int(lib().nectar_quadrature_workspace_size(dims, p, nq))
-    if workspace is None and ws_bytes > 0:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    a = _out(a, "a", torch.float32, Q.shape[:4], Q.device)
+    A_theta = _out(A_theta, "A_theta", torch.float32, Q.shape, Q.device)
+    workspace = _workspace(workspace, int(lib().nectar_quadrature_workspace_size(dims, p, nq)), Q.device)
     st = lib().nectar_quadrature_forward(dims, _ptr(W), _ptr(Z), p, _ptr(Q), nq, float(scale), _ptr(a),
                                          _ptr(A_theta), _ptr(workspace),
                                          0 if workspace is None else workspace.numel(), _stream(stream))
@@ -505,10 +535,11 @@ def fit_metrics(alpha, A, a, A_theta, Q, metrics=None, stream=None):
     is metrics[..., 2].sum()."""
     dims, nq = dims_of(Q)
     _need(Q, "Q", torch.bfloat16)
-    for t, nm in ((alpha, "alpha"), (A, "A"), (a, "a"), (A_theta, "A_theta")):
-        _need(t, nm, torch.float32)
-    if metrics is None:
-        metrics = torch.empty((dims.L, dims.Hkv, 3), dtype=torch.float64, device=Q.device)
+    for t, nm in ((alpha, "alpha"), (a, "a")):
+        _need(t, nm, torch.float32, Q.shape[:4], Q.device)
+    for t, nm in ((A, "A"), (A_theta, "A_theta")):
+        _need(t, nm, torch.float32, Q.shape, Q.device)
+    metrics = _out(metrics, "metrics", torch.float64, (dims.L, dims.Hkv, 3), Q.device)
     st = lib().nectar_fit_metrics(dims, nq, _ptr(alpha), _ptr(A), _ptr(a), _ptr(A_theta), _ptr(Q), _ptr(metrics),
                                   _stream(stream))
     _check(st, "nectar_fit_metrics")

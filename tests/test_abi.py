@@ -219,3 +219,76 @@ def test_cache_attn_workspace_needs_a_device():
     assert nx.cache_attn_workspace_size(2, 2, 2, 4096, 1) == 0
     dims = nx.Dims(2, 2, 2, 128)
     assert nx.lib().nectar_quadrature_workspace_size(dims, 512, 1) == 0
+
+
+def _toy_host_inputs(L=2, Hkv=2, G=2, nq=3, n=16, B=2, T=8):
+    bf = torch.bfloat16
+    K = torch.zeros(L, Hkv, n, 128, dtype=bf)
+    Q = torch.zeros(L, Hkv, G, nq, 128, dtype=bf)
+    loc = (torch.zeros(nq, dtype=torch.int32), torch.zeros(nq, dtype=torch.int32),
+           torch.zeros(L, Hkv, B, T, 128, dtype=bf), torch.zeros(L, Hkv, B, T, 128, dtype=bf),
+           torch.full((B,), T, dtype=torch.int32))
+    a = torch.zeros(L, Hkv, G, nq)
+    A = torch.zeros(L, Hkv, G, nq, 128)
+    return K, Q, loc, a, A
+
+
+def test_binding_refuses_host_tensors():
+    """No compute call runs on host memory: the library sees raw pointers,
+    so the binding refuses CPU tensors instead of passing them on (and there
+    is no CPU fallback to take instead)."""
+    K, Q, loc, a, A = _toy_host_inputs()
+    mods = _host_set(2, 2, [64, 64], 2)
+    calls = [
+        lambda: nx.cache_attn_lse(K, K, Q),
+        lambda: nx.cache_attn_lse_static(K, K, Q),
+        lambda: nx.module_forward(mods, Q),
+        lambda: nx.merge_local(a, A, Q, *loc),
+        lambda: nx.decode(mods, Q, *loc),
+        lambda: nx.decode_layer_out(mods, Q, *loc),
+        lambda: nx.quadrature_init(K, K, 4),
+        lambda: nx.quadrature_forward(K, K, Q),
+        lambda: nx.fit_metrics(a, A, a, A, Q),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="CUDA"):
+            call()
+
+
+class _SeenAsCuda(torch.Tensor):
+    """A host tensor that claims to be on a CUDA device, so that the checks
+    after the device check can be reached on a machine without one.  Every
+    case below is refused before the library is called."""
+
+    @property
+    def is_cuda(self):
+        return True
+
+
+def test_binding_checks_shapes_and_dtypes():
+    """Inputs and caller-given outputs must have the shapes the call implies:
+    a short buffer would otherwise be read or written past its end."""
+    K, Q, loc, a, A = (x.as_subclass(_SeenAsCuda) if isinstance(x, torch.Tensor)
+                       else tuple(t.as_subclass(_SeenAsCuda) for t in x) for x in _toy_host_inputs())
+    with pytest.raises(ValueError, match="K must have shape"):
+        nx.cache_attn_lse(K[:1], K[:1], Q)                       # one layer of cache, two of queries
+    with pytest.raises(ValueError, match="V must have shape"):
+        nx.cache_attn_lse(K, K[:, :, :8], Q)                     # V shorter than K
+    with pytest.raises(ValueError, match="Kloc must have shape"):
+        nx.merge_local(a, A, Q, loc[0], loc[1], loc[2][:, :1], loc[3], loc[4])
+    with pytest.raises(ValueError, match="local_len must have shape"):
+        nx.merge_local(a, A, Q, loc[0], loc[1], loc[2], loc[3], loc[4][:1])
+    with pytest.raises(ValueError, match="q_pos must have shape"):
+        nx.merge_local(a, A, Q, loc[0], loc[1][:2], loc[2], loc[3], loc[4])
+    with pytest.raises(ValueError, match="a must have shape"):
+        nx.fit_metrics(a, A, a[:, :, :1], A, Q)
+    with pytest.raises(TypeError, match="A_theta must be torch.float32"):
+        nx.fit_metrics(a, A, a, A.double(), Q)
+    with pytest.raises(ValueError, match="Q must be a tensor"):
+        nx.module_forward(_host_set(2, 2, [64, 64], 2), Q[0])
+    with pytest.raises(ValueError, match="out must have shape"):
+        nx._out(torch.zeros(3), "out", torch.float32, (2, 2), None)
+    with pytest.raises(ValueError, match="module set is for L=1"):
+        nx._need_mods(_host_set(1, 2, [64], 2), nx.Dims(2, 2, 2, 128))
+    with pytest.raises(ValueError, match="module weights must be on a CUDA device"):
+        nx._need_mods(_host_set(2, 2, [64, 64], 2), nx.Dims(2, 2, 2, 128))

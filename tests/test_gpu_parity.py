@@ -445,3 +445,27 @@ def test_decode_workspace_checked():
     ref = nx.decode(mods, *args)
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
+
+
+def test_binding_refuses_mismatched_buffers():
+    """Caller-given outputs and module sets are checked against Q before any
+    launch; matching ones are written in place."""
+    wl = make_workload("toy", n=100, T=1, with_local=False, with_modules=True, seed=1, L=2, Hkv=2, G=2, nq=5,
+                       widths=[64, 64], depth=2)
+    K, V, Q = cuda(wl.K), cuda(wl.V), cuda(wl.Q)
+    with pytest.raises(ValueError, match="alpha must have shape"):
+        nx.cache_attn_lse(K, V, Q, alpha=torch.empty(2, 2, 2, 4, device="cuda"))
+    with pytest.raises(ValueError, match="A must be a CUDA tensor"):
+        nx.cache_attn_lse(K, V, Q, A=torch.empty(Q.shape))
+    with pytest.raises(TypeError, match="workspace must be torch.uint8"):
+        nx.cache_attn_lse(K, V, Q, workspace=torch.empty(1024, device="cuda"))
+    mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G)
+    with pytest.raises(ValueError, match="module set is for L=1"):
+        nx.module_forward(mods.layer(0), Q)
+    alpha = torch.empty(Q.shape[:4], device="cuda")
+    A = torch.empty(Q.shape, device="cuda")
+    got = nx.cache_attn_lse(K, V, Q, alpha=alpha, A=A)
+    assert got[0] is alpha and got[1] is A
+    ref = nx.cache_attn_lse(K, V, Q)
+    torch.cuda.synchronize()
+    assert torch.equal(alpha, ref[0]) and torch.equal(A, ref[1])
