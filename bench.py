@@ -35,7 +35,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from nectar_inputs import PRESETS, make_workload  # noqa: E402
+from nectar_inputs import PRESETS, make_workload, workload_shape  # noqa: E402
 
 METRIC = "Nectar decode queries/s & exact (α,A) HBM GB/s at 1 B200; % of roofline"
 UNIT = "queries/s"
@@ -167,9 +167,14 @@ class ClockSampler:
 # workload bookkeeping
 # ---------------------------------------------------------------------------
 def describe(wl):
-    H = sorted(set(wl.widths)) if wl.widths else []
-    return (f"{wl.name}: L={wl.L} Hkv={wl.Hkv} G={wl.G} d={wl.d} n={wl.n} B={wl.B} T={wl.T} "
-            f"nq={wl.nq} H={H[0] if len(H) == 1 else H} depth={wl.depth}")
+    return describe_shape(dict(name=wl.name, L=wl.L, Hkv=wl.Hkv, G=wl.G, d=wl.d, n=wl.n, B=wl.B, T=wl.T, nq=wl.nq,
+                               widths=wl.widths or [], depth=wl.depth))
+
+
+def describe_shape(s: dict) -> str:
+    H = sorted(set(s["widths"]))
+    return (f"{s['name']}: L={s['L']} Hkv={s['Hkv']} G={s['G']} d={s['d']} n={s['n']} B={s['B']} T={s['T']} "
+            f"nq={s['nq']} H={H[0] if len(H) == 1 else H} depth={s['depth']}")
 
 
 def queries_per_step(wl) -> int:
@@ -687,8 +692,12 @@ def run_reference(args):
         return
     import oracle
     oracle.build()
-    over = workload_overrides(args)
-    over["L"] = 1
+    # layer 0 of the full workload: its module width is the full workload's
+    # (widths solved per layer from rho depend on L)
+    full = workload_shape(args.workload, **workload_overrides(args))
+    over = dict(workload_overrides(args), L=1)
+    if full["widths"]:
+        over["widths"] = full["widths"][:1]
     wl = make_workload(args.workload, seed=args.seed, device="cpu", **over)
     host = _host_view(wl, [0], token_cap=_token_cap(wl))
     cores = oracle.num_threads()
@@ -698,7 +707,6 @@ def run_reference(args):
         done += _oracle_sample(host, [0])
     dt = time.perf_counter() - t0
     value = done / dt
-    full = PRESETS[args.workload]
     sample = (f"each step = the whole path over layer 0 of {full['L']} ({wl.Hkv} KV heads, {host.nq} of {wl.nq} "
               f"tokens x {wl.G} query heads) of {args.workload}")
     line = {
@@ -715,17 +723,13 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": describe_preset(args.workload), "parallelism": f"{cores} host threads"},
+        "config": {"workload": describe_shape(full), "global_batch": full["B"] * ws, "seq_len": full["n"],
+                   "parallelism": f"{cores} host threads",
+                   "queries_per_step_per_gpu": full["L"] * full["Hkv"] * full["G"] * full["nq"]},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
-
-
-def describe_preset(name):
-    p = PRESETS[name]
-    return (f"{name}: L={p['L']} Hkv={p['Hkv']} G={p['G']} d=128 n={p['n']} B={p['B']} T={p['T']} "
-            f"nq={p['nq']} H={p.get('H')}")
 
 
 def main():

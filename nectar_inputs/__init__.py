@@ -255,6 +255,32 @@ def make_modules_general(L: int, Hkv: int, d: int, seed: int, device, depths: Se
     return mods
 
 
+def _module_widths(cfg: dict, L: int, n: int, d: int) -> List[int]:
+    """Per-layer widths of a workload's modules: explicit, uniform H, or
+    solved per layer from the capacity rho."""
+    if "widths" in cfg:
+        return list(cfg["widths"])
+    if cfg.get("H"):
+        return [int(cfg["H"])] * L
+    return nonuniform_widths(cfg["rho"], L, n, d)
+
+
+def workload_shape(name: str, **overrides) -> dict:
+    """The sizes make_workload(name, **overrides) builds, without building
+    anything: name, L, Hkv, G, d, n, B, T, nq, and the modules' per-layer
+    widths (empty without modules) and depth."""
+    cfg = dict(PRESETS[name])
+    cfg.update(overrides)
+    L, n = cfg["L"], cfg["n"]
+    d = cfg.get("d", D_HEAD)
+    nq = cfg["nq"]
+    if cfg["mode"] == "decode":
+        nq = cfg.get("nq", cfg["B"]) if "nq" in overrides else cfg["B"]
+    with_modules = cfg.get("with_modules", cfg.get("modules", False))
+    return dict(name=name, L=L, Hkv=cfg["Hkv"], G=cfg["G"], d=d, n=n, B=cfg["B"], T=cfg["T"], nq=nq,
+                widths=_module_widths(cfg, L, n, d) if with_modules else [], depth=cfg.get("depth", 2))
+
+
 def make_workload(name: str, *, seed: int = 0, device="cpu", **overrides) -> Workload:
     """Build a preset workload (optionally with overridden sizes).
 
@@ -323,12 +349,7 @@ def make_workload(name: str, *, seed: int = 0, device="cpu", **overrides) -> Wor
 
     with_modules = cfg.get("with_modules", cfg.get("modules", False))
     if with_modules:
-        if "widths" in cfg:
-            widths = list(cfg["widths"])
-        elif cfg.get("H"):
-            widths = [int(cfg["H"])] * L
-        else:
-            widths = nonuniform_widths(cfg["rho"], L, n, d)
+        widths = _module_widths(cfg, L, n, d)
         wl.widths = widths
         wl.depth = cfg.get("depth", 2)
         wl.modules = make_modules(L, Hkv, widths, d, seed, dev, wl.depth)

@@ -52,3 +52,31 @@ def test_bench_single_process_identity():
     import bench
     assert bench.reduce_max(3.5) == 3.5
     assert bench.aggregate(448, 10.0, steps=10) == pytest.approx(448 * 10 / 0.010)
+
+
+@pytest.mark.parametrize("name,over", [
+    ("toy", {}),
+    ("qwen3_1p7b", dict(L=3, n=256)),
+    ("qwen3_4b_targets", dict(L=2, n=256, nq=8)),
+    ("qwen25_7b_decode", dict(L=2, n=256, B=3, T=8)),
+    ("llama8b_sweep", dict(L=10, n=1024, B=2, T=8)),          # widths solved per layer from rho
+])
+def test_workload_shape_is_what_make_workload_builds(name, over):
+    from nectar_inputs import make_workload, workload_shape
+    import bench
+    s = workload_shape(name, **over)
+    wl = make_workload(name, **over)
+    for k in ("L", "Hkv", "G", "d", "n", "B", "T", "nq"):
+        assert s[k] == getattr(wl, k), k
+    assert s["widths"] == (wl.widths or [])
+    assert bench.describe_shape(s) == bench.describe(wl)
+
+
+def test_reference_sample_is_layer_0_of_the_full_workload():
+    """With widths solved from rho, layer 0 of a 32-layer set is wider than a
+    one-layer set of the same capacity: the reference arm's one-layer sample
+    must take the full workload's layer-0 width."""
+    from nectar_inputs import workload_shape
+    full = workload_shape("llama8b_sweep")
+    alone = workload_shape("llama8b_sweep", L=1)
+    assert full["widths"][0] > alone["widths"][0]
