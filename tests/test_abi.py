@@ -292,3 +292,24 @@ def test_binding_checks_shapes_and_dtypes():
         nx._need_mods(_host_set(1, 2, [64], 2), nx.Dims(2, 2, 2, 128))
     with pytest.raises(ValueError, match="module weights must be on a CUDA device"):
         nx._need_mods(_host_set(2, 2, [64, 64], 2), nx.Dims(2, 2, 2, 128))
+
+
+def test_plain_c_client(tmp_path):
+    """The boundary is usable from C alone: tests/c_client/c_client.c
+    includes only include/nectar.h (C99, -pedantic -Werror), links
+    libnectar.so and exercises the entry points that need no GPU."""
+    import os
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not found")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(nx.LIB_PATH)
+    exe = str(tmp_path / "c_client")
+    r = subprocess.run([gcc, "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                        "-I", os.path.join(root, "include"), os.path.join(root, "tests", "c_client", "c_client.c"),
+                        "-L", libdir, "-lnectar", f"-Wl,-rpath,{libdir}", "-o", exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.startswith("ok "), r.stdout + r.stderr
