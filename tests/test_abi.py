@@ -297,7 +297,8 @@ def test_binding_checks_shapes_and_dtypes():
 def test_plain_c_client(tmp_path):
     """The boundary is usable from C alone: tests/c_client/c_client.c
     includes only include/nectar.h (C99, -pedantic -Werror), links
-    libnectar.so and exercises the entry points that need no GPU."""
+    libnectar.so and exercises the entry points that need no GPU, and the
+    per-thread error text from two threads at once."""
     import os
     import shutil
     import subprocess
@@ -309,7 +310,7 @@ def test_plain_c_client(tmp_path):
     exe = str(tmp_path / "c_client")
     r = subprocess.run([gcc, "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror",
                         "-I", os.path.join(root, "include"), os.path.join(root, "tests", "c_client", "c_client.c"),
-                        "-L", libdir, "-lnectar", f"-Wl,-rpath,{libdir}", "-o", exe], capture_output=True, text=True)
+                        "-L", libdir, "-lnectar", f"-Wl,-rpath,{libdir}", "-pthread", "-o", exe], capture_output=True, text=True)
     assert r.returncode == 0, r.stdout + r.stderr
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.startswith("ok "), r.stdout + r.stderr
