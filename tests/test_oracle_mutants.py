@@ -1,7 +1,8 @@
 """Strength of the oracle pins: plausible mistakes planted in a copy of the
 oracle's C source must each make tests/test_oracle_pins.py fail.
 
-Every mutant is one textual change of oracle/nectar_oracle.c -- a dropped
+Every mutant is one textual change of oracle/nectar_oracle.c (or of the
+oracle's Python side: parameter order, head selection) -- a dropped
 term or factor, a wrong sign, a transposed operand, an off-by-one index --
 applied to a scratch copy of the oracle package together with the pin tests
 and their golden files; the copy builds its own library and the pins run
@@ -17,6 +18,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "nectar_oracle.c")
+PY = os.path.join(ROOT, "oracle", "__init__.py")
 
 # (name, old text, new text): each old text occurs exactly once in the source
 MUTANTS = [
@@ -68,12 +70,24 @@ MUTANTS = [
     ("score error not squared", "s_sum += ds * ds;", "s_sum += ds;"),
 ]
 
+# the same for the oracle's Python side (parameter order, head selection)
+PY_MUTANTS = [
+    ("flatten_net: U_k before V_k", "parts += [Vs[k][h], U[k][h], b[k][h]]", "parts += [U[k][h], Vs[k][h], b[k][h]]"),
+    ("flatten_chain: U_k before V_k", "else [V[h], U[h], b[h]]", "else [U[h], V[h], b[h]]"),
+    ("module_forward: heads in reverse", "X = wl.Q[l, hs].reshape(len(hs), wl.rows, wl.d)",
+     "X = wl.Q[l, hs[::-1]].reshape(len(hs), wl.rows, wl.d)"),
+    ("quadrature: W and Z swapped", "return cache_attn(W, Z, Q, scale)", "return cache_attn(Z, W, Q, scale)"),
+    ("RTE summed over the wrong column", "float(out[:, 2].sum())", "float(out[:, 1].sum())"),
+]
 
-def _tree(base: str, source: str) -> str:
-    """A scratch repository holding the oracle (with `source` as its C file),
-    the input generators, the pin tests and their golden files."""
+
+def _tree(base: str, source: str, py_source: str) -> str:
+    """A scratch repository holding the oracle (with `source` as its C file
+    and `py_source` as its Python module), the input generators, the pin
+    tests and their golden files."""
     os.makedirs(os.path.join(base, "oracle"))
-    shutil.copy(os.path.join(ROOT, "oracle", "__init__.py"), os.path.join(base, "oracle"))
+    with open(os.path.join(base, "oracle", "__init__.py"), "w") as f:
+        f.write(py_source)
     with open(os.path.join(base, "oracle", "nectar_oracle.c"), "w") as f:
         f.write(source)
     shutil.copytree(os.path.join(ROOT, "nectar_inputs"), os.path.join(base, "nectar_inputs"),
@@ -98,17 +112,24 @@ def test_every_planted_mistake_fails_a_pin(tmp_path):
         pytest.skip("gcc not found")
     with open(SRC) as f:
         source = f.read()
+    with open(PY) as f:
+        py_source = f.read()
+    for name, old, _ in PY_MUTANTS:
+        assert py_source.count(old) == 1, f"mutant '{name}': its text occurs {py_source.count(old)} times"
     for name, old, new in MUTANTS:
         assert source.count(old) == 1, f"mutant '{name}': its text occurs {source.count(old)} times"
         chk = subprocess.run(["gcc", "-fsyntax-only", "-std=c11", "-fopenmp", "-x", "c", "-"],
                              input=source.replace(old, new), capture_output=True, text=True)
         assert chk.returncode == 0, f"mutant '{name}' does not compile:\n{chk.stderr}"
-    control = _run_pins(_tree(str(tmp_path / "control"), source))
+    control = _run_pins(_tree(str(tmp_path / "control"), source, py_source))
     assert control.returncode == 0, "the unmutated copy must pass:\n" + control.stdout[-3000:]
     jobs = {}
     with cf.ThreadPoolExecutor(max_workers=max(1, min(8, (os.cpu_count() or 2) // 2))) as ex:
         for k, (name, old, new) in enumerate(MUTANTS):
-            base = _tree(str(tmp_path / f"m{k}"), source.replace(old, new))
+            base = _tree(str(tmp_path / f"m{k}"), source.replace(old, new), py_source)
+            jobs[name] = ex.submit(_run_pins, base)
+        for k, (name, old, new) in enumerate(PY_MUTANTS):
+            base = _tree(str(tmp_path / f"p{k}"), source, py_source.replace(old, new))
             jobs[name] = ex.submit(_run_pins, base)
     survivors = [name for name, fut in jobs.items() if fut.result().returncode == 0]
     assert not survivors, f"mutants no pin catches: {survivors}"
