@@ -100,7 +100,8 @@ def read_net(blob, off, H, depth, dout, d=128):
     return out, off
 
 
-@pytest.mark.parametrize("widths,depth,hkv", [([64, 32], 2, 2), ([48], 3, 1), ([16, 208], 1, 3), ([272], 2, 1)])
+@pytest.mark.parametrize("widths,depth,hkv", [([64, 32], 2, 2), ([48], 3, 1), ([16, 208], 1, 3), ([272], 2, 1),
+                                               ([96, 1024], 4, 1)])   # the depth and width limits
 def test_pack_layout(widths, depth, hkv):
     mods = make_modules(len(widths), hkv, widths, 128, seed=3, device="cpu", depth=depth)
     ms = nx.pack_modules(mods, widths, depth, hkv, G=2, device=None)
@@ -314,3 +315,19 @@ def test_plain_c_client(tmp_path):
     assert r.returncode == 0, r.stdout + r.stderr
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.startswith("ok "), r.stdout + r.stderr
+
+
+def test_layer_depth_and_width_limits_on_the_host():
+    """NECTAR_MAX_LAYERS, NECTAR_MAX_DEPTH and NECTAR_MAX_WIDTH: the limit
+    itself is accepted, one past it is refused with the reason."""
+    L = nx.lib()
+    assert nx.packed_elems(256, 1, 1, [16] * 256, 1) > 0
+    assert nx.packed_elems(257, 1, 1, [16] * 257, 1) <= 0
+    assert b"L = 257" in L.nectar_last_error()
+    assert nx.packed_elems(1, 1, 1, [1024], 4) > 0
+    assert nx.packed_elems(1, 1, 1, [64], 5) <= 0
+    assert b"depth 5" in L.nectar_last_error()
+    assert nx.packed_elems(1, 1, 1, [1040], 2) <= 0
+    # a backbone chain counts against the depth limit as a whole
+    assert nx.Arch((2, 2, 1), [64], [64], [64]).packed_elems(1) > 0
+    assert nx.Arch((2, 3, 1), [64], [64], [64]).packed_elems(1) <= 0
