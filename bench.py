@@ -438,6 +438,8 @@ def next_rows(wl, mods, alpha, A, has_decode, dev, hbm_peak, tc_peak) -> dict:
     alone (inputs larger than L2 unless noted):
       quadrature: the Quadrature module forward at p = 10% of n;
       fit_metrics: score / target MSE and RTE over this step's targets;
+      layer_out_decode: the decode as a base-model attention layer (bf16,
+        layer layout);
       backbone_decode: the decode with a (2, 1, 2) module set (backbone,
         score, target depths) of this workload's widths."""
     import long_context_attention_split_b200 as nx
@@ -475,6 +477,20 @@ def next_rows(wl, mods, alpha, A, has_decode, dev, hbm_peak, tc_peak) -> dict:
                           "l2": "inputs smaller than L2" if fbytes < 126e6 else "inputs larger than L2"}
     del a, At, mws
     if has_decode:
+        # f1: the decode written as a base-model attention layer, bf16 in the
+        # layer layout [L][nq][Hkv*G][d]; bytes as the fused decode's with a
+        # 2-byte output
+        lo = torch.empty((wl.L, wl.nq, wl.Hkv * wl.G, wl.d), dtype=torch.bfloat16, device=dev)
+        lws_bytes = int(nx.lib().nectar_decode_layer_out_workspace_size(nx.Dims(wl.L, wl.Hkv, wl.G, wl.d), mods.c(),
+                                                                         wl.nq))
+        lws = torch.empty(max(lws_bytes, 16), dtype=torch.uint8, device=dev)
+        largs = (wl.Q, wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len)
+        t = _timed(lambda: nx.decode_layer_out(mods, *largs, out=lo, workspace=lws))
+        lbytes = decode_bytes(wl, mods.bytes) - wl.heads * wl.rows * 2 * wl.d
+        l_roof_us = max(lbytes / (hbm_peak * 1e9), decode_flops(wl) / (tc_peak * 1e12)) * 1e6
+        res["layer_out_decode"] = {"ms": t, "alg_bytes": lbytes, "roofline_us": l_roof_us,
+                                   "frac": l_roof_us / (t * 1e3)}
+        del lo, lws
         widths = list(wl.widths)
         gm = make_modules_general(wl.L, wl.Hkv, 128, 1, dev, (2, 1, 2), widths, widths, widths)
         arch = nx.Arch((2, 1, 2), widths, widths, widths)
