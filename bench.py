@@ -650,10 +650,37 @@ def cpu_baseline(wl, budget_s=12.0, layers_per_sample=1):
         if time.perf_counter() - t0 > budget_s or samples >= 400:
             break
     dt = time.perf_counter() - t0
+    # the same sample on one thread, for a quarter of the budget
+    oracle.set_threads(1)
+    try:
+        t1 = time.perf_counter()
+        done1 = samples1 = 0
+        while True:
+            done1 += _oracle_sample(host, list(range(len(layers))))
+            samples1 += 1
+            if time.perf_counter() - t1 > budget_s / 4 or samples1 >= 100:
+                break
+        dt1 = time.perf_counter() - t1
+    finally:
+        oracle.set_threads(cores)
     return {"value": done / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "value_1core": done1 / dt1, "cpu_model": cpu_model(),
             "sample": f"{samples} pass(es) of the whole path over layer(s) {layers} "
                       f"({len(layers) * wl.Hkv} of {wl.heads} KV heads, {host.nq} of {wl.nq} tokens x {wl.G} "
-                      f"query heads), {dt:.1f} s on {cores} threads; queries/s = query vectors done / time"}
+                      f"query heads), {dt:.1f} s on {cores} threads; queries/s = query vectors done / time; "
+                      f"value_1core: {samples1} pass(es) in {dt1:.1f} s on one thread"}
+
+
+def cpu_model() -> str:
+    """The host CPU's model name, as the kernel reports it."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def _token_cap(wl) -> int:
@@ -742,7 +769,8 @@ def run_reference(args):
         "config": {"workload": describe_shape(full), "global_batch": full["B"] * ws, "seq_len": full["n"],
                    "parallelism": f"{cores} host threads",
                    "queries_per_step_per_gpu": full["L"] * full["Hkv"] * full["G"] * full["nq"]},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                         "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
