@@ -309,7 +309,12 @@ def run_ours(args):
                 "unit": "GB/s", "frac": achieved / hbm_peak, "alg_bytes_per_launch": ab}
 
     # ---- the same step as L per-layer calls captured in one CUDA graph ----
-    per_layer = per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args)
+    pp = parts(wl, attn_avg, dec_avg, ab, db, qps, hbm_peak, tc_peak, has_decode)
+    exact_roof_us = max(ab / (hbm_peak * 1e9), af / (tc_peak * 1e12)) * 1e6
+    dec_roof_us = pp.get("decode_roofline_us_full", 0.0)
+    per_layer = per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args,
+                                roof_us={"step": exact_roof_us + dec_roof_us, "exact": exact_roof_us,
+                                         "decode": dec_roof_us})
     nextr = next_rows(wl, mods, alpha, A, has_decode, dev, hbm_peak, tc_peak) if args.next_rows else None
 
     # ---- end to end through the public API with host buffers ----
@@ -350,7 +355,9 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, budget_s=args.cpu_budget)
+        torch.cuda.synchronize(dev)
+        gpu_out = {"alpha": alpha, "A": A, "out": out if has_decode else None}
+        cpu = cpu_baseline(wl, budget_s=args.cpu_budget, gpu_out=gpu_out)
 
     if rank == 0:
         traffic = traffic_from_profile(args.workload)
@@ -375,8 +382,7 @@ def run_ours(args):
                 "queries_per_step_per_gpu": qps,
                 "l2": l2_note(ab),
             },
-            "parts": dict(parts(wl, attn_avg, dec_avg, ab, db, qps, hbm_peak, tc_peak, has_decode),
-                          per_layer_graph=per_layer, **({"next_rows": nextr} if nextr else {})),
+            "parts": dict(pp, per_layer_graph=per_layer, **({"next_rows": nextr} if nextr else {})),
             "roofline": dict(kernel=("cache_attn_tc+combine" if wl.rows > 8 else "cache_attn_split+combine")
                              + " (exact alpha, A)", traffic=traffic, **roof),
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -528,10 +534,13 @@ def l2_note(attn_bytes: float) -> str:
     return f"inputs of {attn_bytes / 1e6:.1f} MB fit in L2 (parity-size workload, not a bandwidth measurement)"
 
 
-def per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args):
+def per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args, roof_us=None):
     """ms per step when the step is issued as L per-layer calls (exact
     attention, then the decode, per layer) captured in one CUDA graph and
-    replayed; None when the workload has one layer."""
+    replayed -- the form a model that runs layer after layer gives -- and the
+    same for each half alone; None when the workload has one layer.
+    roof_us: {"step": .., "exact": .., "decode": ..} roofline times (us) of
+    the whole step and its halves, for the fractions."""
     if wl.L < 2:
         return None
     import long_context_attention_split_b200 as nx
@@ -543,35 +552,47 @@ def per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args):
         dws = torch.empty(max(max(nx.decode_workspace_size(m, wl.G, wl.nq) for m in lmods) if has_decode else 16, 16),
                           dtype=torch.uint8, device=dev)
 
-        def issue():
+        def issue(exact=True, decode=True):
             for l in range(wl.L):
                 sl = slice(l, l + 1)
-                nx.cache_attn_lse(wl.K[sl], wl.V[sl], Q[sl], alpha=alpha[sl], A=A[sl], workspace=ws, stream=s)
-                if has_decode:
+                if exact:
+                    nx.cache_attn_lse(wl.K[sl], wl.V[sl], Q[sl], alpha=alpha[sl], A=A[sl], workspace=ws, stream=s)
+                if decode and has_decode:
                     nx.decode(lmods[l], Q[sl], wl.q_seq, wl.q_pos, wl.Kloc[sl], wl.Vloc[sl], wl.local_len,
                               out=out[sl], workspace=dws, stream=s)
 
-        s.wait_stream(torch.cuda.current_stream(dev))
-        with torch.cuda.stream(s):
-            issue()                     # first calls outside the capture (device setup)
-        torch.cuda.synchronize(dev)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=s, capture_error_mode="relaxed"):
-            issue()
-        for _ in range(args.warmup):
-            g.replay()
-        torch.cuda.synchronize(dev)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(s):
-            e0.record(s)
-            for _ in range(args.steps):
+        def timed(**kw):
+            s.wait_stream(torch.cuda.current_stream(dev))
+            with torch.cuda.stream(s):
+                issue(**kw)             # first calls outside the capture (device setup)
+            torch.cuda.synchronize(dev)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s, capture_error_mode="relaxed"):
+                issue(**kw)
+            for _ in range(args.warmup):
                 g.replay()
-            e1.record(s)
-        torch.cuda.synchronize(dev)
-        ms = e0.elapsed_time(e1) / args.steps
-        del g
-        return {"ms_per_step": ms, "calls_per_step": wl.L * (2 if has_decode else 1)}
+            torch.cuda.synchronize(dev)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(s):
+                e0.record(s)
+                for _ in range(args.steps):
+                    g.replay()
+                e1.record(s)
+            torch.cuda.synchronize(dev)
+            del g
+            return e0.elapsed_time(e1) / args.steps
+
+        res = {"ms_per_step": timed(), "calls_per_step": wl.L * (2 if has_decode else 1)}
+        res["exact_ms"] = timed(decode=False)
+        if has_decode:
+            res["decode_ms"] = timed(exact=False)
+        if roof_us:
+            res["frac_step"] = roof_us["step"] / (res["ms_per_step"] * 1e3)
+            res["frac_exact"] = roof_us["exact"] / (res["exact_ms"] * 1e3)
+            if has_decode:
+                res["frac_decode_full"] = roof_us["decode"] / (res["decode_ms"] * 1e3)
+        return res
     except Exception as ex:  # report, do not fail the bench line
         return {"error": f"{type(ex).__name__}: {ex}"[:200]}
 
@@ -611,10 +632,11 @@ def traffic_from_profile(workload: str):
 # ---------------------------------------------------------------------------
 # CPU oracle baseline
 # ---------------------------------------------------------------------------
-def _oracle_sample(wl, layers):
+def _oracle_sample(wl, layers, keep=None):
     """One pass of the whole path on the oracle for the given layers (all
     their KV heads, the tokens kept in the host view).  Returns query
-    vectors processed."""
+    vectors processed; with keep (a dict) also leaves the outputs there:
+    alpha [H, rows], A [H, rows, d], out [H, rows, d] (H = layers x Hkv)."""
     import numpy as np
     import oracle
     H = len(layers) * wl.Hkv
@@ -622,18 +644,59 @@ def _oracle_sample(wl, layers):
     V = wl.V[layers].reshape(H, wl.n, wl.d)
     Q = wl.Q[layers].reshape(H, wl.rows, wl.d)
     alpha, A = oracle.cache_attn(K, V, Q, wl.scale)
+    if keep is not None:
+        keep.update(alpha=alpha, A=A)
     if wl.modules is None:
         return H * wl.rows
     sel = [(l, h) for l in layers for h in range(wl.Hkv)]
     a, At = oracle.module_forward(wl, sel)
     a = np.stack([a[k] for k in sel])
     At = np.stack([At[k] for k in sel])
-    oracle.merge_local(a, At, Q, wl.q_seq, wl.q_pos, wl.Kloc[layers].reshape(H, wl.B, wl.T, wl.d),
-                       wl.Vloc[layers].reshape(H, wl.B, wl.T, wl.d), wl.local_len, wl.scale)
+    out = oracle.merge_local(a, At, Q, wl.q_seq, wl.q_pos, wl.Kloc[layers].reshape(H, wl.B, wl.T, wl.d),
+                             wl.Vloc[layers].reshape(H, wl.B, wl.T, wl.d), wl.local_len, wl.scale)
+    if keep is not None:
+        keep.update(out=out, a=a, At=At)
     return H * wl.rows
 
 
-def cpu_baseline(wl, budget_s=12.0, layers_per_sample=1):
+def _sample_parity(wl, host, layers, ref, gpu_out) -> dict:
+    """Max errors of the timed step's GPU outputs on the oracle sample's
+    heads (layers `layers` of the workload, the host view's tokens), with
+    the tolerances the parity tests use: alpha 1e-3 absolute, A 2e-3 of
+    max|V|, the decode's out within the fused-decode bound (MLP 1e-2
+    relative carried through the merge)."""
+    import numpy as np
+    idx = torch.tensor(layers)
+    nq = host.nq
+
+    def rows(t):          # [L, Hkv, G, nq, ...] -> [H, G * nq, ...] of the sample's layers and tokens
+        t = t[idx.to(t.device)][:, :, :, :nq].cpu().numpy()
+        return t.reshape(len(layers) * wl.Hkv, wl.G * nq, *t.shape[4:])
+
+    res = {"heads": len(layers) * wl.Hkv, "layers": layers, "tokens": nq}
+    vmax = float(host.V.float().abs().max())
+    res["alpha_max_err"] = float(np.abs(rows(gpu_out["alpha"]) - ref["alpha"]).max())
+    res["A_max_err"] = float(np.abs(rows(gpu_out["A"]) - ref["A"]).max())
+    res["alpha_tol"] = 1e-3
+    res["A_tol"] = 2e-3 * vmax
+    ok = res["alpha_max_err"] <= res["alpha_tol"] and res["A_max_err"] <= res["A_tol"]
+    if gpu_out.get("out") is not None and "out" in ref:
+        a, At, o = ref["a"], ref["At"], ref["out"]
+        vl = max(float(host.Vloc.float().abs().max()), float(np.abs(At).max()))
+        bound = 1e-2 * np.abs(a).max() * (np.abs(At).max() + np.abs(o).max()) + 1e-2 * np.abs(At).max() + 2e-3 * vl
+        res["out_max_err"] = float(np.abs(rows(gpu_out["out"]) - o).max())
+        res["out_tol"] = float(bound)
+        ok = ok and res["out_max_err"] <= res["out_tol"]
+    res["pass"] = bool(ok)
+    return res
+
+
+def cpu_baseline(wl, budget_s=12.0, layers_per_sample=1, gpu_out=None):
+    """The oracle timed on the host cores on a bounded sample of the
+    workload (layer 0, all its KV heads).  With gpu_out (the timed step's
+    alpha, A and out on the device) the sample's oracle outputs, and those
+    of one more untimed pass over the last layer, also give the agreement of
+    the step's GPU outputs on those heads ("parity")."""
     import oracle
     oracle.build()
     cores = oracle.num_threads()
@@ -644,8 +707,9 @@ def cpu_baseline(wl, budget_s=12.0, layers_per_sample=1):
     t0 = time.perf_counter()
     done = 0
     samples = 0
+    first = {}
     while True:
-        done += _oracle_sample(host, list(range(len(layers))))
+        done += _oracle_sample(host, list(range(len(layers))), keep=first if samples == 0 else None)
         samples += 1
         if time.perf_counter() - t0 > budget_s or samples >= 400:
             break
@@ -663,12 +727,22 @@ def cpu_baseline(wl, budget_s=12.0, layers_per_sample=1):
         dt1 = time.perf_counter() - t1
     finally:
         oracle.set_threads(cores)
-    return {"value": done / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "value_1core": done1 / dt1, "cpu_model": cpu_model(),
-            "sample": f"{samples} pass(es) of the whole path over layer(s) {layers} "
-                      f"({len(layers) * wl.Hkv} of {wl.heads} KV heads, {host.nq} of {wl.nq} tokens x {wl.G} "
-                      f"query heads), {dt:.1f} s on {cores} threads; queries/s = query vectors done / time; "
-                      f"value_1core: {samples1} pass(es) in {dt1:.1f} s on one thread"}
+    res = {"value": done / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+           "value_1core": done1 / dt1, "cpu_model": cpu_model(),
+           "sample": f"{samples} pass(es) of the whole path over layer(s) {layers} "
+                     f"({len(layers) * wl.Hkv} of {wl.heads} KV heads, {host.nq} of {wl.nq} tokens x {wl.G} "
+                     f"query heads), {dt:.1f} s on {cores} threads; queries/s = query vectors done / time; "
+                     f"value_1core: {samples1} pass(es) in {dt1:.1f} s on one thread"}
+    if gpu_out is not None:
+        par = [_sample_parity(wl, host, layers, first, gpu_out)]
+        if wl.L > 1:
+            last = [wl.L - 1]
+            hl = _host_view(wl, last, token_cap=_token_cap(wl))
+            ref = {}
+            _oracle_sample(hl, [0], keep=ref)
+            par.append(_sample_parity(wl, hl, last, ref, gpu_out))
+        res["parity"] = par
+    return res
 
 
 def cpu_model() -> str:

@@ -121,8 +121,11 @@ NECTAR_API nectar_status nectar_cache_attn_lse(nectar_dims dims, const nectar_bf
  * (nectar_cache_attn_workspace_size) exceeds it returns
  * NECTAR_ERR_WORKSPACE with the two sizes in nectar_last_error().
  *  - The first call on a device looks up the area's device address (with
- *    that device current) and remembers it; make that first call before
- *    any stream capture.
+ *    that device current) and remembers it for the current CUDA context;
+ *    make that first call before any stream capture.  A later context on
+ *    the device (after cudaDeviceReset, or another context made current)
+ *    is detected by its id, and its first call looks the address up again,
+ *    so that call too belongs before any capture.
  *  - All calls on a device share the one area, and it keeps whatever the
  *    last call left there.  Nothing in it has to start at zero (every value
  *    read is first written by the same call), but two calls that overlap on
@@ -131,6 +134,10 @@ NECTAR_API nectar_status nectar_cache_attn_lse(nectar_dims dims, const nectar_bf
  * Arguments and outputs as for nectar_cache_attn_lse.
  * ------------------------------------------------------------------------ */
 #define NECTAR_STATIC_SCRATCH_BYTES (48u << 20)
+
+/* Size in bytes of the static scratch area this library was built with
+ * (NECTAR_STATIC_SCRATCH_BYTES).  Host only; never fails. */
+NECTAR_API size_t nectar_static_scratch_bytes(void);
 
 NECTAR_API nectar_status nectar_cache_attn_lse_static(nectar_dims dims, const nectar_bf16 *K,
                                                       const nectar_bf16 *V, int64_t n,
@@ -378,6 +385,16 @@ NECTAR_API const char *nectar_last_error(void);
  * of range, bit 2 = a local_len entry out of range.  SYNCHRONISES the
  * device; meant for tests and debugging, not for the hot path. */
 NECTAR_API nectar_status nectar_device_error_flags(int32_t *flags, int32_t clear);
+/* Self-check of the failure handling behind bit 0.  Every wait inside the
+ * library's kernels is bounded: it gives up after a time limit, sets bit 0
+ * of the device error word, and the kernel finishes without touching the
+ * data the wait guarded, so a lost arrival never hangs the GPU.  This call
+ * enqueues one small kernel whose thread waits, through that same bounded
+ * wait, on a barrier that nothing arrives on, with a limit of `limit_us`
+ * microseconds (1 .. 1000000): the wait runs out, bit 0 is set, the kernel
+ * returns and the context stays usable.  NECTAR_ERR_INVALID_ARG for a limit
+ * out of range.  For tests and health checks, not for the hot path. */
+NECTAR_API nectar_status nectar_check_wait_timeout(int32_t limit_us, nectar_stream_t stream);
 /* Library version, "major.minor.patch". */
 NECTAR_API const char *nectar_version(void);
 

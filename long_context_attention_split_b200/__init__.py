@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
     L.nectar_cache_attn_lse.restype = S
     L.nectar_cache_attn_lse_static.argtypes = [Dims, P, P, I64, P, I64, F, P, P, P]
     L.nectar_cache_attn_lse_static.restype = S
+    L.nectar_static_scratch_bytes.argtypes = []
+    L.nectar_static_scratch_bytes.restype = ctypes.c_size_t
     L.nectar_module_packed_elems.argtypes = [Dims, I32, P]
     L.nectar_module_packed_elems.restype = I64
     L.nectar_module_pack.argtypes = [Dims, I32, P, P, P, I64]
@@ -116,6 +118,8 @@ def lib() -> ctypes.CDLL:
     L.nectar_device_error_flags.argtypes = [ctypes.POINTER(ctypes.c_int32), I32]
     L.nectar_device_error_flags.restype = S
     L.nectar_version.restype = ctypes.c_char_p
+    L.nectar_check_wait_timeout.argtypes = [I32, P]
+    L.nectar_check_wait_timeout.restype = S
     _lib = L
     return L
 
@@ -250,7 +254,10 @@ def cache_attn_lse_static(K, V, Q, scale: Optional[float] = None, alpha=None, A=
     return alpha, A
 
 
-STATIC_SCRATCH_BYTES = 48 << 20
+def static_scratch_bytes() -> int:
+    """Size of the library's static scratch area (what
+    nectar_cache_attn_lse_static can use), as the library reports it."""
+    return int(lib().nectar_static_scratch_bytes())
 
 
 # ---------------------------------------------------------------------------
@@ -552,3 +559,10 @@ def device_error_flags(clear: bool = True) -> int:
     v = ctypes.c_int32(0)
     _check(lib().nectar_device_error_flags(ctypes.byref(v), 1 if clear else 0), "nectar_device_error_flags")
     return int(v.value)
+
+
+def check_wait_timeout(limit_us: int, stream=None) -> None:
+    """Enqueue the library's bounded-wait self-check: a wait that nothing
+    completes gives up after limit_us and sets bit 0 of the device error
+    word (read it with device_error_flags)."""
+    _check(lib().nectar_check_wait_timeout(int(limit_us), _stream(stream)), "nectar_check_wait_timeout")

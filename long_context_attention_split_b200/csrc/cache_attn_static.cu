@@ -12,9 +12,11 @@
 // the process exits.
 //
 // The array's name in host code is only a host-side handle, not a device
-// address, so the address is looked up once per device with
-// cudaGetSymbolAddress (with that device current) on the first call there,
-// and the kernels get that device address.
+// address, so the address is looked up with cudaGetSymbolAddress (with the
+// device current) on the first call in each CUDA context, and the kernels
+// get that device address.  A new context on the device (after
+// cudaDeviceReset, say) has a new id, and its first call looks the address
+// up again.
 #include <cuda_runtime.h>
 #include <stdio.h>
 
@@ -31,11 +33,17 @@ static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBy
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+struct ScratchAddr {
+  unsigned long long ctx = 0;   // id of the context the address belongs to
+  void* addr = nullptr;
+};
+ScratchAddr g_scratch_addr[kMaxDevices];
 
 }  // namespace
 
 extern "C" {
+
+NECTAR_API size_t nectar_static_scratch_bytes(void) { return kStaticScratchBytes; }
 
 NECTAR_API nectar_status nectar_cache_attn_lse_static(nectar_dims dims, const nectar_bf16* K, const nectar_bf16* V,
                                                       int64_t n, const nectar_bf16* Q, int64_t nq, float scale,
@@ -59,8 +67,11 @@ NECTAR_API nectar_status nectar_cache_attn_lse_static(nectar_dims dims, const ne
       return NECTAR_ERR_CUDA;
     }
     std::lock_guard<std::mutex> lk(g_mu);
-    if (g_scratch_addr[dev] == nullptr) {
+    ScratchAddr& c = g_scratch_addr[dev];
+    const unsigned long long ctx = nectar::current_context_id();
+    if (c.addr == nullptr || ctx == 0 || c.ctx != ctx) {
       void* addr = nullptr;
+      // also makes the device's primary context current if none is
       const cudaError_t e = cudaGetSymbolAddress(&addr, g_static_scratch);
       if (e != cudaSuccess || addr == nullptr) {
         char msg[256];
@@ -68,9 +79,10 @@ NECTAR_API nectar_status nectar_cache_attn_lse_static(nectar_dims dims, const ne
         nectar::set_last_error(msg);
         return NECTAR_ERR_CUDA;
       }
-      g_scratch_addr[dev] = addr;
+      c.addr = addr;
+      c.ctx = nectar::current_context_id();
     }
-    scratch = g_scratch_addr[dev];
+    scratch = c.addr;
   }
   return nectar_cache_attn_lse(dims, K, V, n, Q, nq, scale, alpha, A, scratch, need > 0 ? kStaticScratchBytes : 0,
                                stream);

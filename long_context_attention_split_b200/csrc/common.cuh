@@ -285,10 +285,11 @@ __device__ __forceinline__ int visible_local(const int32_t* q_seq, const int32_t
     record_error(err, DEVERR_BAD_LEN);
     len = len < 0 ? 0 : T;
   }
-  int nv = q_pos[i] + 1;
+  // in 64 bits, so that q_pos = INT_MAX sees all len keys rather than wrapping
+  int64_t nv = static_cast<int64_t>(q_pos[i]) + 1;
   if (nv > len) nv = len;
   if (nv < 0) nv = 0;
-  return nv;
+  return static_cast<int>(nv);
 }
 
 }  // namespace nectar

@@ -10,6 +10,9 @@ namespace nectar {
 
 // Sets the thread's nectar_last_error() text (defined with the C ABI).
 void set_last_error(const char* msg);
+// Id of the CUDA context current on the calling thread (0: none, or the
+// driver cannot tell).
+unsigned long long current_context_id();
 
 // ----- (i) split-n decode attention (CUDA cores) + LSE combine -------------
 struct DecParams {

@@ -30,6 +30,35 @@ thread_local char t_last_error[512] = "";
 
 void nectar::set_last_error(const char* msg) { snprintf(t_last_error, sizeof t_last_error, "%s", msg); }
 
+// cuCtxGetCurrent and cuCtxGetId through the runtime's driver entry points
+// (no link-time dependency on libcuda).  A context id is unique for the
+// life of the process, so a context made after a cudaDeviceReset has a new
+// one even where the driver reuses the handle.
+unsigned long long nectar::current_context_id() {
+  using GetCurrentFn = CUresult (*)(CUcontext*);
+  using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(ptr);
+    ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(ptr);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext c = nullptr;
+  if (get_current(&c) != CUDA_SUCCESS || c == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 namespace {
 
 nectar_status fail(nectar_status s, const char* fmt, ...) {
@@ -70,23 +99,35 @@ struct DeviceInfo {
   int* err = nullptr;   // device address of g_error_word on this device
 };
 
+// The SM count and the error word's device address of the current device.
+// The address belongs to the CUDA context it was looked up in, so the cache
+// is keyed on that context's id: after a cudaDeviceReset (or with another
+// context current) the next call looks it up again.
 DeviceInfo device_info() {
+  struct Entry {
+    unsigned long long ctx = 0;
+    DeviceInfo info;
+  };
   static std::mutex mu;
-  static std::vector<DeviceInfo> cache;
+  static std::vector<Entry> cache;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DeviceInfo{};
   std::lock_guard<std::mutex> lk(mu);
   if (static_cast<int>(cache.size()) <= dev) cache.resize(dev + 1);
-  if (cache[dev].sms == 0) {
+  Entry& e = cache[dev];
+  const unsigned long long ctx = current_context_id();
+  if (e.info.sms == 0 || ctx == 0 || e.ctx != ctx) {
     int sms = 0;
     void* err = nullptr;
+    // the symbol lookup also makes the device's primary context current
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaGetSymbolAddress(&err, nectar::g_error_word) != cudaSuccess)
       return DeviceInfo{};
-    cache[dev].err = static_cast<int*>(err);
-    cache[dev].sms = sms;
+    e.info.err = static_cast<int*>(err);
+    e.info.sms = sms;
+    e.ctx = current_context_id();
   }
-  return cache[dev];
+  return e.info;
 }
 
 // Query rows per KV head up to which exact attention stays on the CUDA-core
@@ -143,9 +184,32 @@ nectar_status make_tmap(CUtensorMap* map, const void* base, int rank, const cuui
 
 }  // namespace
 
+// One thread waits, through the library's bounded wait, on an mbarrier
+// that nothing arrives on; the wait gives up after limit_ns, records
+// DEVERR_WAIT_TIMEOUT and the kernel returns.
+__global__ void wait_timeout_kernel(uint64_t limit_ns, int* err) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(smem_u32(&bar), 0, err, limit_ns);
+}
+
 extern "C" {
 
 const char* nectar_version(void) { return "0.1.0"; }
+
+nectar_status nectar_check_wait_timeout(int32_t limit_us, nectar_stream_t stream) {
+  if (limit_us < 1 || limit_us > 1000000) return fail(NECTAR_ERR_INVALID_ARG, "limit_us = %d: need 1..1000000", limit_us);
+  const DeviceInfo di = device_info();
+  if (di.sms == 0) return fail(NECTAR_ERR_CUDA, "no CUDA device");
+  wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_us) * 1000u,
+                                                                           di.err);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "wait timeout check kernel");
+}
 
 const char* nectar_status_string(nectar_status s) {
   switch (s) {

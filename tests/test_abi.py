@@ -35,6 +35,15 @@ def test_status_strings_and_version():
     assert nx.version().count(".") == 2
 
 
+def test_static_scratch_size_is_the_headers():
+    # the size the library reports is the one include/nectar.h states
+    import re
+    with open(nx.HEADER_PATH) as f:
+        m = re.search(r"#define NECTAR_STATIC_SCRATCH_BYTES \((\d+)u << (\d+)\)", f.read())
+    assert m, "NECTAR_STATIC_SCRATCH_BYTES not found in the header"
+    assert nx.static_scratch_bytes() == int(m.group(1)) << int(m.group(2))
+
+
 def test_host_validation_without_device():
     L = nx.lib()
     bad_d = nx.Dims(1, 1, 1, 64)
@@ -56,6 +65,10 @@ def test_host_validation_without_device():
     assert L.nectar_module_packed_elems(nx.Dims(1, 1, 1, 128), 2, w) == 0
     w = (ctypes.c_int32 * 1)(64)
     assert L.nectar_module_packed_elems(nx.Dims(1, 1, 1, 128), 0, w) == 0
+    # the bounded-wait self-check takes 1 us .. 1 s, checked before any launch
+    for bad in (0, -1, 1000001):
+        assert L.nectar_check_wait_timeout(bad, None) == 1
+        assert b"limit_us" in L.nectar_last_error()
 
 
 # -- independent reader of the packed layout (as documented in module_layout.h) --

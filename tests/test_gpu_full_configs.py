@@ -38,23 +38,59 @@ def check_exact(wl, alpha, A, heads, tokens):
         assert np.abs(Ag - Ao).max() <= ATT_TOL * vmax, ((l, h), np.abs(Ag - Ao).max())
 
 
-def check_decode(wl, out, heads, tokens):
+def check_decode(wl, out, heads, tokens, a_gpu=None, At_gpu=None):
     """Fused decode output of the rows of `tokens` against the oracle's
-    module forward + merge for those rows."""
+    module forward + merge for those rows.  With the GPU's own module
+    outputs (a_gpu, At_gpu from nx.module_forward) the merge step is also
+    checked alone, at the attention tolerance: those outputs through the
+    oracle's merge (Eqs. (3.4)-(3.5)) must give the decode's out."""
     tok = torch.as_tensor(tokens)
     for (l, h) in heads:
         H = wl.widths[l]
         X = wl.Q[l, h][:, tok].reshape(1, -1, 128).cpu()
         a = oracle.mlp(oracle.flatten_net(wl.modules[l]["score"], [h]), X, wl.depth, H, 1)[..., 0]
         At = oracle.mlp(oracle.flatten_net(wl.modules[l]["target"], [h]), X, wl.depth, H, 128)
-        ref = oracle.merge_local(a, At, X, wl.q_seq[tok].cpu(), wl.q_pos[tok].cpu(),
-                                 wl.Kloc[l, h][None].cpu(), wl.Vloc[l, h][None].cpu(), wl.local_len.cpu(), wl.scale)
+        loc = (wl.q_seq[tok].cpu(), wl.q_pos[tok].cpu(), wl.Kloc[l, h][None].cpu(), wl.Vloc[l, h][None].cpu(),
+               wl.local_len.cpu())
+        ref = oracle.merge_local(a, At, X, *loc, wl.scale)
         got = out[l, h][:, tok].reshape(1, -1, 128).cpu().numpy()
-        vmax = max(wl.Vloc[l, h].float().abs().max().item(), np.abs(At).max())
+        vloc = wl.Vloc[l, h].float().abs().max().item()
+        vmax = max(vloc, np.abs(At).max())
         bound = MLP_TOL * np.abs(a).max() * (np.abs(At).max() + np.abs(ref).max()) + MLP_TOL * np.abs(At).max() \
             + ATT_TOL * vmax
         err = np.abs(got - ref).max()
         assert err <= bound, ((l, h), err, bound)
+        if a_gpu is not None:
+            ag = a_gpu[l, h][:, tok].reshape(1, -1).cpu().numpy()
+            Atg = At_gpu[l, h][:, tok].reshape(1, -1, 128).cpu().numpy()
+            # the module outputs themselves, at the MLP tolerance
+            assert np.abs(ag - a).max() <= MLP_TOL * np.abs(a).max(), (l, h)
+            assert np.abs(Atg - At).max() <= MLP_TOL * np.abs(At).max(), (l, h)
+            ref_m = oracle.merge_local(ag, Atg, X, *loc, wl.scale)
+            tol_m = ATT_TOL * max(vloc, np.abs(Atg).max())
+            err_m = np.abs(got - ref_m).max()
+            assert err_m <= tol_m, ((l, h), err_m, tol_m)
+
+
+def test_qwen3_1p7b_decode_full():
+    """The headline step exactly as bench.py runs it: 28 x 8 KV heads, G = 2,
+    n = 32768 with per-head key scales, H = 512, one decode token after 512
+    local tokens (the one-launch decode with its local CTAs first, and the
+    split exact-attention kernel at 2 rows per KV head).  Every (l, h) is
+    checked: exact (alpha, A), the module outputs, the merge step alone and
+    the decode output."""
+    wl = make_workload("qwen3_1p7b", device="cuda")
+    mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G, device="cuda")
+    alpha, A = nx.cache_attn_lse(wl.K, wl.V, wl.Q)
+    out = nx.decode(mods, wl.Q, wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len)
+    a, At = nx.module_forward(mods, wl.Q)
+    torch.cuda.synchronize()
+    assert nx.device_error_flags() == 0
+    heads = [(l, h) for l in range(wl.L) for h in range(wl.Hkv)]
+    check_exact(wl, alpha, A, heads, [0])
+    check_decode(wl, out, heads, [0], a, At)
+    del wl, mods, alpha, A, out, a, At
+    torch.cuda.empty_cache()
 
 
 def test_qwen3_4b_targets_full():
@@ -75,11 +111,12 @@ def test_qwen25_7b_decode_full():
     alpha, A = nx.cache_attn_lse(wl.K, wl.V, wl.Q)
     out = nx.decode(mods, wl.Q, wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len)
     full = nx.merge_local(alpha, A, wl.Q, wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len)
+    a, At = nx.module_forward(mods, wl.Q)
     torch.cuda.synchronize()
     assert nx.device_error_flags() == 0
     heads = sample_heads(wl, 3, 2)
     check_exact(wl, alpha, A, heads, [0, 37, 63])
-    check_decode(wl, out, heads, [0, 37, 63])
+    check_decode(wl, out, heads, [0, 37, 63], a, At)
     # Eq. (3.4): merging the exact (alpha, A) is full attention over document + local
     (l, h) = heads[0]
     tok = torch.tensor([5])
@@ -90,7 +127,7 @@ def test_qwen25_7b_decode_full():
     got = full[l, h][:, tok].reshape(1, -1, 128).cpu().numpy()
     vmax = max(wl.V[l, h].float().abs().max().item(), wl.Vloc[l, h].float().abs().max().item())
     assert np.abs(got - ref).max() <= ATT_TOL * vmax
-    del wl, mods, alpha, A, out, full
+    del wl, mods, alpha, A, out, full, a, At
     torch.cuda.empty_cache()
 
 
@@ -101,11 +138,12 @@ def test_llama8b_sweep_full(B, rho):
     mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G, device="cuda")
     alpha, A = nx.cache_attn_lse(wl.K, wl.V, wl.Q)
     out = nx.decode(mods, wl.Q, wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len)
+    a, At = nx.module_forward(mods, wl.Q)
     torch.cuda.synchronize()
     assert nx.device_error_flags() == 0
     heads = sample_heads(wl, 3, B)
     tokens = sorted({0, B // 2, B - 1})
     check_exact(wl, alpha, A, heads, tokens)
-    check_decode(wl, out, heads, tokens)
-    del wl, mods, alpha, A, out
+    check_decode(wl, out, heads, tokens, a, At)
+    del wl, mods, alpha, A, out, a, At
     torch.cuda.empty_cache()

@@ -87,6 +87,45 @@ def test_fit_metrics_against_oracle():
 # ---------------------------------------------------------------------------
 # the decode as a base-model attention layer: bf16, layer layout
 # ---------------------------------------------------------------------------
+MLP_TOL = 1e-2
+
+
+def _to_layer_layout(x, wl):
+    """[heads, rows, d] (rows = g * nq + i) -> [L, nq, Hkv * G, d]."""
+    return x.reshape(wl.L, wl.Hkv, wl.G, wl.nq, 128).transpose(0, 3, 1, 2, 4).reshape(wl.L, wl.nq, wl.Hkv * wl.G,
+                                                                                        128)
+
+
+def _check_layer_out_against_oracle(wl, mods, args, got):
+    """bf16 layer-layout output against the oracle, through the bf16 rounding
+    (at most 2^-8 of the value, with margin): (1) the GPU's own module outputs
+    through the oracle's merge, at the attention tolerance; (2) the oracle's
+    module forward + merge, at the fused-decode bound."""
+    a, At = nx.module_forward(mods, args[0])
+    torch.cuda.synchronize()
+    H = wl.heads
+    loc = (wl.q_seq, wl.q_pos, wl.Kloc.reshape(H, wl.B, wl.T, 128), wl.Vloc.reshape(H, wl.B, wl.T, 128),
+           wl.local_len, wl.scale)
+    Qr = wl.Q.reshape(H, wl.rows, 128)
+    g = got.float().cpu().numpy()
+    rnd = 2.0 ** -8 * np.abs(g) * 1.01
+    vloc = wl.Vloc.float().abs().max().item()
+    ag = a.cpu().numpy().reshape(H, wl.rows)
+    Atg = At.cpu().numpy().reshape(H, wl.rows, 128)
+    ref_m = _to_layer_layout(oracle.merge_local(ag, Atg, Qr, *loc), wl)
+    tol_m = ATT_TOL * max(vloc, np.abs(Atg).max())
+    assert np.all(np.abs(g - ref_m) <= rnd + tol_m), np.abs(g - ref_m).max()
+    ao, Ao = oracle.module_forward(wl)
+    keys = [(l, h) for l in range(wl.L) for h in range(wl.Hkv)]
+    a_o = np.stack([ao[k] for k in keys])
+    A_o = np.stack([Ao[k] for k in keys])
+    ref = oracle.merge_local(a_o, A_o, Qr, *loc)
+    bound = MLP_TOL * np.abs(a_o).max() * (np.abs(A_o).max() + np.abs(ref).max()) + MLP_TOL * np.abs(A_o).max() \
+        + ATT_TOL * max(vloc, np.abs(A_o).max())
+    ref = _to_layer_layout(ref, wl)
+    assert np.all(np.abs(g - ref) <= rnd + bound), np.abs(g - ref).max()
+
+
 @pytest.mark.parametrize("kw", [
     dict(L=2, Hkv=2, G=2, n=16, B=3, T=40, widths=[256, 128]),   # 2 rows per KV head: one-launch path
     dict(L=2, Hkv=2, G=4, n=16, B=40, T=50, widths=[256, 512]),  # 160 rows: grouped-GEMM path
@@ -100,6 +139,7 @@ def test_decode_layer_out_is_decode_in_layer_layout(kw):
     torch.cuda.synchronize()
     want = ref.permute(0, 3, 1, 2, 4).reshape(wl.L, wl.nq, wl.Hkv * wl.G, 128).to(torch.bfloat16)
     assert torch.equal(got, want)
+    _check_layer_out_against_oracle(wl, mods, args, got)
 
 
 def test_decode_layer_out_prefill_causal():
@@ -112,3 +152,22 @@ def test_decode_layer_out_prefill_causal():
     torch.cuda.synchronize()
     want = ref.permute(0, 3, 1, 2, 4).reshape(wl.L, wl.nq, wl.Hkv * wl.G, 128).to(torch.bfloat16)
     assert torch.equal(got, want)
+    _check_layer_out_against_oracle(wl, mods, args, got)
+
+
+def test_decode_layer_out_prompt_several_sequences():
+    # prompts of 3 sequences at once (64 tokens of each, token t at local
+    # position t), the bf16 layer layout against the oracle
+    T = 64
+    B = 3
+    nq = B * T
+    q_seq = [b for b in range(B) for _ in range(T)]
+    q_pos = [t for _ in range(B) for t in range(T)]
+    wl = make_workload("toy", seed=12, L=2, Hkv=2, G=2, n=16, B=B, T=T, nq=nq, widths=[256, 128],
+                       q_seq=q_seq, q_pos=q_pos, local_len=[T, T - 5, 40])
+    mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G)
+    args = tuple(t.cuda() for t in (wl.Q, wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len))
+    got = nx.decode_layer_out(mods, *args)
+    torch.cuda.synchronize()
+    assert nx.device_error_flags() == 0
+    _check_layer_out_against_oracle(wl, mods, args, got)

@@ -208,12 +208,16 @@ def test_merge_prefill_causal():
 
 def test_merge_edge_cases():
     # q_pos 0; local_len 1; local_len = T_max; local_len 0 -> out = A_doc;
-    # q_pos past local_len (sees local_len tokens)
+    # q_pos past local_len (sees local_len tokens); q_pos = INT32_MAX (sees
+    # all local_len tokens: the visible count q_pos + 1 must not wrap)
     T = 9
-    out, Ad = merge_case(3, 5, 4, T, [0, 1, 2, 3, 1], [0, 5, T - 1, 2, 8], [T, 1, T, 0], seed=4)
-    o = out.cpu().reshape(2, 3, 5, 128)
-    A = Ad.reshape(2, 3, 5, 128)
+    out, Ad = merge_case(3, 6, 4, T, [0, 1, 2, 3, 1, 2], [0, 5, T - 1, 2, 8, 2**31 - 1], [T, 1, T, 0], seed=4)
+    o = out.cpu().reshape(2, 3, 6, 128)
+    A = Ad.reshape(2, 3, 6, 128)
     assert torch.equal(o[:, :, 3], A[:, :, 3])
+    # the INT32_MAX token and a token at the last position see the same keys
+    out2, _ = merge_case(3, 6, 4, T, [0, 1, 2, 3, 1, 2], [0, 5, T - 1, 2, 8, T - 1], [T, 1, T, 0], seed=4)
+    assert torch.equal(out[..., 5, :], out2[..., 5, :])
 
 
 def test_merge_bad_metadata_flags():
@@ -247,6 +251,7 @@ def test_merge_many_tokens(G, T):
     local_len = [T, 0, 1, T // 2 + 3, T - 1]
     q_pos = torch.randint(0, T, (nq,), generator=g).tolist()
     q_pos[0] = 0
+    q_pos[1] = 2**31 - 1          # sees its whole sequence
     out, Ad = merge_case(G, nq, B, T, q_seq, q_pos, local_len, seed=G + T)
     # tokens of the sequence with no local tokens keep the document term
     o = out.cpu().reshape(2, G, nq, 128)
@@ -397,6 +402,16 @@ def decode_case(wl):
     bound = da * (np.abs(A_o).max() + np.abs(ref).max()) + dA + ATT_TOL * vmax
     err = np.abs(got - ref).max()
     assert err <= bound, (err, bound)
+    # the merge step alone, at the attention tolerance: the GPU's own
+    # (a_theta, A_theta) through the oracle's merge (Eqs. (3.4)-(3.5))
+    ag = a.cpu().numpy().reshape(H, wl.rows)
+    Atg = At.cpu().numpy().reshape(H, wl.rows, 128)
+    ref_m = oracle.merge_local(ag, Atg, wl.Q.reshape(H, wl.rows, 128), wl.q_seq, wl.q_pos,
+                               wl.Kloc.reshape(H, wl.B, wl.T, 128), wl.Vloc.reshape(H, wl.B, wl.T, 128),
+                               wl.local_len, wl.scale)
+    vmax_m = max(wl.Vloc.float().abs().max().item(), np.abs(Atg).max())
+    err_m = np.abs(got - ref_m).max()
+    assert err_m <= ATT_TOL * vmax_m, (err_m, ATT_TOL * vmax_m)
     # fused == unfused on the GPU (same arithmetic, different summation order)
     assert torch.allclose(out, out2, rtol=0, atol=1e-4 * max(1.0, out2.abs().max().item()))
 
