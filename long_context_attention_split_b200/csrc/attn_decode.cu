@@ -84,6 +84,18 @@ cache_attn_split_kernel(const DecParams p) {
   if (warp == kDecWarps) {
     // ---------------- producer ----------------
     if (lane == 0) {
+      // the first stages' K and V towards L2 while an earlier kernel finishes
+      for (int64_t tt = t0; tt < t1 && tt < t0 + kDecStages; ++tt) {
+        const int64_t hd = tt / p.tph;
+        const int64_t j0 = (tt - hd * p.tph) * TILE;
+        const int64_t cnt = (p.n - j0 < TILE) ? (p.n - j0) : TILE;
+        const size_t off = (static_cast<size_t>(hd) * p.n + j0) * kD;
+        prefetch_l2(p.K + off, static_cast<uint32_t>(cnt) * kRowBytes);
+        prefetch_l2(p.V + off, static_cast<uint32_t>(cnt) * kRowBytes);
+      }
+    }
+    griddep_wait();
+    if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       int64_t i = 0;
       for (int64_t tt = t0; tt < t1; ++tt, ++i) {
@@ -100,8 +112,10 @@ cache_attn_split_kernel(const DecParams p) {
         bulk_g2s(smem_u32(sV + s * TILE * kRowBytes), p.V + off, bytes, full0 + 8 * s, pol);
       }
     }
+    griddep_launch();
     return;
   }
+  griddep_wait();
 
   // ---------------- consumers ----------------
   const int g = lane / LPK, t = lane % LPK;
@@ -206,6 +220,7 @@ cache_attn_split_kernel(const DecParams p) {
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * s);
   }
+  griddep_launch();               // the combine may start launching
   if (cur >= 0) finalize(cur);
 }
 
@@ -214,6 +229,8 @@ cache_attn_split_kernel(const DecParams p) {
 // 2^{m_s - M} / sum_s l_s 2^{m_s - M}.
 __global__ void cache_attn_combine_kernel(const DecParams p, float* __restrict__ alpha,
                                           float* __restrict__ A) {
+  griddep_wait();
+  griddep_launch();
   const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= static_cast<int64_t>(p.heads) * p.rows_total) return;
@@ -255,8 +272,7 @@ static cudaError_t launch_split(const DecParams& p, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(cache_attn_split_kernel<R, LPK, NRG>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  cache_attn_split_kernel<R, LPK, NRG><<<p.C, kDecThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_k(cache_attn_split_kernel<R, LPK, NRG>, dim3(p.C), dim3(kDecThreads), smem, stream, 1, p);
 }
 
 int dec_max_rows() { return 8; }
@@ -341,8 +357,8 @@ cudaError_t launch_cache_attn_combine(const DecParams& p, float* alpha, float* A
   if (warps == 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = (warps * 32 + threads - 1) / threads;
-  cache_attn_combine_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(p, alpha, A);
-  return cudaGetLastError();
+  return launch_k(cache_attn_combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream, 1, p,
+                  alpha, A);
 }
 
 }  // namespace nectar

@@ -1,0 +1,646 @@
+// Nectar decode for few query rows per KV head, one thread-block cluster per
+// (layer l, KV head h): the score and target nets of Eq. (3.6) and the merge
+// of Eqs. (3.4)-(3.5) with the exact causal attention over the local tokens
+// (§2.2, §2.4 of "Nectar: Neural Estimation of Cached-Token Attention via
+// Regression"), all in one launch and with no workspace.
+//
+// Why a cluster.  At a few query rows per KV head the module forward is a
+// weight stream: every weight is used once per row.  One CTA per (l, h)
+// streams the head's whole module through one SM, which is slow when a call
+// has few heads (one layer of a model run layer after layer: 8 heads on 148
+// SMs).  Here the hidden units of every layer of both nets are cut into
+// kClusterCtas slices of a multiple of 64 units, one per CTA of the
+// cluster, so the head's weights stream through kClusterCtas SMs at once.
+//
+// Per CTA (rank r, units [u0, u0 + slen) of each net):
+//  - hidden layer k: the rows of W_k for its units (A, swap-AB: M = 128
+//    units -- a 64-unit slice uses the lanes 0-63 of an M = 128 tile whose
+//    other rows it ignores --, N = the head's query rows, K = d or d + H),
+//    streamed from the packed blob by bulk copies through a ring, times
+//    X = [q | h_{k-1}] (B, resident, K-major, 128-byte swizzle) into TMEM;
+//    the epilogue adds the bias, applies SiLU, writes its slice of h_k into
+//    its own X as bf16 and copies that slice into the X of every other CTA
+//    of the cluster (DSMEM bulk copies that complete on the receiver's
+//    mbarrier: point to point, no multicast).  The next layer starts once
+//    every slice has landed.  Depth >= 3 alternates two h buffers, so that
+//    a buffer is written again only two layers after it was sent, when every
+//    receiver has it (and so every copy out of it has read it); the target's
+//    last layer writes a region of its own, the readout's input.
+//  - last hidden layer: the score net's readout w . h is summed over the
+//    CTA's units in the epilogue registers; the target net's readout
+//    W_out[:, slice] h_slice is one more MMA (M = d, K = the slice).
+//  - local attention: 4 warps score the CTA's share of every query token's
+//    visible local keys (the keys cut into kClusterCtas ranges) on the CUDA
+//    cores, leaving a partial (m, l, acc) per row.
+//  - reduction and merge: CTA o owns output dims [16 o, 16 o + 16).  Every
+//    CTA stores its partials into the owners' shared memory (score partial
+//    of each row to all, target and local partials of each dim to that
+//    dim's owner), one cluster barrier, and each owner sums the partials in
+//    a fixed order (deterministic), joins the local partials by
+//    log-sum-exp and merges: out = (2^{a'} A_theta + 2^{m} acc) /
+//    (2^{a'} + 2^{m} l) with a' = a_theta log2 e (Eqs. (3.4)-(3.5)).
+// Warp roles: 0 TMA producer, 1 MMA issuer (+ TMEM owner), 2-5 score-net
+// epilogue, 6-9 target-net epilogue, 10-13 local attention; all take part in
+// the merge's reduction.  Every mbarrier wait is bounded; every thread
+// reaches both cluster barriers (no early return).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "module_layout.h"
+#include "out_layout.cuh"
+
+namespace nectar {
+
+namespace {
+
+constexpr int kCl = kClusterCtas;
+constexpr int kOwnDims = kD / kCl;               // output dims merged by each CTA
+constexpr uint32_t kStage = 32 * 1024;           // weight ring stage
+constexpr uint32_t kPad = 8 * 1024;              // read (not used) past the ring by a 64-row tile
+constexpr int kEpiWarps = 8;
+constexpr int kLocWarps = 4;
+constexpr int kThreads = (2 + kEpiWarps + kLocWarps) * 32;
+constexpr int kLocKPG = 2;                        // keys per lane group per step
+
+struct ClSmem {
+  uint32_t ring, xq, xh, xro, rt, rl, rs, rml, sp, lscr, bars, tslot, total;
+};
+
+// 64-unit granules: the h slices exchanged between CTAs are whole 64-column
+// chunks of X
+__host__ __device__ inline int cl_slice(int H) {
+  const int s = (H + kCl - 1) / kCl;
+  return (s + 63) / 64 * 64;
+}
+__host__ __device__ inline int cl_slice_len(int H, int r) {
+  const int S = cl_slice(H);
+  const int len = H - r * S;
+  return len < 0 ? 0 : (len < S ? len : S);
+}
+
+// byte offsets from the 1024-aligned dynamic shared memory base
+__host__ __device__ inline ClSmem cl_layout(int Hmax, int N, int nb, int stages, int rg) {
+  ClSmem s{};
+  uint32_t off = 0;
+  s.ring = off;
+  off += static_cast<uint32_t>(stages) * kStage + kPad;
+  s.xq = off;                                                   // q: 2 chunks of [N][128 B]
+  off += 2u * N * 128;
+  s.xh = off;                                                   // h: [net][buf][chunk][N][128 B]
+  off += 2u * nb * layout::kchunks(Hmax) * N * 128;
+  s.xro = off;                                                  // the target readout's input: own slice
+  off += static_cast<uint32_t>(layout::kchunks(cl_slice(Hmax))) * N * 128;
+  s.rt = off;                                                   // target partials [src][dim][row]
+  off += static_cast<uint32_t>(kCl * kOwnDims * N) * 4;
+  s.rl = off;                                                   // local acc partials [src][row][dim]
+  off += static_cast<uint32_t>(kCl * N * kOwnDims) * 4;
+  s.rs = off;                                                   // score partials [src][row]
+  off += static_cast<uint32_t>(kCl * N) * 4;
+  s.rml = off;                                                  // local (m, l) [src][row][2]
+  off += static_cast<uint32_t>(kCl * N * 2) * 4;
+  s.sp = off;                                                   // score sums by lane quarter [4][N]
+  off += static_cast<uint32_t>(4 * N) * 4;
+  s.lscr = off;                                                 // local warps' states [warp][rg][d + 2]
+  off += static_cast<uint32_t>(kLocWarps * rg * (kD + 2)) * 4;
+  off = (off + 15) & ~15u;
+  s.bars = off;
+  off += 32 * 8;
+  s.tslot = off;
+  off += 16;
+  s.total = off;
+  return s;
+}
+
+__device__ __forceinline__ uint8_t* cl_aligned(uint8_t* raw) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ float cl_silu(float v) { return __fdividef(v, 1.0f + ex2(-v * kLog2e)); }
+
+// element (row n, column c) of a swizzled K-major [N][64]-chunk matrix
+__device__ __forceinline__ uint32_t cl_xoff(int N, int n, int c) {
+  return static_cast<uint32_t>((c >> 6) * (N * 128) + n * 128 + ((((c & 63) >> 3) ^ (n & 7)) << 4) +
+                               ((c & 7) << 1));
+}
+
+template <int RG>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = cl_aligned(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = static_cast<int>(cluster_ctarank());
+  const int ci = static_cast<int>(blockIdx.x) / kCl;
+  const int li = ci / p.Hkv, h = ci % p.Hkv;
+  const int l = p.order[li];
+  const int H = p.width[l];
+  const int depth = p.depth;
+  const int N = p.N;
+  const int nb = p.nb;
+  const int HC = layout::kchunks(p.Hmax);
+  const int S_ = p.stages;
+  const ClSmem SL = cl_layout(p.Hmax, N, nb, S_, RG);
+  const int S = cl_slice(H);
+  const int u0 = r * S;
+  const int slen = cl_slice_len(H, r);
+  const int MT = (slen + 127) / 128;                       // M tiles of the slice (0: empty slice)
+  const int MTmax = (cl_slice(p.Hmax) + 127) / 128;        // TMEM columns are planned for the widest layer
+  const int64_t sbase = p.layer_base[l] + static_cast<int64_t>(h) * layout::head_elems(H, depth);
+  const int64_t tbase = sbase + layout::net_elems(H, depth, 1);
+  const int64_t hd = static_cast<int64_t>(l) * p.Hkv + h;
+  const int R = p.G * static_cast<int>(p.nq);               // query rows of the head (<= N)
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL.bars);
+  const uint32_t b_full = smem_u32(bars);                   // [8]
+  const uint32_t b_empty = smem_u32(bars + 8);              // [8]
+  const uint32_t b_q = smem_u32(bars + 16);
+  const uint32_t b_acc = smem_u32(bars + 17);               // [2]: one per net
+  const uint32_t b_hr = smem_u32(bars + 19);                // [2]: h_k of every slice landed, k parity
+  const uint32_t b_ror = smem_u32(bars + 21);               // target h_{D-1} slice written: readout may run
+  const uint32_t b_rof = smem_u32(bars + 22);               // readout accumulated
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SL.tslot);
+  const uint32_t xq = smem_u32(smem + SL.xq);
+  const uint32_t xh = smem_u32(smem + SL.xh);
+  const uint32_t ring = smem_u32(smem + SL.ring);
+  const uint32_t xro = smem_u32(smem + SL.xro);
+  // X chunk c of net `net` as layer input: q (c < 2) or chunk c - 2 of h buffer `buf`
+  auto xchunk = [&](int net, int buf, int c) -> uint32_t {
+    return c < 2 ? xq + static_cast<uint32_t>(c * N * 128)
+                 : xh + static_cast<uint32_t>(((net * nb + buf) * HC + (c - 2)) * N * 128);
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S_; ++s) {
+      mbar_init(b_full + 8 * s, 1);
+      mbar_init(b_empty + 8 * s, 1);
+    }
+    mbar_init(b_q, 1);
+    mbar_init(b_acc, 1);
+    mbar_init(b_acc + 8, 1);
+    mbar_init(b_hr, 2);            // the two nets' epilogue leaders; the peers' slices as transactions
+    mbar_init(b_hr + 8, 2);
+    mbar_init(b_ror, 1);
+    mbar_init(b_rof, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tslot), static_cast<uint32_t>(p.tmem_cols));
+    tmem_relinquish();
+  }
+  if (warp >= 2) {
+    // h buffers start at 0 (their padding columns are read as 0 by the MMA);
+    // q rows past the R that TMA writes are 0
+    const int t = threadIdx.x - 64, nt = kThreads - 64;
+    uint4* xz = reinterpret_cast<uint4*>(smem + SL.xh);
+    const int n16 = static_cast<int>((SL.rt - SL.xh) / 16);    // h buffers and the readout input
+    for (int i = t; i < n16; i += nt) xz[i] = make_uint4(0, 0, 0, 0);
+    for (int i = t; i < 2 * N * 8; i += nt) {
+      const int c = i / (N * 8), rem = i % (N * 8), n = rem / 8;
+      if (n >= R) reinterpret_cast<uint4*>(smem + SL.xq + c * N * 128 + n * 128)[rem % 8] = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();              // every CTA's barriers are initialised before any DSMEM traffic
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  griddep_launch();                // the next kernel may take the SMs this call leaves idle
+
+  if (warp == 0 && lane == 0) {
+    // this CTA's weights towards L2 while an earlier kernel finishes
+    for (int k = 0; k < depth; ++k) {
+      const int K = layout::hidden_k(H, k), kc = layout::kchunks(K);
+      for (int net = 0; net < 2; ++net) {
+        const __nv_bfloat16* W = p.blob + (net ? tbase : sbase) + layout::hidden_w_off(H, depth, k);
+        for (int j = 0; j < MT; ++j) {
+          const int gu = u0 + 128 * j, m = gu >> 7, r0 = gu & 127;
+          const int rv = (slen - 128 * j < 128) ? (slen - 128 * j) : 128;
+          for (int c = 0; c < kc; ++c)
+            prefetch_l2(W + layout::tile_chunk_off(H, K, m, c) + r0 * 64, static_cast<uint32_t>(rv * 128));
+        }
+      }
+    }
+    if (MT > 0)
+      prefetch_l2(p.blob + tbase + layout::out_w_off(H, depth) + layout::tile_chunk_off(kD, H, 0, u0 / 64),
+                  static_cast<uint32_t>((slen + 63) / 64 * 128 * 128));
+  }
+  griddep_wait();                  // inputs and outputs are touched only from here on
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      prefetch_tmap(&tmap_q);
+      const uint64_t pol = policy_evict_first();
+      mbar_arrive_expect_tx(b_q, static_cast<uint32_t>(2 * R * 128));
+      tma_load_4d(xq, &tmap_q, 0, 0, 0, static_cast<int>(hd), b_q, pol);
+      tma_load_4d(xq + N * 128, &tmap_q, 64, 0, 0, static_cast<int>(hd), b_q, pol);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int k = 0; k < depth && ok; ++k) {
+        const int K = layout::hidden_k(H, k), kc = layout::kchunks(K);
+        for (int net = 0; net < 2 && ok; ++net) {
+          const __nv_bfloat16* W = p.blob + (net ? tbase : sbase) + layout::hidden_w_off(H, depth, k);
+          for (int j = 0; j < MT && ok; ++j) {
+            const int gu = u0 + 128 * j, m = gu >> 7, r0 = gu & 127;
+            const int rv = (slen - 128 * j < 128) ? (slen - 128 * j) : 128;
+            const int rvp = rv <= 64 ? 64 : 128;
+            const int cpg = static_cast<int>(kStage / (rvp * 128));
+            const bool whole = (r0 == 0 && rv == 128);              // whole 128-row tiles are contiguous
+            for (int c0 = 0; c0 < kc; c0 += cpg, ++it) {
+              const uint32_t s = it % S_;
+              if (it >= static_cast<uint32_t>(S_) && !mbar_wait(b_empty + 8 * s, ((it / S_) - 1) & 1, p.err)) {
+                ok = false;
+                break;
+              }
+              const int nc = (kc - c0 < cpg) ? (kc - c0) : cpg;
+              mbar_arrive_expect_tx(b_full + 8 * s, static_cast<uint32_t>(nc * rv * 128));
+              const uint32_t dst = ring + s * kStage;
+              if (whole) {
+                bulk_g2s(dst, W + layout::tile_chunk_off(H, K, m, c0), static_cast<uint32_t>(nc * 128 * 128),
+                         b_full + 8 * s, pol);
+              } else {
+                for (int cl = 0; cl < nc; ++cl)
+                  bulk_g2s(dst + cl * rvp * 128, W + layout::tile_chunk_off(H, K, m, c0 + cl) + r0 * 64,
+                           static_cast<uint32_t>(rv * 128), b_full + 8 * s, pol);
+              }
+            }
+          }
+        }
+      }
+      if (ok && MT > 0) {
+        // the target readout's K range: chunks of the slice of W_out [d][H]
+        const __nv_bfloat16* Wo = p.blob + tbase + layout::out_w_off(H, depth);
+        const int cb = u0 / 64, nch = (slen + 63) / 64;
+        for (int c0 = 0; c0 < nch; c0 += 2, ++it) {
+          const uint32_t s = it % S_;
+          if (it >= static_cast<uint32_t>(S_) && !mbar_wait(b_empty + 8 * s, ((it / S_) - 1) & 1, p.err)) break;
+          const int nc = (nch - c0 < 2) ? (nch - c0) : 2;
+          mbar_arrive_expect_tx(b_full + 8 * s, static_cast<uint32_t>(nc * 128 * 128));
+          bulk_g2s(ring + s * kStage, Wo + layout::tile_chunk_off(kD, H, 0, cb + c0),
+                   static_cast<uint32_t>(nc * 128 * 128), b_full + 8 * s, pol);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      bool ok = mbar_wait(b_q, 0, p.err);
+      uint32_t it = 0;
+      const uint32_t idesc = idesc_bf16_f32(128, N, 0, 0);
+      for (int k = 0; k < depth && ok; ++k) {
+        if (k > 0) {
+          // every CTA's slice of h_{k-1} (both nets) is in this CTA's X
+          ok = mbar_wait(b_hr + 8 * ((k - 1) & 1), ((k - 1) >> 1) & 1, p.err);
+          if (!ok) break;
+        }
+        tc_fence_after();
+        const int kc = layout::kchunks(layout::hidden_k(H, k));
+        const int buf = (k - 1 + nb) % nb;
+        for (int net = 0; net < 2 && ok; ++net) {
+          if (MT == 0) continue;
+          for (int j = 0; j < MT && ok; ++j) {
+            const int rv = (slen - 128 * j < 128) ? (slen - 128 * j) : 128;
+            const int rvp = rv <= 64 ? 64 : 128;
+            const int cpg = static_cast<int>(kStage / (rvp * 128));
+            const uint32_t dcol = tmem + static_cast<uint32_t>((net * MTmax + j) * N);
+            for (int c0 = 0; c0 < kc; c0 += cpg, ++it) {
+              const uint32_t s = it % S_;
+              if (!mbar_wait(b_full + 8 * s, (it / S_) & 1, p.err)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const int nc = (kc - c0 < cpg) ? (kc - c0) : cpg;
+              for (int cl = 0; cl < nc; ++cl) {
+                const uint32_t a = ring + s * kStage + cl * rvp * 128;
+                const uint32_t b = xchunk(net, buf, c0 + cl);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_bf16_ss(dcol, sdesc_sw128(a + kk * 32, 16, 1024), sdesc_sw128(b + kk * 32, 16, 1024), idesc,
+                              (c0 + cl + kk) != 0);
+              }
+              mma_commit(b_empty + 8 * s);
+            }
+          }
+          mma_commit(b_acc + 8 * net);
+        }
+      }
+      if (ok && MT > 0) {
+        // target readout: A_theta partial [d][rows] over this CTA's units
+        ok = mbar_wait(b_ror, 0, p.err);
+        tc_fence_after();
+        const int nch = (slen + 63) / 64;
+        const uint32_t dcol = tmem + static_cast<uint32_t>(2 * MTmax * N);
+        for (int c0 = 0; c0 < nch && ok; c0 += 2, ++it) {
+          const uint32_t s = it % S_;
+          if (!mbar_wait(b_full + 8 * s, (it / S_) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nc = (nch - c0 < 2) ? (nch - c0) : 2;
+          for (int cl = 0; cl < nc; ++cl) {
+            const uint32_t a = ring + s * kStage + cl * 128 * 128;
+            const uint32_t b = xro + static_cast<uint32_t>((c0 + cl) * N * 128);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss(dcol, sdesc_sw128(a + kk * 32, 16, 1024), sdesc_sw128(b + kk * 32, 16, 1024), idesc,
+                          (c0 + cl + kk) != 0);
+          }
+          mma_commit(b_empty + 8 * s);
+        }
+        mma_commit(b_rof);
+      }
+    }
+  } else if (warp < 2 + kEpiWarps) {
+    // ------------------------------ epilogues ------------------------------
+    const int net = (warp - 2) >> 2;                 // 0 score, 1 target
+    const int q4 = warp & 3;                         // TMEM lane quarter of this warp
+    const int et = ((warp - 2) & 3) * 32 + lane;     // 0..127 within the net's warps
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const int64_t nbase = net ? tbase : sbase;
+    float* sp = reinterpret_cast<float*>(smem + SL.sp);
+    bool ok = true;
+    for (int k = 0; k < depth; ++k) {
+      const bool last = (k == depth - 1);
+      const int buf = k % nb;
+      const bool reduce = last && net == 0;           // the score readout: w . h summed here
+      if (MT > 0) {
+        if (ok) ok = mbar_wait(b_acc + 8 * net, k & 1, p.err);
+        tc_fence_after();
+        const __nv_bfloat16* bias = p.blob + nbase + layout::hidden_b_off(H, depth, k);
+        const __nv_bfloat16* wsc = p.blob + sbase + layout::out_w_off(H, depth);
+        for (int n0 = 0; n0 < N; n0 += 16) {
+          float part[16];
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) part[jj] = 0.f;
+          for (int j = 0; j < MT; ++j) {
+            const int u = j * 128 + q4 * 32 + lane;
+            const bool valid = u < slen && ok;
+            const int gu = u0 + u;
+            const float bv = valid ? __bfloat162float(bias[gu]) : 0.f;
+            const float wv = (valid && reduce) ? __bfloat162float(wsc[gu]) : 0.f;
+            uint32_t v[16];
+            NECTAR_TMEM_LD16(trow + static_cast<uint32_t>((net * MTmax + j) * N + n0), v);
+            tmem_ld_wait();
+            if (valid) {
+#pragma unroll
+              for (int jj = 0; jj < 16; jj += 2) {
+                const uint32_t w = pack_bf16x2(cl_silu(__uint_as_float(v[jj]) + bv),
+                                               cl_silu(__uint_as_float(v[jj + 1]) + bv));
+                if (reduce) {
+                  part[jj] = fmaf(wv, bf16lo(w), part[jj]);
+                  part[jj + 1] = fmaf(wv, bf16hi(w), part[jj + 1]);
+                } else {
+                  // h_k into the h buffer (to be exchanged), or -- the target's
+                  // last layer -- into the readout input, columns from the slice start
+                  uint8_t* dst = last ? smem + SL.xro : smem + SL.xq + (xchunk(net, buf, 2) - xq);
+                  const int col = last ? u : gu;
+                  *reinterpret_cast<uint16_t*>(dst + cl_xoff(N, n0 + jj, col)) = static_cast<uint16_t>(w & 0xFFFFu);
+                  *reinterpret_cast<uint16_t*>(dst + cl_xoff(N, n0 + jj + 1, col)) = static_cast<uint16_t>(w >> 16);
+                }
+              }
+            }
+          }
+          if (reduce) {
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+#pragma unroll
+              for (int off = 16; off >= 1; off >>= 1) part[jj] += __shfl_xor_sync(0xffffffffu, part[jj], off);
+            }
+            if (lane == 0) {
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj) sp[q4 * N + n0 + jj] = part[jj];
+            }
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(1 + net, 128);
+      if (!last) {
+        if (et == 0) {
+          // own arrival, expecting the other CTAs' slices of this net as transactions
+          uint32_t peer = 0;
+          for (int o = 0; o < kCl; ++o) {
+            const int sl = cl_slice_len(H, o);
+            if (o != r && sl > 0) peer += static_cast<uint32_t>((sl + 63) / 64 * N * 128);
+          }
+          const uint32_t hr = b_hr + 8 * (k & 1);
+          mbar_arrive_expect_tx(hr, peer);
+          if (MT > 0) {
+            const uint32_t src = xchunk(net, buf, 2 + u0 / 64);
+            const uint32_t bytes = static_cast<uint32_t>((slen + 63) / 64 * N * 128);
+            for (int o = 0; o < kCl; ++o)
+              if (o != r) bulk_s2cluster(mapa_shared(src, o), src, bytes, mapa_shared(hr, o));
+          }
+        }
+      } else if (net == 0) {
+        // score partial of every row, to every CTA
+        if (et < R) {
+          const float v = MT > 0 ? (sp[et] + sp[N + et]) + (sp[2 * N + et] + sp[3 * N + et]) : 0.f;
+          const uint32_t dst = smem_u32(smem + SL.rs) + static_cast<uint32_t>((r * N + et) * 4);
+          for (int o = 0; o < kCl; ++o) st_cluster_f32(mapa_shared(dst, o), v);
+        }
+      } else {
+        // target readout partial [dim][row], to the owner of the dim
+        const int dim = q4 * 32 + lane;
+        const int o = dim / kOwnDims, dl = dim % kOwnDims;
+        const uint32_t dst = mapa_shared(smem_u32(smem + SL.rt) + static_cast<uint32_t>(((r * kOwnDims + dl) * N) * 4), o);
+        if (MT > 0) {
+          if (et == 0) mbar_arrive(b_ror);
+          if (ok) ok = mbar_wait(b_rof, 0, p.err);
+          tc_fence_after();
+          for (int n0 = 0; n0 < N; n0 += 16) {
+            uint32_t v[16];
+            NECTAR_TMEM_LD16(trow + static_cast<uint32_t>(2 * MTmax * N + n0), v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int jj = 0; jj < 16; jj += 4)
+              st_cluster_v4f(dst + (n0 + jj) * 4, __uint_as_float(v[jj]), __uint_as_float(v[jj + 1]),
+                             __uint_as_float(v[jj + 2]), __uint_as_float(v[jj + 3]));
+          }
+        } else {
+          for (int n0 = 0; n0 < N; n0 += 4) st_cluster_v4f(dst + n0 * 4, 0.f, 0.f, 0.f, 0.f);
+        }
+      }
+    }
+    tc_fence_before();
+  } else {
+    // ------------------------------ local attention ------------------------------
+    using St = RowState<RG, 16>;
+    constexpr int NG = St::NG;
+    constexpr int KPS = kLocWarps * NG * kLocKPG;    // keys per step of the 4 warps
+    const int lw = warp - 2 - kEpiWarps;
+    const int g = lane / 16, tl = lane % 16;
+    float* lscr = reinterpret_cast<float*>(smem + SL.lscr);
+    const int gblocks = (p.G + RG - 1) / RG;
+    const uint32_t rl0 = smem_u32(smem + SL.rl), rml0 = smem_u32(smem + SL.rml);
+    for (int t = 0; t < static_cast<int>(p.nq); ++t) {
+      int b = 0;
+      const int nv = visible_local(p.q_seq, p.q_pos, p.local_len, t, p.B, p.T, &b, p.err);
+      const int lo = static_cast<int>(static_cast<int64_t>(nv) * r / kCl);
+      const int hi = static_cast<int>(static_cast<int64_t>(nv) * (r + 1) / kCl);
+      const uint8_t* kb = reinterpret_cast<const uint8_t*>(p.Kloc) + ((hd * p.B + b) * p.T) * kRowBytes;
+      const uint8_t* vb = reinterpret_cast<const uint8_t*>(p.Vloc) + ((hd * p.B + b) * p.T) * kRowBytes;
+      for (int gb = 0; gb < gblocks; ++gb) {
+        const int g0 = gb * RG;
+        const int nr = (p.G - g0 < RG) ? (p.G - g0) : RG;
+        St st;
+        st.reset();
+        st.load_q(p.Q + ((hd * p.G + g0) * p.nq + t) * kD, p.nq * kD, nr, tl, p.qmul);
+        for (int j0 = lo + lw * NG * kLocKPG; j0 < hi; j0 += KPS) {
+          const uint8_t* kr[kLocKPG];
+          const uint8_t* vr[kLocKPG];
+          bool valid[kLocKPG];
+#pragma unroll
+          for (int k = 0; k < kLocKPG; ++k) {
+            const int key = j0 + k * NG + g;
+            valid[k] = key < hi;
+            kr[k] = kb + static_cast<int64_t>(key) * kRowBytes;
+            vr[k] = vb + static_cast<int64_t>(key) * kRowBytes;
+          }
+          st.template step<kLocKPG, GlobalLoader, true>(kr, vr, valid, tl, GlobalLoader{});
+        }
+        st.merge_groups();
+        if (g == 0) {
+          float* dst = lscr + (lw * RG) * (kD + 2);
+#pragma unroll
+          for (int rr = 0; rr < RG; ++rr) {
+#pragma unroll
+            for (int cc = 0; cc < St::CPL; ++cc)
+#pragma unroll
+              for (int e = 0; e < 8; ++e) dst[rr * (kD + 2) + St::dim_of(tl, cc, e)] = st.acc[rr][cc * 8 + e];
+            if (tl == 0) {
+              dst[rr * (kD + 2) + kD] = st.m[rr];
+              dst[rr * (kD + 2) + kD + 1] = st.l[rr];
+            }
+          }
+        }
+        named_bar_sync(3, kLocWarps * 32);
+        // join the 4 warps' states of each row; send each dim to its owner
+        for (int item = lw * 32 + lane; item < nr * kD; item += kLocWarps * 32) {
+          const int rr = item / kD, dim = item % kD;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kLocWarps; ++w) M = fmaxf(M, lscr[(w * RG + rr) * (kD + 2) + kD]);
+          float ls = 0.f, as = 0.f;
+#pragma unroll
+          for (int w = 0; w < kLocWarps; ++w) {
+            const float* src = lscr + (w * RG + rr) * (kD + 2);
+            const float wgt = exp2_shift(src[kD], M);
+            ls = fmaf(src[kD + 1], wgt, ls);
+            as = fmaf(src[dim], wgt, as);
+          }
+          const int n = (g0 + rr) * static_cast<int>(p.nq) + t;
+          const int o = dim / kOwnDims;
+          st_cluster_f32(mapa_shared(rl0 + static_cast<uint32_t>(((r * N + n) * kOwnDims + dim % kOwnDims) * 4), o),
+                         as);
+          if (dim < kCl) {
+            const uint32_t d2 = mapa_shared(rml0 + static_cast<uint32_t>((r * N + n) * 2 * 4), dim);
+            st_cluster_f32(d2, M);
+            st_cluster_f32(d2 + 4, ls);
+          }
+        }
+        named_bar_sync(3, kLocWarps * 32);
+      }
+    }
+  }
+
+  // ------------------------------ reduction and merge ------------------------------
+  __syncwarp();
+  cluster_sync_all();              // every partial is in its owner's shared memory
+  if (warp >= 2) {
+    const float* rs = reinterpret_cast<const float*>(smem + SL.rs);
+    const float* rt = reinterpret_cast<const float*>(smem + SL.rt);
+    const float* rl = reinterpret_cast<const float*>(smem + SL.rl);
+    const float* rml = reinterpret_cast<const float*>(smem + SL.rml);
+    const float cs = __bfloat162float(p.blob[sbase + layout::out_b_off(H, depth, 1)]);
+    const __nv_bfloat16* ct = p.blob + tbase + layout::out_b_off(H, depth, kD);
+    const int64_t rows = R;
+    for (int item = threadIdx.x - 64; item < R * kOwnDims; item += kThreads - 64) {
+      const int n = item / kOwnDims, dl = item % kOwnDims;
+      const int dim = r * kOwnDims + dl;
+      float a = 0.f, at = 0.f, Ml = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kCl; ++c) {
+        a += rs[c * N + n];
+        at += rt[(c * kOwnDims + dl) * N + n];
+        Ml = fmaxf(Ml, rml[(c * N + n) * 2]);
+      }
+      a += cs;
+      at += __bfloat162float(ct[dim]);
+      float ll = 0.f, al = 0.f;
+#pragma unroll
+      for (int c = 0; c < kCl; ++c) {
+        const float wgt = exp2_shift(rml[(c * N + n) * 2], Ml);
+        ll = fmaf(rml[(c * N + n) * 2 + 1], wgt, ll);
+        al = fmaf(rl[(c * N + n) * kOwnDims + dl], wgt, al);
+      }
+      const float ad = a * kLog2e;                     // document logit in log2 units
+      const float M = fmaxf(ad, Ml);
+      const float wd = exp2_shift(ad, M), wl = exp2_shift(Ml, M);
+      const float v = (wd * at + wl * al) / (wd + wl * ll);
+      const int64_t row = hd * rows + n;
+      if (p.out_bf16 != nullptr)
+        p.out_bf16[layer_layout_index(row, dim, p.Hkv, p.G, p.nq)] = __float2bfloat16_rn(v);
+      else
+        p.out[row * kD + dim] = v;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, static_cast<uint32_t>(p.tmem_cols));
+  }
+}
+
+template <int RG>
+cudaError_t launch_cl(const CUtensorMap& tq, const ClusterParams& p, int heads, size_t smem, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(decode_cluster_kernel<RG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_k(decode_cluster_kernel<RG>, dim3(static_cast<unsigned>(heads * kCl)), dim3(kThreads), smem, stream,
+                  kCl, tq, p);
+}
+
+}  // namespace
+
+int cluster_rg(int G) { return G <= 2 ? 2 : 4; }
+
+ClusterShape cluster_shape(int G, int64_t nq, int Hmax, int depth) {
+  ClusterShape sh{};
+  const int64_t R = static_cast<int64_t>(G) * nq;
+  if (R < 1 || R > 64 || nq > 256 || depth < 1 || depth > 4) return sh;
+  sh.N = static_cast<int>((R + 15) / 16 * 16);
+  sh.nb = depth >= 3 ? 2 : 1;
+  const int rg = cluster_rg(G);
+  constexpr size_t kMax = 227 * 1024;
+  for (int st = 6; st >= 2; --st) {
+    const size_t smem = cl_layout(Hmax, sh.N, sh.nb, st, rg).total + 1024;
+    if (smem <= kMax) {
+      sh.stages = st;
+      sh.smem = smem;
+      break;
+    }
+  }
+  if (sh.stages == 0) return sh;
+  const int MTmax = (cl_slice(Hmax) + 127) / 128;
+  const int cols = (2 * MTmax + 1) * sh.N;
+  int c = 32;
+  while (c < cols) c <<= 1;
+  sh.tmem_cols = c;
+  sh.ok = c <= 512;
+  return sh;
+}
+
+cudaError_t launch_decode_cluster(const CUtensorMap& tq, const ClusterParams& p, int heads, size_t smem,
+                                  cudaStream_t stream) {
+  return cluster_rg(p.G) == 2 ? launch_cl<2>(tq, p, heads, smem, stream) : launch_cl<4>(tq, p, heads, smem, stream);
+}
+
+}  // namespace nectar

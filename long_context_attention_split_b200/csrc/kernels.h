@@ -5,6 +5,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 namespace nectar {
 
@@ -13,6 +14,45 @@ void set_last_error(const char* msg);
 // Id of the CUDA context current on the calling thread (0: none, or the
 // driver cannot tell).
 unsigned long long current_context_id();
+
+// Launch with programmatic dependent launch allowed (the kernel calls
+// griddep_wait before it touches global memory; see ptx.cuh) and, with
+// cluster > 1, as clusters of `cluster` CTAs along x.  NECTAR_PDL=0 (read
+// once per process) launches without the attribute.
+inline bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("NECTAR_PDL");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  return on;
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, int cluster,
+                     Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[2];
+  unsigned na = 0;
+  if (pdl_enabled()) {
+    at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (cluster > 1) {
+    at[na].id = cudaLaunchAttributeClusterDimension;
+    at[na].val.clusterDim.x = static_cast<unsigned>(cluster);
+    at[na].val.clusterDim.y = 1;
+    at[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = na;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
 
 // ----- (i) split-n decode attention (CUDA cores) + LSE combine -------------
 struct DecParams {
@@ -134,6 +174,44 @@ struct ModParams {
   int64_t layer_base[kModMaxLayers];   // blob element offset of layer l
   uint8_t order[kModMaxLayers];        // layers by decreasing width
 };
+// One-launch decode with one thread-block cluster per (l, h) (decode_cluster.cu):
+// the hidden units of every layer are sliced over the cluster's CTAs, for
+// calls with few heads (a model's decode run layer after layer).
+constexpr int kClusterCtas = 8;
+struct ClusterParams {
+  int Hkv, G, depth;
+  int64_t nq;
+  int N;                // activation rows: G * nq rounded up to 16 (<= 64)
+  int Hmax, stages, tmem_cols;
+  int nb;               // hidden-state buffers per net: 2 when depth >= 3
+  const __nv_bfloat16* blob;
+  const __nv_bfloat16* Q;
+  const int32_t* q_seq;
+  const int32_t* q_pos;
+  const __nv_bfloat16* Kloc;
+  const __nv_bfloat16* Vloc;
+  const int32_t* local_len;
+  int B, T;
+  float qmul;           // scale * log2(e)
+  float* out;           // fp32 [L][Hkv][G][nq][d], or
+  __nv_bfloat16* out_bf16;   // bf16 layer layout [L][nq][Hkv][G][d]
+  int* err;
+  int32_t width[kModMaxLayers];
+  int64_t layer_base[kModMaxLayers];
+  uint8_t order[kModMaxLayers];
+};
+struct ClusterShape {
+  bool ok;
+  int N, nb, stages, tmem_cols;
+  size_t smem;
+};
+// Plan of the cluster decode for G query heads x nq tokens per KV head;
+// ok = false when it does not apply (more than 64 rows, depth > 4, or the
+// shared memory or TMEM plan does not fit).
+ClusterShape cluster_shape(int G, int64_t nq, int Hmax, int depth);
+cudaError_t launch_decode_cluster(const CUtensorMap& tq, const ClusterParams& p, int heads, size_t smem,
+                                  cudaStream_t stream);
+
 // Layer-by-layer grouped GEMM path of the module forward (module_gemm.cu),
 // used when a KV head has at least kGemmMinRows query rows.
 constexpr int kGemmMaxStages = 8;

@@ -162,6 +162,7 @@ __device__ __forceinline__ void module_cta(const CUtensorMap* tmap_q, const ModP
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  griddep_wait();                 // inputs and outputs only from here on (launched after another kernel)
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
@@ -424,6 +425,7 @@ __device__ __forceinline__ void local_state_cta(const ModParams& p, int64_t luni
     fence_barrier_init();
   }
   __syncthreads();
+  griddep_wait();
   if (warp == kDecLocCW) {
     if (lane == 0) local_produce<RG>(J, hd, i, 1, smem_u32(ring), kDecLocStages, full0, empty0);
   } else if (warp < kDecLocCW) {
@@ -459,12 +461,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_q, const ModParams p) {
     if (b < p.n_local) local_state_cta<RG>(p, b, smem);
     else module_cta<kNetSplit>(&tmap_q, p, static_cast<int>(b - p.n_local), smem);
   }
+  griddep_launch();               // the merge may start launching
 }
 
 // Merge of every row's document term (a_theta from the workspace, A_theta
 // in A_out) with its local state, Eqs. (3.4)-(3.5), into out (in place when
 // A_out is out) or, bf16, into out_bf16 in the layer layout.
 __global__ void decode_merge_kernel(const ModParams p, int64_t nrows) {
+  griddep_wait();
+  griddep_launch();
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= nrows * kD) return;
   const int64_t row = idx / kD;
@@ -539,8 +544,8 @@ static cudaError_t launch_decode_s(const CUtensorMap& tq, const ModParams& q, si
   cudaError_t e = cudaFuncSetAttribute(decode_kernel<RG, kNetSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  decode_kernel<RG, kNetSplit><<<static_cast<unsigned>(q.n_local + q.n_module), kModThreads, smem, stream>>>(tq, q);
-  return cudaGetLastError();
+  return launch_k(decode_kernel<RG, kNetSplit>, dim3(static_cast<unsigned>(q.n_local + q.n_module)), dim3(kModThreads),
+                  smem, stream, 1, tq, q);
 }
 
 template <int RG>
@@ -553,8 +558,8 @@ static cudaError_t launch_decode_t(const CUtensorMap& tq, const ModParams& p, in
   if (e != cudaSuccess) return e;
   const int64_t nrows = static_cast<int64_t>(p.n_local / p.nq) * p.G * p.nq;
   const int64_t threads = nrows * kD;
-  decode_merge_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p, nrows);
-  return cudaGetLastError();
+  return launch_k(decode_merge_kernel, dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256), 0, stream, 1, p,
+                  nrows);
 }
 
 template <int RG>

@@ -1078,6 +1078,25 @@ size_t nectar_decode_layer_out_workspace_size(nectar_dims dims, const nectar_mod
 
 namespace {
 
+// Calls with at most this many (layer, KV head) pairs take the cluster
+// decode (decode_cluster.cu) when it applies; more heads keep the one-launch
+// kernel with one CTA per (l, h) (or per net), which then fills the GPU.
+#ifndef NECTAR_CLUSTER_MAX_HEADS
+#define NECTAR_CLUSTER_MAX_HEADS 32
+#endif
+
+// NECTAR_DECODE_CLUSTER=0 never takes the cluster decode, =1 takes it
+// whenever it applies; unset: by the head count above.
+bool use_cluster_decode(const nectar_dims& dims, int64_t nq, const Arch& ar, int Hmax) {
+  if (ar.general || static_cast<int64_t>(dims.G) * nq > 64) return false;
+  const char* env = getenv("NECTAR_DECODE_CLUSTER");
+  const int mode = (env != nullptr && env[0] != 0) ? atoi(env) : -1;
+  if (mode == 0) return false;
+  if (!cluster_shape(dims.G, nq, Hmax, ar.Ds).ok) return false;
+  if (mode == 1) return true;
+  return static_cast<int64_t>(dims.L) * dims.Hkv <= NECTAR_CLUSTER_MAX_HEADS;
+}
+
 // The decode, into out (fp32, per KV head) or out_bf16 (bf16, layer layout).
 nectar_status decode_impl(nectar_dims dims, const nectar_module_set* mods, const nectar_bf16* Q, int64_t nq,
                           const int32_t* q_seq, const int32_t* q_pos, const nectar_bf16* Kloc,
@@ -1134,6 +1153,47 @@ nectar_status decode_impl(nectar_dims dims, const nectar_module_set* mods, const
     }
     return run_module_gemm(dims, p, Q, nq, nullptr, out, p.ws_loc,
                            base + align256(static_cast<size_t>(rows) * (kD + 2) * sizeof(float)), st, out_bf16);
+  }
+  if (use_cluster_decode(dims, nq, ar, p.Hmax)) {
+    const ClusterShape cs = cluster_shape(dims.G, nq, p.Hmax, ar.Ds);
+    ClusterParams c;
+    memset(&c, 0, sizeof(c));
+    c.Hkv = dims.Hkv;
+    c.G = dims.G;
+    c.depth = ar.Ds;
+    c.nq = nq;
+    c.N = cs.N;
+    c.Hmax = p.Hmax;
+    c.stages = cs.stages;
+    c.tmem_cols = cs.tmem_cols;
+    c.nb = cs.nb;
+    c.blob = p.blob;
+    c.Q = p.Q;
+    c.q_seq = q_seq;
+    c.q_pos = q_pos;
+    c.Kloc = p.Kloc;
+    c.Vloc = p.Vloc;
+    c.local_len = local_len;
+    c.B = B;
+    c.T = T_max;
+    c.qmul = p.qmul;
+    c.out = out;
+    c.out_bf16 = out_bf16;
+    c.err = p.err;
+    for (int l = 0; l < dims.L; ++l) {
+      c.width[l] = p.width[l];
+      c.layer_base[l] = p.layer_base[l];
+      c.order[l] = p.order[l];
+    }
+    // queries: [heads][G][nq][128]; box = 64 columns x all nq tokens x G heads x 1
+    CUtensorMap tqc;
+    const cuuint64_t dimsq[4] = {128, static_cast<cuuint64_t>(nq), static_cast<cuuint64_t>(dims.G),
+                                 static_cast<cuuint64_t>(heads)};
+    const cuuint64_t strq[3] = {256, static_cast<cuuint64_t>(nq) * 256, static_cast<cuuint64_t>(nq) * 256 * dims.G};
+    const cuuint32_t boxq[4] = {64, static_cast<cuuint32_t>(nq), static_cast<cuuint32_t>(dims.G), 1};
+    NECTAR_TRY(make_tmap(&tqc, Q, 4, dimsq, strq, boxq, "queries (cluster decode)"));
+    cudaError_t e = launch_decode_cluster(tqc, c, static_cast<int>(heads), cs.smem, st);
+    return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "cluster decode kernel");
   }
   p.a_out = reinterpret_cast<float*>(base);
   p.ws_loc = reinterpret_cast<float*>(base + decode_ws_a_bytes(rows));

@@ -114,6 +114,20 @@ __device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uin
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch.  A kernel launched with the
+// programmatic-stream-serialization attribute may start (its prologue: shared
+// memory, barriers, TMEM) while the kernel before it on the stream is still
+// finishing.  griddep_wait blocks until that kernel has completed and its
+// memory writes are visible: every thread calls it before it reads or
+// writes global memory (an L2 prefetch is only a hint and may come before).
+// griddep_launch lets the next such kernel start launching once every CTA
+// of this one has called it or exited.  Both do nothing in a kernel
+// launched without the attribute.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // bulk copies (TMA engine).  Every copy lands in the issuing CTA's own
 // shared memory: none is shared across a cluster.
 // ---------------------------------------------------------------------------
@@ -140,6 +154,11 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(bar), "l"(policy)
       : "memory");
+}
+// Bring [src, src + bytes) into L2 (a hint: nothing is written anywhere);
+// src 16-B aligned, bytes % 16 == 0.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 // Tiled tensor loads.  c0 is the innermost coordinate; callers keep
 // c0 * element size a multiple of 16 bytes.
@@ -222,6 +241,22 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
       return false;
     }
   }
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_v4f(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+// Copy `bytes` of this CTA's shared memory into another CTA of the cluster
+// (dst and its mbarrier `bar` are shared::cluster addresses from mapa); the
+// copy completes `bytes` of transactions on that mbarrier.  A plain
+// point-to-point DSMEM copy, not a multicast.  16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_s2cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "r"(src), "r"(bytes), "r"(bar)
+               : "memory");
 }
 // all threads of all CTAs of the cluster
 __device__ __forceinline__ void cluster_sync_all() {

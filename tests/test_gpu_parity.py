@@ -439,6 +439,47 @@ def test_decode_shapes(kw):
     decode_case(wl)
 
 
+# The cluster decode (one 8-CTA cluster per (l, h), hidden units sliced over
+# the cluster, merge in-cluster) on the shapes it takes: at most 64 rows per
+# KV head.  Widths cover 64-unit slices (512), partial and empty slices (208:
+# 4 of 8 CTAs hold units, the last 16), 128-unit slices (1024) next to a
+# layer held by one CTA (64), depths 1 and 3 (no exchange; two h buffers),
+# G = 12 (three head blocks of the local warps), 64 rows (N = 64).
+@pytest.mark.parametrize("kw", [
+    dict(L=2, Hkv=2, G=2, n=16, B=3, T=40, widths=[512, 512]),
+    dict(L=1, Hkv=2, G=7, n=16, B=2, T=33, widths=[208]),
+    dict(L=2, Hkv=1, G=4, n=16, B=5, T=17, widths=[1024, 64]),
+    dict(L=2, Hkv=2, G=2, n=16, B=3, T=70, widths=[256, 128], depth=1),
+    dict(L=2, Hkv=2, G=2, n=16, B=3, T=70, widths=[256, 384], depth=3),
+    dict(L=1, Hkv=1, G=12, n=16, B=4, T=45, widths=[128]),
+    dict(L=1, Hkv=2, G=16, n=16, B=4, T=300, widths=[256]),
+    dict(L=2, Hkv=2, G=2, n=16, B=1, T=512, widths=[512, 512]),     # the headline's shape per layer
+])
+def test_decode_cluster_shapes(kw, monkeypatch):
+    monkeypatch.setenv("NECTAR_DECODE_CLUSTER", "1")
+    wl = make_workload("qwen3_1p7b", seed=7, key_scale=None, **kw)
+    wl.local_len = torch.randint(0, wl.T + 1, (wl.B,), generator=torch.Generator().manual_seed(5)).to(torch.int32)
+    wl.q_pos = (wl.local_len[wl.q_seq.long()] - 1).clamp(min=0).to(torch.int32)
+    decode_case(wl)
+
+
+def test_decode_cluster_matches_one_launch(monkeypatch):
+    # the same decode through the cluster kernel and the one-CTA-per-head
+    # kernel: same arithmetic up to the order of the sums
+    wl = make_workload("qwen3_1p7b", seed=8, key_scale=None, L=3, Hkv=2, G=2, n=16, B=2, T=100, widths=[512] * 3)
+    mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G)
+    args = (cuda(wl.Q), cuda(wl.q_seq), cuda(wl.q_pos), cuda(wl.Kloc), cuda(wl.Vloc), cuda(wl.local_len))
+    monkeypatch.setenv("NECTAR_DECODE_CLUSTER", "1")
+    o1 = nx.decode(mods, *args)
+    l1 = nx.decode_layer_out(mods, *args)
+    monkeypatch.setenv("NECTAR_DECODE_CLUSTER", "0")
+    o0 = nx.decode(mods, *args)
+    torch.cuda.synchronize()
+    assert nx.device_error_flags(clear=True) == 0
+    assert torch.allclose(o1, o0, rtol=0, atol=1e-4 * max(1.0, o0.abs().max().item()))
+    assert torch.equal(l1, o1.permute(0, 3, 1, 2, 4).reshape(wl.L, wl.nq, wl.Hkv * wl.G, 128).to(torch.bfloat16))
+
+
 def test_decode_workspace_checked():
     wl = make_workload("toy", seed=4)
     mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G)
