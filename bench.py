@@ -525,6 +525,8 @@ def workload_overrides(args) -> dict:
         over["B"] = args.batch
     if args.rho:
         over["rho"] = args.rho
+    if args.width:
+        over["H"] = args.width
     return over
 
 
@@ -865,6 +867,8 @@ def main():
                     help="also time the Quadrature module, the fit metrics and a decode with a shared backbone")
     ap.add_argument("--batch", type=int, default=0, help="decode batch B (llama8b_sweep: 1, 16, 256)")
     ap.add_argument("--rho", type=float, default=0.0, help="module capacity (llama8b_sweep: 0.01, 0.05, 0.10)")
+    ap.add_argument("--width", type=int, default=0,
+                    help="module hidden width H for every layer (qwen25_7b_decode at rho = 10 %%: 1152)")
     ap.add_argument("--layers", type=int, default=0,
                     help="run only the first LAYERS layers (small cases for profiling; not a bench line)")
     args = ap.parse_args()

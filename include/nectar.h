@@ -71,7 +71,7 @@ typedef struct {
 
 #define NECTAR_MAX_DEPTH 4
 #define NECTAR_MAX_LAYERS 256
-#define NECTAR_MAX_WIDTH 1024
+#define NECTAR_MAX_WIDTH 2048
 
 /* ------------------------------------------------------------------------
  * (i) Exact cached-token attention, Eq. (3.1), §2.1:
@@ -171,14 +171,14 @@ NECTAR_API nectar_status nectar_cache_attn_lse_static(nectar_dims dims, const ne
 typedef struct {
   int32_t depth_b;          /* backbone layers, 0..NECTAR_MAX_DEPTH - 1 */
   int32_t depth_s, depth_t; /* branch layers, >= 1; depth_b + max(depth_s, depth_t) <= NECTAR_MAX_DEPTH */
-  const int32_t *width_b;   /* HOST [L], multiples of 16 in [16, 1024]; may be NULL when depth_b = 0 */
+  const int32_t *width_b;   /* HOST [L], multiples of 16 in [16, 2048]; may be NULL when depth_b = 0 */
   const int32_t *width_s;   /* HOST [L] */
   const int32_t *width_t;   /* HOST [L] */
 } nectar_module_arch;
 
 typedef struct {
   int32_t depth;          /* hidden layers per net, 1..NECTAR_MAX_DEPTH (classic sets) */
-  const int32_t *width;   /* HOST [L]: H_l, a multiple of 16 in [16, 1024] (classic sets) */
+  const int32_t *width;   /* HOST [L]: H_l, a multiple of 16 in [16, 2048] (classic sets) */
   const nectar_bf16 *weights;   /* DEVICE packed blob */
   int64_t weights_elems;  /* bf16 elements in the blob */
   const nectar_module_arch *arch;   /* HOST; NULL: the classic set (depth, width); else the
@@ -227,15 +227,19 @@ NECTAR_API nectar_status nectar_module_pack(nectar_dims dims, int32_t depth, con
  *   A_theta[row] = A_theta(q)     DEVICE fp32 [L][Hkv][G][nq][d]
  * Runs on the tensor cores (tcgen05, bf16 operands, fp32 accumulation);
  * hidden activations are rounded to bf16 between layers.  Fewer than 64
- * query rows per KV head (classic sets): one launch, each CTA carrying
- * <= 64 rows through all layers in shared memory (workspace unused, may be
- * NULL).  More rows, or a set with a backbone or unequal branches:
+ * query rows per KV head (classic sets) and ceil(Hmax / 128) *
+ * round16(G) <= 512 (Hmax the widest layer: the one-launch kernel keeps a
+ * layer's 128-unit tiles side by side in 512 TMEM columns): one launch,
+ * each CTA carrying <= 64 rows through all layers in shared memory
+ * (workspace unused, may be NULL).  Otherwise, or for a set with a backbone
+ * or unequal branches:
  * one grouped-GEMM launch per hidden layer plus one for the readouts, the
  * hidden activations kept in `workspace` (DEVICE, 256-byte aligned, owned
  * by the caller, overwritten; NECTAR_ERR_WORKSPACE when missing or small).
  * ------------------------------------------------------------------------ */
 /* Workspace of nectar_module_forward, in bytes: 0 when the one-launch path
- * runs (classic sets, fewer than 64 query rows G * nq per KV head), else
+ * runs (classic sets, fewer than 64 query rows G * nq per KV head, and the
+ * TMEM condition above), else
  * the hidden activations of the layer-by-layer path,
  * (S >= 2 ? 2 : 1) * align256(2 * rows * Hp * 2) + align256(rows * ceil(Hsmax / 128) * 4),
  * with rows = L * Hkv * G * nq, S the hidden layers of the longest chain

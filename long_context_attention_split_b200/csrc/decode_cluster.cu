@@ -8,19 +8,21 @@
 // weight stream: every weight is used once per row.  One CTA per (l, h)
 // streams the head's whole module through one SM, which is slow when a call
 // has few heads (one layer of a model run layer after layer: 8 heads on 148
-// SMs).  Here the hidden units of every layer of both nets are cut into
-// kClusterCtas slices of a multiple of 64 units, one per CTA of the
-// cluster, so the head's weights stream through kClusterCtas SMs at once.
+// SMs).  Here the hidden units of every layer of each net are cut into 8
+// slices of a multiple of 64 units, and the cluster's CTAs share them: with
+// 8 CTAs each holds one slice of both nets; with 16 (a non-portable cluster
+// size) CTAs 0-7 hold the score net's slices and 8-15 the target net's, so
+// that a CTA's weights fit its shared-memory ring whole.
 //
-// Per CTA (rank r, units [u0, u0 + slen) of each net):
+// Per CTA (slice si = rank mod 8, units [u0, u0 + slen) of each net it holds):
 //  - hidden layer k: the rows of W_k for its units (A, swap-AB: M = 128
 //    units -- a 64-unit slice uses the lanes 0-63 of an M = 128 tile whose
 //    other rows it ignores --, N = the head's query rows, K = d or d + H),
 //    streamed from the packed blob by bulk copies through a ring, times
 //    X = [q | h_{k-1}] (B, resident, K-major, 128-byte swizzle) into TMEM;
 //    the epilogue adds the bias, applies SiLU, writes its slice of h_k into
-//    its own X as bf16 and copies that slice into the X of every other CTA
-//    of the cluster (DSMEM bulk copies that complete on the receiver's
+//    its own X as bf16 and copies that slice into the X of the other CTAs
+//    holding the same net (DSMEM bulk copies that complete on the receiver's
 //    mbarrier: point to point, no multicast).  The next layer starts once
 //    every slice has landed.  Depth >= 3 alternates two h buffers, so that
 //    a buffer is written again only two layers after it was sent, when every
@@ -30,19 +32,20 @@
 //    CTA's units in the epilogue registers; the target net's readout
 //    W_out[:, slice] h_slice is one more MMA (M = d, K = the slice).
 //  - local attention: 4 warps score the CTA's share of every query token's
-//    visible local keys (the keys cut into kClusterCtas ranges) on the CUDA
+//    visible local keys (the keys cut into one range per CTA) on the CUDA
 //    cores, leaving a partial (m, l, acc) per row.
-//  - reduction and merge: CTA o owns output dims [16 o, 16 o + 16).  Every
+//  - reduction and merge: each CTA owns d / cluster output dims.  Every
 //    CTA stores its partials into the owners' shared memory (score partial
 //    of each row to all, target and local partials of each dim to that
 //    dim's owner), one cluster barrier, and each owner sums the partials in
 //    a fixed order (deterministic), joins the local partials by
 //    log-sum-exp and merges: out = (2^{a'} A_theta + 2^{m} acc) /
 //    (2^{a'} + 2^{m} l) with a' = a_theta log2 e (Eqs. (3.4)-(3.5)).
-// Warp roles: 0 TMA producer, 1 MMA issuer (+ TMEM owner), 2-5 score-net
-// epilogue, 6-9 target-net epilogue, 10-13 local attention; all take part in
-// the merge's reduction.  Every mbarrier wait is bounded; every thread
-// reaches both cluster barriers (no early return).
+// Warp roles: 0 TMA producer, 1 MMA issuer (+ TMEM owner), 2-5 and 6-9 the
+// epilogues of the CTA's first and second net (with one net per CTA, 6-9
+// only join the barriers), 10-13 local attention; all take part in the
+// merge.  Every mbarrier wait is bounded; every thread reaches both cluster
+// barriers (no early return).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -55,14 +58,14 @@ namespace nectar {
 
 namespace {
 
-constexpr int kCl = kClusterCtas;
-constexpr int kOwnDims = kD / kCl;               // output dims merged by each CTA
+constexpr int kSlices = 8;                       // slices of every net's hidden units
 constexpr uint32_t kStage = 32 * 1024;           // weight ring stage
 constexpr uint32_t kPad = 8 * 1024;              // read (not used) past the ring by a 64-row tile
 constexpr int kEpiWarps = 8;
 constexpr int kLocWarps = 4;
 constexpr int kThreads = (2 + kEpiWarps + kLocWarps) * 32;
 constexpr int kLocKPG = 2;                        // keys per lane group per step
+constexpr int kMaxStages = 8;
 
 struct ClSmem {
   uint32_t ring, xq, xh, xro, rt, rl, rs, rml, sp, lscr, bars, tslot, total;
@@ -71,35 +74,39 @@ struct ClSmem {
 // 64-unit granules: the h slices exchanged between CTAs are whole 64-column
 // chunks of X
 __host__ __device__ inline int cl_slice(int H) {
-  const int s = (H + kCl - 1) / kCl;
+  const int s = (H + kSlices - 1) / kSlices;
   return (s + 63) / 64 * 64;
 }
-__host__ __device__ inline int cl_slice_len(int H, int r) {
+__host__ __device__ inline int cl_slice_len(int H, int si) {
   const int S = cl_slice(H);
-  const int len = H - r * S;
+  const int len = H - si * S;
   return len < 0 ? 0 : (len < S ? len : S);
 }
+// rows of the partials exchanged in the reduction: R rounded up to 4
+__host__ __device__ inline int cl_rp(int R) { return (R + 3) / 4 * 4; }
 
-// byte offsets from the 1024-aligned dynamic shared memory base
-__host__ __device__ inline ClSmem cl_layout(int Hmax, int N, int nb, int stages, int rg) {
+// byte offsets from the 1024-aligned dynamic shared memory base, for a
+// cluster of kC CTAs each holding npc nets
+__host__ __device__ inline ClSmem cl_layout(int kC, int npc, int Hmax, int N, int R, int nb, int stages, int rg) {
   ClSmem s{};
+  const int own = kD / kC, Rp = cl_rp(R);
   uint32_t off = 0;
   s.ring = off;
   off += static_cast<uint32_t>(stages) * kStage + kPad;
   s.xq = off;                                                   // q: 2 chunks of [N][128 B]
   off += 2u * N * 128;
   s.xh = off;                                                   // h: [net][buf][chunk][N][128 B]
-  off += 2u * nb * layout::kchunks(Hmax) * N * 128;
+  off += static_cast<uint32_t>(npc * nb * layout::kchunks(Hmax) * N * 128);
   s.xro = off;                                                  // the target readout's input: own slice
   off += static_cast<uint32_t>(layout::kchunks(cl_slice(Hmax))) * N * 128;
-  s.rt = off;                                                   // target partials [src][dim][row]
-  off += static_cast<uint32_t>(kCl * kOwnDims * N) * 4;
-  s.rl = off;                                                   // local acc partials [src][row][dim]
-  off += static_cast<uint32_t>(kCl * N * kOwnDims) * 4;
-  s.rs = off;                                                   // score partials [src][row]
-  off += static_cast<uint32_t>(kCl * N) * 4;
-  s.rml = off;                                                  // local (m, l) [src][row][2]
-  off += static_cast<uint32_t>(kCl * N * 2) * 4;
+  s.rt = off;                                                   // target partials [slice][dim][row]
+  off += static_cast<uint32_t>(kSlices * own * Rp) * 4;
+  s.rl = off;                                                   // local acc partials [cta][row][dim]
+  off += static_cast<uint32_t>(kC * Rp * own) * 4;
+  s.rs = off;                                                   // score partials [slice][row]
+  off += static_cast<uint32_t>(kSlices * Rp) * 4;
+  s.rml = off;                                                  // local (m, l) [cta][row][2]
+  off += static_cast<uint32_t>(kC * Rp * 2) * 4;
   s.sp = off;                                                   // score sums by lane quarter [4][N]
   off += static_cast<uint32_t>(4 * N) * 4;
   s.lscr = off;                                                 // local warps' states [warp][rg][d + 2]
@@ -125,14 +132,21 @@ __device__ __forceinline__ uint32_t cl_xoff(int N, int n, int c) {
                                ((c & 7) << 1));
 }
 
-template <int RG>
+template <int RG, int kC>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterParams p) {
+  constexpr int kNPC = kC == 2 * kSlices ? 1 : 2;   // nets per CTA
+  constexpr int kOwn = kD / kC;                      // output dims merged by each CTA
+  static_assert(kC == kSlices || kC == 2 * kSlices, "8 or 16 CTAs per cluster");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = cl_aligned(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = static_cast<int>(cluster_ctarank());
-  const int ci = static_cast<int>(blockIdx.x) / kCl;
+  const int si = r % kSlices;                       // slice of the units
+  const int n0 = kNPC == 1 ? r / kSlices : 0;       // the CTA's first net (0 score, 1 target)
+  const int pbase = kNPC == 1 ? n0 * kSlices : 0;   // rank of slice 0 of the CTA's nets
+  const bool has_target = n0 + kNPC - 1 == 1;
+  const int ci = static_cast<int>(blockIdx.x) / kC;
   const int li = ci / p.Hkv, h = ci % p.Hkv;
   const int l = p.order[li];
   const int H = p.width[l];
@@ -141,34 +155,35 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
   const int nb = p.nb;
   const int HC = layout::kchunks(p.Hmax);
   const int S_ = p.stages;
-  const ClSmem SL = cl_layout(p.Hmax, N, nb, S_, RG);
+  const int R = p.G * static_cast<int>(p.nq);               // query rows of the head (<= N)
+  const int Rp = cl_rp(R);
+  const ClSmem SL = cl_layout(kC, kNPC, p.Hmax, N, R, nb, S_, RG);
   const int S = cl_slice(H);
-  const int u0 = r * S;
-  const int slen = cl_slice_len(H, r);
+  const int u0 = si * S;
+  const int slen = cl_slice_len(H, si);
   const int MT = (slen + 127) / 128;                       // M tiles of the slice (0: empty slice)
   const int MTmax = (cl_slice(p.Hmax) + 127) / 128;        // TMEM columns are planned for the widest layer
   const int64_t sbase = p.layer_base[l] + static_cast<int64_t>(h) * layout::head_elems(H, depth);
   const int64_t tbase = sbase + layout::net_elems(H, depth, 1);
   const int64_t hd = static_cast<int64_t>(l) * p.Hkv + h;
-  const int R = p.G * static_cast<int>(p.nq);               // query rows of the head (<= N)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL.bars);
-  const uint32_t b_full = smem_u32(bars);                   // [8]
-  const uint32_t b_empty = smem_u32(bars + 8);              // [8]
-  const uint32_t b_q = smem_u32(bars + 16);
-  const uint32_t b_acc = smem_u32(bars + 17);               // [2]: one per net
-  const uint32_t b_hr = smem_u32(bars + 19);                // [2]: h_k of every slice landed, k parity
-  const uint32_t b_ror = smem_u32(bars + 21);               // target h_{D-1} slice written: readout may run
-  const uint32_t b_rof = smem_u32(bars + 22);               // readout accumulated
+  const uint32_t b_full = smem_u32(bars);                   // [kMaxStages]
+  const uint32_t b_empty = smem_u32(bars + kMaxStages);     // [kMaxStages]
+  const uint32_t b_q = smem_u32(bars + 2 * kMaxStages);
+  const uint32_t b_acc = smem_u32(bars + 2 * kMaxStages + 1);   // [2]: one per local net
+  const uint32_t b_hr = smem_u32(bars + 2 * kMaxStages + 3);    // [2]: h_k of every slice landed, k parity
+  const uint32_t b_ror = smem_u32(bars + 2 * kMaxStages + 5);   // target h_{D-1} slice written
+  const uint32_t b_rof = smem_u32(bars + 2 * kMaxStages + 6);   // readout accumulated
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SL.tslot);
   const uint32_t xq = smem_u32(smem + SL.xq);
   const uint32_t xh = smem_u32(smem + SL.xh);
   const uint32_t ring = smem_u32(smem + SL.ring);
   const uint32_t xro = smem_u32(smem + SL.xro);
-  // X chunk c of net `net` as layer input: q (c < 2) or chunk c - 2 of h buffer `buf`
-  auto xchunk = [&](int net, int buf, int c) -> uint32_t {
+  // X chunk c of local net j as layer input: q (c < 2) or chunk c - 2 of h buffer `buf`
+  auto xchunk = [&](int j, int buf, int c) -> uint32_t {
     return c < 2 ? xq + static_cast<uint32_t>(c * N * 128)
-                 : xh + static_cast<uint32_t>(((net * nb + buf) * HC + (c - 2)) * N * 128);
+                 : xh + static_cast<uint32_t>(((j * nb + buf) * HC + (c - 2)) * N * 128);
   };
 
   if (threadIdx.x == 0) {
@@ -179,8 +194,8 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
     mbar_init(b_q, 1);
     mbar_init(b_acc, 1);
     mbar_init(b_acc + 8, 1);
-    mbar_init(b_hr, 2);            // the two nets' epilogue leaders; the peers' slices as transactions
-    mbar_init(b_hr + 8, 2);
+    mbar_init(b_hr, kNPC);         // the nets' epilogue leaders; the peers' slices as transactions
+    mbar_init(b_hr + 8, kNPC);
     mbar_init(b_ror, 1);
     mbar_init(b_rof, 1);
     fence_barrier_init();
@@ -209,21 +224,24 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
   const uint32_t tmem = *tslot;
   griddep_launch();                // the next kernel may take the SMs this call leaves idle
 
-  if (warp == 0 && lane == 0) {
-    // this CTA's weights towards L2 while an earlier kernel finishes
+  if (warp == 0) {
+    // this CTA's weights towards L2 while an earlier kernel finishes (a
+    // hint only; the lanes share the chunks)
+    int q = 0;
     for (int k = 0; k < depth; ++k) {
       const int K = layout::hidden_k(H, k), kc = layout::kchunks(K);
-      for (int net = 0; net < 2; ++net) {
-        const __nv_bfloat16* W = p.blob + (net ? tbase : sbase) + layout::hidden_w_off(H, depth, k);
-        for (int j = 0; j < MT; ++j) {
-          const int gu = u0 + 128 * j, m = gu >> 7, r0 = gu & 127;
-          const int rv = (slen - 128 * j < 128) ? (slen - 128 * j) : 128;
-          for (int c = 0; c < kc; ++c)
-            prefetch_l2(W + layout::tile_chunk_off(H, K, m, c) + r0 * 64, static_cast<uint32_t>(rv * 128));
+      for (int j = 0; j < kNPC; ++j) {
+        const __nv_bfloat16* W = p.blob + (n0 + j ? tbase : sbase) + layout::hidden_w_off(H, depth, k);
+        for (int t = 0; t < MT; ++t) {
+          const int gu = u0 + 128 * t, m = gu >> 7, r0 = gu & 127;
+          const int rv = (slen - 128 * t < 128) ? (slen - 128 * t) : 128;
+          for (int c = 0; c < kc; ++c, ++q)
+            if ((q & 31) == lane)
+              prefetch_l2(W + layout::tile_chunk_off(H, K, m, c) + r0 * 64, static_cast<uint32_t>(rv * 128));
         }
       }
     }
-    if (MT > 0)
+    if (has_target && MT > 0 && lane == 31)
       prefetch_l2(p.blob + tbase + layout::out_w_off(H, depth) + layout::tile_chunk_off(kD, H, 0, u0 / 64),
                   static_cast<uint32_t>((slen + 63) / 64 * 128 * 128));
   }
@@ -241,11 +259,11 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
       bool ok = true;
       for (int k = 0; k < depth && ok; ++k) {
         const int K = layout::hidden_k(H, k), kc = layout::kchunks(K);
-        for (int net = 0; net < 2 && ok; ++net) {
-          const __nv_bfloat16* W = p.blob + (net ? tbase : sbase) + layout::hidden_w_off(H, depth, k);
-          for (int j = 0; j < MT && ok; ++j) {
-            const int gu = u0 + 128 * j, m = gu >> 7, r0 = gu & 127;
-            const int rv = (slen - 128 * j < 128) ? (slen - 128 * j) : 128;
+        for (int j = 0; j < kNPC && ok; ++j) {
+          const __nv_bfloat16* W = p.blob + (n0 + j ? tbase : sbase) + layout::hidden_w_off(H, depth, k);
+          for (int t = 0; t < MT && ok; ++t) {
+            const int gu = u0 + 128 * t, m = gu >> 7, r0 = gu & 127;
+            const int rv = (slen - 128 * t < 128) ? (slen - 128 * t) : 128;
             const int rvp = rv <= 64 ? 64 : 128;
             const int cpg = static_cast<int>(kStage / (rvp * 128));
             const bool whole = (r0 == 0 && rv == 128);              // whole 128-row tiles are contiguous
@@ -270,7 +288,7 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
           }
         }
       }
-      if (ok && MT > 0) {
+      if (ok && has_target && MT > 0) {
         // the target readout's K range: chunks of the slice of W_out [d][H]
         const __nv_bfloat16* Wo = p.blob + tbase + layout::out_w_off(H, depth);
         const int cb = u0 / 64, nch = (slen + 63) / 64;
@@ -292,20 +310,20 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
       const uint32_t idesc = idesc_bf16_f32(128, N, 0, 0);
       for (int k = 0; k < depth && ok; ++k) {
         if (k > 0) {
-          // every CTA's slice of h_{k-1} (both nets) is in this CTA's X
+          // every slice of h_{k-1} (of the CTA's nets) is in this CTA's X
           ok = mbar_wait(b_hr + 8 * ((k - 1) & 1), ((k - 1) >> 1) & 1, p.err);
           if (!ok) break;
         }
         tc_fence_after();
         const int kc = layout::kchunks(layout::hidden_k(H, k));
         const int buf = (k - 1 + nb) % nb;
-        for (int net = 0; net < 2 && ok; ++net) {
+        for (int j = 0; j < kNPC && ok; ++j) {
           if (MT == 0) continue;
-          for (int j = 0; j < MT && ok; ++j) {
-            const int rv = (slen - 128 * j < 128) ? (slen - 128 * j) : 128;
+          for (int t = 0; t < MT && ok; ++t) {
+            const int rv = (slen - 128 * t < 128) ? (slen - 128 * t) : 128;
             const int rvp = rv <= 64 ? 64 : 128;
             const int cpg = static_cast<int>(kStage / (rvp * 128));
-            const uint32_t dcol = tmem + static_cast<uint32_t>((net * MTmax + j) * N);
+            const uint32_t dcol = tmem + static_cast<uint32_t>((j * MTmax + t) * N);
             for (int c0 = 0; c0 < kc; c0 += cpg, ++it) {
               const uint32_t s = it % S_;
               if (!mbar_wait(b_full + 8 * s, (it / S_) & 1, p.err)) {
@@ -316,7 +334,7 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
               const int nc = (kc - c0 < cpg) ? (kc - c0) : cpg;
               for (int cl = 0; cl < nc; ++cl) {
                 const uint32_t a = ring + s * kStage + cl * rvp * 128;
-                const uint32_t b = xchunk(net, buf, c0 + cl);
+                const uint32_t b = xchunk(j, buf, c0 + cl);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                   mma_bf16_ss(dcol, sdesc_sw128(a + kk * 32, 16, 1024), sdesc_sw128(b + kk * 32, 16, 1024), idesc,
@@ -325,15 +343,15 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
               mma_commit(b_empty + 8 * s);
             }
           }
-          mma_commit(b_acc + 8 * net);
+          mma_commit(b_acc + 8 * j);
         }
       }
-      if (ok && MT > 0) {
+      if (ok && has_target && MT > 0) {
         // target readout: A_theta partial [d][rows] over this CTA's units
         ok = mbar_wait(b_ror, 0, p.err);
         tc_fence_after();
         const int nch = (slen + 63) / 64;
-        const uint32_t dcol = tmem + static_cast<uint32_t>(2 * MTmax * N);
+        const uint32_t dcol = tmem + static_cast<uint32_t>(kNPC * MTmax * N);
         for (int c0 = 0; c0 < nch && ok; c0 += 2, ++it) {
           const uint32_t s = it % S_;
           if (!mbar_wait(b_full + 8 * s, (it / S_) & 1, p.err)) {
@@ -357,118 +375,124 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
     }
   } else if (warp < 2 + kEpiWarps) {
     // ------------------------------ epilogues ------------------------------
-    const int net = (warp - 2) >> 2;                 // 0 score, 1 target
+    const int j = (warp - 2) >> 2;                   // local net of this warp group
     const int q4 = warp & 3;                         // TMEM lane quarter of this warp
-    const int et = ((warp - 2) & 3) * 32 + lane;     // 0..127 within the net's warps
-    const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    const int64_t nbase = net ? tbase : sbase;
-    float* sp = reinterpret_cast<float*>(smem + SL.sp);
-    bool ok = true;
-    for (int k = 0; k < depth; ++k) {
-      const bool last = (k == depth - 1);
-      const int buf = k % nb;
-      const bool reduce = last && net == 0;           // the score readout: w . h summed here
-      if (MT > 0) {
-        if (ok) ok = mbar_wait(b_acc + 8 * net, k & 1, p.err);
-        tc_fence_after();
-        const __nv_bfloat16* bias = p.blob + nbase + layout::hidden_b_off(H, depth, k);
-        const __nv_bfloat16* wsc = p.blob + sbase + layout::out_w_off(H, depth);
-        for (int n0 = 0; n0 < N; n0 += 16) {
-          float part[16];
+    const int et = ((warp - 2) & 3) * 32 + lane;     // 0..127 within the group
+    if (j < kNPC) {
+      const int net = n0 + j;                        // 0 score, 1 target
+      const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+      const int64_t nbase = net ? tbase : sbase;
+      float* sp = reinterpret_cast<float*>(smem + SL.sp);
+      bool ok = true;
+      for (int k = 0; k < depth; ++k) {
+        const bool last = (k == depth - 1);
+        const int buf = k % nb;
+        const bool reduce = last && net == 0;           // the score readout: w . h summed here
+        if (MT > 0) {
+          if (ok) ok = mbar_wait(b_acc + 8 * j, k & 1, p.err);
+          tc_fence_after();
+          const __nv_bfloat16* bias = p.blob + nbase + layout::hidden_b_off(H, depth, k);
+          const __nv_bfloat16* wsc = p.blob + sbase + layout::out_w_off(H, depth);
+          for (int n0r = 0; n0r < N; n0r += 16) {
+            float part[16];
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) part[jj] = 0.f;
-          for (int j = 0; j < MT; ++j) {
-            const int u = j * 128 + q4 * 32 + lane;
-            const bool valid = u < slen && ok;
-            const int gu = u0 + u;
-            const float bv = valid ? __bfloat162float(bias[gu]) : 0.f;
-            const float wv = (valid && reduce) ? __bfloat162float(wsc[gu]) : 0.f;
-            uint32_t v[16];
-            NECTAR_TMEM_LD16(trow + static_cast<uint32_t>((net * MTmax + j) * N + n0), v);
-            tmem_ld_wait();
-            if (valid) {
+            for (int jj = 0; jj < 16; ++jj) part[jj] = 0.f;
+            for (int t = 0; t < MT; ++t) {
+              const int u = t * 128 + q4 * 32 + lane;
+              const bool valid = u < slen && ok;
+              const int gu = u0 + u;
+              const float bv = valid ? __bfloat162float(bias[gu]) : 0.f;
+              const float wv = (valid && reduce) ? __bfloat162float(wsc[gu]) : 0.f;
+              uint32_t v[16];
+              NECTAR_TMEM_LD16(trow + static_cast<uint32_t>((j * MTmax + t) * N + n0r), v);
+              tmem_ld_wait();
+              if (valid) {
 #pragma unroll
-              for (int jj = 0; jj < 16; jj += 2) {
-                const uint32_t w = pack_bf16x2(cl_silu(__uint_as_float(v[jj]) + bv),
-                                               cl_silu(__uint_as_float(v[jj + 1]) + bv));
-                if (reduce) {
-                  part[jj] = fmaf(wv, bf16lo(w), part[jj]);
-                  part[jj + 1] = fmaf(wv, bf16hi(w), part[jj + 1]);
-                } else {
-                  // h_k into the h buffer (to be exchanged), or -- the target's
-                  // last layer -- into the readout input, columns from the slice start
-                  uint8_t* dst = last ? smem + SL.xro : smem + SL.xq + (xchunk(net, buf, 2) - xq);
-                  const int col = last ? u : gu;
-                  *reinterpret_cast<uint16_t*>(dst + cl_xoff(N, n0 + jj, col)) = static_cast<uint16_t>(w & 0xFFFFu);
-                  *reinterpret_cast<uint16_t*>(dst + cl_xoff(N, n0 + jj + 1, col)) = static_cast<uint16_t>(w >> 16);
+                for (int jj = 0; jj < 16; jj += 2) {
+                  const uint32_t w = pack_bf16x2(cl_silu(__uint_as_float(v[jj]) + bv),
+                                                 cl_silu(__uint_as_float(v[jj + 1]) + bv));
+                  if (reduce) {
+                    part[jj] = fmaf(wv, bf16lo(w), part[jj]);
+                    part[jj + 1] = fmaf(wv, bf16hi(w), part[jj + 1]);
+                  } else {
+                    // h_k into the h buffer (to be exchanged), or -- the target's
+                    // last layer -- into the readout input, columns from the slice start
+                    uint8_t* dst = last ? smem + SL.xro : smem + SL.xq + (xchunk(j, buf, 2) - xq);
+                    const int col = last ? u : gu;
+                    *reinterpret_cast<uint16_t*>(dst + cl_xoff(N, n0r + jj, col)) = static_cast<uint16_t>(w & 0xFFFFu);
+                    *reinterpret_cast<uint16_t*>(dst + cl_xoff(N, n0r + jj + 1, col)) = static_cast<uint16_t>(w >> 16);
+                  }
                 }
               }
             }
-          }
-          if (reduce) {
+            if (reduce) {
 #pragma unroll
-            for (int jj = 0; jj < 16; ++jj) {
+              for (int jj = 0; jj < 16; ++jj) {
 #pragma unroll
-              for (int off = 16; off >= 1; off >>= 1) part[jj] += __shfl_xor_sync(0xffffffffu, part[jj], off);
+                for (int off = 16; off >= 1; off >>= 1) part[jj] += __shfl_xor_sync(0xffffffffu, part[jj], off);
+              }
+              if (lane == 0) {
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) sp[q4 * N + n0r + jj] = part[jj];
+              }
             }
-            if (lane == 0) {
-#pragma unroll
-              for (int jj = 0; jj < 16; ++jj) sp[q4 * N + n0 + jj] = part[jj];
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar_sync(1 + j, 128);
+        if (!last) {
+          if (et == 0) {
+            // own arrival, expecting the other slices of this net as transactions
+            uint32_t peer = 0;
+            for (int o = 0; o < kSlices; ++o) {
+              const int sl = cl_slice_len(H, o);
+              if (o != si && sl > 0) peer += static_cast<uint32_t>((sl + 63) / 64 * N * 128);
+            }
+            const uint32_t hr = b_hr + 8 * (k & 1);
+            mbar_arrive_expect_tx(hr, peer);
+            if (MT > 0) {
+              const uint32_t src = xchunk(j, buf, 2 + u0 / 64);
+              const uint32_t bytes = static_cast<uint32_t>((slen + 63) / 64 * N * 128);
+              for (int o = 0; o < kSlices; ++o)
+                if (o != si)
+                  bulk_s2cluster(mapa_shared(src, pbase + o), src, bytes, mapa_shared(hr, pbase + o));
             }
           }
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      named_bar_sync(1 + net, 128);
-      if (!last) {
-        if (et == 0) {
-          // own arrival, expecting the other CTAs' slices of this net as transactions
-          uint32_t peer = 0;
-          for (int o = 0; o < kCl; ++o) {
-            const int sl = cl_slice_len(H, o);
-            if (o != r && sl > 0) peer += static_cast<uint32_t>((sl + 63) / 64 * N * 128);
-          }
-          const uint32_t hr = b_hr + 8 * (k & 1);
-          mbar_arrive_expect_tx(hr, peer);
-          if (MT > 0) {
-            const uint32_t src = xchunk(net, buf, 2 + u0 / 64);
-            const uint32_t bytes = static_cast<uint32_t>((slen + 63) / 64 * N * 128);
-            for (int o = 0; o < kCl; ++o)
-              if (o != r) bulk_s2cluster(mapa_shared(src, o), src, bytes, mapa_shared(hr, o));
-          }
-        }
-      } else if (net == 0) {
-        // score partial of every row, to every CTA
-        if (et < R) {
-          const float v = MT > 0 ? (sp[et] + sp[N + et]) + (sp[2 * N + et] + sp[3 * N + et]) : 0.f;
-          const uint32_t dst = smem_u32(smem + SL.rs) + static_cast<uint32_t>((r * N + et) * 4);
-          for (int o = 0; o < kCl; ++o) st_cluster_f32(mapa_shared(dst, o), v);
-        }
-      } else {
-        // target readout partial [dim][row], to the owner of the dim
-        const int dim = q4 * 32 + lane;
-        const int o = dim / kOwnDims, dl = dim % kOwnDims;
-        const uint32_t dst = mapa_shared(smem_u32(smem + SL.rt) + static_cast<uint32_t>(((r * kOwnDims + dl) * N) * 4), o);
-        if (MT > 0) {
-          if (et == 0) mbar_arrive(b_ror);
-          if (ok) ok = mbar_wait(b_rof, 0, p.err);
-          tc_fence_after();
-          for (int n0 = 0; n0 < N; n0 += 16) {
-            uint32_t v[16];
-            NECTAR_TMEM_LD16(trow + static_cast<uint32_t>(2 * MTmax * N + n0), v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int jj = 0; jj < 16; jj += 4)
-              st_cluster_v4f(dst + (n0 + jj) * 4, __uint_as_float(v[jj]), __uint_as_float(v[jj + 1]),
-                             __uint_as_float(v[jj + 2]), __uint_as_float(v[jj + 3]));
+        } else if (net == 0) {
+          // score partial of every row, to every CTA
+          if (et < Rp) {
+            const float v = (MT > 0 && et < R) ? (sp[et] + sp[N + et]) + (sp[2 * N + et] + sp[3 * N + et]) : 0.f;
+            const uint32_t dst = smem_u32(smem + SL.rs) + static_cast<uint32_t>((si * Rp + et) * 4);
+            for (int o = 0; o < kC; ++o) st_cluster_f32(mapa_shared(dst, o), v);
           }
         } else {
-          for (int n0 = 0; n0 < N; n0 += 4) st_cluster_v4f(dst + n0 * 4, 0.f, 0.f, 0.f, 0.f);
+          // target readout partial [dim][row], to the owner of the dim
+          const int dim = q4 * 32 + lane;
+          const int o = dim / kOwn, dl = dim % kOwn;
+          const uint32_t dst =
+              mapa_shared(smem_u32(smem + SL.rt) + static_cast<uint32_t>(((si * kOwn + dl) * Rp) * 4), o);
+          if (MT > 0) {
+            if (et == 0) mbar_arrive(b_ror);
+            if (ok) ok = mbar_wait(b_rof, 0, p.err);
+            tc_fence_after();
+            for (int n0r = 0; n0r < Rp; n0r += 16) {
+              uint32_t v[16];
+              NECTAR_TMEM_LD16(trow + static_cast<uint32_t>(kNPC * MTmax * N + n0r), v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int jj = 0; jj < 16; jj += 4)
+                if (n0r + jj < Rp)
+                  st_cluster_v4f(dst + (n0r + jj) * 4, __uint_as_float(v[jj]), __uint_as_float(v[jj + 1]),
+                                 __uint_as_float(v[jj + 2]), __uint_as_float(v[jj + 3]));
+            }
+          } else {
+            for (int n = 0; n < Rp; n += 4) st_cluster_v4f(dst + n * 4, 0.f, 0.f, 0.f, 0.f);
+          }
         }
       }
+      tc_fence_before();
     }
-    tc_fence_before();
   } else {
     // ------------------------------ local attention ------------------------------
     using St = RowState<RG, 16>;
@@ -482,8 +506,8 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
     for (int t = 0; t < static_cast<int>(p.nq); ++t) {
       int b = 0;
       const int nv = visible_local(p.q_seq, p.q_pos, p.local_len, t, p.B, p.T, &b, p.err);
-      const int lo = static_cast<int>(static_cast<int64_t>(nv) * r / kCl);
-      const int hi = static_cast<int>(static_cast<int64_t>(nv) * (r + 1) / kCl);
+      const int lo = static_cast<int>(static_cast<int64_t>(nv) * r / kC);
+      const int hi = static_cast<int>(static_cast<int64_t>(nv) * (r + 1) / kC);
       const uint8_t* kb = reinterpret_cast<const uint8_t*>(p.Kloc) + ((hd * p.B + b) * p.T) * kRowBytes;
       const uint8_t* vb = reinterpret_cast<const uint8_t*>(p.Vloc) + ((hd * p.B + b) * p.T) * kRowBytes;
       for (int gb = 0; gb < gblocks; ++gb) {
@@ -536,11 +560,10 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
             as = fmaf(src[dim], wgt, as);
           }
           const int n = (g0 + rr) * static_cast<int>(p.nq) + t;
-          const int o = dim / kOwnDims;
-          st_cluster_f32(mapa_shared(rl0 + static_cast<uint32_t>(((r * N + n) * kOwnDims + dim % kOwnDims) * 4), o),
-                         as);
-          if (dim < kCl) {
-            const uint32_t d2 = mapa_shared(rml0 + static_cast<uint32_t>((r * N + n) * 2 * 4), dim);
+          const int o = dim / kOwn;
+          st_cluster_f32(mapa_shared(rl0 + static_cast<uint32_t>(((r * Rp + n) * kOwn + dim % kOwn) * 4), o), as);
+          if (dim < kC) {
+            const uint32_t d2 = mapa_shared(rml0 + static_cast<uint32_t>((r * Rp + n) * 2 * 4), dim);
             st_cluster_f32(d2, M);
             st_cluster_f32(d2 + 4, ls);
           }
@@ -560,31 +583,31 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
     const float* rml = reinterpret_cast<const float*>(smem + SL.rml);
     const float cs = __bfloat162float(p.blob[sbase + layout::out_b_off(H, depth, 1)]);
     const __nv_bfloat16* ct = p.blob + tbase + layout::out_b_off(H, depth, kD);
-    const int64_t rows = R;
-    for (int item = threadIdx.x - 64; item < R * kOwnDims; item += kThreads - 64) {
-      const int n = item / kOwnDims, dl = item % kOwnDims;
-      const int dim = r * kOwnDims + dl;
+    for (int item = threadIdx.x - 64; item < R * kOwn; item += kThreads - 64) {
+      const int n = item / kOwn, dl = item % kOwn;
+      const int dim = r * kOwn + dl;
       float a = 0.f, at = 0.f, Ml = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kCl; ++c) {
-        a += rs[c * N + n];
-        at += rt[(c * kOwnDims + dl) * N + n];
-        Ml = fmaxf(Ml, rml[(c * N + n) * 2]);
+      for (int c = 0; c < kSlices; ++c) {
+        a += rs[c * Rp + n];
+        at += rt[(c * kOwn + dl) * Rp + n];
       }
+#pragma unroll
+      for (int c = 0; c < kC; ++c) Ml = fmaxf(Ml, rml[(c * Rp + n) * 2]);
       a += cs;
       at += __bfloat162float(ct[dim]);
       float ll = 0.f, al = 0.f;
 #pragma unroll
-      for (int c = 0; c < kCl; ++c) {
-        const float wgt = exp2_shift(rml[(c * N + n) * 2], Ml);
-        ll = fmaf(rml[(c * N + n) * 2 + 1], wgt, ll);
-        al = fmaf(rl[(c * N + n) * kOwnDims + dl], wgt, al);
+      for (int c = 0; c < kC; ++c) {
+        const float wgt = exp2_shift(rml[(c * Rp + n) * 2], Ml);
+        ll = fmaf(rml[(c * Rp + n) * 2 + 1], wgt, ll);
+        al = fmaf(rl[(c * Rp + n) * kOwn + dl], wgt, al);
       }
       const float ad = a * kLog2e;                     // document logit in log2 units
       const float M = fmaxf(ad, Ml);
       const float wd = exp2_shift(ad, M), wl = exp2_shift(Ml, M);
       const float v = (wd * at + wl * al) / (wd + wl * ll);
-      const int64_t row = hd * rows + n;
+      const int64_t row = hd * R + n;
       if (p.out_bf16 != nullptr)
         p.out_bf16[layer_layout_index(row, dim, p.Hkv, p.G, p.nq)] = __float2bfloat16_rn(v);
       else
@@ -599,29 +622,65 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
   }
 }
 
-template <int RG>
-cudaError_t launch_cl(const CUtensorMap& tq, const ClusterParams& p, int heads, size_t smem, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(decode_cluster_kernel<RG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <int RG, int kC>
+cudaError_t set_attrs(size_t smem) {
+  cudaError_t e = cudaFuncSetAttribute(decode_cluster_kernel<RG, kC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
+  if (e == cudaSuccess && kC > 8)
+    e = cudaFuncSetAttribute(decode_cluster_kernel<RG, kC>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
+
+template <int RG, int kC>
+cudaError_t launch_cl(const CUtensorMap& tq, const ClusterParams& p, int heads, size_t smem, cudaStream_t stream) {
+  const cudaError_t e = set_attrs<RG, kC>(smem);
   if (e != cudaSuccess) return e;
-  return launch_k(decode_cluster_kernel<RG>, dim3(static_cast<unsigned>(heads * kCl)), dim3(kThreads), smem, stream,
-                  kCl, tq, p);
+  return launch_k(decode_cluster_kernel<RG, kC>, dim3(static_cast<unsigned>(heads * kC)), dim3(kThreads), smem,
+                  stream, kC, tq, p);
+}
+
+// Clusters of this shape that can be resident at once (0: none, or unknown).
+template <int RG, int kC>
+int max_clusters(size_t smem) {
+  if (set_attrs<RG, kC>(smem) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kC);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = kC;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, decode_cluster_kernel<RG, kC>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
 }
 
 }  // namespace
 
 int cluster_rg(int G) { return G <= 2 ? 2 : 4; }
 
-ClusterShape cluster_shape(int G, int64_t nq, int Hmax, int depth) {
+ClusterShape cluster_shape(int cluster, int G, int64_t nq, int Hmax, int depth) {
   ClusterShape sh{};
   const int64_t R = static_cast<int64_t>(G) * nq;
-  if (R < 1 || R > 64 || nq > 256 || depth < 1 || depth > 4) return sh;
+  if ((cluster != 8 && cluster != 16) || R < 1 || R > 64 || nq > 256 || depth < 1 || depth > 4) return sh;
+  sh.cluster = cluster;
   sh.N = static_cast<int>((R + 15) / 16 * 16);
   sh.nb = depth >= 3 ? 2 : 1;
+  const int npc = cluster == 16 ? 1 : 2;
   const int rg = cluster_rg(G);
   constexpr size_t kMax = 227 * 1024;
-  for (int st = 6; st >= 2; --st) {
-    const size_t smem = cl_layout(Hmax, sh.N, sh.nb, st, rg).total + 1024;
+  for (int st = kMaxStages; st >= 2; --st) {
+    const size_t smem = cl_layout(cluster, npc, Hmax, sh.N, static_cast<int>(R), sh.nb, st, rg).total + 1024;
     if (smem <= kMax) {
       sh.stages = st;
       sh.smem = smem;
@@ -629,8 +688,21 @@ ClusterShape cluster_shape(int G, int64_t nq, int Hmax, int depth) {
     }
   }
   if (sh.stages == 0) return sh;
+  // no longer a ring than one CTA's weights of the widest layer need
+  {
+    const int S = cl_slice(Hmax);
+    int64_t groups = 0;                  // ring stages the producer fills, as it groups the chunks
+    const int cpg = S <= 64 ? 4 : 2;
+    for (int k = 0; k < depth; ++k)
+      groups += npc * ((S + 127) / 128) * ((layout::kchunks(layout::hidden_k(Hmax, k)) + cpg - 1) / cpg);
+    groups += (layout::kchunks(S) + 1) / 2;
+    if (groups < sh.stages) {
+      sh.stages = groups < 2 ? 2 : static_cast<int>(groups);
+      sh.smem = cl_layout(cluster, npc, Hmax, sh.N, static_cast<int>(R), sh.nb, sh.stages, rg).total + 1024;
+    }
+  }
   const int MTmax = (cl_slice(Hmax) + 127) / 128;
-  const int cols = (2 * MTmax + 1) * sh.N;
+  const int cols = (npc * MTmax + 1) * sh.N;
   int c = 32;
   while (c < cols) c <<= 1;
   sh.tmem_cols = c;
@@ -638,9 +710,19 @@ ClusterShape cluster_shape(int G, int64_t nq, int Hmax, int depth) {
   return sh;
 }
 
-cudaError_t launch_decode_cluster(const CUtensorMap& tq, const ClusterParams& p, int heads, size_t smem,
+int cluster_max_active(const ClusterShape& sh, int G) {
+  if (!sh.ok) return 0;
+  const bool rg2 = cluster_rg(G) == 2;
+  if (sh.cluster == 16) return rg2 ? max_clusters<2, 16>(sh.smem) : max_clusters<4, 16>(sh.smem);
+  return rg2 ? max_clusters<2, 8>(sh.smem) : max_clusters<4, 8>(sh.smem);
+}
+
+cudaError_t launch_decode_cluster(const CUtensorMap& tq, const ClusterParams& p, int cluster, int heads, size_t smem,
                                   cudaStream_t stream) {
-  return cluster_rg(p.G) == 2 ? launch_cl<2>(tq, p, heads, smem, stream) : launch_cl<4>(tq, p, heads, smem, stream);
+  const bool rg2 = cluster_rg(p.G) == 2;
+  if (cluster == 16)
+    return rg2 ? launch_cl<2, 16>(tq, p, heads, smem, stream) : launch_cl<4, 16>(tq, p, heads, smem, stream);
+  return rg2 ? launch_cl<2, 8>(tq, p, heads, smem, stream) : launch_cl<4, 8>(tq, p, heads, smem, stream);
 }
 
 }  // namespace nectar

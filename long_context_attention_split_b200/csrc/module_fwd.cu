@@ -268,8 +268,9 @@ __device__ __forceinline__ void module_cta(const CUtensorMap* tmap_q, const ModP
         const __nv_bfloat16* bias = blob + nb + layout::hidden_b_off(H, depth, k);
         const bool readout = (net == 0 && k == depth - 1);   // score net: reduce w . h here
         const __nv_bfloat16* wsc = blob + nb + layout::out_w_off(H, depth);
-        // this thread's biases (and readout weights) do not depend on the
-        // accumulators: fetch them while the layer's MMAs run
+        // this thread's biases (and readout weights) of the first 8 row tiles
+        // do not depend on the accumulators: fetch them while the layer's
+        // MMAs run (wider layers read the rest when they need them)
         float bvs[8], wvs[8];
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
@@ -296,12 +297,17 @@ __device__ __forceinline__ void module_cta(const CUtensorMap* tmap_q, const ModP
               const int i = (m0 + mm) * 128 + u;
               if (mm < mc && ok && i < H) {
                 float bv = 0.f, wv = 0.f;
+                if (m0 + mm < 8) {
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                  if (q == m0 + mm) {
-                    bv = bvs[q];
-                    wv = wvs[q];
-                  }
+                  for (int q = 0; q < 8; ++q)
+                    if (q == m0 + mm) {
+                      bv = bvs[q];
+                      wv = wvs[q];
+                    }
+                } else {
+                  bv = __bfloat162float(bias[i]);
+                  wv = readout ? __bfloat162float(wsc[i]) : 0.f;
+                }
                 uint32_t ws[8];
 #pragma unroll
                 for (int j = 0; j < 16; j += 2) {
@@ -498,12 +504,14 @@ ModShape mod_shape(int G, int64_t nq, int Hmax, bool fuse) {
   int tpc = 64 / G;
   if (tpc < 1) tpc = 1;
   if (tpc > nq) tpc = static_cast<int>(nq);
+  const int mt = (Hmax + 127) / 128;
   while (true) {
     const int N = (G * tpc + 15) / 16 * 16;
     sh.TPC = tpc;
     sh.N = N;
     sh.smem = mod_smem_layout(Hmax, N, 3, 1).total + 1024;
-    if (sh.smem <= kBudget || tpc == 1) break;
+    // the layer's M tiles sit side by side in TMEM: mt * N <= 512 columns
+    if ((sh.smem <= kBudget && mt * N <= 512) || tpc == 1) break;
     tpc = (tpc + 1) / 2;
   }
   // plans that fit half an SM run two CTAs per SM
@@ -517,7 +525,6 @@ ModShape mod_shape(int G, int64_t nq, int Hmax, bool fuse) {
   sh.smem = mod_smem_layout(Hmax, sh.N, stages, cps).total + 1024;
   if (sh.smem < floor_smem) sh.smem = floor_smem;   // the decode's local CTAs share the launch
   sh.nblk = static_cast<int>((nq + sh.TPC - 1) / sh.TPC);
-  const int mt = (Hmax + 127) / 128;
   sh.tmem_cols = mod_tmem_cols(mt, sh.N);
   return sh;
 }

@@ -223,6 +223,8 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  griddep_wait();                 // inputs and outputs only from here on (launched after another kernel)
+  griddep_launch();
 
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
@@ -470,14 +472,12 @@ cudaError_t launch_module_gemm(const CUtensorMap& tq, const CUtensorMap& th, con
     cudaError_t e = cudaFuncSetAttribute(module_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    module_gemm_kernel<true><<<grid, kGemmThreads, smem, stream>>>(tq, th, p);
-  } else {
-    cudaError_t e = cudaFuncSetAttribute(module_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    module_gemm_kernel<false><<<grid, kGemmThreads, smem, stream>>>(tq, th, p);
+    return launch_k(module_gemm_kernel<true>, dim3(grid), dim3(kGemmThreads), smem, stream, 1, tq, th, p);
   }
-  return cudaGetLastError();
+  cudaError_t e = cudaFuncSetAttribute(module_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_k(module_gemm_kernel<false>, dim3(grid), dim3(kGemmThreads), smem, stream, 1, tq, th, p);
 }
 
 }  // namespace nectar

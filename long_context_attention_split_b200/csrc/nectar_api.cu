@@ -774,9 +774,14 @@ size_t decode_ws_a_bytes(int64_t rows) { return align256(static_cast<size_t>(row
 
 // Many query rows per KV head, or a set with a backbone or unequal nets:
 // the module runs layer by layer as grouped GEMMs (module_gemm.cu) instead
-// of one CTA per block of <= 64 rows.
-bool use_gemm_path(const nectar_dims& dims, int64_t nq, bool general) {
-  return general || static_cast<int64_t>(dims.G) * nq >= kGemmMinRows;
+// of one CTA per block of <= 64 rows.  So do widths whose M tiles, side by
+// side for the G rows of one token, would need more than 512 TMEM columns
+// in the one-CTA kernel.
+int arch_hmax(const nectar_dims& dims, const Arch& a);
+bool use_gemm_path(const nectar_dims& dims, int64_t nq, bool general, int Hmax) {
+  if (general || static_cast<int64_t>(dims.G) * nq >= kGemmMinRows) return true;
+  const int mt = (Hmax + 127) / 128;
+  return mt * ((dims.G + 15) / 16 * 16) > 512;
 }
 
 // widest layer of any part, widest score net, hidden layers of the longest chain
@@ -923,7 +928,7 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
     int64_t acc = 0;
     for (int li = 0; li < dims.L; ++li) {
       g.tile_start[li] = acc;
-      const int l = mp.order[li];
+      const int l = g.order[li];
       const int j = stage - mp.depth_b;
       int mt;                                   // 128-unit tiles per head, as gemm_tile counts them
       if (g.readout) mt = 1;
@@ -933,6 +938,7 @@ nectar_status run_module_gemm(const nectar_dims& dims, const ModParams& mp, cons
     }
     g.tile_start[dims.L] = acc;
     g.ntiles = acc;
+    if (acc == 0) continue;
     const int grid = static_cast<int>(acc < di.sms ? acc : di.sms);
     const CUtensorMap& tin = g.readout ? thr : (stage == 0 ? tq : th[(stage - 1) & 1]);
     cudaError_t e = launch_module_gemm(tq, tin, g, grid, ss.smem, st);
@@ -984,9 +990,11 @@ nectar_status prepare_modules(const nectar_dims& dims, const nectar_module_set* 
   for (int l = 0; l < dims.L; ++l) p->order[l] = static_cast<uint8_t>(ord[l]);
   const int Hmax = arch_hmax(dims, ar);
   p->Hmax = Hmax;
-  if (use_gemm_path(dims, nq, ar.general)) return NECTAR_OK;   // the layer-by-layer path needs no fused shape
+  if (use_gemm_path(dims, nq, ar.general, arch_hmax(dims, ar))) return NECTAR_OK;   // the layer-by-layer path needs no fused shape
   *sh = mod_shape(dims.G, nq, Hmax, fuse);
   if (sh->smem > 227 * 1024) return fail(NECTAR_ERR_UNSUPPORTED, "width %d needs too much shared memory", Hmax);
+  if (sh->tmem_cols > 512)
+    return fail(NECTAR_ERR_UNSUPPORTED, "width %d with G = %d needs more than 512 TMEM columns", Hmax, dims.G);
   // one CTA per net when every layer's net streams at least 1 MB of weights:
   // then the two streams side by side on different SMs outweigh the extra
   // CTA start-up (measured: H = 720 / 912 gains 8 %, H = 512 loses 3 %)
@@ -1022,7 +1030,7 @@ size_t nectar_module_workspace_size(nectar_dims dims, const nectar_module_set* m
   if (check_dims(dims) != NECTAR_OK || nq <= 0 || mods == nullptr) return 0;
   Arch ar;
   if (arch_of(dims, mods, &ar) != NECTAR_OK) return 0;
-  if (!use_gemm_path(dims, nq, ar.general)) return 0;
+  if (!use_gemm_path(dims, nq, ar.general, arch_hmax(dims, ar))) return 0;
   return gemm_ws_bytes(dims, ar, nq);
 }
 
@@ -1039,7 +1047,7 @@ nectar_status nectar_module_forward(nectar_dims dims, const nectar_module_set* m
   ModShape sh;
   NECTAR_TRY(prepare_modules(dims, mods, Q, nq, false, &p, &tq, &sh));
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (use_gemm_path(dims, nq, p.general)) {
+  if (use_gemm_path(dims, nq, p.general, p.Hmax)) {
     const size_t need = nectar_module_workspace_size(dims, mods, nq);
     if (workspace == nullptr || workspace_bytes < need)
       return fail(NECTAR_ERR_WORKSPACE, "module workspace of %zu bytes given, %zu needed",
@@ -1061,14 +1069,14 @@ size_t nectar_decode_workspace_size(nectar_dims dims, const nectar_module_set* m
   if (arch_of(dims, mods, &ar) != NECTAR_OK) return 0;
   const int64_t rows = static_cast<int64_t>(dims.L) * dims.Hkv * dims.G * nq;
   const size_t loc = align256(static_cast<size_t>(rows) * (kD + 2) * sizeof(float));
-  if (use_gemm_path(dims, nq, ar.general)) return loc + gemm_ws_bytes(dims, ar, nq);
+  if (use_gemm_path(dims, nq, ar.general, arch_hmax(dims, ar))) return loc + gemm_ws_bytes(dims, ar, nq);
   return decode_ws_a_bytes(rows) + loc;
 }
 
 size_t nectar_decode_layer_out_workspace_size(nectar_dims dims, const nectar_module_set* mods, int64_t nq) {
   const size_t base = nectar_decode_workspace_size(dims, mods, nq);
   Arch ar;
-  if (base == 0 || arch_of(dims, mods, &ar) != NECTAR_OK || use_gemm_path(dims, nq, ar.general)) return base;
+  if (base == 0 || arch_of(dims, mods, &ar) != NECTAR_OK || use_gemm_path(dims, nq, ar.general, arch_hmax(dims, ar))) return base;
   // the one-launch path keeps A_theta in fp32 until the merge
   const int64_t rows = static_cast<int64_t>(dims.L) * dims.Hkv * dims.G * nq;
   return base + align256(static_cast<size_t>(rows) * kD * sizeof(float));
@@ -1085,16 +1093,51 @@ namespace {
 #define NECTAR_CLUSTER_MAX_HEADS 32
 #endif
 
-// NECTAR_DECODE_CLUSTER=0 never takes the cluster decode, =1 takes it
-// whenever it applies; unset: by the head count above.
-bool use_cluster_decode(const nectar_dims& dims, int64_t nq, const Arch& ar, int Hmax) {
-  if (ar.general || static_cast<int64_t>(dims.G) * nq > 64) return false;
+// Resident clusters of a cluster-decode plan on the current device, cached.
+int cached_max_active(const ClusterShape& sh, int G) {
+  struct Key {
+    int dev, cluster, rg2;
+    size_t smem;
+    int n;
+  };
+  static std::mutex mu;
+  static std::vector<Key> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const int rg2 = G <= 2 ? 1 : 0;
+  std::lock_guard<std::mutex> lk(mu);
+  for (const Key& k : cache)
+    if (k.dev == dev && k.cluster == sh.cluster && k.rg2 == rg2 && k.smem == sh.smem) return k.n;
+  const int n = cluster_max_active(sh, G);
+  cache.push_back(Key{dev, sh.cluster, rg2, sh.smem, n});
+  return n;
+}
+
+// The cluster size (8 or 16) the decode takes, or 0 for the one-launch
+// kernel.  NECTAR_DECODE_CLUSTER=0 never takes the cluster decode, =8 or
+// =16 takes that size whenever it applies; unset: with at most
+// NECTAR_CLUSTER_MAX_HEADS (l, h) pairs, 8-CTA clusters (both nets per CTA;
+// measured faster than 16 on one Qwen3-1.7B layer: 17.4 against 27.4 us per
+// layer in a graph), or 16-CTA ones where only those fit.
+int cluster_decode_size(const nectar_dims& dims, int64_t nq, const Arch& ar, int Hmax, ClusterShape* out) {
+  if (ar.general || static_cast<int64_t>(dims.G) * nq > 64) return 0;
   const char* env = getenv("NECTAR_DECODE_CLUSTER");
   const int mode = (env != nullptr && env[0] != 0) ? atoi(env) : -1;
-  if (mode == 0) return false;
-  if (!cluster_shape(dims.G, nq, Hmax, ar.Ds).ok) return false;
-  if (mode == 1) return true;
-  return static_cast<int64_t>(dims.L) * dims.Hkv <= NECTAR_CLUSTER_MAX_HEADS;
+  if (mode == 0) return 0;
+  const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
+  if (mode == 8 || mode == 16) {
+    *out = cluster_shape(mode, dims.G, nq, Hmax, ar.Ds);
+    return out->ok && cached_max_active(*out, dims.G) > 0 ? mode : 0;
+  }
+  if (heads > NECTAR_CLUSTER_MAX_HEADS) return 0;
+  for (const int size : {8, 16}) {
+    const ClusterShape sh = cluster_shape(size, dims.G, nq, Hmax, ar.Ds);
+    if (sh.ok && cached_max_active(sh, dims.G) > 0) {
+      *out = sh;
+      return size;
+    }
+  }
+  return 0;
 }
 
 // The decode, into out (fp32, per KV head) or out_bf16 (bf16, layer layout).
@@ -1124,7 +1167,7 @@ nectar_status decode_impl(nectar_dims dims, const nectar_module_set* mods, const
   NECTAR_TRY(prepare_modules(dims, mods, Q, nq, true, &p, &tq, &sh));
   const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
   const int64_t rows = heads * dims.G * nq;
-  const bool gemm = use_gemm_path(dims, nq, ar.general);
+  const bool gemm = use_gemm_path(dims, nq, ar.general, arch_hmax(dims, ar));
   if (heads * nq + (gemm ? 0 : (p.net_split ? 2 : 1) * static_cast<int64_t>(dims.L) * dims.Hkv * sh.nblk) >
       0x7fffffffLL)
     return fail(NECTAR_ERR_UNSUPPORTED, "too many CTAs for one launch");
@@ -1154,8 +1197,8 @@ nectar_status decode_impl(nectar_dims dims, const nectar_module_set* mods, const
     return run_module_gemm(dims, p, Q, nq, nullptr, out, p.ws_loc,
                            base + align256(static_cast<size_t>(rows) * (kD + 2) * sizeof(float)), st, out_bf16);
   }
-  if (use_cluster_decode(dims, nq, ar, p.Hmax)) {
-    const ClusterShape cs = cluster_shape(dims.G, nq, p.Hmax, ar.Ds);
+  ClusterShape cs{};
+  if (const int csize = cluster_decode_size(dims, nq, ar, p.Hmax, &cs)) {
     ClusterParams c;
     memset(&c, 0, sizeof(c));
     c.Hkv = dims.Hkv;
@@ -1192,7 +1235,7 @@ nectar_status decode_impl(nectar_dims dims, const nectar_module_set* mods, const
     const cuuint64_t strq[3] = {256, static_cast<cuuint64_t>(nq) * 256, static_cast<cuuint64_t>(nq) * 256 * dims.G};
     const cuuint32_t boxq[4] = {64, static_cast<cuuint32_t>(nq), static_cast<cuuint32_t>(dims.G), 1};
     NECTAR_TRY(make_tmap(&tqc, Q, 4, dimsq, strq, boxq, "queries (cluster decode)"));
-    cudaError_t e = launch_decode_cluster(tqc, c, static_cast<int>(heads), cs.smem, st);
+    cudaError_t e = launch_decode_cluster(tqc, c, csize, static_cast<int>(heads), cs.smem, st);
     return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "cluster decode kernel");
   }
   p.a_out = reinterpret_cast<float*>(base);

@@ -61,7 +61,7 @@ def test_host_validation_without_device():
     assert st == 1
     w = (ctypes.c_int32 * 2)(64, 40)      # 40 is not a multiple of 16
     assert L.nectar_module_packed_elems(nx.Dims(2, 1, 1, 128), 2, w) == 0
-    w = (ctypes.c_int32 * 1)(2048)        # too wide
+    w = (ctypes.c_int32 * 1)(2064)        # too wide
     assert L.nectar_module_packed_elems(nx.Dims(1, 1, 1, 128), 2, w) == 0
     w = (ctypes.c_int32 * 1)(64)
     assert L.nectar_module_packed_elems(nx.Dims(1, 1, 1, 128), 0, w) == 0
@@ -114,7 +114,7 @@ def read_net(blob, off, H, depth, dout, d=128):
 
 
 @pytest.mark.parametrize("widths,depth,hkv", [([64, 32], 2, 2), ([48], 3, 1), ([16, 208], 1, 3), ([272], 2, 1),
-                                               ([96, 1024], 4, 1)])   # the depth and width limits
+                                               ([96, 2048], 4, 1)])   # the depth and width limits
 def test_pack_layout(widths, depth, hkv):
     mods = make_modules(len(widths), hkv, widths, 128, seed=3, device="cpu", depth=depth)
     ms = nx.pack_modules(mods, widths, depth, hkv, G=2, device=None)
@@ -168,7 +168,7 @@ def test_arch_validation_on_the_host():
                                ((0, 1, 0), [], [32, 16], [48, 96]),
                                ((3, 1, 2), [64, 32], [32, 16], [48, 96]),     # chain of 5 > NECTAR_MAX_DEPTH
                                ((1, 1, 1), [64, 40], [32, 16], [48, 96]),     # width not a multiple of 16
-                               ((0, 2, 2), [], [32, 2048], [48, 96]),         # width above the maximum
+                               ((0, 2, 2), [], [32, 2064], [48, 96]),         # width above the maximum
                                ((-1, 1, 1), [], [32, 16], [48, 96])]:
         assert nx.Arch(depths, wb, ws, wt).packed_elems(2) == 0, depths
 
@@ -186,17 +186,19 @@ def _host_set(L, Hkv, widths, depth, arch=None):
     return nx.ModuleSet(torch.zeros(n, dtype=torch.bfloat16), widths, depth, L, Hkv)
 
 
-@pytest.mark.parametrize("widths,depth", [([256, 512, 384], 2), ([208, 144, 80], 1), ([128, 128, 1024], 3)])
-@pytest.mark.parametrize("G,nq", [(2, 1), (4, 8), (2, 32), (8, 40)])
+@pytest.mark.parametrize("widths,depth", [([256, 512, 384], 2), ([208, 144, 80], 1), ([128, 128, 1024], 3),
+                                          ([2048, 1152], 2)])
+@pytest.mark.parametrize("G,nq", [(2, 1), (4, 8), (2, 32), (8, 40), (40, 1)])
 def test_workspace_sizes_follow_the_header(widths, depth, G, nq):
     """nectar_module_workspace_size, nectar_decode_workspace_size and
     nectar_decode_layer_out_workspace_size equal the formulas include/nectar.h
-    states for them (classic sets; 64 query rows per KV head or more take the
-    layer-by-layer path)."""
+    states for them (classic sets; 64 query rows per KV head or more, or
+    widths whose 128-unit tiles for round16(G) rows exceed 512 TMEM columns,
+    take the layer-by-layer path)."""
     L, Hkv, d = len(widths), 2, 128
     mods = _host_set(L, Hkv, widths, depth)
     rows = L * Hkv * G * nq
-    gemm = G * nq >= 64
+    gemm = G * nq >= 64 or math.ceil(max(widths) / 128) * (-(-G // 16) * 16) > 512
     Hp = r64(max(widths))
     mod_ws = ((2 if depth >= 2 else 1) * a256(2 * rows * Hp * 2) + a256(rows * math.ceil(max(widths) / 128) * 4)
               if gemm else 0)
@@ -337,10 +339,10 @@ def test_layer_depth_and_width_limits_on_the_host():
     assert nx.packed_elems(256, 1, 1, [16] * 256, 1) > 0
     assert nx.packed_elems(257, 1, 1, [16] * 257, 1) <= 0
     assert b"L = 257" in L.nectar_last_error()
-    assert nx.packed_elems(1, 1, 1, [1024], 4) > 0
+    assert nx.packed_elems(1, 1, 1, [2048], 4) > 0
     assert nx.packed_elems(1, 1, 1, [64], 5) <= 0
     assert b"depth 5" in L.nectar_last_error()
-    assert nx.packed_elems(1, 1, 1, [1040], 2) <= 0
+    assert nx.packed_elems(1, 1, 1, [2064], 2) <= 0
     # a backbone chain counts against the depth limit as a whole
     assert nx.Arch((2, 2, 1), [64], [64], [64]).packed_elems(1) > 0
     assert nx.Arch((2, 3, 1), [64], [64], [64]).packed_elems(1) <= 0

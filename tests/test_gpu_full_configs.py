@@ -154,6 +154,21 @@ def test_qwen25_7b_decode_full():
     torch.cuda.empty_cache()
 
 
+def test_qwen25_7b_decode_rho10_full():
+    """The Qwen2.5-7B-shaped decode at the stated capacity rho = 10 %: H = 1152
+    (10.12 % of 2nd per (l, h); H = 768 is 4.99 %), 28 x 4 heads, G = 7,
+    n = 131072, 64 sequences x 256 local tokens."""
+    wl = make_workload("qwen25_7b_decode", device="cuda", H=1152)
+    mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G, device="cuda")
+    out = nx.decode(mods, wl.Q, wl.q_seq, wl.q_pos, wl.Kloc, wl.Vloc, wl.local_len)
+    a, At = nx.module_forward(mods, wl.Q)
+    torch.cuda.synchronize()
+    assert nx.device_error_flags() == 0
+    check_decode(wl, out, sample_heads(wl, 3, 3), [0, 31, 63], a, At)
+    del wl, mods, out, a, At
+    torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("B,rho", [(1, 0.10), (16, 0.10), (256, 0.10), (16, 0.01), (16, 0.05)])
 def test_llama8b_sweep_full(B, rho):
     """32 x 8 heads, G = 4, n = 65536, 128 local tokens, non-uniform widths."""

@@ -369,6 +369,11 @@ def test_module_forward_toy():
     dict(L=1, Hkv=1, G=7, nq=9, widths=[144], depth=2),         # 63 rows: still one CTA per block of tokens
     dict(L=2, Hkv=2, G=2, nq=5, widths=[768, 1024], depth=2),   # >= 1 MB per net: one CTA per net
     dict(L=1, Hkv=1, G=3, nq=4, widths=[1024], depth=3),
+    # widths past 8 row tiles (up to NECTAR_MAX_WIDTH = 2048)
+    dict(L=2, Hkv=1, G=2, nq=3, widths=[2048, 1152], depth=2),  # one launch, 16 and 9 row tiles
+    dict(L=1, Hkv=2, G=7, nq=2, widths=[1152], depth=3),
+    dict(L=1, Hkv=1, G=40, nq=1, widths=[2048], depth=2),       # 16 tiles x 48 rows > 512 TMEM columns: GEMM path
+    dict(L=1, Hkv=2, G=4, nq=40, widths=[2048], depth=2),       # grouped GEMM, 16 units tiles
 ])
 def test_module_forward_shapes(kw):
     kw = dict(kw)
@@ -431,6 +436,8 @@ def test_decode_toy_prefill():
     dict(L=2, Hkv=2, G=4, n=16, B=16, T=40, widths=[256, 128]),   # exactly 64 rows: grouped-GEMM decode
     dict(L=1, Hkv=2, G=16, n=16, B=8, T=300, widths=[256]),    # 128 rows, 16 heads per local job, 3 tiles
     dict(L=2, Hkv=2, G=2, n=16, B=3, T=40, widths=[768, 896]),   # one CTA per net in the one-launch decode
+    dict(L=1, Hkv=2, G=2, n=16, B=3, T=40, widths=[2048]),        # the widest layer, one-launch decode
+    dict(L=1, Hkv=1, G=7, n=16, B=16, T=40, widths=[1152]),       # 112 rows: grouped GEMM at 1152 units
 ])
 def test_decode_shapes(kw):
     wl = make_workload("qwen3_1p7b", seed=2, key_scale=None, **kw)
@@ -455,8 +462,9 @@ def test_decode_shapes(kw):
     dict(L=1, Hkv=2, G=16, n=16, B=4, T=300, widths=[256]),
     dict(L=2, Hkv=2, G=2, n=16, B=1, T=512, widths=[512, 512]),     # the headline's shape per layer
 ])
-def test_decode_cluster_shapes(kw, monkeypatch):
-    monkeypatch.setenv("NECTAR_DECODE_CLUSTER", "1")
+@pytest.mark.parametrize("cluster", ["8", "16"])
+def test_decode_cluster_shapes(kw, cluster, monkeypatch):
+    monkeypatch.setenv("NECTAR_DECODE_CLUSTER", cluster)
     wl = make_workload("qwen3_1p7b", seed=7, key_scale=None, **kw)
     wl.local_len = torch.randint(0, wl.T + 1, (wl.B,), generator=torch.Generator().manual_seed(5)).to(torch.int32)
     wl.q_pos = (wl.local_len[wl.q_seq.long()] - 1).clamp(min=0).to(torch.int32)
@@ -469,15 +477,16 @@ def test_decode_cluster_matches_one_launch(monkeypatch):
     wl = make_workload("qwen3_1p7b", seed=8, key_scale=None, L=3, Hkv=2, G=2, n=16, B=2, T=100, widths=[512] * 3)
     mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G)
     args = (cuda(wl.Q), cuda(wl.q_seq), cuda(wl.q_pos), cuda(wl.Kloc), cuda(wl.Vloc), cuda(wl.local_len))
-    monkeypatch.setenv("NECTAR_DECODE_CLUSTER", "1")
-    o1 = nx.decode(mods, *args)
-    l1 = nx.decode_layer_out(mods, *args)
     monkeypatch.setenv("NECTAR_DECODE_CLUSTER", "0")
     o0 = nx.decode(mods, *args)
-    torch.cuda.synchronize()
-    assert nx.device_error_flags(clear=True) == 0
-    assert torch.allclose(o1, o0, rtol=0, atol=1e-4 * max(1.0, o0.abs().max().item()))
-    assert torch.equal(l1, o1.permute(0, 3, 1, 2, 4).reshape(wl.L, wl.nq, wl.Hkv * wl.G, 128).to(torch.bfloat16))
+    for cluster in ("8", "16"):
+        monkeypatch.setenv("NECTAR_DECODE_CLUSTER", cluster)
+        o1 = nx.decode(mods, *args)
+        l1 = nx.decode_layer_out(mods, *args)
+        torch.cuda.synchronize()
+        assert nx.device_error_flags(clear=True) == 0
+        assert torch.allclose(o1, o0, rtol=0, atol=1e-4 * max(1.0, o0.abs().max().item())), cluster
+        assert torch.equal(l1, o1.permute(0, 3, 1, 2, 4).reshape(wl.L, wl.nq, wl.Hkv * wl.G, 128).to(torch.bfloat16))
 
 
 def test_decode_workspace_checked():
