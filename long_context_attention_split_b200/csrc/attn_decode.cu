@@ -27,9 +27,6 @@ constexpr int kDecWarps = 8;
 constexpr int kDecStages = 3;
 constexpr int kDecThreads = (kDecWarps + 1) * 32;
 
-__host__ __device__ __forceinline__ int first_cta_of_tile(int64_t t, int64_t total, int C) {
-  return static_cast<int>(((t + 1) * static_cast<int64_t>(C) - 1) / total);
-}
 
 // RW: query rows held by one warp (R rows in NRG groups of RW); TILE keys per tile.
 template <int RW, int TILE>

@@ -1,0 +1,437 @@
+// (i) Exact cached-token attention for 3-16 query rows per KV head, on the
+// tensor cores: Eq. (3.1) of "Nectar: Neural Estimation of Cached-Token
+// Attention via Regression" (§2.1), split over n and joined by log-sum-exp.
+//
+// At a few rows per head the CUDA-core split kernel spends ~10 instructions
+// per (key, row, dim) and is bound by the ALU, not by the K/V bytes.  Here
+// the products run on tcgen05, taken transposed so that the keys fill the
+// 128 rows of the tensor-core tile and the TMEM lanes:
+//   S^T = K Q^T   (M = 128 keys of a tile, N = QC = 16 >= rows, K = d; K and Q
+//                  K-major, 128-byte swizzle),
+//   O^T = V^T P^T (M = d, N = QC, K = the tile's keys; V read MN-major).
+// Each of the 128 softmax threads owns one key of a tile and holds its row
+// scores; the online softmax keeps one running maximum per row for the whole
+// CTA: a tile's maximum is reduced over the 128 threads, and the maximum
+// moves only when the tile's exceeds it by 2^8 (log2 units, as in the split
+// kernel), in which case the O^T column is rescaled in TMEM; that decision
+// is the same in every thread.  Each thread keeps its own partial sum of the
+// row weights; they are reduced at the end of a head's range.
+//
+// Schedule and output: the split kernel's.  All heads' 128-key tiles are laid
+// end to end and CTA c takes [c T / C, (c + 1) T / C) (two CTAs per SM, so
+// that one CTA's softmax latency hides under the other's); a CTA leaves one
+// partial (m, l, acc) per head it touched in the workspace, and the split
+// kernel's combine launch joins them.
+//
+// Warp roles: 0 TMA producer (K and V tiles, 32 KB each, into one ring in
+// the order the MMAs consume them: K0 K1 V0 K2 V1 ...; the head's Q rows
+// per head range), 1 MMA issuer (+ TMEM owner), 2-5 softmax and epilogue.
+// S^T and P are double-buffered per tile, Q and O^T per head range, so the
+// tile after next is scored while this one's weights are formed.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nectar {
+
+namespace {
+
+constexpr int kTKeys = kTctTile;                   // keys per tile (TMEM lanes of S^T)
+#ifndef NECTAR_TCT_STAGES
+#define NECTAR_TCT_STAGES (6 / NECTAR_TCT_CTAS_PER_SM)
+#endif
+constexpr int kTStages = NECTAR_TCT_STAGES;         // K / V tile ring
+constexpr uint32_t kTHalf = kTKeys * 128;          // 128 keys x 64 dims bf16: 16 KB
+constexpr uint32_t kTTile = 2 * kTHalf;
+constexpr int kTThreads = 6 * 32;
+
+template <int QC>
+struct TSmem {
+  static constexpr uint32_t kQHalf = QC * 128;                  // QC rows x 64 dims
+  static constexpr uint32_t kQ = 2 * kQHalf;
+  static constexpr uint32_t kPChunk = QC * 128;                 // QC rows x 64 keys
+  static constexpr uint32_t kP = 2 * kPChunk;                   // one tile of P
+  static constexpr uint32_t ring = 0;                           // [kTStages] K or V tiles
+  static constexpr uint32_t q = ring + kTStages * kTTile;       // [2 head ranges]
+  static constexpr uint32_t p = q + 2 * kQ;                     // [2 tiles]
+  static constexpr uint32_t red = p + 2 * kP;                   // float [2 tiles][4 warps][QC] maxima
+  static constexpr uint32_t reds = red + 2 * 4 * QC * 4;        // float [4 warps][QC] sums
+  static constexpr uint32_t bars = reds + 4 * QC * 4;
+  static constexpr uint32_t total = bars + 32 * 8;                 // 30 barriers, the TMEM slot
+};
+
+// byte offset of P[row][key] in one tile's P buffer (two K-major 64-key
+// chunks of QC rows, 128-byte swizzle)
+template <int QC>
+__device__ __forceinline__ uint32_t tp_off(int row, int key) {
+  return static_cast<uint32_t>(((key >> 6) & 1) * TSmem<QC>::kPChunk + row * 128 +
+                               ((((key & 63) >> 3) ^ (row & 7)) << 4) + ((key & 7) << 1));
+}
+
+// NV per-lane values reduced over the 32 lanes of a warp (max or sum):
+// halving steps (a lane keeps one half of its values and sends the other
+// half to its partner), then plain butterfly steps.  Lane L ends with value
+// L / (32 / NV) reduced over all lanes.
+template <int NV, bool kMax>
+__device__ __forceinline__ float twarp_reduce(float (&v)[NV], int lane) {
+  int n = NV;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    if (n > 1) {
+      const int half = n / 2;
+      const bool up = lane & off;
+#pragma unroll
+      for (int j = 0; j < half; ++j) {
+        const float lo = v[j], hi = v[j + half];
+        const float send = up ? lo : hi, keep = up ? hi : lo;
+        const float got = __shfl_xor_sync(0xffffffffu, send, off);
+        v[j] = kMax ? fmaxf(keep, got) : keep + got;
+      }
+      n = half;
+    } else {
+      const float got = __shfl_xor_sync(0xffffffffu, v[0], off);
+      v[0] = kMax ? fmaxf(v[0], got) : v[0] + got;
+    }
+  }
+  return v[0];
+}
+
+template <int QC>
+__device__ __forceinline__ void ttmem_ld(uint32_t taddr, uint32_t (&r)[QC]) {
+  static_assert(QC == 16, "16 columns");
+  NECTAR_TMEM_LD16(taddr, r);
+}
+template <int QC>
+__device__ __forceinline__ void ttmem_st(uint32_t taddr, const uint32_t (&r)[QC]) {
+  static_assert(QC == 16, "16 columns");
+  {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+  }
+}
+
+}  // namespace
+
+template <int QC>
+__global__ void __launch_bounds__(kTThreads, kTctCtasPerSm)
+cache_attn_tct_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                      const __grid_constant__ CUtensorMap tmap_v, const DecParams p) {
+  using SL = TSmem<QC>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (kTctCtasPerSm > 1 && smem != smem_raw) {
+    // two CTAs per SM request no alignment slack: refuse rather than overrun
+    if (threadIdx.x == 0) record_error(p.err, DEVERR_WAIT_TIMEOUT);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL::bars);
+  const uint32_t b_full = smem_u32(bars);               // [kTStages]
+  const uint32_t b_empty = smem_u32(bars + 8);          // [kTStages]
+  const uint32_t b_qfull = smem_u32(bars + 16);         // [2] per head range
+  const uint32_t b_qempty = smem_u32(bars + 18);        // [2]
+  const uint32_t b_sfull = smem_u32(bars + 20);         // [2] per tile
+  const uint32_t b_sfree = smem_u32(bars + 22);         // [2]
+  const uint32_t b_pfull = smem_u32(bars + 24);         // [2]
+  const uint32_t b_pfree = smem_u32(bars + 26);         // [2]
+  const uint32_t b_ofull = smem_u32(bars + 28);         // one phase per tile's O^T update
+  const uint32_t b_ofree = smem_u32(bars + 29);         // [2] per head range
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 31);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x;
+  const int64_t t0 = static_cast<int64_t>(c) * p.total / p.C;
+  const int64_t t1 = static_cast<int64_t>(c + 1) * p.total / p.C;
+  const int ntiles = static_cast<int>(t1 - t0);
+  const int64_t hd0 = t0 / p.tph;
+  const int R = static_cast<int>(p.rows_total);
+  constexpr uint32_t kTmemCols = 4 * QC < 32 ? 32 : 4 * QC;   // S^T [2][QC], O^T [2][QC]
+  const uint32_t kOCol = 2 * QC;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTStages; ++s) {
+      mbar_init(b_full + 8 * s, 1);
+      mbar_init(b_empty + 8 * s, 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(b_qfull + 8 * x, 1);
+      mbar_init(b_qempty + 8 * x, 1);
+      mbar_init(b_sfull + 8 * x, 1);
+      mbar_init(b_sfree + 8 * x, 128);
+      mbar_init(b_pfull + 8 * x, 128);
+      mbar_init(b_pfree + 8 * x, 1);
+      mbar_init(b_ofree + 8 * x, 128);
+    }
+    mbar_init(b_ofull, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tslot), kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp >= 2) {
+    // Q rows past the R that TMA writes stay 0 (their S^T and O^T columns are unused)
+    for (int x = threadIdx.x - 64; x < 2 * 2 * (QC - R) * 8; x += 128) {
+      const int buf = x / (2 * (QC - R) * 8), rem = x % (2 * (QC - R) * 8);
+      const int half = rem / ((QC - R) * 8), rr = rem % ((QC - R) * 8);
+      reinterpret_cast<uint4*>(smem + SL::q + buf * SL::kQ + half * SL::kQHalf + R * 128)[rr] = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  griddep_wait();                 // inputs and outputs only from here on (launched after another kernel)
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      prefetch_tmap(&tmap_q);
+      prefetch_tmap(&tmap_k);
+      prefetch_tmap(&tmap_v);
+      const uint64_t pol = policy_evict_first();
+      uint32_t it = 0;
+      bool ok = true;
+      auto load_tile = [&](const CUtensorMap* map, int64_t t) {
+        const uint32_t s = it % kTStages;
+        if (it >= kTStages) ok = mbar_wait(b_empty + 8 * s, ((it / kTStages) - 1) & 1, p.err);
+        if (!ok) return;
+        const int64_t hd = t / p.tph, kt = t % p.tph;
+        mbar_arrive_expect_tx(b_full + 8 * s, kTTile);
+        tma_load_4d(smem_u32(smem + SL::ring + s * kTTile), map, 0, static_cast<int>(kt * kTKeys), 0,
+                    static_cast<int>(hd), b_full + 8 * s, pol);
+        ++it;
+      };
+      for (int i = 0; i <= ntiles && ok; ++i) {
+        if (i < ntiles) {
+          const int64_t t = t0 + i;
+          const int64_t hd = t / p.tph;
+          if (i == 0 || t % p.tph == 0) {
+            // this head's query rows, one box per 64-column half
+            const int seg = static_cast<int>(hd - hd0);
+            const uint32_t qb = seg & 1;
+            if (seg >= 2 && !(ok = mbar_wait(b_qempty + 8 * qb, ((seg >> 1) - 1) & 1, p.err))) break;
+            mbar_arrive_expect_tx(b_qfull + 8 * qb, static_cast<uint32_t>(2 * R * 128));
+            const uint32_t qd = smem_u32(smem + SL::q + qb * SL::kQ);
+            tma_load_4d(qd, &tmap_q, 0, 0, 0, static_cast<int>(hd), b_qfull + 8 * qb, pol);
+            tma_load_4d(qd + SL::kQHalf, &tmap_q, 0, 0, 1, static_cast<int>(hd), b_qfull + 8 * qb, pol);
+          }
+          load_tile(&tmap_k, t);
+        }
+        if (i >= 1) load_tile(&tmap_v, t0 + i - 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, QC, 0, 0);   // A = K tile, B = Q
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, QC, 1, 0);   // A = V tile (MN-major), B = P
+      bool ok = true;
+      uint32_t it = 0;
+      for (int i = 0; i <= ntiles && ok; ++i) {
+        if (i < ntiles) {
+          // S^T of tile i
+          const int64_t t = t0 + i;
+          const int seg = static_cast<int>(t / p.tph - hd0);
+          const uint32_t qb = seg & 1, sb = i & 1;
+          if ((i == 0 || t % p.tph == 0) && !(ok = mbar_wait(b_qfull + 8 * qb, (seg >> 1) & 1, p.err))) break;
+          if (i >= 2 && !(ok = mbar_wait(b_sfree + 8 * sb, ((i >> 1) - 1) & 1, p.err))) break;
+          const uint32_t s = it % kTStages;
+          if (!(ok = mbar_wait(b_full + 8 * s, (it / kTStages) & 1, p.err))) break;
+          tc_fence_after();
+          const uint32_t ka = smem_u32(smem + SL::ring + s * kTTile);
+          const uint32_t qa = smem_u32(smem + SL::q + qb * SL::kQ);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ss(tmem + sb * QC, sdesc_sw128(ka + (kk >> 2) * kTHalf + (kk & 3) * 32, 16, 1024),
+                        sdesc_sw128(qa + (kk >> 2) * SL::kQHalf + (kk & 3) * 32, 16, 1024), idesc_s, kk != 0);
+          mma_commit(b_empty + 8 * s);
+          ++it;
+          mma_commit(b_sfull + 8 * sb);
+          if (i == ntiles - 1 || (t + 1) % p.tph == 0) mma_commit(b_qempty + 8 * qb);
+        }
+        if (i >= 1) {
+          // O^T += V^T P^T of tile j = i - 1, once its weights are in P
+          const int j = i - 1;
+          const int64_t t = t0 + j;
+          const int seg = static_cast<int>(t / p.tph - hd0);
+          const bool first = (j == 0 || t % p.tph == 0);
+          const uint32_t pb = j & 1;
+          if (!(ok = mbar_wait(b_pfull + 8 * pb, (j >> 1) & 1, p.err))) break;
+          if (first && seg >= 2 && !(ok = mbar_wait(b_ofree + 8 * (seg & 1), ((seg >> 1) - 1) & 1, p.err))) break;
+          const uint32_t s = it % kTStages;
+          if (!(ok = mbar_wait(b_full + 8 * s, (it / kTStages) & 1, p.err))) break;
+          tc_fence_after();
+          const uint32_t va = smem_u32(smem + SL::ring + s * kTTile);
+          const uint32_t pa = smem_u32(smem + SL::p + pb * SL::kP);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ss(tmem + kOCol + (seg & 1) * QC, sdesc_sw128(va + kk * 2048, kTHalf, 1024),
+                        sdesc_sw128(pa + (kk >> 2) * SL::kPChunk + (kk & 3) * 32, 16, 1024), idesc_o,
+                        (!first || kk != 0) ? 1u : 0u);
+          mma_commit(b_empty + 8 * s);
+          ++it;
+          mma_commit(b_pfree + 8 * pb);
+          mma_commit(b_ofull);
+        }
+      }
+    }
+  } else {
+    // --------------------- softmax + epilogue (128 threads) ---------------------
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;                // key of a tile (S^T) / dim (O^T)
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    constexpr int kLanesPer = 32 / QC;                // lanes holding one reduced value
+    float* red = reinterpret_cast<float*>(smem + SL::red);
+    float* reds = reinterpret_cast<float*>(smem + SL::reds);
+    bool ok = true;
+    float M[QC], lp[QC];
+    for (int i = 0; i < ntiles; ++i) {
+      const int64_t t = t0 + i;
+      const int64_t hd = t / p.tph, kt = t % p.tph;
+      const int seg = static_cast<int>(hd - hd0);
+      const bool first = (i == 0 || kt == 0);
+      const bool last = (i == ntiles - 1 || (t + 1) % p.tph == 0);
+      const uint32_t sb = i & 1;
+      if (first) {
+#pragma unroll
+        for (int q = 0; q < QC; ++q) {
+          M[q] = -INFINITY;
+          lp[q] = 0.f;
+        }
+      }
+      if (ok) ok = mbar_wait(b_sfull + 8 * sb, (i >> 1) & 1, p.err);
+      tc_fence_after();
+      float s[QC];
+      {
+        uint32_t v[QC];
+        ttmem_ld<QC>(tmem + sb * QC + lane_base, v);
+        tmem_ld_wait();
+        const bool valid = kt * kTKeys + r < p.n;
+#pragma unroll
+        for (int q = 0; q < QC; ++q) s[q] = (valid && q < R) ? __uint_as_float(v[q]) * p.qmul : -INFINITY;
+      }
+      tc_fence_before();
+      mbar_arrive(b_sfree + 8 * sb);
+      // the tile's maximum per row over its 128 keys
+      {
+        float mx[QC];
+#pragma unroll
+        for (int q = 0; q < QC; ++q) mx[q] = s[q];
+        const float w = twarp_reduce<QC, true>(mx, lane);
+        if (lane % kLanesPer == 0) red[(sb * 4 + quarter) * QC + lane / kLanesPer] = w;
+      }
+      named_bar_sync(1, 128);
+      float corr[QC];
+      bool need = false;
+#pragma unroll
+      for (int q = 0; q < QC; ++q) {
+        const float* rq = red + sb * 4 * QC + q;
+        const float mt = fmaxf(fmaxf(rq[0], rq[QC]), fmaxf(rq[2 * QC], rq[3 * QC]));
+        corr[q] = 1.f;
+        if (mt > M[q] + kRescaleSlack) {             // also the head's first finite maximum
+          corr[q] = exp2_shift(M[q], mt);
+          M[q] = mt;
+          need = true;
+        }
+        lp[q] *= corr[q];
+      }
+      if (need && !first) {
+        // the running O^T holds the tiles up to i - 1: rescale its columns
+        if (ok) ok = mbar_wait(b_ofull, (i - 1) & 1, p.err);
+        tc_fence_after();
+        uint32_t o[QC];
+        const uint32_t oaddr = tmem + kOCol + (seg & 1) * QC + lane_base;
+        ttmem_ld<QC>(oaddr, o);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < QC; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * corr[q]);
+        ttmem_st<QC>(oaddr, o);
+        tmem_st_wait();
+      }
+      // the weights, bf16 into P (row, key): what the P V product and the
+      // row sums both use
+      if (i >= 2 && ok) ok = mbar_wait(b_pfree + 8 * sb, ((i >> 1) - 1) & 1, p.err);
+      uint8_t* pt = smem + SL::p + sb * SL::kP;
+#pragma unroll
+      for (int q = 0; q < QC; ++q) {
+        const __nv_bfloat16 w = __float2bfloat16_rn(exp2_shift(s[q], M[q]));
+        lp[q] += __bfloat162float(w);
+        *reinterpret_cast<__nv_bfloat16*>(pt + tp_off<QC>(q, r)) = w;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(b_pfull + 8 * sb);
+      if (last) {
+        // the head's partial: O^T (this thread: dim r), the row sums, M.
+        // ofull completes one phase per tile's O^T update, in order, and a
+        // parity wait only tells the current phase from the one before: so
+        // O(i - 1) first (it was issued after S(i), and may still be running
+        // -- a wait for phase i alone would pass on phase i - 1's parity),
+        // then O(i).  (The rescale's wait for O(i - 1) needs no such step:
+        // S(i), complete by then, was issued after O(i - 2).)
+        if (ok && i >= 1) ok = mbar_wait(b_ofull, (i - 1) & 1, p.err);
+        if (ok) ok = mbar_wait(b_ofull, i & 1, p.err);
+        tc_fence_after();
+        uint32_t o[QC];
+        ttmem_ld<QC>(tmem + kOCol + (seg & 1) * QC + lane_base, o);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(b_ofree + 8 * (seg & 1));
+        float ls[QC];
+#pragma unroll
+        for (int q = 0; q < QC; ++q) ls[q] = lp[q];
+        const float w = twarp_reduce<QC, false>(ls, lane);
+        if (lane % kLanesPer == 0) reds[quarter * QC + lane / kLanesPer] = w;
+        named_bar_sync(2, 128);
+        const int slot = c - first_cta_of_tile(hd * p.tph, p.total, p.C);
+        if (ok) {
+#pragma unroll
+          for (int q = 0; q < QC; ++q) {
+            if (q < R) {
+              const int64_t prow = (hd * p.S_max + slot) * p.rows_total + q;
+              p.ws_acc[prow * kD + r] = __uint_as_float(o[q]);
+              if (r == 0) {
+                p.ws_ml[prow * 2] = M[q];
+                p.ws_ml[prow * 2 + 1] = (reds[q] + reds[QC + q]) + (reds[2 * QC + q] + reds[3 * QC + q]);
+              }
+            }
+          }
+        }
+        named_bar_sync(2, 128);                     // the sums are read before the next head's
+      }
+    }
+  }
+  griddep_launch();                 // the combine may start launching
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// N = 16 query columns whatever the rows (3..16): a kind::f16 MMA with
+// M = 128 takes N in multiples of 16, so narrower S^T / O^T tiles are not
+// an option.
+size_t cache_attn_tct_smem(int rows) {
+  (void)rows;
+  return TSmem<16>::total + (kTctCtasPerSm > 1 ? 0 : 1024);
+}
+
+cudaError_t launch_cache_attn_tct(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                  const DecParams& p, cudaStream_t stream) {
+  const size_t smem = cache_attn_tct_smem(static_cast<int>(p.rows_total));
+  cudaError_t e = cudaFuncSetAttribute(cache_attn_tct_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_k(cache_attn_tct_kernel<16>, dim3(p.C), dim3(kTThreads), smem, stream, 1, tq, tk, tv, p);
+}
+
+}  // namespace nectar

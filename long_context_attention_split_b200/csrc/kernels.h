@@ -84,13 +84,38 @@ struct DecPlan {
 // 0.683 ms on a 28 x 8-head, 32768-key, 2-row document), 64 above (at 4
 // rows the 64-key tiles with two CTAs per SM measured 1 % faster; from 5
 // rows the row state needs the registers of a smaller tile).
-__host__ __device__ constexpr int dec_tile(int R) { return R <= 2 ? 128 : 64; }
+#ifndef NECTAR_SPLIT_TILE_R4
+#define NECTAR_SPLIT_TILE_R4 64
+#endif
+__host__ __device__ constexpr int dec_tile(int R) { return R <= 2 ? 128 : (R <= 4 ? NECTAR_SPLIT_TILE_R4 : 64); }
 DecPlan plan_decode(int heads, int64_t n, int num_sms, int ctas_per_sm, int tile);
+// The CTA of a stream-K split whose range [c*total/C, (c+1)*total/C) holds
+// tile t: a head's partial slot s is written by CTA first_cta_of_tile(its
+// first tile) + s.
+__host__ __device__ __forceinline__ int first_cta_of_tile(int64_t t, int64_t total, int C) {
+  return static_cast<int>(((t + 1) * static_cast<int64_t>(C) - 1) / total);
+}
 int dec_max_rows();
 int dec_ctas_per_sm(int R);
 size_t dec_smem_for_rows(int R);
 cudaError_t launch_cache_attn_split(const DecParams& p, int R, cudaStream_t stream);
 cudaError_t launch_cache_attn_combine(const DecParams& p, float* alpha, float* A, cudaStream_t stream);
+
+// ----- (i) 3-16 query rows per head: transposed tensor-core split ---------
+// Same stream-K plan (128-key tiles), partial layout and combine as the
+// split kernel.
+constexpr int kTctTile = 128;
+constexpr int kTctMaxRows = 16;
+// Resident CTAs per SM (each with a ring of 6 / this K or V stages): two
+// measured 1.29 ms against 1.72 for one on a 32 x 8-head, 65536-key
+// document at 4 rows (6.67 against 5.00 TB/s).
+#ifndef NECTAR_TCT_CTAS_PER_SM
+#define NECTAR_TCT_CTAS_PER_SM 2
+#endif
+constexpr int kTctCtasPerSm = NECTAR_TCT_CTAS_PER_SM;
+size_t cache_attn_tct_smem(int rows);
+cudaError_t launch_cache_attn_tct(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                  const DecParams& p, cudaStream_t stream);
 
 // ----- (i) tensor-core path for many query rows per head -------------------
 struct TcParams {

@@ -135,8 +135,18 @@ DeviceInfo device_info() {
 #ifndef NECTAR_TC_ROUTE_ROWS
 #define NECTAR_TC_ROUTE_ROWS 8
 #endif
-// More query rows per KV head than that: the tensor-core kernel.
+// 3 to 16 query rows per KV head: the transposed tensor-core split kernel
+// (attn_tct.cu), where the CUDA-core split kernel is bound by its ALU work
+// (measured on a Llama-8B-shaped document at 4 rows: the CUDA-core kernel
+// reaches 68 % of the HBM copy bandwidth).  NECTAR_TCT=0
+// keeps those rows on the CUDA-core kernel (up to NECTAR_TC_ROUTE_ROWS).
+bool use_tct_attn(int64_t rows) {
+  const char* e = getenv("NECTAR_TCT");
+  return !(e != nullptr && e[0] == '0') && rows >= 3 && rows <= kTctMaxRows;
+}
+// More query rows per KV head than those: the tensor-core kernel.
 bool use_tc_attn(int64_t rows) {
+  if (use_tct_attn(rows)) return false;
   const int64_t lim = NECTAR_TC_ROUTE_ROWS < dec_max_rows() ? NECTAR_TC_ROUTE_ROWS : dec_max_rows();
   return rows > lim;
 }
@@ -145,6 +155,7 @@ int dec_row_block(int64_t rows) { return rows < dec_max_rows() ? static_cast<int
 
 DecPlan cache_attn_plan(const nectar_dims& d, int64_t n, int64_t nq, int sms) {
   const int64_t rows = static_cast<int64_t>(d.G) * nq;
+  if (use_tct_attn(rows)) return plan_decode(d.L * d.Hkv, n, sms, kTctCtasPerSm, kTctTile);
   const int R = dec_row_block(rows);
   return plan_decode(d.L * d.Hkv, n, sms, dec_ctas_per_sm(R < 1 ? 1 : R), dec_tile(R < 1 ? 1 : R));
 }
@@ -340,6 +351,24 @@ nectar_status nectar_cache_attn_lse(nectar_dims dims, const nectar_bf16* K, cons
   const int64_t prow = static_cast<int64_t>(heads) * pl.S_max * rows;
   p.ws_acc = reinterpret_cast<float*>(workspace);
   p.ws_ml = p.ws_acc + prow * kD;
+  if (use_tct_attn(rows)) {
+    // K, V as [heads][2 halves of d][n][64]: one box = 128 keys, both halves;
+    // Q as [heads][2 halves][rows][64]: one box per half
+    CUtensorMap tq, tk, tv;
+    const cuuint64_t dq[4] = {64, static_cast<cuuint64_t>(rows), 2, static_cast<cuuint64_t>(heads)};
+    const cuuint64_t sq[3] = {256, 128, static_cast<cuuint64_t>(rows) * 256};
+    const cuuint64_t dk[4] = {64, static_cast<cuuint64_t>(n), 2, static_cast<cuuint64_t>(heads)};
+    const cuuint64_t sk[3] = {256, 128, static_cast<cuuint64_t>(n) * 256};
+    const cuuint32_t boxq[4] = {64, static_cast<cuuint32_t>(rows), 1, 1};
+    const cuuint32_t boxk[4] = {64, static_cast<cuuint32_t>(kTctTile), 2, 1};
+    NECTAR_TRY(make_tmap(&tq, Q, 4, dq, sq, boxq, "Q"));
+    NECTAR_TRY(make_tmap(&tk, K, 4, dk, sk, boxk, "K"));
+    NECTAR_TRY(make_tmap(&tv, V, 4, dk, sk, boxk, "V"));
+    cudaError_t e = launch_cache_attn_tct(tq, tk, tv, p, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cache_attn transposed tensor-core kernel");
+    e = launch_cache_attn_combine(p, alpha, A, st);
+    return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "cache_attn combine kernel");
+  }
 
   const int RB = dec_row_block(rows);
   for (int64_t r0 = 0; r0 < rows; r0 += RB) {

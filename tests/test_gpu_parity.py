@@ -82,6 +82,66 @@ def test_cache_attn_parity(L, Hkv, G, n, nq):
     check_attn(ag, Ag, ao, Ao, wl.V.float().abs().max().item(), f"n={n}")
 
 
+# 3-16 query rows per KV head: the transposed tensor-core split kernel
+# (keys on the TMEM lanes).  Cases: a ragged single tile, many short heads per
+# CTA range (each CTA crosses 4 heads: the double-buffered Q and O^T are
+# reused), a head cut over several CTAs, 16 rows, and the same shapes on the
+# CUDA-core kernel (NECTAR_TCT=0) for comparison.
+@pytest.mark.parametrize("L,Hkv,G,n,nq", [
+    (1, 2, 3, 100, 1),        # 3 rows, n < one 128-key tile
+    (30, 20, 4, 100, 1),      # 600 one-tile heads: ~4 head ranges per CTA
+    (2, 4, 5, 20000, 1),      # 5 rows, each head cut over ~18 CTAs
+    (1, 3, 8, 1537, 2),       # 16 rows, ragged tail of 1 key
+    (2, 2, 2, 5000, 6),       # 12 rows (QC = 16)
+])
+def test_cache_attn_tct(L, Hkv, G, n, nq, monkeypatch):
+    wl, ag, Ag, ao, Ao = run_cache_attn(L, Hkv, G, n, nq, seed=n + 7 * G)
+    vmax = wl.V.float().abs().max().item()
+    check_attn(ag, Ag, ao, Ao, vmax, f"tct n={n}")
+    if G * nq <= 8:
+        monkeypatch.setenv("NECTAR_TCT", "0")
+        _, ag0, Ag0, _, _ = run_cache_attn(L, Hkv, G, n, nq, seed=n + 7 * G)
+        check_attn(ag0, Ag0, ao, Ao, vmax, f"split n={n}")
+        assert np.abs(ag - ag0).max() <= ALPHA_TOL and np.abs(Ag - Ag0).max() <= ATT_TOL * vmax
+
+
+def test_cache_attn_tct_repeatable():
+    # a head spread over several CTAs with several tiles each: ten calls give
+    # the same bits (the partials are summed in a fixed order; a call that
+    # read a head's O^T before its last tiles had landed would not)
+    wl = make_workload("toy", L=2, Hkv=4, G=5, n=20000, nq=1, T=1, with_local=False, with_modules=False, seed=3)
+    K, V, Q = wl.K.cuda(), wl.V.cuda(), wl.Q.cuda()
+    a0, A0 = nx.cache_attn_lse(K, V, Q)
+    for _ in range(9):
+        a1, A1 = nx.cache_attn_lse(K, V, Q)
+        torch.cuda.synchronize()
+        assert torch.equal(a1, a0) and torch.equal(A1, A0)
+    ao, Ao = oracle.cache_attn(wl.K, wl.V, wl.Q.reshape(2, 4, 5, 128), wl.scale)
+    check_attn(a0.cpu().numpy().reshape(ao.shape), A0.cpu().numpy().reshape(Ao.shape), ao, Ao,
+               wl.V.float().abs().max().item(), "tct repeat")
+
+
+def test_cache_attn_tct_running_max_moves():
+    # 4 rows: after 40 tiles of ordinary scores a key scores ~ +10 (natural
+    # log units) higher for two of the rows, so the running maximum of those
+    # rows moves past the 2^8 slack and their O^T columns are rescaled in TMEM
+    L, Hkv, G, nq, n = 1, 2, 4, 1, 9000
+    g = torch.Generator().manual_seed(21)
+    K = torch.randn(L, Hkv, n, 128, generator=g)
+    V = torch.randn(L, Hkv, n, 128, generator=g)
+    Q = torch.randn(L, Hkv, G, nq, 128, generator=g)
+    u = Q[0, 1, 1, 0] / Q[0, 1, 1, 0].norm()
+    K[0, 1, 5123] = 40.0 * u
+    w = Q[0, 0, 3, 0] / Q[0, 0, 3, 0].norm()
+    K[0, 0, 8999] = 45.0 * w             # the very last key of a head
+    K, V, Q = K.to(torch.bfloat16), V.to(torch.bfloat16), Q.to(torch.bfloat16)
+    alpha, A = nx.cache_attn_lse(cuda(K), cuda(V), cuda(Q))
+    torch.cuda.synchronize()
+    ao, Ao = oracle.cache_attn(K, V, Q.reshape(L, Hkv, G * nq, 128), 1 / math.sqrt(128))
+    check_attn(alpha.cpu().numpy().reshape(ao.shape), A.cpu().numpy().reshape(Ao.shape), ao, Ao,
+               V.float().abs().max().item(), "tct rescale")
+
+
 def test_cache_attn_key_scale_and_heavy_hitters():
     wl, ag, Ag, ao, Ao = run_cache_attn(2, 2, 2, 3000, 2, seed=5, key_scale=(0.5, 2.0))
     check_attn(ag, Ag, ao, Ao, wl.V.float().abs().max().item())
