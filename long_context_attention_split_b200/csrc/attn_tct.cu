@@ -1,4 +1,4 @@
-// (i) Exact cached-token attention for 3-16 query rows per KV head, on the
+// (i) Exact cached-token attention for 3-32 query rows per KV head, on the
 // tensor cores: Eq. (3.1) of "Nectar: Neural Estimation of Cached-Token
 // Attention via Regression" (§2.1), split over n and joined by log-sum-exp.
 //
@@ -25,7 +25,8 @@
 //
 // Warp roles: 0 TMA producer (K and V tiles, 32 KB each, into one ring in
 // the order the MMAs consume them: K0 K1 V0 K2 V1 ...; the head's Q rows
-// per head range), 1 MMA issuer (+ TMEM owner), 2-5 softmax and epilogue.
+// per head range), 1 MMA issuer (+ TMEM owner), then one softmax and
+// epilogue warpgroup per 16 query columns (each thread: one key, 16 rows).
 // S^T and P are double-buffered per tile, Q and O^T per head range, so the
 // tile after next is scored while this one's weights are formed.
 #include <cuda.h>
@@ -42,10 +43,19 @@ constexpr int kTKeys = kTctTile;                   // keys per tile (TMEM lanes 
 #ifndef NECTAR_TCT_STAGES
 #define NECTAR_TCT_STAGES (6 / NECTAR_TCT_CTAS_PER_SM)
 #endif
-constexpr int kTStages = NECTAR_TCT_STAGES;         // K / V tile ring
+// Per query-column count QC: resident CTAs per SM and K / V ring stages.
+// 16 columns: two CTAs of NECTAR_TCT_STAGES stages; 32 and 64 columns (Q,
+// P and the row state grow with QC): one CTA, with the stages that fit.
+template <int QC>
+struct TCfg {
+  static constexpr int wgs = QC / 16;                     // softmax warpgroups
+  static constexpr int threads = 64 + 128 * wgs;
+  static constexpr int ctas = QC == 16 ? kTctCtasPerSm : 1;
+  static constexpr int stages = QC == 16 ? NECTAR_TCT_STAGES : (QC == 32 ? 6 : 4);
+};
 constexpr uint32_t kTHalf = kTKeys * 128;          // 128 keys x 64 dims bf16: 16 KB
 constexpr uint32_t kTTile = 2 * kTHalf;
-constexpr int kTThreads = 6 * 32;
+// one softmax warpgroup (128 threads) per 16 query columns
 
 template <int QC>
 struct TSmem {
@@ -53,13 +63,15 @@ struct TSmem {
   static constexpr uint32_t kQ = 2 * kQHalf;
   static constexpr uint32_t kPChunk = QC * 128;                 // QC rows x 64 keys
   static constexpr uint32_t kP = 2 * kPChunk;                   // one tile of P
-  static constexpr uint32_t ring = 0;                           // [kTStages] K or V tiles
-  static constexpr uint32_t q = ring + kTStages * kTTile;       // [2 head ranges]
+  static constexpr uint32_t ring = 0;                           // [stages] K or V tiles
+  static constexpr uint32_t q = ring + TCfg<QC>::stages * kTTile;   // [2 head ranges]
   static constexpr uint32_t p = q + 2 * kQ;                     // [2 tiles]
   static constexpr uint32_t red = p + 2 * kP;                   // float [2 tiles][4 warps][QC] maxima
   static constexpr uint32_t reds = red + 2 * 4 * QC * 4;        // float [4 warps][QC] sums
-  static constexpr uint32_t bars = reds + 4 * QC * 4;
-  static constexpr uint32_t total = bars + 32 * 8;                 // 30 barriers, the TMEM slot
+  static constexpr uint32_t corrs = reds + 4 * QC * 4;          // float [QC] a tile's rescale factors
+  static constexpr uint32_t bars = corrs + QC * 4;
+  // 2 x stages ring barriers, 15 more, the TMEM slot (8 bytes each)
+  static constexpr uint32_t total = bars + (2 * TCfg<QC>::stages + 16) * 8;
 };
 
 // byte offset of P[row][key] in one tile's P buffer (two K-major 64-key
@@ -98,50 +110,44 @@ __device__ __forceinline__ float twarp_reduce(float (&v)[NV], int lane) {
   return v[0];
 }
 
-template <int QC>
-__device__ __forceinline__ void ttmem_ld(uint32_t taddr, uint32_t (&r)[QC]) {
-  static_assert(QC == 16, "16 columns");
-  NECTAR_TMEM_LD16(taddr, r);
-}
-template <int QC>
-__device__ __forceinline__ void ttmem_st(uint32_t taddr, const uint32_t (&r)[QC]) {
-  static_assert(QC == 16, "16 columns");
-  {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-            taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-  }
+// 16 columns of 32 lanes of TMEM <-> registers (warp-collective)
+__device__ __forceinline__ void ttmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
 }
 
 }  // namespace
 
 template <int QC>
-__global__ void __launch_bounds__(kTThreads, kTctCtasPerSm)
+__global__ void __launch_bounds__(TCfg<QC>::threads, TCfg<QC>::ctas)
 cache_attn_tct_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const DecParams p) {
   using SL = TSmem<QC>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  if (kTctCtasPerSm > 1 && smem != smem_raw) {
+  if (TCfg<QC>::ctas > 1 && smem != smem_raw) {
     // two CTAs per SM request no alignment slack: refuse rather than overrun
     if (threadIdx.x == 0) record_error(p.err, DEVERR_WAIT_TIMEOUT);
     return;
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL::bars);
-  const uint32_t b_full = smem_u32(bars);               // [kTStages]
-  const uint32_t b_empty = smem_u32(bars + 8);          // [kTStages]
-  const uint32_t b_qfull = smem_u32(bars + 16);         // [2] per head range
-  const uint32_t b_qempty = smem_u32(bars + 18);        // [2]
-  const uint32_t b_sfull = smem_u32(bars + 20);         // [2] per tile
-  const uint32_t b_sfree = smem_u32(bars + 22);         // [2]
-  const uint32_t b_pfull = smem_u32(bars + 24);         // [2]
-  const uint32_t b_pfree = smem_u32(bars + 26);         // [2]
-  const uint32_t b_ofull = smem_u32(bars + 28);         // one phase per tile's O^T update
-  const uint32_t b_ofree = smem_u32(bars + 29);         // [2] per head range
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 31);
+  constexpr int kTStages = TCfg<QC>::stages;
+  const uint32_t b_full = smem_u32(bars);                    // [kTStages]
+  const uint32_t b_empty = smem_u32(bars + kTStages);        // [kTStages]
+  uint64_t* const bx = bars + 2 * kTStages;
+  const uint32_t b_qfull = smem_u32(bx + 0);         // [2] per head range
+  const uint32_t b_qempty = smem_u32(bx + 2);        // [2]
+  const uint32_t b_sfull = smem_u32(bx + 4);         // [2] per tile
+  const uint32_t b_sfree = smem_u32(bx + 6);         // [2]
+  const uint32_t b_pfull = smem_u32(bx + 8);         // [2]
+  const uint32_t b_pfree = smem_u32(bx + 10);        // [2]
+  const uint32_t b_ofull = smem_u32(bx + 12);        // one phase per tile's O^T update
+  const uint32_t b_ofree = smem_u32(bx + 13);        // [2] per head range
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bx + 15);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x;
   const int64_t t0 = static_cast<int64_t>(c) * p.total / p.C;
@@ -150,6 +156,9 @@ cache_attn_tct_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
   const int64_t hd0 = t0 / p.tph;
   const int R = static_cast<int>(p.rows_total);
   constexpr uint32_t kTmemCols = 4 * QC < 32 ? 32 : 4 * QC;   // S^T [2][QC], O^T [2][QC]
+  constexpr int kWG = TCfg<QC>::wgs;
+  constexpr int kThreadsAll = TCfg<QC>::threads;
+  static_assert(QC % 16 == 0 && QC <= 64, "16, 32 or 64 query columns");
   const uint32_t kOCol = 2 * QC;
 
   if (threadIdx.x == 0) {
@@ -161,10 +170,10 @@ cache_attn_tct_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
       mbar_init(b_qfull + 8 * x, 1);
       mbar_init(b_qempty + 8 * x, 1);
       mbar_init(b_sfull + 8 * x, 1);
-      mbar_init(b_sfree + 8 * x, 128);
-      mbar_init(b_pfull + 8 * x, 128);
+      mbar_init(b_sfree + 8 * x, 128 * kWG);
+      mbar_init(b_pfull + 8 * x, 128 * kWG);
       mbar_init(b_pfree + 8 * x, 1);
-      mbar_init(b_ofree + 8 * x, 128);
+      mbar_init(b_ofree + 8 * x, 128 * kWG);
     }
     mbar_init(b_ofull, 1);
     fence_barrier_init();
@@ -175,7 +184,7 @@ cache_attn_tct_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
   }
   if (warp >= 2) {
     // Q rows past the R that TMA writes stay 0 (their S^T and O^T columns are unused)
-    for (int x = threadIdx.x - 64; x < 2 * 2 * (QC - R) * 8; x += 128) {
+    for (int x = threadIdx.x - 64; x < 2 * 2 * (QC - R) * 8; x += kThreadsAll - 64) {
       const int buf = x / (2 * (QC - R) * 8), rem = x % (2 * (QC - R) * 8);
       const int half = rem / ((QC - R) * 8), rr = rem % ((QC - R) * 8);
       reinterpret_cast<uint4*>(smem + SL::q + buf * SL::kQ + half * SL::kQHalf + R * 128)[rr] = make_uint4(0, 0, 0, 0);
@@ -282,15 +291,18 @@ cache_attn_tct_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
       }
     }
   } else {
-    // --------------------- softmax + epilogue (128 threads) ---------------------
+    // ------------- softmax + epilogue (one warpgroup per 16 columns) -------------
+    const int wg = (warp - 2) >> 2;                  // softmax warpgroup: columns [16 wg, 16 wg + 16)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                // key of a tile (S^T) / dim (O^T)
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    constexpr int kLanesPer = 32 / QC;                // lanes holding one reduced value
+    constexpr int CH = 16;
+    const int cb = wg * CH;
     float* red = reinterpret_cast<float*>(smem + SL::red);
     float* reds = reinterpret_cast<float*>(smem + SL::reds);
+    float* corrs = reinterpret_cast<float*>(smem + SL::corrs);
     bool ok = true;
-    float M[QC], lp[QC];
+    float M[CH], lp[CH];
     for (int i = 0; i < ntiles; ++i) {
       const int64_t t = t0 + i;
       const int64_t hd = t / p.tph, kt = t % p.tph;
@@ -300,72 +312,76 @@ cache_attn_tct_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
       const uint32_t sb = i & 1;
       if (first) {
 #pragma unroll
-        for (int q = 0; q < QC; ++q) {
-          M[q] = -INFINITY;
-          lp[q] = 0.f;
+        for (int j = 0; j < CH; ++j) {
+          M[j] = -INFINITY;
+          lp[j] = 0.f;
         }
       }
       if (ok) ok = mbar_wait(b_sfull + 8 * sb, (i >> 1) & 1, p.err);
       tc_fence_after();
-      float s[QC];
+      const bool valid = kt * kTKeys + r < p.n;
+      // pass 1: the tile's maximum per row over its 128 keys
       {
-        uint32_t v[QC];
-        ttmem_ld<QC>(tmem + sb * QC + lane_base, v);
+        uint32_t v[CH];
+        NECTAR_TMEM_LD16(tmem + sb * QC + cb + lane_base, v);
         tmem_ld_wait();
-        const bool valid = kt * kTKeys + r < p.n;
+        float mx[CH];
 #pragma unroll
-        for (int q = 0; q < QC; ++q) s[q] = (valid && q < R) ? __uint_as_float(v[q]) * p.qmul : -INFINITY;
+        for (int j = 0; j < CH; ++j) mx[j] = (valid && cb + j < R) ? __uint_as_float(v[j]) * p.qmul : -INFINITY;
+        const float w = twarp_reduce<CH, true>(mx, lane);
+        if ((lane & 1) == 0) red[(sb * 4 + quarter) * QC + cb + (lane >> 1)] = w;
       }
-      tc_fence_before();
-      mbar_arrive(b_sfree + 8 * sb);
-      // the tile's maximum per row over its 128 keys
-      {
-        float mx[QC];
-#pragma unroll
-        for (int q = 0; q < QC; ++q) mx[q] = s[q];
-        const float w = twarp_reduce<QC, true>(mx, lane);
-        if (lane % kLanesPer == 0) red[(sb * 4 + quarter) * QC + lane / kLanesPer] = w;
-      }
-      named_bar_sync(1, 128);
-      float corr[QC];
+      named_bar_sync(1 + wg, 128);
       bool need = false;
+      float my_corr = 1.f;                            // the factor of column cb + r (r < CH)
 #pragma unroll
-      for (int q = 0; q < QC; ++q) {
-        const float* rq = red + sb * 4 * QC + q;
+      for (int j = 0; j < CH; ++j) {
+        const float* rq = red + sb * 4 * QC + cb + j;
         const float mt = fmaxf(fmaxf(rq[0], rq[QC]), fmaxf(rq[2 * QC], rq[3 * QC]));
-        corr[q] = 1.f;
-        if (mt > M[q] + kRescaleSlack) {             // also the head's first finite maximum
-          corr[q] = exp2_shift(M[q], mt);
-          M[q] = mt;
+        float corr = 1.f;
+        if (mt > M[j] + kRescaleSlack) {             // also the head's first finite maximum
+          corr = exp2_shift(M[j], mt);
+          M[j] = mt;
           need = true;
         }
-        lp[q] *= corr[q];
+        lp[j] *= corr;
+        if (j == r) my_corr = corr;
       }
       if (need && !first) {
-        // the running O^T holds the tiles up to i - 1: rescale its columns
+        // the running O^T holds the tiles up to i - 1: rescale this
+        // warpgroup's columns (the same decision in its every thread)
+        if (r < CH) corrs[cb + r] = my_corr;
+        named_bar_sync(9 + wg, 128);
         if (ok) ok = mbar_wait(b_ofull, (i - 1) & 1, p.err);
         tc_fence_after();
-        uint32_t o[QC];
-        const uint32_t oaddr = tmem + kOCol + (seg & 1) * QC + lane_base;
-        ttmem_ld<QC>(oaddr, o);
+        const uint32_t oaddr = tmem + kOCol + (seg & 1) * QC + cb + lane_base;
+        uint32_t o[CH];
+        NECTAR_TMEM_LD16(oaddr, o);
         tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < QC; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * corr[q]);
-        ttmem_st<QC>(oaddr, o);
+        for (int j = 0; j < CH; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * corrs[cb + j]);
+        ttmem_st16(oaddr, o);
         tmem_st_wait();
       }
-      // the weights, bf16 into P (row, key): what the P V product and the
-      // row sums both use
+      // pass 2: the weights, bf16 into P (row, key): what the P V product and
+      // the row sums both use
       if (i >= 2 && ok) ok = mbar_wait(b_pfree + 8 * sb, ((i >> 1) - 1) & 1, p.err);
       uint8_t* pt = smem + SL::p + sb * SL::kP;
+      {
+        uint32_t v[CH];
+        NECTAR_TMEM_LD16(tmem + sb * QC + cb + lane_base, v);
+        tmem_ld_wait();
 #pragma unroll
-      for (int q = 0; q < QC; ++q) {
-        const __nv_bfloat16 w = __float2bfloat16_rn(exp2_shift(s[q], M[q]));
-        lp[q] += __bfloat162float(w);
-        *reinterpret_cast<__nv_bfloat16*>(pt + tp_off<QC>(q, r)) = w;
+        for (int j = 0; j < CH; ++j) {
+          const float sc = (valid && cb + j < R) ? __uint_as_float(v[j]) * p.qmul : -INFINITY;
+          const __nv_bfloat16 w = __float2bfloat16_rn(exp2_shift(sc, M[j]));
+          lp[j] += __bfloat162float(w);
+          *reinterpret_cast<__nv_bfloat16*>(pt + tp_off<QC>(cb + j, r)) = w;
+        }
       }
-      fence_proxy_async_smem();
       tc_fence_before();
+      mbar_arrive(b_sfree + 8 * sb);                  // S^T of this tile read for the last time
+      fence_proxy_async_smem();
       mbar_arrive(b_pfull + 8 * sb);
       if (last) {
         // the head's partial: O^T (this thread: dim r), the row sums, M.
@@ -378,32 +394,36 @@ cache_attn_tct_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
         if (ok && i >= 1) ok = mbar_wait(b_ofull, (i - 1) & 1, p.err);
         if (ok) ok = mbar_wait(b_ofull, i & 1, p.err);
         tc_fence_after();
-        uint32_t o[QC];
-        ttmem_ld<QC>(tmem + kOCol + (seg & 1) * QC + lane_base, o);
+        const int slot = c - first_cta_of_tile(hd * p.tph, p.total, p.C);
+        uint32_t o[CH];
+        NECTAR_TMEM_LD16(tmem + kOCol + (seg & 1) * QC + cb + lane_base, o);
         tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(b_ofree + 8 * (seg & 1));
-        float ls[QC];
+        float ls[CH];
 #pragma unroll
-        for (int q = 0; q < QC; ++q) ls[q] = lp[q];
-        const float w = twarp_reduce<QC, false>(ls, lane);
-        if (lane % kLanesPer == 0) reds[quarter * QC + lane / kLanesPer] = w;
-        named_bar_sync(2, 128);
-        const int slot = c - first_cta_of_tile(hd * p.tph, p.total, p.C);
+        for (int j = 0; j < CH; ++j) ls[j] = lp[j];
+        const float w = twarp_reduce<CH, false>(ls, lane);
+        if ((lane & 1) == 0) reds[quarter * QC + cb + (lane >> 1)] = w;
         if (ok) {
 #pragma unroll
-          for (int q = 0; q < QC; ++q) {
-            if (q < R) {
-              const int64_t prow = (hd * p.S_max + slot) * p.rows_total + q;
-              p.ws_acc[prow * kD + r] = __uint_as_float(o[q]);
-              if (r == 0) {
-                p.ws_ml[prow * 2] = M[q];
-                p.ws_ml[prow * 2 + 1] = (reds[q] + reds[QC + q]) + (reds[2 * QC + q] + reds[3 * QC + q]);
-              }
-            }
+          for (int j = 0; j < CH; ++j) {
+            const int q = cb + j;
+            if (q < R) p.ws_acc[((hd * p.S_max + slot) * p.rows_total + q) * kD + r] = __uint_as_float(o[j]);
           }
         }
-        named_bar_sync(2, 128);                     // the sums are read before the next head's
+        named_bar_sync(5 + wg, 128);
+        if (ok && r < CH && cb + r < R) {
+          const int64_t prow = (hd * p.S_max + slot) * p.rows_total + cb + r;
+          float mr = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < CH; ++j)
+            if (j == r) mr = M[j];
+          const float* rs = reds + cb + r;
+          p.ws_ml[prow * 2] = mr;
+          p.ws_ml[prow * 2 + 1] = (rs[0] + rs[QC]) + (rs[2 * QC] + rs[3 * QC]);
+        }
+        named_bar_sync(5 + wg, 128);                // the sums are read before the next head's
       }
     }
   }
@@ -417,21 +437,39 @@ cache_attn_tct_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
   }
 }
 
-// N = 16 query columns whatever the rows (3..16): a kind::f16 MMA with
-// M = 128 takes N in multiples of 16, so narrower S^T / O^T tiles are not
-// an option.
-size_t cache_attn_tct_smem(int rows) {
-  (void)rows;
-  return TSmem<16>::total + (kTctCtasPerSm > 1 ? 0 : 1024);
+// N = 16, 32 or 64 query columns (at least the rows): a kind::f16 MMA
+// with M = 128 takes N in multiples of 16.
+static int tct_qc(int64_t rows) { return rows <= 16 ? 16 : (rows <= 32 ? 32 : 64); }
+
+int cache_attn_tct_ctas_per_sm(int64_t rows) {
+  const int qc = tct_qc(rows);
+  return qc == 16 ? TCfg<16>::ctas : (qc == 32 ? TCfg<32>::ctas : TCfg<64>::ctas);
+}
+
+size_t cache_attn_tct_smem(int64_t rows) {
+  const int qc = tct_qc(rows);
+  const size_t slack = 1024;      // the dynamic base is rounded up to 1024 bytes
+  if (qc == 16) return TSmem<16>::total + (TCfg<16>::ctas > 1 ? 0 : slack);
+  return (qc == 32 ? TSmem<32>::total : TSmem<64>::total) + slack;
+}
+
+template <int QC>
+static cudaError_t launch_tct(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                              const DecParams& p, cudaStream_t stream) {
+  const size_t smem = cache_attn_tct_smem(p.rows_total);
+  cudaError_t e = cudaFuncSetAttribute(cache_attn_tct_kernel<QC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_k(cache_attn_tct_kernel<QC>, dim3(p.C), dim3(TCfg<QC>::threads), smem, stream, 1, tq, tk, tv, p);
 }
 
 cudaError_t launch_cache_attn_tct(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                   const DecParams& p, cudaStream_t stream) {
-  const size_t smem = cache_attn_tct_smem(static_cast<int>(p.rows_total));
-  cudaError_t e = cudaFuncSetAttribute(cache_attn_tct_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  return launch_k(cache_attn_tct_kernel<16>, dim3(p.C), dim3(kTThreads), smem, stream, 1, tq, tk, tv, p);
+  switch (tct_qc(p.rows_total)) {
+    case 16: return launch_tct<16>(tq, tk, tv, p, stream);
+    case 32: return launch_tct<32>(tq, tk, tv, p, stream);
+    default: return launch_tct<64>(tq, tk, tv, p, stream);
+  }
 }
 
 }  // namespace nectar

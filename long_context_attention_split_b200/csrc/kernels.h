@@ -101,11 +101,18 @@ size_t dec_smem_for_rows(int R);
 cudaError_t launch_cache_attn_split(const DecParams& p, int R, cudaStream_t stream);
 cudaError_t launch_cache_attn_combine(const DecParams& p, float* alpha, float* A, cudaStream_t stream);
 
-// ----- (i) 3-16 query rows per head: transposed tensor-core split ---------
+// ----- (i) 3-32 query rows per head: transposed tensor-core split ---------
 // Same stream-K plan (128-key tiles), partial layout and combine as the
 // split kernel.
 constexpr int kTctTile = 128;
-constexpr int kTctMaxRows = 16;
+// Up to this many rows per head: measured against the M = 128 tensor-core
+// kernel on Llama-8B-shaped documents, 32 rows 1.94 vs 2.06 ms, 64 rows
+// 2.60 vs 2.07 ms (one CTA per SM with four softmax warpgroups is bound
+// by the softmax chain of each tile).
+#ifndef NECTAR_TCT_MAX_ROWS
+#define NECTAR_TCT_MAX_ROWS 32
+#endif
+constexpr int kTctMaxRows = NECTAR_TCT_MAX_ROWS;
 // Resident CTAs per SM (each with a ring of 6 / this K or V stages): two
 // measured 1.29 ms against 1.72 for one on a 32 x 8-head, 65536-key
 // document at 4 rows (6.67 against 5.00 TB/s).
@@ -113,7 +120,8 @@ constexpr int kTctMaxRows = 16;
 #define NECTAR_TCT_CTAS_PER_SM 2
 #endif
 constexpr int kTctCtasPerSm = NECTAR_TCT_CTAS_PER_SM;
-size_t cache_attn_tct_smem(int rows);
+size_t cache_attn_tct_smem(int64_t rows);
+int cache_attn_tct_ctas_per_sm(int64_t rows);
 cudaError_t launch_cache_attn_tct(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                   const DecParams& p, cudaStream_t stream);
 

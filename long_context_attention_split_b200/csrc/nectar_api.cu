@@ -135,10 +135,10 @@ DeviceInfo device_info() {
 #ifndef NECTAR_TC_ROUTE_ROWS
 #define NECTAR_TC_ROUTE_ROWS 8
 #endif
-// 3 to 16 query rows per KV head: the transposed tensor-core split kernel
-// (attn_tct.cu), where the CUDA-core split kernel is bound by its ALU work
-// (measured on a Llama-8B-shaped document at 4 rows: the CUDA-core kernel
-// reaches 68 % of the HBM copy bandwidth).  NECTAR_TCT=0
+// 3 to kTctMaxRows query rows per KV head: the transposed tensor-core split
+// kernel (attn_tct.cu), where the CUDA-core split kernel is bound by its ALU
+// work (measured on a Llama-8B-shaped document at 4 rows: the CUDA-core
+// kernel reaches 68 % of the HBM copy bandwidth).  NECTAR_TCT=0
 // keeps those rows on the CUDA-core kernel (up to NECTAR_TC_ROUTE_ROWS).
 bool use_tct_attn(int64_t rows) {
   const char* e = getenv("NECTAR_TCT");
@@ -155,7 +155,7 @@ int dec_row_block(int64_t rows) { return rows < dec_max_rows() ? static_cast<int
 
 DecPlan cache_attn_plan(const nectar_dims& d, int64_t n, int64_t nq, int sms) {
   const int64_t rows = static_cast<int64_t>(d.G) * nq;
-  if (use_tct_attn(rows)) return plan_decode(d.L * d.Hkv, n, sms, kTctCtasPerSm, kTctTile);
+  if (use_tct_attn(rows)) return plan_decode(d.L * d.Hkv, n, sms, cache_attn_tct_ctas_per_sm(rows), kTctTile);
   const int R = dec_row_block(rows);
   return plan_decode(d.L * d.Hkv, n, sms, dec_ctas_per_sm(R < 1 ? 1 : R), dec_tile(R < 1 ? 1 : R));
 }

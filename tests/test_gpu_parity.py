@@ -93,6 +93,9 @@ def test_cache_attn_parity(L, Hkv, G, n, nq):
     (2, 4, 5, 20000, 1),      # 5 rows, each head cut over ~18 CTAs
     (1, 3, 8, 1537, 2),       # 16 rows, ragged tail of 1 key
     (2, 2, 2, 5000, 6),       # 12 rows (QC = 16)
+    (1, 2, 4, 5000, 5),       # 20 rows: 32 query columns
+    (2, 3, 4, 3000, 16),      # 64 rows: 64 query columns, heads cut over CTAs
+    (1, 2, 8, 1000, 6),       # 48 rows, ragged tail
 ])
 def test_cache_attn_tct(L, Hkv, G, n, nq, monkeypatch):
     wl, ag, Ag, ao, Ao = run_cache_attn(L, Hkv, G, n, nq, seed=n + 7 * G)
@@ -105,27 +108,30 @@ def test_cache_attn_tct(L, Hkv, G, n, nq, monkeypatch):
         assert np.abs(ag - ag0).max() <= ALPHA_TOL and np.abs(Ag - Ag0).max() <= ATT_TOL * vmax
 
 
-def test_cache_attn_tct_repeatable():
+@pytest.mark.parametrize("G,nq", [(5, 1), (4, 16)])
+def test_cache_attn_tct_repeatable(G, nq):
     # a head spread over several CTAs with several tiles each: ten calls give
     # the same bits (the partials are summed in a fixed order; a call that
     # read a head's O^T before its last tiles had landed would not)
-    wl = make_workload("toy", L=2, Hkv=4, G=5, n=20000, nq=1, T=1, with_local=False, with_modules=False, seed=3)
+    wl = make_workload("toy", L=2, Hkv=4, G=G, n=20000, nq=nq, T=1, with_local=False, with_modules=False, seed=3)
     K, V, Q = wl.K.cuda(), wl.V.cuda(), wl.Q.cuda()
     a0, A0 = nx.cache_attn_lse(K, V, Q)
     for _ in range(9):
         a1, A1 = nx.cache_attn_lse(K, V, Q)
         torch.cuda.synchronize()
         assert torch.equal(a1, a0) and torch.equal(A1, A0)
-    ao, Ao = oracle.cache_attn(wl.K, wl.V, wl.Q.reshape(2, 4, 5, 128), wl.scale)
+    ao, Ao = oracle.cache_attn(wl.K, wl.V, wl.Q.reshape(2, 4, G * nq, 128), wl.scale)
     check_attn(a0.cpu().numpy().reshape(ao.shape), A0.cpu().numpy().reshape(Ao.shape), ao, Ao,
                wl.V.float().abs().max().item(), "tct repeat")
 
 
-def test_cache_attn_tct_running_max_moves():
-    # 4 rows: after 40 tiles of ordinary scores a key scores ~ +10 (natural
-    # log units) higher for two of the rows, so the running maximum of those
-    # rows moves past the 2^8 slack and their O^T columns are rescaled in TMEM
-    L, Hkv, G, nq, n = 1, 2, 4, 1, 9000
+@pytest.mark.parametrize("nq", [1, 12])
+def test_cache_attn_tct_running_max_moves(nq):
+    # 4 or 48 rows: after 40 tiles of ordinary scores a key scores ~ +10
+    # (natural log units) higher for two of the rows, so the running maximum
+    # of those rows moves past the 2^8 slack and their O^T columns are
+    # rescaled in TMEM
+    L, Hkv, G, n = 1, 2, 4, 9000
     g = torch.Generator().manual_seed(21)
     K = torch.randn(L, Hkv, n, 128, generator=g)
     V = torch.randn(L, Hkv, n, 128, generator=g)
