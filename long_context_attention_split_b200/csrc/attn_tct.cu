@@ -6,7 +6,7 @@
 // per (key, row, dim) and is bound by the ALU, not by the K/V bytes.  Here
 // the products run on tcgen05, taken transposed so that the keys fill the
 // 128 rows of the tensor-core tile and the TMEM lanes:
-//   S^T = K Q^T   (M = 128 keys of a tile, N = QC = 16 >= rows, K = d; K and Q
+//   S^T = K Q^T   (M = 128 keys of a tile, N = QC = 16 or 32 >= rows, K = d; K, Q
 //                  K-major, 128-byte swizzle),
 //   O^T = V^T P^T (M = d, N = QC, K = the tile's keys; V read MN-major).
 // Each of the 128 softmax threads owns one key of a tile and holds its row
@@ -44,14 +44,14 @@ constexpr int kTKeys = kTctTile;                   // keys per tile (TMEM lanes 
 #define NECTAR_TCT_STAGES (6 / NECTAR_TCT_CTAS_PER_SM)
 #endif
 // Per query-column count QC: resident CTAs per SM and K / V ring stages.
-// 16 columns: two CTAs of NECTAR_TCT_STAGES stages; 32 and 64 columns (Q,
-// P and the row state grow with QC): one CTA, with the stages that fit.
+// 16 columns: two CTAs of NECTAR_TCT_STAGES stages; 32 columns (Q, P and
+// the row state grow with QC): one CTA of six stages.
 template <int QC>
 struct TCfg {
   static constexpr int wgs = QC / 16;                     // softmax warpgroups
   static constexpr int threads = 64 + 128 * wgs;
   static constexpr int ctas = QC == 16 ? kTctCtasPerSm : 1;
-  static constexpr int stages = QC == 16 ? NECTAR_TCT_STAGES : (QC == 32 ? 6 : 4);
+  static constexpr int stages = QC == 16 ? NECTAR_TCT_STAGES : 6;
 };
 constexpr uint32_t kTHalf = kTKeys * 128;          // 128 keys x 64 dims bf16: 16 KB
 constexpr uint32_t kTTile = 2 * kTHalf;
@@ -158,7 +158,7 @@ cache_attn_tct_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
   constexpr uint32_t kTmemCols = 4 * QC < 32 ? 32 : 4 * QC;   // S^T [2][QC], O^T [2][QC]
   constexpr int kWG = TCfg<QC>::wgs;
   constexpr int kThreadsAll = TCfg<QC>::threads;
-  static_assert(QC % 16 == 0 && QC <= 64, "16, 32 or 64 query columns");
+  static_assert(QC == 16 || QC == 32, "16 or 32 query columns");
   const uint32_t kOCol = 2 * QC;
 
   if (threadIdx.x == 0) {
@@ -437,20 +437,20 @@ cache_attn_tct_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
   }
 }
 
-// N = 16, 32 or 64 query columns (at least the rows): a kind::f16 MMA
-// with M = 128 takes N in multiples of 16.
-static int tct_qc(int64_t rows) { return rows <= 16 ? 16 : (rows <= 32 ? 32 : 64); }
+// N = 16 or 32 query columns (at least the rows): a kind::f16 MMA with
+// M = 128 takes N in multiples of 16.
+static int tct_qc(int64_t rows) { return rows <= 16 ? 16 : 32; }
 
 int cache_attn_tct_ctas_per_sm(int64_t rows) {
   const int qc = tct_qc(rows);
-  return qc == 16 ? TCfg<16>::ctas : (qc == 32 ? TCfg<32>::ctas : TCfg<64>::ctas);
+  return qc == 16 ? TCfg<16>::ctas : TCfg<32>::ctas;
 }
 
 size_t cache_attn_tct_smem(int64_t rows) {
   const int qc = tct_qc(rows);
   const size_t slack = 1024;      // the dynamic base is rounded up to 1024 bytes
   if (qc == 16) return TSmem<16>::total + (TCfg<16>::ctas > 1 ? 0 : slack);
-  return (qc == 32 ? TSmem<32>::total : TSmem<64>::total) + slack;
+  return TSmem<32>::total + slack;
 }
 
 template <int QC>
@@ -467,8 +467,7 @@ cudaError_t launch_cache_attn_tct(const CUtensorMap& tq, const CUtensorMap& tk, 
                                   const DecParams& p, cudaStream_t stream) {
   switch (tct_qc(p.rows_total)) {
     case 16: return launch_tct<16>(tq, tk, tv, p, stream);
-    case 32: return launch_tct<32>(tq, tk, tv, p, stream);
-    default: return launch_tct<64>(tq, tk, tv, p, stream);
+    default: return launch_tct<32>(tq, tk, tv, p, stream);
   }
 }
 

@@ -108,10 +108,12 @@ constexpr int kTctTile = 128;
 // Up to this many rows per head: measured against the M = 128 tensor-core
 // kernel on Llama-8B-shaped documents, 32 rows 1.94 vs 2.06 ms, 64 rows
 // 2.60 vs 2.07 ms (one CTA per SM with four softmax warpgroups is bound
-// by the softmax chain of each tile).
+// by the softmax chain of each tile), so the kernel is built for 16 and 32
+// query columns only.
 #ifndef NECTAR_TCT_MAX_ROWS
 #define NECTAR_TCT_MAX_ROWS 32
 #endif
+static_assert(NECTAR_TCT_MAX_ROWS >= 2 && NECTAR_TCT_MAX_ROWS <= 32, "transposed kernel: at most 32 rows");
 constexpr int kTctMaxRows = NECTAR_TCT_MAX_ROWS;
 // Resident CTAs per SM (each with a ring of 6 / this K or V stages): two
 // measured 1.29 ms against 1.72 for one on a 32 x 8-head, 65536-key
