@@ -232,20 +232,47 @@ __global__ void cache_attn_combine_kernel(const DecParams p, float* __restrict__
   }
   const int f = first_cta_of_tile(hd * p.tph, p.total, p.C);
   const int la = first_cta_of_tile(hd * p.tph + p.tph - 1, p.total, p.C);
+  const int ns = la - f + 1;                    // partials of this head
+  const float* ml = p.ws_ml + (hd * p.S_max * p.rows_total + r) * 2;     // partial s at ml[s * rows_total * 2]
+  const float* ac = p.ws_acc + (hd * p.S_max * p.rows_total + r) * kD;   // partial s at ac[s * rows_total * d]
+  const int64_t sml = static_cast<int64_t>(p.rows_total) * 2, sac = static_cast<int64_t>(p.rows_total) * kD;
+  // the partials' maxima, one partial per lane (all loads in flight at once)
   float M = -INFINITY;
-  for (int s = 0; s <= la - f; ++s) M = fmaxf(M, p.ws_ml[((hd * p.S_max + s) * p.rows_total + r) * 2]);
+  for (int s = lane; s < ns; s += 32) M = fmaxf(M, ml[s * sml]);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  // weights 2^(m_s - M), the sum of the row weights, and the weighted sum of
+  // the partial value sums, 32 partials at a time
   float ls = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s <= la - f; ++s) {
-    const int64_t prow = (hd * p.S_max + s) * p.rows_total + r;
-    const float w = exp2_shift(p.ws_ml[prow * 2], M);
-    ls = fmaf(p.ws_ml[prow * 2 + 1], w, ls);
-    const float4 a4 = reinterpret_cast<const float4*>(p.ws_acc + prow * kD)[lane];
-    acc.x = fmaf(a4.x, w, acc.x);
-    acc.y = fmaf(a4.y, w, acc.y);
-    acc.z = fmaf(a4.z, w, acc.z);
-    acc.w = fmaf(a4.w, w, acc.w);
+  for (int s0 = 0; s0 < ns; s0 += 32) {
+    const int s = s0 + lane;
+    float w = 0.f;
+    if (s < ns) {
+      w = exp2_shift(ml[s * sml], M);
+      ls = fmaf(ml[s * sml + 1], w, ls);
+    }
+    const int cnt = ns - s0 < 32 ? ns - s0 : 32;
+    for (int j0 = 0; j0 < cnt; j0 += 8) {
+      float4 a4[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        a4[j] = j0 + j < cnt ? reinterpret_cast<const float4*>(ac + (s0 + j0 + j) * sac)[lane]
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, w, (j0 + j) & 31);
+        if (j0 + j < cnt) {
+          acc.x = fmaf(a4[j].x, wj, acc.x);
+          acc.y = fmaf(a4[j].y, wj, acc.y);
+          acc.z = fmaf(a4[j].z, wj, acc.z);
+          acc.w = fmaf(a4[j].w, wj, acc.w);
+        }
+      }
+    }
   }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
   const float inv = 1.0f / ls;
   *out = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   if (lane == 0) alpha[gw] = (M + log2f(ls)) * kLn2;
