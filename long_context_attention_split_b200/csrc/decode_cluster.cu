@@ -58,7 +58,6 @@ namespace nectar {
 
 namespace {
 
-constexpr int kSlices = 8;                       // slices of every net's hidden units
 constexpr uint32_t kStage = 32 * 1024;           // weight ring stage
 constexpr uint32_t kPad = 8 * 1024;              // read (not used) past the ring by a 64-row tile
 constexpr int kEpiWarps = 8;
@@ -66,19 +65,22 @@ constexpr int kLocWarps = 4;
 constexpr int kThreads = (2 + kEpiWarps + kLocWarps) * 32;
 constexpr int kLocKPG = 2;                        // keys per lane group per step
 constexpr int kMaxStages = 8;
+constexpr int kMaxSliceTiles = 4;                 // 128-unit M tiles of a slice (H <= 2048, 4 slices)
 
 struct ClSmem {
   uint32_t ring, xq, xh, xro, rt, rl, rs, rml, sp, lscr, bars, tslot, total;
 };
 
-// 64-unit granules: the h slices exchanged between CTAs are whole 64-column
-// chunks of X
-__host__ __device__ inline int cl_slice(int H) {
-  const int s = (H + kSlices - 1) / kSlices;
+// Slices of each net's hidden units: one per CTA holding that net, so
+// cluster * nets per CTA / 2.  64-unit granules: the h slices exchanged
+// between CTAs are whole 64-column chunks of X.
+__host__ __device__ constexpr int cl_slices(int kC, int npc) { return kC * npc / 2; }
+__host__ __device__ inline int cl_slice(int H, int ksl) {
+  const int s = (H + ksl - 1) / ksl;
   return (s + 63) / 64 * 64;
 }
-__host__ __device__ inline int cl_slice_len(int H, int si) {
-  const int S = cl_slice(H);
+__host__ __device__ inline int cl_slice_len(int H, int si, int ksl) {
+  const int S = cl_slice(H, ksl);
   const int len = H - si * S;
   return len < 0 ? 0 : (len < S ? len : S);
 }
@@ -89,7 +91,7 @@ __host__ __device__ inline int cl_rp(int R) { return (R + 3) / 4 * 4; }
 // cluster of kC CTAs each holding npc nets
 __host__ __device__ inline ClSmem cl_layout(int kC, int npc, int Hmax, int N, int R, int nb, int stages, int rg) {
   ClSmem s{};
-  const int own = kD / kC, Rp = cl_rp(R);
+  const int own = kD / kC, Rp = cl_rp(R), ksl = cl_slices(kC, npc);
   uint32_t off = 0;
   s.ring = off;
   off += static_cast<uint32_t>(stages) * kStage + kPad;
@@ -98,13 +100,13 @@ __host__ __device__ inline ClSmem cl_layout(int kC, int npc, int Hmax, int N, in
   s.xh = off;                                                   // h: [net][buf][chunk][N][128 B]
   off += static_cast<uint32_t>(npc * nb * layout::kchunks(Hmax) * N * 128);
   s.xro = off;                                                  // the target readout's input: own slice
-  off += static_cast<uint32_t>(layout::kchunks(cl_slice(Hmax))) * N * 128;
+  off += static_cast<uint32_t>(layout::kchunks(cl_slice(Hmax, ksl))) * N * 128;
   s.rt = off;                                                   // target partials [slice][dim][row]
-  off += static_cast<uint32_t>(kSlices * own * Rp) * 4;
+  off += static_cast<uint32_t>(ksl * own * Rp) * 4;
   s.rl = off;                                                   // local acc partials [cta][row][dim]
   off += static_cast<uint32_t>(kC * Rp * own) * 4;
   s.rs = off;                                                   // score partials [slice][row]
-  off += static_cast<uint32_t>(kSlices * Rp) * 4;
+  off += static_cast<uint32_t>(ksl * Rp) * 4;
   s.rml = off;                                                  // local (m, l) [cta][row][2]
   off += static_cast<uint32_t>(kC * Rp * 2) * 4;
   s.sp = off;                                                   // score sums by lane quarter [4][N]
@@ -132,19 +134,20 @@ __device__ __forceinline__ uint32_t cl_xoff(int N, int n, int c) {
                                ((c & 7) << 1));
 }
 
-template <int RG, int kC>
+template <int RG, int kC, int kNPC>
 __global__ void __launch_bounds__(kThreads, 1)
-decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterParams p) {
-  constexpr int kNPC = kC == 2 * kSlices ? 1 : 2;   // nets per CTA
+decode_cluster_kernel(const ClusterParams p) {
+  constexpr int kSl = cl_slices(kC, kNPC);           // slices of each net
   constexpr int kOwn = kD / kC;                      // output dims merged by each CTA
-  static_assert(kC == kSlices || kC == 2 * kSlices, "8 or 16 CTAs per cluster");
+  static_assert((kC == 8 && (kNPC == 1 || kNPC == 2)) || (kC == 16 && kNPC == 1),
+                "8 CTAs holding one or both nets, or 16 holding one");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = cl_aligned(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = static_cast<int>(cluster_ctarank());
-  const int si = r % kSlices;                       // slice of the units
-  const int n0 = kNPC == 1 ? r / kSlices : 0;       // the CTA's first net (0 score, 1 target)
-  const int pbase = kNPC == 1 ? n0 * kSlices : 0;   // rank of slice 0 of the CTA's nets
+  const int si = r % kSl;                           // slice of the units
+  const int n0 = kNPC == 1 ? r / kSl : 0;           // the CTA's first net (0 score, 1 target)
+  const int pbase = kNPC == 1 ? n0 * kSl : 0;       // rank of slice 0 of the CTA's nets
   const bool has_target = n0 + kNPC - 1 == 1;
   const int ci = static_cast<int>(blockIdx.x) / kC;
   const int li = ci / p.Hkv, h = ci % p.Hkv;
@@ -158,11 +161,11 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
   const int R = p.G * static_cast<int>(p.nq);               // query rows of the head (<= N)
   const int Rp = cl_rp(R);
   const ClSmem SL = cl_layout(kC, kNPC, p.Hmax, N, R, nb, S_, RG);
-  const int S = cl_slice(H);
+  const int S = cl_slice(H, kSl);
   const int u0 = si * S;
-  const int slen = cl_slice_len(H, si);
+  const int slen = cl_slice_len(H, si, kSl);
   const int MT = (slen + 127) / 128;                       // M tiles of the slice (0: empty slice)
-  const int MTmax = (cl_slice(p.Hmax) + 127) / 128;        // TMEM columns are planned for the widest layer
+  const int MTmax = (cl_slice(p.Hmax, kSl) + 127) / 128;   // TMEM columns are planned for the widest layer
   const int64_t sbase = p.layer_base[l] + static_cast<int64_t>(h) * layout::head_elems(H, depth);
   const int64_t tbase = sbase + layout::net_elems(H, depth, 1);
   const int64_t hd = static_cast<int64_t>(l) * p.Hkv + h;
@@ -231,11 +234,7 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
-      prefetch_tmap(&tmap_q);
       const uint64_t pol = policy_evict_first();
-      mbar_arrive_expect_tx(b_q, static_cast<uint32_t>(2 * R * 128));
-      tma_load_4d(xq, &tmap_q, 0, 0, 0, static_cast<int>(hd), b_q, pol);
-      tma_load_4d(xq + N * 128, &tmap_q, 64, 0, 0, static_cast<int>(hd), b_q, pol);
       uint32_t it = 0;
       bool ok = true;
       for (int k = 0; k < depth && ok; ++k) {
@@ -261,9 +260,16 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
                 bulk_g2s(dst, W + layout::tile_chunk_off(H, K, m, c0), static_cast<uint32_t>(nc * 128 * 128),
                          b_full + 8 * s, pol);
               } else {
-                for (int cl = 0; cl < nc; ++cl)
+                // a slice that starts inside a 128-row tile of the blob takes
+                // its first rows from tile m and the rest from tile m + 1
+                const int r1 = rv < 128 - r0 ? rv : 128 - r0;
+                for (int cl = 0; cl < nc; ++cl) {
                   bulk_g2s(dst + cl * rvp * 128, W + layout::tile_chunk_off(H, K, m, c0 + cl) + r0 * 64,
-                           static_cast<uint32_t>(rv * 128), b_full + 8 * s, pol);
+                           static_cast<uint32_t>(r1 * 128), b_full + 8 * s, pol);
+                  if (rv > r1)
+                    bulk_g2s(dst + cl * rvp * 128 + r1 * 128, W + layout::tile_chunk_off(H, K, m + 1, c0 + cl),
+                             static_cast<uint32_t>((rv - r1) * 128), b_full + 8 * s, pol);
+                }
               }
             }
           }
@@ -287,13 +293,22 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
     // ------------------------------ MMA issuer ------------------------------
     if (lane == 0) {
       bool ok = mbar_wait(b_q, 0, p.err);
-      uint32_t it = 0;
       const uint32_t idesc = idesc_bf16_f32(128, N, 0, 0);
+      const uint64_t dK = sdesc_sw128(0, 16, 1024);    // K-major, 128-byte swizzle, at address 0
+      int s = 0;                                      // ring stage and its phase
+      uint32_t ph = 0;
+      auto next_stage = [&]() {
+        if (++s == S_) {
+          s = 0;
+          ph ^= 1u;
+        }
+      };
       for (int k = 0; k < depth && ok; ++k) {
         if (k > 0) {
           // every slice of h_{k-1} (of the CTA's nets) is in this CTA's X
-          ok = mbar_wait(b_hr + 8 * ((k - 1) & 1), ((k - 1) >> 1) & 1, p.err);
+          ok = mbar_wait_cluster(b_hr + 8 * ((k - 1) & 1), ((k - 1) >> 1) & 1, p.err);
           if (!ok) break;
+          fence_proxy_async_smem();    // the peers' stores, to the tensor core's reads
         }
         tc_fence_after();
         const int kc = layout::kchunks(layout::hidden_k(H, k));
@@ -305,23 +320,24 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
             const int rvp = rv <= 64 ? 64 : 128;
             const int cpg = static_cast<int>(kStage / (rvp * 128));
             const uint32_t dcol = tmem + static_cast<uint32_t>((j * MTmax + t) * N);
-            for (int c0 = 0; c0 < kc; c0 += cpg, ++it) {
-              const uint32_t s = it % S_;
-              if (!mbar_wait(b_full + 8 * s, (it / S_) & 1, p.err)) {
+            for (int c0 = 0; c0 < kc; c0 += cpg) {
+              // (bulk copies into the ring and the MMAs' reads of it are both
+              // async-proxy operations ordered by the barrier; no tcgen05
+              // fence is needed here, and one per stage costs ~0.1 us)
+              if (!mbar_wait(b_full + 8 * s, ph, p.err)) {
                 ok = false;
                 break;
               }
-              tc_fence_after();
               const int nc = (kc - c0 < cpg) ? (kc - c0) : cpg;
               for (int cl = 0; cl < nc; ++cl) {
-                const uint32_t a = ring + s * kStage + cl * rvp * 128;
-                const uint32_t b = xchunk(j, buf, c0 + cl);
+                const uint64_t da = sdesc_at(dK, ring + s * kStage + cl * rvp * 128);
+                const uint64_t db = sdesc_at(dK, xchunk(j, buf, c0 + cl));
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                  mma_bf16_ss(dcol, sdesc_sw128(a + kk * 32, 16, 1024), sdesc_sw128(b + kk * 32, 16, 1024), idesc,
-                              (c0 + cl + kk) != 0);
+                for (int kk = 0; kk < 4; ++kk)   // 16 columns (32 bytes) of K per MMA
+                  mma_bf16_ss(dcol, da + 2 * kk, db + 2 * kk, idesc, (c0 + cl + kk) != 0);
               }
               mma_commit(b_empty + 8 * s);
+              next_stage();
             }
           }
           mma_commit(b_acc + 8 * j);
@@ -333,23 +349,21 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
         tc_fence_after();
         const int nch = (slen + 63) / 64;
         const uint32_t dcol = tmem + static_cast<uint32_t>(kNPC * MTmax * N);
-        for (int c0 = 0; c0 < nch && ok; c0 += 2, ++it) {
-          const uint32_t s = it % S_;
-          if (!mbar_wait(b_full + 8 * s, (it / S_) & 1, p.err)) {
+        for (int c0 = 0; c0 < nch && ok; c0 += 2) {
+          if (!mbar_wait(b_full + 8 * s, ph, p.err)) {
             ok = false;
             break;
           }
-          tc_fence_after();
           const int nc = (nch - c0 < 2) ? (nch - c0) : 2;
           for (int cl = 0; cl < nc; ++cl) {
-            const uint32_t a = ring + s * kStage + cl * 128 * 128;
-            const uint32_t b = xro + static_cast<uint32_t>((c0 + cl) * N * 128);
+            const uint64_t da = sdesc_at(dK, ring + s * kStage + cl * 128 * 128);
+            const uint64_t db = sdesc_at(dK, xro + static_cast<uint32_t>((c0 + cl) * N * 128));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(dcol, sdesc_sw128(a + kk * 32, 16, 1024), sdesc_sw128(b + kk * 32, 16, 1024), idesc,
-                          (c0 + cl + kk) != 0);
+              mma_bf16_ss(dcol, da + 2 * kk, db + 2 * kk, idesc, (c0 + cl + kk) != 0);
           }
           mma_commit(b_empty + 8 * s);
+          next_stage();
         }
         mma_commit(b_rof);
       }
@@ -359,31 +373,62 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
     const int j = (warp - 2) >> 2;                   // local net of this warp group
     const int q4 = warp & 3;                         // TMEM lane quarter of this warp
     const int et = ((warp - 2) & 3) * 32 + lane;     // 0..127 within the group
+    if (j == 0) {
+      // the head's R query rows (contiguous, 256 bytes each) into X's q
+      // chunks, 16 bytes per load, swizzled as the MMA reads them; a few
+      // hundred bytes, so plain loads: the TMA unit keeps to the weights
+      const uint4* qg = reinterpret_cast<const uint4*>(p.Q + hd * R * kD);
+      for (int i = et; i < R * 16; i += 128) {
+        const int n = i >> 4, c16 = i & 15;
+        const uint4 v = qg[i];
+        *reinterpret_cast<uint4*>(smem + SL.xq + (c16 >> 3) * N * 128 + n * 128 + (((c16 & 7) ^ (n & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (et == 0) mbar_arrive(b_q);
+    }
     if (j < kNPC) {
       const int net = n0 + j;                        // 0 score, 1 target
       const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
       const int64_t nbase = net ? tbase : sbase;
       float* sp = reinterpret_cast<float*>(smem + SL.sp);
       bool ok = true;
+      uint32_t peer = 0;                             // bytes of h_k the other slices send here
+      for (int o = 0; o < kSl; ++o) {
+        const int sl = cl_slice_len(H, o, kSl);
+        if (o != si && sl > 0) peer += static_cast<uint32_t>((sl + 63) / 64 * N * 128);
+      }
       for (int k = 0; k < depth; ++k) {
         const bool last = (k == depth - 1);
         const int buf = k % nb;
         const bool reduce = last && net == 0;           // the score readout: w . h summed here
         if (MT > 0) {
-          if (ok) ok = mbar_wait(b_acc + 8 * j, k & 1, p.err);
-          tc_fence_after();
+          // this thread's biases (and score readout weights), read while the
+          // layer's MMAs run
           const __nv_bfloat16* bias = p.blob + nbase + layout::hidden_b_off(H, depth, k);
           const __nv_bfloat16* wsc = p.blob + sbase + layout::out_w_off(H, depth);
+          float bvr[kMaxSliceTiles], wvr[kMaxSliceTiles];
+#pragma unroll
+          for (int t = 0; t < kMaxSliceTiles; ++t) {
+            const int u = t * 128 + q4 * 32 + lane;
+            const bool valid = t < MT && u < slen;
+            bvr[t] = valid ? __bfloat162float(bias[u0 + u]) : 0.f;
+            wvr[t] = (valid && reduce) ? __bfloat162float(wsc[u0 + u]) : 0.f;
+          }
+          if (ok) ok = mbar_wait(b_acc + 8 * j, k & 1, p.err);
+          tc_fence_after();
           for (int n0r = 0; n0r < N; n0r += 16) {
             float part[16];
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) part[jj] = 0.f;
-            for (int t = 0; t < MT; ++t) {
+#pragma unroll
+            for (int t = 0; t < kMaxSliceTiles; ++t) {
+              if (t >= MT) break;
               const int u = t * 128 + q4 * 32 + lane;
               const bool valid = u < slen && ok;
               const int gu = u0 + u;
-              const float bv = valid ? __bfloat162float(bias[gu]) : 0.f;
-              const float wv = (valid && reduce) ? __bfloat162float(wsc[gu]) : 0.f;
+              const float bv = bvr[t];
+              const float wv = wvr[t];
               uint32_t v[16];
               NECTAR_TMEM_LD16(trow + static_cast<uint32_t>((j * MTmax + t) * N + n0r), v);
               tmem_ld_wait();
@@ -423,21 +468,20 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
         tc_fence_before();
         named_bar_sync(1 + j, 128);
         if (!last) {
-          if (et == 0) {
-            // own arrival, expecting the other slices of this net as transactions
-            uint32_t peer = 0;
-            for (int o = 0; o < kSlices; ++o) {
-              const int sl = cl_slice_len(H, o);
-              if (o != si && sl > 0) peer += static_cast<uint32_t>((sl + 63) / 64 * N * 128);
-            }
-            const uint32_t hr = b_hr + 8 * (k & 1);
-            mbar_arrive_expect_tx(hr, peer);
-            if (MT > 0) {
-              const uint32_t src = xchunk(j, buf, 2 + u0 / 64);
-              const uint32_t bytes = static_cast<uint32_t>((slen + 63) / 64 * N * 128);
-              for (int o = 0; o < kSlices; ++o)
-                if (o != si)
-                  bulk_s2cluster(mapa_shared(src, pbase + o), src, bytes, mapa_shared(hr, pbase + o));
+          const uint32_t hr = b_hr + 8 * (k & 1);
+          // own arrival, expecting the other slices of this net as transactions
+          if (et == 0) mbar_arrive_expect_tx(hr, peer);
+          if (MT > 0) {
+            // this slice of h_k into the same place of every other CTA holding
+            // the net: 16-byte stores by the group's threads, each completing
+            // its bytes on the receiver's barrier (point to point, no multicast)
+            const uint32_t src = xchunk(j, buf, 2 + u0 / 64);
+            const int n16 = (slen + 63) / 64 * N * 8;
+            for (int i = et; i < n16; i += 128) {
+              const uint4 v = ld_shared_v4(src + 16 * i);
+#pragma unroll
+              for (int o = 0; o < kSl; ++o)
+                if (o != si) st_async_v4(mapa_shared(src + 16 * i, pbase + o), v, mapa_shared(hr, pbase + o));
             }
           }
         } else if (net == 0) {
@@ -555,6 +599,23 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
   }
 
   // ------------------------------ reduction and merge ------------------------------
+  // the readout biases this thread's merge items need, read before the barrier
+  constexpr int kMergeThreads = kThreads - 64;
+  constexpr int kMaxItems = (64 * kOwn + kMergeThreads - 1) / kMergeThreads;   // R <= 64
+  // (raw bits: the loads are in flight across the barrier, converted after it)
+  uint16_t csb = 0, ctb[kMaxItems];
+#pragma unroll
+  for (int q = 0; q < kMaxItems; ++q) ctb[q] = 0;
+  if (warp >= 2) {
+    const uint16_t* bits = reinterpret_cast<const uint16_t*>(p.blob);
+    csb = bits[sbase + layout::out_b_off(H, depth, 1)];
+    const uint16_t* ct = bits + tbase + layout::out_b_off(H, depth, kD);
+#pragma unroll
+    for (int q = 0; q < kMaxItems; ++q) {
+      const int item = threadIdx.x - 64 + q * kMergeThreads;
+      if (item < R * kOwn) ctb[q] = ct[r * kOwn + item % kOwn];
+    }
+  }
   __syncwarp();
   cluster_sync_all();              // every partial is in its owner's shared memory
   if (warp >= 2) {
@@ -562,21 +623,22 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
     const float* rt = reinterpret_cast<const float*>(smem + SL.rt);
     const float* rl = reinterpret_cast<const float*>(smem + SL.rl);
     const float* rml = reinterpret_cast<const float*>(smem + SL.rml);
-    const float cs = __bfloat162float(p.blob[sbase + layout::out_b_off(H, depth, 1)]);
-    const __nv_bfloat16* ct = p.blob + tbase + layout::out_b_off(H, depth, kD);
-    for (int item = threadIdx.x - 64; item < R * kOwn; item += kThreads - 64) {
+#pragma unroll
+    for (int q = 0; q < kMaxItems; ++q) {
+      const int item = threadIdx.x - 64 + q * kMergeThreads;
+      if (item >= R * kOwn) break;
       const int n = item / kOwn, dl = item % kOwn;
       const int dim = r * kOwn + dl;
       float a = 0.f, at = 0.f, Ml = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kSlices; ++c) {
+      for (int c = 0; c < kSl; ++c) {
         a += rs[c * Rp + n];
         at += rt[(c * kOwn + dl) * Rp + n];
       }
 #pragma unroll
       for (int c = 0; c < kC; ++c) Ml = fmaxf(Ml, rml[(c * Rp + n) * 2]);
-      a += cs;
-      at += __bfloat162float(ct[dim]);
+      a += __uint_as_float(static_cast<uint32_t>(csb) << 16);
+      at += __uint_as_float(static_cast<uint32_t>(ctb[q]) << 16);
       float ll = 0.f, al = 0.f;
 #pragma unroll
       for (int c = 0; c < kC; ++c) {
@@ -603,27 +665,28 @@ decode_cluster_kernel(const __grid_constant__ CUtensorMap tmap_q, const ClusterP
   }
 }
 
-template <int RG, int kC>
+template <int RG, int kC, int kNPC>
 cudaError_t set_attrs(size_t smem) {
-  cudaError_t e = cudaFuncSetAttribute(decode_cluster_kernel<RG, kC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(decode_cluster_kernel<RG, kC, kNPC>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e == cudaSuccess && kC > 8)
-    e = cudaFuncSetAttribute(decode_cluster_kernel<RG, kC>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = cudaFuncSetAttribute(decode_cluster_kernel<RG, kC, kNPC>, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                             1);
   return e;
 }
 
-template <int RG, int kC>
-cudaError_t launch_cl(const CUtensorMap& tq, const ClusterParams& p, int heads, size_t smem, cudaStream_t stream) {
-  const cudaError_t e = set_attrs<RG, kC>(smem);
+template <int RG, int kC, int kNPC>
+cudaError_t launch_cl(const ClusterParams& p, int heads, size_t smem, cudaStream_t stream) {
+  const cudaError_t e = set_attrs<RG, kC, kNPC>(smem);
   if (e != cudaSuccess) return e;
-  return launch_k(decode_cluster_kernel<RG, kC>, dim3(static_cast<unsigned>(heads * kC)), dim3(kThreads), smem,
-                  stream, kC, tq, p);
+  return launch_k(decode_cluster_kernel<RG, kC, kNPC>, dim3(static_cast<unsigned>(heads * kC)), dim3(kThreads),
+                  smem, stream, kC, p);
 }
 
 // Clusters of this shape that can be resident at once (0: none, or unknown).
-template <int RG, int kC>
+template <int RG, int kC, int kNPC>
 int max_clusters(size_t smem) {
-  if (set_attrs<RG, kC>(smem) != cudaSuccess) {
+  if (set_attrs<RG, kC, kNPC>(smem) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -639,7 +702,7 @@ int max_clusters(size_t smem) {
   cfg.attrs = at;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, decode_cluster_kernel<RG, kC>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, decode_cluster_kernel<RG, kC, kNPC>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -650,14 +713,18 @@ int max_clusters(size_t smem) {
 
 int cluster_rg(int G) { return G <= 2 ? 2 : 4; }
 
-ClusterShape cluster_shape(int cluster, int G, int64_t nq, int Hmax, int depth) {
+ClusterShape cluster_shape(int cluster, int npc, int G, int64_t nq, int Hmax, int depth) {
   ClusterShape sh{};
   const int64_t R = static_cast<int64_t>(G) * nq;
-  if ((cluster != 8 && cluster != 16) || R < 1 || R > 64 || nq > 256 || depth < 1 || depth > 4) return sh;
+  const bool shape_ok = (cluster == 8 && (npc == 1 || npc == 2)) || (cluster == 16 && npc == 1);
+  if (!shape_ok || R < 1 || R > 64 || nq > 256 || depth < 1 || depth > 4) return sh;
+  const int ksl = cl_slices(cluster, npc);
+  const int S = cl_slice(Hmax, ksl);
+  if (S > 128 * kMaxSliceTiles) return sh;
   sh.cluster = cluster;
+  sh.npc = npc;
   sh.N = static_cast<int>((R + 15) / 16 * 16);
   sh.nb = depth >= 3 ? 2 : 1;
-  const int npc = cluster == 16 ? 1 : 2;
   const int rg = cluster_rg(G);
   constexpr size_t kMax = 227 * 1024;
   for (int st = kMaxStages; st >= 2; --st) {
@@ -671,7 +738,6 @@ ClusterShape cluster_shape(int cluster, int G, int64_t nq, int Hmax, int depth) 
   if (sh.stages == 0) return sh;
   // no longer a ring than one CTA's weights of the widest layer need
   {
-    const int S = cl_slice(Hmax);
     int64_t groups = 0;                  // ring stages the producer fills, as it groups the chunks
     const int cpg = S <= 64 ? 4 : 2;
     for (int k = 0; k < depth; ++k)
@@ -682,7 +748,7 @@ ClusterShape cluster_shape(int cluster, int G, int64_t nq, int Hmax, int depth) 
       sh.smem = cl_layout(cluster, npc, Hmax, sh.N, static_cast<int>(R), sh.nb, sh.stages, rg).total + 1024;
     }
   }
-  const int MTmax = (cl_slice(Hmax) + 127) / 128;
+  const int MTmax = (S + 127) / 128;
   const int cols = (npc * MTmax + 1) * sh.N;
   int c = 32;
   while (c < cols) c <<= 1;
@@ -694,16 +760,17 @@ ClusterShape cluster_shape(int cluster, int G, int64_t nq, int Hmax, int depth) 
 int cluster_max_active(const ClusterShape& sh, int G) {
   if (!sh.ok) return 0;
   const bool rg2 = cluster_rg(G) == 2;
-  if (sh.cluster == 16) return rg2 ? max_clusters<2, 16>(sh.smem) : max_clusters<4, 16>(sh.smem);
-  return rg2 ? max_clusters<2, 8>(sh.smem) : max_clusters<4, 8>(sh.smem);
+  if (sh.cluster == 16) return rg2 ? max_clusters<2, 16, 1>(sh.smem) : max_clusters<4, 16, 1>(sh.smem);
+  if (sh.npc == 1) return rg2 ? max_clusters<2, 8, 1>(sh.smem) : max_clusters<4, 8, 1>(sh.smem);
+  return rg2 ? max_clusters<2, 8, 2>(sh.smem) : max_clusters<4, 8, 2>(sh.smem);
 }
 
-cudaError_t launch_decode_cluster(const CUtensorMap& tq, const ClusterParams& p, int cluster, int heads, size_t smem,
-                                  cudaStream_t stream) {
+cudaError_t launch_decode_cluster(const ClusterParams& p, const ClusterShape& sh, int heads, cudaStream_t stream) {
   const bool rg2 = cluster_rg(p.G) == 2;
-  if (cluster == 16)
-    return rg2 ? launch_cl<2, 16>(tq, p, heads, smem, stream) : launch_cl<4, 16>(tq, p, heads, smem, stream);
-  return rg2 ? launch_cl<2, 8>(tq, p, heads, smem, stream) : launch_cl<4, 8>(tq, p, heads, smem, stream);
+  const size_t smem = sh.smem;
+  if (sh.cluster == 16) return rg2 ? launch_cl<2, 16, 1>(p, heads, smem, stream) : launch_cl<4, 16, 1>(p, heads, smem, stream);
+  if (sh.npc == 1) return rg2 ? launch_cl<2, 8, 1>(p, heads, smem, stream) : launch_cl<4, 8, 1>(p, heads, smem, stream);
+  return rg2 ? launch_cl<2, 8, 2>(p, heads, smem, stream) : launch_cl<4, 8, 2>(p, heads, smem, stream);
 }
 
 }  // namespace nectar

@@ -237,18 +237,18 @@ struct ClusterParams {
 };
 struct ClusterShape {
   bool ok;
-  int cluster, N, nb, stages, tmem_cols;
+  int cluster, npc, N, nb, stages, tmem_cols;   // npc: nets per CTA (1 or 2)
   size_t smem;
 };
-// Plan of the cluster decode with `cluster` (8 or 16) CTAs per (l, h) for G
-// query heads x nq tokens per KV head; ok = false when it does not apply
+// Plan of the cluster decode with `cluster` (8 or 16) CTAs per (l, h), each
+// holding npc of the two nets (8 CTAs: 1 or 2; 16 CTAs: 1), for G query
+// heads x nq tokens per KV head; ok = false when it does not apply
 // (more than 64 rows, depth > 4, or the shared memory or TMEM plan does not
 // fit).
-ClusterShape cluster_shape(int cluster, int G, int64_t nq, int Hmax, int depth);
+ClusterShape cluster_shape(int cluster, int npc, int G, int64_t nq, int Hmax, int depth);
 // Clusters of that plan that can be resident on the device at once.
 int cluster_max_active(const ClusterShape& sh, int G);
-cudaError_t launch_decode_cluster(const CUtensorMap& tq, const ClusterParams& p, int cluster, int heads, size_t smem,
-                                  cudaStream_t stream);
+cudaError_t launch_decode_cluster(const ClusterParams& p, const ClusterShape& sh, int heads, cudaStream_t stream);
 
 // Layer-by-layer grouped GEMM path of the module forward (module_gemm.cu),
 // used when a KV head has at least kGemmMinRows query rows.

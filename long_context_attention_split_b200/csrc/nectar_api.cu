@@ -1125,7 +1125,7 @@ namespace {
 // Resident clusters of a cluster-decode plan on the current device, cached.
 int cached_max_active(const ClusterShape& sh, int G) {
   struct Key {
-    int dev, cluster, rg2;
+    int dev, cluster, npc, rg2;
     size_t smem;
     int n;
   };
@@ -1136,18 +1136,21 @@ int cached_max_active(const ClusterShape& sh, int G) {
   const int rg2 = G <= 2 ? 1 : 0;
   std::lock_guard<std::mutex> lk(mu);
   for (const Key& k : cache)
-    if (k.dev == dev && k.cluster == sh.cluster && k.rg2 == rg2 && k.smem == sh.smem) return k.n;
+    if (k.dev == dev && k.cluster == sh.cluster && k.npc == sh.npc && k.rg2 == rg2 && k.smem == sh.smem) return k.n;
   const int n = cluster_max_active(sh, G);
-  cache.push_back(Key{dev, sh.cluster, rg2, sh.smem, n});
+  cache.push_back(Key{dev, sh.cluster, sh.npc, rg2, sh.smem, n});
   return n;
 }
 
-// The cluster size (8 or 16) the decode takes, or 0 for the one-launch
-// kernel.  NECTAR_DECODE_CLUSTER=0 never takes the cluster decode, =8 or
-// =16 takes that size whenever it applies; unset: with at most
-// NECTAR_CLUSTER_MAX_HEADS (l, h) pairs, 8-CTA clusters (both nets per CTA;
-// measured faster than 16 on one Qwen3-1.7B layer: 17.4 against 27.4 us per
-// layer in a graph), or 16-CTA ones where only those fit.
+// The cluster plan the decode takes; returns its size (8 or 16), or 0 for
+// the one-launch kernel.  NECTAR_DECODE_CLUSTER=0 never takes the cluster
+// decode, =8 or =16 takes that size whenever it applies (with
+// NECTAR_DECODE_CLUSTER_NETS=1 or 2 nets per CTA for size 8; default 1);
+// unset: with at most NECTAR_CLUSTER_MAX_HEADS (l, h) pairs, the first plan
+// that applies of: 8 CTAs holding one net each (4 slices per net), 8 CTAs
+// holding both nets (8 slices), 16 CTAs holding one net each.  On one
+// Qwen3-1.7B layer in a graph: 17.4 us with both nets per CTA against
+// 27.4 with 16 CTAs, whose non-portable clusters do not all fit at once.
 int cluster_decode_size(const nectar_dims& dims, int64_t nq, const Arch& ar, int Hmax, ClusterShape* out) {
   if (ar.general || static_cast<int64_t>(dims.G) * nq > 64) return 0;
   const char* env = getenv("NECTAR_DECODE_CLUSTER");
@@ -1155,15 +1158,18 @@ int cluster_decode_size(const nectar_dims& dims, int64_t nq, const Arch& ar, int
   if (mode == 0) return 0;
   const int64_t heads = static_cast<int64_t>(dims.L) * dims.Hkv;
   if (mode == 8 || mode == 16) {
-    *out = cluster_shape(mode, dims.G, nq, Hmax, ar.Ds);
+    const char* envn = getenv("NECTAR_DECODE_CLUSTER_NETS");
+    const int npc = mode == 16 ? 1 : ((envn != nullptr && envn[0] == '2') ? 2 : 1);
+    *out = cluster_shape(mode, npc, dims.G, nq, Hmax, ar.Ds);
     return out->ok && cached_max_active(*out, dims.G) > 0 ? mode : 0;
   }
   if (heads > NECTAR_CLUSTER_MAX_HEADS) return 0;
-  for (const int size : {8, 16}) {
-    const ClusterShape sh = cluster_shape(size, dims.G, nq, Hmax, ar.Ds);
+  const int plans[3][2] = {{8, 1}, {8, 2}, {16, 1}};
+  for (const auto& pl : plans) {
+    const ClusterShape sh = cluster_shape(pl[0], pl[1], dims.G, nq, Hmax, ar.Ds);
     if (sh.ok && cached_max_active(sh, dims.G) > 0) {
       *out = sh;
-      return size;
+      return pl[0];
     }
   }
   return 0;
@@ -1257,14 +1263,7 @@ nectar_status decode_impl(nectar_dims dims, const nectar_module_set* mods, const
       c.layer_base[l] = p.layer_base[l];
       c.order[l] = p.order[l];
     }
-    // queries: [heads][G][nq][128]; box = 64 columns x all nq tokens x G heads x 1
-    CUtensorMap tqc;
-    const cuuint64_t dimsq[4] = {128, static_cast<cuuint64_t>(nq), static_cast<cuuint64_t>(dims.G),
-                                 static_cast<cuuint64_t>(heads)};
-    const cuuint64_t strq[3] = {256, static_cast<cuuint64_t>(nq) * 256, static_cast<cuuint64_t>(nq) * 256 * dims.G};
-    const cuuint32_t boxq[4] = {64, static_cast<cuuint32_t>(nq), static_cast<cuuint32_t>(dims.G), 1};
-    NECTAR_TRY(make_tmap(&tqc, Q, 4, dimsq, strq, boxq, "queries (cluster decode)"));
-    cudaError_t e = launch_decode_cluster(tqc, c, csize, static_cast<int>(heads), cs.smem, st);
+    cudaError_t e = launch_decode_cluster(c, cs, static_cast<int>(heads), st);
     return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "cluster decode kernel");
   }
   p.a_out = reinterpret_cast<float*>(base);

@@ -249,6 +249,21 @@ __device__ __forceinline__ void st_cluster_v4f(uint32_t addr, float a, float b, 
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
 }
+// Store 16 bytes into another CTA of the cluster (addr and its mbarrier
+// `bar` are shared::cluster addresses from mapa); the store completes 16
+// bytes of transactions on that mbarrier.  Issued by the thread itself, so
+// it does not queue behind the CTA's bulk copies.
+__device__ __forceinline__ void st_async_v4(uint32_t addr, uint4 v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+               ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
 // Copy `bytes` of this CTA's shared memory into another CTA of the cluster
 // (dst and its mbarrier `bar` are shared::cluster addresses from mapa); the
 // copy completes `bytes` of transactions on that mbarrier.  A plain
@@ -327,6 +342,11 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   d |= uint64_t(2) << 61;
   return d;
 }
+
+// The descriptor `base` (built with start address 0) at shared address
+// saddr: the start-address field is the low 14 bits, and a shared-memory
+// address (< 256 KB) shifted right by 4 fits them, so this is one add.
+__device__ __forceinline__ uint64_t sdesc_at(uint64_t base, uint32_t saddr) { return base + (saddr >> 4); }
 
 // 32 lanes x 32 columns of 32-bit TMEM -> 32 registers per thread.
 #define NECTAR_TMEM_LD32(taddr, r)                                                               \

@@ -512,12 +512,16 @@ def test_decode_shapes(kw):
     decode_case(wl)
 
 
-# The cluster decode (one 8-CTA cluster per (l, h), hidden units sliced over
-# the cluster, merge in-cluster) on the shapes it takes: at most 64 rows per
-# KV head.  Widths cover 64-unit slices (512), partial and empty slices (208:
-# 4 of 8 CTAs hold units, the last 16), 128-unit slices (1024) next to a
-# layer held by one CTA (64), depths 1 and 3 (no exchange; two h buffers),
-# G = 12 (three head blocks of the local warps), 64 rows (N = 64).
+# The cluster decode (one cluster per (l, h), hidden units sliced over the
+# CTAs holding each net, merge in-cluster) on the shapes it takes: at most 64
+# rows per KV head, in its three plans (8 CTAs with one net each: 4 slices
+# per net; 8 CTAs with both nets: 8 slices; 16 CTAs with one net each).
+# Widths cover 64- and 128-unit slices (512), partial and empty slices (208),
+# 128- and 256-unit slices (1024) next to a layer held by one CTA (64), a
+# 512-unit slice (2048: four M tiles per CTA), slices that start inside a
+# 128-row weight tile (768 and 1152), depths 1 and 3 (no exchange;
+# two h buffers), G = 12 (three head blocks of the local warps), 64 rows
+# (N = 64).
 @pytest.mark.parametrize("kw", [
     dict(L=2, Hkv=2, G=2, n=16, B=3, T=40, widths=[512, 512]),
     dict(L=1, Hkv=2, G=7, n=16, B=2, T=33, widths=[208]),
@@ -527,10 +531,14 @@ def test_decode_shapes(kw):
     dict(L=1, Hkv=1, G=12, n=16, B=4, T=45, widths=[128]),
     dict(L=1, Hkv=2, G=16, n=16, B=4, T=300, widths=[256]),
     dict(L=2, Hkv=2, G=2, n=16, B=1, T=512, widths=[512, 512]),     # the headline's shape per layer
+    dict(L=1, Hkv=1, G=4, n=16, B=2, T=64, widths=[2048]),
+    dict(L=2, Hkv=1, G=2, n=16, B=2, T=40, widths=[768, 1152]),   # slices that start inside a 128-row tile
 ])
-@pytest.mark.parametrize("cluster", ["8", "16"])
+@pytest.mark.parametrize("cluster", ["8:1", "8:2", "16:1"])
 def test_decode_cluster_shapes(kw, cluster, monkeypatch):
-    monkeypatch.setenv("NECTAR_DECODE_CLUSTER", cluster)
+    size, nets = cluster.split(":")
+    monkeypatch.setenv("NECTAR_DECODE_CLUSTER", size)
+    monkeypatch.setenv("NECTAR_DECODE_CLUSTER_NETS", nets)
     wl = make_workload("qwen3_1p7b", seed=7, key_scale=None, **kw)
     wl.local_len = torch.randint(0, wl.T + 1, (wl.B,), generator=torch.Generator().manual_seed(5)).to(torch.int32)
     wl.q_pos = (wl.local_len[wl.q_seq.long()] - 1).clamp(min=0).to(torch.int32)
@@ -545,8 +553,10 @@ def test_decode_cluster_matches_one_launch(monkeypatch):
     args = (cuda(wl.Q), cuda(wl.q_seq), cuda(wl.q_pos), cuda(wl.Kloc), cuda(wl.Vloc), cuda(wl.local_len))
     monkeypatch.setenv("NECTAR_DECODE_CLUSTER", "0")
     o0 = nx.decode(mods, *args)
-    for cluster in ("8", "16"):
-        monkeypatch.setenv("NECTAR_DECODE_CLUSTER", cluster)
+    for cluster in ("8:1", "8:2", "16:1"):
+        size, nets = cluster.split(":")
+        monkeypatch.setenv("NECTAR_DECODE_CLUSTER", size)
+        monkeypatch.setenv("NECTAR_DECODE_CLUSTER_NETS", nets)
         o1 = nx.decode(mods, *args)
         l1 = nx.decode_layer_out(mods, *args)
         torch.cuda.synchronize()
