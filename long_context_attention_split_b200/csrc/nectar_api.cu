@@ -1024,14 +1024,18 @@ nectar_status prepare_modules(const nectar_dims& dims, const nectar_module_set* 
   if (sh->smem > 227 * 1024) return fail(NECTAR_ERR_UNSUPPORTED, "width %d needs too much shared memory", Hmax);
   if (sh->tmem_cols > 512)
     return fail(NECTAR_ERR_UNSUPPORTED, "width %d with G = %d needs more than 512 TMEM columns", Hmax, dims.G);
-  // one CTA per net when every layer's net streams at least 1 MB of weights:
-  // then the two streams side by side on different SMs outweigh the extra
-  // CTA start-up (measured: H = 720 / 912 gains 8 %, H = 512 loses 3 %)
+  // one CTA per net when every layer's net streams at least 256 KB of
+  // weights: the two streams then run side by side on different SMs, and
+  // the smaller CTAs even out the bytes per SM (measured with the module
+  // CTAs first in the decode grid: Qwen3-1.7B, H = 512, 95.6 -> 89.8 us;
+  // Llama-8B b = 1 at rho = 10 %, 185 -> 169 us)
   {
     int64_t min_net = INT64_MAX;
     for (int l = 0; l < dims.L; ++l)
       min_net = std::min(min_net, layout::net_elems(ar.ws[l], ar.Ds, 1) * 2);
-    p->net_split = min_net >= (int64_t(1) << 20) ? 1 : 0;
+    p->net_split = min_net >= (int64_t(256) << 10) ? 1 : 0;
+    const char* ns = getenv("NECTAR_NET_SPLIT");   // =0 or =1 overrides the choice
+    if (ns != nullptr && (ns[0] == '0' || ns[0] == '1')) p->net_split = ns[0] - '0';
   }
   p->N = sh->N;
   p->TPC = sh->TPC;
@@ -1274,15 +1278,16 @@ nectar_status decode_impl(nectar_dims dims, const nectar_module_set* mods, const
                            : reinterpret_cast<float*>(base + decode_ws_a_bytes(rows) +
                                                       align256(static_cast<size_t>(rows) * (kD + 2) * sizeof(float)));
   const int units = (p.net_split ? 2 : 1) * dims.L * dims.Hkv * sh.nblk;
-  // local CTAs last when each streams under a tenth of a module CTA's
-  // weights (measured: 4-7 % faster on llama8b_sweep b = 1 with 128 local
-  // tokens; with 512 local tokens, qwen3_1p7b, first is 1 % faster)
+  // Module CTAs first in the grid, local CTAs after them.  With the local
+  // CTAs first the block scheduler was seen to place one CTA per SM until
+  // the first ones ended (a per-CTA timeline of the Qwen3-1.7B decode: 148
+  // local CTAs resident for the first 16 us, then the module CTAs), which
+  // left the SMs' second slots and most of HBM idle; module CTAs first:
+  // 102.5 -> 96.0 us in the bench step.  NECTAR_DECODE_ORDER=local puts the
+  // local CTAs first.
   {
-    int64_t wsum = 0;
-    for (int l = 0; l < dims.L; ++l) wsum += arch_head_elems(ar, l) * 2;
-    const int64_t module_bytes = wsum / dims.L / (p.net_split ? 2 : 1);
-    const int64_t local_bytes = static_cast<int64_t>(T_max) * kD * 2 * 2;
-    p.module_first = local_bytes * 10 < module_bytes ? 1 : 0;
+    const char* ord = getenv("NECTAR_DECODE_ORDER");
+    p.module_first = (ord != nullptr && ord[0] == 'l') ? 0 : 1;
   }
   cudaError_t e = launch_decode(tq, p, units, sh.smem, st);
   return e == cudaSuccess ? NECTAR_OK : cuda_fail(e, "decode kernels");
