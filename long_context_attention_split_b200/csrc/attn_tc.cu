@@ -31,7 +31,13 @@
 // second softmax warpgroup idle; its key range is then split between the
 // two warpgroups (interleaved in the K / V ring, both reading query tile
 // 0), and warpgroup 1 hands its (m, l, O) to warpgroup 0 through shared
-// memory at the end of the unit.
+// memory at the end of the unit.  With at most 64 rows (kDup), rows 64..127
+// of the query tile repeat rows 0..63, and the thread of row r scores only
+// the keys [32 h, 32 h + 32) of each key tile, h = r / 64: P row r holds
+// that half's weights and zeros elsewhere, so O rows r and r + 64 are two
+// partial states of one query row, joined by log-sum-exp at the end of the
+// unit.  Each softmax thread then does half the work of a full tile, none
+// of it on padding rows.
 //
 // Warps: 0..3 softmax / epilogue of query tile 0, 4..7 of tile 1 (thread =
 // row = TMEM lane), 8 Q and K producer, 9 V producer, 10 MMA issuer.
@@ -54,6 +60,14 @@ constexpr int kTcKeys = 64;                        // keys per tile
 // slower (the special-function unit is not its limit)
 constexpr int kTcPolyPairs = NECTAR_TC_POLY_PAIRS;
 constexpr int kTcStages = 3;                       // K and V ring depth
+#ifndef NECTAR_TC_PV_LAG
+#define NECTAR_TC_PV_LAG 1
+#endif
+// key tiles by which the P V products trail the S products (1: P V of a
+// tile right after the S of the next; 2 measured 1-3 % slower on every
+// tensor-core workload)
+constexpr int kPvLag = NECTAR_TC_PV_LAG;
+static_assert(kPvLag >= 1 && kPvLag < kTcStages, "the V ring holds the trailing tiles");
 constexpr int kTcThreads = 11 * 32;
 constexpr uint32_t kQBytes = kTcRows * kD * 2;     // 32 KB
 constexpr uint32_t kKVBytes = kTcKeys * kD * 2;    // 16 KB
@@ -67,6 +81,12 @@ struct TcSmem {
   static constexpr uint32_t xml = p + 4 * kPBytes;                  // split units: (m, l) of warpgroup 1
   static constexpr uint32_t bars = xml + 2 * kTcRows * 4;           // 40 barriers
   static constexpr uint32_t tslot = bars + 40 * 8;
+  // K / V ring stage s (s < kTcStages: its own area; s = kTcStages: the
+  // second query tile's area, free in the one-query-tile instance)
+  static __device__ __forceinline__ uint32_t k_at(int s) { return s < kTcStages ? k + s * kKVBytes : q + kQBytes; }
+  static __device__ __forceinline__ uint32_t v_at(int s) {
+    return s < kTcStages ? v + s * kKVBytes : q + kQBytes + kKVBytes;
+  }
   static constexpr uint32_t total = tslot + 16;
 };
 
@@ -244,10 +264,65 @@ __device__ __noinline__ void tc_unit_epilogue_split(const TcParams& p, uint8_t* 
   tc_unit_epilogue<true>(p, smem, tO, b_ofree_t, sg, split, t, row, m, l, ok, c);
 }
 
+// kDup, end of a unit for softmax warpgroup t (its last P V complete):
+// fold row r + 64's partial state (the keys of the second half) into row
+// r -- its O row and (m, l) through this warpgroup's own P buffers (free
+// now), then log-sum-exp.  Returns row r's joined (m, l); O rows 0..63 of
+// the tile hold the joined state.  Out of line, as the split hand-off: it
+// would take registers from the softmax loop.
+__device__ __noinline__ float2 tc_dup_fold(uint8_t* smem, uint32_t tO, int t, int row, float m, float l) {
+  float4* park = reinterpret_cast<float4*>(smem + TcSmem::p + 2 * t * kPBytes);   // 64 rows x 512 B
+  float* xm = reinterpret_cast<float*>(smem + TcSmem::xml) + t * kTcRows;
+  const int q = row & 63;
+  if (row >= 64) {
+#pragma unroll
+    for (int cb = 0; cb < kD; cb += 16) {
+      uint32_t v[16];
+      NECTAR_TMEM_LD16(tO + cb, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4)
+        park[q * (kD / 4) + (((cb >> 2) + q4) ^ (q & 31))] =
+            make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]), __uint_as_float(v[4 * q4 + 2]),
+                        __uint_as_float(v[4 * q4 + 3]));
+    }
+    xm[q] = m;
+    xm[64 + q] = l;
+  }
+  named_bar_sync(2 + t, kTcRows);
+  if (row < 64) {
+    const float m1 = xm[q], l1 = xm[64 + q];
+    const float M = fmaxf(m, m1);
+    const float w0 = exp2_shift(m, M), w1 = exp2_shift(m1, M);
+    l = w0 * l + w1 * l1;
+    m = M;
+#pragma unroll
+    for (int cb = 0; cb < kD; cb += 32) {
+      uint32_t v[32];
+      NECTAR_TMEM_LD32(tO + cb, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 o1 = park[q * (kD / 4) + (((cb >> 2) + q4) ^ (q & 31))];
+        v[4 * q4] = __float_as_uint(w0 * __uint_as_float(v[4 * q4]) + w1 * o1.x);
+        v[4 * q4 + 1] = __float_as_uint(w0 * __uint_as_float(v[4 * q4 + 1]) + w1 * o1.y);
+        v[4 * q4 + 2] = __float_as_uint(w0 * __uint_as_float(v[4 * q4 + 2]) + w1 * o1.z);
+        v[4 * q4 + 3] = __float_as_uint(w0 * __uint_as_float(v[4 * q4 + 3]) + w1 * o1.w);
+      }
+      NECTAR_TMEM_ST32(tO + cb, v);
+    }
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  named_bar_sync(2 + t, kTcRows);       // the parked rows are read
+  tc_fence_after();
+  return make_float2(m, l);
+}
+
 // kSplit: units with one query tile split their keys between the two
 // softmax warpgroups (compiled only into the instance used when every unit
 // has one query tile: the hand-off costs registers)
-template <bool kSplit>
+template <bool kSplit, bool kDup>
 __global__ void __launch_bounds__(kTcThreads, 1)
 cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const TcParams p) {
@@ -255,14 +330,19 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TcSmem::bars);
   const uint32_t b_qfull = smem_u32(bars + 0), b_qempty = smem_u32(bars + 1);
-  const uint32_t b_kfull = smem_u32(bars + 2), b_kempty = smem_u32(bars + 5);     // [3]
-  const uint32_t b_vfull = smem_u32(bars + 8), b_vempty = smem_u32(bars + 11);    // [3]
+  // K / V ring depth: one more stage in the one-query-tile instance, in the
+  // unused second query tile (a head of <= 128 rows streams its K / V at
+  // HBM speed there, so more bytes in flight)
+  constexpr int kSt = kSplit ? kTcStages + 1 : kTcStages;
+  const uint32_t b_kfull = smem_u32(bars + 2), b_kempty = smem_u32(bars + 6);     // [4]
+  const uint32_t b_vfull = smem_u32(bars + 10), b_vempty = smem_u32(bars + 14);   // [4]
   // [tile t][buf b] at + 8 * (2 t + b)
-  const uint32_t b_sfull = smem_u32(bars + 14), b_sfree = smem_u32(bars + 18);
-  const uint32_t b_pfull = smem_u32(bars + 22), b_pvdone = smem_u32(bars + 26);
-  const uint32_t b_ofree = smem_u32(bars + 30);                                   // [tile]
+  const uint32_t b_sfull = smem_u32(bars + 18), b_sfree = smem_u32(bars + 22);
+  const uint32_t b_pfull = smem_u32(bars + 26), b_pvdone = smem_u32(bars + 30);
+  const uint32_t b_ofree = smem_u32(bars + 34);                                   // [tile]
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + TcSmem::tslot);
 
+  static_assert(kSplit || !kDup, "repeated rows only in the one-query-tile instance");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x;
   const int nseg = tc_num_segs(p, c);
@@ -270,7 +350,7 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
   if (threadIdx.x == 0) {
     mbar_init(b_qfull, 1);
     mbar_init(b_qempty, 1);
-    for (int s = 0; s < kTcStages; ++s) {
+    for (int s = 0; s < kSt; ++s) {
       mbar_init(b_kfull + 8 * s, 1);
       mbar_init(b_kempty + 8 * s, 1);
       mbar_init(b_vfull + 8 * s, 1);
@@ -317,17 +397,26 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         if (qn > 0 && !(ok = mbar_wait(b_qempty, (qn - 1) & 1, p.err))) break;
         const bool two = two_tiles(sg.unit);
         mbar_arrive_expect_tx(b_qfull, (two ? 2 : 1) * kQBytes);
-        tma_load_4d(smem_u32(smem + TcSmem::q), &tmap_q, 0, qp * kTcUnitRows, 0, static_cast<int>(hd), b_qfull, pol_q);
+        if constexpr (kDup) {
+          // rows 0..63 of each 64-column half, twice (box: 64 rows, one half)
+#pragma unroll
+          for (int hq = 0; hq < 4; ++hq)
+            tma_load_4d(smem_u32(smem + TcSmem::q + hq * (kQBytes / 4)), &tmap_q, 0, qp * kTcUnitRows, hq >> 1,
+                        static_cast<int>(hd), b_qfull, pol_q);
+        } else {
+          tma_load_4d(smem_u32(smem + TcSmem::q), &tmap_q, 0, qp * kTcUnitRows, 0, static_cast<int>(hd), b_qfull,
+                      pol_q);
+        }
         if (two)
           tma_load_4d(smem_u32(smem + TcSmem::q + kQBytes), &tmap_q, 0, qp * kTcUnitRows + kTcRows, 0,
                       static_cast<int>(hd), b_qfull, pol_q);
         ++qn;
         for (int64_t i = 0; i < sg.k1 - sg.k0; ++i, ++it) {
           const int64_t kt = tc_item<kSplit>(sg, two, i).kt;
-          const uint32_t s = it % kTcStages;
-          if (it >= kTcStages && !(ok = mbar_wait(b_kempty + 8 * s, ((it / kTcStages) - 1) & 1, p.err))) break;
+          const uint32_t s = it % kSt;
+          if (it >= kSt && !(ok = mbar_wait(b_kempty + 8 * s, ((it / kSt) - 1) & 1, p.err))) break;
           mbar_arrive_expect_tx(b_kfull + 8 * s, kKVBytes);
-          tma_load_4d(smem_u32(smem + TcSmem::k + s * kKVBytes), &tmap_k, 0, static_cast<int>(kt * kTcKeys), 0,
+          tma_load_4d(smem_u32(smem + TcSmem::k_at(s)), &tmap_k, 0, static_cast<int>(kt * kTcKeys), 0,
                       static_cast<int>(hd), b_kfull + 8 * s, pol_kv);
         }
       }
@@ -345,10 +434,10 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         const bool two = two_tiles(sg.unit);
         for (int64_t i = 0; i < sg.k1 - sg.k0; ++i, ++it) {
           const int64_t kt = tc_item<kSplit>(sg, two, i).kt;
-          const uint32_t s = it % kTcStages;
-          if (it >= kTcStages && !(ok = mbar_wait(b_vempty + 8 * s, ((it / kTcStages) - 1) & 1, p.err))) break;
+          const uint32_t s = it % kSt;
+          if (it >= kSt && !(ok = mbar_wait(b_vempty + 8 * s, ((it / kSt) - 1) & 1, p.err))) break;
           mbar_arrive_expect_tx(b_vfull + 8 * s, kKVBytes);
-          tma_load_4d(smem_u32(smem + TcSmem::v + s * kKVBytes), &tmap_v, 0, static_cast<int>(kt * kTcKeys), 0,
+          tma_load_4d(smem_u32(smem + TcSmem::v_at(s)), &tmap_v, 0, static_cast<int>(kt * kTcKeys), 0,
                       static_cast<int>(hd), b_vfull + 8 * s, pol_kv);
         }
       }
@@ -365,8 +454,8 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
       uint32_t un[2] = {0, 0};   // units whose O was started, per query tile
       // O_t += P_t V for the ring entry `vit`, for every warpgroup t in mask
       auto issue_pv = [&](uint32_t vit, uint32_t mask, bool first) {
-        const uint32_t vs = vit % kTcStages;
-        if (ok) ok = mbar_wait(b_vfull + 8 * vs, (vit / kTcStages) & 1, p.err);
+        const uint32_t vs = vit % kSt;
+        if (ok) ok = mbar_wait(b_vfull + 8 * vs, (vit / kSt) & 1, p.err);
         for (int t = 0; t < 2; ++t) {
           if (!(mask >> t & 1u)) continue;
           const uint32_t b = cp[t] & 1;
@@ -377,7 +466,7 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
           if (!ok) continue;
           tc_fence_after();
           const uint32_t pa = smem_u32(smem + TcSmem::p + (2 * t + b) * kPBytes);
-          const uint32_t vb = smem_u32(smem + TcSmem::v + vs * kKVBytes);
+          const uint32_t vb = smem_u32(smem + TcSmem::v_at(vs));
 #pragma unroll
           for (int kk = 0; kk < kTcKeys / 16; ++kk) {
             // A = P (K-major, one 64-key chunk): keys 16 kk.. at byte 32 kk.
@@ -390,8 +479,14 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         }
         mma_commit(b_vempty + 8 * vs);
       };
-      uint32_t prev_mask = 0;
-      bool prev_first = false, have_prev = false;
+      // the P V products trail the S products by kPvLag key tiles, so that
+      // the S of the next tiles is not held up behind a softmax
+      struct PendPv {
+        uint32_t vit, mask;
+        bool first;
+      };
+      PendPv pend[kPvLag];
+      int npend = 0;
       for (int si = 0; si < nseg && ok; ++si) {
         const TcSeg sg = tc_seg(p, c, si);
         const bool two = two_tiles(sg.unit);
@@ -400,8 +495,8 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         const int64_t nit = sg.k1 - sg.k0;
         for (int64_t i = 0; i < nit && ok; ++i, ++it) {
           const TcItem itm = tc_item<kSplit>(sg, two, i);
-          const uint32_t ks = it % kTcStages;
-          if (!(ok = mbar_wait(b_kfull + 8 * ks, (it / kTcStages) & 1, p.err))) break;
+          const uint32_t ks = it % kSt;
+          if (!(ok = mbar_wait(b_kfull + 8 * ks, (it / kSt) & 1, p.err))) break;
           for (int t = 0; t < 2 && ok; ++t) {
             if (!(itm.mask >> t & 1u)) continue;
             const uint32_t b = cs[t] & 1;
@@ -409,7 +504,7 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
             tc_fence_after();
             // one query tile (split or not): both warpgroups read tile 0
             const uint32_t qa = smem_u32(smem + TcSmem::q + (two ? t : 0) * kQBytes);
-            const uint32_t kb = smem_u32(smem + TcSmem::k + ks * kKVBytes);
+            const uint32_t kb = smem_u32(smem + TcSmem::k_at(ks));
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               // d 16 kk..: half kk / 4, byte (kk % 4) * 32 inside the 128-B rows
@@ -422,13 +517,16 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
           }
           mma_commit(b_kempty + 8 * ks);
           if (i + 1 == nit) mma_commit(b_qempty);
-          if (have_prev) issue_pv(it - 1, prev_mask, prev_first);
-          prev_mask = itm.mask;
-          prev_first = itm.first;
-          have_prev = true;
+          if (npend == kPvLag) {
+            issue_pv(pend[0].vit, pend[0].mask, pend[0].first);
+#pragma unroll
+            for (int q = 1; q < kPvLag; ++q) pend[q - 1] = pend[q];
+            --npend;
+          }
+          pend[npend++] = PendPv{it, itm.mask, itm.first};
         }
       }
-      if (ok && have_prev) issue_pv(it - 1, prev_mask, prev_first);
+      for (int q = 0; q < npend && ok; ++q) issue_pv(pend[q].vit, pend[q].mask, pend[q].first);
     }
   } else {
     // --------------------- softmax + epilogue (tile t) ---------------------
@@ -455,13 +553,17 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         tc_fence_after();
         // a whole tile of valid keys (every tile but a head's last): keep
         // the raw scores, take the max on them and fold the scale into the
-        // exponent's FMA; the last tile scales and masks element by element
-        const bool full = nvalid >= kTcKeys;
-        float sc[kTcKeys];
+        // exponent's FMA; the last tile scales and masks element by element.
+        // kDup: this thread's columns are the 32 keys of its half hh.
+        constexpr int kCols = kDup ? kTcKeys / 2 : kTcKeys;
+        const int hh = kDup ? (row >> 6) : 0;
+        const int64_t nv = nvalid - hh * kCols;          // valid keys among this thread's columns
+        const bool full = nv >= kCols;
+        float sc[kCols];
 #pragma unroll
-        for (int cb = 0; cb < kTcKeys; cb += 32) {
+        for (int cb = 0; cb < kCols; cb += 32) {
           uint32_t v[32];
-          NECTAR_TMEM_LD32(tS + 64 * b + lane_base + cb, v);
+          NECTAR_TMEM_LD32(tS + 64 * b + lane_base + hh * kCols + cb, v);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) sc[cb + e] = __uint_as_float(v[e]);
@@ -475,14 +577,14 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
           float x0 = sc[0], x1 = sc[1];
           if (p.qmul >= 0.f) {
 #pragma unroll
-            for (int e = 2; e < kTcKeys; e += 2) {
+            for (int e = 2; e < kCols; e += 2) {
               x0 = fmaxf(x0, sc[e]);
               x1 = fmaxf(x1, sc[e + 1]);
             }
             bm = fmaxf(x0, x1) * p.qmul;
           } else {
 #pragma unroll
-            for (int e = 2; e < kTcKeys; e += 2) {
+            for (int e = 2; e < kCols; e += 2) {
               x0 = fminf(x0, sc[e]);
               x1 = fminf(x1, sc[e + 1]);
             }
@@ -490,8 +592,8 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < kTcKeys; ++e) {
-            sc[e] = (e < nvalid) ? sc[e] * p.qmul : -INFINITY;
+          for (int e = 0; e < kCols; ++e) {
+            sc[e] = (e < nv) ? sc[e] * p.qmul : -INFINITY;
             bm = fmaxf(bm, sc[e]);
           }
         }
@@ -525,10 +627,11 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         // the row sum adds the rounded weights that P V uses; full tiles and
         // the last (masked) tile in separate loops, so that the unrolled
         // loop body carries no per-pair branch
+        const int col0 = hh * kCols;
         if (full) {
           const float2 q2 = make_float2(p.qmul, p.qmul), nm2 = make_float2(-m, -m);
 #pragma unroll
-          for (int c8 = 0; c8 < kTcKeys / 8; ++c8) {
+          for (int c8 = 0; c8 < kCols / 8; ++c8) {
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -539,19 +642,25 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
               else w[e] = pack_bf16x2(ex2(x.x), ex2(x.y));
               rs2[e & 1] = fadd2(rs2[e & 1], make_float2(bf16lo(w[e]), bf16hi(w[e])));
             }
-            *reinterpret_cast<uint4*>(pt + p_off(row, c8 * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(pt + p_off(row, col0 + c8 * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         } else {
 #pragma unroll
-          for (int c8 = 0; c8 < kTcKeys / 8; ++c8) {
+          for (int c8 = 0; c8 < kCols / 8; ++c8) {
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               w[e] = pack_bf16x2(exp2_shift(sc[c8 * 8 + 2 * e], m), exp2_shift(sc[c8 * 8 + 2 * e + 1], m));
               rs2[e & 1] = fadd2(rs2[e & 1], make_float2(bf16lo(w[e]), bf16hi(w[e])));
             }
-            *reinterpret_cast<uint4*>(pt + p_off(row, c8 * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(pt + p_off(row, col0 + c8 * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
+        }
+        if constexpr (kDup) {
+          // the other half's keys carry no weight in this row
+#pragma unroll
+          for (int c8 = 0; c8 < kCols / 8; ++c8)
+            *reinterpret_cast<uint4*>(pt + p_off(row, (kCols - col0) + c8 * 8)) = make_uint4(0, 0, 0, 0);
         }
         l += (rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y);
         fence_proxy_async_smem();
@@ -562,6 +671,11 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
       const uint32_t pc = cnt - 1;
       if (ok) ok = mbar_wait(b_pvdone + 8 * (2 * t + (pc & 1)), (pc >> 1) & 1, p.err);
       tc_fence_after();
+      if constexpr (kDup) {
+        const float2 ml = tc_dup_fold(smem, tO + lane_base, t, row, m, l);
+        m = ml.x;
+        l = ml.y;
+      }
       if constexpr (kSplit) {
         tc_unit_epilogue_split(p, smem, tmem + 256 + 128 * t + lane_base, b_ofree + 8 * t, sg, split, t, row, m, l,
                                ok, c);
@@ -642,19 +756,33 @@ TcPlan plan_tc(int heads, int64_t n, int64_t rows, int num_sms) {
   return pl;
 }
 
+// At most 64 rows per head: the one-query-tile instance with the rows
+// repeated and the keys of each tile halved between a row's two threads.
+// NECTAR_TC_DUP=0 keeps one thread per row over all 64 keys of a tile.
+bool cache_attn_tc_dup(int64_t rows) {
+  const char* e = getenv("NECTAR_TC_DUP");
+  return rows <= kTcRows / 2 && !(e != nullptr && e[0] == '0');
+}
+
+template <bool kSplit, bool kDup>
+static cudaError_t launch_tc_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const TcParams& p,
+                               size_t smem, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(cache_attn_tc_kernel<kSplit, kDup>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  cache_attn_tc_kernel<kSplit, kDup><<<p.C, kTcThreads, smem, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_cache_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                  const TcParams& p, cudaStream_t stream) {
   const size_t smem = TcSmem::total + 1024;
-  // every unit has one query tile when a head has at most 128 rows
+  // every unit has one query tile when a head has at most 128 rows; the
+  // query tensor map's box is 64 rows when the rows are repeated
   const bool split = p.rows_total <= kTcRows;
-  cudaError_t e = split ? cudaFuncSetAttribute(cache_attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(smem))
-                        : cudaFuncSetAttribute(cache_attn_tc_kernel<false>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  if (split) cache_attn_tc_kernel<true><<<p.C, kTcThreads, smem, stream>>>(tq, tk, tv, p);
-  else cache_attn_tc_kernel<false><<<p.C, kTcThreads, smem, stream>>>(tq, tk, tv, p);
-  e = cudaGetLastError();
+  cudaError_t e = !split ? launch_tc_t<false, false>(tq, tk, tv, p, smem, stream)
+                  : cache_attn_tc_dup(p.rows_total) ? launch_tc_t<true, true>(tq, tk, tv, p, smem, stream)
+                                                    : launch_tc_t<true, false>(tq, tk, tv, p, smem, stream);
   if (e != cudaSuccess) return e;
   if (p.sk_units == 0) return cudaSuccess;
   const int64_t warps = static_cast<int64_t>(p.heads) * p.rows_total;

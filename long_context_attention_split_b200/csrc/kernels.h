@@ -153,6 +153,8 @@ struct TcPlan {
   size_t ws_bytes, smem;
 };
 TcPlan plan_tc(int heads, int64_t n, int64_t rows, int num_sms);
+// the query map's box is {64, 64, 1, 1} when this is true, else {64, 128, 2, 1}
+bool cache_attn_tc_dup(int64_t rows);
 cudaError_t launch_cache_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                  const TcParams& p, cudaStream_t stream);
 

@@ -340,7 +340,8 @@ nectar_status nectar_cache_attn_lse(nectar_dims dims, const nectar_bf16* K, cons
     const cuuint64_t sq[3] = {256, 128, static_cast<cuuint64_t>(rows) * 256};
     const cuuint64_t dk[4] = {64, static_cast<cuuint64_t>(n), 2, static_cast<cuuint64_t>(heads)};
     const cuuint64_t sk[3] = {256, 128, static_cast<cuuint64_t>(n) * 256};
-    const cuuint32_t boxq[4] = {64, 128, 2, 1};
+    const bool dup = cache_attn_tc_dup(rows);
+    const cuuint32_t boxq[4] = {64, dup ? 64u : 128u, dup ? 1u : 2u, 1};
     const cuuint32_t boxk[4] = {64, 64, 2, 1};
     NECTAR_TRY(make_tmap(&tq, Q, 4, dq, sq, boxq, "Q"));
     NECTAR_TRY(make_tmap(&tk, K, 4, dk, sk, boxk, "K"));

@@ -108,6 +108,29 @@ def test_cache_attn_tct(L, Hkv, G, n, nq, monkeypatch):
         assert np.abs(ag - ag0).max() <= ALPHA_TOL and np.abs(Ag - Ag0).max() <= ATT_TOL * vmax
 
 
+# 33-64 query rows per KV head: the tensor-core kernel with the rows of the
+# query tile repeated, each row's keys of a tile halved between two
+# threads, and the two halves joined at the end.  Cases: both halves of the
+# last tile partly valid, the second half of the last tile empty, one key
+# tile (one warpgroup, no key split), n < 32 (the second half never holds a
+# key), heads cut over CTAs (partials); each also with NECTAR_TC_DUP=0.
+@pytest.mark.parametrize("L,Hkv,G,n,nq", [
+    (1, 2, 3, 700, 11),       # 33 rows, last tile 60 keys
+    (1, 3, 4, 650, 16),       # 64 rows, last tile 10 keys
+    (2, 2, 7, 64, 9),         # 63 rows, exactly one key tile
+    (1, 1, 8, 40, 8),         # 64 rows, n = 40
+    (3, 4, 4, 20000, 16),     # 64 rows, heads cut over CTAs
+])
+def test_cache_attn_tc_repeated_rows(L, Hkv, G, n, nq, monkeypatch):
+    wl, ag, Ag, ao, Ao = run_cache_attn(L, Hkv, G, n, nq, seed=n + 11 * G)
+    vmax = wl.V.float().abs().max().item()
+    check_attn(ag, Ag, ao, Ao, vmax, f"repeated rows n={n}")
+    monkeypatch.setenv("NECTAR_TC_DUP", "0")
+    _, ag0, Ag0, _, _ = run_cache_attn(L, Hkv, G, n, nq, seed=n + 11 * G)
+    check_attn(ag0, Ag0, ao, Ao, vmax, f"one thread per row n={n}")
+    assert np.abs(ag - ag0).max() <= ALPHA_TOL and np.abs(Ag - Ag0).max() <= ATT_TOL * vmax
+
+
 @pytest.mark.parametrize("G,nq", [(5, 1), (4, 16)])
 def test_cache_attn_tct_repeatable(G, nq):
     # a head spread over several CTAs with several tiles each: ten calls give
