@@ -560,13 +560,14 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         const int64_t nv = nvalid - hh * kCols;          // valid keys among this thread's columns
         const bool full = nv >= kCols;
         float sc[kCols];
+        {
+          // every load of the tile issued before the one wait
+          uint32_t v[kCols];
 #pragma unroll
-        for (int cb = 0; cb < kCols; cb += 32) {
-          uint32_t v[32];
-          NECTAR_TMEM_LD32(tS + 64 * b + lane_base + hh * kCols + cb, v);
+          for (int cb = 0; cb < kCols; cb += 32) NECTAR_TMEM_LD32(tS + 64 * b + lane_base + hh * kCols + cb, (v + cb));
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) sc[cb + e] = __uint_as_float(v[e]);
+          for (int e = 0; e < kCols; ++e) sc[e] = __uint_as_float(v[e]);
         }
         tc_fence_before();
         mbar_arrive(b_sfree + 8 * (2 * t + b));
