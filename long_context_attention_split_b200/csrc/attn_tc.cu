@@ -40,7 +40,8 @@
 // of it on padding rows.
 //
 // Warps: 0..3 softmax / epilogue of query tile 0, 4..7 of tile 1 (thread =
-// row = TMEM lane), 8 Q and K producer, 9 V producer, 10 MMA issuer.
+// row = TMEM lane), 8 Q and K producer, 9 V producer, 10 S issuer (and
+// TMEM owner), 11 P V issuer.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -60,15 +61,7 @@ constexpr int kTcKeys = 64;                        // keys per tile
 // slower (the special-function unit is not its limit)
 constexpr int kTcPolyPairs = NECTAR_TC_POLY_PAIRS;
 constexpr int kTcStages = 3;                       // K and V ring depth
-#ifndef NECTAR_TC_PV_LAG
-#define NECTAR_TC_PV_LAG 1
-#endif
-// key tiles by which the P V products trail the S products (1: P V of a
-// tile right after the S of the next; 2 measured 1-3 % slower on every
-// tensor-core workload)
-constexpr int kPvLag = NECTAR_TC_PV_LAG;
-static_assert(kPvLag >= 1 && kPvLag < kTcStages, "the V ring holds the trailing tiles");
-constexpr int kTcThreads = 11 * 32;
+constexpr int kTcThreads = 12 * 32;
 constexpr uint32_t kQBytes = kTcRows * kD * 2;     // 32 KB
 constexpr uint32_t kKVBytes = kTcKeys * kD * 2;    // 16 KB
 constexpr uint32_t kPBytes = kTcRows * kTcKeys * 2;   // 16 KB
@@ -443,50 +436,12 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
       }
     }
   } else if (warp == 10) {
-    // ---------------------------- MMA issuer ----------------------------
+    // ---------------------- S issuer (+ TMEM owner) ----------------------
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, kTcKeys, 0, 0);
-      const uint32_t idesc_o = idesc_bf16_f32(128, kD, 0, 1);
       bool ok = true;
       uint32_t qn = 0, it = 0;
       uint32_t cs[2] = {0, 0};   // S tiles issued per query tile
-      uint32_t cp[2] = {0, 0};   // P V products issued per query tile
-      uint32_t un[2] = {0, 0};   // units whose O was started, per query tile
-      // O_t += P_t V for the ring entry `vit`, for every warpgroup t in mask
-      auto issue_pv = [&](uint32_t vit, uint32_t mask, bool first) {
-        const uint32_t vs = vit % kSt;
-        if (ok) ok = mbar_wait(b_vfull + 8 * vs, (vit / kSt) & 1, p.err);
-        for (int t = 0; t < 2; ++t) {
-          if (!(mask >> t & 1u)) continue;
-          const uint32_t b = cp[t] & 1;
-          if (ok) ok = mbar_wait(b_pfull + 8 * (2 * t + b), (cp[t] >> 1) & 1, p.err);
-          if (ok && first && un[t] > 0) ok = mbar_wait(b_ofree + 8 * t, (un[t] - 1) & 1, p.err);
-          if (first) ++un[t];
-          ++cp[t];
-          if (!ok) continue;
-          tc_fence_after();
-          const uint32_t pa = smem_u32(smem + TcSmem::p + (2 * t + b) * kPBytes);
-          const uint32_t vb = smem_u32(smem + TcSmem::v_at(vs));
-#pragma unroll
-          for (int kk = 0; kk < kTcKeys / 16; ++kk) {
-            // A = P (K-major, one 64-key chunk): keys 16 kk.. at byte 32 kk.
-            // B = V (MN-major): 16 keys = two 8-row groups of 128 B; the two
-            // 64-wide d halves are kKVBytes / 2 apart
-            mma_bf16_ss(tmem + 256 + 128 * t, sdesc_sw128(pa + kk * 32, 16, 1024),
-                        sdesc_sw128(vb + kk * 2048, kKVBytes / 2, 1024), idesc_o, (first && kk == 0) ? 0u : 1u);
-          }
-          mma_commit(b_pvdone + 8 * (2 * t + b));
-        }
-        mma_commit(b_vempty + 8 * vs);
-      };
-      // the P V products trail the S products by kPvLag key tiles, so that
-      // the S of the next tiles is not held up behind a softmax
-      struct PendPv {
-        uint32_t vit, mask;
-        bool first;
-      };
-      PendPv pend[kPvLag];
-      int npend = 0;
       for (int si = 0; si < nseg && ok; ++si) {
         const TcSeg sg = tc_seg(p, c, si);
         const bool two = two_tiles(sg.unit);
@@ -517,16 +472,54 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
           }
           mma_commit(b_kempty + 8 * ks);
           if (i + 1 == nit) mma_commit(b_qempty);
-          if (npend == kPvLag) {
-            issue_pv(pend[0].vit, pend[0].mask, pend[0].first);
-#pragma unroll
-            for (int q = 1; q < kPvLag; ++q) pend[q - 1] = pend[q];
-            --npend;
-          }
-          pend[npend++] = PendPv{it, itm.mask, itm.first};
         }
       }
-      for (int q = 0; q < npend && ok; ++q) issue_pv(pend[q].vit, pend[q].mask, pend[q].first);
+    }
+  } else if (warp == 11) {
+    // ----------------------------- P V issuer -----------------------------
+    // A thread of its own, so that the S of the next key tiles is issued as
+    // soon as its K tile and S buffer are there, not behind a softmax (a
+    // per-tile timeline showed the softmax warpgroups waiting 0.95 us of
+    // each 1.76 us tile for their S while one thread issued both products).
+    if (lane == 0) {
+      const uint32_t idesc_o = idesc_bf16_f32(128, kD, 0, 1);
+      bool ok = true;
+      uint32_t it = 0;
+      uint32_t cp[2] = {0, 0};   // P V products issued per query tile
+      uint32_t un[2] = {0, 0};   // units whose O was started, per query tile
+      for (int si = 0; si < nseg && ok; ++si) {
+        const TcSeg sg = tc_seg(p, c, si);
+        const bool two = two_tiles(sg.unit);
+        for (int64_t i = 0; i < sg.k1 - sg.k0 && ok; ++i, ++it) {
+          const TcItem itm = tc_item<kSplit>(sg, two, i);
+          const bool first = itm.first;
+          // O_t += P_t V for the ring entry `it`, for every warpgroup t in the mask
+          const uint32_t vs = it % kSt;
+          if (ok) ok = mbar_wait(b_vfull + 8 * vs, (it / kSt) & 1, p.err);
+          for (int t = 0; t < 2; ++t) {
+            if (!(itm.mask >> t & 1u)) continue;
+            const uint32_t b = cp[t] & 1;
+            if (ok) ok = mbar_wait(b_pfull + 8 * (2 * t + b), (cp[t] >> 1) & 1, p.err);
+            if (ok && first && un[t] > 0) ok = mbar_wait(b_ofree + 8 * t, (un[t] - 1) & 1, p.err);
+            if (first) ++un[t];
+            ++cp[t];
+            if (!ok) continue;
+            tc_fence_after();
+            const uint32_t pa = smem_u32(smem + TcSmem::p + (2 * t + b) * kPBytes);
+            const uint32_t vb = smem_u32(smem + TcSmem::v_at(vs));
+#pragma unroll
+            for (int kk = 0; kk < kTcKeys / 16; ++kk) {
+              // A = P (K-major, one 64-key chunk): keys 16 kk.. at byte 32 kk.
+              // B = V (MN-major): 16 keys = two 8-row groups of 128 B; the two
+              // 64-wide d halves are kKVBytes / 2 apart
+              mma_bf16_ss(tmem + 256 + 128 * t, sdesc_sw128(pa + kk * 32, 16, 1024),
+                          sdesc_sw128(vb + kk * 2048, kKVBytes / 2, 1024), idesc_o, (first && kk == 0) ? 0u : 1u);
+            }
+            mma_commit(b_pvdone + 8 * (2 * t + b));
+          }
+          mma_commit(b_vempty + 8 * vs);
+        }
+      }
     }
   } else {
     // --------------------- softmax + epilogue (tile t) ---------------------
