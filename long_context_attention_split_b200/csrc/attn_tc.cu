@@ -61,6 +61,11 @@ constexpr int kTcKeys = 64;                        // keys per tile
 // slower (the special-function unit is not its limit)
 constexpr int kTcPolyPairs = NECTAR_TC_POLY_PAIRS;
 constexpr int kTcStages = 3;                       // K and V ring depth
+#ifndef NECTAR_TC_PINGPONG
+#define NECTAR_TC_PINGPONG 1
+#endif
+constexpr bool kPingPong = NECTAR_TC_PINGPONG != 0;
+constexpr int kPingBar = 4;                         // named barriers 4, 5
 constexpr int kTcThreads = 12 * 32;
 constexpr uint32_t kQBytes = kTcRows * kD * 2;     // 32 KB
 constexpr uint32_t kKVBytes = kTcKeys * kD * 2;    // 16 KB
@@ -534,6 +539,11 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
       const bool two = two_tiles(sg.unit);
       const bool split = tc_split<kSplit>(sg, two);
       if (t == 1 && !two && !split) continue;
+      // two query tiles: the warpgroups take turns at the exponentials of a
+      // key tile (warpgroup 0 first), so that one's run on the special-
+      // function unit overlaps the other's maximum, stores and waits
+      const bool pp = kPingPong && two;
+      const int64_t nk = sg.k1 - sg.k0;
       float m = -INFINITY, l = 0.f;
       for (int64_t i = 0; i < sg.k1 - sg.k0; ++i) {
         const TcItem itm = tc_item<kSplit>(sg, two, i);
@@ -618,6 +628,12 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
         if (ci >= 2 && ok) ok = mbar_wait(b_pvdone + 8 * (2 * t + b), ((ci >> 1) - 1) & 1, p.err);
         uint8_t* pt = smem + TcSmem::p + (2 * t + b) * kPBytes;
         float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        if (pp) {
+          // warpgroup 0 waits for warpgroup 1's exponentials of the previous
+          // key tile, warpgroup 1 for warpgroup 0's of this one
+          if (t == 1) named_bar_sync(kPingBar + 1, 2 * kTcRows);
+          else if (i > 0) named_bar_sync(kPingBar, 2 * kTcRows);
+        }
         // the row sum adds the rounded weights that P V uses; full tiles and
         // the last (masked) tile in separate loops, so that the unrolled
         // loop body carries no per-pair branch
@@ -649,6 +665,10 @@ cache_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_co
             }
             *reinterpret_cast<uint4*>(pt + p_off(row, col0 + c8 * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
+        }
+        if (pp) {
+          if (t == 0) named_bar_arrive(kPingBar + 1, 2 * kTcRows);
+          else if (i + 1 < nk) named_bar_arrive(kPingBar, 2 * kTcRows);
         }
         if constexpr (kDup) {
           // the other half's keys carry no weight in this row
