@@ -76,6 +76,7 @@ def run_cache_attn(L, Hkv, G, n, nq, seed=0, key_scale=None):
     (1, 2, 4, 266, 16),       # 64 rows, 5 key tiles: halves of 3 and 2, ragged last tile
     (2, 8, 4, 3000, 16),      # 64 rows, 16 heads: units cut into short segments between CTAs
     (1, 1, 2, 64 * 2, 40),    # 80 rows, exactly two key tiles: one each
+    (256, 1, 2, 200, 1),      # 256 layers (NECTAR_MAX_LAYERS)
 ])
 def test_cache_attn_parity(L, Hkv, G, n, nq):
     wl, ag, Ag, ao, Ao = run_cache_attn(L, Hkv, G, n, nq, seed=n + G)
@@ -463,6 +464,12 @@ def test_module_forward_toy():
     dict(L=1, Hkv=2, G=7, nq=2, widths=[1152], depth=3),
     dict(L=1, Hkv=1, G=40, nq=1, widths=[2048], depth=2),       # 16 tiles x 48 rows > 512 TMEM columns: GEMM path
     dict(L=1, Hkv=2, G=4, nq=40, widths=[2048], depth=2),       # grouped GEMM, 16 units tiles
+    # the API's limits: depth 4 (NECTAR_MAX_DEPTH) on both paths, 256 layers (NECTAR_MAX_LAYERS)
+    dict(L=1, Hkv=2, G=2, nq=3, widths=[256], depth=4),         # one launch
+    dict(L=1, Hkv=1, G=4, nq=20, widths=[128], depth=4),        # 80 rows: grouped GEMM
+    # 256 layers, 16 rows per head (with 2 rows the score readout of a head
+    # can cancel towards 0, where the relative measure is ill-posed)
+    dict(L=256, Hkv=1, G=2, nq=8, widths=[16, 32, 48, 64] * 64, depth=1),
 ])
 def test_module_forward_shapes(kw):
     kw = dict(kw)
@@ -527,8 +534,16 @@ def test_decode_toy_prefill():
     dict(L=2, Hkv=2, G=2, n=16, B=3, T=40, widths=[768, 896]),   # one CTA per net in the one-launch decode
     dict(L=1, Hkv=2, G=2, n=16, B=3, T=40, widths=[2048]),        # the widest layer, one-launch decode
     dict(L=1, Hkv=1, G=7, n=16, B=16, T=40, widths=[1152]),       # 112 rows: grouped GEMM at 1152 units
+    dict(L=1, Hkv=2, G=2, n=16, B=3, T=40, widths=[256], depth=4),   # depth 4: three h exchanges
+    dict(L=1, Hkv=1, G=4, n=16, B=20, T=40, widths=[128], depth=4),  # depth 4, 80 rows: grouped GEMM
+    dict(L=256, Hkv=1, G=2, n=16, B=1, T=8, widths=[16, 64] * 128, depth=1),   # 256 layers
 ])
-def test_decode_shapes(kw):
+@pytest.mark.parametrize("cluster", ["auto", "0"])
+def test_decode_shapes(kw, cluster, monkeypatch):
+    # "auto": calls of <= 32 (l, h) pairs and <= 64 rows per head take the
+    # cluster decode; "0": the one-launch decode for every shape
+    if cluster == "0":
+        monkeypatch.setenv("NECTAR_DECODE_CLUSTER", "0")
     wl = make_workload("qwen3_1p7b", seed=2, key_scale=None, **kw)
     wl.local_len = torch.randint(0, wl.T + 1, (wl.B,), generator=torch.Generator().manual_seed(3)).to(torch.int32)
     wl.q_pos = (wl.local_len[wl.q_seq.long()] - 1).clamp(min=0).to(torch.int32)
