@@ -452,15 +452,21 @@ decode_cluster_kernel(const ClusterParams p) {
               }
             }
             if (reduce) {
+              // the warp's 32 units summed for each of the 16 rows by a
+              // halving transpose (16 shuffles, not 16 x 5): after it, lanes
+              // 2 r and 2 r + 1 hold row r's sum
 #pragma unroll
-              for (int jj = 0; jj < 16; ++jj) {
+              for (int off = 16, nv = 8; off >= 2; off >>= 1, nv >>= 1) {
+                const bool upper = (lane & off) != 0;
 #pragma unroll
-                for (int off = 16; off >= 1; off >>= 1) part[jj] += __shfl_xor_sync(0xffffffffu, part[jj], off);
+                for (int q = 0; q < nv; ++q) {
+                  const float send = upper ? part[q] : part[q + nv];
+                  const float keep = upper ? part[q + nv] : part[q];
+                  part[q] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                }
               }
-              if (lane == 0) {
-#pragma unroll
-                for (int jj = 0; jj < 16; ++jj) sp[q4 * N + n0r + jj] = part[jj];
-              }
+              const float tot = part[0] + __shfl_xor_sync(0xffffffffu, part[0], 1);
+              if ((lane & 1) == 0) sp[q4 * N + n0r + (lane >> 1)] = tot;
             }
           }
         }
