@@ -155,11 +155,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       "l"(src), "r"(bytes), "r"(bar), "l"(policy)
       : "memory");
 }
-// Bring [src, src + bytes) into L2 (a hint: nothing is written anywhere);
-// src 16-B aligned, bytes % 16 == 0.
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
 // Tiled tensor loads.  c0 is the innermost coordinate; callers keep
 // c0 * element size a multiple of 16 bytes.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
@@ -217,17 +212,7 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
-               "r"(v.w)
-               : "memory");
-}
-// arrive on an mbarrier of another CTA of the cluster, releasing this
-// thread's prior writes at cluster scope
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-// bounded wait that acquires at cluster scope (pairs with the remote arrive)
+// bounded wait that acquires at cluster scope (the peers' st.async bytes)
 __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, int* err) {
   const uint64_t t0 = globaltimer();
   while (true) {
@@ -267,15 +252,6 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
                : "memory");
   return v;
-}
-// Copy `bytes` of this CTA's shared memory into another CTA of the cluster
-// (dst and its mbarrier `bar` are shared::cluster addresses from mapa); the
-// copy completes `bytes` of transactions on that mbarrier.  A plain
-// point-to-point DSMEM copy, not a multicast.  16-byte aligned, bytes % 16 == 0.
-__device__ __forceinline__ void bulk_s2cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-               ::"r"(dst), "r"(src), "r"(bytes), "r"(bar)
-               : "memory");
 }
 // all threads of all CTAs of the cluster
 __device__ __forceinline__ void cluster_sync_all() {
