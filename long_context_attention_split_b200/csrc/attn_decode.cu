@@ -56,6 +56,7 @@ cache_attn_split_kernel(const DecParams p) {
   constexpr int KPW = TILE / WPG;            // keys per warp per tile
   constexpr int KPG = KPW / NG;              // keys per group per tile
   static_assert(KPG >= 1, "tile too small");
+  static_assert(KPW * WPG == TILE && KPG * NG == KPW, "a tile's keys split evenly over the warps and lane groups");
 
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* sK = smem;
@@ -236,39 +237,58 @@ __global__ void cache_attn_combine_kernel(const DecParams p, float* __restrict__
   const float* ml = p.ws_ml + (hd * p.S_max * p.rows_total + r) * 2;     // partial s at ml[s * rows_total * 2]
   const float* ac = p.ws_acc + (hd * p.S_max * p.rows_total + r) * kD;   // partial s at ac[s * rows_total * d]
   const int64_t sml = static_cast<int64_t>(p.rows_total) * 2, sac = static_cast<int64_t>(p.rows_total) * kD;
-  // the partials' maxima, one partial per lane (all loads in flight at once)
-  float M = -INFINITY;
-  for (int s = lane; s < ns; s += 32) M = fmaxf(M, ml[s * sml]);
+  // the first kFirst partials' value sums, this lane's 4 dims, loaded before
+  // anything waits on them: with the (m, l) loads below, one round trip to L2
+  // for a head of up to kFirst partials (a one-layer call: ~19)
+  constexpr int kFirst = 24;
+  float4 a4[kFirst];
+#pragma unroll
+  for (int j = 0; j < kFirst; ++j)
+    a4[j] = j < ns ? reinterpret_cast<const float4*>(ac + j * sac)[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+  // the partials' maxima and row sums, one partial per lane
+  float mv = -INFINITY, lv = 0.f;
+  if (lane < ns) {
+    mv = ml[lane * sml];
+    lv = ml[lane * sml + 1];
+  }
+  float M = mv;
+  for (int s = lane + 32; s < ns; s += 32) M = fmaxf(M, ml[s * sml]);
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   // weights 2^(m_s - M), the sum of the row weights, and the weighted sum of
-  // the partial value sums, 32 partials at a time
-  float ls = 0.f;
+  // the partial value sums
+  float w = lane < ns ? exp2_shift(mv, M) : 0.f;
+  float ls = lv * w;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < ns; s0 += 32) {
-    const int s = s0 + lane;
-    float w = 0.f;
-    if (s < ns) {
-      w = exp2_shift(ml[s * sml], M);
-      ls = fmaf(ml[s * sml + 1], w, ls);
+#pragma unroll
+  for (int j = 0; j < kFirst; ++j) {
+    const float wj = __shfl_sync(0xffffffffu, w, j);
+    acc.x = fmaf(a4[j].x, wj, acc.x);
+    acc.y = fmaf(a4[j].y, wj, acc.y);
+    acc.z = fmaf(a4[j].z, wj, acc.z);
+    acc.w = fmaf(a4[j].w, wj, acc.w);
+  }
+  // partials past kFirst (heads cut over more CTAs), 32 at a time
+  for (int s0 = kFirst; s0 < ns; s0 += 32) {
+    const int sl = s0 + lane;
+    const float wlow = __shfl_sync(0xffffffffu, w, sl & 31);   // partials < 32: lane sl holds the weight
+    float w2 = 0.f;
+    if (sl < ns) {
+      if (sl >= 32) {
+        w2 = exp2_shift(ml[sl * sml], M);
+        ls = fmaf(ml[sl * sml + 1], w2, ls);
+      } else {
+        w2 = wlow;            // (its row sum was added with the first 32)
+      }
     }
     const int cnt = ns - s0 < 32 ? ns - s0 : 32;
-    for (int j0 = 0; j0 < cnt; j0 += 8) {
-      float4 a4[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        a4[j] = j0 + j < cnt ? reinterpret_cast<const float4*>(ac + (s0 + j0 + j) * sac)[lane]
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float wj = __shfl_sync(0xffffffffu, w, (j0 + j) & 31);
-        if (j0 + j < cnt) {
-          acc.x = fmaf(a4[j].x, wj, acc.x);
-          acc.y = fmaf(a4[j].y, wj, acc.y);
-          acc.z = fmaf(a4[j].z, wj, acc.z);
-          acc.w = fmaf(a4[j].w, wj, acc.w);
-        }
-      }
+    for (int jj = 0; jj < cnt; ++jj) {
+      const float wj = __shfl_sync(0xffffffffu, w2, jj);
+      const float4 b4 = reinterpret_cast<const float4*>(ac + (s0 + jj) * sac)[lane];
+      acc.x = fmaf(b4.x, wj, acc.x);
+      acc.y = fmaf(b4.y, wj, acc.y);
+      acc.z = fmaf(b4.z, wj, acc.z);
+      acc.w = fmaf(b4.w, wj, acc.w);
     }
   }
 #pragma unroll

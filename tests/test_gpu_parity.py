@@ -77,6 +77,9 @@ def run_cache_attn(L, Hkv, G, n, nq, seed=0, key_scale=None):
     (2, 8, 4, 3000, 16),      # 64 rows, 16 heads: units cut into short segments between CTAs
     (1, 1, 2, 64 * 2, 40),    # 80 rows, exactly two key tiles: one each
     (256, 1, 2, 200, 1),      # 256 layers (NECTAR_MAX_LAYERS)
+    # one head cut over every CTA: more partials per head than a warp has lanes
+    (1, 1, 2, 65536, 1),      # 1024 key tiles over all CTAs
+    (1, 1, 1, 1900, 1),       # ~30 one-tile partials
 ])
 def test_cache_attn_parity(L, Hkv, G, n, nq):
     wl, ag, Ag, ao, Ao = run_cache_attn(L, Hkv, G, n, nq, seed=n + G)
@@ -97,6 +100,7 @@ def test_cache_attn_parity(L, Hkv, G, n, nq):
     (1, 2, 4, 5000, 5),       # 20 rows: 32 query columns
     (2, 3, 4, 3000, 16),      # 64 rows: 64 query columns, heads cut over CTAs
     (1, 2, 8, 1000, 6),       # 48 rows, ragged tail
+    (1, 1, 5, 131072, 1),     # 5 rows, one head cut over every CTA
 ])
 def test_cache_attn_tct(L, Hkv, G, n, nq, monkeypatch):
     wl, ag, Ag, ao, Ao = run_cache_attn(L, Hkv, G, n, nq, seed=n + 7 * G)
