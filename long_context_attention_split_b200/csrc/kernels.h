@@ -136,8 +136,11 @@ struct TcParams {
   int tile;             // keys per tile: dec_tile(rows of a pass)
   int64_t tph;          // tiles per head
   int C;                // CTAs (one per SM)
-  int dp_rounds;        // whole-unit rounds before the stream-K part
-  int64_t sk_units;     // units cut by key tiles across the CTAs
+  int dp_rounds;        // whole-unit rounds before the rest
+  int64_t sk_units;     // the rest: units cut by key tiles across the CTAs
+  int sk_parts;         // 0: the rest as one stream-K range list; S > 0: each unit of the rest in S
+                        // equal key parts, item p * sk_units + u on CTA item % C (the query units of
+                        // a head then read each key part at the same time)
   float qmul;           // scale * log2(e)
   float* alpha;
   float* A;
@@ -150,6 +153,7 @@ struct TcPlan {
   int64_t tph;
   int C, dp_rounds;
   int64_t sk_units;
+  int sk_parts;
   size_t ws_bytes, smem;
 };
 TcPlan plan_tc(int heads, int64_t n, int64_t rows, int num_sms);

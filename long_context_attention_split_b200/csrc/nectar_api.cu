@@ -326,6 +326,7 @@ nectar_status nectar_cache_attn_lse(nectar_dims dims, const nectar_bf16* K, cons
     tpar.C = tp.C;
     tpar.dp_rounds = tp.dp_rounds;
     tpar.sk_units = tp.sk_units;
+    tpar.sk_parts = tp.sk_parts;
     tpar.qmul = scale * kLog2e;
     tpar.alpha = alpha;
     tpar.A = A;

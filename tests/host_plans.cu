@@ -11,10 +11,12 @@
 //                  slots a head gets in the workspace) is the largest number
 //                  of CTAs whose range touches one head;
 //   tensor cores   dp_rounds whole rounds of C units plus sk_units units cut
-//                  by key tiles make up all units, every CTA's range cuts at
-//                  most the 2 units it has partial slots for (the first and
-//                  the last of its range), and the workspace holds 2 slots of
-//                  256 rows of (d + 2) floats per CTA;
+//                  by key tiles make up all units; a stream-K rest cuts at
+//                  most the 2 units of each CTA's range it has partial slots
+//                  for (the first and the last), a lockstep rest puts every
+//                  key tile of its units in exactly one of at most 2 items
+//                  per CTA, within 10 % of the even cut; the workspace holds
+//                  2 slots of 256 rows of (d + 2) floats per CTA;
 //   shared memory  every split launch fits 227 KB per CTA, and the launches
 //                  bounded to two CTAs per SM fit the SM's 228 KB twice.
 // Prints "ok <cases>" and exits 0, or prints the first failure and exits 1.
@@ -87,14 +89,49 @@ bool check_tc(int heads, int64_t n, int64_t rows, int sms) {
   CHECK(pl.dp_rounds >= 0 && pl.sk_units >= 0, "dp %d sk %lld", pl.dp_rounds, (long long)pl.sk_units);
   CHECK(static_cast<int64_t>(pl.dp_rounds) * pl.C + pl.sk_units == units, "dp %d x C %d + sk %lld != units %lld",
         pl.dp_rounds, pl.C, (long long)pl.sk_units, (long long)units);
-  // whole rounds are taken only while at least one round of units is left
-  // to cut, so no CTA idles through the stream-K part
-  if (pl.sk_units > 0 && pl.dp_rounds > 0)
-    CHECK(pl.sk_units >= pl.C && pl.sk_units < 2 * static_cast<int64_t>(pl.C), "sk %lld C %d",
-          (long long)pl.sk_units, pl.C);
   CHECK(pl.ws_bytes >= static_cast<size_t>(pl.C) * 2 * kUnitRows * (kD + 2) * sizeof(float), "ws %zu",
         pl.ws_bytes);
   CHECK(pl.smem <= kMaxSmemPerCta, "smem %zu", pl.smem);
+  if (pl.sk_parts > 0) {
+    // lockstep rest: every whole round, the rest (< C units) in S equal key
+    // parts, item q * U + u on CTA item % C, slot item / C (two slots)
+    const int64_t U = pl.sk_units, S = pl.sk_parts, items = U * S;
+    CHECK(pl.qpairs > 1 && U > 0 && U < pl.C, "lockstep with qpairs %d, rest %lld, C %d", pl.qpairs, (long long)U,
+          pl.C);
+    CHECK(pl.dp_rounds == units / pl.C, "lockstep rounds %d, units %lld", pl.dp_rounds, (long long)units);
+    CHECK(S <= pl.tph && items <= 2 * static_cast<int64_t>(pl.C), "S %lld items %lld C %d tph %lld", (long long)S,
+          (long long)items, pl.C, (long long)pl.tph);
+    // every key tile of every rest unit in exactly one (CTA, slot); no slot used twice
+    std::vector<int> seen(static_cast<size_t>(U * pl.tph), 0);
+    std::vector<int> slot_used(static_cast<size_t>(pl.C) * 2, 0);
+    int64_t longest = 0;
+    for (int64_t c = 0; c < pl.C; ++c) {
+      int64_t tiles = 0;
+      for (int j = 0; c + j * static_cast<int64_t>(pl.C) < items; ++j) {
+        const int64_t item = c + j * static_cast<int64_t>(pl.C);
+        const int64_t q = item / U, u = item % U;
+        const int64_t k0 = q * pl.tph / S, k1 = (q + 1) * pl.tph / S;
+        CHECK(k1 > k0, "empty part %lld of %lld (tph %lld)", (long long)q, (long long)S, (long long)pl.tph);
+        CHECK(j < 2, "CTA %lld has a third item", (long long)c);
+        ++slot_used[c * 2 + j];
+        for (int64_t k = k0; k < k1; ++k) ++seen[u * pl.tph + k];
+        tiles += k1 - k0;
+      }
+      longest = std::max(longest, tiles);
+    }
+    for (size_t i = 0; i < seen.size(); ++i)
+      CHECK(seen[i] == 1, "rest tile %zu covered %d times", i, seen[i]);
+    for (size_t i = 0; i < slot_used.size(); ++i) CHECK(slot_used[i] <= 1, "slot %zu used twice", i);
+    // within 10 % of cutting the rest evenly over the CTAs
+    const int64_t even = cdiv(U * pl.tph, pl.C);
+    CHECK(longest * 10 <= even * 11, "longest CTA %lld tiles, even cut %lld", (long long)longest, (long long)even);
+    return true;
+  }
+  // stream-K rest: whole rounds are taken only while at least one round of
+  // units is left to cut, so no CTA idles through the stream-K part
+  if (pl.sk_units > 0 && pl.dp_rounds > 0)
+    CHECK(pl.sk_units >= pl.C && pl.sk_units < 2 * static_cast<int64_t>(pl.C), "sk %lld C %d",
+          (long long)pl.sk_units, pl.C);
   const int64_t Tsk = pl.sk_units * pl.tph;
   for (int64_t c = 0; c < pl.C && Tsk > 0; ++c) {
     const int64_t s0 = c * Tsk / pl.C, s1 = (c + 1) * Tsk / pl.C;

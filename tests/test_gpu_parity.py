@@ -86,6 +86,21 @@ def test_cache_attn_parity(L, Hkv, G, n, nq):
     check_attn(ag, Ag, ao, Ao, wl.V.float().abs().max().item(), f"n={n}")
 
 
+# The tensor-core kernel's lockstep rest: after the whole rounds, each
+# remaining unit (two or more query units per head) in S equal key parts,
+# item p * U + u on CTA item % C.  On 148 SMs: 4 heads x 2 query units, 148
+# key tiles -> no whole round, S = 37, two items on every CTA (both partial
+# slots); 75 heads x 2 query units, 37 key tiles -> one whole round, then 2
+# units in 37 one-tile parts.
+@pytest.mark.parametrize("L,Hkv,G,n,nq", [
+    (1, 4, 4, 148 * 64, 128),
+    (1, 75, 2, 37 * 64, 129),
+])
+def test_cache_attn_tc_lockstep_rest(L, Hkv, G, n, nq):
+    wl, ag, Ag, ao, Ao = run_cache_attn(L, Hkv, G, n, nq, seed=n + Hkv)
+    check_attn(ag, Ag, ao, Ao, wl.V.float().abs().max().item(), f"lockstep n={n}")
+
+
 # 3-16 query rows per KV head: the transposed tensor-core split kernel
 # (keys on the TMEM lanes).  Cases: a ragged single tile, many short heads per
 # CTA range (each CTA crosses 4 heads: the double-buffered Q and O^T are

@@ -35,7 +35,9 @@ PLAN_MUTANTS = [
     ("attn_decode.cu", "S_max one short", "if (la - f + 1 > pl.S_max) pl.S_max = la - f + 1;",
      "if (la - f > pl.S_max) pl.S_max = la - f;"),
     ("attn_decode.cu", "C not clamped to the tile count", "  if (C > pl.total) C = pl.total;\n", ""),
-    ("attn_tc.cu", "no whole round left for the stream-K part", "  if (units % C != 0 && R > 0) R -= 1;\n", ""),
+    ("attn_tc.cu", "no whole round left for the stream-K part", "  if (best_s == 0 && rest != 0 && R > 0) R -= 1;\n",
+     ""),
+    ("attn_tc.cu", "lockstep balance ignored", "if (best_s > 0 && best * 10 > even * 11) best_s = 0;", ""),
     ("attn_tc.cu", "one partial slot per CTA",
      "pl.ws_bytes = static_cast<size_t>(pl.C) * 2 * kTcUnitRows", "pl.ws_bytes = static_cast<size_t>(pl.C) * 1 * kTcUnitRows"),
 ]
