@@ -540,11 +540,17 @@ def per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args, roof_us=N
     """ms per step when the step is issued as L per-layer calls captured in
     one CUDA graph and replayed -- the form a model that runs layer after
     layer gives -- and the same for each half alone; None when the workload
-    has one layer.  Two forms of the whole step: `ms_per_step` runs each
-    layer's decode on a second stream beside its exact attention (the two
-    calls of a layer share no data), and the next layer starts when both
-    have ended; `serial_ms_per_step` issues exact attention, then the
-    decode, on one stream.
+    has one layer.  Three forms of the whole step, each with the
+    dependencies a model that runs its layers in turn has (layer l + 1's
+    query depends on layer l's decode output):
+      `ms_per_step`: the decodes are the model's chain, on one stream; the
+        exact attention of layer l (regression targets, which no later layer
+        reads) starts on a second stream once layer l's query exists, i.e.
+        after the decode of layer l - 1, and the step ends when both
+        streams have;
+      `beside_ms_per_step`: each layer's decode on a second stream beside
+        its exact attention, the next layer after both;
+      `serial_ms_per_step`: exact attention, then the decode, on one stream.
     roof_us: {"step": .., "exact": .., "decode": ..} roofline times (us) of
     the whole step and its halves, for the fractions."""
     if wl.L < 2:
@@ -560,8 +566,21 @@ def per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args, roof_us=N
                           dtype=torch.uint8, device=dev)
 
         evs = [(torch.cuda.Event(), torch.cuda.Event()) for _ in range(wl.L)]
+        end_b = torch.cuda.Event()
 
-        def issue(exact=True, decode=True, beside=False):
+        def issue(exact=True, decode=True, beside=False, pipelined=False):
+            if pipelined and exact and decode and has_decode:
+                for l in range(wl.L):
+                    sl = slice(l, l + 1)
+                    q_ready = evs[l][0]
+                    q_ready.record(s)            # after the decode of layer l - 1 (the step's start for l = 0)
+                    s2.wait_event(q_ready)
+                    nx.cache_attn_lse(wl.K[sl], wl.V[sl], Q[sl], alpha=alpha[sl], A=A[sl], workspace=ws, stream=s2)
+                    nx.decode(lmods[l], Q[sl], wl.q_seq, wl.q_pos, wl.Kloc[sl], wl.Vloc[sl], wl.local_len,
+                              out=out[sl], workspace=dws, stream=s)
+                end_b.record(s2)
+                s.wait_event(end_b)
+                return
             for l in range(wl.L):
                 sl = slice(l, l + 1)
                 if beside and exact and decode and has_decode:
@@ -605,9 +624,11 @@ def per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args, roof_us=N
             del g
             return e0.elapsed_time(e1) / args.steps
 
-        res = {"ms_per_step": timed(beside=True), "calls_per_step": wl.L * (2 if has_decode else 1)}
         if has_decode:
-            res["serial_ms_per_step"] = timed()
+            res = {"ms_per_step": timed(pipelined=True), "calls_per_step": wl.L * 2,
+                   "beside_ms_per_step": timed(beside=True), "serial_ms_per_step": timed()}
+        else:
+            res = {"ms_per_step": timed(), "calls_per_step": wl.L}
         res["exact_ms"] = timed(decode=False)
         if has_decode:
             res["decode_ms"] = timed(exact=False)

@@ -382,16 +382,21 @@ cache_attn_tct_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
       tc_fence_before();
       mbar_arrive(b_sfree + 8 * sb);                  // S^T of this tile read for the last time
       fence_proxy_async_smem();
+      // ofull completes one phase per tile's O^T update, in order, and a
+      // parity wait only tells the current phase from the one before.  At a
+      // head range's last tile this thread waits for O(i), so first for
+      // O(i - 1) (issued after S(i), it may still be running: a wait for
+      // phase i alone would pass on phase i - 1's parity) -- and that before
+      // its P(i) lets O(i) be issued: waited after, O(i) could complete
+      // first, and the parity of phase i - 1 would then name phase i + 1,
+      // which waits on this thread's next P (seen as a wait that ran out
+      // when another kernel ran beside this one).  (The rescale's wait for
+      // O(i - 1) needs no such step: S(i), complete by then, was issued
+      // after O(i - 2), and P(i) is not written yet.)
+      if (last && ok && i >= 1) ok = mbar_wait(b_ofull, (i - 1) & 1, p.err);
       mbar_arrive(b_pfull + 8 * sb);
       if (last) {
-        // the head's partial: O^T (this thread: dim r), the row sums, M.
-        // ofull completes one phase per tile's O^T update, in order, and a
-        // parity wait only tells the current phase from the one before: so
-        // O(i - 1) first (it was issued after S(i), and may still be running
-        // -- a wait for phase i alone would pass on phase i - 1's parity),
-        // then O(i).  (The rescale's wait for O(i - 1) needs no such step:
-        // S(i), complete by then, was issued after O(i - 2).)
-        if (ok && i >= 1) ok = mbar_wait(b_ofull, (i - 1) & 1, p.err);
+        // the head's partial: O^T (this thread: dim r), the row sums, M
         if (ok) ok = mbar_wait(b_ofull, i & 1, p.err);
         tc_fence_after();
         const int slot = c - first_cta_of_tile(hd * p.tph, p.total, p.C);

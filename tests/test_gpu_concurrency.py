@@ -1,0 +1,80 @@
+"""The library's calls running side by side on two streams, as a model that
+runs its layers in turn issues them: each layer's decode on one stream (the
+model's chain), the same layer's exact attention of Eq. (3.1) ("Nectar:
+Neural Estimation of Cached-Token Attention via Regression", §2.1) on a
+second stream once the layer's query exists, i.e. after the decode of the
+layer before.
+
+At the Llama-8B decode shapes (b = 1: 4 query rows per KV head) the exact
+attention runs the transposed tensor-core kernel and the decode the
+8-CTA-cluster kernel.  Replayed this way, the transposed kernel's wait for
+the O^T update of a head range's next-to-last key tile could miss it (two
+phases of one barrier completing before a parity wait), so the wait ran
+out after its time limit in about 1 replay of 7.  The test replays the
+captured step 30 times, and after each checks the device error word and
+that every output equals the one-stream run bit for bit (neither kernel's
+arithmetic depends on the scheduling)."""
+import pytest
+import torch
+
+import long_context_attention_split_b200 as nx
+from nectar_inputs import make_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def test_exact_attention_beside_the_layer_chain_of_decodes():
+    dev = torch.device("cuda")
+    wl = make_workload("llama8b_sweep", device="cuda", B=1, rho=0.10)
+    mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G, device="cuda")
+    lmods = [mods.layer(l) for l in range(wl.L)]
+    Q = wl.Q
+    ws = torch.empty(nx.cache_attn_workspace_size(1, wl.Hkv, wl.G, wl.n, wl.nq), dtype=torch.uint8, device=dev)
+    dws = torch.empty(max(nx.decode_workspace_size(m, wl.G, wl.nq) for m in lmods), dtype=torch.uint8, device=dev)
+    alpha = torch.empty(Q.shape[:4], device=dev)
+    A = torch.empty(Q.shape, device=dev)
+    out = torch.empty(Q.shape, device=dev)
+    nx.device_error_flags(clear=True)
+
+    # reference: every call on one stream, one after the other
+    ref_a, ref_A, ref_o = torch.empty_like(alpha), torch.empty_like(A), torch.empty_like(out)
+    for l in range(wl.L):
+        sl = slice(l, l + 1)
+        nx.cache_attn_lse(wl.K[sl], wl.V[sl], Q[sl], alpha=ref_a[sl], A=ref_A[sl], workspace=ws)
+        nx.decode(lmods[l], Q[sl], wl.q_seq, wl.q_pos, wl.Kloc[sl], wl.Vloc[sl], wl.local_len, out=ref_o[sl],
+                  workspace=dws)
+    torch.cuda.synchronize()
+    assert nx.device_error_flags(clear=True) == 0
+
+    s, s2 = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    q_ready = [torch.cuda.Event() for _ in range(wl.L)]
+    done = torch.cuda.Event()
+
+    def issue():
+        for l in range(wl.L):
+            sl = slice(l, l + 1)
+            q_ready[l].record(s)            # after the decode of layer l - 1
+            s2.wait_event(q_ready[l])
+            nx.cache_attn_lse(wl.K[sl], wl.V[sl], Q[sl], alpha=alpha[sl], A=A[sl], workspace=ws, stream=s2)
+            nx.decode(lmods[l], Q[sl], wl.q_seq, wl.q_pos, wl.Kloc[sl], wl.Vloc[sl], wl.local_len, out=out[sl],
+                      workspace=dws, stream=s)
+        done.record(s2)
+        s.wait_event(done)
+
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        issue()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s, capture_error_mode="relaxed"):
+        issue()
+    for rep in range(30):
+        for t in (alpha, A, out):
+            t.fill_(float("nan"))
+        with torch.cuda.stream(s):
+            s.wait_stream(torch.cuda.current_stream(dev))
+            g.replay()
+        torch.cuda.synchronize()
+        assert nx.device_error_flags(clear=True) == 0, f"replay {rep}: a bounded wait ran out"
+        assert torch.equal(alpha, ref_a) and torch.equal(A, ref_A) and torch.equal(out, ref_o), f"replay {rep}"
+    del g
