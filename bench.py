@@ -550,7 +550,11 @@ def per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args, roof_us=N
         streams have;
       `beside_ms_per_step`: each layer's decode on a second stream beside
         its exact attention, the next layer after both;
-      `serial_ms_per_step`: exact attention, then the decode, on one stream.
+      `serial_ms_per_step`: exact attention, then the decode, on one stream;
+      `grouped4_ms_per_step`: as `ms_per_step`, but the exact attention
+        runs for 4 layers at a time, once the last of their queries exists
+        (not per-layer exact calls: the targets of a layer are ready up to
+        3 layers later).
     roof_us: {"step": .., "exact": .., "decode": ..} roofline times (us) of
     the whole step and its halves, for the fractions."""
     if wl.L < 2:
@@ -561,6 +565,8 @@ def per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args, roof_us=N
         s2 = torch.cuda.Stream(dev)
         ws = torch.empty(max(nx.cache_attn_workspace_size(1, wl.Hkv, wl.G, wl.n, wl.nq), 16), dtype=torch.uint8,
                          device=dev)
+        wsg = torch.empty(max(max(nx.cache_attn_workspace_size(k, wl.Hkv, wl.G, wl.n, wl.nq) for k in (1, 4)), 16),
+                          dtype=torch.uint8, device=dev)
         lmods = [mods.layer(l) for l in range(wl.L)] if has_decode else None
         dws = torch.empty(max(max(nx.decode_workspace_size(m, wl.G, wl.nq) for m in lmods) if has_decode else 16, 16),
                           dtype=torch.uint8, device=dev)
@@ -568,14 +574,18 @@ def per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args, roof_us=N
         evs = [(torch.cuda.Event(), torch.cuda.Event()) for _ in range(wl.L)]
         end_b = torch.cuda.Event()
 
-        def issue(exact=True, decode=True, beside=False, pipelined=False):
+        def issue(exact=True, decode=True, beside=False, pipelined=False, group=1):
             if pipelined and exact and decode and has_decode:
                 for l in range(wl.L):
                     sl = slice(l, l + 1)
                     q_ready = evs[l][0]
                     q_ready.record(s)            # after the decode of layer l - 1 (the step's start for l = 0)
-                    s2.wait_event(q_ready)
-                    nx.cache_attn_lse(wl.K[sl], wl.V[sl], Q[sl], alpha=alpha[sl], A=A[sl], workspace=ws, stream=s2)
+                    if (l + 1) % group == 0 or l + 1 == wl.L:
+                        g0 = l + 1 - ((l % group) + 1)
+                        gs = slice(g0, l + 1)
+                        s2.wait_event(q_ready)
+                        nx.cache_attn_lse(wl.K[gs], wl.V[gs], Q[gs], alpha=alpha[gs], A=A[gs], workspace=wsg,
+                                          stream=s2)
                     nx.decode(lmods[l], Q[sl], wl.q_seq, wl.q_pos, wl.Kloc[sl], wl.Vloc[sl], wl.local_len,
                               out=out[sl], workspace=dws, stream=s)
                 end_b.record(s2)
@@ -626,7 +636,8 @@ def per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args, roof_us=N
 
         if has_decode:
             res = {"ms_per_step": timed(pipelined=True), "calls_per_step": wl.L * 2,
-                   "beside_ms_per_step": timed(beside=True), "serial_ms_per_step": timed()}
+                   "beside_ms_per_step": timed(beside=True), "serial_ms_per_step": timed(),
+                   "grouped4_ms_per_step": timed(pipelined=True, group=4)}
         else:
             res = {"ms_per_step": timed(), "calls_per_step": wl.L}
         res["exact_ms"] = timed(decode=False)
