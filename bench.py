@@ -107,7 +107,10 @@ def aggregate(units_per_rank: float, max_ms: float, steps: int) -> float:
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples every 20 ms from a little before the timed region
+    to a little after it; summary() keeps the samples whose timestamp falls
+    inside [mark_start(), mark_end()] (host clock), and says how many."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -117,6 +120,13 @@ class ClockSampler:
         # the samples go to $NECTAR_CLOCKS_DIR (default: the system temp directory)
         out_dir = os.environ.get("NECTAR_CLOCKS_DIR") or tempfile.gettempdir()
         self.path = os.path.join(out_dir, f"clocks_gpu{gpu_index}.csv")
+        self.t_start = self.t_end = None
+
+    def mark_start(self):
+        self.t_start = time.time()
+
+    def mark_end(self):
+        self.t_end = time.time()
 
     def __enter__(self):
         try:
@@ -145,22 +155,25 @@ class ClockSampler:
             rows = [ln.split(",") for ln in open(self.path).read().strip().splitlines() if ln.strip()]
         except Exception:
             rows = []
-        sm = []
-        mx = None
-        reasons = set()
+        import datetime
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        parsed = []
         for r in rows:
             try:
-                sm.append(float(r[1]))
-                mx = float(r[2])
-                for nm, v in zip(names, r[5:9]):
-                    if v.strip().lower() == "active":
-                        reasons.add(nm)
+                ts = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                parsed.append((ts, float(r[2]), float(r[3]), [v.strip().lower() == "active" for v in r[6:10]]))
             except Exception:
                 pass
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        inside = [x for x in parsed
+                  if self.t_start is not None and self.t_end is not None and self.t_start <= x[0] <= self.t_end]
+        use = inside if inside else parsed
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0,
+                    "samples_in_timed_region": 0}
+        reasons = sorted({nm for x in use for nm, on in zip(names, x[3]) if on})
+        return {"sm_mhz": statistics.median(x[1] for x in use), "sm_max_mhz": use[-1][2], "reasons": reasons,
+                "samples": len(parsed), "samples_in_timed_region": len(inside),
+                "window": "timed region" if inside else "around the timed region (no sample inside it)"}
 
 
 # ---------------------------------------------------------------------------
@@ -273,11 +286,13 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
+        clk.mark_start()
         t0.record(stream)
         for i in range(args.steps):
             step(i)
         t1.record(stream)
         torch.cuda.synchronize(dev)
+        clk.mark_end()
         barrier(dev)
     total_ms = t0.elapsed_time(t1)
     max_ms = reduce_max(total_ms, dev)
@@ -909,7 +924,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="qwen3_1p7b", choices=sorted(PRESETS))
