@@ -16,7 +16,7 @@ independent replica (the path has no exchange step), value = all ranks'
 queries / max-over-ranks time, scaling "weak".
 
 --impl reference times the CPU oracle (oracle/, plain C in fp64) on the
-box's host cores on a bounded sample of the same workload.
+host's cores on a bounded sample of the same workload.
 """
 from __future__ import annotations
 
@@ -872,7 +872,7 @@ def _host_view(wl, layers, token_cap=None):
 
 
 def run_reference(args):
-    """The CPU oracle, as it stands, on the machine's host cores: each step is one
+    """The CPU oracle, as it stands, on the host's cores: each step is one
     pass of the whole path over layer 0 (all KV heads, all query rows) of the
     workload -- a bounded sample of the GPU arm's step."""
     ws, rank, _ = dist_env()
