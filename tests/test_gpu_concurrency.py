@@ -12,8 +12,11 @@ the O^T update of a head range's next-to-last key tile could miss it (two
 phases of one barrier completing before a parity wait), so the wait ran
 out after its time limit in about 1 replay of 7.  The test replays the
 captured step 30 times, and after each checks the device error word and
-that every output equals the one-stream run bit for bit (neither kernel's
-arithmetic depends on the scheduling)."""
+the outputs against the one-stream run: bit for bit with one layer per
+exact call (neither kernel's arithmetic depends on the scheduling); with 4
+layers per call the keys are split another way, so (alpha, A) within the
+attention tolerances.  At Qwen3-1.7B shapes the exact attention is the
+CUDA-core split kernel instead."""
 import pytest
 import torch
 
@@ -23,13 +26,25 @@ from nectar_inputs import make_workload
 pytestmark = pytest.mark.gpu
 
 
-def test_exact_attention_beside_the_layer_chain_of_decodes():
+WORKLOADS = {
+    "llama8b_b1": ("llama8b_sweep", dict(B=1, rho=0.10)),   # transposed tensor-core exact kernel
+    "qwen3_1p7b": ("qwen3_1p7b", {}),                       # CUDA-core split kernel
+}
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+@pytest.mark.parametrize("group", [1, 4])
+def test_exact_attention_beside_the_layer_chain_of_decodes(name, group):
+    """group: layers per exact-attention call (4: once the last of their
+    queries exists)."""
     dev = torch.device("cuda")
-    wl = make_workload("llama8b_sweep", device="cuda", B=1, rho=0.10)
+    preset, kw = WORKLOADS[name]
+    wl = make_workload(preset, device="cuda", **kw)
     mods = nx.pack_modules(wl.modules, wl.widths, wl.depth, wl.Hkv, wl.G, device="cuda")
     lmods = [mods.layer(l) for l in range(wl.L)]
     Q = wl.Q
-    ws = torch.empty(nx.cache_attn_workspace_size(1, wl.Hkv, wl.G, wl.n, wl.nq), dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(nx.cache_attn_workspace_size(k, wl.Hkv, wl.G, wl.n, wl.nq) for k in (1, group)),
+                     dtype=torch.uint8, device=dev)
     dws = torch.empty(max(nx.decode_workspace_size(m, wl.G, wl.nq) for m in lmods), dtype=torch.uint8, device=dev)
     alpha = torch.empty(Q.shape[:4], device=dev)
     A = torch.empty(Q.shape, device=dev)
@@ -54,8 +69,10 @@ def test_exact_attention_beside_the_layer_chain_of_decodes():
         for l in range(wl.L):
             sl = slice(l, l + 1)
             q_ready[l].record(s)            # after the decode of layer l - 1
-            s2.wait_event(q_ready[l])
-            nx.cache_attn_lse(wl.K[sl], wl.V[sl], Q[sl], alpha=alpha[sl], A=A[sl], workspace=ws, stream=s2)
+            if (l + 1) % group == 0 or l + 1 == wl.L:
+                gs = slice(l - l % group, l + 1)
+                s2.wait_event(q_ready[l])
+                nx.cache_attn_lse(wl.K[gs], wl.V[gs], Q[gs], alpha=alpha[gs], A=A[gs], workspace=ws, stream=s2)
             nx.decode(lmods[l], Q[sl], wl.q_seq, wl.q_pos, wl.Kloc[sl], wl.Vloc[sl], wl.local_len, out=out[sl],
                       workspace=dws, stream=s)
         done.record(s2)
@@ -76,5 +93,11 @@ def test_exact_attention_beside_the_layer_chain_of_decodes():
             g.replay()
         torch.cuda.synchronize()
         assert nx.device_error_flags(clear=True) == 0, f"replay {rep}: a bounded wait ran out"
-        assert torch.equal(alpha, ref_a) and torch.equal(A, ref_A) and torch.equal(out, ref_o), f"replay {rep}"
+        assert torch.equal(out, ref_o), f"replay {rep}"
+        if group == 1:      # (a call over 4 layers splits their keys another way)
+            assert torch.equal(alpha, ref_a) and torch.equal(A, ref_A), f"replay {rep}"
+        else:
+            vmax = wl.V.float().abs().max().item()
+            assert (alpha - ref_a).abs().max().item() <= 1e-3, f"replay {rep}"
+            assert (A - ref_A).abs().max().item() <= 2e-3 * vmax, f"replay {rep}"
     del g
