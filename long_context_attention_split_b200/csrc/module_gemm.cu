@@ -299,22 +299,38 @@ module_gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     const uint32_t tlane = static_cast<uint32_t>(q4 * 32) << 16;
     uint32_t tc = 0;
     bool ok = true;
+    // A tile's decode and its per-thread constants (bias; the score
+    // readout's w) are fetched one tile ahead, as raw bf16 bits, so that the
+    // search over the per-layer tables and the global loads (~1.3 us a tile
+    // on a per-tile timeline of stage 0, where the epilogue bounds the tile
+    // rate) run under the previous tile's epilogue.
+    const uint16_t* blob16 = reinterpret_cast<const uint16_t*>(p.blob);
+    auto fetch = [&](int64_t tt, GemmTile& gg, uint16_t& braw, uint16_t& wraw) {
+      gg = gemm_tile<kReadout>(p, tt);
+      const int ii = gg.m * 128 + u;
+      braw = 0;
+      wraw = 0;
+      if (kReadout) {
+        braw = blob16[gg.b_off + u];
+      } else if (ii < gg.H) {
+        braw = blob16[gg.b_off + ii];
+        if (gg.score_last) wraw = blob16[gg.aux_off + ii];
+      }
+    };
+    GemmTile gnext{};
+    uint16_t bnext = 0, wnext = 0;
+    if (blockIdx.x < p.ntiles) fetch(blockIdx.x, gnext, bnext, wnext);
     for (int64_t t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++tc) {
-      const GemmTile g = gemm_tile<kReadout>(p, t);
+      const GemmTile g = gnext;
+      const float bias = __uint_as_float(static_cast<uint32_t>(bnext) << 16);
+      const float wsc = __uint_as_float(static_cast<uint32_t>(wnext) << 16);
+      if (t + gridDim.x < p.ntiles) fetch(t + gridDim.x, gnext, bnext, wnext);
       const uint32_t b = tc & 1;
       const int r0 = g.rt * NR;
       // rows of this tile; a 32-column batch may run 16 columns past NR
       const int rend = (R < r0 + NR) ? R : r0 + NR;
-      // per-thread constants, fetched before the accumulator is ready
       const int i = g.m * 128 + u;
-      float bias = 0.f, wsc = 0.f;
       const bool score_last = g.score_last;
-      if (kReadout) {
-        bias = __bfloat162float(p.blob[g.b_off + u]);
-      } else if (i < g.H) {
-        bias = __bfloat162float(p.blob[g.b_off + i]);
-        if (score_last) wsc = __bfloat162float(p.blob[g.aux_off + i]);
-      }
       const float hbias = 0.5f * bias;
       if (ok) ok = mbar_wait_sleep(b_accf + 8 * b, (tc >> 1) & 1, p.err);   // waits out a main loop
       ok = __all_sync(0xffffffffu, ok);         // keeps the shuffles below warp-uniform
