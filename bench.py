@@ -555,7 +555,7 @@ def per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args, roof_us=N
     """ms per step when the step is issued as L per-layer calls captured in
     one CUDA graph and replayed -- the form a model that runs layer after
     layer gives -- and the same for each half alone; None when the workload
-    has one layer.  Three forms of the whole step, each with the
+    has one layer.  Four forms of the whole step, each with the
     dependencies a model that runs its layers in turn has (layer l + 1's
     query depends on layer l's decode output):
       `ms_per_step`: the decodes are the model's chain, on one stream; the
@@ -596,8 +596,7 @@ def per_layer_graph(wl, mods, Q, alpha, A, out, has_decode, dev, args, roof_us=N
                     q_ready = evs[l][0]
                     q_ready.record(s)            # after the decode of layer l - 1 (the step's start for l = 0)
                     if (l + 1) % group == 0 or l + 1 == wl.L:
-                        g0 = l + 1 - ((l % group) + 1)
-                        gs = slice(g0, l + 1)
+                        gs = slice(l - l % group, l + 1)
                         s2.wait_event(q_ready)
                         nx.cache_attn_lse(wl.K[gs], wl.V[gs], Q[gs], alpha=alpha[gs], A=A[gs], workspace=wsg,
                                           stream=s2)
