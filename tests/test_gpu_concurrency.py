@@ -16,7 +16,8 @@ the outputs against the one-stream run: bit for bit with one layer per
 exact call (neither kernel's arithmetic depends on the scheduling); with 4
 layers per call the keys are split another way, so (alpha, A) within the
 attention tolerances.  At Qwen3-1.7B shapes the exact attention is the
-CUDA-core split kernel instead."""
+CUDA-core split kernel instead; at b = 16 and 256 the M = 128 tensor-core
+kernel runs beside the local-attention states and the grouped GEMMs."""
 import pytest
 import torch
 
@@ -27,8 +28,10 @@ pytestmark = pytest.mark.gpu
 
 
 WORKLOADS = {
-    "llama8b_b1": ("llama8b_sweep", dict(B=1, rho=0.10)),   # transposed tensor-core exact kernel
-    "qwen3_1p7b": ("qwen3_1p7b", {}),                       # CUDA-core split kernel
+    "llama8b_b1": ("llama8b_sweep", dict(B=1, rho=0.10)),     # transposed tensor-core exact kernel, cluster decode
+    "qwen3_1p7b": ("qwen3_1p7b", {}),                         # CUDA-core split kernel, cluster decode
+    "llama8b_b16": ("llama8b_sweep", dict(B=16, rho=0.10)),   # tensor-core kernel (rows repeated), local_tct + GEMMs
+    "llama8b_b256": ("llama8b_sweep", dict(B=256, rho=0.10)), # tensor-core kernel, local_tct + grouped GEMMs
 }
 
 
